@@ -1,0 +1,77 @@
+"""Float64 restatements of the iterative inverse-root solvers (diagnostic).
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).  Never used as a parity
+gate: the gate is the exact root of ``oracle.shampoo.inverse_root``.  These
+mirrors take the same steps as the CUDA solvers in float64, so that when a
+parity check fails one can tell "not converged / method error" from "fp32
+rounding".
+
+Both start from the Frobenius-scaled, damped matrix A' = (A + eps I) / s,
+s = ||A + eps I||_F (spec(A') in (0, 1]), and unscale by s^{-1/p} at the end.
+
+* Coupled Newton for A'^{-1/p} (Guo & Higham, "A Schur-Newton method for the
+  matrix p-th root and its inverse", 2006): X_0 = I, M_0 = A';
+  T = ((p + 1) I - M) / p;  X <- X T;  M <- T^p M.  M -> I, X -> A'^{-1/p}.
+* Newton-DB, read as the coupled Denman-Beavers-family square-root iteration
+  in its multiplication-only (Newton-Schulz) form (Higham, "Functions of
+  Matrices", 2008, sec. 6.3 and 6.8): Y_0 = A', Z_0 = I;
+  T = (3 I - Z Y) / 2;  Y <- Y T;  Z <- T Z.  Y -> A'^{1/2}, Z -> A'^{-1/2}.
+  p = 2 takes Z; p = 4 runs the iteration a second time on A'' = Y (the first
+  run's square root) and takes that run's Z = A'^{-1/4}.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def frobenius_scale(A: np.ndarray, eps: float):
+    n = A.shape[0]
+    Ad = np.asarray(A, dtype=np.float64) + eps * np.eye(n)
+    s = float(np.linalg.norm(Ad))
+    return Ad / s, s
+
+
+def coupled_newton(A: np.ndarray, p: int, eps: float, iters: int, tol: float = 0.0):
+    """Returns (X, iterations run, final residual ||M - I||_F / sqrt(n))."""
+    M, s = frobenius_scale(A, eps)
+    n = M.shape[0]
+    eye = np.eye(n)
+    X = eye.copy()
+    res = np.linalg.norm(M - eye) / np.sqrt(n)
+    k = 0
+    while k < iters and not (tol > 0.0 and res <= tol):
+        T = ((p + 1) * eye - M) / p
+        X = X @ T
+        M = np.linalg.matrix_power(T, p) @ M
+        res = np.linalg.norm(M - eye) / np.sqrt(n)
+        k += 1
+    return X * s ** (-1.0 / p), k, res
+
+
+def newton_schulz_sqrt(A1: np.ndarray, iters: int, tol: float = 0.0):
+    """One Newton-DB stage on a matrix with spectrum in (0, 1].
+    Returns (Y ~ A1^{1/2}, Z ~ A1^{-1/2}, iterations, ||Z Y - I||_F / sqrt(n))."""
+    n = A1.shape[0]
+    eye = np.eye(n)
+    Y = A1.copy()
+    Z = eye.copy()
+    k = 0
+    res = np.linalg.norm(Z @ Y - eye) / np.sqrt(n)
+    while k < iters and not (tol > 0.0 and res <= tol):
+        T = 0.5 * (3.0 * eye - Z @ Y)
+        Y, Z = Y @ T, T @ Z
+        res = np.linalg.norm(Z @ Y - eye) / np.sqrt(n)
+        k += 1
+    return Y, Z, k, res
+
+
+def newton_db(A: np.ndarray, p: int, eps: float, iters: int, tol: float = 0.0):
+    """Returns (X, total iterations, final residual)."""
+    A1, s = frobenius_scale(A, eps)
+    Y, Z, k1, res = newton_schulz_sqrt(A1, iters, tol)
+    if p == 2:
+        return Z * s ** -0.5, k1, res
+    if p != 4:
+        raise ValueError("Newton-DB supports p = 2 and p = 4")
+    _, Z2, k2, res2 = newton_schulz_sqrt(Y, iters, tol)
+    return Z2 * s ** -0.25, k1 + k2, res2
