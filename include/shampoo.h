@@ -1,0 +1,229 @@
+/*
+ * shampoo.h - C ABI of the blocked Shampoo optimizer step on one NVIDIA B200
+ * (sm_100a).  Library: libshampoo.so (shampoo_family_second_b200/).
+ *
+ * What it computes ("Shampoo optimizer" notes, "Key Components" and the
+ * simplified matrix-case listing; podcast transcript "Preconditioned
+ * optimization without the full matrix cost", cues 20-28; DASH abstract):
+ * every weight W (m x n) is cut into B x B blocks (ragged edges zero-padded),
+ * and for every block, each step,
+ *     L <- beta L + G G^T,   R <- beta R + G^T G              (statistics)
+ *     XL = (L + eps I)^{-1/p},  XR = (R + eps I)^{-1/p}      (every refresh_every steps)
+ *     W <- W - lr * XL G XR                                  (update)
+ * with p = 4 by default (the notes' -1/4 powers) and p = 2 allowed (SOAP
+ * abstract: Shampoo with the 1/2 power).  The roots come from an iterative
+ * solver (coupled Newton, Newton-DB or Chebyshev) on Frobenius-scaled, damped
+ * statistics.  All products run on the tensor cores as 3xTF32 (fp32-accurate)
+ * tcgen05 MMAs.
+ *
+ * Conventions (all entry points):
+ *  - Ownership: the caller owns every device buffer (weights, gradients,
+ *    state, scratch, inputs, outputs).  The library never allocates device
+ *    memory; it owns only the small host-side handle.
+ *  - Streams: work is enqueued on the caller's cudaStream_t, passed as void*
+ *    (NULL = legacy default stream).  shampoo_step and inv_root_batched never
+ *    synchronise the host.
+ *  - Errors: argument errors return a negative SHAMPOO_ERR_* code before any
+ *    work is enqueued; shampoo_last_error() describes the last one on the
+ *    calling thread.  Conditions found on the device (non-finite values,
+ *    no convergence, a bounded wait that timed out) are OR-ed as
+ *    SHAMPOO_DEVFLAG_* bits into a device status word (see shampoo_get_status
+ *    and the d_status argument of inv_root_batched).
+ *  - Layout: matrices are row-major fp32 unless stated.  Stacks are
+ *    (batch, n, n).  A "split" stack is (batch, 2, n, n): per matrix a
+ *    tf32-exact high plane then a low plane; the value is high + low.
+ *  - Thread safety: a handle is not thread-safe; separate handles are
+ *    independent.  The profiling counters are process-wide.
+ */
+#ifndef SHAMPOO_B200_H
+#define SHAMPOO_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SHAMPOO_API __attribute__((visibility("default")))
+#else
+#define SHAMPOO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+enum {
+  SHAMPOO_OK = 0,
+  SHAMPOO_ERR_INVALID_ARG = -1, /* bad pointer, size, shape or config value */
+  SHAMPOO_ERR_UNSUPPORTED = -2, /* valid but not supported (e.g. alignment) */
+  SHAMPOO_ERR_WORKSPACE = -3,   /* state or scratch smaller than required */
+  SHAMPOO_ERR_CUDA = -4,        /* a CUDA runtime call failed */
+  SHAMPOO_ERR_DEVICE = -5       /* get_status: the device status word is non-zero */
+};
+
+/* Device status bits (OR-ed into the status word by the kernels). */
+enum {
+  SHAMPOO_DEVFLAG_NONFINITE = 1,     /* a NaN or Inf was produced */
+  SHAMPOO_DEVFLAG_NOT_CONVERGED = 2, /* tol > 0 and a residual stayed above tol after iters */
+  SHAMPOO_DEVFLAG_TIMEOUT = 4        /* a bounded on-chip wait gave up (kernel unwound) */
+};
+
+/* Inverse-root solvers (DASH abstract names Newton-DB and Chebyshev). */
+enum {
+  SHAMPOO_SOLVER_NEWTON = 0,    /* coupled Newton for A^{-1/p} (Guo & Higham 2006) */
+  SHAMPOO_SOLVER_NEWTON_DB = 1, /* coupled Y/Z square-root iteration, twice for p = 4 */
+  SHAMPOO_SOLVER_CHEBYSHEV = 2  /* Chebyshev interpolant of x^{-1/p}, Clenshaw evaluation */
+};
+
+/* Gradient element types. */
+enum { SHAMPOO_F32 = 0, SHAMPOO_BF16 = 1 };
+
+/* Profiler kernel kinds (shampoo_profile_read). */
+enum {
+  SHAMPOO_KERNEL_GEMM = 0,     /* tensor-core GEMM (stats, roots, apply) */
+  SHAMPOO_KERNEL_STACK = 1,    /* partition / stack of the gradient blocks */
+  SHAMPOO_KERNEL_NORM = 2,     /* Frobenius norms of the damped statistics */
+  SHAMPOO_KERNEL_PROLOGUE = 3, /* damping + scaling + first iterate */
+  SHAMPOO_KERNEL_CHECK = 4,    /* residual check */
+  SHAMPOO_KERNEL_FINALIZE = 5, /* unscale + output */
+  SHAMPOO_KERNEL_CHEB_COEF = 6,/* Chebyshev coefficients */
+  SHAMPOO_KERNEL_KINDS = 7
+};
+
+/* Hyper-parameters of the blocked step.
+ *  block          B: multiple of 32 in [32, 1024].
+ *  beta           statistics decay (beta = 1: plain running sum as in the notes' listing).
+ *  eps            damping: roots of (L + eps I); >= 0.
+ *  lr             learning rate eta.
+ *  root_p         2 or 4.
+ *  solver         SHAMPOO_SOLVER_*.
+ *  iters          iterations (tol = 0) or iteration cap (tol > 0) per Newton / Newton-DB
+ *                 stage, >= 1; ignored by Chebyshev.
+ *  tol            0: fixed iteration count; > 0: stop a matrix once
+ *                 ||M - I||_F / sqrt(n) (Newton) or ||Z Y - I||_F / sqrt(n) (Newton-DB) <= tol.
+ *  refresh_every  roots recomputed at steps t with t % refresh_every == 0 (t from 0), >= 1.
+ *  cheb_degree    Chebyshev degree d in [2, 64].
+ *  cheb_lo        Chebyshev interval: [lo / s, 1] with lo = cheb_lo if > 0 else eps,
+ *                 s = ||A + eps I||_F.
+ *  grad_dtype     SHAMPOO_F32 or SHAMPOO_BF16 (weights and statistics are always fp32). */
+typedef struct {
+  int32_t block;
+  float beta;
+  float eps;
+  float lr;
+  int32_t root_p;
+  int32_t solver;
+  int32_t iters;
+  float tol;
+  int32_t refresh_every;
+  int32_t cheb_degree;
+  float cheb_lo;
+  int32_t grad_dtype;
+} shampoo_config;
+
+typedef struct shampoo_ctx* shampoo_handle;
+
+/* Human-readable name of a return code or device status word.  Never NULL. */
+SHAMPOO_API const char* shampoo_status_string(int code);
+
+/* Description of the last error returned on the calling thread ("" if none). */
+SHAMPOO_API const char* shampoo_last_error(void);
+
+/* Sizes of the caller-owned device buffers for a parameter set.
+ * rows[i] x cols[i] is the shape of weight i (nparams in [1, 1024]).
+ * state_bytes: persistent state (statistics, roots, block table, status word).
+ * scratch_bytes: per-step scratch (stacked gradient blocks, solver iterates).
+ * Host-only; no CUDA call.  Source: the notes' "Key Components" (one m x m and
+ * one n x n preconditioner per block: O(m^2 + n^2) memory). */
+SHAMPOO_API int shampoo_query_sizes(const shampoo_config* cfg, int32_t nparams, const int64_t* rows, const int64_t* cols,
+                        size_t* state_bytes, size_t* scratch_bytes);
+
+/* Create a handle over caller-owned state and scratch (device pointers,
+ * 256-byte aligned, at least the queried sizes).  Zeroes the statistics
+ * (the notes' listing initialises L and R; eps enters as damping, see
+ * shampoo_config.eps), uploads the block table (stream-ordered on `stream`)
+ * and sets the step counter to 0. */
+SHAMPOO_API int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows, const int64_t* cols,
+                 void* d_state, size_t state_bytes, void* d_scratch, size_t scratch_bytes, void* stream,
+                 shampoo_handle* out);
+
+/* One optimizer step (the notes' loop body, for every block): accumulate the
+ * statistics from the gradients, recompute the roots if step % refresh_every
+ * == 0, then W <- W - lr XL G XR in place.  d_weights[i]: fp32 row-major
+ * rows[i] x cols[i]; d_grads[i]: same shape, grad_dtype.  Both are host arrays
+ * of nparams device pointers.  Enqueued on `stream`; no host sync. */
+SHAMPOO_API int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d_grads, void* stream);
+
+/* Synchronises the handle's last stream, reads the device status word into
+ * *status (0 = clean; else SHAMPOO_DEVFLAG_* bits) and returns SHAMPOO_OK, or
+ * SHAMPOO_ERR_CUDA if the device reported an error.  reset != 0 clears the word. */
+SHAMPOO_API int shampoo_get_status(shampoo_handle h, int32_t* status, int32_t reset);
+
+/* Block table: *nb blocks; if table != NULL it receives nb rows of
+ * {param, row0, col0, rows, cols} (int64, host memory), in stack order
+ * (param, block row, block column).  DASH abstract: blocks stacked into 3D tensors. */
+SHAMPOO_API int shampoo_block_table(shampoo_handle h, int32_t* nb, int64_t* table);
+
+/* Device pointers into the state (owned by the caller's state buffer):
+ * L: plain stack (nb, B, B) of left statistics; R: (nb, B, B) right statistics;
+ * rootL / rootR: split stacks (nb, 2, B, B) of XL and XR; *step: steps taken.
+ * Ragged blocks hold zeros outside their r x r / c x c valid region. */
+SHAMPOO_API int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, float** rootR, int64_t* step);
+
+/* Sets the step counter (checkpoint resume: restore the state buffer bytes,
+ * then the counter). */
+SHAMPOO_API int shampoo_set_step(shampoo_handle h, int64_t step);
+
+/* Frees the host-side handle (the caller's device buffers are untouched). */
+SHAMPOO_API void shampoo_destroy(shampoo_handle h);
+
+/* Scratch bytes inv_root_batched needs to solve all `batch` matrices in one
+ * pass.  Less (but at least the size for one matrix plus 64 KiB) makes it work
+ * through the batch in chunks.  Host-only. */
+SHAMPOO_API int inv_root_scratch_bytes(int64_t batch, int32_t n, int32_t solver, size_t* bytes);
+
+/* Batched inverse p-th roots: X_i ~ (A_i + eps I)^{-1/p} for symmetric
+ * positive semi-definite A_i (the notes' L^{-1/4}, R^{-1/4}; SOAP abstract's
+ * p = 2).  DASH abstract: batched inverse-root solvers with matrix scaling.
+ *  d_A, d_X      device plain stacks (batch, n, n); n a multiple of 32 in [32, 1024].
+ *                A is symmetrised ((A + A^T)/2) before use.
+ *  p             2 or 4.   eps  damping >= 0.
+ *  solver, iters, tol, cheb_degree, cheb_lo   as in shampoo_config.
+ *  d_scratch     device scratch, 256-byte aligned (see inv_root_scratch_bytes).
+ *  d_iters_used  nullable device int32[batch]: iterations run per matrix
+ *                (Newton-DB p = 4: both stages; Chebyshev: the degree); negative
+ *                when tol > 0 and the cap was reached without convergence.
+ *  d_status      nullable device int32: OR of SHAMPOO_DEVFLAG_* (not cleared).
+ *  stream        cudaStream_t as void*.  Enqueued; no host sync. */
+SHAMPOO_API int inv_root_batched(const float* d_A, float* d_X, int64_t batch, int32_t n, int32_t p, float eps, int32_t solver,
+                     int32_t iters, float tol, int32_t cheb_degree, float cheb_lo, void* d_scratch,
+                     size_t scratch_bytes, int32_t* d_iters_used, int32_t* d_status, void* stream);
+
+/* The batched fp32-accurate product every stage uses, as a utility:
+ * D_i = alpha A_i op(B_i) + beta C_i + gamma I for plain stacks (batch, n, n),
+ * op(B) = B^T (op_b = 0) or B (op_b = 1);
+ * d_C may be NULL (then beta is ignored) and may equal d_D.  n a multiple of
+ * 32 in [32, 4096].  Operands are split into tf32 hi/lo planes in d_scratch
+ * (see shampoo_gemm_scratch_bytes), then multiplied as 3xTF32 on the tensor
+ * cores.  Enqueued on `stream`; no host sync. */
+SHAMPOO_API int shampoo_gemm_scratch_bytes(int64_t batch, int32_t n, size_t* bytes);
+SHAMPOO_API int shampoo_gemm_batched(const float* d_A, const float* d_B, const float* d_C, float* d_D, int64_t batch, int32_t n,
+                         int32_t op_b, float alpha, float beta, float gamma, void* d_scratch, size_t scratch_bytes,
+                         int32_t* d_status, void* stream);
+
+/* Profiling (process-wide).  When enabled, every kernel launch of the library
+ * is bracketed by CUDA events on its own stream and tallied per kind with its
+ * algorithmic flops (GEMM: executed tiles only) and bytes.
+ * shampoo_profile_read synchronises the recorded events. */
+SHAMPOO_API void shampoo_profile_enable(int32_t on);
+SHAMPOO_API void shampoo_profile_reset(void);
+SHAMPOO_API int shampoo_profile_read(int32_t kind, int64_t* launches, double* total_ms, double* alg_flops, double* alg_bytes);
+
+/* Number of kernels this library has launched in this process. */
+SHAMPOO_API uint64_t shampoo_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SHAMPOO_B200_H */

@@ -1,0 +1,462 @@
+// C ABI of the blocked Shampoo step (include/shampoo.h): argument checking,
+// caller-owned state / scratch layout, and the order of work in one step.
+//
+// Step order ("Shampoo optimizer" notes, matrix-case listing: preconditioners
+// first, then the parameters; podcast "Preconditioned optimization without the
+// full matrix cost", cue 28: roots recomputed only every so many steps):
+//   1. stack     gradient blocks -> Gs (B x B, split) and Gt (transposed)
+//   2. stats     L <- beta L + Gs Gs^T, R <- beta R + Gt Gt^T     (one GEMM launch)
+//   3. roots     if step % refresh_every == 0: XL, XR of the damped, scaled stats
+//   4. apply     T = XL G (GEMM), then W -= lr T XR fused into the second
+//                GEMM's epilogue, masked to each block's real extent.
+#include <algorithm>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/shampoo.h"
+#include "internal.h"
+
+using namespace shampoo;
+
+namespace {
+
+constexpr size_t kAlignBytes = 256;
+constexpr size_t kRootBudget = size_t(16) << 30;  // solver scratch per step (chunks beyond)
+
+size_t al(size_t x) { return (x + kAlignBytes - 1) / kAlignBytes * kAlignBytes; }
+
+struct Shapes {
+  int nb = 0;
+  std::vector<int> table;  // nb x {param, row0, col0, r, c}
+};
+
+int validate_config(const shampoo_config* c) {
+  if (!c) return set_error(SHAMPOO_ERR_INVALID_ARG, "config is NULL");
+  if (c->block < 32 || c->block > 1024 || c->block % 32)
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "block %d: need a multiple of 32 in [32, 1024]", c->block);
+  if (!(c->beta >= 0.f) || !(c->beta <= 1.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "beta must be in [0, 1]");
+  if (!(c->eps >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "eps must be >= 0");
+  if (!(c->lr == c->lr)) return set_error(SHAMPOO_ERR_INVALID_ARG, "lr is NaN");
+  if (c->root_p != 2 && c->root_p != 4) return set_error(SHAMPOO_ERR_INVALID_ARG, "root_p must be 2 or 4");
+  if (c->solver < 0 || c->solver > 2) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", c->solver);
+  if (c->solver != SHAMPOO_SOLVER_CHEBYSHEV && (c->iters < 1 || c->iters > 1000))
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "iters must be in [1, 1000]");
+  if (!(c->tol >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "tol must be >= 0");
+  if (c->refresh_every < 1) return set_error(SHAMPOO_ERR_INVALID_ARG, "refresh_every must be >= 1");
+  if (c->solver == SHAMPOO_SOLVER_CHEBYSHEV) {
+    if (c->cheb_degree < 2 || c->cheb_degree > kMaxChebDegree)
+      return set_error(SHAMPOO_ERR_INVALID_ARG, "cheb_degree must be in [2, %d]", kMaxChebDegree);
+    if (!(c->cheb_lo > 0.f) && !(c->eps > 0.f))
+      return set_error(SHAMPOO_ERR_INVALID_ARG, "Chebyshev needs cheb_lo > 0 or eps > 0");
+  }
+  if (c->grad_dtype != SHAMPOO_F32 && c->grad_dtype != SHAMPOO_BF16)
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "grad_dtype must be SHAMPOO_F32 or SHAMPOO_BF16");
+  return SHAMPOO_OK;
+}
+
+int build_table(int B, int32_t nparams, const int64_t* rows, const int64_t* cols, Shapes& out) {
+  if (nparams < 1 || nparams > kMaxParams)
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "nparams %d: need 1..%d", nparams, kMaxParams);
+  if (!rows || !cols) return set_error(SHAMPOO_ERR_INVALID_ARG, "rows/cols is NULL");
+  out.table.clear();
+  for (int i = 0; i < nparams; ++i) {
+    if (rows[i] < 1 || cols[i] < 1 || rows[i] > (1 << 20) || cols[i] > (1 << 20))
+      return set_error(SHAMPOO_ERR_INVALID_ARG, "param %d has shape %lld x %lld", i, (long long)rows[i],
+                       (long long)cols[i]);
+    for (int64_t r0 = 0; r0 < rows[i]; r0 += B)
+      for (int64_t c0 = 0; c0 < cols[i]; c0 += B) {
+        out.table.push_back(i);
+        out.table.push_back(static_cast<int>(r0));
+        out.table.push_back(static_cast<int>(c0));
+        out.table.push_back(static_cast<int>(std::min<int64_t>(B, rows[i] - r0)));
+        out.table.push_back(static_cast<int>(std::min<int64_t>(B, cols[i] - c0)));
+      }
+  }
+  out.nb = static_cast<int>(out.table.size() / 5);
+  if (out.nb > 65535) return set_error(SHAMPOO_ERR_UNSUPPORTED, "%d blocks exceed 65535", out.nb);
+  return SHAMPOO_OK;
+}
+
+// State layout (bytes, each part 256-aligned):
+//   status word | block table (nb x 5 int32) | valid extents (2nb int32: r of L_b, c of R_b)
+//   | wrows (nb) | wcols (nb) | stats plain (2nb, B, B) | roots split (2nb, 2, B, B)
+struct StateLayout {
+  size_t status, table, valid, wrows, wcols, stats, roots, total;
+};
+StateLayout state_layout(int nb, int B) {
+  StateLayout s;
+  size_t o = 0;
+  s.status = o, o += al(4);
+  s.table = o, o += al(size_t(nb) * 5 * 4);
+  s.valid = o, o += al(size_t(2) * nb * 4);
+  s.wrows = o, o += al(size_t(nb) * 4);
+  s.wcols = o, o += al(size_t(nb) * 4);
+  s.stats = o, o += al(plain_floats(2 * nb, B) * 4);
+  s.roots = o, o += al(split_floats(2 * nb, B) * 4);
+  s.total = o;
+  return s;
+}
+// Scratch layout: Gs | Gt | Tapply (split, nb each) | blk_wptr (nb ptrs) | blk_ld (nb) | solver scratch
+struct ScratchLayout {
+  size_t gs, gt, tap, wptr, ld, root, root_bytes, total;
+};
+ScratchLayout scratch_layout(int nb, int B, int solver) {
+  ScratchLayout s;
+  size_t o = 0;
+  s.gs = o, o += al(split_floats(nb, B) * 4);
+  s.gt = o, o += al(split_floats(nb, B) * 4);
+  s.tap = o, o += al(split_floats(nb, B) * 4);
+  s.wptr = o, o += al(size_t(nb) * 8);
+  s.ld = o, o += al(size_t(nb) * 4);
+  s.root = o;
+  const size_t per = root_scratch_per_matrix(B, solver);
+  const size_t want = root_scratch_header() + per * size_t(2 * nb);
+  s.root_bytes = std::min(want, std::max(kRootBudget, root_scratch_header() + per));
+  o += al(s.root_bytes);
+  s.total = o;
+  return s;
+}
+
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+
+}  // namespace
+
+struct shampoo_ctx {
+  shampoo_config cfg;
+  int nparams = 0;
+  std::vector<int64_t> rows, cols;
+  Shapes shapes;
+  StateLayout sl;
+  ScratchLayout xl;
+  char* state = nullptr;
+  char* scratch = nullptr;
+  int* d_status = nullptr;
+  int* d_table = nullptr;
+  int* d_valid = nullptr;
+  int* d_wrows = nullptr;
+  int* d_wcols = nullptr;
+  float* stats = nullptr;
+  float* roots = nullptr;
+  float* Gs = nullptr;
+  float* Gt = nullptr;
+  float* Tap = nullptr;
+  float** blk_wptr = nullptr;
+  int* blk_ld = nullptr;
+  StackMaps mGs, mGt, mRoots, mTap;
+  double stats_flops_L = 0, stats_flops_R = 0, stack_bytes = 0;
+  int64_t step = 0;
+  cudaStream_t last_stream = nullptr;
+};
+
+extern "C" {
+
+const char* shampoo_status_string(int code) {
+  switch (code) {
+    case SHAMPOO_OK: return "SHAMPOO_OK";
+    case SHAMPOO_ERR_INVALID_ARG: return "SHAMPOO_ERR_INVALID_ARG";
+    case SHAMPOO_ERR_UNSUPPORTED: return "SHAMPOO_ERR_UNSUPPORTED";
+    case SHAMPOO_ERR_WORKSPACE: return "SHAMPOO_ERR_WORKSPACE";
+    case SHAMPOO_ERR_CUDA: return "SHAMPOO_ERR_CUDA";
+    case SHAMPOO_ERR_DEVICE: return "SHAMPOO_ERR_DEVICE";
+    default: return "SHAMPOO_UNKNOWN_STATUS";
+  }
+}
+
+int shampoo_query_sizes(const shampoo_config* cfg, int32_t nparams, const int64_t* rows, const int64_t* cols,
+                        size_t* state_bytes, size_t* scratch_bytes) {
+  int rc = validate_config(cfg);
+  if (rc) return rc;
+  Shapes sh;
+  if ((rc = build_table(cfg->block, nparams, rows, cols, sh))) return rc;
+  if (!state_bytes || !scratch_bytes) return set_error(SHAMPOO_ERR_INVALID_ARG, "output pointer is NULL");
+  *state_bytes = state_layout(sh.nb, cfg->block).total;
+  *scratch_bytes = scratch_layout(sh.nb, cfg->block, cfg->solver).total;
+  return SHAMPOO_OK;
+}
+
+int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows, const int64_t* cols, void* d_state,
+                 size_t state_bytes, void* d_scratch, size_t scratch_bytes, void* stream, shampoo_handle* out) {
+  int rc = validate_config(cfg);
+  if (rc) return rc;
+  if (!out) return set_error(SHAMPOO_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  Shapes sh;
+  if ((rc = build_table(cfg->block, nparams, rows, cols, sh))) return rc;
+  if (!d_state || !d_scratch) return set_error(SHAMPOO_ERR_INVALID_ARG, "state/scratch is NULL");
+  if (!aligned256(d_state) || !aligned256(d_scratch))
+    return set_error(SHAMPOO_ERR_UNSUPPORTED, "state/scratch must be 256-byte aligned");
+  const int B = cfg->block, nb = sh.nb;
+  StateLayout sl = state_layout(nb, B);
+  ScratchLayout xl = scratch_layout(nb, B, cfg->solver);
+  if (state_bytes < sl.total) return set_error(SHAMPOO_ERR_WORKSPACE, "state %zu < %zu bytes", state_bytes, sl.total);
+  if (scratch_bytes < xl.total)
+    return set_error(SHAMPOO_ERR_WORKSPACE, "scratch %zu < %zu bytes", scratch_bytes, xl.total);
+
+  shampoo_ctx* h = new (std::nothrow) shampoo_ctx;
+  if (!h) return set_error(SHAMPOO_ERR_INVALID_ARG, "out of host memory");
+  h->cfg = *cfg;
+  h->nparams = nparams;
+  h->rows.assign(rows, rows + nparams);
+  h->cols.assign(cols, cols + nparams);
+  h->shapes = sh;
+  h->sl = sl;
+  h->xl = xl;
+  h->state = static_cast<char*>(d_state);
+  h->scratch = static_cast<char*>(d_scratch);
+  h->d_status = reinterpret_cast<int*>(h->state + sl.status);
+  h->d_table = reinterpret_cast<int*>(h->state + sl.table);
+  h->d_valid = reinterpret_cast<int*>(h->state + sl.valid);
+  h->d_wrows = reinterpret_cast<int*>(h->state + sl.wrows);
+  h->d_wcols = reinterpret_cast<int*>(h->state + sl.wcols);
+  h->stats = reinterpret_cast<float*>(h->state + sl.stats);
+  h->roots = reinterpret_cast<float*>(h->state + sl.roots);
+  h->Gs = reinterpret_cast<float*>(h->scratch + xl.gs);
+  h->Gt = reinterpret_cast<float*>(h->scratch + xl.gt);
+  h->Tap = reinterpret_cast<float*>(h->scratch + xl.tap);
+  h->blk_wptr = reinterpret_cast<float**>(h->scratch + xl.wptr);
+  h->blk_ld = reinterpret_cast<int*>(h->scratch + xl.ld);
+
+  std::vector<int> valid(2 * nb), wr(nb), wc(nb);
+  double fl = 0, fr = 0, sb = 0;
+  for (int b = 0; b < nb; ++b) {
+    const double r = sh.table[5 * b + 3], c = sh.table[5 * b + 4];
+    valid[b] = sh.table[5 * b + 3];
+    valid[nb + b] = sh.table[5 * b + 4];
+    wr[b] = sh.table[5 * b + 3];
+    wc[b] = sh.table[5 * b + 4];
+    fl += 2 * r * r * c;
+    fr += 2 * r * c * c;
+    sb += r * c * (cfg->grad_dtype == SHAMPOO_BF16 ? 2 : 4) + 4.0 * 8.0 * B * B;
+  }
+  h->stats_flops_L = fl / nb;
+  h->stats_flops_R = fr / nb;
+  h->stack_bytes = sb;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  auto up = [&](void* dst, const void* src, size_t bytes) {
+    return check_cuda(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st), "upload block table");
+  };
+  if ((rc = up(h->d_table, sh.table.data(), sh.table.size() * 4)) || (rc = up(h->d_valid, valid.data(), valid.size() * 4)) ||
+      (rc = up(h->d_wrows, wr.data(), wr.size() * 4)) || (rc = up(h->d_wcols, wc.data(), wc.size() * 4)) ||
+      (rc = check_cuda(cudaMemsetAsync(h->d_status, 0, 4, st), "zero status")) ||
+      (rc = check_cuda(cudaMemsetAsync(h->stats, 0, plain_floats(2 * nb, B) * 4, st), "zero statistics")) ||
+      (rc = check_cuda(cudaMemsetAsync(h->roots, 0, split_floats(2 * nb, B) * 4, st), "zero roots")) ||
+      (rc = check_cuda(cudaStreamSynchronize(st), "init sync"))) {
+    delete h;
+    return rc;
+  }
+  if ((rc = make_stack_maps(h->mGs, h->Gs, nb, B)) || (rc = make_stack_maps(h->mGt, h->Gt, nb, B)) ||
+      (rc = make_stack_maps(h->mRoots, h->roots, 2 * nb, B)) || (rc = make_stack_maps(h->mTap, h->Tap, nb, B))) {
+    delete h;
+    return rc;
+  }
+  *out = h;
+  return SHAMPOO_OK;
+}
+
+int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d_grads, void* stream) {
+  if (!h) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle is NULL");
+  if (!d_weights || !d_grads) return set_error(SHAMPOO_ERR_INVALID_ARG, "weights/grads array is NULL");
+  const shampoo_config& c = h->cfg;
+  const int B = c.block, nb = h->shapes.nb;
+  StackArgs args;
+  for (int i = 0; i < h->nparams; ++i) {
+    if (!d_weights[i] || !d_grads[i]) return set_error(SHAMPOO_ERR_INVALID_ARG, "param %d has a NULL pointer", i);
+    args.g[i] = d_grads[i];
+    args.w[i] = d_weights[i];
+    args.ld[i] = static_cast<int>(h->cols[i]);
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  int rc;
+  // 1. partition / stack
+  if ((rc = launch_stack(args, h->d_table, nb, B, c.grad_dtype, h->Gs, h->Gt, h->blk_wptr, h->blk_ld, st,
+                         h->stack_bytes)))
+    return rc;
+  // 2. statistics: L <- beta L + G G^T (first nb matrices), R <- beta R + G^T G (next nb)
+  {
+    Builder b;
+    Epilogue& eL = b.add(nb, B, h->mGs, 0, h->mGs, 0, h->stats_flops_L);
+    eL.beta = c.beta;
+    eL.C = h->stats;
+    eL.D = h->stats;
+    eL.flags = h->d_status;
+    Epilogue& eR = b.add(nb, B, h->mGt, 0, h->mGt, 0, h->stats_flops_R);
+    eR.beta = c.beta;
+    eR.C = h->stats + plain_floats(nb, B);
+    eR.D = h->stats + plain_floats(nb, B);
+    eR.flags = h->d_status;
+    if ((rc = b.launch(st))) return rc;
+  }
+  // 3. roots of all 2 nb damped statistics, every refresh_every steps
+  if (h->step % c.refresh_every == 0) {
+    RootJob job;
+    job.batch = 2 * nb;
+    job.n = B;
+    job.p = c.root_p;
+    job.solver = c.solver;
+    job.iters = c.iters;
+    job.cheb_degree = c.cheb_degree;
+    job.eps = c.eps;
+    job.tol = c.tol;
+    job.cheb_lo = c.cheb_lo;
+    job.A = h->stats;
+    job.valid = h->d_valid;
+    job.X_plain = nullptr;
+    job.X_split = h->roots;
+    job.iters_used = nullptr;
+    job.flags = h->d_status;
+    if ((rc = run_inverse_roots(job, h->scratch + h->xl.root, h->xl.root_bytes, st))) return rc;
+  }
+  // 4. apply: T = XL G, then W -= lr T XR (masked scatter into the weights)
+  {
+    Builder b;
+    Epilogue& e = b.add(nb, B, h->mRoots, 0, h->mGt, 0, h->stats_flops_L);
+    e.D = h->Tap;
+    e.d_split = 1;
+    e.flags = h->d_status;
+    if ((rc = b.launch(st))) return rc;
+  }
+  {
+    Builder b;
+    Epilogue& e = b.add(nb, B, h->mTap, 0, h->mRoots, nb, h->stats_flops_R);
+    e.wptr = h->blk_wptr;
+    e.wld = h->blk_ld;
+    e.wrows = h->d_wrows;
+    e.wcols = h->d_wcols;
+    e.lr = c.lr;
+    e.flags = h->d_status;
+    if ((rc = b.launch(st))) return rc;
+  }
+  h->step += 1;
+  return SHAMPOO_OK;
+}
+
+int shampoo_get_status(shampoo_handle h, int32_t* status, int32_t reset) {
+  if (!h || !status) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle/status is NULL");
+  int rc = check_cuda(cudaStreamSynchronize(h->last_stream), "status sync");
+  if (rc) return rc;
+  int v = 0;
+  if ((rc = check_cuda(cudaMemcpy(&v, h->d_status, 4, cudaMemcpyDeviceToHost), "read status"))) return rc;
+  *status = v;
+  if (reset && (rc = check_cuda(cudaMemset(h->d_status, 0, 4), "reset status"))) return rc;
+  return SHAMPOO_OK;
+}
+
+int shampoo_block_table(shampoo_handle h, int32_t* nb, int64_t* table) {
+  if (!h || !nb) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle/nb is NULL");
+  *nb = h->shapes.nb;
+  if (table)
+    for (size_t i = 0; i < h->shapes.table.size(); ++i) table[i] = h->shapes.table[i];
+  return SHAMPOO_OK;
+}
+
+int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, float** rootR, int64_t* step) {
+  if (!h) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle is NULL");
+  const int nb = h->shapes.nb, B = h->cfg.block;
+  if (L) *L = h->stats;
+  if (R) *R = h->stats + plain_floats(nb, B);
+  if (rootL) *rootL = h->roots;
+  if (rootR) *rootR = h->roots + split_floats(nb, B);
+  if (step) *step = h->step;
+  return SHAMPOO_OK;
+}
+
+int shampoo_set_step(shampoo_handle h, int64_t step) {
+  if (!h || step < 0) return set_error(SHAMPOO_ERR_INVALID_ARG, "bad handle or step");
+  h->step = step;
+  return SHAMPOO_OK;
+}
+
+void shampoo_destroy(shampoo_handle h) { delete h; }
+
+int inv_root_scratch_bytes(int64_t batch, int32_t n, int32_t solver, size_t* bytes) {
+  if (!bytes) return set_error(SHAMPOO_ERR_INVALID_ARG, "bytes is NULL");
+  if (batch < 0 || n < 32 || n > 1024 || n % 32 || solver < 0 || solver > 2)
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "bad batch / n / solver");
+  *bytes = root_scratch_header() + root_scratch_per_matrix(n, solver) * static_cast<size_t>(std::max<int64_t>(batch, 1));
+  return SHAMPOO_OK;
+}
+
+int inv_root_batched(const float* d_A, float* d_X, int64_t batch, int32_t n, int32_t p, float eps, int32_t solver,
+                     int32_t iters, float tol, int32_t cheb_degree, float cheb_lo, void* d_scratch,
+                     size_t scratch_bytes, int32_t* d_iters_used, int32_t* d_status, void* stream) {
+  if (batch < 0) return set_error(SHAMPOO_ERR_INVALID_ARG, "batch < 0");
+  if (batch == 0) return SHAMPOO_OK;
+  if (!d_A || !d_X || !d_scratch) return set_error(SHAMPOO_ERR_INVALID_ARG, "NULL device pointer");
+  if (n < 32 || n > 1024 || n % 32) return set_error(SHAMPOO_ERR_INVALID_ARG, "n %d: need a multiple of 32 in [32, 1024]", n);
+  if (p != 2 && p != 4) return set_error(SHAMPOO_ERR_INVALID_ARG, "p must be 2 or 4");
+  if (!(eps >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "eps must be >= 0");
+  if (solver < 0 || solver > 2) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", solver);
+  if (solver != SHAMPOO_SOLVER_CHEBYSHEV && (iters < 1 || iters > 1000))
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "iters must be in [1, 1000]");
+  if (!(tol >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "tol must be >= 0");
+  if (solver == SHAMPOO_SOLVER_CHEBYSHEV) {
+    if (cheb_degree < 2 || cheb_degree > kMaxChebDegree)
+      return set_error(SHAMPOO_ERR_INVALID_ARG, "cheb_degree must be in [2, %d]", kMaxChebDegree);
+    if (!(cheb_lo > 0.f) && !(eps > 0.f))
+      return set_error(SHAMPOO_ERR_INVALID_ARG, "Chebyshev needs cheb_lo > 0 or eps > 0");
+  }
+  if (!aligned256(d_scratch) || (reinterpret_cast<uintptr_t>(d_A) & 15) || (reinterpret_cast<uintptr_t>(d_X) & 15))
+    return set_error(SHAMPOO_ERR_UNSUPPORTED, "scratch must be 256-byte and A, X 16-byte aligned");
+  RootJob job;
+  job.batch = batch;
+  job.n = n;
+  job.p = p;
+  job.solver = solver;
+  job.iters = iters;
+  job.cheb_degree = cheb_degree;
+  job.eps = eps;
+  job.tol = tol;
+  job.cheb_lo = cheb_lo;
+  job.A = d_A;
+  job.valid = nullptr;
+  job.X_plain = d_X;
+  job.X_split = nullptr;
+  job.iters_used = d_iters_used;
+  job.flags = d_status;
+  return run_inverse_roots(job, d_scratch, scratch_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int shampoo_gemm_scratch_bytes(int64_t batch, int32_t n, size_t* bytes) {
+  if (!bytes || batch < 0 || n < 32 || n > 4096 || n % 32)
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "bad arguments");
+  *bytes = 2 * al(split_floats(batch, n) * 4);
+  return SHAMPOO_OK;
+}
+
+int shampoo_gemm_batched(const float* d_A, const float* d_B, const float* d_C, float* d_D, int64_t batch, int32_t n,
+                         int32_t op_b, float alpha, float beta, float gamma, void* d_scratch, size_t scratch_bytes,
+                         int32_t* d_status, void* stream) {
+  if (batch < 0 || n < 32 || n > 4096 || n % 32) return set_error(SHAMPOO_ERR_INVALID_ARG, "bad batch / n");
+  if (op_b != 0 && op_b != 1) return set_error(SHAMPOO_ERR_INVALID_ARG, "op_b must be 0 (B^T) or 1 (B)");
+  if (batch == 0) return SHAMPOO_OK;
+  if (batch > 0x7fffffff / 32) return set_error(SHAMPOO_ERR_UNSUPPORTED, "batch too large");
+  if (!d_A || !d_B || !d_D || !d_scratch) return set_error(SHAMPOO_ERR_INVALID_ARG, "NULL device pointer");
+  size_t need = 0;
+  shampoo_gemm_scratch_bytes(batch, n, &need);
+  if (scratch_bytes < need) return set_error(SHAMPOO_ERR_WORKSPACE, "scratch %zu < %zu bytes", scratch_bytes, need);
+  if (!aligned256(d_scratch) || (reinterpret_cast<uintptr_t>(d_A) & 15) || (reinterpret_cast<uintptr_t>(d_B) & 15) ||
+      (reinterpret_cast<uintptr_t>(d_D) & 15) || (reinterpret_cast<uintptr_t>(d_C) & 15))
+    return set_error(SHAMPOO_ERR_UNSUPPORTED, "scratch must be 256-byte and A, B, C, D 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* As = static_cast<float*>(d_scratch);
+  float* Bs = reinterpret_cast<float*>(static_cast<char*>(d_scratch) + al(split_floats(batch, n) * 4));
+  int rc;
+  if ((rc = launch_split_plain(d_A, As, batch, n, st)) || (rc = launch_split_plain(d_B, Bs, batch, n, st))) return rc;
+  StackMaps ma, mb;
+  if ((rc = make_stack_maps(ma, As, batch, n)) || (rc = make_stack_maps(mb, Bs, batch, n))) return rc;
+  Builder b;
+  Epilogue& e = b.add(static_cast<int>(batch), n, ma, 0, mb, 0, 2.0 * n * double(n) * n, op_b);
+  e.alpha = alpha;
+  e.beta = d_C ? beta : 0.f;
+  e.gamma = gamma;
+  e.C = d_C;
+  e.D = d_D;
+  e.flags = d_status;
+  return b.launch(st);
+}
+
+}  // extern "C"

@@ -1,0 +1,186 @@
+// Internal (host + device) declarations of the blocked Shampoo library.
+// Nothing here is part of the public C ABI (include/shampoo.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>  // CUtensorMap (type only; the driver entry point is fetched at run time)
+#include <cuda_runtime.h>
+
+namespace shampoo {
+
+// ---------------------------------------------------------------------------
+// Storage formats
+//   plain stack : (batch, n, n) fp32, row-major matrices back to back.
+//   split stack : (batch, 2, n, n) fp32; matrix i holds its tf32-exact "hi"
+//                 plane then its "lo" plane (value = hi + lo, see split_tf32).
+// Split stacks are the operand format of the tensor-core GEMM.
+// ---------------------------------------------------------------------------
+inline size_t plain_floats(int64_t batch, int n) { return static_cast<size_t>(batch) * n * n; }
+inline size_t split_floats(int64_t batch, int n) { return 2 * static_cast<size_t>(batch) * n * n; }
+
+constexpr int kMaxGroups = 4;
+constexpr int kMaxMaps = 2 * kMaxGroups;
+constexpr int kMaxParams = 1024;
+constexpr int kMaxChebDegree = 64;
+
+// Epilogue of one GEMM group.  For matrix i of the group and element (r, c):
+//   v = scale_i * (alpha * acc + beta * C_i[r][c] + gamma_i * [r == c])
+// with acc = (A_i B_i^T)[r][c], gamma_i = gamma_vec[i * gamma_stride] when
+// gamma_vec is set (else gamma) and scale_i = scale_vec[i] (else 1).
+// All per-matrix pointers are already offset to the group's first matrix.
+struct Epilogue {
+  float alpha, beta, gamma;
+  const float* gamma_vec;
+  int gamma_stride;
+  const float* scale_vec;
+  const float* C;  // optional input stack
+  int c_split;     // C is a split stack (else plain)
+  float* D;        // optional main output stack
+  int d_split;     // D is a split stack (else plain)
+  float* E;        // optional second output (split): e_mul * v + e_add * [r == c]
+  float e_mul, e_add;
+  float* res;        // optional: res[i] += sum over the valid region of (acc - [r == c])^2
+  const int* valid;  // per-matrix valid extent (nullable: n)
+  const int* skip;   // per-matrix "done" flags: a set flag skips the matrix
+  int* flags;        // device status word (nullable)
+  // Weight update: W_i[r * ld_i + c] -= lr * v for r < wrows_i, c < wcols_i,
+  // W_i = wptr[i] (a pointer to the block's top-left weight element).
+  float* const* wptr;
+  const int* wld;
+  const int* wrows;
+  const int* wcols;
+  float lr;
+};
+
+struct GemmGroup {
+  int batch;       // matrices in this group
+  int n;           // square size (multiple of 32)
+  int a_map, b_map;  // tensor-map slots (A as 128-row boxes, B as 256-row boxes)
+  int a_off, b_off;  // matrix index offsets into the mapped stacks
+  int a_rows, b_rows;  // box rows of the two maps (min(tile, n))
+  int b_mn;            // 1: B is read MN-major (D = A B); 0: K-major (D = A B^T)
+  int tiles_m, tiles_n, cta_begin;  // filled by launch_gemm
+  double flops_per_matrix;          // algorithmic flops (profiling only)
+  Epilogue ep;
+};
+
+struct GemmLaunch {
+  int ngroups;
+  int profile;  // accumulate executed algorithmic flops into the profiler slot
+  int prof_slot;
+  GemmGroup g[kMaxGroups];
+};
+
+struct TmaMaps {
+  CUtensorMap m[kMaxMaps];
+};
+
+// GEMM tile geometry (tcgen05 kind::tf32, one CTA per tile).
+constexpr int kTileM = 128;
+constexpr int kTileN = 256;
+constexpr int kTileK = 32;
+
+// Host helpers -------------------------------------------------------------
+int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout = 0);
+int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st);
+Epilogue epilogue_defaults();
+
+// Errors: codes from include/shampoo.h; message kept per thread.
+int set_error(int code, const char* fmt, ...);
+int check_cuda(cudaError_t e, const char* what);
+
+// Profiler (process-wide).  Kinds index the per-kernel tallies.
+enum KernelKind : int {
+  K_GEMM = 0,
+  K_STACK = 1,
+  K_NORM = 2,
+  K_PROLOGUE = 3,
+  K_CHECK = 4,
+  K_FINALIZE = 5,
+  K_CHEB_COEF = 6,
+  K_COUNT = 7,
+};
+struct ProfScope {
+  ProfScope(int kind, cudaStream_t st, double alg_flops, double alg_bytes);
+  ~ProfScope();
+  int kind;
+  cudaStream_t st;
+  double flops, bytes;
+  int active;
+  int ev;
+};
+void count_launch();
+bool profiling_enabled();
+double* device_flop_slots();  // device address of the executed-flop accumulators
+
+
+// A GEMM launch under construction: groups plus the tensor maps they reference.
+struct StackMaps {
+  CUtensorMap a, b;  // the split stack as A (128-row boxes) and as K-major B (256-row boxes)
+  CUtensorMap mn;    // as MN-major B: 32 x 32 boxes (32 rows of K, 32 columns of N)
+  float* base;
+  int a_rows, b_rows;
+};
+int make_stack_maps(StackMaps& sm, float* base, int64_t batch, int n);
+
+struct Builder {
+  GemmLaunch L;
+  TmaMaps M;
+  int nmaps;
+  Builder();
+  // Adds a group D_i = epi(A_i B_i^T) (b_mn = 0) or epi(A_i B_i) (b_mn = 1)
+  // over matrices a_off.. of `a` and b_off.. of `b`.
+  Epilogue& add(int batch, int n, const StackMaps& a, int a_off, const StackMaps& b, int b_off,
+                double flops_per_matrix, int b_mn = 0);
+  int launch(cudaStream_t st) { return launch_gemm(L, M, st); }
+};
+
+int launch_report(const int* iters, const int* add, const int* done, int64_t batch, int default_iters, int* out,
+                  int* flags, bool residual, cudaStream_t st);
+int launch_split_plain(const float* src, float* dst, int64_t batch, int n, cudaStream_t st);
+
+// Elementwise / reduction kernels (kernels_elem.cu) ---------------------------
+struct StackArgs {
+  const void* g[kMaxParams];
+  float* w[kMaxParams];
+  int ld[kMaxParams];
+};
+int launch_stack(const StackArgs& args, const int* d_table, int nb, int B, int grad_dtype, float* Gs, float* Gts,
+                 float** blk_wptr, int* blk_ld, cudaStream_t st, double alg_bytes);
+
+int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, float eps, int p, float* s, float* sc,
+                     cudaStream_t st);
+// kind: 0 = Newton (M0, T0 = ((p+1)I - M0)/p, X1 = T0)
+//       1 = Newton-DB (Y0 = A', T0 = (3I - A')/2, Z1 = T0)
+int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const int* valid, float eps, int p,
+                         const float* s, float* out0, float* out1, float* out2, cudaStream_t st);
+// Second Newton-DB stage: Y0' = Y_par(i) (parity from iters), T0 = (3I - Y0')/2, Z1 = T0.
+int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters, int64_t batch, int n,
+                              float* Ynew0, float* T, float* Z1, cudaStream_t st);
+int launch_check(float* res, int* done, int* iters, const int* valid, int64_t batch, int n, float tol, int it,
+                 int* flags, cudaStream_t st);
+int launch_finalize(const float* X0, const float* X1, const int* iters, int default_iters, const float* sc,
+                    int64_t batch, int n, float* out_plain, float* out_split, int* flags, cudaStream_t st);
+int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int degree,
+                      float lo, const float* s, float* coef, float* sc, float* Xt, float* bd, float* bd1,
+                      cudaStream_t st);
+int launch_fill_iters(int* iters, int64_t batch, int value, cudaStream_t st);
+
+// Inverse-root solver (solver.cu) ---------------------------------------------
+struct RootJob {
+  int64_t batch;
+  int n, p, solver, iters, cheb_degree;
+  float eps, tol, cheb_lo;
+  const float* A;    // plain stack input
+  const int* valid;  // device valid extents (nullable)
+  float* X_plain;    // plain output (nullable)
+  float* X_split;    // split output (nullable)
+  int* iters_used;   // device per-matrix iterations (nullable)
+  int* flags;        // device status word (nullable)
+};
+size_t root_scratch_per_matrix(int n, int solver);
+size_t root_scratch_header();
+int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, cudaStream_t st);
+
+}  // namespace shampoo

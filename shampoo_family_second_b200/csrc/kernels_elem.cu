@@ -1,0 +1,441 @@
+// Memory-bound kernels of the blocked Shampoo step: the block partitioner /
+// stacker, the damping + Frobenius pre-scaling prologues of the inverse-root
+// solvers, the residual check, the unscale / output pass, and the Chebyshev
+// coefficient setup.  All reads and writes are coalesced (transposes go through
+// a 32 x 33 shared-memory tile) and each kernel touches each byte once.
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace shampoo {
+namespace {
+
+__device__ __forceinline__ float load_grad(const void* g, size_t idx, int dtype) {
+  if (dtype == 1) {
+    const uint16_t bits = reinterpret_cast<const uint16_t*>(g)[idx];
+    return __uint_as_float(static_cast<uint32_t>(bits) << 16);
+  }
+  return reinterpret_cast<const float*>(g)[idx];
+}
+
+__device__ __forceinline__ void store_split(float* stack, size_t mat, size_t nn, size_t idx, float v) {
+  float h, l;
+  split_tf32(v, h, l);
+  stack[mat * 2 * nn + idx] = h;
+  stack[mat * 2 * nn + nn + idx] = l;
+}
+
+// ---------------------------------------------------------------------------
+// A1 partition / stack.  DASH abstract: preconditioner blocks stacked into 3D
+// tensors.  Block b of the table {param, row0, col0, r, c} is copied from the
+// row-major gradient into Gs[b] (B x B, split) and its transpose into Gt[b],
+// zero-padded beyond (r, c).  Also records where the block's weights live.
+// grid (B/32, B/32, nb), block (32, 8).
+// ---------------------------------------------------------------------------
+__global__ void stack_split_kernel(const __grid_constant__ StackArgs args, const int* __restrict__ table, int B,
+                                   int dtype, float* __restrict__ Gs, float* __restrict__ Gt, float** blk_wptr,
+                                   int* blk_ld) {
+  __shared__ float tile[32][33];
+  const int b = blockIdx.z;
+  const int bi = blockIdx.y, bj = blockIdx.x;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int param = table[5 * b + 0];
+  const int row0 = table[5 * b + 1], col0 = table[5 * b + 2];
+  const int r = table[5 * b + 3], c = table[5 * b + 4];
+  const void* g = args.g[param];
+  const int ld = args.ld[param];
+  const size_t nn = static_cast<size_t>(B) * B;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int row = bi * 32 + ty + 8 * k;
+    const int col = bj * 32 + tx;
+    float v = 0.f;
+    if (row < r && col < c) v = load_grad(g, static_cast<size_t>(row0 + row) * ld + col0 + col, dtype);
+    tile[ty + 8 * k][tx] = v;
+    store_split(Gs, b, nn, static_cast<size_t>(row) * B + col, v);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int row = bj * 32 + ty + 8 * k;  // row of G^T = column of G
+    const int col = bi * 32 + tx;
+    store_split(Gt, b, nn, static_cast<size_t>(row) * B + col, tile[tx][ty + 8 * k]);
+  }
+  if (bi == 0 && bj == 0 && tx == 0 && ty == 0) {
+    blk_wptr[b] = args.w[param] + static_cast<size_t>(row0) * ld + col0;
+    blk_ld[b] = ld;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// s_i = ||A_i + eps I||_F over the valid region, and sc_i = s_i^{-1/p}
+// (Frobenius pre-scaling; DASH abstract: matrix scaling).  One CTA per matrix,
+// float64 accumulation.
+// ---------------------------------------------------------------------------
+__global__ void frob_norm_kernel(const float* __restrict__ A, int n, const int* __restrict__ valid, float eps,
+                                 double inv_p, float* __restrict__ s, float* __restrict__ sc) {
+  const int i = blockIdx.x;
+  const int v = valid ? valid[i] : n;
+  const float* a = A + static_cast<size_t>(i) * n * n;
+  double acc = 0.0;
+  for (int r = threadIdx.y; r < v; r += blockDim.y) {
+    const float* row = a + static_cast<size_t>(r) * n;
+    for (int c = threadIdx.x; c < v; c += blockDim.x) {
+      const double x = static_cast<double>(row[c]) + ((r == c) ? static_cast<double>(eps) : 0.0);
+      acc += x * x;
+    }
+  }
+  __shared__ double red[32];
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  const int tid = threadIdx.y * blockDim.x + threadIdx.x;
+  if ((tid & 31) == 0) red[tid >> 5] = acc;
+  __syncthreads();
+  if (tid < 32) {
+    const int nw = (blockDim.x * blockDim.y) >> 5;
+    double x = (tid < nw) ? red[tid] : 0.0;
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (tid == 0) {
+      double sv = sqrt(x);
+      if (!(sv > 0.0)) sv = 1.0;  // all-zero matrix with eps = 0: keep the scale finite
+      s[i] = static_cast<float>(sv);
+      sc[i] = static_cast<float>(pow(sv, -inv_p));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Solver prologues.  A' = (sym(A) + eps I) / s on the valid region; the padded
+// region of a ragged block gets the identity (its root is then exactly the
+// identity times s^{-1/p} and never slows convergence).
+//   kind 0, coupled Newton: out0 = M0 = A', out1 = T0 = ((p+1) I - A') / p,
+//                           out2 = X1 = T0.
+//   kind 1, Newton-DB:      out0 = Y0 = A', out1 = T0 = (3 I - A') / 2,
+//                           out2 = Z1 = T0.
+// grid (n/32, n/32, batch), block (32, 8).
+// ---------------------------------------------------------------------------
+__global__ void root_prologue_kernel(int kind, const float* __restrict__ A, int n, const int* __restrict__ valid,
+                                     float eps, int p, const float* __restrict__ s, float* __restrict__ out0,
+                                     float* __restrict__ out1, float* __restrict__ out2) {
+  __shared__ float t1[32][33];
+  __shared__ float t2[32][33];
+  const int i = blockIdx.z;
+  const int bi = blockIdx.y, bj = blockIdx.x;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const size_t nn = static_cast<size_t>(n) * n;
+  const float* a = A + i * nn;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    t1[ty + 8 * k][tx] = a[static_cast<size_t>(bi * 32 + ty + 8 * k) * n + bj * 32 + tx];
+    t2[ty + 8 * k][tx] = a[static_cast<size_t>(bj * 32 + ty + 8 * k) * n + bi * 32 + tx];
+  }
+  __syncthreads();
+  const int v = valid ? valid[i] : n;
+  const float inv_s = 1.f / s[i];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = bi * 32 + ty + 8 * k, c = bj * 32 + tx;
+    const float sym = 0.5f * (t1[ty + 8 * k][tx] + t2[tx][ty + 8 * k]);
+    const float d = (r == c) ? 1.f : 0.f;
+    const float m = (r < v && c < v) ? (sym + d * eps) * inv_s : d;
+    float t;
+    if (kind == 0)
+      t = (static_cast<float>(p + 1) * d - m) / static_cast<float>(p);
+    else
+      t = 0.5f * (3.f * d - m);
+    const size_t idx = static_cast<size_t>(r) * n + c;
+    store_split(out0, i, nn, idx, m);
+    store_split(out1, i, nn, idx, t);
+    store_split(out2, i, nn, idx, t);
+  }
+}
+
+// Second Newton-DB stage (p = 4): its input is the first stage's Y (~A'^{1/2},
+// spectrum in (0, 1]); Y0' = Y, T0 = (3 I - Y) / 2, Z1 = T0.  Elementwise.
+__global__ void db_stage2_kernel(const float* Y0, const float* Y1, const int* __restrict__ iters, int n,
+                                 float* Ynew0, float* __restrict__ T, float* __restrict__ Z1) {
+  const int i = blockIdx.y;
+  const size_t nn = static_cast<size_t>(n) * n;
+  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= nn) return;
+  const float* src = (iters[i] & 1) ? Y1 : Y0;
+  const float y = src[i * 2 * nn + idx] + src[i * 2 * nn + nn + idx];
+  const int r = static_cast<int>(idx / n), c = static_cast<int>(idx % n);
+  const float t = 0.5f * (3.f * ((r == c) ? 1.f : 0.f) - y);
+  store_split(Ynew0, i, nn, idx, y);
+  store_split(T, i, nn, idx, t);
+  store_split(Z1, i, nn, idx, t);
+}
+
+// Residual check after iteration `it`: ||acc - I||_F / sqrt(valid) <= tol
+// marks the matrix done (its later GEMM tiles are skipped).
+__global__ void check_kernel(float* res, int* done, int* iters, const int* valid, int batch, int n, float tol,
+                             int it, int* flags) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= batch) return;
+  if (done[i]) {
+    res[i] = 0.f;
+    return;
+  }
+  const int v = valid ? valid[i] : n;
+  const float r = sqrtf(res[i] / static_cast<float>(v));
+  res[i] = 0.f;
+  iters[i] = it;
+  if (!isfinite(r)) {
+    done[i] = 1;
+    raise_flag(flags, DEV_FLAG_NONFINITE);
+  } else if (r <= tol) {
+    done[i] = 1;
+  }
+}
+
+// Output pass: X = (hi + lo of the final iterate) * s^{-1/p}; the final iterate
+// sits in buffer (iters[i] & 1).  Writes a plain and/or a split stack.
+__global__ void finalize_kernel(const float* __restrict__ X0, const float* __restrict__ X1,
+                                const int* __restrict__ iters, int default_iters, const float* __restrict__ sc, int n,
+                                float* __restrict__ out_plain, float* __restrict__ out_split, int* flags) {
+  const int i = blockIdx.y;
+  const size_t nn = static_cast<size_t>(n) * n;
+  const size_t idx = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (idx >= nn) return;
+  const int it = iters ? iters[i] : default_iters;
+  const float* src = (it & 1) ? X1 : X0;
+  const float4 h = *reinterpret_cast<const float4*>(src + i * 2 * nn + idx);
+  const float4 l = *reinterpret_cast<const float4*>(src + i * 2 * nn + nn + idx);
+  const float f = sc[i];
+  float v[4] = {(h.x + l.x) * f, (h.y + l.y) * f, (h.z + l.z) * f, (h.w + l.w) * f};
+  bool bad = false;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) bad |= !isfinite(v[q]);
+  if (bad) raise_flag(flags, DEV_FLAG_NONFINITE);
+  if (out_plain) *reinterpret_cast<float4*>(out_plain + i * nn + idx) = make_float4(v[0], v[1], v[2], v[3]);
+  if (out_split) {
+    float hh[4], ll[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) split_tf32(v[q], hh[q], ll[q]);
+    *reinterpret_cast<float4*>(out_split + i * 2 * nn + idx) = make_float4(hh[0], hh[1], hh[2], hh[3]);
+    *reinterpret_cast<float4*>(out_split + i * 2 * nn + nn + idx) = make_float4(ll[0], ll[1], ll[2], ll[3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Chebyshev setup (DASH abstract names Chebyshev approximation; reading:
+// interpolation of x^{-1/p} on [a, 1] at first-kind Chebyshev points, with
+// a = lo / s, lo = cheb_lo if > 0 else eps, a >= 1 clamped to 1/2).
+// coef layout per matrix: c_0 .. c_d (c_0 halved), then a.  One CTA per matrix,
+// float64 arithmetic.
+// ---------------------------------------------------------------------------
+__global__ void cheb_coef_kernel(const float* __restrict__ s, int degree, int p, float eps, float lo,
+                                 float* __restrict__ coef, float* __restrict__ sc) {
+  const int i = blockIdx.x;
+  const double sv = s[i];
+  const double base = (lo > 0.f) ? static_cast<double>(lo) : static_cast<double>(eps);
+  double a = base / sv;
+  if (a >= 1.0) a = 0.5;
+  const int d = degree;
+  const double pi = 3.14159265358979323846;
+  float* ci = coef + static_cast<size_t>(i) * (d + 2);
+  for (int k = threadIdx.x; k <= d; k += blockDim.x) {
+    double acc = 0.0;
+    for (int j = 0; j <= d; ++j) {
+      const double th = pi * (j + 0.5) / (d + 1);
+      const double x = 0.5 * (1.0 - a) * cos(th) + 0.5 * (1.0 + a);
+      acc += pow(x, -1.0 / p) * cos(k * th);
+    }
+    acc *= 2.0 / (d + 1);
+    if (k == 0) acc *= 0.5;
+    ci[k] = static_cast<float>(acc);
+  }
+  if (threadIdx.x == 0) {
+    ci[d + 1] = static_cast<float>(a);
+    sc[i] = static_cast<float>(pow(sv, -1.0 / p));
+  }
+}
+
+// Xt = (2 A' - (1 + a) I) / (1 - a) on the valid region (identity on the pad),
+// b_d = c_d I and b_{d-1} = 2 c_d Xt + c_{d-1} I (first two Clenshaw terms).
+__global__ void cheb_prologue_kernel(const float* __restrict__ A, int n, const int* __restrict__ valid, float eps,
+                                     const float* __restrict__ s, const float* __restrict__ coef, int degree,
+                                     float* __restrict__ Xt, float* __restrict__ bd, float* __restrict__ bd1) {
+  __shared__ float t1[32][33];
+  __shared__ float t2[32][33];
+  const int i = blockIdx.z;
+  const int bi = blockIdx.y, bj = blockIdx.x;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const size_t nn = static_cast<size_t>(n) * n;
+  const float* a_in = A + i * nn;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    t1[ty + 8 * k][tx] = a_in[static_cast<size_t>(bi * 32 + ty + 8 * k) * n + bj * 32 + tx];
+    t2[ty + 8 * k][tx] = a_in[static_cast<size_t>(bj * 32 + ty + 8 * k) * n + bi * 32 + tx];
+  }
+  __syncthreads();
+  const int v = valid ? valid[i] : n;
+  const float inv_s = 1.f / s[i];
+  const float* ci = coef + static_cast<size_t>(i) * (degree + 2);
+  const float a = ci[degree + 1];
+  const float cd = ci[degree], cd1 = ci[degree - 1];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = bi * 32 + ty + 8 * k, c = bj * 32 + tx;
+    const float sym = 0.5f * (t1[ty + 8 * k][tx] + t2[tx][ty + 8 * k]);
+    const float d = (r == c) ? 1.f : 0.f;
+    const float m = (r < v && c < v) ? (sym + d * eps) * inv_s : d;
+    const float x = (2.f * m - (1.f + a) * d) / (1.f - a);
+    const size_t idx = static_cast<size_t>(r) * n + c;
+    store_split(Xt, i, nn, idx, x);
+    store_split(bd, i, nn, idx, cd * d);
+    store_split(bd1, i, nn, idx, 2.f * cd * x + cd1 * d);
+  }
+}
+
+__global__ void fill_int_kernel(int* p, int64_t count, int value) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < count) p[i] = value;
+}
+
+}  // namespace
+
+int launch_stack(const StackArgs& args, const int* d_table, int nb, int B, int grad_dtype, float* Gs, float* Gts,
+                 float** blk_wptr, int* blk_ld, cudaStream_t st, double alg_bytes) {
+  if (nb == 0) return 0;
+  ProfScope ps(K_STACK, st, 0.0, alg_bytes);
+  dim3 grid(B / 32, B / 32, nb), block(32, 8);
+  stack_split_kernel<<<grid, block, 0, st>>>(args, d_table, B, grad_dtype, Gs, Gts, blk_wptr, blk_ld);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "stack_split_kernel");
+}
+
+int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, float eps, int p, float* s, float* sc,
+                     cudaStream_t st) {
+  if (batch == 0) return 0;
+  ProfScope ps(K_NORM, st, 0.0, 4.0 * batch * n * n);
+  frob_norm_kernel<<<static_cast<unsigned>(batch), dim3(32, 16), 0, st>>>(A, n, valid, eps, 1.0 / p, s, sc);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "frob_norm_kernel");
+}
+
+int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const int* valid, float eps, int p,
+                         const float* s, float* out0, float* out1, float* out2, cudaStream_t st) {
+  if (batch == 0) return 0;
+  ProfScope ps(K_PROLOGUE, st, 0.0, (4.0 + 3 * 8.0) * batch * n * n);
+  dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
+  root_prologue_kernel<<<grid, block, 0, st>>>(kind, A, n, valid, eps, p, s, out0, out1, out2);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "root_prologue_kernel");
+}
+
+int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters, int64_t batch, int n, float* Ynew0,
+                              float* T, float* Z1, cudaStream_t st) {
+  if (batch == 0) return 0;
+  ProfScope ps(K_PROLOGUE, st, 0.0, (8.0 + 3 * 8.0) * batch * n * n);
+  const size_t nn = static_cast<size_t>(n) * n;
+  dim3 grid(static_cast<unsigned>((nn + 255) / 256), static_cast<unsigned>(batch));
+  db_stage2_kernel<<<grid, 256, 0, st>>>(Y0, Y1, iters, n, Ynew0, T, Z1);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "db_stage2_kernel");
+}
+
+int launch_check(float* res, int* done, int* iters, const int* valid, int64_t batch, int n, float tol, int it,
+                 int* flags, cudaStream_t st) {
+  if (batch == 0) return 0;
+  ProfScope ps(K_CHECK, st, 0.0, 16.0 * batch);
+  check_kernel<<<static_cast<unsigned>((batch + 255) / 256), 256, 0, st>>>(res, done, iters, valid,
+                                                                           static_cast<int>(batch), n, tol, it, flags);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "check_kernel");
+}
+
+int launch_finalize(const float* X0, const float* X1, const int* iters, int default_iters, const float* sc,
+                    int64_t batch, int n, float* out_plain, float* out_split, int* flags, cudaStream_t st) {
+  if (batch == 0) return 0;
+  const double bytes = (8.0 + (out_plain ? 4.0 : 0.0) + (out_split ? 8.0 : 0.0)) * batch * n * n;
+  ProfScope ps(K_FINALIZE, st, 0.0, bytes);
+  const size_t nn4 = static_cast<size_t>(n) * n / 4;
+  dim3 grid(static_cast<unsigned>((nn4 + 255) / 256), static_cast<unsigned>(batch));
+  finalize_kernel<<<grid, 256, 0, st>>>(X0, X1, iters, default_iters, sc, n, out_plain, out_split, flags);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "finalize_kernel");
+}
+
+int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int degree, float lo,
+                      const float* s, float* coef, float* sc, float* Xt, float* bd, float* bd1, cudaStream_t st) {
+  if (batch == 0) return 0;
+  {
+    ProfScope ps(K_CHEB_COEF, st, 0.0, 8.0 * batch);
+    cheb_coef_kernel<<<static_cast<unsigned>(batch), 128, 0, st>>>(s, degree, p, eps, lo, coef, sc);
+    count_launch();
+    int rc = check_cuda(cudaGetLastError(), "cheb_coef_kernel");
+    if (rc) return rc;
+  }
+  ProfScope ps(K_PROLOGUE, st, 0.0, (4.0 + 3 * 8.0) * batch * n * n);
+  dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
+  cheb_prologue_kernel<<<grid, block, 0, st>>>(A, n, valid, eps, s, coef, degree, Xt, bd, bd1);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "cheb_prologue_kernel");
+}
+
+int launch_fill_iters(int* iters, int64_t batch, int value, cudaStream_t st) {
+  if (batch == 0) return 0;
+  fill_int_kernel<<<static_cast<unsigned>((batch + 255) / 256), 256, 0, st>>>(iters, batch, value);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "fill_int_kernel");
+}
+
+}  // namespace shampoo
+
+namespace shampoo {
+namespace {
+
+// Per-matrix iteration report: out[i] = iterations (+ add[i]); negated when
+// the residual never reached tol (and DEV_FLAG_NOT_CONVERGED is raised).
+__global__ void report_kernel(const int* iters, const int* add, const int* done, int batch, int default_iters,
+                              int* out, int* flags, int residual) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= batch) return;
+  int it = iters ? iters[i] : default_iters;
+  if (add) it += add[i];
+  const bool failed = residual && done && !done[i];
+  if (failed) raise_flag(flags, DEV_FLAG_NOT_CONVERGED);
+  if (out) out[i] = failed ? -it : it;
+}
+
+// Plain stack -> split stack (hi / lo planes).
+__global__ void split_plain_kernel(const float* __restrict__ src, float* __restrict__ dst, int n) {
+  const int i = blockIdx.y;
+  const size_t nn = static_cast<size_t>(n) * n;
+  const size_t idx = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (idx >= nn) return;
+  const float4 v = *reinterpret_cast<const float4*>(src + i * nn + idx);
+  float h[4], l[4];
+  split_tf32(v.x, h[0], l[0]);
+  split_tf32(v.y, h[1], l[1]);
+  split_tf32(v.z, h[2], l[2]);
+  split_tf32(v.w, h[3], l[3]);
+  *reinterpret_cast<float4*>(dst + i * 2 * nn + idx) = make_float4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<float4*>(dst + i * 2 * nn + nn + idx) = make_float4(l[0], l[1], l[2], l[3]);
+}
+
+}  // namespace
+
+int launch_report(const int* iters, const int* add, const int* done, int64_t batch, int default_iters, int* out,
+                  int* flags, bool residual, cudaStream_t st) {
+  if (batch == 0) return 0;
+  ProfScope ps(K_CHECK, st, 0.0, 16.0 * batch);
+  report_kernel<<<static_cast<unsigned>((batch + 255) / 256), 256, 0, st>>>(
+      iters, add, done, static_cast<int>(batch), default_iters, out, flags, residual ? 1 : 0);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "report_kernel");
+}
+
+int launch_split_plain(const float* src, float* dst, int64_t batch, int n, cudaStream_t st) {
+  if (batch == 0) return 0;
+  ProfScope ps(K_PROLOGUE, st, 0.0, 12.0 * batch * n * n);
+  const size_t nn4 = static_cast<size_t>(n) * n / 4;
+  dim3 grid(static_cast<unsigned>((nn4 + 255) / 256), static_cast<unsigned>(batch));
+  split_plain_kernel<<<grid, 256, 0, st>>>(src, dst, n);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "split_plain_kernel");
+}
+
+}  // namespace shampoo

@@ -1,0 +1,301 @@
+// Batched inverse p-th roots X_i ~ (A_i + eps I)^{-1/p} of stacked symmetric
+// matrices: host-side driver of the tensor-core GEMM and the prologue /
+// check / output kernels.
+//
+// The pages name the solvers (DASH abstract: Newton-DB iteration and Chebyshev
+// polynomial approximation for inverse matrix roots; matrix scaling) without
+// defining them.  The iterations implemented here are published methods:
+//   coupled Newton  (Guo & Higham 2006): X0 = I, M0 = A'; T = ((p+1) I - M)/p;
+//                   X <- X T; M <- T^p M   (4 GEMMs per iteration for p = 4,
+//                   3 for p = 2);
+//   Newton-DB       coupled Denman-Beavers-family square-root iteration in its
+//                   multiplication-only form: Y0 = A', Z0 = I;
+//                   T = (3 I - Z Y)/2; Y <- Y T; Z <- T Z (3 GEMMs); p = 4 runs
+//                   a second stage on Y ~ A'^{1/2};
+//   Chebyshev       Clenshaw evaluation of the degree-d interpolant of x^{-1/p}
+//                   on [a, 1] (d - 1 GEMMs).
+// Every product is a true product A B (B read MN-major): with the implicit
+// transpose of a K-major B, rounding makes the iterates slightly unsymmetric
+// and the Newton-DB fixed point is unstable along that direction.
+// A' = (A + eps I)/||A + eps I||_F (Frobenius pre-scaling); the result is
+// unscaled by ||A + eps I||_F^{-1/p}.  With tol > 0 the residual
+// ||M - I||_F / sqrt(n) (Newton) or ||Z Y - I||_F / sqrt(n) (Newton-DB) is
+// checked after every iteration and converged matrices drop out of later
+// launches (their tiles exit at once); iters is then the cap.
+#include <algorithm>
+#include <cstring>
+#include <vector>
+
+#include "internal.h"
+
+namespace shampoo {
+namespace {
+
+int stacks_for(int solver) {
+  switch (solver) {
+    case 0: return 7;  // M0 M1 X0 X1 T T2 T4
+    case 1: return 5;  // Y0 Y1 Z0 Z1 T
+    default: return 4; // Xt b0 b1 b2
+  }
+}
+
+constexpr size_t kAlign = 256;
+constexpr size_t kHeader = 64 * 1024;  // covers the alignment padding of the arrays
+constexpr int kVecInts = 6;            // s sc res done iters iters1
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  float* s;
+  float* sc;
+  float* res;
+  int* done;
+  int* iters;
+  int* iters1;
+  float* coef;
+  float* stack[7];
+};
+
+Layout carve(void* base, int64_t cb, int n, int solver) {
+  Layout L;
+  std::memset(&L, 0, sizeof(L));
+  char* p = static_cast<char*>(base);
+  auto take = [&](size_t bytes) {
+    char* r = p;
+    p += align_up(bytes);
+    return r;
+  };
+  L.s = reinterpret_cast<float*>(take(cb * 4));
+  L.sc = reinterpret_cast<float*>(take(cb * 4));
+  L.res = reinterpret_cast<float*>(take(cb * 4));
+  L.done = reinterpret_cast<int*>(take(cb * 4));
+  L.iters = reinterpret_cast<int*>(take(cb * 4));
+  L.iters1 = reinterpret_cast<int*>(take(cb * 4));
+  L.coef = reinterpret_cast<float*>(take(cb * 4 * (kMaxChebDegree + 2)));
+  for (int k = 0; k < stacks_for(solver); ++k) L.stack[k] = reinterpret_cast<float*>(take(split_floats(cb, n) * 4));
+  return L;
+}
+
+}  // namespace
+
+size_t root_scratch_header() { return kHeader; }
+
+size_t root_scratch_per_matrix(int n, int solver) {
+  return static_cast<size_t>(stacks_for(solver)) * split_floats(1, n) * 4 + 4 * (kVecInts + kMaxChebDegree + 2);
+}
+
+int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, cudaStream_t st) {
+  const int n = job.n;
+  const int p = job.p;
+  const bool residual = job.tol > 0.f && job.solver != 2;
+  const size_t per = root_scratch_per_matrix(n, job.solver);
+  if (scratch_bytes < kHeader + per) return set_error(-3, "inverse-root scratch too small: %zu < %zu bytes",
+                                                      scratch_bytes, kHeader + per);
+  const int64_t cb_max = std::min<int64_t>(job.batch, static_cast<int64_t>((scratch_bytes - kHeader) / per));
+  const int64_t cb_cap = std::min<int64_t>(cb_max, 65535);  // grid.z limit of the prologues
+  const double f1 = 2.0 * n * static_cast<double>(n) * n;  // one GEMM(n), algorithmic
+  int rc = 0;
+  for (int64_t off = 0; off < job.batch; off += cb_cap) {
+    const int64_t cb = std::min<int64_t>(cb_cap, job.batch - off);
+    const int cbi = static_cast<int>(cb);
+    Layout S = carve(scratch, cb, n, job.solver);
+    const float* A = job.A + off * static_cast<int64_t>(n) * n;
+    const int* valid = job.valid ? job.valid + off : nullptr;
+    float* out_plain = job.X_plain ? job.X_plain + off * static_cast<int64_t>(n) * n : nullptr;
+    float* out_split = job.X_split ? job.X_split + off * 2 * static_cast<int64_t>(n) * n : nullptr;
+    int* iters_out = job.iters_used ? job.iters_used + off : nullptr;
+    StackMaps sm[7];
+    for (int k = 0; k < stacks_for(job.solver); ++k)
+      if ((rc = make_stack_maps(sm[k], S.stack[k], cb, n))) return rc;
+    if ((rc = launch_frob_norm(A, cb, n, valid, job.eps, p, S.s, S.sc, st))) return rc;
+    if (residual) {
+      if ((rc = check_cuda(cudaMemsetAsync(S.done, 0, cb * 4, st), "memset done"))) return rc;
+      if ((rc = check_cuda(cudaMemsetAsync(S.res, 0, cb * 4, st), "memset res"))) return rc;
+    }
+    const int* skip = residual ? S.done : nullptr;
+
+    if (job.solver == 0) {
+      // ------------------------------------------------------------ coupled Newton
+      StackMaps* M = &sm[0];  // M[0], M[1]
+      StackMaps* X = &sm[2];  // X[0], X[1]
+      StackMaps& T = sm[4];
+      StackMaps& T2 = sm[5];
+      StackMaps& T4 = sm[6];
+      if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, M[0].base, T.base, X[1].base, st)))
+        return rc;
+      for (int j = 0; j < job.iters; ++j) {
+        {
+          Builder b;
+          Epilogue& e = b.add(cbi, n, T, 0, T, 0, f1, 1);
+          e.D = T2.base;
+          e.d_split = 1;
+          e.skip = skip;
+          e.flags = job.flags;
+          if (j >= 1) {
+            Epilogue& ex = b.add(cbi, n, X[j & 1], 0, T, 0, f1, 1);
+            ex.D = X[(j + 1) & 1].base;
+            ex.d_split = 1;
+            ex.skip = skip;
+            ex.flags = job.flags;
+          }
+          if ((rc = b.launch(st))) return rc;
+        }
+        if (!residual && j == job.iters - 1) break;
+        StackMaps* P = &T2;
+        if (p == 4) {
+          Builder b;
+          Epilogue& e = b.add(cbi, n, T2, 0, T2, 0, f1, 1);
+          e.D = T4.base;
+          e.d_split = 1;
+          e.skip = skip;
+          e.flags = job.flags;
+          if ((rc = b.launch(st))) return rc;
+          P = &T4;
+        }
+        {
+          Builder b;
+          Epilogue& e = b.add(cbi, n, *P, 0, M[j & 1], 0, f1, 1);
+          e.D = M[(j + 1) & 1].base;
+          e.d_split = 1;
+          e.E = T.base;
+          e.e_mul = -1.f / p;
+          e.e_add = static_cast<float>(p + 1) / p;
+          e.res = residual ? S.res : nullptr;
+          e.valid = valid;
+          e.skip = skip;
+          e.flags = job.flags;
+          if ((rc = b.launch(st))) return rc;
+        }
+        if (residual &&
+            (rc = launch_check(S.res, S.done, S.iters, valid, cb, n, job.tol, j + 1, job.flags, st)))
+          return rc;
+      }
+      if ((rc = launch_finalize(X[0].base, X[1].base, residual ? S.iters : nullptr, job.iters, S.sc, cb, n, out_plain,
+                                out_split, job.flags, st)))
+        return rc;
+      if (iters_out && (rc = launch_report(residual ? S.iters : nullptr, nullptr, residual ? S.done : nullptr, cb,
+                                           job.iters, iters_out, job.flags, residual, st)))
+        return rc;
+      if (!iters_out && residual &&
+          (rc = launch_report(S.iters, nullptr, S.done, cb, job.iters, nullptr, job.flags, residual, st)))
+        return rc;
+    } else if (job.solver == 1) {
+      // ------------------------------------------------------------ Newton-DB
+      StackMaps* Y = &sm[0];
+      StackMaps* Z = &sm[2];
+      StackMaps& T = sm[4];
+      if ((rc = launch_root_prologue(1, A, cb, n, valid, job.eps, p, S.s, Y[0].base, T.base, Z[1].base, st)))
+        return rc;
+      const int stages = (p == 4) ? 2 : 1;
+      for (int stage = 0; stage < stages; ++stage) {
+        if (stage == 1) {
+          // Stage-1 results: Y_final at parity iters1; its square root seeds stage 2.
+          if (residual) {
+            // Flags stage-1 matrices that reached the cap (per-matrix signs report stage 2).
+            if ((rc = launch_report(S.iters, nullptr, S.done, cb, job.iters, nullptr, job.flags, true, st))) return rc;
+            if ((rc = check_cuda(cudaMemcpyAsync(S.iters1, S.iters, cb * 4, cudaMemcpyDeviceToDevice, st),
+                                 "copy iters")))
+              return rc;
+            if ((rc = check_cuda(cudaMemsetAsync(S.done, 0, cb * 4, st), "memset done"))) return rc;
+            if ((rc = check_cuda(cudaMemsetAsync(S.res, 0, cb * 4, st), "memset res"))) return rc;
+          } else {
+            if ((rc = launch_fill_iters(S.iters1, cb, job.iters, st))) return rc;
+          }
+          if ((rc = launch_db_stage2_prologue(Y[0].base, Y[1].base, S.iters1, cb, n, Y[0].base, T.base, Z[1].base,
+                                              st)))
+            return rc;
+        }
+        for (int j = 0; j < job.iters; ++j) {
+          {
+            Builder b;
+            Epilogue& ey = b.add(cbi, n, Y[j & 1], 0, T, 0, f1, 1);
+            ey.D = Y[(j + 1) & 1].base;
+            ey.d_split = 1;
+            ey.skip = skip;
+            ey.flags = job.flags;
+            if (j >= 1) {
+              Epilogue& ez = b.add(cbi, n, T, 0, Z[j & 1], 0, f1, 1);
+              ez.D = Z[(j + 1) & 1].base;
+              ez.d_split = 1;
+              ez.skip = skip;
+              ez.flags = job.flags;
+            }
+            if ((rc = b.launch(st))) return rc;
+          }
+          if (!residual && j == job.iters - 1) break;
+          {
+            Builder b;
+            Epilogue& e = b.add(cbi, n, Z[(j + 1) & 1], 0, Y[(j + 1) & 1], 0, f1, 1);
+            e.alpha = -0.5f;
+            e.gamma = 1.5f;
+            e.D = T.base;
+            e.d_split = 1;
+            e.res = residual ? S.res : nullptr;
+            e.valid = valid;
+            e.skip = skip;
+            e.flags = job.flags;
+            if ((rc = b.launch(st))) return rc;
+          }
+          if (residual &&
+              (rc = launch_check(S.res, S.done, S.iters, valid, cb, n, job.tol, j + 1, job.flags, st)))
+            return rc;
+        }
+      }
+      if ((rc = launch_finalize(Z[0].base, Z[1].base, residual ? S.iters : nullptr, job.iters, S.sc, cb, n, out_plain,
+                                out_split, job.flags, st)))
+        return rc;
+      const int* add = (p == 4) ? S.iters1 : nullptr;
+      if (p == 4 && !residual) add = nullptr;
+      const int default_total = (p == 4) ? 2 * job.iters : job.iters;
+      if ((iters_out || residual) &&
+          (rc = launch_report(residual ? S.iters : nullptr, residual ? add : nullptr, residual ? S.done : nullptr, cb,
+                              default_total, iters_out, job.flags, residual, st)))
+        return rc;
+    } else {
+      // ------------------------------------------------------------ Chebyshev
+      const int d = job.cheb_degree;
+      StackMaps& Xt = sm[0];
+      StackMaps* b = &sm[1];  // b[k % 3]
+      if ((rc = launch_cheb_setup(A, cb, n, valid, job.eps, p, d, job.cheb_lo, S.s, S.coef, S.sc, Xt.base,
+                                  b[d % 3].base, b[(d - 1) % 3].base, st)))
+        return rc;
+      for (int k = d - 2; k >= 1; --k) {
+        Builder bl;
+        Epilogue& e = bl.add(cbi, n, Xt, 0, b[(k + 1) % 3], 0, f1, 1);
+        e.alpha = 2.f;
+        e.beta = -1.f;
+        e.C = b[(k + 2) % 3].base;
+        e.c_split = 1;
+        e.gamma_vec = S.coef + k;
+        e.gamma_stride = d + 2;
+        e.D = b[k % 3].base;
+        e.d_split = 1;
+        e.flags = job.flags;
+        if ((rc = bl.launch(st))) return rc;
+      }
+      {
+        Builder bl;
+        Epilogue& e = bl.add(cbi, n, Xt, 0, b[1], 0, f1, 1);
+        e.alpha = 1.f;
+        e.beta = -1.f;
+        e.C = b[2].base;
+        e.c_split = 1;
+        e.gamma_vec = S.coef;
+        e.gamma_stride = d + 2;
+        e.scale_vec = S.sc;
+        if (out_split) {
+          e.D = out_split;
+          e.d_split = 1;
+        } else {
+          e.D = out_plain;
+          e.d_split = 0;
+        }
+        e.flags = job.flags;
+        if ((rc = bl.launch(st))) return rc;
+      }
+      if (iters_out && (rc = launch_fill_iters(iters_out, cb, d, st))) return rc;
+    }
+  }
+  return 0;
+}
+
+}  // namespace shampoo

@@ -1,0 +1,117 @@
+"""C-ABI boundary without a GPU: the library loads, exports every symbol that
+include/shampoo.h declares, and its host-only entry points validate
+arguments and compute sizes (no CUDA call is made by these)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def sb():
+    import shampoo_family_second_b200 as sb
+    return sb
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "shampoo.h")).read()
+    return re.findall(r"^SHAMPOO_API [^(]*?\b(\w+)\(", text, flags=re.M)
+
+
+def test_library_exports_every_declared_symbol(sb):
+    declared = header_functions()
+    assert len(declared) >= 15
+    lib = ctypes.CDLL(sb.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert tuple(declared) == sb.EXPORTS
+
+
+def test_status_strings(sb):
+    assert sb.lib.shampoo_status_string(0) == b"SHAMPOO_OK"
+    assert sb.lib.shampoo_status_string(-3) == b"SHAMPOO_ERR_WORKSPACE"
+    assert sb.lib.shampoo_status_string(12345) == b"SHAMPOO_UNKNOWN_STATUS"
+
+
+def test_query_sizes_memory_is_quadratic_per_block(sb):
+    """One B x B statistic per side per block (notes' "Key Components":
+    O(m^2 + n^2) memory): state = stats (2 nb B^2 fp32) + split roots
+    (2 nb 2 B^2 fp32) + a small table."""
+    for name in ("tiny", "lowrank", "gpt2", "llama"):
+        wl = workloads.workload(name)
+        cfg = sb.config_from_workload(wl)
+        state, scratch = sb.query_sizes(cfg, wl.shapes)
+        nb = len(oracle.block_table(wl.shapes, wl.block))
+        core = 2 * nb * wl.block ** 2 * 4 * 3
+        assert core <= state <= core + 64 * 1024 + 64 * nb
+        assert scratch > 3 * 2 * nb * wl.block ** 2 * 4
+
+
+@pytest.mark.parametrize("field,value", [("block", 48), ("block", 2048), ("root_p", 3), ("solver", 7),
+                                         ("iters", 0), ("refresh_every", 0), ("beta", 1.5), ("eps", -1.0),
+                                         ("grad_dtype", 5)])
+def test_config_validation(sb, field, value):
+    cfg = sb.make_config(32, 1.0, 1e-6, 1e-3)
+    setattr(cfg, field, value)
+    with pytest.raises(sb.ShampooError) as e:
+        sb.query_sizes(cfg, [(64, 32)])
+    assert e.value.code == sb.ERR_INVALID_ARG
+    assert sb.last_error()
+
+
+def test_chebyshev_needs_interval(sb):
+    cfg = sb.make_config(32, 1.0, 0.0, 1e-3, solver=sb.SOLVER_CHEBYSHEV, cheb_degree=16, cheb_lo=0.0)
+    with pytest.raises(sb.ShampooError):
+        sb.query_sizes(cfg, [(64, 32)])
+    cfg.cheb_degree = 1
+    cfg.eps = 1e-3
+    with pytest.raises(sb.ShampooError):
+        sb.query_sizes(cfg, [(64, 32)])
+
+
+def test_bad_shapes(sb):
+    cfg = sb.make_config(32, 1.0, 1e-6, 1e-3)
+    with pytest.raises(sb.ShampooError):
+        sb.query_sizes(cfg, [(0, 32)])
+    with pytest.raises(sb.ShampooError):
+        sb.query_sizes(cfg, [])
+
+
+def test_inv_root_argument_errors_before_any_launch(sb):
+    L = sb.lib
+    n0 = sb.launch_count()
+    # NULL pointers, bad n, bad p: all rejected on the host.
+    assert L.inv_root_batched(None, None, 4, 64, 4, 0.0, 0, 10, 0.0, 16, 0.0, None, 0, None, None, None) == -1
+    assert L.inv_root_batched(1024, 1024, 4, 65, 4, 0.0, 0, 10, 0.0, 16, 0.0, 4096, 1 << 20, None, None, None) == -1
+    assert L.inv_root_batched(1024, 1024, 4, 64, 3, 0.0, 0, 10, 0.0, 16, 0.0, 4096, 1 << 20, None, None, None) == -1
+    assert L.inv_root_batched(1024, 1024, 4, 64, 4, 0.0, 0, 0, 0.0, 16, 0.0, 4096, 1 << 20, None, None, None) == -1
+    assert L.inv_root_batched(1024, 1024, 0, 64, 4, 0.0, 0, 10, 0.0, 16, 0.0, 4096, 1 << 20, None, None, None) == 0
+    assert sb.launch_count() == n0
+
+
+def test_scratch_sizes(sb):
+    a = sb.inv_root_scratch_bytes(64, 1024, sb.SOLVER_NEWTON)
+    b = sb.inv_root_scratch_bytes(128, 1024, sb.SOLVER_NEWTON)
+    per = b - a
+    assert per == 64 * (7 * 2 * 1024 * 1024 * 4 + 4 * (6 + 64 + 2))
+    assert sb.inv_root_scratch_bytes(64, 1024, sb.SOLVER_NEWTON_DB) < a
+    assert sb.gemm_scratch_bytes(3, 256) == 2 * 3 * 2 * 256 * 256 * 4
+    with pytest.raises(sb.ShampooError):
+        sb.inv_root_scratch_bytes(4, 100, 0)
+
+
+def test_init_rejects_missing_buffers_without_cuda(sb):
+    cfg = sb.make_config(32, 1.0, 1e-6, 1e-3)
+    rows = (ctypes.c_int64 * 1)(64)
+    cols = (ctypes.c_int64 * 1)(32)
+    h = ctypes.c_void_p()
+    assert sb.lib.shampoo_init(ctypes.byref(cfg), 1, rows, cols, None, 0, None, 0, None, ctypes.byref(h)) == -1
+    assert sb.lib.shampoo_init(ctypes.byref(cfg), 1, rows, cols, 256, 0, 512, 0, None, ctypes.byref(h)) == -3
+    assert sb.lib.shampoo_init(ctypes.byref(cfg), 1, rows, cols, 255, 1 << 30, 512, 1 << 30, None,
+                               ctypes.byref(h)) == -2

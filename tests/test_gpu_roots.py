@@ -1,0 +1,98 @@
+"""Batched inverse p-th roots on the GPU vs the float64 oracle.
+
+Inputs: SPD stacks Q diag(lam) Q^T with an exact condition number (the solver
+sweep's recipe), cast to fp32; the oracle takes the same fp32 values.
+Gates: relative Frobenius error per root <= 2e-3 against the exact root for
+coupled Newton and Newton-DB where the fp32 conditioning floor allows it
+(kappa <= 1e4); Chebyshev against the float64 Clenshaw evaluation of the same
+polynomial (its distance to the exact root is a property of the degree).
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle
+from oracle import chebyshev as och
+import workloads
+from parity import root_gate
+
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def sb():
+    import shampoo_family_second_b200 as sb
+    return sb
+
+
+def run(sb, A32, **kw):
+    X, it, st = sb.inv_root_batched(torch.from_numpy(A32).cuda(), **kw)
+    torch.cuda.synchronize()
+    return X.cpu().numpy().astype(np.float64), it.cpu().numpy(), int(st.item())
+
+
+@pytest.mark.parametrize("n,batch", [(64, 4), (256, 3), (384, 2)])
+@pytest.mark.parametrize("p", [2, 4])
+@pytest.mark.parametrize("kappa", [1e2, 1e4])
+def test_newton_fixed(sb, n, batch, p, kappa):
+    A32 = workloads.spd_batch(batch, n, kappa, seed=n + p).astype(np.float32)
+    X, it, st = run(sb, A32, p=p, eps=0.0, solver=sb.SOLVER_NEWTON, iters=30, tol=0.0)
+    assert st == 0
+    assert np.all(it == 30)
+    for b in range(batch):
+        A = A32[b].astype(np.float64)
+        ref = oracle.inverse_root(A, p, 0.0)
+        assert oracle.rel_fro(X[b], ref) < root_gate(A, p, 0.0), (b, oracle.rel_fro(X[b], ref))
+
+
+@pytest.mark.parametrize("p", [2, 4])
+def test_newton_residual_mode(sb, p):
+    A32 = workloads.spd_batch(4, 128, 1e3, seed=5).astype(np.float32)
+    X, it, st = run(sb, A32, p=p, eps=1e-6, solver=sb.SOLVER_NEWTON, iters=40, tol=1e-5)
+    assert st == 0
+    assert np.all(it > 0) and np.all(it < 40)
+    for b in range(4):
+        ref = oracle.inverse_root(A32[b].astype(np.float64), p, 1e-6)
+        assert oracle.rel_fro(X[b], ref) < TOL
+
+
+@pytest.mark.parametrize("p", [2, 4])
+@pytest.mark.parametrize("tol", [0.0, 1e-5])
+def test_newton_db(sb, p, tol):
+    A32 = workloads.spd_batch(3, 256, 1e3, seed=9).astype(np.float32)
+    X, it, st = run(sb, A32, p=p, eps=0.0, solver=sb.SOLVER_NEWTON_DB, iters=30, tol=tol)
+    assert st == 0
+    for b in range(3):
+        ref = oracle.inverse_root(A32[b].astype(np.float64), p, 0.0)
+        assert oracle.rel_fro(X[b], ref) < TOL, oracle.rel_fro(X[b], ref)
+
+
+@pytest.mark.parametrize("p", [2, 4])
+@pytest.mark.parametrize("degree", [16, 32])
+def test_chebyshev_polynomial_parity(sb, p, degree):
+    kappa = 1e2
+    A32 = workloads.spd_batch(3, 256, kappa, seed=11).astype(np.float32)
+    lo = 0.999 / kappa                       # lower spectral bound of A (lam_min = 1/kappa)
+    X, it, st = run(sb, A32, p=p, eps=0.0, solver=sb.SOLVER_CHEBYSHEV, cheb_degree=degree, cheb_lo=lo)
+    assert st == 0
+    assert np.all(it == degree)
+    for b in range(3):
+        ref = och.chebyshev_inverse_root(A32[b].astype(np.float64), p, 0.0, degree, lo=lo)
+        assert oracle.rel_fro(X[b], ref) < TOL, oracle.rel_fro(X[b], ref)
+
+
+def test_not_converged_flag(sb):
+    A32 = workloads.spd_batch(2, 64, 1e6, seed=13).astype(np.float32)
+    X, it, st = run(sb, A32, p=4, eps=0.0, solver=sb.SOLVER_NEWTON, iters=2, tol=1e-6)
+    assert st & sb.DEVFLAG_NOT_CONVERGED
+    assert np.all(it == -2)
+
+
+def test_nonfinite_flag(sb):
+    A32 = workloads.spd_batch(2, 64, 1e2, seed=14).astype(np.float32)
+    A32[1, 3, 5] = np.nan
+    X, it, st = run(sb, A32, p=4, eps=0.0, solver=sb.SOLVER_NEWTON, iters=5, tol=0.0)
+    assert st & sb.DEVFLAG_NONFINITE
+    assert np.all(np.isfinite(X[0]))

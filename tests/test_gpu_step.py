@@ -1,0 +1,181 @@
+"""The full blocked Shampoo step on the GPU vs the float64 oracle.
+
+Per step and per block: statistics (GPU fp32 L, R vs the float64 oracle's,
+1e-5 relative Frobenius), roots (the GPU roots vs the oracle's exact root of
+the GPU's own fp32 statistics: isolates the solver from fp32 statistics
+rounding), and the update P_b = -(W_t - W_{t-1}) / lr against the fully
+float64 pipeline, <= 2e-3 relative Frobenius per block.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle
+import workloads
+from parity import root_gate
+
+TOL_UPDATE = 2e-3
+TOL_ROOT = 2e-3
+TOL_STATS = 1e-5
+
+
+@pytest.fixture(scope="module")
+def sb():
+    import shampoo_family_second_b200 as sb
+    return sb
+
+
+def bf16_tensor(x32):
+    return torch.from_numpy(workloads.bf16_bits(x32).view(np.int16)).view(torch.bfloat16)
+
+
+def run_parity(sb, wl, steps, check_roots=True, blocks=None):
+    cfg = sb.config_from_workload(wl)
+    opt = sb.Shampoo(wl.shapes, cfg)
+    W = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    ref = oracle.ShampooOracle(wl.shapes, wl.block, wl.beta, wl.eps, wl.lr, wl.root_p, wl.refresh_every,
+                               blocks=blocks)
+    table = opt.block_table()
+    assert [tuple(t) for t in table] == [(b.param, b.row0, b.col0, b.r, b.c) for b in ref.table]
+    stream = workloads.GradientStream(wl)
+    worst = {"update": 0.0, "root": 0.0, "stats": 0.0}
+    for t in range(steps):
+        grads = stream.next()
+        if wl.grad_dtype == workloads.DTYPE_BF16:
+            G = [bf16_tensor(g).cuda() for g in grads]
+        else:
+            G = [torch.from_numpy(g).cuda() for g in grads]
+        before = [w.clone() for w in W]
+        opt.step(W, G)
+        P_ref = ref.step(grads)
+        torch.cuda.synchronize()
+        dW = [((b - a) / wl.lr).cpu().numpy().astype(np.float64) for a, b in zip(W, before)]
+        L, R = opt.statistics()
+        L, R = L.cpu().numpy().astype(np.float64), R.cpu().numpy().astype(np.float64)
+        if check_roots and t % wl.refresh_every == 0:
+            XL, XR = opt.roots()
+            XL, XR = XL.cpu().numpy().astype(np.float64), XR.cpu().numpy().astype(np.float64)
+        for b in ref.active:
+            blk = ref.table[b]
+            Pg = dW[blk.param][blk.row0:blk.row0 + blk.r, blk.col0:blk.col0 + blk.c]
+            e = oracle.rel_fro(Pg, P_ref[b])
+            worst["update"] = max(worst["update"], e)
+            assert e < TOL_UPDATE, (t, b, "update", e)
+            es = max(oracle.rel_fro(L[b, :blk.r, :blk.r], ref.L[b]), oracle.rel_fro(R[b, :blk.c, :blk.c], ref.R[b]))
+            worst["stats"] = max(worst["stats"], es)
+            assert es < TOL_STATS, (t, b, "stats", es)
+            if check_roots and t % wl.refresh_every == 0:
+                for X, S, v in ((XL, L, blk.r), (XR, R, blk.c)):
+                    xr = oracle.inverse_root(S[b, :v, :v], wl.root_p, wl.eps)
+                    er = oracle.rel_fro(X[b, :v, :v], xr)
+                    worst["root"] = max(worst["root"], er)
+                    assert er < root_gate(S[b, :v, :v], wl.root_p, wl.eps), (t, b, "root", er)
+    assert opt.status() == 0
+    return worst
+
+
+def test_tiny_workload(sb):
+    """Tiny: one 64x32 weight, block 32, 10 steps, beta = 1, Newton 20 iterations."""
+    wl = workloads.workload("tiny")
+    run_parity(sb, wl, wl.steps)
+
+
+@pytest.mark.parametrize("shapes", [((33, 47),), ((64, 45), (20, 96)), ((100, 33),)])
+def test_ragged_blocks(sb, shapes):
+    wl = workloads.workload("tiny", shapes=shapes, steps=4, iters=40, tol=1e-6, beta=0.9, eps=1e-4)
+    run_parity(sb, wl, wl.steps)
+
+
+@pytest.mark.parametrize("solver", [1, 2])
+def test_other_solvers_in_step(sb, solver):
+    # Chebyshev needs a spectral lower bound: eps large enough that a = eps / s
+    # keeps the degree-32 interpolant within tolerance.
+    over = dict(solver=solver, iters=30, tol=0.0)
+    if solver == 2:
+        over.update(eps=1.0, cheb_degree=32, cheb_lo=0.0)
+    wl = workloads.workload("tiny", steps=3, **over)
+    cfg = sb.config_from_workload(wl)
+    opt = sb.Shampoo(wl.shapes, cfg)
+    W = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    stream = workloads.GradientStream(wl)
+    from oracle import chebyshev as och
+    for t in range(wl.steps):
+        G = stream.next()
+        opt.step(W, [torch.from_numpy(g).cuda() for g in G])
+        torch.cuda.synchronize()
+        L, R = opt.statistics()
+        XL, XR = opt.roots()
+        L, R, XL, XR = [x.cpu().numpy().astype(np.float64) for x in (L, R, XL, XR)]
+        for b in range(opt.nb):
+            for X, S in ((XL, L), (XR, R)):
+                if solver == 2:
+                    ref = och.chebyshev_inverse_root(S[b], wl.root_p, wl.eps, wl.cheb_degree, lo=0.0)
+                else:
+                    ref = oracle.inverse_root(S[b], wl.root_p, wl.eps)
+                assert oracle.rel_fro(X[b], ref) < TOL_ROOT
+    assert opt.status() == 0
+
+
+def test_p2_step(sb):
+    wl = workloads.workload("tiny", root_p=2, steps=3, iters=30)
+    run_parity(sb, wl, wl.steps)
+
+
+def test_bf16_gradients(sb):
+    wl = workloads.workload("tiny", shapes=((64, 96),), grad_dtype=workloads.DTYPE_BF16, steps=3, iters=30)
+    run_parity(sb, wl, wl.steps)
+
+
+def test_refresh_schedule(sb):
+    wl = workloads.workload("tiny", steps=7, refresh_every=3, iters=30, beta=0.9)
+    run_parity(sb, wl, wl.steps)
+
+
+def test_checkpoint_resume_bit_identical(sb):
+    wl = workloads.workload("tiny", shapes=((64, 96),), steps=6, iters=25)
+    cfg = sb.config_from_workload(wl)
+    grads = [[torch.from_numpy(g).cuda() for g in gs]
+             for gs in (workloads.GradientStream(wl).next() for _ in range(1))]
+    stream = workloads.GradientStream(wl)
+    grads = [[torch.from_numpy(g).cuda() for g in stream.next()] for _ in range(wl.steps)]
+    a = sb.Shampoo(wl.shapes, cfg)
+    Wa = [torch.zeros(s, device="cuda") for s in wl.shapes]
+    for t in range(wl.steps):
+        a.step(Wa, grads[t])
+        if t == 2:
+            ckpt = a.state_dict()
+            Wckpt = [w.clone() for w in Wa]
+    b = sb.Shampoo(wl.shapes, cfg)
+    b.load_state_dict(ckpt)
+    Wb = Wckpt
+    for t in range(3, wl.steps):
+        b.step(Wb, grads[t])
+    torch.cuda.synchronize()
+    for x, y in zip(Wa, Wb):
+        assert torch.equal(x, y)
+    assert b.step_count == a.step_count == wl.steps
+
+
+def test_nonfinite_gradient_sets_status(sb):
+    wl = workloads.workload("tiny", steps=1)
+    opt = sb.Shampoo(wl.shapes, sb.config_from_workload(wl))
+    W = [torch.zeros(s, device="cuda") for s in wl.shapes]
+    g = torch.randn(wl.shapes[0], device="cuda")
+    g[5, 7] = float("inf")
+    opt.step(W, [g])
+    st = opt.status(reset=True)
+    assert st & sb.DEVFLAG_NONFINITE
+    assert opt.status() == 0
+
+
+def test_launch_count_increases(sb):
+    wl = workloads.workload("tiny", steps=1)
+    opt = sb.Shampoo(wl.shapes, sb.config_from_workload(wl))
+    W = [torch.zeros(s, device="cuda") for s in wl.shapes]
+    n0 = sb.launch_count()
+    opt.step(W, [torch.randn(wl.shapes[0], device="cuda")])
+    torch.cuda.synchronize()
+    # stack + stats + norm + prologue + 20 + 19 * 2 Newton launches + finalize + 2 apply
+    assert sb.launch_count() - n0 == 1 + 1 + 1 + 1 + 20 + 19 * 2 + 1 + 2
