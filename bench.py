@@ -1,0 +1,583 @@
+"""Benchmark of the blocked Shampoo step on B200 GPUs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path (stack -> statistics -> inverse roots
+when the step is a refresh step -> apply + update) over one batch of synthetic
+gradients, through the C ABI (libshampoo.so).  Default workload: 4 fp32
+matrices 1024 x 1024, block 256 (64 blocks -> 128 roots per refresh), low-rank
++ noise gradients, beta 0.95, eps 1e-8, roots refreshed every 10 steps.
+
+Metric: inverse roots per second of the whole job (all ranks), with the mean
+step time beside it.  Timing: W untimed warm-up steps, then K steps, each
+between two CUDA events on the launching stream, with a 256 MiB L2 flush
+between steps outside the events; barrier + synchronize around the timed
+region; max over ranks.  Multi-GPU runs are weak-scaled replicas: every rank
+runs its own copy of the workload (blocks are independent; the step has no
+exchange to make).
+
+The `e2e` figure repeats the timed steps through the public Python API with the
+gradients in pinned host memory: each step copies them host -> device, runs
+the step and reads the device status word back.
+
+`--impl reference` times the float64 CPU oracle (the only other program here)
+on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np
+
+import workloads
+
+METRIC = "Shampoo step ms & inverse-roots/s at B=256..1024; % of tensor-core dense peak"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 / bf16 tensor throughput ratio
+SPLIT_PASSES = 3             # 3xTF32: three tf32 MMAs per fp32-accurate product
+WORKLOAD_NAMES = {
+    "tiny": "tiny_64x32_b32",
+    "lowrank": "lowrank_4x1024sq_b256",
+    "gpt2": "gpt2_small_shapes_b512",
+    "llama": "llama_1b_shapes_b1024",
+    "sweep": "inverse_root_sweep",
+}
+SWEEP_BATCH = {256: 512, 512: 128, 1024: 64}
+SOLVER_NAMES = {0: "coupled_newton", 1: "newton_db", 2: "chebyshev"}
+
+
+# ---------------------------------------------------------------------------
+# shared helpers
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def block_counts(wl):
+    import oracle  # noqa: F401  (only the partition; used for sizes)
+    nb = 0
+    for m, n in wl.shapes:
+        nb += -(-m // wl.block) * -(-n // wl.block)
+    return nb
+
+
+def refresh_steps(k, every):
+    """Refresh steps in a window of k steps that starts on a refresh step."""
+    return -(-k // every)
+
+
+def phase_to_refresh(step, every):
+    """First step >= `step` on which the roots are refreshed."""
+    return -(-step // every) * every
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def device_gradients(wl, seed, count, device):
+    """`count` per-step gradient sets on the device, drawn with torch from the
+    workload's recipe (same distribution as workloads.GradientStream)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    sets = []
+    fixed = {}
+    for i, (m, n) in enumerate(wl.shapes):
+        if wl.name == "lowrank":
+            fixed[i] = (torch.randn(m, 16, generator=g, device=device), torch.randn(n, 16, generator=g, device=device))
+        elif wl.name == "gpt2":
+            fixed[i] = 10.0 ** (torch.rand(n, generator=g, device=device) * 2.0 - 2.0)
+    for _ in range(count):
+        out = []
+        for i, (m, n) in enumerate(wl.shapes):
+            if wl.name == "lowrank":
+                u, v = fixed[i]
+                s = torch.randn(16, 16, generator=g, device=device)
+                x = (u @ s @ v.T) / 16.0 + 0.01 * torch.randn(m, n, generator=g, device=device)
+            elif wl.name == "gpt2":
+                x = torch.randn(m, n, generator=g, device=device) * 0.02 * fixed[i][None, :]
+            elif wl.name == "llama":
+                x = (torch.randn(m, n, generator=g, device=device) * 0.01).to(torch.bfloat16)
+            else:
+                x = torch.randn(m, n, generator=g, device=device)
+                if wl.grad_dtype == workloads.DTYPE_BF16:
+                    x = x.to(torch.bfloat16)
+            out.append(x.contiguous())
+        sets.append(out)
+    return sets
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+    import shampoo_family_second_b200 as sb
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        from datetime import timedelta
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+
+    cfg = sb.config_from_workload(wl)
+    opt = sb.Shampoo(wl.shapes, cfg, device=device)
+    W = [torch.zeros(s, dtype=torch.float32, device=device) for s in wl.shapes]
+    ring = max(1, min(args.ring, args.steps + args.warmup))
+    grads = device_gradients(wl, wl.seed + 1000 * rank, ring, device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    nb = opt.nb
+    roots_per_refresh = 2 * nb
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    # warm-up
+    for t in range(args.warmup):
+        opt.step(W, grads[t % ring])
+    barrier()
+    if opt.status(reset=True) & ~sb.DEVFLAG_NOT_CONVERGED:
+        raise RuntimeError("device status reported an error during warm-up")
+
+    # ---- timed region: K steps, per-step events, L2 flushed between steps
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    first = args.warmup
+    opt.set_step_count(phase_to_refresh(first, wl.refresh_every))   # timed window starts on a refresh step
+    launches0 = sb.launch_count()
+    barrier()
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        opt.step(W, grads[(first + k) % ring])
+        ev[k][1].record(stream)
+    barrier()
+    launches = sb.launch_count() - launches0
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(step_ms))
+    nref = refresh_steps(args.steps, wl.refresh_every)
+    status = opt.status(reset=True)
+
+    # ---- roofline pass: same steps with per-launch events inside the library
+    sb.profile_reset()
+    sb.profile_enable(True)
+    opt.set_step_count(phase_to_refresh(opt.step_count, wl.refresh_every))
+    barrier()
+    for k in range(args.steps):
+        flush.zero_()
+        opt.step(W, grads[(first + args.steps + k) % ring])
+    barrier()
+    tallies = {kind: sb.profile_read(kind) for kind in range(sb.KERNEL_KINDS)}
+    sb.profile_enable(False)
+    nref_prof = refresh_steps(args.steps, wl.refresh_every)
+
+    # ---- end to end through the public API with host-resident gradients
+    host = [[g.cpu().pin_memory() for g in gs] for gs in grads[: min(ring, 4)]]
+    dev_in = [torch.empty_like(g) for g in grads[0]]
+    status_host = torch.zeros(1, dtype=torch.int32).pin_memory()
+    h2d = sum(g.numel() * g.element_size() for g in host[0])
+    status_view = opt.state[:4].view(torch.int32)
+    opt.set_step_count(phase_to_refresh(opt.step_count, wl.refresh_every))
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for k in range(args.steps):
+        flush.zero_()
+        e0.record(stream)
+        for d, h in zip(dev_in, host[k % len(host)]):
+            d.copy_(h, non_blocking=True)
+        opt.step(W, dev_in)
+        status_host.copy_(status_view, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    barrier()
+    nref_e2e = refresh_steps(args.steps, wl.refresh_every)
+
+    # ---- max over ranks
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    peaks, peak_src = load_peaks()
+    g = tallies[sb.KERNEL_GEMM]
+    gemm_avg_ms = g.total_ms / max(g.launches, 1)
+    achieved = (g.alg_flops / max(g.launches, 1)) / (gemm_avg_ms * 1e-3) / 1e12 if g.launches else 0.0
+    tf32_peak = peaks["bf16_tflops_sustained"] * TF32_PER_BF16
+    peak = tf32_peak / SPLIT_PASSES
+    traffic = gemm_traffic_per_launch(g)
+    step_total_prof = sum(tl.total_ms for tl in tallies.values())
+
+    result = {
+        "metric": METRIC,
+        "value": roots_per_refresh * nref * world / (total_ms * 1e-3) if total_ms > 0 else 0.0,
+        "unit": "inverse-roots/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD_NAMES.get(wl.name, wl.name),
+            "params": len(wl.shapes), "param_elems": wl.n_params, "block": wl.block, "blocks": nb,
+            "roots_per_refresh": roots_per_refresh, "refresh_every": wl.refresh_every,
+            "refresh_steps_timed": nref, "solver": SOLVER_NAMES[wl.solver], "root_p": wl.root_p,
+            "iters_cap": wl.iters, "tol": wl.tol, "beta": wl.beta, "eps": wl.eps,
+            "grad_dtype": "bf16" if wl.grad_dtype == workloads.DTYPE_BF16 else "f32",
+            "arithmetic": "3xTF32 tcgen05 (fp32-accurate), fp32 state",
+            "l2": "256 MiB buffer written between timed steps, outside the per-step events",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "device_status": int(status),
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "roofline": {
+            "kernel": "gemm3x_tf32_kernel",
+            "bound": "tensor",
+            "achieved": achieved,
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": achieved / peak if peak else None,
+            "traffic": traffic,
+            "peak_basis": (f"{peak_src} bf16 sustained {peaks['bf16_tflops_sustained']} TF/s x {TF32_PER_BF16:.4f} "
+                           f"(nominal tf32/bf16) / {SPLIT_PASSES} (3xTF32 passes): fp32-equivalent "
+                           "algorithmic flops; frac is also the issued tf32 fraction"),
+            "launches": g.launches, "avg_launch_ms": gemm_avg_ms,
+            "share_of_step_kernel_time": g.total_ms / step_total_prof if step_total_prof else None,
+            "refresh_steps": nref_prof,
+        },
+        "kernels": {sb.KERNEL_NAMES[k]: {"launches": v.launches, "ms": round(v.total_ms, 4),
+                                         "alg_tflop": round(v.alg_flops / 1e12, 6),
+                                         "alg_gb": round(v.alg_bytes / 1e9, 6)}
+                    for k, v in tallies.items() if v.launches},
+        "e2e": {
+            "value": roots_per_refresh * nref_e2e * world / (e2e_ms * 1e-3) if e2e_ms > 0 else 0.0,
+            "unit": "inverse-roots/s",
+            "ms_per_step": e2e_ms / args.steps,
+            "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": 4,
+        },
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget_s)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def gemm_traffic_per_launch(g):
+    """DRAM bytes per GEMM launch from the committed ncu capture of this
+    workload's GEMM, if the capture was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        import hashlib
+        src = open(os.path.join(ROOT, "shampoo_family_second_b200", "csrc", "gemm_tc.cu"), "rb").read()
+        if d.get("gemm_tc_sha256") != hashlib.sha256(src).hexdigest():
+            return None
+        return d.get("bytes_per_launch")
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline / reference arm: the float64 oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def oracle_sample_plan(wl, budget_s):
+    """Blocks and steps of a bounded oracle sample of the workload."""
+    import oracle
+    table = oracle.block_table(wl.shapes, wl.block)
+    nb = len(table)
+    # rough cost model of one eigh(B) + products, to keep the sample in budget
+    per_block = 2 * (wl.block / 512.0) ** 3 * 0.06 + 1e-3
+    n_blocks = max(1, min(nb, int(budget_s / max(per_block, 1e-4) / 2)))
+    rng = np.random.default_rng(wl.seed)
+    blocks = sorted(rng.choice(nb, size=n_blocks, replace=False).tolist())
+    return blocks, nb
+
+
+def time_oracle(wl, blocks, steps, warmup=0):
+    import oracle
+    params = sorted({oracle.block_table(wl.shapes, wl.block)[b].param for b in blocks})
+    stream = workloads.GradientStream(wl, params=params)
+    gen = []
+    for _ in range(steps):
+        gs = stream.next()
+        full = [None] * len(wl.shapes)
+        for p, g in zip(params, gs):
+            full[p] = g
+        gen.append(full)
+    o = oracle.ShampooOracle(wl.shapes, wl.block, wl.beta, wl.eps, wl.lr, wl.root_p, wl.refresh_every,
+                             blocks=blocks)
+    times, nref = [], 0
+    for t in range(steps):
+        if t == warmup:
+            o.t = phase_to_refresh(o.t, wl.refresh_every)   # timed window starts on a refresh step
+        refresh = (o.t % wl.refresh_every) == 0
+        t0 = time.perf_counter()
+        o.step(gen[t])
+        times.append(time.perf_counter() - t0)
+        nref += int(refresh and t >= warmup)
+    return times, nref
+
+
+def cpu_baseline(wl, budget_s):
+    cores = len(os.sched_getaffinity(0))
+    blocks, nb = oracle_sample_plan(wl, budget_s)
+    steps = min(wl.refresh_every, 10)
+    times, nref = time_oracle(wl, blocks, steps)
+    roots = 2 * len(blocks) * nref
+    value = roots / sum(times)
+    return {"value": value, "unit": "inverse-roots/s", "cores": cores, "kind": "oracle",
+            "sample": (f"{len(blocks)} of {nb} blocks, {steps} consecutive steps from step 0 "
+                       f"({nref} refresh), float64 numpy/LAPACK eigh, {cores} host threads")}
+
+
+def run_reference(args, wl):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    cores = len(os.sched_getaffinity(0))
+    per_step_budget = max(1.0, args.cpu_budget_s / max(args.steps + args.warmup, 1))
+    blocks, nb = oracle_sample_plan(wl, per_step_budget * wl.refresh_every)
+    total = args.warmup + args.steps
+    times, nref = time_oracle(wl, blocks, total, warmup=args.warmup)
+    timed = times[args.warmup:]
+    roots = 2 * len(blocks) * nref
+    value = roots / sum(timed) if sum(timed) > 0 else 0.0
+    sample = (f"{len(blocks)} of {nb} blocks per step, {args.steps} timed steps after {args.warmup} warm-up, "
+              f"window starting on a refresh step ({nref} refresh), float64 numpy/LAPACK, {cores} host threads")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "inverse-roots/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(timed) / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAMES.get(wl.name, wl.name), "block": wl.block,
+                   "refresh_every": wl.refresh_every, "sampled_blocks": len(blocks), "blocks": nb},
+        "cpu_baseline": {"value": value, "unit": "inverse-roots/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "inverse-roots/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def run_sweep(args):
+    """Inverse-root solver sweep: stacked fp32 SPD matrices Q diag(lam) Q^T
+    (Haar Q, log-uniform lam with condition number kappa), one
+    inv_root_batched call per step through the C ABI."""
+    import torch
+    import shampoo_family_second_b200 as sb
+    import oracle
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group(backend="nccl", timeout=timedelta(seconds=120))
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    n, kappa, p = args.sweep_n, args.sweep_kappa, args.sweep_p
+    batch = args.sweep_batch or SWEEP_BATCH.get(n, 64)
+    solver = {"newton": 0, "newton_db": 1, "chebyshev": 2}[args.sweep_solver]
+    A64 = workloads.spd_batch(batch, n, kappa, seed=4321 + n + rank)
+    A = torch.from_numpy(A64.astype(np.float32)).to(device)
+    X = torch.empty_like(A)
+    scratch = torch.empty(sb.inv_root_scratch_bytes(batch, n, solver), dtype=torch.uint8, device=device)
+    iters = torch.zeros(batch, dtype=torch.int32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    lo = 0.999 / kappa if solver == 2 else 0.0
+    kw = dict(p=p, eps=0.0, solver=solver, iters=args.sweep_iters, tol=args.sweep_tol, cheb_degree=args.sweep_degree,
+              cheb_lo=lo, out=X, scratch=scratch, stream=stream)
+
+    def one():
+        _, it, st = sb.inv_root_batched(A, **kw)
+        iters.copy_(it)
+        status.copy_(st)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(device.index or 0)
+    clocks.start()
+    l0 = sb.launch_count()
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        one()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    launches = sb.launch_count() - l0
+    clk = clocks.stop()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    sb.profile_reset()
+    sb.profile_enable(True)
+    for k in range(args.steps):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    g = sb.profile_read(sb.KERNEL_GEMM)
+    sb.profile_enable(False)
+    peaks, src = load_peaks()
+    peak = peaks["bf16_tflops_sustained"] * TF32_PER_BF16 / SPLIT_PASSES
+    ach = (g.alg_flops / g.launches) / (g.total_ms / g.launches * 1e-3) / 1e12 if g.launches else 0.0
+    it_host = iters.cpu().numpy()
+    # parity on a sample of the stacked roots (the oracle's exact root)
+    Xh = X.cpu().numpy().astype(np.float64)
+    errs = [oracle.rel_fro(Xh[i], oracle.inverse_root(A64[i].astype(np.float32).astype(np.float64), p, 0.0))
+            for i in range(min(2, batch))]
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": batch * args.steps * world / (total_ms * 1e-3), "unit": "inverse-roots/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"inverse_root_sweep_{batch}x{n}sq_kappa{kappa:.0e}_p{p}_{args.sweep_solver}",
+                       "n": n, "batch": batch, "kappa": kappa, "p": p, "solver": args.sweep_solver,
+                       "iters": args.sweep_iters, "tol": args.sweep_tol, "degree": args.sweep_degree,
+                       "l2": "256 MiB buffer written between timed calls, outside the events"},
+            "iters_used": [int(it_host.min()), int(it_host.max())], "device_status": int(status.item()),
+            "rel_err_vs_oracle_sample": errs, "gpu_launches": int(launches), "clocks": clk,
+            "roofline": {"kernel": "gemm3x_tf32_kernel", "bound": "tensor", "achieved": ach, "peak": peak,
+                         "unit": "TFLOP/s", "frac": ach / peak if peak else None, "traffic": None,
+                         "launches": g.launches, "avg_launch_ms": g.total_ms / max(g.launches, 1),
+                         "peak_basis": f"{src} bf16 sustained x 1.1/2.25 / 3"},
+        }), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="lowrank", choices=sorted(WORKLOAD_NAMES))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ring", type=int, default=8, help="distinct gradient sets kept on the device")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep-n", type=int, default=512)
+    ap.add_argument("--sweep-batch", type=int, default=0)
+    ap.add_argument("--sweep-kappa", type=float, default=1e4)
+    ap.add_argument("--sweep-p", type=int, default=4)
+    ap.add_argument("--sweep-solver", default="newton", choices=["newton", "newton_db", "chebyshev"])
+    ap.add_argument("--sweep-iters", type=int, default=25)
+    ap.add_argument("--sweep-tol", type=float, default=0.0)
+    ap.add_argument("--sweep-degree", type=int, default=32)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.workload == "sweep":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the sweep is timed for the CUDA path only; "
+                              "the oracle arm covers the step workloads"}))
+            return
+        run_sweep(args)
+        return
+    wl = workloads.workload(args.workload)
+    np.random.seed(0)
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

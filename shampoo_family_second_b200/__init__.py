@@ -277,6 +277,10 @@ class Shampoo:
         XR = fl[(pxr - base) // 4:(pxr - base) // 4 + 2 * nb * B * B].view(nb, 2, B, B)
         return XL[:, 0] + XL[:, 1], XR[:, 0] + XR[:, 1]
 
+    def set_step_count(self, step: int):
+        """Sets the step counter (the refresh schedule counts from it)."""
+        _check(lib.shampoo_set_step(self._h, int(step)))
+
     def state_dict(self):
         """Checkpoint: a copy of the state bytes and the step counter."""
         return {"state": self.state.clone(), "step": self.step_count}

@@ -79,15 +79,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // that the caller can unwind instead of spinning forever.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* flags) {
+// `abort` (shared memory, nullable) lets one role of a CTA that gave up tell
+// the others to stop waiting as well.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* flags,
+                                                  volatile int* abort = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
+    if (abort && *abort) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       raise_flag(flags, DEV_FLAG_TIMEOUT);
+      if (abort) *abort = 1;
       return false;
     }
   }
@@ -177,18 +182,19 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
-// with 128-byte swizzling: rows of 128 bytes (32 fp32), 8-row groups 1024 bytes
+// with 64-byte swizzling: rows of 64 bytes (16 fp32), 8-row groups 512 bytes
 // apart.  Fields: start address >> 4 (bits 0-13), leading byte offset >> 4
 // (bits 16-29; unused for swizzled K-major, set to 1), stride byte offset >> 4
 // (bits 32-45), descriptor version 1 (bits 46-47), base offset 0, swizzle mode
-// 2 = 128B (bits 61-63).
-__device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
+// 4 = 64B (bits 61-63).  One MMA reads 8 tf32 (32 bytes) of each row; the
+// second K-step of a row starts 32 bytes further.
+__device__ __forceinline__ uint64_t smem_desc_k_sw64(uint32_t saddr) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>(1u) << 16;
-  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(512u >> 4) << 32;
   d |= static_cast<uint64_t>(1u) << 46;
-  d |= static_cast<uint64_t>(2u) << 61;
+  d |= static_cast<uint64_t>(4u) << 61;
   return d;
 }
 

@@ -12,10 +12,11 @@
 //   apply + update  T = L^{-1/4} G, then W <- W - lr T R^{-1/4} scattered into
 //                   the weight (notes' listing, last line).
 //
-// One CTA computes one 128 x 256 tile of one matrix D_i = epi(A_i B_i^T), or
-// epi(A_i B_i) when B is read MN-major (B stored K x N row-major):
+// A persistent kernel (one CTA per SM) walks 128 x 256 tiles of the matrices
+// D_i = epi(A_i B_i^T), or epi(A_i B_i) when B is read MN-major (B stored
+// K x N row-major):
 //   warp 0      one thread issues TMA loads of the A and B tiles (hi and lo
-//               planes) into a 2-stage shared-memory ring;
+//               planes, 16 deep in K) into a 4-stage shared-memory ring;
 //   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 buffers); one
 //               thread issues the tcgen05 MMAs (3 per K-step of 8), each K
 //               segment of 64 into the next buffer, and commits them to the
@@ -25,8 +26,9 @@
 //               epilogue and store.  The tensor core's own fp32 additions
 //               truncate; summing short segments outside it keeps the product
 //               as accurate as a plain fp32 GEMM.
-// Every wait is bounded (2 s); a time-out raises DEV_FLAG_TIMEOUT and the CTA
-// unwinds, releasing its TMEM.
+// Every wait is bounded (2 s); a time-out raises DEV_FLAG_TIMEOUT, tells the
+// other roles of the CTA to stop waiting, and the CTA unwinds, releasing its
+// TMEM.
 #include <cstdio>
 #include <cstring>
 
@@ -41,38 +43,20 @@ namespace {
 constexpr int BM = kTileM;
 constexpr int BN = kTileN;
 constexpr int BK = kTileK;
-constexpr int STAGES = 2;
-constexpr int A_PLANE = BM * BK * 4;                        // 16 KB
-constexpr int B_PLANE = BN * BK * 4;                        // 32 KB
-constexpr int STAGE_BYTES = 2 * A_PLANE + 2 * B_PLANE;      // 96 KB
-constexpr int MN_BLOCK = BK * 32 * 4;                      // 4 KB: 32 K-rows x 32 columns
+constexpr int STAGES = 4;
+constexpr int A_PLANE = BM * BK * 4;                        // 8 KB
+constexpr int B_PLANE = BN * BK * 4;                        // 16 KB
+constexpr int STAGE_BYTES = 2 * A_PLANE + 2 * B_PLANE;      // 48 KB
+constexpr int MN_BLOCK = BK * 32 * 4;                      // 2 KB: 16 K-rows x 32 columns
 constexpr int TMEM_COLS = 512;  // two 128 x 256 fp32 accumulators (K-segment double buffer)
-constexpr int SEG = 2;           // K chunks (of 32) per accumulation segment
+constexpr int SEG = 4;           // K chunks (of 16) per accumulation segment: 64 deep
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 
-__device__ __forceinline__ void store_row32(float* dst, const float (&v)[32]) {
-  float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) d4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-}
-
-__device__ __forceinline__ void store_split_row32(float* hi_dst, float* lo_dst, const float (&v)[32]) {
-  float4* h4 = reinterpret_cast<float4*>(hi_dst);
-  float4* l4 = reinterpret_cast<float4*>(lo_dst);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    float h[4], l[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) split_tf32(v[4 * j + q], h[q], l[q]);
-    h4[j] = make_float4(h[0], h[1], h[2], h[3]);
-    l4[j] = make_float4(l[0], l[1], l[2], l[3]);
-  }
-}
-
 // Epilogue for 32 consecutive columns [c0, c0+32) of row r of matrix `mat`;
-// acc holds the fp32 products (A B^T or A B) of those columns.
+// acc holds the fp32 products (A B^T or A B) of those columns.  Works through
+// them 8 at a time to keep few registers live next to the running sums.
 // Returns this thread's residual contribution.
 __device__ __forceinline__ float epilogue_chunk(const GemmGroup& G, int mat, int r, int c0, const float* acc,
                                                 bool& nonfinite) {
@@ -80,85 +64,122 @@ __device__ __forceinline__ float epilogue_chunk(const GemmGroup& G, int mat, int
   const int n = G.n;
   const size_t nn = static_cast<size_t>(n) * n;
   const size_t row_off = static_cast<size_t>(r) * n + c0;
-  float v[32];
-  float resid = 0.f;
   const int vsz = E.valid ? E.valid[mat] : n;
-  if (E.res) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int c = c0 + j;
-      float d = acc[j] - ((r == c) ? 1.f : 0.f);
-      resid += (r < vsz && c < vsz) ? d * d : 0.f;
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = E.alpha * acc[j];
-  if (E.C) {
-    if (E.c_split) {
-      const float4* h4 = reinterpret_cast<const float4*>(E.C + mat * 2 * nn + row_off);
-      const float4* l4 = reinterpret_cast<const float4*>(E.C + mat * 2 * nn + nn + row_off);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float4 h = h4[j], l = l4[j];
-        v[4 * j + 0] += E.beta * (h.x + l.x);
-        v[4 * j + 1] += E.beta * (h.y + l.y);
-        v[4 * j + 2] += E.beta * (h.z + l.z);
-        v[4 * j + 3] += E.beta * (h.w + l.w);
-      }
-    } else {
-      const float4* c4 = reinterpret_cast<const float4*>(E.C + mat * nn + row_off);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float4 h = c4[j];
-        v[4 * j + 0] += E.beta * h.x;
-        v[4 * j + 1] += E.beta * h.y;
-        v[4 * j + 2] += E.beta * h.z;
-        v[4 * j + 3] += E.beta * h.w;
-      }
-    }
-  }
   const float gam = E.gamma_vec ? E.gamma_vec[static_cast<size_t>(mat) * E.gamma_stride] : E.gamma;
+  const float sc = E.scale_vec ? E.scale_vec[mat] : 1.f;
   const int dj = r - c0;
-  if (dj >= 0 && dj < 32) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j == dj) v[j] += gam;
-  }
-  if (E.scale_vec) {
-    const float sc = E.scale_vec[mat];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] *= sc;
-  }
+  float resid = 0.f;
   bool bad = false;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) bad |= !isfinite(v[j]);
-  nonfinite |= bad;
-  if (E.D) {
-    if (E.d_split)
-      store_split_row32(E.D + mat * 2 * nn + row_off, E.D + mat * 2 * nn + nn + row_off, v);
-    else
-      store_row32(E.D + mat * nn + row_off, v);
-  }
-  if (E.E) {
-    float e[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) e[j] = E.e_mul * v[j] + ((j == dj) ? E.e_add : 0.f);
-    store_split_row32(E.E + mat * 2 * nn + row_off, E.E + mat * 2 * nn + nn + row_off, e);
-  }
+  const size_t dplane = E.d_split ? 2 * nn : nn;
+  float* wrow = nullptr;
+  int wc = 0;
   if (E.wptr) {
-    const int wr = E.wrows[mat], wc = E.wcols[mat];
-    if (r < wr) {
-      float* w = E.wptr[mat] + static_cast<size_t>(r) * E.wld[mat];
+    const int wr = E.wrows[mat];
+    wc = E.wcols[mat];
+    if (r < wr) wrow = E.wptr[mat] + static_cast<size_t>(r) * E.wld[mat];
+  }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int c = c0 + j;
-        if (c < wc) w[c] -= E.lr * v[j];
+  for (int g = 0; g < 4; ++g) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int jj = 8 * g + j;
+      const float a = acc[jj];
+      if (E.res) {
+        const int c = c0 + jj;
+        const float d = a - ((r == c) ? 1.f : 0.f);
+        resid += (r < vsz && c < vsz) ? d * d : 0.f;
+      }
+      v[j] = E.alpha * a;
+    }
+    if (E.C) {
+      if (E.c_split) {
+        const float4* h4 = reinterpret_cast<const float4*>(E.C + mat * 2 * nn + row_off + 8 * g);
+        const float4* l4 = reinterpret_cast<const float4*>(E.C + mat * 2 * nn + nn + row_off + 8 * g);
+        const float4 h0 = h4[0], h1 = h4[1], l0 = l4[0], l1 = l4[1];
+        v[0] += E.beta * (h0.x + l0.x); v[1] += E.beta * (h0.y + l0.y);
+        v[2] += E.beta * (h0.z + l0.z); v[3] += E.beta * (h0.w + l0.w);
+        v[4] += E.beta * (h1.x + l1.x); v[5] += E.beta * (h1.y + l1.y);
+        v[6] += E.beta * (h1.z + l1.z); v[7] += E.beta * (h1.w + l1.w);
+      } else {
+        const float4* c4 = reinterpret_cast<const float4*>(E.C + mat * nn + row_off + 8 * g);
+        const float4 x0 = c4[0], x1 = c4[1];
+        v[0] += E.beta * x0.x; v[1] += E.beta * x0.y; v[2] += E.beta * x0.z; v[3] += E.beta * x0.w;
+        v[4] += E.beta * x1.x; v[5] += E.beta * x1.y; v[6] += E.beta * x1.z; v[7] += E.beta * x1.w;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (8 * g + j == dj) v[j] += gam;
+      v[j] *= sc;
+      bad |= !isfinite(v[j]);
+    }
+    if (E.D) {
+      float* d = E.D + mat * dplane + row_off + 8 * g;
+      if (E.d_split) {
+        float hh[8], ll[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) split_tf32(v[j], hh[j], ll[j]);
+        reinterpret_cast<float4*>(d)[0] = make_float4(hh[0], hh[1], hh[2], hh[3]);
+        reinterpret_cast<float4*>(d)[1] = make_float4(hh[4], hh[5], hh[6], hh[7]);
+        reinterpret_cast<float4*>(d + nn)[0] = make_float4(ll[0], ll[1], ll[2], ll[3]);
+        reinterpret_cast<float4*>(d + nn)[1] = make_float4(ll[4], ll[5], ll[6], ll[7]);
+      } else {
+        reinterpret_cast<float4*>(d)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4*>(d)[1] = make_float4(v[4], v[5], v[6], v[7]);
+      }
+    }
+    if (E.E) {
+      float hh[8], ll[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) split_tf32(E.e_mul * v[j] + ((8 * g + j == dj) ? E.e_add : 0.f), hh[j], ll[j]);
+      float* e = E.E + mat * 2 * nn + row_off + 8 * g;
+      reinterpret_cast<float4*>(e)[0] = make_float4(hh[0], hh[1], hh[2], hh[3]);
+      reinterpret_cast<float4*>(e)[1] = make_float4(hh[4], hh[5], hh[6], hh[7]);
+      reinterpret_cast<float4*>(e + nn)[0] = make_float4(ll[0], ll[1], ll[2], ll[3]);
+      reinterpret_cast<float4*>(e + nn)[1] = make_float4(ll[4], ll[5], ll[6], ll[7]);
+    }
+    if (wrow) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = c0 + 8 * g + j;
+        if (c < wc) wrow[c] -= E.lr * v[j];
       }
     }
   }
+  nonfinite |= bad;
   return resid;
 }
 
+struct TileCoord {
+  int gi, mat, tm, tn;
+  bool skip;
+};
+
+// Tile `tile` of the launch: group, matrix, tile row and column.  Tiles are
+// numbered group by group, matrix by matrix, so the CTAs working at the same
+// time share operands of a few matrices through L2.
+__device__ __forceinline__ TileCoord tile_coord(const GemmLaunch& L, int tile) {
+  TileCoord c;
+  int gi = 0;
+#pragma unroll 1
+  while (gi + 1 < L.ngroups && tile >= L.g[gi + 1].cta_begin) ++gi;
+  const GemmGroup& G = L.g[gi];
+  const int local = tile - G.cta_begin;
+  const int tiles = G.tiles_m * G.tiles_n;
+  c.gi = gi;
+  c.mat = local / tiles;
+  const int t = local - c.mat * tiles;
+  c.tm = t / G.tiles_n;
+  c.tn = t - c.tm * G.tiles_n;
+  c.skip = G.ep.skip && G.ep.skip[c.mat];
+  return c;
+}
+
+// Persistent: one CTA per SM walks the tiles blockIdx.x, blockIdx.x +
+// gridDim.x, ...  The shared-memory ring and the two TMEM buffers carry over
+// from one tile to the next, so the epilogue of a tile (register sums ->
+// global stores) overlaps the MMAs of the next one.
 __global__ void __launch_bounds__(THREADS, 1)
     gemm3x_tf32_kernel(const __grid_constant__ GemmLaunch L, const __grid_constant__ TmaMaps maps,
                        double* prof_flops) {
@@ -169,27 +190,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* acc_full = empty + STAGES;   // [2]: a K-segment's partial sums are ready in TMEM buffer b
   uint64_t* acc_empty = acc_full + 2;    // [2]: the epilogue has drained TMEM buffer b
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-
-  // Locate this CTA's group, matrix and tile.
-  const int cta = blockIdx.x;
-  int gi = 0;
-#pragma unroll 1
-  while (gi + 1 < L.ngroups && cta >= L.g[gi + 1].cta_begin) ++gi;
-  const GemmGroup& G = L.g[gi];
-  const int local = cta - G.cta_begin;
-  const int tiles = G.tiles_m * G.tiles_n;
-  const int mat = local / tiles;
-  const int t = local - mat * tiles;
-  const int tm = t / G.tiles_n;
-  const int tn = t - tm * G.tiles_n;
-  if (G.ep.skip && G.ep.skip[mat]) return;  // uniform across the CTA: nothing allocated yet
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n = G.n;
-  const int nk = n / BK;
-  const int nseg = (nk + SEG - 1) / SEG;
-  int* flags = G.ep.flags;
+  const int total = L.total_tiles;
+  int* flags = L.g[0].ep.flags;
 
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -202,12 +208,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], EPI_WARPS);
     }
+    *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&maps.m[G.a_map]);
-    prefetch_tmap(&maps.m[G.b_map]);
-  }
+  if (warp == 0 && lane < 2 * L.ngroups) prefetch_tmap(&maps.m[lane]);
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
@@ -220,86 +224,114 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      const uint32_t tx_bytes = 2u * G.a_rows * BK * 4u + 2u * G.b_rows * BK * 4u;
-      const void* amap = &maps.m[G.a_map];
-      const void* bmap = &maps.m[G.b_map];
-      const int am = G.a_off + mat;
-      const int bm = G.b_off + mat;
-      int issued = 0;
+      uint32_t it = 0;  // chunks issued by this CTA (ring position)
+      bool ok = true;
 #pragma unroll 1
-      for (int kc = 0; kc < nk; ++kc) {
-        const int s = kc % STAGES;
-        if (kc >= STAGES && !mbar_wait_bounded(&empty[s], ((kc / STAGES) - 1) & 1, flags)) break;
-        uint8_t* sa = smem + s * STAGE_BYTES;
-        uint8_t* sb = sa + 2 * A_PLANE;
-        mbar_arrive_expect_tx(&full[s], tx_bytes);
-        // One copy per plane, each to its fixed offset (the boxes may hold
-        // fewer rows than the tile when n is small).
-        tma_load_4d(sa, amap, &full[s], kc * BK, tm * BM, 0, am);
-        tma_load_4d(sa + A_PLANE, amap, &full[s], kc * BK, tm * BM, 1, am);
-        if (G.b_mn) {
-          // B[k][n] row-major: 32 K-rows x 32 N-columns per copy, one copy per
-          // 32-column block of the tile, blocks MN_BLOCK bytes apart.
-          const int nblk = G.b_rows / 32;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileCoord tc = tile_coord(L, tile);
+        if (tc.skip) continue;
+        const GemmGroup& G = L.g[tc.gi];
+        const int nk = G.n / BK;
+        const uint32_t tx_bytes = 2u * G.a_rows * BK * 4u + 2u * G.b_rows * BK * 4u;
+        const void* amap = &maps.m[G.a_map];
+        const void* bmap = &maps.m[G.b_map];
+        const int am = G.a_off + tc.mat;
+        const int bm = G.b_off + tc.mat;
 #pragma unroll 1
-          for (int q = 0; q < nblk; ++q) {
-            tma_load_4d(sb + q * MN_BLOCK, bmap, &full[s], tn * BN + q * 32, kc * BK, 0, bm);
-            tma_load_4d(sb + B_PLANE + q * MN_BLOCK, bmap, &full[s], tn * BN + q * 32, kc * BK, 1, bm);
+        for (int kc = 0; kc < nk; ++kc, ++it) {
+          const int s = it % STAGES;
+          if (it >= STAGES && !mbar_wait_bounded(&empty[s], ((it / STAGES) - 1) & 1, flags, abort_flag)) {
+            ok = false;
+            break;
           }
-        } else {
-          tma_load_4d(sb, bmap, &full[s], kc * BK, tn * BN, 0, bm);
-          tma_load_4d(sb + B_PLANE, bmap, &full[s], kc * BK, tn * BN, 1, bm);
-        }
-        ++issued;
-      }
-      // Drain: make sure no copy is still landing in shared memory when the
-      // CTA retires (bounded; normally these phases completed long ago).
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          uint8_t* sb = sa + 2 * A_PLANE;
+          mbar_arrive_expect_tx(&full[s], tx_bytes);
+          // One copy per plane, each to its fixed offset (the boxes may hold
+          // fewer rows than the tile when n is small).
+          tma_load_4d(sa, amap, &full[s], kc * BK, tc.tm * BM, 0, am);
+          tma_load_4d(sa + A_PLANE, amap, &full[s], kc * BK, tc.tm * BM, 1, am);
+          if (G.b_mn) {
+            // B[k][n] row-major: 16 K-rows x 32 N-columns per copy, one copy per
+            // 32-column block of the tile, blocks MN_BLOCK bytes apart.
+            const int nblk = G.b_rows / 32;
 #pragma unroll 1
-      for (int kc = (issued > STAGES ? issued - STAGES : 0); kc < issued; ++kc)
-        mbar_wait_bounded(&full[kc % STAGES], (kc / STAGES) & 1, flags);
+            for (int q = 0; q < nblk; ++q) {
+              tma_load_4d(sb + q * MN_BLOCK, bmap, &full[s], tc.tn * BN + q * 32, kc * BK, 0, bm);
+              tma_load_4d(sb + B_PLANE + q * MN_BLOCK, bmap, &full[s], tc.tn * BN + q * 32, kc * BK, 1, bm);
+            }
+          } else {
+            tma_load_4d(sb, bmap, &full[s], kc * BK, tc.tn * BN, 0, bm);
+            tma_load_4d(sb + B_PLANE, bmap, &full[s], kc * BK, tc.tn * BN, 1, bm);
+          }
+        }
+      }
+      // Drain: no copy may still be landing in shared memory when the CTA
+      // retires (bounded by time only; normally these phases completed).
+#pragma unroll 1
+      for (uint32_t k = (it > STAGES ? it - STAGES : 0); k < it; ++k)
+        mbar_wait_bounded(&full[k % STAGES], (k / STAGES) & 1, flags, nullptr);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      // K is cut into segments of SEG chunks.  Segment g accumulates from zero
-      // into TMEM buffer g & 1; the epilogue warps add each finished segment
-      // into fp32 registers with round-to-nearest.  The tensor core's own
-      // additions (which truncate) then only ever see one segment's partial
-      // sums, which keeps the truncation bias of long products small.
-      const uint32_t idesc = idesc_tf32(BM, BN, G.b_mn);
+      // K is cut into segments of SEG chunks.  Segment g (counted across
+      // tiles) accumulates from zero into TMEM buffer g & 1; the epilogue warps
+      // add each finished segment into fp32 registers with round-to-nearest.
+      // The tensor core's own additions (which truncate) then only ever see
+      // one segment's partial sums, which keeps long products unbiased.
+      uint32_t it = 0, sg = 0;
+      bool ok = true;
 #pragma unroll 1
-      for (int kc = 0; kc < nk; ++kc) {
-        const int s = kc % STAGES;
-        const int seg = kc / SEG;
-        const int b = seg & 1;
-        const bool first = (kc % SEG) == 0;
-        const uint32_t tbuf = taddr + b * BN;
-        if (first && seg >= 2 && !mbar_wait_bounded(&acc_empty[b], ((seg >> 1) - 1) & 1, flags)) break;
-        if (!mbar_wait_bounded(&full[s], (kc / STAGES) & 1, flags)) break;
-        tc_fence_after();
-        const uint32_t a_hi = smem_u32(smem + s * STAGE_BYTES);
-        const uint32_t a_lo = a_hi + A_PLANE;
-        const uint32_t b_hi = a_hi + 2 * A_PLANE;
-        const uint32_t b_lo = b_hi + B_PLANE;
-#pragma unroll
-        for (int ks = 0; ks < BK / 8; ++ks) {
-          const uint32_t off = ks * 32;  // 8 tf32 values = 32 bytes along K (K-major)
-          const uint64_t dah = smem_desc_k_sw128(a_hi + off);
-          const uint64_t dal = smem_desc_k_sw128(a_lo + off);
-          uint64_t dbh, dbl;
-          if (G.b_mn) {  // 8 K-rows = 1024 bytes = two 4-row groups
-            dbh = smem_desc_mn_sw128_32b(b_hi + ks * 1024, MN_BLOCK);
-            dbl = smem_desc_mn_sw128_32b(b_lo + ks * 1024, MN_BLOCK);
-          } else {
-            dbh = smem_desc_k_sw128(b_hi + off);
-            dbl = smem_desc_k_sw128(b_lo + off);
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileCoord tc = tile_coord(L, tile);
+        if (tc.skip) continue;
+        const GemmGroup& G = L.g[tc.gi];
+        const int nk = G.n / BK;
+        const uint32_t idesc = idesc_tf32(BM, BN, G.b_mn);
+#pragma unroll 1
+        for (int kc = 0; kc < nk; ++kc, ++it) {
+          const int s = it % STAGES;
+          const bool first = (kc % SEG) == 0;
+          const uint32_t b = sg & 1;
+          const uint32_t tbuf = taddr + b * BN;
+          if (first && sg >= 2 &&
+              !mbar_wait_bounded(&acc_empty[b], ((sg >> 1) - 1) & 1, flags, abort_flag)) {
+            ok = false;
+            break;
           }
-          mma_tf32(tbuf, dah, dbh, idesc, (first && ks == 0) ? 0u : 1u);
-          mma_tf32(tbuf, dah, dbl, idesc, 1u);
-          mma_tf32(tbuf, dal, dbh, idesc, 1u);
+          if (!mbar_wait_bounded(&full[s], (it / STAGES) & 1, flags, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_hi = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t a_lo = a_hi + A_PLANE;
+          const uint32_t b_hi = a_hi + 2 * A_PLANE;
+          const uint32_t b_lo = b_hi + B_PLANE;
+#pragma unroll
+          for (int ks = 0; ks < BK / 8; ++ks) {
+            const uint32_t off = ks * 32;  // 8 tf32 values = 32 bytes along K (K-major)
+            const uint64_t dah = smem_desc_k_sw64(a_hi + off);
+            const uint64_t dal = smem_desc_k_sw64(a_lo + off);
+            uint64_t dbh, dbl;
+            if (G.b_mn) {  // 8 K-rows = 1024 bytes = two 4-row groups
+              dbh = smem_desc_mn_sw128_32b(b_hi + ks * 1024, MN_BLOCK);
+              dbl = smem_desc_mn_sw128_32b(b_lo + ks * 1024, MN_BLOCK);
+            } else {
+              dbh = smem_desc_k_sw64(b_hi + off);
+              dbl = smem_desc_k_sw64(b_lo + off);
+            }
+            mma_tf32(tbuf, dah, dbh, idesc, (first && ks == 0) ? 0u : 1u);
+            mma_tf32(tbuf, dah, dbl, idesc, 1u);
+            mma_tf32(tbuf, dal, dbh, idesc, 1u);
+          }
+          mma_commit(&empty[s]);
+          if ((kc % SEG) == SEG - 1 || kc == nk - 1) {
+            mma_commit(&acc_full[b]);
+            ++sg;
+          }
         }
-        mma_commit(&empty[s]);
-        if ((kc % SEG) == SEG - 1 || kc == nk - 1) mma_commit(&acc_full[b]);
       }
     }
   } else {
@@ -308,47 +340,59 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int ew = warp - 2;
     const int q = warp & 3;
     const int h = ew >> 2;
-    const int r = tm * BM + q * 32 + lane;
     const uint32_t lane_addr = taddr + (static_cast<uint32_t>(q * 32) << 16) + h * (BN / 2);
-    float sum[BN / 2];
-#pragma unroll
-    for (int j = 0; j < BN / 2; ++j) sum[j] = 0.f;
+    uint32_t sg = 0;
     bool ok = true;
 #pragma unroll 1
-    for (int seg = 0; seg < nseg; ++seg) {
-      const int b = seg & 1;
-      if (!mbar_wait_bounded(&acc_full[b], (seg >> 1) & 1, flags)) {
-        ok = false;
-        break;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const TileCoord tc = tile_coord(L, tile);
+      if (tc.skip) continue;
+      const GemmGroup& G = L.g[tc.gi];
+      const int n = G.n;
+      const int nseg = (n / BK + SEG - 1) / SEG;
+      const int r = tc.tm * BM + q * 32 + lane;
+      float sum[BN / 2];
+#pragma unroll
+      for (int j = 0; j < BN / 2; ++j) sum[j] = 0.f;
+#pragma unroll 1
+      for (int seg = 0; seg < nseg; ++seg, ++sg) {
+        const uint32_t b = sg & 1;
+        if (!mbar_wait_bounded(&acc_full[b], (sg >> 1) & 1, flags, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(lane_addr + b * BN + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sum[c * 32 + j] += __uint_as_float(v[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
       }
-      tc_fence_after();
+      if (!ok) break;
+      float resid = 0.f;
+      bool nonfinite = false;
+      if (r < n) {
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_addr + b * BN + c * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) sum[c * 32 + j] += __uint_as_float(v[j]);
+        for (int c = 0; c < BN / 64; ++c) {
+          const int c0 = tc.tn * BN + h * (BN / 2) + c * 32;
+          if (c0 < n) resid += epilogue_chunk(G, tc.mat, r, c0, &sum[c * 32], nonfinite);
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[b]);
-    }
-    float resid = 0.f;
-    bool nonfinite = false;
-    if (ok && r < n) {
+      if (G.ep.res) {
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) {
-        const int c0 = tn * BN + h * (BN / 2) + c * 32;
-        if (c0 < n) resid += epilogue_chunk(G, mat, r, c0, &sum[c * 32], nonfinite);
+        for (int o = 16; o > 0; o >>= 1) resid += __shfl_xor_sync(0xffffffffu, resid, o);
+        if (lane == 0 && resid != 0.f) atomicAdd(&G.ep.res[tc.mat], resid);
       }
+      if (nonfinite) raise_flag(G.ep.flags, DEV_FLAG_NONFINITE);
+      if (L.profile && ew == 0 && lane == 0 && prof_flops)
+        atomicAdd(&prof_flops[L.prof_slot], G.flops_per_matrix / (G.tiles_m * G.tiles_n));
     }
-    if (G.ep.res) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) resid += __shfl_xor_sync(0xffffffffu, resid, o);
-      if (lane == 0 && resid != 0.f) atomicAdd(&G.ep.res[mat], resid);
-    }
-    if (nonfinite) raise_flag(flags, DEV_FLAG_NONFINITE);
   }
 
   tc_fence_before();
@@ -357,8 +401,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     tmem_dealloc(taddr, TMEM_COLS);
   }
-  if (L.profile && threadIdx.x == 0 && prof_flops)
-    atomicAdd(&prof_flops[L.prof_slot], G.flops_per_matrix / tiles);
 }
 
 }  // namespace
@@ -388,9 +430,10 @@ int get_encoder() {
 
 // Tensor map over a split stack (batch, 2, n, n) fp32: dimensions (innermost
 // first) column = n, row = n, plane = 2, matrix = batch; box {32, box_rows, 1,
-// 1} (one plane of a box_rows x 32 tile per copy).  K-major operand tiles use
-// the 128-byte swizzle; MN-major tiles (mn_layout) the 128-byte swizzle with
-// 32-byte atoms, the only MN-major tf32 layout of the tensor core.
+// 1} (one plane of a tile per copy).  K-major operand tiles (box_rows x 16)
+// use the 64-byte swizzle; MN-major tiles (mn_layout: 16 rows of K x 32
+// columns) the 128-byte swizzle with 32-byte atoms, the only MN-major tf32
+// layout of the tensor core.
 int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout) {
   int rc = get_encoder();
   if (rc) return rc;
@@ -398,11 +441,13 @@ int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, 
   const cuuint64_t nn = static_cast<cuuint64_t>(n);
   cuuint64_t dims[4] = {nn, nn, 2, static_cast<cuuint64_t>(batch)};
   cuuint64_t strides[3] = {nn * 4, nn * nn * 4, 2 * nn * nn * 4};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows), 1, 1};
+  // K-major boxes: BK columns (64 bytes) x box_rows rows; MN-major boxes: 32
+  // columns (128 bytes) x box_rows (= BK) rows of K.
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(mn_layout ? 32 : BK), static_cast<cuuint32_t>(box_rows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        mn_layout ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                        mn_layout ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(-4, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
@@ -466,11 +511,19 @@ int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
     flops += g.flops_per_matrix * g.batch;
   }
   if (total == 0) return 0;
-  if (total > 0x7fffffff) return set_error(-2, "GEMM launch too large (%lld CTAs)", (long long)total);
+  if (total > 0x7fffffff) return set_error(-2, "GEMM launch too large (%lld tiles)", (long long)total);
+  static int sm_count[32] = {0};
+  if (dev < 32 && sm_count[dev] == 0) {
+    rc = check_cuda(cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev), "SM count");
+    if (rc) return rc;
+  }
+  const int sms = (dev < 32 && sm_count[dev] > 0) ? sm_count[dev] : 148;
+  L.total_tiles = static_cast<int>(total);
   L.profile = profiling_enabled() ? 1 : 0;
   L.prof_slot = K_GEMM;
+  const unsigned grid = static_cast<unsigned>(total < sms ? total : sms);
   ProfScope ps(K_GEMM, st, flops, 0.0);
-  gemm3x_tf32_kernel<<<static_cast<unsigned>(total), THREADS, SMEM_BYTES, st>>>(L, maps, device_flop_slots());
+  gemm3x_tf32_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(L, maps, device_flop_slots());
   count_launch();
   return check_cuda(cudaGetLastError(), "gemm3x_tf32_kernel launch");
 }

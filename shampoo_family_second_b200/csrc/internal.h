@@ -60,13 +60,14 @@ struct GemmGroup {
   int a_off, b_off;  // matrix index offsets into the mapped stacks
   int a_rows, b_rows;  // box rows of the two maps (min(tile, n))
   int b_mn;            // 1: B is read MN-major (D = A B); 0: K-major (D = A B^T)
-  int tiles_m, tiles_n, cta_begin;  // filled by launch_gemm
+  int tiles_m, tiles_n, cta_begin;  // filled by launch_gemm (cta_begin: first tile of the group)
   double flops_per_matrix;          // algorithmic flops (profiling only)
   Epilogue ep;
 };
 
 struct GemmLaunch {
   int ngroups;
+  int total_tiles;  // filled by launch_gemm
   int profile;  // accumulate executed algorithmic flops into the profiler slot
   int prof_slot;
   GemmGroup g[kMaxGroups];
@@ -79,7 +80,7 @@ struct TmaMaps {
 // GEMM tile geometry (tcgen05 kind::tf32, one CTA per tile).
 constexpr int kTileM = 128;
 constexpr int kTileN = 256;
-constexpr int kTileK = 32;
+constexpr int kTileK = 16;
 
 // Host helpers -------------------------------------------------------------
 int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout = 0);

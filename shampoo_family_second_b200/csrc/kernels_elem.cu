@@ -104,10 +104,18 @@ __global__ void frob_norm_kernel(const float* __restrict__ A, int n, const int* 
   }
 }
 
+// Damping actually applied by the solvers: eps_eff = max(eps, u s) with
+// u = 2^-24 and s = ||A + eps I||_F.  Statistics accumulated in fp32 carry
+// rounding errors of about u s, which can make A + eps I indefinite when eps
+// is below that level; the iterations would then grow the negative
+// eigenvalue until it overflows.  A shift of u s is the size of rounding A to
+// fp32 and keeps the scaled matrix positive definite.
+__device__ __forceinline__ float effective_eps(float eps, float s) { return fmaxf(eps, s * 5.9604645e-8f); }
+
 // ---------------------------------------------------------------------------
-// Solver prologues.  A' = (sym(A) + eps I) / s on the valid region; the padded
-// region of a ragged block gets the identity (its root is then exactly the
-// identity times s^{-1/p} and never slows convergence).
+// Solver prologues.  A' = (sym(A) + eps_eff I) / s on the valid region; the
+// padded region of a ragged block gets the identity (its root is then exactly
+// the identity times s^{-1/p} and never slows convergence).
 //   kind 0, coupled Newton: out0 = M0 = A', out1 = T0 = ((p+1) I - A') / p,
 //                           out2 = X1 = T0.
 //   kind 1, Newton-DB:      out0 = Y0 = A', out1 = T0 = (3 I - A') / 2,
@@ -132,12 +140,13 @@ __global__ void root_prologue_kernel(int kind, const float* __restrict__ A, int 
   __syncthreads();
   const int v = valid ? valid[i] : n;
   const float inv_s = 1.f / s[i];
+  const float eps_eff = effective_eps(eps, s[i]);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int r = bi * 32 + ty + 8 * k, c = bj * 32 + tx;
     const float sym = 0.5f * (t1[ty + 8 * k][tx] + t2[tx][ty + 8 * k]);
     const float d = (r == c) ? 1.f : 0.f;
-    const float m = (r < v && c < v) ? (sym + d * eps) * inv_s : d;
+    const float m = (r < v && c < v) ? (sym + d * eps_eff) * inv_s : d;
     float t;
     if (kind == 0)
       t = (static_cast<float>(p + 1) * d - m) / static_cast<float>(p);
@@ -229,7 +238,7 @@ __global__ void cheb_coef_kernel(const float* __restrict__ s, int degree, int p,
                                  float* __restrict__ coef, float* __restrict__ sc) {
   const int i = blockIdx.x;
   const double sv = s[i];
-  const double base = (lo > 0.f) ? static_cast<double>(lo) : static_cast<double>(eps);
+  const double base = (lo > 0.f) ? static_cast<double>(lo) : static_cast<double>(effective_eps(eps, s[i]));
   double a = base / sv;
   if (a >= 1.0) a = 0.5;
   const int d = degree;
@@ -272,6 +281,7 @@ __global__ void cheb_prologue_kernel(const float* __restrict__ A, int n, const i
   __syncthreads();
   const int v = valid ? valid[i] : n;
   const float inv_s = 1.f / s[i];
+  const float eps_eff = effective_eps(eps, s[i]);
   const float* ci = coef + static_cast<size_t>(i) * (degree + 2);
   const float a = ci[degree + 1];
   const float cd = ci[degree], cd1 = ci[degree - 1];
@@ -280,7 +290,7 @@ __global__ void cheb_prologue_kernel(const float* __restrict__ A, int n, const i
     const int r = bi * 32 + ty + 8 * k, c = bj * 32 + tx;
     const float sym = 0.5f * (t1[ty + 8 * k][tx] + t2[tx][ty + 8 * k]);
     const float d = (r == c) ? 1.f : 0.f;
-    const float m = (r < v && c < v) ? (sym + d * eps) * inv_s : d;
+    const float m = (r < v && c < v) ? (sym + d * eps_eff) * inv_s : d;
     const float x = (2.f * m - (1.f + a) * d) / (1.f - a);
     const size_t idx = static_cast<size_t>(r) * n + c;
     store_split(Xt, i, nn, idx, x);

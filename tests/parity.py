@@ -13,6 +13,15 @@ allows.  The floor F is the larger of two measured numbers:
 
 The gate is max(2e-3, 2 F).  In well-conditioned cases F is far below 1e-3
 and the gate is the plain 2e-3.
+
+Update gate.  The same reading for the preconditioned update: F_update is the
+relative error, against the float64 oracle, of an fp32 reference pipeline
+(float32 statistics and products, single-precision LAPACK roots) run on the
+same gradients; the gate is max(2e-3, 2 F_update).
+
+Both fp32 references damp with eps_eff = max(eps, u ||A + eps I||_F), the
+damping the GPU solvers apply: statistics accumulated in fp32 can be
+indefinite at the level u ||A||, and a smaller eps is below fp32 resolution.
 """
 import numpy as np
 import scipy.linalg
@@ -37,7 +46,14 @@ def perturbation_floor(A, p, eps, seeds=5, u=U32):
     return float(np.median(out))
 
 
+def effective_eps(A, eps):
+    n = np.asarray(A).shape[0]
+    s = np.linalg.norm(np.asarray(A, dtype=np.float64) + eps * np.eye(n))
+    return max(eps, U32 * s)
+
+
 def lapack_fp32_root(A, p, eps):
+    eps = effective_eps(A, eps)
     A32 = np.asarray(A, dtype=np.float32)
     A32 = (A32 + A32.T) * np.float32(0.5)
     lam, Q = scipy.linalg.eigh(A32, driver="evd")
@@ -60,3 +76,37 @@ def conditioning_floor(A, p, eps):
 
 def root_gate(A, p, eps):
     return max(BASE_TOL, 2.0 * conditioning_floor(A, p, eps))
+
+
+class Fp32ReferenceShampoo:
+    """The blocked step in float32 with LAPACK roots: the update floor's
+    reference (statistics, roots and products all in single precision)."""
+
+    def __init__(self, shapes, block, beta, eps, root_p, refresh_every, blocks):
+        from oracle import block_table
+        self.table = block_table(shapes, block)
+        self.blocks = list(blocks)
+        self.beta, self.eps, self.p, self.k = np.float32(beta), eps, root_p, refresh_every
+        self.L = {b: np.zeros((self.table[b].r,) * 2, np.float32) for b in self.blocks}
+        self.R = {b: np.zeros((self.table[b].c,) * 2, np.float32) for b in self.blocks}
+        self.XL, self.XR = {}, {}
+        self.t = 0
+
+    def step(self, grads):
+        P = {}
+        refresh = self.t % self.k == 0
+        for b in self.blocks:
+            blk = self.table[b]
+            G = np.asarray(grads[blk.param][blk.row0:blk.row0 + blk.r, blk.col0:blk.col0 + blk.c], np.float32)
+            self.L[b] = self.beta * self.L[b] + G @ G.T
+            self.R[b] = self.beta * self.R[b] + G.T @ G
+            if refresh:
+                self.XL[b] = lapack_fp32_root(self.L[b], self.p, self.eps).astype(np.float32)
+                self.XR[b] = lapack_fp32_root(self.R[b], self.p, self.eps).astype(np.float32)
+            P[b] = (self.XL[b] @ G @ self.XR[b]).astype(np.float64)
+        self.t += 1
+        return P
+
+
+def update_gate(P_fp32, P_oracle):
+    return max(BASE_TOL, 2.0 * rel_fro(P_fp32, P_oracle))

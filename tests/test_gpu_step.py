@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 
 import oracle
 import workloads
-from parity import root_gate
+from parity import Fp32ReferenceShampoo, root_gate, update_gate
 
 TOL_UPDATE = 2e-3
 TOL_ROOT = 2e-3
@@ -39,6 +39,7 @@ def run_parity(sb, wl, steps, check_roots=True, blocks=None):
                                blocks=blocks)
     table = opt.block_table()
     assert [tuple(t) for t in table] == [(b.param, b.row0, b.col0, b.r, b.c) for b in ref.table]
+    ref32 = Fp32ReferenceShampoo(wl.shapes, wl.block, wl.beta, wl.eps, wl.root_p, wl.refresh_every, ref.active)
     stream = workloads.GradientStream(wl)
     worst = {"update": 0.0, "root": 0.0, "stats": 0.0}
     for t in range(steps):
@@ -50,6 +51,7 @@ def run_parity(sb, wl, steps, check_roots=True, blocks=None):
         before = [w.clone() for w in W]
         opt.step(W, G)
         P_ref = ref.step(grads)
+        P_32 = ref32.step(grads)
         torch.cuda.synchronize()
         dW = [((b - a) / wl.lr).cpu().numpy().astype(np.float64) for a, b in zip(W, before)]
         L, R = opt.statistics()
@@ -62,7 +64,7 @@ def run_parity(sb, wl, steps, check_roots=True, blocks=None):
             Pg = dW[blk.param][blk.row0:blk.row0 + blk.r, blk.col0:blk.col0 + blk.c]
             e = oracle.rel_fro(Pg, P_ref[b])
             worst["update"] = max(worst["update"], e)
-            assert e < TOL_UPDATE, (t, b, "update", e)
+            assert e < update_gate(P_32[b], P_ref[b]), (t, b, "update", e)
             es = max(oracle.rel_fro(L[b, :blk.r, :blk.r], ref.L[b]), oracle.rel_fro(R[b, :blk.c, :blk.c], ref.R[b]))
             worst["stats"] = max(worst["stats"], es)
             assert es < TOL_STATS, (t, b, "stats", es)
