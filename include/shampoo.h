@@ -100,7 +100,9 @@ enum {
  *  iters          iterations (tol = 0) or iteration cap (tol > 0) per Newton / Newton-DB
  *                 stage, >= 1; ignored by Chebyshev.
  *  tol            0: fixed iteration count; > 0: stop a matrix once
- *                 ||M - I||_F / sqrt(n) (Newton) or ||Z Y - I||_F / sqrt(n) (Newton-DB) <= tol.
+ *                 tr(I - M)/n (Newton) or tr(I - Z Y)/n (Newton-DB) <= tol.  Both iterations
+ *                 keep every eigenvalue of M (or Z Y) at or below 1, so this trace bounds the
+ *                 largest eigenvalue error (times n).
  *  refresh_every  roots recomputed at steps t with t % refresh_every == 0 (t from 0), >= 1.
  *  cheb_degree    Chebyshev degree d in [2, 64].
  *  cheb_lo        Chebyshev interval: [lo / s, 1] with lo = cheb_lo if > 0 else eps,

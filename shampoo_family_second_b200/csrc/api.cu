@@ -315,7 +315,7 @@ int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d
     Builder b;
     Epilogue& e = b.add(nb, B, h->mRoots, 0, h->mGt, 0, h->stats_flops_L);
     e.D = h->Tap;
-    e.d_split = 1;
+    e.d_planes = 2;
     e.flags = h->d_status;
     if ((rc = b.launch(st))) return rc;
   }
@@ -449,7 +449,8 @@ int shampoo_gemm_batched(const float* d_A, const float* d_B, const float* d_C, f
   StackMaps ma, mb;
   if ((rc = make_stack_maps(ma, As, batch, n)) || (rc = make_stack_maps(mb, Bs, batch, n))) return rc;
   Builder b;
-  Epilogue& e = b.add(static_cast<int>(batch), n, ma, 0, mb, 0, 2.0 * n * double(n) * n, op_b);
+  Epilogue& e = b.add(static_cast<int>(batch), n, ma, 0, mb, 0, 2.0 * n * double(n) * n,
+                      op_b ? B_MN_MAJOR : B_TRANSPOSED);
   e.alpha = alpha;
   e.beta = d_C ? beta : 0.f;
   e.gamma = gamma;

@@ -70,7 +70,7 @@ __device__ __forceinline__ float epilogue_chunk(const GemmGroup& G, int mat, int
   const int dj = r - c0;
   float resid = 0.f;
   bool bad = false;
-  const size_t dplane = E.d_split ? 2 * nn : nn;
+  const size_t dstride = static_cast<size_t>(E.d_planes) * nn;
   float* wrow = nullptr;
   int wc = 0;
   if (E.wptr) {
@@ -87,15 +87,15 @@ __device__ __forceinline__ float epilogue_chunk(const GemmGroup& G, int mat, int
       const float a = acc[jj];
       if (E.res) {
         const int c = c0 + jj;
-        const float d = a - ((r == c) ? 1.f : 0.f);
-        resid += (r < vsz && c < vsz) ? d * d : 0.f;
+        resid += (r == c && r < vsz) ? 1.f - a : 0.f;
       }
       v[j] = E.alpha * a;
     }
     if (E.C) {
-      if (E.c_split) {
-        const float4* h4 = reinterpret_cast<const float4*>(E.C + mat * 2 * nn + row_off + 8 * g);
-        const float4* l4 = reinterpret_cast<const float4*>(E.C + mat * 2 * nn + nn + row_off + 8 * g);
+      if (E.c_planes >= 2) {
+        const float* cb = E.C + mat * static_cast<size_t>(E.c_planes) * nn + row_off + 8 * g;
+        const float4* h4 = reinterpret_cast<const float4*>(cb);
+        const float4* l4 = reinterpret_cast<const float4*>(cb + nn);
         const float4 h0 = h4[0], h1 = h4[1], l0 = l4[0], l1 = l4[1];
         v[0] += E.beta * (h0.x + l0.x); v[1] += E.beta * (h0.y + l0.y);
         v[2] += E.beta * (h0.z + l0.z); v[3] += E.beta * (h0.w + l0.w);
@@ -115,8 +115,9 @@ __device__ __forceinline__ float epilogue_chunk(const GemmGroup& G, int mat, int
       bad |= !isfinite(v[j]);
     }
     if (E.D) {
-      float* d = E.D + mat * dplane + row_off + 8 * g;
-      if (E.d_split) {
+      float* dm = E.D + mat * dstride;
+      float* d = dm + row_off + 8 * g;
+      if (E.d_planes >= 2) {
         float hh[8], ll[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) split_tf32(v[j], hh[j], ll[j]);
@@ -410,6 +411,9 @@ Epilogue epilogue_defaults() {
   std::memset(&e, 0, sizeof(e));
   e.alpha = 1.f;
   e.gamma_stride = 1;
+  e.c_planes = 1;
+  e.d_planes = 1;
+  e.e_planes = 2;
   return e;
 }
 
@@ -434,13 +438,14 @@ int get_encoder() {
 // use the 64-byte swizzle; MN-major tiles (mn_layout: 16 rows of K x 32
 // columns) the 128-byte swizzle with 32-byte atoms, the only MN-major tf32
 // layout of the tensor core.
-int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout) {
+int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout,
+                     int planes) {
   int rc = get_encoder();
   if (rc) return rc;
   if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return set_error(-2, "stack base not 16-byte aligned");
   const cuuint64_t nn = static_cast<cuuint64_t>(n);
   cuuint64_t dims[4] = {nn, nn, 2, static_cast<cuuint64_t>(batch)};
-  cuuint64_t strides[3] = {nn * 4, nn * nn * 4, 2 * nn * nn * 4};
+  cuuint64_t strides[3] = {nn * 4, nn * nn * 4, static_cast<cuuint64_t>(planes) * nn * nn * 4};
   // K-major boxes: BK columns (64 bytes) x box_rows rows; MN-major boxes: 32
   // columns (128 bytes) x box_rows (= BK) rows of K.
   cuuint32_t box[4] = {static_cast<cuuint32_t>(mn_layout ? 32 : BK), static_cast<cuuint32_t>(box_rows), 1, 1};
@@ -454,14 +459,15 @@ int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, 
   return 0;
 }
 
-int make_stack_maps(StackMaps& sm, float* base, int64_t batch, int n) {
+int make_stack_maps(StackMaps& sm, float* base, int64_t batch, int n, int planes) {
   sm.base = base;
+  sm.planes = planes;
   sm.a_rows = n < BM ? n : BM;
   sm.b_rows = n < BN ? n : BN;
-  int rc = encode_split_map(&sm.a, base, batch, n, sm.a_rows);
+  int rc = encode_split_map(&sm.a, base, batch, n, sm.a_rows, 0, planes);
   if (rc) return rc;
-  if ((rc = encode_split_map(&sm.mn, base, batch, n, BK, 1))) return rc;
-  return encode_split_map(&sm.b, base, batch, n, sm.b_rows);
+  if ((rc = encode_split_map(&sm.mn, base, batch, n, BK, 1, planes))) return rc;
+  return encode_split_map(&sm.b, base, batch, n, sm.b_rows, 0, planes);
 }
 
 Builder::Builder() : nmaps(0) {
@@ -470,15 +476,15 @@ Builder::Builder() : nmaps(0) {
 }
 
 Epilogue& Builder::add(int batch, int n, const StackMaps& a, int a_off, const StackMaps& b, int b_off,
-                       double flops_per_matrix, int b_mn) {
+                       double flops_per_matrix, int bmode) {
   GemmGroup& g = L.g[L.ngroups++];
   g.batch = batch;
   g.n = n;
   M.m[nmaps] = a.a;
   g.a_map = nmaps++;
-  M.m[nmaps] = b_mn ? b.mn : b.b;
+  M.m[nmaps] = bmode == B_MN_MAJOR ? b.mn : b.b;
   g.b_map = nmaps++;
-  g.b_mn = b_mn;
+  g.b_mn = bmode == B_MN_MAJOR ? 1 : 0;
   g.a_off = a_off;
   g.b_off = b_off;
   g.a_rows = a.a_rows;

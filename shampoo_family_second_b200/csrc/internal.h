@@ -10,14 +10,17 @@
 namespace shampoo {
 
 // ---------------------------------------------------------------------------
-// Storage formats
-//   plain stack : (batch, n, n) fp32, row-major matrices back to back.
-//   split stack : (batch, 2, n, n) fp32; matrix i holds its tf32-exact "hi"
-//                 plane then its "lo" plane (value = hi + lo, see split_tf32).
+// Storage formats (P = planes per matrix, matrix stride P n^2 floats)
+//   plain stack  (P = 1): (batch, n, n) fp32, row-major matrices back to back.
+//   split stack  (P = 2): matrix i holds its tf32-exact "hi" plane then its
+//                "lo" plane (value = hi + lo, see split_tf32).
 // Split stacks are the operand format of the tensor-core GEMM.
 // ---------------------------------------------------------------------------
 inline size_t plain_floats(int64_t batch, int n) { return static_cast<size_t>(batch) * n * n; }
 inline size_t split_floats(int64_t batch, int n) { return 2 * static_cast<size_t>(batch) * n * n; }
+inline size_t stack_floats(int64_t batch, int n, int planes) {
+  return static_cast<size_t>(planes) * batch * n * n;
+}
 
 constexpr int kMaxGroups = 4;
 constexpr int kMaxMaps = 2 * kMaxGroups;
@@ -34,13 +37,14 @@ struct Epilogue {
   const float* gamma_vec;
   int gamma_stride;
   const float* scale_vec;
-  const float* C;  // optional input stack
-  int c_split;     // C is a split stack (else plain)
+  const float* C;  // optional input stack (its value planes are read)
+  int c_planes;    // 1 (plain) or 2 (split)
   float* D;        // optional main output stack
-  int d_split;     // D is a split stack (else plain)
+  int d_planes;    // 1 (plain) or 2 (split)
   float* E;        // optional second output (split): e_mul * v + e_add * [r == c]
+  int e_planes;    // 2
   float e_mul, e_add;
-  float* res;        // optional: res[i] += sum over the valid region of (acc - [r == c])^2
+  float* res;        // optional: res[i] += sum over the valid diagonal of (1 - acc): tr(I - acc)
   const int* valid;  // per-matrix valid extent (nullable: n)
   const int* skip;   // per-matrix "done" flags: a set flag skips the matrix
   int* flags;        // device status word (nullable)
@@ -83,7 +87,8 @@ constexpr int kTileN = 256;
 constexpr int kTileK = 16;
 
 // Host helpers -------------------------------------------------------------
-int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout = 0);
+int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout,
+                     int planes);
 int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st);
 Epilogue epilogue_defaults();
 
@@ -118,12 +123,17 @@ double* device_flop_slots();  // device address of the executed-flop accumulator
 
 // A GEMM launch under construction: groups plus the tensor maps they reference.
 struct StackMaps {
-  CUtensorMap a, b;  // the split stack as A (128-row boxes) and as K-major B (256-row boxes)
-  CUtensorMap mn;    // as MN-major B: 32 x 32 boxes (32 rows of K, 32 columns of N)
+  CUtensorMap a, b;  // the stack as A (128-row boxes) and as K-major B (256-row boxes)
+  CUtensorMap mn;    // as MN-major B: 16 rows of K x 32 columns of N
   float* base;
+  int planes;
   int a_rows, b_rows;
 };
-int make_stack_maps(StackMaps& sm, float* base, int64_t batch, int n);
+int make_stack_maps(StackMaps& sm, float* base, int64_t batch, int n, int planes = 2);
+
+// How a group reads its B operand: as B^T (K-major; D = A B^T) or as B
+// (MN-major; D = A B).
+enum BMode : int { B_TRANSPOSED = 0, B_MN_MAJOR = 1 };
 
 struct Builder {
   GemmLaunch L;
@@ -133,7 +143,7 @@ struct Builder {
   // Adds a group D_i = epi(A_i B_i^T) (b_mn = 0) or epi(A_i B_i) (b_mn = 1)
   // over matrices a_off.. of `a` and b_off.. of `b`.
   Epilogue& add(int batch, int n, const StackMaps& a, int a_off, const StackMaps& b, int b_off,
-                double flops_per_matrix, int b_mn = 0);
+                double flops_per_matrix, int bmode = B_TRANSPOSED);
   int launch(cudaStream_t st) { return launch_gemm(L, M, st); }
 };
 
@@ -155,17 +165,19 @@ int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, flo
 // kind: 0 = Newton (M0, T0 = ((p+1)I - M0)/p, X1 = T0)
 //       1 = Newton-DB (Y0 = A', T0 = (3I - A')/2, Z1 = T0)
 int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const int* valid, float eps, int p,
-                         const float* s, float* out0, float* out1, float* out2, cudaStream_t st);
+                         const float* s, float* out0, float* out1, float* out2, int planes0, int planes1, int planes2,
+                         cudaStream_t st);
 // Second Newton-DB stage: Y0' = Y_par(i) (parity from iters), T0 = (3I - Y0')/2, Z1 = T0.
 int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters, int64_t batch, int n,
                               float* Ynew0, float* T, float* Z1, cudaStream_t st);
 int launch_check(float* res, int* done, int* iters, const int* valid, int64_t batch, int n, float tol, int it,
                  int* flags, cudaStream_t st);
-int launch_finalize(const float* X0, const float* X1, const int* iters, int default_iters, const float* sc,
-                    int64_t batch, int n, float* out_plain, float* out_split, int* flags, cudaStream_t st);
+int launch_finalize(const float* X0, const float* X1, int src_planes, const int* iters, int default_iters,
+                    const float* sc, int64_t batch, int n, float* out_plain, float* out_split, int* flags,
+                    cudaStream_t st);
 int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int degree,
                       float lo, const float* s, float* coef, float* sc, float* Xt, float* bd, float* bd1,
-                      cudaStream_t st);
+                      int xt_planes, int b_planes, cudaStream_t st);
 int launch_fill_iters(int* iters, int64_t batch, int value, cudaStream_t st);
 
 // Inverse-root solver (solver.cu) ---------------------------------------------

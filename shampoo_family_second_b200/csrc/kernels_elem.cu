@@ -26,6 +26,15 @@ __device__ __forceinline__ void store_split(float* stack, size_t mat, size_t nn,
   stack[mat * 2 * nn + nn + idx] = l;
 }
 
+// Matrix `mat` of a stack with `planes` planes per matrix (2: split).
+__device__ __forceinline__ void store_sym(float* stack, int planes, size_t mat, size_t nn, size_t idx, float v) {
+  float h, l;
+  split_tf32(v, h, l);
+  float* m = stack + mat * planes * nn;
+  m[idx] = h;
+  m[nn + idx] = l;
+}
+
 // ---------------------------------------------------------------------------
 // A1 partition / stack.  DASH abstract: preconditioner blocks stacked into 3D
 // tensors.  Block b of the table {param, row0, col0, r, c} is copied from the
@@ -124,7 +133,8 @@ __device__ __forceinline__ float effective_eps(float eps, float s) { return fmax
 // ---------------------------------------------------------------------------
 __global__ void root_prologue_kernel(int kind, const float* __restrict__ A, int n, const int* __restrict__ valid,
                                      float eps, int p, const float* __restrict__ s, float* __restrict__ out0,
-                                     float* __restrict__ out1, float* __restrict__ out2) {
+                                     float* __restrict__ out1, float* __restrict__ out2, int planes0, int planes1,
+                                     int planes2) {
   __shared__ float t1[32][33];
   __shared__ float t2[32][33];
   const int i = blockIdx.z;
@@ -153,9 +163,9 @@ __global__ void root_prologue_kernel(int kind, const float* __restrict__ A, int 
     else
       t = 0.5f * (3.f * d - m);
     const size_t idx = static_cast<size_t>(r) * n + c;
-    store_split(out0, i, nn, idx, m);
-    store_split(out1, i, nn, idx, t);
-    store_split(out2, i, nn, idx, t);
+    store_sym(out0, planes0, i, nn, idx, m);
+    store_sym(out1, planes1, i, nn, idx, t);
+    store_sym(out2, planes2, i, nn, idx, t);
   }
 }
 
@@ -176,8 +186,8 @@ __global__ void db_stage2_kernel(const float* Y0, const float* Y1, const int* __
   store_split(Z1, i, nn, idx, t);
 }
 
-// Residual check after iteration `it`: ||acc - I||_F / sqrt(valid) <= tol
-// marks the matrix done (its later GEMM tiles are skipped).
+// Residual check after iteration `it`: |tr(I - acc)| / valid <= tol marks the
+// matrix done (its later GEMM tiles are skipped).
 __global__ void check_kernel(float* res, int* done, int* iters, const int* valid, int batch, int n, float tol,
                              int it, int* flags) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -187,7 +197,7 @@ __global__ void check_kernel(float* res, int* done, int* iters, const int* valid
     return;
   }
   const int v = valid ? valid[i] : n;
-  const float r = sqrtf(res[i] / static_cast<float>(v));
+  const float r = fabsf(res[i]) / static_cast<float>(v);
   res[i] = 0.f;
   iters[i] = it;
   if (!isfinite(r)) {
@@ -198,33 +208,43 @@ __global__ void check_kernel(float* res, int* done, int* iters, const int* valid
   }
 }
 
-// Output pass: X = (hi + lo of the final iterate) * s^{-1/p}; the final iterate
-// sits in buffer (iters[i] & 1).  Writes a plain and/or a split stack.
-__global__ void finalize_kernel(const float* __restrict__ X0, const float* __restrict__ X1,
+// Output pass: X = sym(hi + lo of the final iterate) * s^{-1/p}, with
+// sym(Y) = (Y + Y^T)/2.  The principal root is symmetric; the iterates pick
+// up a small antisymmetric rounding component (the products are formed as
+// A B^T), which this removes.  The final iterate sits in buffer
+// (iters[i] & 1).  Writes a plain and/or a split stack.
+// grid (n/32, n/32, batch), block (32, 8).
+__global__ void finalize_kernel(const float* __restrict__ X0, const float* __restrict__ X1, int src_planes,
                                 const int* __restrict__ iters, int default_iters, const float* __restrict__ sc, int n,
                                 float* __restrict__ out_plain, float* __restrict__ out_split, int* flags) {
-  const int i = blockIdx.y;
+  __shared__ float t1[32][33];
+  __shared__ float t2[32][33];
+  const int i = blockIdx.z;
+  const int bi = blockIdx.y, bj = blockIdx.x;
+  const int tx = threadIdx.x, ty = threadIdx.y;
   const size_t nn = static_cast<size_t>(n) * n;
-  const size_t idx = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
-  if (idx >= nn) return;
   const int it = iters ? iters[i] : default_iters;
-  const float* src = (it & 1) ? X1 : X0;
-  const float4 h = *reinterpret_cast<const float4*>(src + i * 2 * nn + idx);
-  const float4 l = *reinterpret_cast<const float4*>(src + i * 2 * nn + nn + idx);
+  const float* src = ((it & 1) ? X1 : X0) + i * static_cast<size_t>(src_planes) * nn;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const size_t a = static_cast<size_t>(bi * 32 + ty + 8 * k) * n + bj * 32 + tx;
+    const size_t b = static_cast<size_t>(bj * 32 + ty + 8 * k) * n + bi * 32 + tx;
+    t1[ty + 8 * k][tx] = src[a] + src[nn + a];
+    t2[ty + 8 * k][tx] = src[b] + src[nn + b];
+  }
+  __syncthreads();
   const float f = sc[i];
-  float v[4] = {(h.x + l.x) * f, (h.y + l.y) * f, (h.z + l.z) * f, (h.w + l.w) * f};
   bool bad = false;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) bad |= !isfinite(v[q]);
-  if (bad) raise_flag(flags, DEV_FLAG_NONFINITE);
-  if (out_plain) *reinterpret_cast<float4*>(out_plain + i * nn + idx) = make_float4(v[0], v[1], v[2], v[3]);
-  if (out_split) {
-    float hh[4], ll[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) split_tf32(v[q], hh[q], ll[q]);
-    *reinterpret_cast<float4*>(out_split + i * 2 * nn + idx) = make_float4(hh[0], hh[1], hh[2], hh[3]);
-    *reinterpret_cast<float4*>(out_split + i * 2 * nn + nn + idx) = make_float4(ll[0], ll[1], ll[2], ll[3]);
+  for (int k = 0; k < 4; ++k) {
+    const int r = bi * 32 + ty + 8 * k, c = bj * 32 + tx;
+    const float v = 0.5f * (t1[ty + 8 * k][tx] + t2[tx][ty + 8 * k]) * f;
+    bad |= !isfinite(v);
+    const size_t idx = static_cast<size_t>(r) * n + c;
+    if (out_plain) out_plain[i * nn + idx] = v;
+    if (out_split) store_split(out_split, i, nn, idx, v);
   }
+  if (bad) raise_flag(flags, DEV_FLAG_NONFINITE);
 }
 
 // ---------------------------------------------------------------------------
@@ -265,7 +285,8 @@ __global__ void cheb_coef_kernel(const float* __restrict__ s, int degree, int p,
 // b_d = c_d I and b_{d-1} = 2 c_d Xt + c_{d-1} I (first two Clenshaw terms).
 __global__ void cheb_prologue_kernel(const float* __restrict__ A, int n, const int* __restrict__ valid, float eps,
                                      const float* __restrict__ s, const float* __restrict__ coef, int degree,
-                                     float* __restrict__ Xt, float* __restrict__ bd, float* __restrict__ bd1) {
+                                     float* __restrict__ Xt, float* __restrict__ bd, float* __restrict__ bd1,
+                                     int xt_planes, int b_planes) {
   __shared__ float t1[32][33];
   __shared__ float t2[32][33];
   const int i = blockIdx.z;
@@ -293,9 +314,9 @@ __global__ void cheb_prologue_kernel(const float* __restrict__ A, int n, const i
     const float m = (r < v && c < v) ? (sym + d * eps_eff) * inv_s : d;
     const float x = (2.f * m - (1.f + a) * d) / (1.f - a);
     const size_t idx = static_cast<size_t>(r) * n + c;
-    store_split(Xt, i, nn, idx, x);
-    store_split(bd, i, nn, idx, cd * d);
-    store_split(bd1, i, nn, idx, 2.f * cd * x + cd1 * d);
+    store_sym(Xt, xt_planes, i, nn, idx, x);
+    store_sym(bd, b_planes, i, nn, idx, cd * d);
+    store_sym(bd1, b_planes, i, nn, idx, 2.f * cd * x + cd1 * d);
   }
 }
 
@@ -326,11 +347,13 @@ int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, flo
 }
 
 int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const int* valid, float eps, int p,
-                         const float* s, float* out0, float* out1, float* out2, cudaStream_t st) {
+                         const float* s, float* out0, float* out1, float* out2, int planes0, int planes1, int planes2,
+                         cudaStream_t st) {
   if (batch == 0) return 0;
-  ProfScope ps(K_PROLOGUE, st, 0.0, (4.0 + 3 * 8.0) * batch * n * n);
+  ProfScope ps(K_PROLOGUE, st, 0.0, (4.0 + 4.0 * (planes0 + planes1 + planes2)) * batch * n * n);
   dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
-  root_prologue_kernel<<<grid, block, 0, st>>>(kind, A, n, valid, eps, p, s, out0, out1, out2);
+  root_prologue_kernel<<<grid, block, 0, st>>>(kind, A, n, valid, eps, p, s, out0, out1, out2, planes0, planes1,
+                                               planes2);
   count_launch();
   return check_cuda(cudaGetLastError(), "root_prologue_kernel");
 }
@@ -356,20 +379,22 @@ int launch_check(float* res, int* done, int* iters, const int* valid, int64_t ba
   return check_cuda(cudaGetLastError(), "check_kernel");
 }
 
-int launch_finalize(const float* X0, const float* X1, const int* iters, int default_iters, const float* sc,
-                    int64_t batch, int n, float* out_plain, float* out_split, int* flags, cudaStream_t st) {
+int launch_finalize(const float* X0, const float* X1, int src_planes, const int* iters, int default_iters,
+                    const float* sc, int64_t batch, int n, float* out_plain, float* out_split, int* flags,
+                    cudaStream_t st) {
   if (batch == 0) return 0;
   const double bytes = (8.0 + (out_plain ? 4.0 : 0.0) + (out_split ? 8.0 : 0.0)) * batch * n * n;
   ProfScope ps(K_FINALIZE, st, 0.0, bytes);
-  const size_t nn4 = static_cast<size_t>(n) * n / 4;
-  dim3 grid(static_cast<unsigned>((nn4 + 255) / 256), static_cast<unsigned>(batch));
-  finalize_kernel<<<grid, 256, 0, st>>>(X0, X1, iters, default_iters, sc, n, out_plain, out_split, flags);
+  dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
+  finalize_kernel<<<grid, block, 0, st>>>(X0, X1, src_planes, iters, default_iters, sc, n, out_plain, out_split,
+                                          flags);
   count_launch();
   return check_cuda(cudaGetLastError(), "finalize_kernel");
 }
 
 int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int degree, float lo,
-                      const float* s, float* coef, float* sc, float* Xt, float* bd, float* bd1, cudaStream_t st) {
+                      const float* s, float* coef, float* sc, float* Xt, float* bd, float* bd1, int xt_planes,
+                      int b_planes, cudaStream_t st) {
   if (batch == 0) return 0;
   {
     ProfScope ps(K_CHEB_COEF, st, 0.0, 8.0 * batch);
@@ -378,9 +403,9 @@ int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, fl
     int rc = check_cuda(cudaGetLastError(), "cheb_coef_kernel");
     if (rc) return rc;
   }
-  ProfScope ps(K_PROLOGUE, st, 0.0, (4.0 + 3 * 8.0) * batch * n * n);
+  ProfScope ps(K_PROLOGUE, st, 0.0, (4.0 + 4.0 * (xt_planes + 2 * b_planes)) * batch * n * n);
   dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
-  cheb_prologue_kernel<<<grid, block, 0, st>>>(A, n, valid, eps, s, coef, degree, Xt, bd, bd1);
+  cheb_prologue_kernel<<<grid, block, 0, st>>>(A, n, valid, eps, s, coef, degree, Xt, bd, bd1, xt_planes, b_planes);
   count_launch();
   return check_cuda(cudaGetLastError(), "cheb_prologue_kernel");
 }

@@ -14,14 +14,23 @@
 //                   a second stage on Y ~ A'^{1/2};
 //   Chebyshev       Clenshaw evaluation of the degree-d interpolant of x^{-1/p}
 //                   on [a, 1] (d - 1 GEMMs).
-// Every product is a true product A B (B read MN-major): with the implicit
-// transpose of a K-major B, rounding makes the iterates slightly unsymmetric
-// and the Newton-DB fixed point is unstable along that direction.
+// Operand orientation.  The tensor core computes A B^T from row-major stacks
+// fastest (both operands K-major).  The iterates are symmetric in exact
+// arithmetic, so A B^T is the wanted product up to rounding, which leaves a
+// small antisymmetric component in the iterates.  Coupled Newton and the
+// Clenshaw recurrence are stable under it (it neither grows nor disturbs the
+// symmetric part), so they use A B^T.  The Newton-DB fixed point is unstable
+// along that direction (the error grows about 1.5x per iteration), so its
+// products are true products A B with B read MN-major.
+// Convergence is measured by tr(I - M)/n (Newton) or tr(I - Z Y)/n (Newton-DB):
+// both iterations keep every eigenvalue of M (or Z Y) at or below 1, so the
+// trace bounds the largest eigenvalue error and ignores the antisymmetric
+// rounding component.
 // A' = (A + eps I)/||A + eps I||_F (Frobenius pre-scaling); the result is
 // unscaled by ||A + eps I||_F^{-1/p}.  With tol > 0 the residual
-// ||M - I||_F / sqrt(n) (Newton) or ||Z Y - I||_F / sqrt(n) (Newton-DB) is
-// checked after every iteration and converged matrices drop out of later
-// launches (their tiles exit at once); iters is then the cap.
+// tr(I - M)/n (Newton) or tr(I - Z Y)/n (Newton-DB) is checked after every
+// iteration and converged matrices drop out of later launches (their tiles
+// exit at once); iters is then the cap.
 #include <algorithm>
 #include <cstring>
 #include <vector>
@@ -31,12 +40,24 @@
 namespace shampoo {
 namespace {
 
-int stacks_for(int solver) {
-  switch (solver) {
-    case 0: return 7;  // M0 M1 X0 X1 T T2 T4
-    case 1: return 5;  // Y0 Y1 Z0 Z1 T
-    default: return 4; // Xt b0 b1 b2
-  }
+constexpr int NEWTON_B = B_TRANSPOSED;
+
+// Planes per matrix of each scratch stack, by solver (all split stacks).
+//   Newton    : M0 M1 X0 X1 T T2 T4
+//   Newton-DB : Y0 Y1 Z0 Z1 T
+//   Chebyshev : Xt b0 b1 b2
+constexpr int kNewtonPlanes[7] = {2, 2, 2, 2, 2, 2, 2};
+constexpr int kDbPlanes[5] = {2, 2, 2, 2, 2};
+constexpr int kChebPlanes[4] = {2, 2, 2, 2};
+
+int stacks_for(int solver) { return solver == 0 ? 7 : (solver == 1 ? 5 : 4); }
+int planes_of(int solver, int k) {
+  return solver == 0 ? kNewtonPlanes[k] : (solver == 1 ? kDbPlanes[k] : kChebPlanes[k]);
+}
+int total_planes(int solver) {
+  int t = 0;
+  for (int k = 0; k < stacks_for(solver); ++k) t += planes_of(solver, k);
+  return t;
 }
 
 constexpr size_t kAlign = 256;
@@ -71,7 +92,8 @@ Layout carve(void* base, int64_t cb, int n, int solver) {
   L.iters = reinterpret_cast<int*>(take(cb * 4));
   L.iters1 = reinterpret_cast<int*>(take(cb * 4));
   L.coef = reinterpret_cast<float*>(take(cb * 4 * (kMaxChebDegree + 2)));
-  for (int k = 0; k < stacks_for(solver); ++k) L.stack[k] = reinterpret_cast<float*>(take(split_floats(cb, n) * 4));
+  for (int k = 0; k < stacks_for(solver); ++k)
+    L.stack[k] = reinterpret_cast<float*>(take(stack_floats(cb, n, planes_of(solver, k)) * 4));
   return L;
 }
 
@@ -80,7 +102,7 @@ Layout carve(void* base, int64_t cb, int n, int solver) {
 size_t root_scratch_header() { return kHeader; }
 
 size_t root_scratch_per_matrix(int n, int solver) {
-  return static_cast<size_t>(stacks_for(solver)) * split_floats(1, n) * 4 + 4 * (kVecInts + kMaxChebDegree + 2);
+  return static_cast<size_t>(total_planes(solver)) * n * n * 4 + 4 * (kVecInts + kMaxChebDegree + 2);
 }
 
 int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, cudaStream_t st) {
@@ -88,8 +110,8 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
   const int p = job.p;
   const bool residual = job.tol > 0.f && job.solver != 2;
   const size_t per = root_scratch_per_matrix(n, job.solver);
-  if (scratch_bytes < kHeader + per) return set_error(-3, "inverse-root scratch too small: %zu < %zu bytes",
-                                                      scratch_bytes, kHeader + per);
+  if (scratch_bytes < kHeader + per)
+    return set_error(-3, "inverse-root scratch too small: %zu < %zu bytes", scratch_bytes, kHeader + per);
   const int64_t cb_max = std::min<int64_t>(job.batch, static_cast<int64_t>((scratch_bytes - kHeader) / per));
   const int64_t cb_cap = std::min<int64_t>(cb_max, 65535);  // grid.z limit of the prologues
   const double f1 = 2.0 * n * static_cast<double>(n) * n;  // one GEMM(n), algorithmic
@@ -105,37 +127,39 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
     int* iters_out = job.iters_used ? job.iters_used + off : nullptr;
     StackMaps sm[7];
     for (int k = 0; k < stacks_for(job.solver); ++k)
-      if ((rc = make_stack_maps(sm[k], S.stack[k], cb, n))) return rc;
+      if ((rc = make_stack_maps(sm[k], S.stack[k], cb, n, planes_of(job.solver, k)))) return rc;
     if ((rc = launch_frob_norm(A, cb, n, valid, job.eps, p, S.s, S.sc, st))) return rc;
     if (residual) {
       if ((rc = check_cuda(cudaMemsetAsync(S.done, 0, cb * 4, st), "memset done"))) return rc;
       if ((rc = check_cuda(cudaMemsetAsync(S.res, 0, cb * 4, st), "memset res"))) return rc;
     }
     const int* skip = residual ? S.done : nullptr;
+    auto common = [&](Epilogue& e) {
+      e.skip = skip;
+      e.flags = job.flags;
+    };
 
     if (job.solver == 0) {
       // ------------------------------------------------------------ coupled Newton
-      StackMaps* M = &sm[0];  // M[0], M[1]
-      StackMaps* X = &sm[2];  // X[0], X[1]
-      StackMaps& T = sm[4];
-      StackMaps& T2 = sm[5];
-      StackMaps& T4 = sm[6];
-      if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, M[0].base, T.base, X[1].base, st)))
+      StackMaps* M = &sm[0];  // M[0], M[1]  (paired)
+      StackMaps* X = &sm[2];  // X[0], X[1]  (split)
+      StackMaps& T = sm[4];   // paired
+      StackMaps& T2 = sm[5];  // paired
+      StackMaps& T4 = sm[6];  // split
+      if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, M[0].base, T.base, X[1].base, 2, 2, 2, st)))
         return rc;
       for (int j = 0; j < job.iters; ++j) {
         {
           Builder b;
-          Epilogue& e = b.add(cbi, n, T, 0, T, 0, f1, 1);
+          Epilogue& e = b.add(cbi, n, T, 0, T, 0, f1, NEWTON_B);  // T2 = T T
           e.D = T2.base;
-          e.d_split = 1;
-          e.skip = skip;
-          e.flags = job.flags;
+          e.d_planes = 2;
+          common(e);
           if (j >= 1) {
-            Epilogue& ex = b.add(cbi, n, X[j & 1], 0, T, 0, f1, 1);
+            Epilogue& ex = b.add(cbi, n, X[j & 1], 0, T, 0, f1, NEWTON_B);  // X <- X T
             ex.D = X[(j + 1) & 1].base;
-            ex.d_split = 1;
-            ex.skip = skip;
-            ex.flags = job.flags;
+            ex.d_planes = 2;
+            common(ex);
           }
           if ((rc = b.launch(st))) return rc;
         }
@@ -143,47 +167,44 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
         StackMaps* P = &T2;
         if (p == 4) {
           Builder b;
-          Epilogue& e = b.add(cbi, n, T2, 0, T2, 0, f1, 1);
+          Epilogue& e = b.add(cbi, n, T2, 0, T2, 0, f1, NEWTON_B);  // T4 = T2 T2
           e.D = T4.base;
-          e.d_split = 1;
-          e.skip = skip;
-          e.flags = job.flags;
+          e.d_planes = 2;
+          common(e);
           if ((rc = b.launch(st))) return rc;
           P = &T4;
         }
         {
           Builder b;
-          Epilogue& e = b.add(cbi, n, *P, 0, M[j & 1], 0, f1, 1);
+          Epilogue& e = b.add(cbi, n, *P, 0, M[j & 1], 0, f1, NEWTON_B);  // M <- T^p M
           e.D = M[(j + 1) & 1].base;
-          e.d_split = 1;
-          e.E = T.base;
+          e.d_planes = 2;
+          e.E = T.base;  // next T = ((p+1) I - M) / p
+          e.e_planes = 2;
           e.e_mul = -1.f / p;
           e.e_add = static_cast<float>(p + 1) / p;
           e.res = residual ? S.res : nullptr;
           e.valid = valid;
-          e.skip = skip;
-          e.flags = job.flags;
+          common(e);
           if ((rc = b.launch(st))) return rc;
         }
         if (residual &&
             (rc = launch_check(S.res, S.done, S.iters, valid, cb, n, job.tol, j + 1, job.flags, st)))
           return rc;
       }
-      if ((rc = launch_finalize(X[0].base, X[1].base, residual ? S.iters : nullptr, job.iters, S.sc, cb, n, out_plain,
-                                out_split, job.flags, st)))
+      if ((rc = launch_finalize(X[0].base, X[1].base, 2, residual ? S.iters : nullptr, job.iters, S.sc, cb, n,
+                                out_plain, out_split, job.flags, st)))
         return rc;
-      if (iters_out && (rc = launch_report(residual ? S.iters : nullptr, nullptr, residual ? S.done : nullptr, cb,
-                                           job.iters, iters_out, job.flags, residual, st)))
-        return rc;
-      if (!iters_out && residual &&
-          (rc = launch_report(S.iters, nullptr, S.done, cb, job.iters, nullptr, job.flags, residual, st)))
+      if ((iters_out || residual) &&
+          (rc = launch_report(residual ? S.iters : nullptr, nullptr, residual ? S.done : nullptr, cb, job.iters,
+                              iters_out, job.flags, residual, st)))
         return rc;
     } else if (job.solver == 1) {
       // ------------------------------------------------------------ Newton-DB
       StackMaps* Y = &sm[0];
       StackMaps* Z = &sm[2];
       StackMaps& T = sm[4];
-      if ((rc = launch_root_prologue(1, A, cb, n, valid, job.eps, p, S.s, Y[0].base, T.base, Z[1].base, st)))
+      if ((rc = launch_root_prologue(1, A, cb, n, valid, job.eps, p, S.s, Y[0].base, T.base, Z[1].base, 2, 2, 2, st)))
         return rc;
       const int stages = (p == 4) ? 2 : 1;
       for (int stage = 0; stage < stages; ++stage) {
@@ -207,32 +228,29 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
         for (int j = 0; j < job.iters; ++j) {
           {
             Builder b;
-            Epilogue& ey = b.add(cbi, n, Y[j & 1], 0, T, 0, f1, 1);
+            Epilogue& ey = b.add(cbi, n, Y[j & 1], 0, T, 0, f1, B_MN_MAJOR);  // Y <- Y T
             ey.D = Y[(j + 1) & 1].base;
-            ey.d_split = 1;
-            ey.skip = skip;
-            ey.flags = job.flags;
+            ey.d_planes = 2;
+            common(ey);
             if (j >= 1) {
-              Epilogue& ez = b.add(cbi, n, T, 0, Z[j & 1], 0, f1, 1);
+              Epilogue& ez = b.add(cbi, n, T, 0, Z[j & 1], 0, f1, B_MN_MAJOR);  // Z <- T Z
               ez.D = Z[(j + 1) & 1].base;
-              ez.d_split = 1;
-              ez.skip = skip;
-              ez.flags = job.flags;
+              ez.d_planes = 2;
+              common(ez);
             }
             if ((rc = b.launch(st))) return rc;
           }
           if (!residual && j == job.iters - 1) break;
           {
             Builder b;
-            Epilogue& e = b.add(cbi, n, Z[(j + 1) & 1], 0, Y[(j + 1) & 1], 0, f1, 1);
+            Epilogue& e = b.add(cbi, n, Z[(j + 1) & 1], 0, Y[(j + 1) & 1], 0, f1, B_MN_MAJOR);  // T = (3I - Z Y)/2
             e.alpha = -0.5f;
             e.gamma = 1.5f;
             e.D = T.base;
-            e.d_split = 1;
+            e.d_planes = 2;
             e.res = residual ? S.res : nullptr;
             e.valid = valid;
-            e.skip = skip;
-            e.flags = job.flags;
+            common(e);
             if ((rc = b.launch(st))) return rc;
           }
           if (residual &&
@@ -240,55 +258,49 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
             return rc;
         }
       }
-      if ((rc = launch_finalize(Z[0].base, Z[1].base, residual ? S.iters : nullptr, job.iters, S.sc, cb, n, out_plain,
-                                out_split, job.flags, st)))
+      if ((rc = launch_finalize(Z[0].base, Z[1].base, 2, residual ? S.iters : nullptr, job.iters, S.sc, cb, n,
+                                out_plain, out_split, job.flags, st)))
         return rc;
-      const int* add = (p == 4) ? S.iters1 : nullptr;
-      if (p == 4 && !residual) add = nullptr;
+      const int* add = (p == 4 && residual) ? S.iters1 : nullptr;
       const int default_total = (p == 4) ? 2 * job.iters : job.iters;
       if ((iters_out || residual) &&
-          (rc = launch_report(residual ? S.iters : nullptr, residual ? add : nullptr, residual ? S.done : nullptr, cb,
-                              default_total, iters_out, job.flags, residual, st)))
+          (rc = launch_report(residual ? S.iters : nullptr, add, residual ? S.done : nullptr, cb, default_total,
+                              iters_out, job.flags, residual, st)))
         return rc;
     } else {
       // ------------------------------------------------------------ Chebyshev
       const int d = job.cheb_degree;
       StackMaps& Xt = sm[0];
-      StackMaps* b = &sm[1];  // b[k % 3]
+      StackMaps* b = &sm[1];  // b[k % 3], paired
       if ((rc = launch_cheb_setup(A, cb, n, valid, job.eps, p, d, job.cheb_lo, S.s, S.coef, S.sc, Xt.base,
-                                  b[d % 3].base, b[(d - 1) % 3].base, st)))
+                                  b[d % 3].base, b[(d - 1) % 3].base, 2, 2, st)))
         return rc;
-      for (int k = d - 2; k >= 1; --k) {
+      for (int k = d - 2; k >= 1; --k) {  // b_k = 2 Xt b_{k+1} - b_{k+2} + c_k I
         Builder bl;
-        Epilogue& e = bl.add(cbi, n, Xt, 0, b[(k + 1) % 3], 0, f1, 1);
+        Epilogue& e = bl.add(cbi, n, Xt, 0, b[(k + 1) % 3], 0, f1, B_TRANSPOSED);
         e.alpha = 2.f;
         e.beta = -1.f;
         e.C = b[(k + 2) % 3].base;
-        e.c_split = 1;
+        e.c_planes = 2;
         e.gamma_vec = S.coef + k;
         e.gamma_stride = d + 2;
         e.D = b[k % 3].base;
-        e.d_split = 1;
+        e.d_planes = 2;
         e.flags = job.flags;
         if ((rc = bl.launch(st))) return rc;
       }
-      {
+      {  // X = s^{-1/p} (Xt b_1 - b_2 + c_0 I)
         Builder bl;
-        Epilogue& e = bl.add(cbi, n, Xt, 0, b[1], 0, f1, 1);
+        Epilogue& e = bl.add(cbi, n, Xt, 0, b[1], 0, f1, B_TRANSPOSED);
         e.alpha = 1.f;
         e.beta = -1.f;
         e.C = b[2].base;
-        e.c_split = 1;
+        e.c_planes = 2;
         e.gamma_vec = S.coef;
         e.gamma_stride = d + 2;
         e.scale_vec = S.sc;
-        if (out_split) {
-          e.D = out_split;
-          e.d_split = 1;
-        } else {
-          e.D = out_plain;
-          e.d_split = 0;
-        }
+        e.D = out_split ? out_split : out_plain;
+        e.d_planes = out_split ? 2 : 1;
         e.flags = job.flags;
         if ((rc = bl.launch(st))) return rc;
       }

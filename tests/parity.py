@@ -74,8 +74,8 @@ def conditioning_floor(A, p, eps):
     return max(perturbation_floor(A, p, eps), lapack_fp32_floor(A, p, eps))
 
 
-def root_gate(A, p, eps):
-    return max(BASE_TOL, 2.0 * conditioning_floor(A, p, eps))
+def root_gate(A, p, eps, factor=2.0):
+    return max(BASE_TOL, factor * conditioning_floor(A, p, eps))
 
 
 class Fp32ReferenceShampoo:

@@ -99,7 +99,7 @@ def test_scratch_sizes(sb):
     a = sb.inv_root_scratch_bytes(64, 1024, sb.SOLVER_NEWTON)
     b = sb.inv_root_scratch_bytes(128, 1024, sb.SOLVER_NEWTON)
     per = b - a
-    assert per == 64 * (7 * 2 * 1024 * 1024 * 4 + 4 * (6 + 64 + 2))
+    assert per == 64 * (14 * 1024 * 1024 * 4 + 4 * (6 + 64 + 2))   # Newton: 7 split stacks per matrix
     assert sb.inv_root_scratch_bytes(64, 1024, sb.SOLVER_NEWTON_DB) < a
     assert sb.gemm_scratch_bytes(3, 256) == 2 * 3 * 2 * 256 * 256 * 4
     with pytest.raises(sb.ShampooError):
