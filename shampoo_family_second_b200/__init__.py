@@ -6,7 +6,7 @@ inverse roots, preconditioned update) runs in the library's CUDA kernels.
 PyTorch supplies device memory and streams.  There is no CPU fallback: if the
 library is missing, importing this package fails.
 
-Build the library with ``python -m shampoo_family_second_b200.build``.
+Build the library with ``python shampoo_family_second_b200/build.py``.
 """
 from __future__ import annotations
 
@@ -86,7 +86,7 @@ def config_from_workload(wl) -> Config:
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m shampoo_family_second_b200.build` "
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python shampoo_family_second_b200/build.py` "
                           "(the CUDA library is required; there is no fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     P = ctypes.c_void_p

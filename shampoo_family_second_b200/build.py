@@ -1,6 +1,6 @@
 """Builds libshampoo.so (the C-ABI library) in-tree for sm_100a.
 
-    python -m shampoo_family_second_b200.build [--force] [--verbose]
+    python shampoo_family_second_b200/build.py [--force] [--verbose] [--ptxas-info]
 
 Each .cu under csrc/ is compiled with nvcc (-gencode arch=compute_100a,
 code=sm_100a -lineinfo -O3) into _build/, then linked with the CUDA runtime

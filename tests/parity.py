@@ -32,9 +32,12 @@ U32 = 2.0 ** -24
 BASE_TOL = 2e-3
 
 
-def perturbation_floor(A, p, eps, seeds=5, u=U32):
+def perturbation_floor(A, p, eps, seeds=5, u=U32, basis=None):
+    """Median relative change of the root under u ||A||_2 symmetric
+    perturbations; measured on Q^T X Q when a basis Q is given."""
     A = np.asarray(A, dtype=np.float64)
-    ex = inverse_root(A, p, eps)
+    proj = (lambda M: M) if basis is None else (lambda M: basis.T @ M @ basis)
+    ex = proj(inverse_root(A, p, eps))
     norm2 = np.linalg.norm(A, 2)
     out = []
     for sd in range(seeds):
@@ -42,7 +45,7 @@ def perturbation_floor(A, p, eps, seeds=5, u=U32):
         E = rng.standard_normal(A.shape)
         E = E + E.T
         E *= u * norm2 / np.linalg.norm(E, 2)
-        out.append(rel_fro(inverse_root(A + E, p, eps), ex))
+        out.append(rel_fro(proj(inverse_root(A + E, p, eps)), ex))
     return float(np.median(out))
 
 
@@ -110,3 +113,44 @@ class Fp32ReferenceShampoo:
 
 def update_gate(P_fp32, P_oracle):
     return max(BASE_TOL, 2.0 * rel_fro(P_fp32, P_oracle))
+
+
+def split_range_null(S, eps):
+    """Eigen-split of symmetric statistics S: the range space (eigenvalues
+    above 10 eps and above 100 u ||S||_2, i.e. determined by the gradients)
+    and the rest (determined by the damping eps and rounding)."""
+    S = 0.5 * (np.asarray(S, dtype=np.float64) + np.asarray(S, dtype=np.float64).T)
+    lam, Q = np.linalg.eigh(S)
+    thr = max(10.0 * eps, 100.0 * U32 * max(abs(lam[-1]), 1e-300))
+    keep = lam > thr
+    return Q[:, keep], Q[:, ~keep], lam
+
+
+def root_checks(X, S, p, eps):
+    """(range error, range gate, null-space eigenvalue spread or None).
+
+    For full-rank statistics the range space is everything and this is the
+    plain root gate.  Otherwise the root is compared on the range space (the
+    part the preconditioned gradient uses, since a gradient block lies in the
+    range of its own statistics) and, on the null space, its eigenvalues are
+    returned relative to (eps_eff + lam)^{-1/p} for a validity check."""
+    X = np.asarray(X, dtype=np.float64)
+    S = np.asarray(S, dtype=np.float64)
+    Qr, Qn, lam = split_range_null(S, eps)
+    ref = inverse_root(S, p, eps)
+    if Qn.shape[1] == 0:
+        return rel_fro(X, ref), root_gate(S, p, eps), None
+    pr = lambda M: Qr.T @ M @ Qr
+    err = rel_fro(pr(X), pr(ref))
+    f32 = rel_fro(pr(lapack_fp32_root(S, p, eps)), pr(ref))
+    gate = max(BASE_TOL, 2.0 * max(f32, perturbation_floor(S, p, eps, basis=Qr)))
+    Xn = Qn.T @ (0.5 * (X + X.T)) @ Qn
+    mu = np.linalg.eigvalsh(Xn)
+    lam_n = np.maximum(lam[: Qn.shape[1]], 0.0)
+    e = effective_eps(S, eps)
+    lo = (lam_n.max() + e) ** (-1.0 / p)      # the band the null-space root must lie in
+    hi = (lam_n.min() + e) ** (-1.0 / p)
+    below = np.maximum(0.0, lo - mu) / lo
+    above = np.maximum(0.0, mu - hi) / hi
+    spread = float(max(below.max(), above.max()))
+    return err, gate, spread

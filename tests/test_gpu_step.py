@@ -6,13 +6,16 @@ the GPU's own fp32 statistics: isolates the solver from fp32 statistics
 rounding), and the update P_b = -(W_t - W_{t-1}) / lr against the fully
 float64 pipeline, <= max(2e-3, 2 F_update) relative Frobenius per block.
 
-Roots in these small-block tests are gated at max(2e-3, 4 F): their
-statistics are built from a few 32-wide gradient blocks, so they are rank
-deficient or nearly singular (condition numbers 1e5-1e7), and there the
-coupled Newton iteration's error, which sits in the null-space directions,
-is up to 4x that of single-precision LAPACK.  Those directions carry no
-gradient, so the update (gated at 2 F) is unaffected; the full-size
-workloads and the solver sweep gate roots at 2 F.
+Small ragged blocks have rank-deficient statistics (a 32 x 15 gradient
+block gives a 32 x 32 L of rank 15).  On the null space the root is set by
+eps and by rounding noise alone, and an iterative fp32 solver's error there
+is larger than single-precision LAPACK's; the gradient has no component
+there, so the update does not see it.  Roots are therefore compared on the
+range space of the statistics at max(2e-3, 2 F) (F measured on the same
+projection), and on the null space the root's eigenvalues must lie within
+10% of the band [(lam_max + eps)^{-1/p}, (lam_min + eps)^{-1/p}] spanned by
+the null-space eigenvalues lam (tests/parity.py, root_checks).
+Full-rank statistics get the plain 2 F gate.
 """
 import numpy as np
 import pytest
@@ -22,11 +25,11 @@ pytestmark = pytest.mark.gpu
 
 import oracle
 import workloads
-from parity import Fp32ReferenceShampoo, root_gate, update_gate
+from parity import Fp32ReferenceShampoo, root_checks, root_gate, update_gate
 
 TOL_UPDATE = 2e-3
 TOL_ROOT = 2e-3
-ROOT_FACTOR = 4.0
+NULL_SPREAD = 0.10
 TOL_STATS = 1e-5
 
 
@@ -79,10 +82,11 @@ def run_parity(sb, wl, steps, check_roots=True, blocks=None):
             assert es < TOL_STATS, (t, b, "stats", es)
             if check_roots and t % wl.refresh_every == 0:
                 for X, S, v in ((XL, L, blk.r), (XR, R, blk.c)):
-                    xr = oracle.inverse_root(S[b, :v, :v], wl.root_p, wl.eps)
-                    er = oracle.rel_fro(X[b, :v, :v], xr)
+                    er, gate, spread = root_checks(X[b, :v, :v], S[b, :v, :v], wl.root_p, wl.eps)
                     worst["root"] = max(worst["root"], er)
-                    assert er < root_gate(S[b, :v, :v], wl.root_p, wl.eps, ROOT_FACTOR), (t, b, "root", er)
+                    assert er < gate, (t, b, "root", er, gate)
+                    if spread is not None:
+                        assert spread < NULL_SPREAD, (t, b, "null-space root", spread)
     assert opt.status() == 0
     return worst
 
@@ -95,7 +99,7 @@ def test_tiny_workload(sb):
 
 @pytest.mark.parametrize("shapes", [((33, 47),), ((64, 45), (20, 96)), ((100, 33),)])
 def test_ragged_blocks(sb, shapes):
-    wl = workloads.workload("tiny", shapes=shapes, steps=4, iters=40, tol=1e-6, beta=0.9, eps=1e-4)
+    wl = workloads.workload("tiny", shapes=shapes, steps=4, iters=40, tol=1e-5, beta=0.9, eps=1e-4)
     run_parity(sb, wl, wl.steps)
 
 
