@@ -201,6 +201,25 @@ SHAMPOO_API int inv_root_batched(const float* d_A, float* d_X, int64_t batch, in
                      int32_t iters, float tol, int32_t cheb_degree, float cheb_lo, void* d_scratch,
                      size_t scratch_bytes, int32_t* d_iters_used, int32_t* d_status, void* stream);
 
+/* inv_root_batched for callers that cannot allocate device memory (no
+ * counterpart on the pages: an addition of this library).  Some callers may
+ * not call cudaMalloc at all, e.g. code running inside a memory-pool region
+ * that forbids allocation, a real-time loop that must not block on the
+ * allocator, or an embedding without an allocator.  This entry point takes the
+ * solver's scratch from a fixed 32 MiB device array inside the library (held
+ * on every GPU that loads the library until the process exits) and allocates
+ * nothing; inputs and outputs are still the caller's, with the same meaning as
+ * in inv_root_batched.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) and should come before any stream capture.
+ * All calls share the array: calls whose work overlaps on the GPU (other
+ * streams or host threads on the same device) race on it.  The solver clears
+ * what must start at zero on every call.  Batches larger than the array are
+ * solved in chunks; sizes whose scratch for one matrix exceeds 32 MiB (e.g.
+ * n = 1024 with coupled Newton) return SHAMPOO_ERR_UNSUPPORTED. */
+SHAMPOO_API int inv_root_batched_noalloc(const float* d_A, float* d_X, int64_t batch, int32_t n, int32_t p, float eps,
+                                         int32_t solver, int32_t iters, float tol, int32_t cheb_degree,
+                                         float cheb_lo, int32_t* d_iters_used, int32_t* d_status, void* stream);
+
 /* The batched fp32-accurate product every stage uses, as a utility:
  * D_i = alpha A_i op(B_i) + beta C_i + gamma I for plain stacks (batch, n, n),
  * op(B) = B^T (op_b = 0) or B (op_b = 1);

@@ -50,7 +50,8 @@ KERNEL_NAMES = ("gemm3x_tf32", "stack_split", "frob_norm", "prologue", "check", 
 EXPORTS = (
     "shampoo_status_string", "shampoo_last_error", "shampoo_query_sizes", "shampoo_init", "shampoo_step",
     "shampoo_get_status", "shampoo_block_table", "shampoo_state_views", "shampoo_set_step", "shampoo_destroy",
-    "inv_root_scratch_bytes", "inv_root_batched", "shampoo_gemm_scratch_bytes", "shampoo_gemm_batched",
+    "inv_root_scratch_bytes", "inv_root_batched", "inv_root_batched_noalloc", "shampoo_gemm_scratch_bytes",
+    "shampoo_gemm_batched",
     "shampoo_profile_enable", "shampoo_profile_reset", "shampoo_profile_read", "shampoo_launch_count",
 )
 
@@ -108,6 +109,7 @@ def _load():
         "shampoo_destroy": (None, [P]),
         "inv_root_scratch_bytes": (ctypes.c_int, [I64, I32, I32, sz]),
         "inv_root_batched": (ctypes.c_int, [P, P, I64, I32, I32, F, I32, I32, F, I32, F, P, ctypes.c_size_t, P, P, P]),
+        "inv_root_batched_noalloc": (ctypes.c_int, [P, P, I64, I32, I32, F, I32, I32, F, I32, F, P, P, P]),
         "shampoo_gemm_scratch_bytes": (ctypes.c_int, [I64, I32, sz]),
         "shampoo_gemm_batched": (ctypes.c_int, [P, P, P, P, I64, I32, I32, F, F, F, P, ctypes.c_size_t, P, P]),
         "shampoo_profile_enable": (None, [I32]),
