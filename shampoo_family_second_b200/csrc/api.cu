@@ -227,7 +227,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
     wc[b] = sh.table[5 * b + 4];
     fl += 2 * r * r * c;
     fr += 2 * r * c * c;
-    sb += r * c * (cfg->grad_dtype == SHAMPOO_BF16 ? 2 : 4) + 4.0 * 8.0 * B * B;
+    sb += r * c * (cfg->grad_dtype == SHAMPOO_BF16 ? 2 : 4) + 16.0 * B * B;  // G read; Gs, Gt split written
   }
   h->stats_flops_L = fl / nb;
   h->stats_flops_R = fr / nb;

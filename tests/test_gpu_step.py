@@ -88,6 +88,8 @@ def run_parity(sb, wl, steps, check_roots=True, blocks=None):
                     if spread is not None:
                         assert spread < NULL_SPREAD, (t, b, "null-space root", spread)
     assert opt.status() == 0
+    print(f"\n{wl.name} {wl.shapes}: worst update {worst['update']:.2e}, root {worst['root']:.2e}, "
+          f"statistics {worst['stats']:.2e}")
     return worst
 
 
