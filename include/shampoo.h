@@ -30,8 +30,7 @@
  *    SHAMPOO_DEVFLAG_* bits into a device status word (see shampoo_get_status
  *    and the d_status argument of inv_root_batched).
  *  - Layout: matrices are row-major fp32 unless stated.  Stacks are
- *    (batch, n, n).  A "split" stack is (batch, 2, n, n): per matrix a
- *    tf32-exact high plane then a low plane; the value is high + low.
+ *    (batch, n, n), matrices back to back.
  *  - Thread safety: a handle is not thread-safe; separate handles are
  *    independent.  The profiling counters are process-wide.
  */
@@ -168,7 +167,7 @@ SHAMPOO_API int shampoo_block_table(shampoo_handle h, int32_t* nb, int64_t* tabl
 
 /* Device pointers into the state (owned by the caller's state buffer):
  * L: plain stack (nb, B, B) of left statistics; R: (nb, B, B) right statistics;
- * rootL / rootR: split stacks (nb, 2, B, B) of XL and XR; *step: steps taken.
+ * rootL / rootR: (nb, B, B) stacks of XL and XR; *step: steps taken.
  * Ragged blocks hold zeros outside their r x r / c x c valid region. */
 SHAMPOO_API int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, float** rootR, int64_t* step);
 
@@ -214,8 +213,9 @@ SHAMPOO_API int inv_root_batched(const float* d_A, float* d_X, int64_t batch, in
  * All calls share the array: calls whose work overlaps on the GPU (other
  * streams or host threads on the same device) race on it.  The solver clears
  * what must start at zero on every call.  Batches larger than the array are
- * solved in chunks; sizes whose scratch for one matrix exceeds 32 MiB (e.g.
- * n = 1024 with coupled Newton) return SHAMPOO_ERR_UNSUPPORTED. */
+ * solved in chunks (the largest need, coupled Newton at n = 1024, is 28 MiB
+ * per matrix); a size whose scratch for one matrix exceeded the array would
+ * return SHAMPOO_ERR_UNSUPPORTED. */
 SHAMPOO_API int inv_root_batched_noalloc(const float* d_A, float* d_X, int64_t batch, int32_t n, int32_t p, float eps,
                                          int32_t solver, int32_t iters, float tol, int32_t cheb_degree,
                                          float cheb_lo, int32_t* d_iters_used, int32_t* d_status, void* stream);
@@ -223,10 +223,12 @@ SHAMPOO_API int inv_root_batched_noalloc(const float* d_A, float* d_X, int64_t b
 /* The batched fp32-accurate product every stage uses, as a utility:
  * D_i = alpha A_i op(B_i) + beta C_i + gamma I for plain stacks (batch, n, n),
  * op(B) = B^T (op_b = 0) or B (op_b = 1);
- * d_C may be NULL (then beta is ignored) and may equal d_D.  n a multiple of
- * 32 in [32, 4096].  Operands are split into tf32 hi/lo planes in d_scratch
- * (see shampoo_gemm_scratch_bytes), then multiplied as 3xTF32 on the tensor
- * cores.  Enqueued on `stream`; no host sync. */
+ * d_C may be NULL (then beta is ignored) and may equal d_D; d_D must not
+ * overlap d_A or d_B.  n a multiple of 32 in [32, 4096]; all four 16-byte
+ * aligned.  The kernel splits operand tiles into tf32 hi/lo parts on chip and
+ * multiplies them as 3xTF32 on the tensor cores.  No scratch is needed
+ * (shampoo_gemm_scratch_bytes returns 0; d_scratch may be NULL).  Enqueued on
+ * `stream`; no host sync. */
 SHAMPOO_API int shampoo_gemm_scratch_bytes(int64_t batch, int32_t n, size_t* bytes);
 SHAMPOO_API int shampoo_gemm_batched(const float* d_A, const float* d_B, const float* d_C, float* d_D, int64_t batch, int32_t n,
                          int32_t op_b, float alpha, float beta, float gamma, void* d_scratch, size_t scratch_bytes,

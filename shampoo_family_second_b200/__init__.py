@@ -44,7 +44,7 @@ KERNEL_CHECK = 4
 KERNEL_FINALIZE = 5
 KERNEL_CHEB_COEF = 6
 KERNEL_KINDS = 7
-KERNEL_NAMES = ("gemm3x_tf32", "stack_split", "frob_norm", "prologue", "check", "finalize", "cheb_coef")
+KERNEL_NAMES = ("gemm3x_tf32", "stack_blocks", "frob_norm", "prologue", "check", "finalize", "cheb_coef")
 
 # Exported symbols, in header order (tests compare this with include/shampoo.h).
 EXPORTS = (
@@ -269,15 +269,15 @@ class Shampoo:
         return L, R
 
     def roots(self):
-        """(XL, XR) as float32 values (nb, B, B): high + low planes of the split roots."""
+        """(XL, XR) as float32 views (nb, B, B) into the state buffer."""
         import torch
         (_, _, pxl, pxr), _ = self._views()
         B, nb = self.cfg.block, self.nb
         base = self.state.data_ptr()
         fl = self.state.view(torch.float32)
-        XL = fl[(pxl - base) // 4:(pxl - base) // 4 + 2 * nb * B * B].view(nb, 2, B, B)
-        XR = fl[(pxr - base) // 4:(pxr - base) // 4 + 2 * nb * B * B].view(nb, 2, B, B)
-        return XL[:, 0] + XL[:, 1], XR[:, 0] + XR[:, 1]
+        XL = fl[(pxl - base) // 4:(pxl - base) // 4 + nb * B * B].view(nb, B, B)
+        XR = fl[(pxr - base) // 4:(pxr - base) // 4 + nb * B * B].view(nb, B, B)
+        return XL, XR
 
     def set_step_count(self, step: int):
         """Sets the step counter (the refresh schedule counts from it)."""

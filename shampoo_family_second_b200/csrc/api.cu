@@ -4,7 +4,7 @@
 // Step order ("Shampoo optimizer" notes, matrix-case listing: preconditioners
 // first, then the parameters; podcast "Preconditioned optimization without the
 // full matrix cost", cue 28: roots recomputed only every so many steps):
-//   1. stack     gradient blocks -> Gs (B x B, split) and Gt (transposed)
+//   1. stack     gradient blocks -> Gs (B x B) and Gt (transposed), zero-padded
 //   2. stats     L <- beta L + Gs Gs^T, R <- beta R + Gt Gt^T     (one GEMM launch)
 //   3. roots     if step % refresh_every == 0: XL, XR of the damped, scaled stats
 //   4. apply     T = XL G (GEMM), then W -= lr T XR fused into the second
@@ -80,7 +80,7 @@ int build_table(int B, int32_t nparams, const int64_t* rows, const int64_t* cols
 
 // State layout (bytes, each part 256-aligned):
 //   status word | block table (nb x 5 int32) | valid extents (2nb int32: r of L_b, c of R_b)
-//   | wrows (nb) | wcols (nb) | stats plain (2nb, B, B) | roots split (2nb, 2, B, B)
+//   | wrows (nb) | wcols (nb) | statistics (2nb, B, B) | roots (2nb, B, B)
 struct StateLayout {
   size_t status, table, valid, wrows, wcols, stats, roots, total;
 };
@@ -93,20 +93,20 @@ StateLayout state_layout(int nb, int B) {
   s.wrows = o, o += al(size_t(nb) * 4);
   s.wcols = o, o += al(size_t(nb) * 4);
   s.stats = o, o += al(plain_floats(2 * nb, B) * 4);
-  s.roots = o, o += al(split_floats(2 * nb, B) * 4);
+  s.roots = o, o += al(plain_floats(2 * nb, B) * 4);
   s.total = o;
   return s;
 }
-// Scratch layout: Gs | Gt | Tapply (split, nb each) | blk_wptr (nb ptrs) | blk_ld (nb) | solver scratch
+// Scratch layout: Gs | Gt | Tapply (nb matrices each) | blk_wptr (nb ptrs) | blk_ld (nb) | solver scratch
 struct ScratchLayout {
   size_t gs, gt, tap, wptr, ld, root, root_bytes, total;
 };
 ScratchLayout scratch_layout(int nb, int B, int solver) {
   ScratchLayout s;
   size_t o = 0;
-  s.gs = o, o += al(split_floats(nb, B) * 4);
-  s.gt = o, o += al(split_floats(nb, B) * 4);
-  s.tap = o, o += al(split_floats(nb, B) * 4);
+  s.gs = o, o += al(plain_floats(nb, B) * 4);
+  s.gt = o, o += al(plain_floats(nb, B) * 4);
+  s.tap = o, o += al(plain_floats(nb, B) * 4);
   s.wptr = o, o += al(size_t(nb) * 8);
   s.ld = o, o += al(size_t(nb) * 4);
   s.root = o;
@@ -227,7 +227,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
     wc[b] = sh.table[5 * b + 4];
     fl += 2 * r * r * c;
     fr += 2 * r * c * c;
-    sb += r * c * (cfg->grad_dtype == SHAMPOO_BF16 ? 2 : 4) + 16.0 * B * B;  // G read; Gs, Gt split written
+    sb += r * c * (cfg->grad_dtype == SHAMPOO_BF16 ? 2 : 4) + 8.0 * B * B;  // G read; Gs, Gt written
   }
   h->stats_flops_L = fl / nb;
   h->stats_flops_R = fr / nb;
@@ -242,7 +242,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
       (rc = up(h->d_wrows, wr.data(), wr.size() * 4)) || (rc = up(h->d_wcols, wc.data(), wc.size() * 4)) ||
       (rc = check_cuda(cudaMemsetAsync(h->d_status, 0, 4, st), "zero status")) ||
       (rc = check_cuda(cudaMemsetAsync(h->stats, 0, plain_floats(2 * nb, B) * 4, st), "zero statistics")) ||
-      (rc = check_cuda(cudaMemsetAsync(h->roots, 0, split_floats(2 * nb, B) * 4, st), "zero roots")) ||
+      (rc = check_cuda(cudaMemsetAsync(h->roots, 0, plain_floats(2 * nb, B) * 4, st), "zero roots")) ||
       (rc = check_cuda(cudaStreamSynchronize(st), "init sync"))) {
     delete h;
     return rc;
@@ -304,8 +304,7 @@ int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d
     job.cheb_lo = c.cheb_lo;
     job.A = h->stats;
     job.valid = h->d_valid;
-    job.X_plain = nullptr;
-    job.X_split = h->roots;
+    job.X = h->roots;
     job.iters_used = nullptr;
     job.flags = h->d_status;
     if ((rc = run_inverse_roots(job, h->scratch + h->xl.root, h->xl.root_bytes, st))) return rc;
@@ -315,7 +314,6 @@ int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d
     Builder b;
     Epilogue& e = b.add(nb, B, h->mRoots, 0, h->mGt, 0, h->stats_flops_L);
     e.D = h->Tap;
-    e.d_planes = 2;
     e.flags = h->d_status;
     if ((rc = b.launch(st))) return rc;
   }
@@ -359,7 +357,7 @@ int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, f
   if (L) *L = h->stats;
   if (R) *R = h->stats + plain_floats(nb, B);
   if (rootL) *rootL = h->roots;
-  if (rootR) *rootR = h->roots + split_floats(nb, B);
+  if (rootR) *rootR = h->roots + plain_floats(nb, B);
   if (step) *step = h->step;
   return SHAMPOO_OK;
 }
@@ -413,8 +411,7 @@ int inv_root_batched(const float* d_A, float* d_X, int64_t batch, int32_t n, int
   job.cheb_lo = cheb_lo;
   job.A = d_A;
   job.valid = nullptr;
-  job.X_plain = d_X;
-  job.X_split = nullptr;
+  job.X = d_X;
   job.iters_used = d_iters_used;
   job.flags = d_status;
   return run_inverse_roots(job, d_scratch, scratch_bytes, static_cast<cudaStream_t>(stream));
@@ -423,31 +420,27 @@ int inv_root_batched(const float* d_A, float* d_X, int64_t batch, int32_t n, int
 int shampoo_gemm_scratch_bytes(int64_t batch, int32_t n, size_t* bytes) {
   if (!bytes || batch < 0 || n < 32 || n > 4096 || n % 32)
     return set_error(SHAMPOO_ERR_INVALID_ARG, "bad arguments");
-  *bytes = 2 * al(split_floats(batch, n) * 4);
+  *bytes = 0;  // the operands are read in place
   return SHAMPOO_OK;
 }
 
 int shampoo_gemm_batched(const float* d_A, const float* d_B, const float* d_C, float* d_D, int64_t batch, int32_t n,
                          int32_t op_b, float alpha, float beta, float gamma, void* d_scratch, size_t scratch_bytes,
                          int32_t* d_status, void* stream) {
+  (void)d_scratch;
+  (void)scratch_bytes;
   if (batch < 0 || n < 32 || n > 4096 || n % 32) return set_error(SHAMPOO_ERR_INVALID_ARG, "bad batch / n");
   if (op_b != 0 && op_b != 1) return set_error(SHAMPOO_ERR_INVALID_ARG, "op_b must be 0 (B^T) or 1 (B)");
   if (batch == 0) return SHAMPOO_OK;
   if (batch > 0x7fffffff / 32) return set_error(SHAMPOO_ERR_UNSUPPORTED, "batch too large");
-  if (!d_A || !d_B || !d_D || !d_scratch) return set_error(SHAMPOO_ERR_INVALID_ARG, "NULL device pointer");
-  size_t need = 0;
-  shampoo_gemm_scratch_bytes(batch, n, &need);
-  if (scratch_bytes < need) return set_error(SHAMPOO_ERR_WORKSPACE, "scratch %zu < %zu bytes", scratch_bytes, need);
-  if (!aligned256(d_scratch) || (reinterpret_cast<uintptr_t>(d_A) & 15) || (reinterpret_cast<uintptr_t>(d_B) & 15) ||
+  if (!d_A || !d_B || !d_D) return set_error(SHAMPOO_ERR_INVALID_ARG, "NULL device pointer");
+  if ((reinterpret_cast<uintptr_t>(d_A) & 15) || (reinterpret_cast<uintptr_t>(d_B) & 15) ||
       (reinterpret_cast<uintptr_t>(d_D) & 15) || (reinterpret_cast<uintptr_t>(d_C) & 15))
-    return set_error(SHAMPOO_ERR_UNSUPPORTED, "scratch must be 256-byte and A, B, C, D 16-byte aligned");
+    return set_error(SHAMPOO_ERR_UNSUPPORTED, "A, B, C, D must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* As = static_cast<float*>(d_scratch);
-  float* Bs = reinterpret_cast<float*>(static_cast<char*>(d_scratch) + al(split_floats(batch, n) * 4));
   int rc;
-  if ((rc = launch_split_plain(d_A, As, batch, n, st)) || (rc = launch_split_plain(d_B, Bs, batch, n, st))) return rc;
   StackMaps ma, mb;
-  if ((rc = make_stack_maps(ma, As, batch, n)) || (rc = make_stack_maps(mb, Bs, batch, n))) return rc;
+  if ((rc = make_stack_maps(ma, d_A, batch, n)) || (rc = make_stack_maps(mb, d_B, batch, n))) return rc;
   Builder b;
   Epilogue& e = b.add(static_cast<int>(batch), n, ma, 0, mb, 0, 2.0 * n * double(n) * n,
                       op_b ? B_MN_MAJOR : B_TRANSPOSED);

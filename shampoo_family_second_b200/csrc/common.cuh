@@ -16,7 +16,9 @@ namespace shampoo {
 // hi keeps the 10 explicit mantissa bits of a tf32 number (rounded to nearest,
 // ties away from zero, by integer arithmetic on the bit pattern); lo = v - hi is
 // exact in fp32.  A product a*b is then a_hi*b_hi + a_hi*b_lo + a_lo*b_hi, with
-// a relative error of about 2^-21 instead of tf32's 2^-11.
+// a relative error of about 2^-21 instead of tf32's 2^-11.  The GEMM kernel
+// applies it to each operand tile in shared memory, so every stack in global
+// memory is plain fp32.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void split_tf32(float v, float& hi, float& lo) {
   uint32_t u = __float_as_uint(v);
@@ -103,16 +105,36 @@ __device__ __forceinline__ void fence_barrier_init() {
 }
 
 // ---------------------------------------------------------------------------
-// TMA: 4-D tiled tensor load into shared memory, completing on an mbarrier.
+// TMA: tiled tensor loads into shared memory, completing on an mbarrier.
 // No multicast: each CTA fetches its own tiles.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, uint64_t* bar, int c0, int c1,
-                                            int c2, int c3) {
+// A plain stack (batch, rows, columns) is mapped as {columns, rows, matrix}.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, uint64_t* bar, int c0, int c1,
+                                            int c2) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+// Orders this thread's ordinary shared-memory stores before later accesses
+// by the async proxy (the tensor core's operand reads, TMA writes).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Per-thread register budget of the executing warpgroup (all four warps must
+// execute the same instruction).  dec returns registers to the CTA's pool,
+// inc blocks until the pool can supply them; the pool is what the CTA was
+// launched with (threads x registers per thread).
+template <int N>
+__device__ __forceinline__ void warpgroup_regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void warpgroup_regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {

@@ -12,23 +12,28 @@
 //   apply + update  T = L^{-1/4} G, then W <- W - lr T R^{-1/4} scattered into
 //                   the weight (notes' listing, last line).
 //
-// A persistent kernel (one CTA per SM) walks 128 x 256 tiles of the matrices
-// D_i = epi(A_i B_i^T), or epi(A_i B_i) when B is read MN-major (B stored
-// K x N row-major):
-//   warp 0      one thread issues TMA loads of the A and B tiles (hi and lo
-//               planes, 16 deep in K) into a 4-stage shared-memory ring;
+// A persistent kernel (one CTA per SM, 16 warps) walks 128 x 256 tiles of the
+// matrices D_i = epi(A_i B_i^T), or epi(A_i B_i) when B is read MN-major (B
+// stored K x N row-major).  All operands and results are plain fp32 stacks.
+//   warp 0      one thread issues TMA loads of the fp32 A and B tiles (16 deep
+//               in K) into a 4-stage shared-memory ring;
 //   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 buffers); one
 //               thread issues the tcgen05 MMAs (3 per K-step of 8), each K
 //               segment of 64 into the next buffer, and commits them to the
 //               ring's "empty" barriers and the buffer's "full" barrier;
-//   warps 2-9   add each finished segment into fp32 registers (round to
+//   warps 2-7   split each landed tile in place into its tf32 hi part and a
+//               separate lo part (split_tf32), then release it to the MMAs;
+//   warps 8-15  add each finished segment into fp32 registers (round to
 //               nearest; one row x 128 columns per thread), then apply the
-//               epilogue and store.  The tensor core's own fp32 additions
-//               truncate; summing short segments outside it keeps the product
-//               as accurate as a plain fp32 GEMM.
-// Every wait is bounded (2 s); a time-out raises DEV_FLAG_TIMEOUT, tells the
-// other roles of the CTA to stop waiting, and the CTA unwinds, releasing its
-// TMEM.
+//               epilogue through a per-warp 32 x 32 shared-memory tile, so
+//               that global loads and stores are whole 128-byte row pieces.
+//               The tensor core's own fp32 additions truncate; summing short
+//               segments outside it keeps the product as accurate as a plain
+//               fp32 GEMM.
+// Warps 0-7 hand registers to warps 8-15 (setmaxnreg), whose running sums
+// need them.  Every wait is bounded (2 s); a time-out raises
+// DEV_FLAG_TIMEOUT, tells the other roles of the CTA to stop waiting, and the
+// CTA unwinds, releasing its TMEM.
 #include <cstdio>
 #include <cstring>
 
@@ -44,113 +49,26 @@ constexpr int BM = kTileM;
 constexpr int BN = kTileN;
 constexpr int BK = kTileK;
 constexpr int STAGES = 4;
-constexpr int A_PLANE = BM * BK * 4;                        // 8 KB
-constexpr int B_PLANE = BN * BK * 4;                        // 16 KB
-constexpr int STAGE_BYTES = 2 * A_PLANE + 2 * B_PLANE;      // 48 KB
-constexpr int MN_BLOCK = BK * 32 * 4;                      // 2 KB: 16 K-rows x 32 columns
+constexpr int A_BYTES = BM * BK * 4;                  // 8 KB
+constexpr int B_BYTES = BN * BK * 4;                  // 16 KB
+constexpr int RAW_BYTES = A_BYTES + B_BYTES;          // TMA destination; becomes the hi parts
+constexpr int STAGE_BYTES = 2 * RAW_BYTES;            // [A hi | B hi | A lo | B lo]
+constexpr int MN_BLOCK = BK * 32 * 4;                 // 2 KB: 16 K-rows x 32 columns
 constexpr int TMEM_COLS = 512;  // two 128 x 256 fp32 accumulators (K-segment double buffer)
 constexpr int SEG = 4;           // K chunks (of 16) per accumulation segment: 64 deep
-constexpr int EPI_WARPS = 8;
-constexpr int THREADS = 64 + 32 * EPI_WARPS;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-
-// Epilogue for 32 consecutive columns [c0, c0+32) of row r of matrix `mat`;
-// acc holds the fp32 products (A B^T or A B) of those columns.  Works through
-// them 8 at a time to keep few registers live next to the running sums.
-// Returns this thread's residual contribution.
-__device__ __forceinline__ float epilogue_chunk(const GemmGroup& G, int mat, int r, int c0, const float* acc,
-                                                bool& nonfinite) {
-  const Epilogue& E = G.ep;
-  const int n = G.n;
-  const size_t nn = static_cast<size_t>(n) * n;
-  const size_t row_off = static_cast<size_t>(r) * n + c0;
-  const int vsz = E.valid ? E.valid[mat] : n;
-  const float gam = E.gamma_vec ? E.gamma_vec[static_cast<size_t>(mat) * E.gamma_stride] : E.gamma;
-  const float sc = E.scale_vec ? E.scale_vec[mat] : 1.f;
-  const int dj = r - c0;
-  float resid = 0.f;
-  bool bad = false;
-  const size_t dstride = static_cast<size_t>(E.d_planes) * nn;
-  float* wrow = nullptr;
-  int wc = 0;
-  if (E.wptr) {
-    const int wr = E.wrows[mat];
-    wc = E.wcols[mat];
-    if (r < wr) wrow = E.wptr[mat] + static_cast<size_t>(r) * E.wld[mat];
-  }
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int jj = 8 * g + j;
-      const float a = acc[jj];
-      if (E.res) {
-        const int c = c0 + jj;
-        resid += (r == c && r < vsz) ? 1.f - a : 0.f;
-      }
-      v[j] = E.alpha * a;
-    }
-    if (E.C) {
-      if (E.c_planes >= 2) {
-        const float* cb = E.C + mat * static_cast<size_t>(E.c_planes) * nn + row_off + 8 * g;
-        const float4* h4 = reinterpret_cast<const float4*>(cb);
-        const float4* l4 = reinterpret_cast<const float4*>(cb + nn);
-        const float4 h0 = h4[0], h1 = h4[1], l0 = l4[0], l1 = l4[1];
-        v[0] += E.beta * (h0.x + l0.x); v[1] += E.beta * (h0.y + l0.y);
-        v[2] += E.beta * (h0.z + l0.z); v[3] += E.beta * (h0.w + l0.w);
-        v[4] += E.beta * (h1.x + l1.x); v[5] += E.beta * (h1.y + l1.y);
-        v[6] += E.beta * (h1.z + l1.z); v[7] += E.beta * (h1.w + l1.w);
-      } else {
-        const float4* c4 = reinterpret_cast<const float4*>(E.C + mat * nn + row_off + 8 * g);
-        const float4 x0 = c4[0], x1 = c4[1];
-        v[0] += E.beta * x0.x; v[1] += E.beta * x0.y; v[2] += E.beta * x0.z; v[3] += E.beta * x0.w;
-        v[4] += E.beta * x1.x; v[5] += E.beta * x1.y; v[6] += E.beta * x1.z; v[7] += E.beta * x1.w;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (8 * g + j == dj) v[j] += gam;
-      v[j] *= sc;
-      bad |= !isfinite(v[j]);
-    }
-    if (E.D) {
-      float* dm = E.D + mat * dstride;
-      float* d = dm + row_off + 8 * g;
-      if (E.d_planes >= 2) {
-        float hh[8], ll[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) split_tf32(v[j], hh[j], ll[j]);
-        reinterpret_cast<float4*>(d)[0] = make_float4(hh[0], hh[1], hh[2], hh[3]);
-        reinterpret_cast<float4*>(d)[1] = make_float4(hh[4], hh[5], hh[6], hh[7]);
-        reinterpret_cast<float4*>(d + nn)[0] = make_float4(ll[0], ll[1], ll[2], ll[3]);
-        reinterpret_cast<float4*>(d + nn)[1] = make_float4(ll[4], ll[5], ll[6], ll[7]);
-      } else {
-        reinterpret_cast<float4*>(d)[0] = make_float4(v[0], v[1], v[2], v[3]);
-        reinterpret_cast<float4*>(d)[1] = make_float4(v[4], v[5], v[6], v[7]);
-      }
-    }
-    if (E.E) {
-      float hh[8], ll[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) split_tf32(E.e_mul * v[j] + ((8 * g + j == dj) ? E.e_add : 0.f), hh[j], ll[j]);
-      float* e = E.E + mat * 2 * nn + row_off + 8 * g;
-      reinterpret_cast<float4*>(e)[0] = make_float4(hh[0], hh[1], hh[2], hh[3]);
-      reinterpret_cast<float4*>(e)[1] = make_float4(hh[4], hh[5], hh[6], hh[7]);
-      reinterpret_cast<float4*>(e + nn)[0] = make_float4(ll[0], ll[1], ll[2], ll[3]);
-      reinterpret_cast<float4*>(e + nn)[1] = make_float4(ll[4], ll[5], ll[6], ll[7]);
-    }
-    if (wrow) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = c0 + 8 * g + j;
-        if (c < wc) wrow[c] -= E.lr * v[j];
-      }
-    }
-  }
-  nonfinite |= bad;
-  return resid;
-}
+constexpr int CONV_WARP0 = 2, CONV_WARPS = 6, CONV_THREADS = 32 * CONV_WARPS;
+constexpr int EPI_WARP0 = 8, EPI_WARPS = 8;
+constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);  // 512
+constexpr int EPI_TILE_FLOATS = 32 * 32;                // per epilogue warp
+constexpr int RING_BYTES = STAGES * STAGE_BYTES;        // 192 KB
+constexpr int EPI_BYTES = EPI_WARPS * EPI_TILE_FLOATS * 4;  // 32 KB
+constexpr int SMEM_BYTES = RING_BYTES + EPI_BYTES + 1024 + 256;
+// Register split: the CTA is launched with 512 x LAUNCH_REGS registers;
+// warps 0-7 keep LIGHT_REGS each, warps 8-15 take the rest.
+constexpr int LAUNCH_REGS = 128, LIGHT_REGS = 64, HEAVY_REGS = 192;
+static_assert(256 * LIGHT_REGS + 256 * HEAVY_REGS == THREADS * LAUNCH_REGS, "register split must match the pool");
+static_assert((RAW_BYTES / 16) % CONV_THREADS == 0, "converter work divides evenly");
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 struct TileCoord {
   int gi, mat, tm, tn;
@@ -177,6 +95,90 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmLaunch& L, int tile) {
   return c;
 }
 
+// Epilogue of one 32 x 32 chunk: rows row0 .. row0+31 (row row0 + lane in this
+// thread's registers, acc = its 32 sums for columns c0 .. c0+31).
+//   phase 1  each thread writes alpha * acc + gamma [r == c] for its row into
+//            the warp's shared tile (16-byte pieces XOR-swizzled by the row, so
+//            neither phase has bank conflicts) and adds its diagonal term to
+//            the residual;
+//   phase 2  each quarter-warp takes one row: 8 lanes x 16 bytes = one
+//            128-byte piece; beta C, the scale, the outputs D, E and the
+//            weight update are applied there.
+__device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int row0, int c0, const float* acc,
+                                               float* tilebuf, int lane, float& resid, bool& bad) {
+  const Epilogue& E = G.ep;
+  const int n = G.n;
+  const int r = row0 + lane;
+  const int dj = r - c0;  // column of this row's diagonal element within the chunk
+  const float gam = E.gamma_vec ? E.gamma_vec[static_cast<size_t>(mat) * E.gamma_stride] : E.gamma;
+  if (E.res) {
+    const int vsz = E.valid ? E.valid[mat] : n;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j == dj && r < vsz) resid += 1.f - acc[j];
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float4 w;
+    w.x = E.alpha * acc[4 * k + 0] + ((4 * k + 0 == dj) ? gam : 0.f);
+    w.y = E.alpha * acc[4 * k + 1] + ((4 * k + 1 == dj) ? gam : 0.f);
+    w.z = E.alpha * acc[4 * k + 2] + ((4 * k + 2 == dj) ? gam : 0.f);
+    w.w = E.alpha * acc[4 * k + 3] + ((4 * k + 3 == dj) ? gam : 0.f);
+    *reinterpret_cast<float4*>(tilebuf + lane * 32 + ((k ^ (lane & 7)) << 2)) = w;
+  }
+  __syncwarp();
+  const size_t nn = static_cast<size_t>(n) * n;
+  const float sc = E.scale_vec ? E.scale_vec[mat] : 1.f;
+  float* wbase = nullptr;
+  int wld = 0, wr = 0, wc = 0;
+  if (E.wptr) {
+    wbase = E.wptr[mat];
+    wld = E.wld[mat];
+    wr = E.wrows[mat];
+    wc = E.wcols[mat];
+  }
+  const int kq = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int R = 4 * i + (lane >> 3);
+    const int gr = row0 + R;
+    const int gc = c0 + 4 * kq;
+    float4 v = *reinterpret_cast<const float4*>(tilebuf + R * 32 + ((kq ^ (R & 7)) << 2));
+    if (gr < n) {
+      const size_t off = static_cast<size_t>(mat) * nn + static_cast<size_t>(gr) * n + gc;
+      if (E.C) {
+        const float4 c = *reinterpret_cast<const float4*>(E.C + off);
+        v.x += E.beta * c.x;
+        v.y += E.beta * c.y;
+        v.z += E.beta * c.z;
+        v.w += E.beta * c.w;
+      }
+      v.x *= sc;
+      v.y *= sc;
+      v.z *= sc;
+      v.w *= sc;
+      bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
+      if (E.D) *reinterpret_cast<float4*>(E.D + off) = v;
+      if (E.E) {
+        float4 e;
+        e.x = E.e_mul * v.x + ((gr == gc + 0) ? E.e_add : 0.f);
+        e.y = E.e_mul * v.y + ((gr == gc + 1) ? E.e_add : 0.f);
+        e.z = E.e_mul * v.z + ((gr == gc + 2) ? E.e_add : 0.f);
+        e.w = E.e_mul * v.w + ((gr == gc + 3) ? E.e_add : 0.f);
+        *reinterpret_cast<float4*>(E.E + off) = e;
+      }
+      if (wbase && gr < wr) {
+        float* wrow = wbase + static_cast<size_t>(gr) * wld + gc;
+        if (gc + 0 < wc) wrow[0] -= E.lr * v.x;
+        if (gc + 1 < wc) wrow[1] -= E.lr * v.y;
+        if (gc + 2 < wc) wrow[2] -= E.lr * v.z;
+        if (gc + 3 < wc) wrow[3] -= E.lr * v.w;
+      }
+    }
+  }
+  __syncwarp();
+}
+
 // Persistent: one CTA per SM walks the tiles blockIdx.x, blockIdx.x +
 // gridDim.x, ...  The shared-memory ring and the two TMEM buffers carry over
 // from one tile to the next, so the epilogue of a tile (register sums ->
@@ -186,8 +188,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                        double* prof_flops) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* empty = full + STAGES;
+  float* epi_tiles = reinterpret_cast<float*>(smem + RING_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + RING_BYTES + EPI_BYTES);  // [STAGES]: TMA landed
+  uint64_t* conv = full + STAGES;        // [STAGES]: operands split, ready for the MMAs
+  uint64_t* empty = conv + STAGES;       // [STAGES]: the MMAs have read the stage
   uint64_t* acc_full = empty + STAGES;   // [2]: a K-segment's partial sums are ready in TMEM buffer b
   uint64_t* acc_empty = acc_full + 2;    // [2]: the epilogue has drained TMEM buffer b
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
@@ -202,6 +206,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
+      mbar_init(&conv[s], CONV_THREADS);
       mbar_init(&empty[s], 1);
     }
 #pragma unroll
@@ -222,126 +227,164 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t taddr = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ producer
-      uint32_t it = 0;  // chunks issued by this CTA (ring position)
-      bool ok = true;
+  if (warp < EPI_WARP0) {
+    // Warps 0-7 (two whole warpgroups) run the light roles; each warpgroup
+    // executes this one setmaxnreg.
+    warpgroup_regs_dec<LIGHT_REGS>();
+    if (warp == 0) {
+      if (lane == 0) {
+        // ------------------------------------------------------------ producer
+        uint32_t it = 0;  // chunks issued by this CTA (ring position)
+        bool ok = true;
 #pragma unroll 1
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const TileCoord tc = tile_coord(L, tile);
-        if (tc.skip) continue;
-        const GemmGroup& G = L.g[tc.gi];
-        const int nk = G.n / BK;
-        const uint32_t tx_bytes = 2u * G.a_rows * BK * 4u + 2u * G.b_rows * BK * 4u;
-        const void* amap = &maps.m[G.a_map];
-        const void* bmap = &maps.m[G.b_map];
-        const int am = G.a_off + tc.mat;
-        const int bm = G.b_off + tc.mat;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+          const TileCoord tc = tile_coord(L, tile);
+          if (tc.skip) continue;
+          const GemmGroup& G = L.g[tc.gi];
+          const int nk = G.n / BK;
+          const uint32_t tx_bytes = static_cast<uint32_t>(G.a_rows + G.b_rows) * BK * 4u;
+          const void* amap = &maps.m[G.a_map];
+          const void* bmap = &maps.m[G.b_map];
+          const int am = G.a_off + tc.mat;
+          const int bm = G.b_off + tc.mat;
 #pragma unroll 1
-        for (int kc = 0; kc < nk; ++kc, ++it) {
-          const int s = it % STAGES;
-          if (it >= STAGES && !mbar_wait_bounded(&empty[s], ((it / STAGES) - 1) & 1, flags, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sa = smem + s * STAGE_BYTES;
-          uint8_t* sb = sa + 2 * A_PLANE;
-          mbar_arrive_expect_tx(&full[s], tx_bytes);
-          // One copy per plane, each to its fixed offset (the boxes may hold
-          // fewer rows than the tile when n is small).
-          tma_load_4d(sa, amap, &full[s], kc * BK, tc.tm * BM, 0, am);
-          tma_load_4d(sa + A_PLANE, amap, &full[s], kc * BK, tc.tm * BM, 1, am);
-          if (G.b_mn) {
-            // B[k][n] row-major: 16 K-rows x 32 N-columns per copy, one copy per
-            // 32-column block of the tile, blocks MN_BLOCK bytes apart.
-            const int nblk = G.b_rows / 32;
-#pragma unroll 1
-            for (int q = 0; q < nblk; ++q) {
-              tma_load_4d(sb + q * MN_BLOCK, bmap, &full[s], tc.tn * BN + q * 32, kc * BK, 0, bm);
-              tma_load_4d(sb + B_PLANE + q * MN_BLOCK, bmap, &full[s], tc.tn * BN + q * 32, kc * BK, 1, bm);
+          for (int kc = 0; kc < nk; ++kc, ++it) {
+            const int s = it % STAGES;
+            if (it >= STAGES && !mbar_wait_bounded(&empty[s], ((it / STAGES) - 1) & 1, flags, abort_flag)) {
+              ok = false;
+              break;
             }
-          } else {
-            tma_load_4d(sb, bmap, &full[s], kc * BK, tc.tn * BN, 0, bm);
-            tma_load_4d(sb + B_PLANE, bmap, &full[s], kc * BK, tc.tn * BN, 1, bm);
+            uint8_t* sa = smem + s * STAGE_BYTES;
+            uint8_t* sb = sa + A_BYTES;
+            mbar_arrive_expect_tx(&full[s], tx_bytes);
+            tma_load_3d(sa, amap, &full[s], kc * BK, tc.tm * BM, am);
+            if (G.b_mn) {
+              // B[k][n] row-major: 16 K-rows x 32 N-columns per copy, one copy per
+              // 32-column block of the tile, blocks MN_BLOCK bytes apart.
+              const int nblk = G.b_rows / 32;
+#pragma unroll 1
+              for (int q = 0; q < nblk; ++q)
+                tma_load_3d(sb + q * MN_BLOCK, bmap, &full[s], tc.tn * BN + q * 32, kc * BK, bm);
+            } else {
+              tma_load_3d(sb, bmap, &full[s], kc * BK, tc.tn * BN, bm);
+            }
+          }
+        }
+        // Drain: no copy may still be landing in shared memory when the CTA
+        // retires (bounded by time only; normally these phases completed).
+#pragma unroll 1
+        for (uint32_t k = (it > STAGES ? it - STAGES : 0); k < it; ++k)
+          mbar_wait_bounded(&full[k % STAGES], (k / STAGES) & 1, flags, nullptr);
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        // K is cut into segments of SEG chunks.  Segment g (counted across
+        // tiles) accumulates from zero into TMEM buffer g & 1; the epilogue warps
+        // add each finished segment into fp32 registers with round-to-nearest.
+        // The tensor core's own additions (which truncate) then only ever see
+        // one segment's partial sums, which keeps long products unbiased.
+        uint32_t it = 0, sg = 0;
+        bool ok = true;
+#pragma unroll 1
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+          const TileCoord tc = tile_coord(L, tile);
+          if (tc.skip) continue;
+          const GemmGroup& G = L.g[tc.gi];
+          const int nk = G.n / BK;
+          const uint32_t idesc = idesc_tf32(BM, BN, G.b_mn);
+#pragma unroll 1
+          for (int kc = 0; kc < nk; ++kc, ++it) {
+            const int s = it % STAGES;
+            const bool first = (kc % SEG) == 0;
+            const uint32_t b = sg & 1;
+            const uint32_t tbuf = taddr + b * BN;
+            if (first && sg >= 2 &&
+                !mbar_wait_bounded(&acc_empty[b], ((sg >> 1) - 1) & 1, flags, abort_flag)) {
+              ok = false;
+              break;
+            }
+            if (!mbar_wait_bounded(&conv[s], (it / STAGES) & 1, flags, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_hi = smem_u32(smem + s * STAGE_BYTES);
+            const uint32_t b_hi = a_hi + A_BYTES;
+            const uint32_t a_lo = a_hi + RAW_BYTES;
+            const uint32_t b_lo = b_hi + RAW_BYTES;
+#pragma unroll
+            for (int ks = 0; ks < BK / 8; ++ks) {
+              const uint32_t off = ks * 32;  // 8 tf32 values = 32 bytes along K (K-major)
+              const uint64_t dah = smem_desc_k_sw64(a_hi + off);
+              const uint64_t dal = smem_desc_k_sw64(a_lo + off);
+              uint64_t dbh, dbl;
+              if (G.b_mn) {  // 8 K-rows = 1024 bytes = two 4-row groups
+                dbh = smem_desc_mn_sw128_32b(b_hi + ks * 1024, MN_BLOCK);
+                dbl = smem_desc_mn_sw128_32b(b_lo + ks * 1024, MN_BLOCK);
+              } else {
+                dbh = smem_desc_k_sw64(b_hi + off);
+                dbl = smem_desc_k_sw64(b_lo + off);
+              }
+              mma_tf32(tbuf, dah, dbh, idesc, (first && ks == 0) ? 0u : 1u);
+              mma_tf32(tbuf, dah, dbl, idesc, 1u);
+              mma_tf32(tbuf, dal, dbh, idesc, 1u);
+            }
+            mma_commit(&empty[s]);
+            if ((kc % SEG) == SEG - 1 || kc == nk - 1) {
+              mma_commit(&acc_full[b]);
+              ++sg;
+            }
           }
         }
       }
-      // Drain: no copy may still be landing in shared memory when the CTA
-      // retires (bounded by time only; normally these phases completed).
-#pragma unroll 1
-      for (uint32_t k = (it > STAGES ? it - STAGES : 0); k < it; ++k)
-        mbar_wait_bounded(&full[k % STAGES], (k / STAGES) & 1, flags, nullptr);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      // K is cut into segments of SEG chunks.  Segment g (counted across
-      // tiles) accumulates from zero into TMEM buffer g & 1; the epilogue warps
-      // add each finished segment into fp32 registers with round-to-nearest.
-      // The tensor core's own additions (which truncate) then only ever see
-      // one segment's partial sums, which keeps long products unbiased.
-      uint32_t it = 0, sg = 0;
+    } else {
+      // ------------------------------------------------------------ converters
+      // Each landed stage (A and B tiles, 24 KB of fp32) is split in place: the
+      // hi parts overwrite the fp32 values, the lo parts go RAW_BYTES further.
+      // The split is elementwise, so the swizzled layout TMA wrote carries over.
+      const int ct = threadIdx.x - 32 * CONV_WARP0;
+      uint32_t it = 0;
       bool ok = true;
 #pragma unroll 1
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileCoord tc = tile_coord(L, tile);
         if (tc.skip) continue;
-        const GemmGroup& G = L.g[tc.gi];
-        const int nk = G.n / BK;
-        const uint32_t idesc = idesc_tf32(BM, BN, G.b_mn);
+        const int nk = L.g[tc.gi].n / BK;
 #pragma unroll 1
         for (int kc = 0; kc < nk; ++kc, ++it) {
           const int s = it % STAGES;
-          const bool first = (kc % SEG) == 0;
-          const uint32_t b = sg & 1;
-          const uint32_t tbuf = taddr + b * BN;
-          if (first && sg >= 2 &&
-              !mbar_wait_bounded(&acc_empty[b], ((sg >> 1) - 1) & 1, flags, abort_flag)) {
-            ok = false;
-            break;
-          }
           if (!mbar_wait_bounded(&full[s], (it / STAGES) & 1, flags, abort_flag)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t a_hi = smem_u32(smem + s * STAGE_BYTES);
-          const uint32_t a_lo = a_hi + A_PLANE;
-          const uint32_t b_hi = a_hi + 2 * A_PLANE;
-          const uint32_t b_lo = b_hi + B_PLANE;
+          uint8_t* base = smem + s * STAGE_BYTES;
 #pragma unroll
-          for (int ks = 0; ks < BK / 8; ++ks) {
-            const uint32_t off = ks * 32;  // 8 tf32 values = 32 bytes along K (K-major)
-            const uint64_t dah = smem_desc_k_sw64(a_hi + off);
-            const uint64_t dal = smem_desc_k_sw64(a_lo + off);
-            uint64_t dbh, dbl;
-            if (G.b_mn) {  // 8 K-rows = 1024 bytes = two 4-row groups
-              dbh = smem_desc_mn_sw128_32b(b_hi + ks * 1024, MN_BLOCK);
-              dbl = smem_desc_mn_sw128_32b(b_lo + ks * 1024, MN_BLOCK);
-            } else {
-              dbh = smem_desc_k_sw64(b_hi + off);
-              dbl = smem_desc_k_sw64(b_lo + off);
-            }
-            mma_tf32(tbuf, dah, dbh, idesc, (first && ks == 0) ? 0u : 1u);
-            mma_tf32(tbuf, dah, dbl, idesc, 1u);
-            mma_tf32(tbuf, dal, dbh, idesc, 1u);
+          for (int i = 0; i < RAW_BYTES / 16 / CONV_THREADS; ++i) {
+            const int off = (i * CONV_THREADS + ct) * 16;
+            const float4 x = *reinterpret_cast<const float4*>(base + off);
+            float4 h, l;
+            split_tf32(x.x, h.x, l.x);
+            split_tf32(x.y, h.y, l.y);
+            split_tf32(x.z, h.z, l.z);
+            split_tf32(x.w, h.w, l.w);
+            *reinterpret_cast<float4*>(base + off) = h;
+            *reinterpret_cast<float4*>(base + RAW_BYTES + off) = l;
           }
-          mma_commit(&empty[s]);
-          if ((kc % SEG) == SEG - 1 || kc == nk - 1) {
-            mma_commit(&acc_full[b]);
-            ++sg;
-          }
+          fence_proxy_async_shared();
+          mbar_arrive(&conv[s]);
         }
       }
     }
   } else {
     // -------------------------------------------------------------- epilogue
     // 8 warps: warp w reads TMEM lane quarter (w & 3) and column half h.
-    const int ew = warp - 2;
+    warpgroup_regs_inc<HEAVY_REGS>();
+    const int ew = warp - EPI_WARP0;
     const int q = warp & 3;
     const int h = ew >> 2;
     const uint32_t lane_addr = taddr + (static_cast<uint32_t>(q * 32) << 16) + h * (BN / 2);
+    float* tilebuf = epi_tiles + ew * EPI_TILE_FLOATS;
     uint32_t sg = 0;
     bool ok = true;
 #pragma unroll 1
@@ -351,7 +394,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       const GemmGroup& G = L.g[tc.gi];
       const int n = G.n;
       const int nseg = (n / BK + SEG - 1) / SEG;
-      const int r = tc.tm * BM + q * 32 + lane;
       float sum[BN / 2];
 #pragma unroll
       for (int j = 0; j < BN / 2; ++j) sum[j] = 0.f;
@@ -378,11 +420,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) break;
       float resid = 0.f;
       bool nonfinite = false;
-      if (r < n) {
+      const int row0 = tc.tm * BM + q * 32;
+      if (row0 < n) {
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c) {
           const int c0 = tc.tn * BN + h * (BN / 2) + c * 32;
-          if (c0 < n) resid += epilogue_chunk(G, tc.mat, r, c0, &sum[c * 32], nonfinite);
+          if (c0 < n) epilogue_chunk(G, tc.mat, row0, c0, &sum[c * 32], tilebuf, lane, resid, nonfinite);
         }
       }
       if (G.ep.res) {
@@ -390,7 +433,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int o = 16; o > 0; o >>= 1) resid += __shfl_xor_sync(0xffffffffu, resid, o);
         if (lane == 0 && resid != 0.f) atomicAdd(&G.ep.res[tc.mat], resid);
       }
-      if (nonfinite) raise_flag(G.ep.flags, DEV_FLAG_NONFINITE);
+      if (__any_sync(0xffffffffu, nonfinite) && lane == 0) raise_flag(G.ep.flags, DEV_FLAG_NONFINITE);
       if (L.profile && ew == 0 && lane == 0 && prof_flops)
         atomicAdd(&prof_flops[L.prof_slot], G.flops_per_matrix / (G.tiles_m * G.tiles_n));
     }
@@ -411,9 +454,6 @@ Epilogue epilogue_defaults() {
   std::memset(&e, 0, sizeof(e));
   e.alpha = 1.f;
   e.gamma_stride = 1;
-  e.c_planes = 1;
-  e.d_planes = 1;
-  e.e_planes = 2;
   return e;
 }
 
@@ -432,25 +472,23 @@ int get_encoder() {
 }
 }  // namespace
 
-// Tensor map over a split stack (batch, 2, n, n) fp32: dimensions (innermost
-// first) column = n, row = n, plane = 2, matrix = batch; box {32, box_rows, 1,
-// 1} (one plane of a tile per copy).  K-major operand tiles (box_rows x 16)
-// use the 64-byte swizzle; MN-major tiles (mn_layout: 16 rows of K x 32
-// columns) the 128-byte swizzle with 32-byte atoms, the only MN-major tf32
-// layout of the tensor core.
-int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout,
-                     int planes) {
+// Tensor map over a plain stack (batch, n, n) fp32: dimensions (innermost
+// first) column = n, row = n, matrix = batch.  K-major operand tiles (box
+// box_rows x 16) use the 64-byte swizzle; MN-major tiles (mn_layout: 16 rows
+// of K x 32 columns) the 128-byte swizzle with 32-byte atoms, the only
+// MN-major tf32 layout of the tensor core.
+int encode_stack_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout) {
   int rc = get_encoder();
   if (rc) return rc;
   if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return set_error(-2, "stack base not 16-byte aligned");
   const cuuint64_t nn = static_cast<cuuint64_t>(n);
-  cuuint64_t dims[4] = {nn, nn, 2, static_cast<cuuint64_t>(batch)};
-  cuuint64_t strides[3] = {nn * 4, nn * nn * 4, static_cast<cuuint64_t>(planes) * nn * nn * 4};
+  cuuint64_t dims[3] = {nn, nn, static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {nn * 4, nn * nn * 4};
   // K-major boxes: BK columns (64 bytes) x box_rows rows; MN-major boxes: 32
   // columns (128 bytes) x box_rows (= BK) rows of K.
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(mn_layout ? 32 : BK), static_cast<cuuint32_t>(box_rows), 1, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(base), dims, strides, box, estr,
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(mn_layout ? 32 : BK), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
                         mn_layout ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -459,15 +497,14 @@ int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, 
   return 0;
 }
 
-int make_stack_maps(StackMaps& sm, float* base, int64_t batch, int n, int planes) {
-  sm.base = base;
-  sm.planes = planes;
+int make_stack_maps(StackMaps& sm, const float* base, int64_t batch, int n) {
+  sm.base = const_cast<float*>(base);
   sm.a_rows = n < BM ? n : BM;
   sm.b_rows = n < BN ? n : BN;
-  int rc = encode_split_map(&sm.a, base, batch, n, sm.a_rows, 0, planes);
+  int rc = encode_stack_map(&sm.a, base, batch, n, sm.a_rows, 0);
   if (rc) return rc;
-  if ((rc = encode_split_map(&sm.mn, base, batch, n, BK, 1, planes))) return rc;
-  return encode_split_map(&sm.b, base, batch, n, sm.b_rows, 0, planes);
+  if ((rc = encode_stack_map(&sm.mn, base, batch, n, BK, 1))) return rc;
+  return encode_stack_map(&sm.b, base, batch, n, sm.b_rows, 0);
 }
 
 Builder::Builder() : nmaps(0) {
@@ -500,6 +537,15 @@ int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
   int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
   if (rc) return rc;
   if (dev < 32 && !(attr_mask & (1u << dev))) {
+    // The register hand-over inside the kernel (setmaxnreg) balances only if
+    // the CTA is launched with exactly LAUNCH_REGS registers per thread; with
+    // fewer, the epilogue warps' request could never be met.
+    cudaFuncAttributes fa;
+    rc = check_cuda(cudaFuncGetAttributes(&fa, gemm3x_tf32_kernel), "cudaFuncGetAttributes(gemm)");
+    if (rc) return rc;
+    if (fa.numRegs != LAUNCH_REGS)
+      return set_error(-2, "gemm3x_tf32_kernel was built with %d registers per thread; the register split "
+                       "needs exactly %d", fa.numRegs, LAUNCH_REGS);
     rc = check_cuda(cudaFuncSetAttribute(gemm3x_tf32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SMEM_BYTES),
                     "cudaFuncSetAttribute(gemm)");

@@ -10,17 +10,11 @@
 namespace shampoo {
 
 // ---------------------------------------------------------------------------
-// Storage formats (P = planes per matrix, matrix stride P n^2 floats)
-//   plain stack  (P = 1): (batch, n, n) fp32, row-major matrices back to back.
-//   split stack  (P = 2): matrix i holds its tf32-exact "hi" plane then its
-//                "lo" plane (value = hi + lo, see split_tf32).
-// Split stacks are the operand format of the tensor-core GEMM.
+// Storage format: every stack is plain fp32, (batch, n, n), row-major matrices
+// back to back.  The tensor-core GEMM splits its operand tiles into tf32 hi /
+// lo parts in shared memory.
 // ---------------------------------------------------------------------------
 inline size_t plain_floats(int64_t batch, int n) { return static_cast<size_t>(batch) * n * n; }
-inline size_t split_floats(int64_t batch, int n) { return 2 * static_cast<size_t>(batch) * n * n; }
-inline size_t stack_floats(int64_t batch, int n, int planes) {
-  return static_cast<size_t>(planes) * batch * n * n;
-}
 
 constexpr int kMaxGroups = 4;
 constexpr int kMaxMaps = 2 * kMaxGroups;
@@ -37,12 +31,9 @@ struct Epilogue {
   const float* gamma_vec;
   int gamma_stride;
   const float* scale_vec;
-  const float* C;  // optional input stack (its value planes are read)
-  int c_planes;    // 1 (plain) or 2 (split)
+  const float* C;  // optional input stack
   float* D;        // optional main output stack
-  int d_planes;    // 1 (plain) or 2 (split)
-  float* E;        // optional second output (split): e_mul * v + e_add * [r == c]
-  int e_planes;    // 2
+  float* E;        // optional second output stack: e_mul * v + e_add * [r == c]
   float e_mul, e_add;
   float* res;        // optional: res[i] += sum over the valid diagonal of (1 - acc): tr(I - acc)
   const int* valid;  // per-matrix valid extent (nullable: n)
@@ -87,8 +78,7 @@ constexpr int kTileN = 256;
 constexpr int kTileK = 16;
 
 // Host helpers -------------------------------------------------------------
-int encode_split_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout,
-                     int planes);
+int encode_stack_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout);
 int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st);
 Epilogue epilogue_defaults();
 
@@ -126,10 +116,9 @@ struct StackMaps {
   CUtensorMap a, b;  // the stack as A (128-row boxes) and as K-major B (256-row boxes)
   CUtensorMap mn;    // as MN-major B: 16 rows of K x 32 columns of N
   float* base;
-  int planes;
   int a_rows, b_rows;
 };
-int make_stack_maps(StackMaps& sm, float* base, int64_t batch, int n, int planes = 2);
+int make_stack_maps(StackMaps& sm, const float* base, int64_t batch, int n);
 
 // How a group reads its B operand: as B^T (K-major; D = A B^T) or as B
 // (MN-major; D = A B).
@@ -149,7 +138,6 @@ struct Builder {
 
 int launch_report(const int* iters, const int* add, const int* done, int64_t batch, int default_iters, int* out,
                   int* flags, bool residual, cudaStream_t st);
-int launch_split_plain(const float* src, float* dst, int64_t batch, int n, cudaStream_t st);
 
 // Elementwise / reduction kernels (kernels_elem.cu) ---------------------------
 struct StackArgs {
@@ -165,19 +153,17 @@ int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, flo
 // kind: 0 = Newton (M0, T0 = ((p+1)I - M0)/p, X1 = T0)
 //       1 = Newton-DB (Y0 = A', T0 = (3I - A')/2, Z1 = T0)
 int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const int* valid, float eps, int p,
-                         const float* s, float* out0, float* out1, float* out2, int planes0, int planes1, int planes2,
-                         cudaStream_t st);
+                         const float* s, float* out0, float* out1, float* out2, cudaStream_t st);
 // Second Newton-DB stage: Y0' = Y_par(i) (parity from iters), T0 = (3I - Y0')/2, Z1 = T0.
 int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters, int64_t batch, int n,
                               float* Ynew0, float* T, float* Z1, cudaStream_t st);
 int launch_check(float* res, int* done, int* iters, const int* valid, int64_t batch, int n, float tol, int it,
                  int* flags, cudaStream_t st);
-int launch_finalize(const float* X0, const float* X1, int src_planes, const int* iters, int default_iters,
-                    const float* sc, int64_t batch, int n, float* out_plain, float* out_split, int* flags,
-                    cudaStream_t st);
+int launch_finalize(const float* X0, const float* X1, const int* iters, int default_iters, const float* sc,
+                    int64_t batch, int n, float* out, int* flags, cudaStream_t st);
 int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int degree,
                       float lo, const float* s, float* coef, float* sc, float* Xt, float* bd, float* bd1,
-                      int xt_planes, int b_planes, cudaStream_t st);
+                      cudaStream_t st);
 int launch_fill_iters(int* iters, int64_t batch, int value, cudaStream_t st);
 
 // Inverse-root solver (solver.cu) ---------------------------------------------
@@ -187,8 +173,7 @@ struct RootJob {
   float eps, tol, cheb_lo;
   const float* A;    // plain stack input
   const int* valid;  // device valid extents (nullable)
-  float* X_plain;    // plain output (nullable)
-  float* X_split;    // split output (nullable)
+  float* X;          // output stack
   int* iters_used;   // device per-matrix iterations (nullable)
   int* flags;        // device status word (nullable)
 };

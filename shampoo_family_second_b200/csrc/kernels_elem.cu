@@ -19,30 +19,14 @@ __device__ __forceinline__ float load_grad(const void* g, size_t idx, int dtype)
   return reinterpret_cast<const float*>(g)[idx];
 }
 
-__device__ __forceinline__ void store_split(float* stack, size_t mat, size_t nn, size_t idx, float v) {
-  float h, l;
-  split_tf32(v, h, l);
-  stack[mat * 2 * nn + idx] = h;
-  stack[mat * 2 * nn + nn + idx] = l;
-}
-
-// Matrix `mat` of a stack with `planes` planes per matrix (2: split).
-__device__ __forceinline__ void store_sym(float* stack, int planes, size_t mat, size_t nn, size_t idx, float v) {
-  float h, l;
-  split_tf32(v, h, l);
-  float* m = stack + mat * planes * nn;
-  m[idx] = h;
-  m[nn + idx] = l;
-}
-
 // ---------------------------------------------------------------------------
 // A1 partition / stack.  DASH abstract: preconditioner blocks stacked into 3D
 // tensors.  Block b of the table {param, row0, col0, r, c} is copied from the
-// row-major gradient into Gs[b] (B x B, split) and its transpose into Gt[b],
+// row-major gradient into Gs[b] (B x B) and its transpose into Gt[b],
 // zero-padded beyond (r, c).  Also records where the block's weights live.
 // grid (B/32, B/32, nb), block (32, 8).
 // ---------------------------------------------------------------------------
-__global__ void stack_split_kernel(const __grid_constant__ StackArgs args, const int* __restrict__ table, int B,
+__global__ void stack_blocks_kernel(const __grid_constant__ StackArgs args, const int* __restrict__ table, int B,
                                    int dtype, float* __restrict__ Gs, float* __restrict__ Gt, float** blk_wptr,
                                    int* blk_ld) {
   __shared__ float tile[32][33];
@@ -62,14 +46,14 @@ __global__ void stack_split_kernel(const __grid_constant__ StackArgs args, const
     float v = 0.f;
     if (row < r && col < c) v = load_grad(g, static_cast<size_t>(row0 + row) * ld + col0 + col, dtype);
     tile[ty + 8 * k][tx] = v;
-    store_split(Gs, b, nn, static_cast<size_t>(row) * B + col, v);
+    Gs[b * nn + static_cast<size_t>(row) * B + col] = v;
   }
   __syncthreads();
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int row = bj * 32 + ty + 8 * k;  // row of G^T = column of G
     const int col = bi * 32 + tx;
-    store_split(Gt, b, nn, static_cast<size_t>(row) * B + col, tile[tx][ty + 8 * k]);
+    Gt[b * nn + static_cast<size_t>(row) * B + col] = tile[tx][ty + 8 * k];
   }
   if (bi == 0 && bj == 0 && tx == 0 && ty == 0) {
     blk_wptr[b] = args.w[param] + static_cast<size_t>(row0) * ld + col0;
@@ -133,8 +117,7 @@ __device__ __forceinline__ float effective_eps(float eps, float s) { return fmax
 // ---------------------------------------------------------------------------
 __global__ void root_prologue_kernel(int kind, const float* __restrict__ A, int n, const int* __restrict__ valid,
                                      float eps, int p, const float* __restrict__ s, float* __restrict__ out0,
-                                     float* __restrict__ out1, float* __restrict__ out2, int planes0, int planes1,
-                                     int planes2) {
+                                     float* __restrict__ out1, float* __restrict__ out2) {
   __shared__ float t1[32][33];
   __shared__ float t2[32][33];
   const int i = blockIdx.z;
@@ -162,10 +145,10 @@ __global__ void root_prologue_kernel(int kind, const float* __restrict__ A, int 
       t = (static_cast<float>(p + 1) * d - m) / static_cast<float>(p);
     else
       t = 0.5f * (3.f * d - m);
-    const size_t idx = static_cast<size_t>(r) * n + c;
-    store_sym(out0, planes0, i, nn, idx, m);
-    store_sym(out1, planes1, i, nn, idx, t);
-    store_sym(out2, planes2, i, nn, idx, t);
+    const size_t idx = i * nn + static_cast<size_t>(r) * n + c;
+    out0[idx] = m;
+    out1[idx] = t;
+    out2[idx] = t;
   }
 }
 
@@ -178,12 +161,12 @@ __global__ void db_stage2_kernel(const float* Y0, const float* Y1, const int* __
   const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= nn) return;
   const float* src = (iters[i] & 1) ? Y1 : Y0;
-  const float y = src[i * 2 * nn + idx] + src[i * 2 * nn + nn + idx];
+  const float y = src[i * nn + idx];
   const int r = static_cast<int>(idx / n), c = static_cast<int>(idx % n);
   const float t = 0.5f * (3.f * ((r == c) ? 1.f : 0.f) - y);
-  store_split(Ynew0, i, nn, idx, y);
-  store_split(T, i, nn, idx, t);
-  store_split(Z1, i, nn, idx, t);
+  Ynew0[i * nn + idx] = y;
+  T[i * nn + idx] = t;
+  Z1[i * nn + idx] = t;
 }
 
 // Residual check after iteration `it`: |tr(I - acc)| / valid <= tol marks the
@@ -208,15 +191,14 @@ __global__ void check_kernel(float* res, int* done, int* iters, const int* valid
   }
 }
 
-// Output pass: X = sym(hi + lo of the final iterate) * s^{-1/p}, with
-// sym(Y) = (Y + Y^T)/2.  The principal root is symmetric; the iterates pick
-// up a small antisymmetric rounding component (the products are formed as
-// A B^T), which this removes.  The final iterate sits in buffer
-// (iters[i] & 1).  Writes a plain and/or a split stack.
+// Output pass: X = sym(final iterate) * s^{-1/p}, with sym(Y) = (Y + Y^T)/2.
+// The principal root is symmetric; the iterates pick up a small
+// antisymmetric rounding component (the products are formed as A B^T), which
+// this removes.  The final iterate sits in buffer (iters[i] & 1).
 // grid (n/32, n/32, batch), block (32, 8).
-__global__ void finalize_kernel(const float* __restrict__ X0, const float* __restrict__ X1, int src_planes,
+__global__ void finalize_kernel(const float* __restrict__ X0, const float* __restrict__ X1,
                                 const int* __restrict__ iters, int default_iters, const float* __restrict__ sc, int n,
-                                float* __restrict__ out_plain, float* __restrict__ out_split, int* flags) {
+                                float* __restrict__ out, int* flags) {
   __shared__ float t1[32][33];
   __shared__ float t2[32][33];
   const int i = blockIdx.z;
@@ -224,13 +206,11 @@ __global__ void finalize_kernel(const float* __restrict__ X0, const float* __res
   const int tx = threadIdx.x, ty = threadIdx.y;
   const size_t nn = static_cast<size_t>(n) * n;
   const int it = iters ? iters[i] : default_iters;
-  const float* src = ((it & 1) ? X1 : X0) + i * static_cast<size_t>(src_planes) * nn;
+  const float* src = ((it & 1) ? X1 : X0) + i * nn;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const size_t a = static_cast<size_t>(bi * 32 + ty + 8 * k) * n + bj * 32 + tx;
-    const size_t b = static_cast<size_t>(bj * 32 + ty + 8 * k) * n + bi * 32 + tx;
-    t1[ty + 8 * k][tx] = src[a] + src[nn + a];
-    t2[ty + 8 * k][tx] = src[b] + src[nn + b];
+    t1[ty + 8 * k][tx] = src[static_cast<size_t>(bi * 32 + ty + 8 * k) * n + bj * 32 + tx];
+    t2[ty + 8 * k][tx] = src[static_cast<size_t>(bj * 32 + ty + 8 * k) * n + bi * 32 + tx];
   }
   __syncthreads();
   const float f = sc[i];
@@ -240,9 +220,7 @@ __global__ void finalize_kernel(const float* __restrict__ X0, const float* __res
     const int r = bi * 32 + ty + 8 * k, c = bj * 32 + tx;
     const float v = 0.5f * (t1[ty + 8 * k][tx] + t2[tx][ty + 8 * k]) * f;
     bad |= !isfinite(v);
-    const size_t idx = static_cast<size_t>(r) * n + c;
-    if (out_plain) out_plain[i * nn + idx] = v;
-    if (out_split) store_split(out_split, i, nn, idx, v);
+    out[i * nn + static_cast<size_t>(r) * n + c] = v;
   }
   if (bad) raise_flag(flags, DEV_FLAG_NONFINITE);
 }
@@ -285,8 +263,7 @@ __global__ void cheb_coef_kernel(const float* __restrict__ s, int degree, int p,
 // b_d = c_d I and b_{d-1} = 2 c_d Xt + c_{d-1} I (first two Clenshaw terms).
 __global__ void cheb_prologue_kernel(const float* __restrict__ A, int n, const int* __restrict__ valid, float eps,
                                      const float* __restrict__ s, const float* __restrict__ coef, int degree,
-                                     float* __restrict__ Xt, float* __restrict__ bd, float* __restrict__ bd1,
-                                     int xt_planes, int b_planes) {
+                                     float* __restrict__ Xt, float* __restrict__ bd, float* __restrict__ bd1) {
   __shared__ float t1[32][33];
   __shared__ float t2[32][33];
   const int i = blockIdx.z;
@@ -313,10 +290,10 @@ __global__ void cheb_prologue_kernel(const float* __restrict__ A, int n, const i
     const float d = (r == c) ? 1.f : 0.f;
     const float m = (r < v && c < v) ? (sym + d * eps_eff) * inv_s : d;
     const float x = (2.f * m - (1.f + a) * d) / (1.f - a);
-    const size_t idx = static_cast<size_t>(r) * n + c;
-    store_sym(Xt, xt_planes, i, nn, idx, x);
-    store_sym(bd, b_planes, i, nn, idx, cd * d);
-    store_sym(bd1, b_planes, i, nn, idx, 2.f * cd * x + cd1 * d);
+    const size_t idx = i * nn + static_cast<size_t>(r) * n + c;
+    Xt[idx] = x;
+    bd[idx] = cd * d;
+    bd1[idx] = 2.f * cd * x + cd1 * d;
   }
 }
 
@@ -332,9 +309,9 @@ int launch_stack(const StackArgs& args, const int* d_table, int nb, int B, int g
   if (nb == 0) return 0;
   ProfScope ps(K_STACK, st, 0.0, alg_bytes);
   dim3 grid(B / 32, B / 32, nb), block(32, 8);
-  stack_split_kernel<<<grid, block, 0, st>>>(args, d_table, B, grad_dtype, Gs, Gts, blk_wptr, blk_ld);
+  stack_blocks_kernel<<<grid, block, 0, st>>>(args, d_table, B, grad_dtype, Gs, Gts, blk_wptr, blk_ld);
   count_launch();
-  return check_cuda(cudaGetLastError(), "stack_split_kernel");
+  return check_cuda(cudaGetLastError(), "stack_blocks_kernel");
 }
 
 int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, float eps, int p, float* s, float* sc,
@@ -347,13 +324,11 @@ int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, flo
 }
 
 int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const int* valid, float eps, int p,
-                         const float* s, float* out0, float* out1, float* out2, int planes0, int planes1, int planes2,
-                         cudaStream_t st) {
+                         const float* s, float* out0, float* out1, float* out2, cudaStream_t st) {
   if (batch == 0) return 0;
-  ProfScope ps(K_PROLOGUE, st, 0.0, (4.0 + 4.0 * (planes0 + planes1 + planes2)) * batch * n * n);
+  ProfScope ps(K_PROLOGUE, st, 0.0, 16.0 * batch * n * n);
   dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
-  root_prologue_kernel<<<grid, block, 0, st>>>(kind, A, n, valid, eps, p, s, out0, out1, out2, planes0, planes1,
-                                               planes2);
+  root_prologue_kernel<<<grid, block, 0, st>>>(kind, A, n, valid, eps, p, s, out0, out1, out2);
   count_launch();
   return check_cuda(cudaGetLastError(), "root_prologue_kernel");
 }
@@ -361,7 +336,7 @@ int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const i
 int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters, int64_t batch, int n, float* Ynew0,
                               float* T, float* Z1, cudaStream_t st) {
   if (batch == 0) return 0;
-  ProfScope ps(K_PROLOGUE, st, 0.0, (8.0 + 3 * 8.0) * batch * n * n);
+  ProfScope ps(K_PROLOGUE, st, 0.0, 16.0 * batch * n * n);
   const size_t nn = static_cast<size_t>(n) * n;
   dim3 grid(static_cast<unsigned>((nn + 255) / 256), static_cast<unsigned>(batch));
   db_stage2_kernel<<<grid, 256, 0, st>>>(Y0, Y1, iters, n, Ynew0, T, Z1);
@@ -379,22 +354,18 @@ int launch_check(float* res, int* done, int* iters, const int* valid, int64_t ba
   return check_cuda(cudaGetLastError(), "check_kernel");
 }
 
-int launch_finalize(const float* X0, const float* X1, int src_planes, const int* iters, int default_iters,
-                    const float* sc, int64_t batch, int n, float* out_plain, float* out_split, int* flags,
-                    cudaStream_t st) {
+int launch_finalize(const float* X0, const float* X1, const int* iters, int default_iters, const float* sc,
+                    int64_t batch, int n, float* out, int* flags, cudaStream_t st) {
   if (batch == 0) return 0;
-  const double bytes = (8.0 + (out_plain ? 4.0 : 0.0) + (out_split ? 8.0 : 0.0)) * batch * n * n;
-  ProfScope ps(K_FINALIZE, st, 0.0, bytes);
+  ProfScope ps(K_FINALIZE, st, 0.0, 8.0 * batch * n * n);
   dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
-  finalize_kernel<<<grid, block, 0, st>>>(X0, X1, src_planes, iters, default_iters, sc, n, out_plain, out_split,
-                                          flags);
+  finalize_kernel<<<grid, block, 0, st>>>(X0, X1, iters, default_iters, sc, n, out, flags);
   count_launch();
   return check_cuda(cudaGetLastError(), "finalize_kernel");
 }
 
 int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int degree, float lo,
-                      const float* s, float* coef, float* sc, float* Xt, float* bd, float* bd1, int xt_planes,
-                      int b_planes, cudaStream_t st) {
+                      const float* s, float* coef, float* sc, float* Xt, float* bd, float* bd1, cudaStream_t st) {
   if (batch == 0) return 0;
   {
     ProfScope ps(K_CHEB_COEF, st, 0.0, 8.0 * batch);
@@ -403,9 +374,9 @@ int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, fl
     int rc = check_cuda(cudaGetLastError(), "cheb_coef_kernel");
     if (rc) return rc;
   }
-  ProfScope ps(K_PROLOGUE, st, 0.0, (4.0 + 4.0 * (xt_planes + 2 * b_planes)) * batch * n * n);
+  ProfScope ps(K_PROLOGUE, st, 0.0, 16.0 * batch * n * n);
   dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
-  cheb_prologue_kernel<<<grid, block, 0, st>>>(A, n, valid, eps, s, coef, degree, Xt, bd, bd1, xt_planes, b_planes);
+  cheb_prologue_kernel<<<grid, block, 0, st>>>(A, n, valid, eps, s, coef, degree, Xt, bd, bd1);
   count_launch();
   return check_cuda(cudaGetLastError(), "cheb_prologue_kernel");
 }
@@ -435,22 +406,6 @@ __global__ void report_kernel(const int* iters, const int* add, const int* done,
   if (out) out[i] = failed ? -it : it;
 }
 
-// Plain stack -> split stack (hi / lo planes).
-__global__ void split_plain_kernel(const float* __restrict__ src, float* __restrict__ dst, int n) {
-  const int i = blockIdx.y;
-  const size_t nn = static_cast<size_t>(n) * n;
-  const size_t idx = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
-  if (idx >= nn) return;
-  const float4 v = *reinterpret_cast<const float4*>(src + i * nn + idx);
-  float h[4], l[4];
-  split_tf32(v.x, h[0], l[0]);
-  split_tf32(v.y, h[1], l[1]);
-  split_tf32(v.z, h[2], l[2]);
-  split_tf32(v.w, h[3], l[3]);
-  *reinterpret_cast<float4*>(dst + i * 2 * nn + idx) = make_float4(h[0], h[1], h[2], h[3]);
-  *reinterpret_cast<float4*>(dst + i * 2 * nn + nn + idx) = make_float4(l[0], l[1], l[2], l[3]);
-}
-
 }  // namespace
 
 int launch_report(const int* iters, const int* add, const int* done, int64_t batch, int default_iters, int* out,
@@ -461,16 +416,6 @@ int launch_report(const int* iters, const int* add, const int* done, int64_t bat
       iters, add, done, static_cast<int>(batch), default_iters, out, flags, residual ? 1 : 0);
   count_launch();
   return check_cuda(cudaGetLastError(), "report_kernel");
-}
-
-int launch_split_plain(const float* src, float* dst, int64_t batch, int n, cudaStream_t st) {
-  if (batch == 0) return 0;
-  ProfScope ps(K_PROLOGUE, st, 0.0, 12.0 * batch * n * n);
-  const size_t nn4 = static_cast<size_t>(n) * n / 4;
-  dim3 grid(static_cast<unsigned>((nn4 + 255) / 256), static_cast<unsigned>(batch));
-  split_plain_kernel<<<grid, 256, 0, st>>>(src, dst, n);
-  count_launch();
-  return check_cuda(cudaGetLastError(), "split_plain_kernel");
 }
 
 }  // namespace shampoo

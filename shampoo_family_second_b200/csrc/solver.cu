@@ -42,23 +42,11 @@ namespace {
 
 constexpr int NEWTON_B = B_TRANSPOSED;
 
-// Planes per matrix of each scratch stack, by solver (all split stacks).
+// Scratch stacks per solver (plain fp32, n x n per matrix):
 //   Newton    : M0 M1 X0 X1 T T2 T4
 //   Newton-DB : Y0 Y1 Z0 Z1 T
 //   Chebyshev : Xt b0 b1 b2
-constexpr int kNewtonPlanes[7] = {2, 2, 2, 2, 2, 2, 2};
-constexpr int kDbPlanes[5] = {2, 2, 2, 2, 2};
-constexpr int kChebPlanes[4] = {2, 2, 2, 2};
-
 int stacks_for(int solver) { return solver == 0 ? 7 : (solver == 1 ? 5 : 4); }
-int planes_of(int solver, int k) {
-  return solver == 0 ? kNewtonPlanes[k] : (solver == 1 ? kDbPlanes[k] : kChebPlanes[k]);
-}
-int total_planes(int solver) {
-  int t = 0;
-  for (int k = 0; k < stacks_for(solver); ++k) t += planes_of(solver, k);
-  return t;
-}
 
 constexpr size_t kAlign = 256;
 constexpr size_t kHeader = 64 * 1024;  // covers the alignment padding of the arrays
@@ -93,7 +81,7 @@ Layout carve(void* base, int64_t cb, int n, int solver) {
   L.iters1 = reinterpret_cast<int*>(take(cb * 4));
   L.coef = reinterpret_cast<float*>(take(cb * 4 * (kMaxChebDegree + 2)));
   for (int k = 0; k < stacks_for(solver); ++k)
-    L.stack[k] = reinterpret_cast<float*>(take(stack_floats(cb, n, planes_of(solver, k)) * 4));
+    L.stack[k] = reinterpret_cast<float*>(take(plain_floats(cb, n) * 4));
   return L;
 }
 
@@ -102,7 +90,7 @@ Layout carve(void* base, int64_t cb, int n, int solver) {
 size_t root_scratch_header() { return kHeader; }
 
 size_t root_scratch_per_matrix(int n, int solver) {
-  return static_cast<size_t>(total_planes(solver)) * n * n * 4 + 4 * (kVecInts + kMaxChebDegree + 2);
+  return static_cast<size_t>(stacks_for(solver)) * n * n * 4 + 4 * (kVecInts + kMaxChebDegree + 2);
 }
 
 int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, cudaStream_t st) {
@@ -122,12 +110,11 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
     Layout S = carve(scratch, cb, n, job.solver);
     const float* A = job.A + off * static_cast<int64_t>(n) * n;
     const int* valid = job.valid ? job.valid + off : nullptr;
-    float* out_plain = job.X_plain ? job.X_plain + off * static_cast<int64_t>(n) * n : nullptr;
-    float* out_split = job.X_split ? job.X_split + off * 2 * static_cast<int64_t>(n) * n : nullptr;
+    float* out = job.X + off * static_cast<int64_t>(n) * n;
     int* iters_out = job.iters_used ? job.iters_used + off : nullptr;
     StackMaps sm[7];
     for (int k = 0; k < stacks_for(job.solver); ++k)
-      if ((rc = make_stack_maps(sm[k], S.stack[k], cb, n, planes_of(job.solver, k)))) return rc;
+      if ((rc = make_stack_maps(sm[k], S.stack[k], cb, n))) return rc;
     if ((rc = launch_frob_norm(A, cb, n, valid, job.eps, p, S.s, S.sc, st))) return rc;
     if (residual) {
       if ((rc = check_cuda(cudaMemsetAsync(S.done, 0, cb * 4, st), "memset done"))) return rc;
@@ -141,24 +128,22 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
 
     if (job.solver == 0) {
       // ------------------------------------------------------------ coupled Newton
-      StackMaps* M = &sm[0];  // M[0], M[1]  (paired)
-      StackMaps* X = &sm[2];  // X[0], X[1]  (split)
-      StackMaps& T = sm[4];   // paired
-      StackMaps& T2 = sm[5];  // paired
-      StackMaps& T4 = sm[6];  // split
-      if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, M[0].base, T.base, X[1].base, 2, 2, 2, st)))
+      StackMaps* M = &sm[0];  // M[0], M[1]
+      StackMaps* X = &sm[2];  // X[0], X[1]
+      StackMaps& T = sm[4];
+      StackMaps& T2 = sm[5];
+      StackMaps& T4 = sm[6];
+      if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, M[0].base, T.base, X[1].base, st)))
         return rc;
       for (int j = 0; j < job.iters; ++j) {
         {
           Builder b;
           Epilogue& e = b.add(cbi, n, T, 0, T, 0, f1, NEWTON_B);  // T2 = T T
           e.D = T2.base;
-          e.d_planes = 2;
           common(e);
           if (j >= 1) {
             Epilogue& ex = b.add(cbi, n, X[j & 1], 0, T, 0, f1, NEWTON_B);  // X <- X T
             ex.D = X[(j + 1) & 1].base;
-            ex.d_planes = 2;
             common(ex);
           }
           if ((rc = b.launch(st))) return rc;
@@ -169,7 +154,6 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
           Builder b;
           Epilogue& e = b.add(cbi, n, T2, 0, T2, 0, f1, NEWTON_B);  // T4 = T2 T2
           e.D = T4.base;
-          e.d_planes = 2;
           common(e);
           if ((rc = b.launch(st))) return rc;
           P = &T4;
@@ -178,9 +162,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
           Builder b;
           Epilogue& e = b.add(cbi, n, *P, 0, M[j & 1], 0, f1, NEWTON_B);  // M <- T^p M
           e.D = M[(j + 1) & 1].base;
-          e.d_planes = 2;
           e.E = T.base;  // next T = ((p+1) I - M) / p
-          e.e_planes = 2;
           e.e_mul = -1.f / p;
           e.e_add = static_cast<float>(p + 1) / p;
           e.res = residual ? S.res : nullptr;
@@ -192,8 +174,8 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
             (rc = launch_check(S.res, S.done, S.iters, valid, cb, n, job.tol, j + 1, job.flags, st)))
           return rc;
       }
-      if ((rc = launch_finalize(X[0].base, X[1].base, 2, residual ? S.iters : nullptr, job.iters, S.sc, cb, n,
-                                out_plain, out_split, job.flags, st)))
+      if ((rc = launch_finalize(X[0].base, X[1].base, residual ? S.iters : nullptr, job.iters, S.sc, cb, n, out,
+                                job.flags, st)))
         return rc;
       if ((iters_out || residual) &&
           (rc = launch_report(residual ? S.iters : nullptr, nullptr, residual ? S.done : nullptr, cb, job.iters,
@@ -204,7 +186,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       StackMaps* Y = &sm[0];
       StackMaps* Z = &sm[2];
       StackMaps& T = sm[4];
-      if ((rc = launch_root_prologue(1, A, cb, n, valid, job.eps, p, S.s, Y[0].base, T.base, Z[1].base, 2, 2, 2, st)))
+      if ((rc = launch_root_prologue(1, A, cb, n, valid, job.eps, p, S.s, Y[0].base, T.base, Z[1].base, st)))
         return rc;
       const int stages = (p == 4) ? 2 : 1;
       for (int stage = 0; stage < stages; ++stage) {
@@ -230,12 +212,10 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
             Builder b;
             Epilogue& ey = b.add(cbi, n, Y[j & 1], 0, T, 0, f1, B_MN_MAJOR);  // Y <- Y T
             ey.D = Y[(j + 1) & 1].base;
-            ey.d_planes = 2;
             common(ey);
             if (j >= 1) {
               Epilogue& ez = b.add(cbi, n, T, 0, Z[j & 1], 0, f1, B_MN_MAJOR);  // Z <- T Z
               ez.D = Z[(j + 1) & 1].base;
-              ez.d_planes = 2;
               common(ez);
             }
             if ((rc = b.launch(st))) return rc;
@@ -247,7 +227,6 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
             e.alpha = -0.5f;
             e.gamma = 1.5f;
             e.D = T.base;
-            e.d_planes = 2;
             e.res = residual ? S.res : nullptr;
             e.valid = valid;
             common(e);
@@ -258,8 +237,8 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
             return rc;
         }
       }
-      if ((rc = launch_finalize(Z[0].base, Z[1].base, 2, residual ? S.iters : nullptr, job.iters, S.sc, cb, n,
-                                out_plain, out_split, job.flags, st)))
+      if ((rc = launch_finalize(Z[0].base, Z[1].base, residual ? S.iters : nullptr, job.iters, S.sc, cb, n, out,
+                                job.flags, st)))
         return rc;
       const int* add = (p == 4 && residual) ? S.iters1 : nullptr;
       const int default_total = (p == 4) ? 2 * job.iters : job.iters;
@@ -271,9 +250,9 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       // ------------------------------------------------------------ Chebyshev
       const int d = job.cheb_degree;
       StackMaps& Xt = sm[0];
-      StackMaps* b = &sm[1];  // b[k % 3], paired
+      StackMaps* b = &sm[1];  // b[k % 3]
       if ((rc = launch_cheb_setup(A, cb, n, valid, job.eps, p, d, job.cheb_lo, S.s, S.coef, S.sc, Xt.base,
-                                  b[d % 3].base, b[(d - 1) % 3].base, 2, 2, st)))
+                                  b[d % 3].base, b[(d - 1) % 3].base, st)))
         return rc;
       for (int k = d - 2; k >= 1; --k) {  // b_k = 2 Xt b_{k+1} - b_{k+2} + c_k I
         Builder bl;
@@ -281,11 +260,9 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
         e.alpha = 2.f;
         e.beta = -1.f;
         e.C = b[(k + 2) % 3].base;
-        e.c_planes = 2;
         e.gamma_vec = S.coef + k;
         e.gamma_stride = d + 2;
         e.D = b[k % 3].base;
-        e.d_planes = 2;
         e.flags = job.flags;
         if ((rc = bl.launch(st))) return rc;
       }
@@ -295,12 +272,10 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
         e.alpha = 1.f;
         e.beta = -1.f;
         e.C = b[2].base;
-        e.c_planes = 2;
         e.gamma_vec = S.coef;
         e.gamma_stride = d + 2;
         e.scale_vec = S.sc;
-        e.D = out_split ? out_split : out_plain;
-        e.d_planes = out_split ? 2 : 1;
+        e.D = out;
         e.flags = job.flags;
         if ((rc = bl.launch(st))) return rc;
       }

@@ -54,10 +54,16 @@ def test_noalloc_matches_inv_root_batched_on_two_calls(sb, solver, n, batch, tol
             assert oracle.rel_fro(Xn[b], Xr[b]) <= TOL
 
 
-def test_noalloc_rejects_sizes_beyond_the_fixed_scratch(sb):
-    A = torch.zeros(1, 1024, 1024, device="cuda")
-    X = torch.empty_like(A)
-    rc = sb.lib.inv_root_batched_noalloc(A.data_ptr(), X.data_ptr(), 1, 1024, 4, 1e-6, 0, 10, 0.0, 32, 0.0,
-                                         None, None, torch.cuda.current_stream().cuda_stream)
-    assert rc == sb.ERR_UNSUPPORTED
-    assert "fixed scratch" in sb.last_error()
+def test_noalloc_largest_block_in_chunks(sb):
+    """n = 1024 with coupled Newton needs 28 MiB of scratch per matrix: the
+    fixed 32 MiB array takes one matrix at a time."""
+    A64 = workloads.spd_batch(2, 1024, 1e3, seed=7)
+    A = torch.from_numpy(A64.astype(np.float32)).cuda()
+    X_ref, it_ref, st_ref = sb.inv_root_batched(A, p=4, eps=1e-6, solver=0, iters=20, tol=0.0)
+    X, it, st = call_noalloc(sb, A, 4, 1e-6, 0, 20, 0.0)
+    torch.cuda.synchronize()
+    assert int(st.item()) == int(st_ref.item()) == 0
+    assert torch.equal(it, it_ref)
+    Xr, Xn = X_ref.cpu().numpy().astype(np.float64), X.cpu().numpy().astype(np.float64)
+    for b in range(2):
+        assert oracle.rel_fro(Xn[b], Xr[b]) <= TOL
