@@ -262,7 +262,7 @@ def run_ours(args, wl):
     for t in range(args.warmup):
         opt.step(W, grads[t % ring])
     barrier()
-    if opt.status(reset=True) & ~sb.DEVFLAG_NOT_CONVERGED:
+    if opt.status(reset=True) & ~(sb.DEVFLAG_NOT_CONVERGED | sb.DEVFLAG_STAGNATED):
         raise RuntimeError("device status reported an error during warm-up")
 
     # ---- timed region: K steps, per-step events, L2 flushed between steps

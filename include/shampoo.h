@@ -64,7 +64,10 @@ enum {
 enum {
   SHAMPOO_DEVFLAG_NONFINITE = 1,     /* a NaN or Inf was produced */
   SHAMPOO_DEVFLAG_NOT_CONVERGED = 2, /* tol > 0 and a residual stayed above tol after iters */
-  SHAMPOO_DEVFLAG_TIMEOUT = 4        /* a bounded on-chip wait gave up (kernel unwound) */
+  SHAMPOO_DEVFLAG_TIMEOUT = 4,       /* a bounded on-chip wait gave up (kernel unwound) */
+  SHAMPOO_DEVFLAG_STAGNATED = 8      /* tol > 0 and a residual stopped improving above tol once every
+                                        eigenvalue above fp32 resolution had converged (the fp32 floor
+                                        of a rank-deficient or ill-conditioned matrix); stopped there */
 };
 
 /* Inverse-root solvers (DASH abstract names Newton-DB and Chebyshev). */
@@ -193,7 +196,8 @@ SHAMPOO_API int inv_root_scratch_bytes(int64_t batch, int32_t n, int32_t solver,
  *  d_scratch     device scratch, 256-byte aligned (see inv_root_scratch_bytes).
  *  d_iters_used  nullable device int32[batch]: iterations run per matrix
  *                (Newton-DB p = 4: both stages; Chebyshev: the degree); negative
- *                when tol > 0 and the cap was reached without convergence.
+ *                when tol > 0 and the residual did not reach tol (cap reached:
+ *                SHAMPOO_DEVFLAG_NOT_CONVERGED; stagnated: SHAMPOO_DEVFLAG_STAGNATED).
  *  d_status      nullable device int32: OR of SHAMPOO_DEVFLAG_* (not cleared).
  *  stream        cudaStream_t as void*.  Enqueued; no host sync. */
 SHAMPOO_API int inv_root_batched(const float* d_A, float* d_X, int64_t batch, int32_t n, int32_t p, float eps, int32_t solver,

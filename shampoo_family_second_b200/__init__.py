@@ -28,6 +28,7 @@ ERR_DEVICE = -5
 DEVFLAG_NONFINITE = 1
 DEVFLAG_NOT_CONVERGED = 2
 DEVFLAG_TIMEOUT = 4
+DEVFLAG_STAGNATED = 8
 
 SOLVER_NEWTON = 0
 SOLVER_NEWTON_DB = 1

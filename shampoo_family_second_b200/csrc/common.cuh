@@ -32,6 +32,7 @@ enum : int {
   DEV_FLAG_NONFINITE = 1,
   DEV_FLAG_NOT_CONVERGED = 2,
   DEV_FLAG_TIMEOUT = 4,
+  DEV_FLAG_STAGNATED = 8,
 };
 
 __device__ __forceinline__ void raise_flag(int* flags, int bit) {

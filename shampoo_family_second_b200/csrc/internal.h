@@ -157,8 +157,11 @@ int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const i
 // Second Newton-DB stage: Y0' = Y_par(i) (parity from iters), T0 = (3I - Y0')/2, Z1 = T0.
 int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters, int64_t batch, int n,
                               float* Ynew0, float* T, float* Z1, cudaStream_t st);
-int launch_check(float* res, int* done, int* iters, const int* valid, int64_t batch, int n, float tol, int it,
-                 int* flags, cudaStream_t st);
+// Residual check after iteration `it`: converged (done = 1) when the residual
+// is at most tol; stagnated (done = 2) when, from iteration kmin on, it failed
+// to improve on the previous iteration's (kept in prev) by a relative 1e-3.
+int launch_check(float* res, float* prev, int* done, int* iters, const int* valid, int64_t batch, int n, float tol,
+                 int it, int kmin, int* flags, cudaStream_t st);
 int launch_finalize(const float* X0, const float* X1, const int* iters, int default_iters, const float* sc,
                     int64_t batch, int n, float* out, int* flags, cudaStream_t st);
 int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int degree,

@@ -169,10 +169,17 @@ __global__ void db_stage2_kernel(const float* Y0, const float* Y1, const int* __
   Z1[i * nn + idx] = t;
 }
 
-// Residual check after iteration `it`: |tr(I - acc)| / valid <= tol marks the
-// matrix done (its later GEMM tiles are skipped).
-__global__ void check_kernel(float* res, int* done, int* iters, const int* valid, int batch, int n, float tol,
-                             int it, int* flags) {
+// Residual check after iteration `it`: r = |tr(I - acc)| / valid.
+//   r <= tol                        done = 1 (converged);
+//   it >= kmin, r >= (1 - 1e-3) r'  done = 2 (stagnated; r' = previous r).
+// Both iterations lift an eigenvalue mu << 1 of M by a fixed factor per
+// iteration (((p+1)/p)^p for coupled Newton, 9/4 for the square-root
+// iteration), so by iteration kmin every eigenvalue above fp32 resolution
+// (2^-24) has converged in exact arithmetic; a residual that no longer falls
+// from there on is held up by rounding, and more iterations cannot lower it.
+// A finished matrix's later GEMM tiles are skipped.
+__global__ void check_kernel(float* res, float* prev, int* done, int* iters, const int* valid, int batch, int n,
+                             float tol, int it, int kmin, int* flags) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= batch) return;
   if (done[i]) {
@@ -188,7 +195,11 @@ __global__ void check_kernel(float* res, int* done, int* iters, const int* valid
     raise_flag(flags, DEV_FLAG_NONFINITE);
   } else if (r <= tol) {
     done[i] = 1;
+  } else if (it >= kmin && r >= 0.999f * prev[i]) {
+    done[i] = 2;
+    raise_flag(flags, DEV_FLAG_STAGNATED);
   }
+  prev[i] = r;
 }
 
 // Output pass: X = sym(final iterate) * s^{-1/p}, with sym(Y) = (Y + Y^T)/2.
@@ -344,12 +355,12 @@ int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters
   return check_cuda(cudaGetLastError(), "db_stage2_kernel");
 }
 
-int launch_check(float* res, int* done, int* iters, const int* valid, int64_t batch, int n, float tol, int it,
-                 int* flags, cudaStream_t st) {
+int launch_check(float* res, float* prev, int* done, int* iters, const int* valid, int64_t batch, int n, float tol,
+                 int it, int kmin, int* flags, cudaStream_t st) {
   if (batch == 0) return 0;
-  ProfScope ps(K_CHECK, st, 0.0, 16.0 * batch);
-  check_kernel<<<static_cast<unsigned>((batch + 255) / 256), 256, 0, st>>>(res, done, iters, valid,
-                                                                           static_cast<int>(batch), n, tol, it, flags);
+  ProfScope ps(K_CHECK, st, 0.0, 24.0 * batch);
+  check_kernel<<<static_cast<unsigned>((batch + 255) / 256), 256, 0, st>>>(
+      res, prev, done, iters, valid, static_cast<int>(batch), n, tol, it, kmin, flags);
   count_launch();
   return check_cuda(cudaGetLastError(), "check_kernel");
 }
@@ -394,15 +405,18 @@ namespace shampoo {
 namespace {
 
 // Per-matrix iteration report: out[i] = iterations (+ add[i]); negated when
-// the residual never reached tol (and DEV_FLAG_NOT_CONVERGED is raised).
+// the residual never reached tol: the cap was reached (done 0, raises
+// DEV_FLAG_NOT_CONVERGED) or the residual stagnated (done 2, flagged by the
+// check).
 __global__ void report_kernel(const int* iters, const int* add, const int* done, int batch, int default_iters,
                               int* out, int* flags, int residual) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= batch) return;
   int it = iters ? iters[i] : default_iters;
   if (add) it += add[i];
-  const bool failed = residual && done && !done[i];
-  if (failed) raise_flag(flags, DEV_FLAG_NOT_CONVERGED);
+  const bool capped = residual && done && done[i] == 0;
+  const bool failed = residual && done && done[i] != 1;
+  if (capped) raise_flag(flags, DEV_FLAG_NOT_CONVERGED);
   if (out) out[i] = failed ? -it : it;
 }
 

@@ -50,13 +50,22 @@ int stacks_for(int solver) { return solver == 0 ? 7 : (solver == 1 ? 5 : 4); }
 
 constexpr size_t kAlign = 256;
 constexpr size_t kHeader = 64 * 1024;  // covers the alignment padding of the arrays
-constexpr int kVecInts = 6;            // s sc res done iters iters1
+constexpr int kVecInts = 7;            // s sc res prev done iters iters1
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// First iteration at which a stalled residual counts as stagnation: an
+// eigenvalue mu of M (scaled input 2^-24 <= mu << 1) grows by ((p+1)/p)^p per
+// coupled-Newton iteration (2.44 at p = 4, 2.25 at p = 2) and by 9/4 per
+// square-root iteration, reaching 1/2 within 18 (resp. 20) iterations; a few
+// quadratic steps and a margin give the values below.
+int kmin_newton(int p) { return p == 4 ? 24 : 26; }
+constexpr int kKminSqrt = 26;
 
 struct Layout {
   float* s;
   float* sc;
   float* res;
+  float* prev;
   int* done;
   int* iters;
   int* iters1;
@@ -76,6 +85,7 @@ Layout carve(void* base, int64_t cb, int n, int solver) {
   L.s = reinterpret_cast<float*>(take(cb * 4));
   L.sc = reinterpret_cast<float*>(take(cb * 4));
   L.res = reinterpret_cast<float*>(take(cb * 4));
+  L.prev = reinterpret_cast<float*>(take(cb * 4));
   L.done = reinterpret_cast<int*>(take(cb * 4));
   L.iters = reinterpret_cast<int*>(take(cb * 4));
   L.iters1 = reinterpret_cast<int*>(take(cb * 4));
@@ -119,6 +129,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
     if (residual) {
       if ((rc = check_cuda(cudaMemsetAsync(S.done, 0, cb * 4, st), "memset done"))) return rc;
       if ((rc = check_cuda(cudaMemsetAsync(S.res, 0, cb * 4, st), "memset res"))) return rc;
+      if ((rc = check_cuda(cudaMemsetAsync(S.prev, 0, cb * 4, st), "memset prev"))) return rc;
     }
     const int* skip = residual ? S.done : nullptr;
     auto common = [&](Epilogue& e) {
@@ -171,7 +182,8 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
           if ((rc = b.launch(st))) return rc;
         }
         if (residual &&
-            (rc = launch_check(S.res, S.done, S.iters, valid, cb, n, job.tol, j + 1, job.flags, st)))
+            (rc = launch_check(S.res, S.prev, S.done, S.iters, valid, cb, n, job.tol, j + 1, kmin_newton(p),
+                               job.flags, st)))
           return rc;
       }
       if ((rc = launch_finalize(X[0].base, X[1].base, residual ? S.iters : nullptr, job.iters, S.sc, cb, n, out,
@@ -200,6 +212,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
               return rc;
             if ((rc = check_cuda(cudaMemsetAsync(S.done, 0, cb * 4, st), "memset done"))) return rc;
             if ((rc = check_cuda(cudaMemsetAsync(S.res, 0, cb * 4, st), "memset res"))) return rc;
+            if ((rc = check_cuda(cudaMemsetAsync(S.prev, 0, cb * 4, st), "memset prev"))) return rc;
           } else {
             if ((rc = launch_fill_iters(S.iters1, cb, job.iters, st))) return rc;
           }
@@ -233,7 +246,8 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
             if ((rc = b.launch(st))) return rc;
           }
           if (residual &&
-              (rc = launch_check(S.res, S.done, S.iters, valid, cb, n, job.tol, j + 1, job.flags, st)))
+              (rc = launch_check(S.res, S.prev, S.done, S.iters, valid, cb, n, job.tol, j + 1, kKminSqrt, job.flags,
+                                 st)))
             return rc;
         }
       }

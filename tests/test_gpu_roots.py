@@ -90,6 +90,25 @@ def test_not_converged_flag(sb):
     assert np.all(it == -2)
 
 
+@pytest.mark.parametrize("solver,kmin", [(0, 24), (1, 26)])
+def test_stagnation_stops_before_the_cap(sb, solver, kmin):
+    """tol = 1e-9 is below what fp32 iterates can reach (their fixed point
+    sits near 1e-6), so the residual stalls: the solver must stop each matrix
+    once the residual no longer improves (from iteration kmin on), flag
+    STAGNATED rather than NOT_CONVERGED, report a negative count below the
+    cap, and still return an accurate root."""
+    A32 = workloads.spd_batch(3, 128, 1e2, seed=31).astype(np.float32)
+    cap = 80
+    X, it, st = run(sb, A32, p=4, eps=0.0, solver=solver, iters=cap, tol=1e-9)
+    assert st & sb.DEVFLAG_STAGNATED
+    assert not st & sb.DEVFLAG_NOT_CONVERGED
+    total_cap = 2 * cap if solver == 1 else cap
+    assert np.all(it < 0) and np.all(-it >= kmin) and np.all(-it < total_cap), it
+    for b in range(3):
+        ref = oracle.inverse_root(A32[b].astype(np.float64), 4, 0.0)
+        assert oracle.rel_fro(X[b], ref) < TOL
+
+
 def test_nonfinite_flag(sb):
     A32 = workloads.spd_batch(2, 64, 1e2, seed=14).astype(np.float32)
     A32[1, 3, 5] = np.nan

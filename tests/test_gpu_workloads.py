@@ -75,7 +75,8 @@ def run_workload(sb, wl, steps, k_blocks):
         del G
     assert all(torch.isfinite(w).all().item() for w in W)
     status = opt.status()
-    assert status & ~sb.DEVFLAG_NOT_CONVERGED == 0, status
+    # rank-deficient ragged blocks stall at the fp32 floor (STAGNATED)
+    assert status & ~(sb.DEVFLAG_NOT_CONVERGED | sb.DEVFLAG_STAGNATED) == 0, status
     print(f"\n{wl.name}: {len(blocks)} sampled blocks x {steps} steps; worst update error "
           f"{max(r[2] for r in report):.2e} (tightest gate {min(r[3] for r in report):.2e}), "
           f"worst statistics error {max(r[4] for r in report):.2e}, device status {status}")
