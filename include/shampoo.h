@@ -246,7 +246,10 @@ SHAMPOO_API void shampoo_profile_enable(int32_t on);
 SHAMPOO_API void shampoo_profile_reset(void);
 SHAMPOO_API int shampoo_profile_read(int32_t kind, int64_t* launches, double* total_ms, double* alg_flops, double* alg_bytes);
 
-/* Number of kernels this library has launched in this process. */
+/* Number of kernels this library has launched in this process, including
+ * the kernels that residual-checked solver loops ran inside CUDA graphs
+ * (counted on the device; once such a loop has run, this call waits for the
+ * device). */
 SHAMPOO_API uint64_t shampoo_launch_count(void);
 
 #ifdef __cplusplus

@@ -101,6 +101,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// mbar_wait_bounded for a whole warp: lane 0 polls the barrier and the warp
+// synchronises on it (bar.warp.sync orders lane 0's acquire before the other
+// lanes' later accesses), so a waiting warp costs one shared-memory poll
+// instead of 32.  Returns the wait's outcome on every lane.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* flags, volatile int* abort) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, flags, abort) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }

@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&conv[s], CONV_THREADS);
+      mbar_init(&conv[s], CONV_WARPS);
       mbar_init(&empty[s], 1);
     }
 #pragma unroll
@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
         for (int kc = 0; kc < nk; ++kc, ++it) {
           const int s = it % STAGES;
-          if (!mbar_wait_bounded(&full[s], (it / STAGES) & 1, flags, abort_flag)) {
+          if (!mbar_wait_warp(&full[s], (it / STAGES) & 1, flags, abort_flag)) {
             ok = false;
             break;
           }
@@ -371,8 +371,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             *reinterpret_cast<float4*>(base + off) = h;
             *reinterpret_cast<float4*>(base + RAW_BYTES + off) = l;
           }
+          // Each lane orders its stores before the tensor core's reads; the
+          // warp then reports once.
           fence_proxy_async_shared();
-          mbar_arrive(&conv[s]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&conv[s]);
         }
       }
     }
@@ -400,7 +403,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
       for (int seg = 0; seg < nseg; ++seg, ++sg) {
         const uint32_t b = sg & 1;
-        if (!mbar_wait_bounded(&acc_full[b], (sg >> 1) & 1, flags, abort_flag)) {
+        if (!mbar_wait_warp(&acc_full[b], (sg >> 1) & 1, flags, abort_flag)) {
           ok = false;
           break;
         }

@@ -107,6 +107,13 @@ struct ProfScope {
   int ev;
 };
 void count_launch();
+// While alive, this thread's launches are being recorded into a graph (not
+// counted as launches; the graph's own execution is counted on the device).
+struct CaptureScope {
+  CaptureScope();
+  ~CaptureScope();
+};
+void note_graph_loop_launch();  // a graph loop ran: shampoo_launch_count adds its device-side count
 bool profiling_enabled();
 double* device_flop_slots();  // device address of the executed-flop accumulators
 
@@ -157,11 +164,20 @@ int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const i
 // Second Newton-DB stage: Y0' = Y_par(i) (parity from iters), T0 = (3I - Y0')/2, Z1 = T0.
 int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters, int64_t batch, int n,
                               float* Ynew0, float* T, float* Z1, cudaStream_t st);
-// Residual check after iteration `it`: converged (done = 1) when the residual
-// is at most tol; stagnated (done = 2) when, from iteration kmin on, it failed
-// to improve on the previous iteration's (kept in prev) by a relative 1e-3.
+// A residual-checked iteration loop captured as a CUDA graph WHILE node: the
+// check kernel of each pass sets the loop condition.
+struct GraphLoop {
+  cudaGraphConditionalHandle cond;
+  int kernels_per_check;  // kernels of one iteration (the check's own included)
+};
+// Residual check after an iteration (one CTA): it = *counter + 1; converged
+// (done = 1) when the residual is at most tol; stagnated (done = 2) when, from
+// iteration kmin on, it failed to improve on the previous one (kept in prev)
+// by a relative 1e-3; capped (done = 3) at it = cap.  Inside a graph loop
+// (loop != NULL) it also sets the loop condition.
 int launch_check(float* res, float* prev, int* done, int* iters, const int* valid, int64_t batch, int n, float tol,
-                 int it, int kmin, int* flags, cudaStream_t st);
+                 int* counter, int cap, int kmin, int* flags, const GraphLoop* loop, cudaStream_t st);
+uint64_t graph_kernel_count();  // kernels run inside graph loops so far (synchronous read)
 int launch_finalize(const float* X0, const float* X1, const int* iters, int default_iters, const float* sc,
                     int64_t batch, int n, float* out, int* flags, cudaStream_t st);
 int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int degree,

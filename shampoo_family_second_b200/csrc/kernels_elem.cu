@@ -9,6 +9,17 @@
 #include "internal.h"
 
 namespace shampoo {
+
+// Kernels executed inside graph loops (added by the loop's check kernel once
+// per pass); read by shampoo_launch_count.
+__device__ unsigned long long g_graph_kernels = 0;
+
+uint64_t graph_kernel_count() {
+  unsigned long long v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_graph_kernels, sizeof(v)) != cudaSuccess) return 0;
+  return v;
+}
+
 namespace {
 
 __device__ __forceinline__ float load_grad(const void* g, size_t idx, int dtype) {
@@ -169,37 +180,65 @@ __global__ void db_stage2_kernel(const float* Y0, const float* Y1, const int* __
   Z1[i * nn + idx] = t;
 }
 
-// Residual check after iteration `it`: r = |tr(I - acc)| / valid.
+// Residual check after an iteration, one CTA for the whole batch.  The
+// iteration number is it = counter[0] + 1 (counter[0] then holds it, and
+// counter[1] the number of matrices still active).  For an
+// active matrix with r = |tr(I - acc)| / valid:
 //   r <= tol                        done = 1 (converged);
-//   it >= kmin, r >= (1 - 1e-3) r'  done = 2 (stagnated; r' = previous r).
+//   it >= kmin, r >= (1 - 1e-3) r'  done = 2 (stagnated; r' = previous r);
+//   it >= cap                       done = 3 (iteration cap reached).
 // Both iterations lift an eigenvalue mu << 1 of M by a fixed factor per
 // iteration (((p+1)/p)^p for coupled Newton, 9/4 for the square-root
 // iteration), so by iteration kmin every eigenvalue above fp32 resolution
 // (2^-24) has converged in exact arithmetic; a residual that no longer falls
 // from there on is held up by rounding, and more iterations cannot lower it.
-// A finished matrix's later GEMM tiles are skipped.
-__global__ void check_kernel(float* res, float* prev, int* done, int* iters, const int* valid, int batch, int n,
-                             float tol, int it, int kmin, int* flags) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= batch) return;
-  if (done[i]) {
+// A finished matrix's later GEMM tiles are skipped.  Inside a graph loop
+// (set_cond) the loop condition becomes "some matrix still active", and
+// graph_kernels (the kernels of one iteration) is added to the device-side
+// launch count.
+__global__ void __launch_bounds__(1024) check_kernel(float* res, float* prev, int* done, int* iters,
+                                                     const int* valid, int batch, int n, float tol, int* counter,
+                                                     int cap, int kmin, int* flags, cudaGraphConditionalHandle cond,
+                                                     int set_cond, int graph_kernels) {
+  __shared__ int active;
+  if (threadIdx.x == 0) active = 0;
+  __syncthreads();
+  const int it = *counter + 1;
+  int mine = 0;
+  for (int i = threadIdx.x; i < batch; i += blockDim.x) {
+    if (done[i]) {
+      res[i] = 0.f;
+      continue;
+    }
+    const int v = valid ? valid[i] : n;
+    const float r = fabsf(res[i]) / static_cast<float>(v);
     res[i] = 0.f;
-    return;
+    iters[i] = it;
+    if (!isfinite(r)) {
+      done[i] = 1;
+      raise_flag(flags, DEV_FLAG_NONFINITE);
+    } else if (r <= tol) {
+      done[i] = 1;
+    } else if (it >= kmin && r >= 0.999f * prev[i]) {
+      done[i] = 2;
+      raise_flag(flags, DEV_FLAG_STAGNATED);
+    } else if (it >= cap) {
+      done[i] = 3;
+    } else {
+      ++mine;
+    }
+    prev[i] = r;
   }
-  const int v = valid ? valid[i] : n;
-  const float r = fabsf(res[i]) / static_cast<float>(v);
-  res[i] = 0.f;
-  iters[i] = it;
-  if (!isfinite(r)) {
-    done[i] = 1;
-    raise_flag(flags, DEV_FLAG_NONFINITE);
-  } else if (r <= tol) {
-    done[i] = 1;
-  } else if (it >= kmin && r >= 0.999f * prev[i]) {
-    done[i] = 2;
-    raise_flag(flags, DEV_FLAG_STAGNATED);
+  if (mine) atomicAdd(&active, mine);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    counter[0] = it;
+    counter[1] = active;
+    if (set_cond) {
+      cudaGraphSetConditional(cond, active > 0 ? 1u : 0u);
+      atomicAdd(&g_graph_kernels, static_cast<unsigned long long>(graph_kernels));
+    }
   }
-  prev[i] = r;
 }
 
 // Output pass: X = sym(final iterate) * s^{-1/p}, with sym(Y) = (Y + Y^T)/2.
@@ -356,11 +395,12 @@ int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters
 }
 
 int launch_check(float* res, float* prev, int* done, int* iters, const int* valid, int64_t batch, int n, float tol,
-                 int it, int kmin, int* flags, cudaStream_t st) {
+                 int* counter, int cap, int kmin, int* flags, const GraphLoop* loop, cudaStream_t st) {
   if (batch == 0) return 0;
   ProfScope ps(K_CHECK, st, 0.0, 24.0 * batch);
-  check_kernel<<<static_cast<unsigned>((batch + 255) / 256), 256, 0, st>>>(
-      res, prev, done, iters, valid, static_cast<int>(batch), n, tol, it, kmin, flags);
+  check_kernel<<<1, 1024, 0, st>>>(res, prev, done, iters, valid, static_cast<int>(batch), n, tol, counter, cap,
+                                   kmin, flags, loop ? loop->cond : cudaGraphConditionalHandle(0), loop ? 1 : 0,
+                                   loop ? loop->kernels_per_check : 0);
   count_launch();
   return check_cuda(cudaGetLastError(), "check_kernel");
 }
@@ -405,7 +445,7 @@ namespace shampoo {
 namespace {
 
 // Per-matrix iteration report: out[i] = iterations (+ add[i]); negated when
-// the residual never reached tol: the cap was reached (done 0, raises
+// the residual never reached tol: the cap was reached (done 0 or 3, raises
 // DEV_FLAG_NOT_CONVERGED) or the residual stagnated (done 2, flagged by the
 // check).
 __global__ void report_kernel(const int* iters, const int* add, const int* done, int batch, int default_iters,
@@ -414,7 +454,7 @@ __global__ void report_kernel(const int* iters, const int* add, const int* done,
   if (i >= batch) return;
   int it = iters ? iters[i] : default_iters;
   if (add) it += add[i];
-  const bool capped = residual && done && done[i] == 0;
+  const bool capped = residual && done && (done[i] == 0 || done[i] == 3);
   const bool failed = residual && done && done[i] != 1;
   if (capped) raise_flag(flags, DEV_FLAG_NOT_CONVERGED);
   if (out) out[i] = failed ? -it : it;

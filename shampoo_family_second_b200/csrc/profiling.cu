@@ -63,7 +63,20 @@ int check_cuda(cudaError_t e, const char* what) {
   return set_error(SHAMPOO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+namespace {
+thread_local int t_capturing = 0;  // > 0 while this thread records launches into a graph
+}
+CaptureScope::CaptureScope() { ++t_capturing; }
+CaptureScope::~CaptureScope() { --t_capturing; }
+
+void count_launch() {
+  if (t_capturing == 0) g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+namespace {
+std::atomic<bool> g_graph_loops_used{false};
+}
+void note_graph_loop_launch() { g_graph_loops_used.store(true, std::memory_order_relaxed); }
 bool profiling_enabled() { return g_enabled.load(std::memory_order_relaxed); }
 
 double* device_flop_slots() {
@@ -103,7 +116,11 @@ extern "C" {
 
 const char* shampoo_last_error(void) { return g_last_error.c_str(); }
 
-uint64_t shampoo_launch_count(void) { return g_launches.load(); }
+uint64_t shampoo_launch_count(void) {
+  // Host-issued launches, plus the kernels graph loops ran on the device
+  // (counted there; reading them waits for the device).
+  return g_launches.load() + (g_graph_loops_used.load() ? graph_kernel_count() : 0);
+}
 
 void shampoo_profile_enable(int32_t on) { g_enabled.store(on != 0); }
 

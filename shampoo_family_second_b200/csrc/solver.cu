@@ -33,6 +33,9 @@
 // exit at once); iters is then the cap.
 #include <algorithm>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
 #include <vector>
 
 #include "internal.h"
@@ -62,6 +65,7 @@ int kmin_newton(int p) { return p == 4 ? 24 : 26; }
 constexpr int kKminSqrt = 26;
 
 struct Layout {
+  int* counter;  // [0] iterations done, [1] matrices still active (written by the check kernel)
   float* s;
   float* sc;
   float* res;
@@ -82,6 +86,7 @@ Layout carve(void* base, int64_t cb, int n, int solver) {
     p += align_up(bytes);
     return r;
   };
+  L.counter = reinterpret_cast<int*>(take(8));
   L.s = reinterpret_cast<float*>(take(cb * 4));
   L.sc = reinterpret_cast<float*>(take(cb * 4));
   L.res = reinterpret_cast<float*>(take(cb * 4));
@@ -93,6 +98,151 @@ Layout carve(void* base, int64_t cb, int n, int solver) {
   for (int k = 0; k < stacks_for(solver); ++k)
     L.stack[k] = reinterpret_cast<float*>(take(plain_floats(cb, n) * 4));
   return L;
+}
+
+// ---------------------------------------------------------------------------
+// Residual-checked loops as CUDA graphs.  After iteration 0, the remaining
+// iterations run as one graph with a WHILE node; its body holds two
+// iterations (so the ping-pong buffers line up again after every pass) and
+// each body's check kernel sets the loop condition to "some matrix still
+// active".  The device ends the loop as soon as every matrix has converged,
+// stagnated or reached the cap, instead of the host launching the cap's worth
+// of iterations.  Executable graphs are cached by everything their kernels'
+// arguments depend on.
+// ---------------------------------------------------------------------------
+struct LoopKey {
+  int dev, solver, p, n, cap;
+  int64_t cb;
+  float tol;
+  const void* scratch;
+  const int* valid;
+  const int* flags;
+  bool operator<(const LoopKey& o) const {
+    return std::tie(dev, solver, p, n, cap, cb, tol, scratch, valid, flags) <
+           std::tie(o.dev, o.solver, o.p, o.n, o.cap, o.cb, o.tol, o.scratch, o.valid, o.flags);
+  }
+};
+
+struct LoopGraph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  uint64_t used = 0;
+};
+
+std::mutex g_loop_mu;
+std::map<LoopKey, LoopGraph> g_loops;
+uint64_t g_loop_clock = 0;
+bool g_loops_unavailable = false;  // a graph call failed once: plain launches from then on
+constexpr size_t kMaxLoopGraphs = 64;
+
+void destroy_loop(LoopGraph& g) {
+  if (g.exec) cudaGraphExecDestroy(g.exec);
+  if (g.graph) cudaGraphDestroy(g.graph);
+  g.exec = nullptr;
+  g.graph = nullptr;
+}
+
+// Graph loops are used unless profiling is on (per-launch events need plain
+// launches), the caller's stream is being captured, or graphs failed before.
+bool use_graph_loop(cudaStream_t st) {
+  if (profiling_enabled()) return false;
+  {
+    std::lock_guard<std::mutex> lk(g_loop_mu);
+    if (g_loops_unavailable) return false;
+  }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return cs == cudaStreamCaptureStatusNone;
+}
+
+// Builds the graph: one WHILE node whose body `body(capture_stream, loop)`
+// issues by stream capture.  Returns 0 or a CUDA error (nothing enqueued).
+template <class Body>
+int build_loop(LoopGraph& out, int kernels_per_iter, Body&& body) {
+  cudaGraph_t g = nullptr;
+  cudaStream_t cs = nullptr;
+  auto fail = [&](cudaError_t e, const char* what) {
+    if (cs) {
+      cudaGraph_t tmp = nullptr;
+      cudaStreamEndCapture(cs, &tmp);
+      cudaStreamDestroy(cs);
+    }
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    return set_error(-4, "graph loop: %s failed (%s)", what, cudaGetErrorString(e));
+  };
+  cudaError_t e = cudaGraphCreate(&g, 0);
+  if (e != cudaSuccess) return fail(e, "cudaGraphCreate");
+  cudaGraphConditionalHandle h;
+  e = cudaGraphConditionalHandleCreate(&h, g, 1, cudaGraphCondAssignDefault);
+  if (e != cudaSuccess) return fail(e, "cudaGraphConditionalHandleCreate");
+  cudaGraphNodeParams np = {cudaGraphNodeTypeConditional};
+  np.conditional.handle = h;
+  np.conditional.type = cudaGraphCondTypeWhile;
+  np.conditional.size = 1;
+  cudaGraphNode_t node;
+  e = cudaGraphAddNode(&node, g, nullptr, 0, &np);
+  if (e != cudaSuccess) return fail(e, "cudaGraphAddNode(while)");
+  cudaGraph_t bodyg = np.conditional.phGraph_out[0];
+  e = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return fail(e, "cudaStreamCreate");
+  e = cudaStreamBeginCaptureToGraph(cs, bodyg, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal);
+  if (e != cudaSuccess) return fail(e, "cudaStreamBeginCaptureToGraph");
+  GraphLoop loop{h, kernels_per_iter};
+  int rc;
+  {
+    CaptureScope capture;  // launches recorded here are not executed launches
+    rc = body(cs, &loop);
+  }
+  cudaGraph_t ended = nullptr;
+  e = cudaStreamEndCapture(cs, &ended);
+  cudaStreamDestroy(cs);
+  cs = nullptr;
+  if (rc) {
+    cudaGraphDestroy(g);
+    return rc;
+  }
+  if (e != cudaSuccess) return fail(e, "cudaStreamEndCapture");
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, g, 0);
+  if (e != cudaSuccess) return fail(e, "cudaGraphInstantiate");
+  out.graph = g;
+  out.exec = exec;
+  return 0;
+}
+
+// Runs the loop for `key` on st (building and caching its graph on first
+// use).  *done = false when graphs are unavailable (the caller then issues
+// the iterations itself; nothing was enqueued).
+template <class Body>
+int run_loop(const LoopKey& key, int kernels_per_iter, Body&& body, cudaStream_t st, bool* done) {
+  *done = false;
+  std::lock_guard<std::mutex> lk(g_loop_mu);
+  auto it = g_loops.find(key);
+  if (it == g_loops.end()) {
+    if (g_loops.size() >= kMaxLoopGraphs) {  // evict the least recently used
+      auto old = g_loops.begin();
+      for (auto i = g_loops.begin(); i != g_loops.end(); ++i)
+        if (i->second.used < old->second.used) old = i;
+      destroy_loop(old->second);
+      g_loops.erase(old);
+    }
+    LoopGraph lg;
+    if (build_loop(lg, kernels_per_iter, body)) {
+      g_loops_unavailable = true;
+      return 0;
+    }
+    it = g_loops.emplace(key, lg).first;
+  }
+  it->second.used = ++g_loop_clock;
+  int rc = check_cuda(cudaGraphLaunch(it->second.exec, st), "cudaGraphLaunch(solver loop)");
+  if (rc) return rc;
+  note_graph_loop_launch();
+  *done = true;
+  return 0;
 }
 
 }  // namespace
@@ -130,8 +280,44 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       if ((rc = check_cuda(cudaMemsetAsync(S.done, 0, cb * 4, st), "memset done"))) return rc;
       if ((rc = check_cuda(cudaMemsetAsync(S.res, 0, cb * 4, st), "memset res"))) return rc;
       if ((rc = check_cuda(cudaMemsetAsync(S.prev, 0, cb * 4, st), "memset prev"))) return rc;
+      if ((rc = check_cuda(cudaMemsetAsync(S.counter, 0, 8, st), "memset counter"))) return rc;
     }
     const int* skip = residual ? S.done : nullptr;
+    int dev = 0;
+    if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+    const LoopKey key{dev, job.solver, p, n, job.iters, cb, job.tol, scratch, valid, job.flags};
+    // Iterations 1.. of a residual-checked loop: one graph with a WHILE node
+    // when available, else plain launches up to the cap.
+    auto run_rest = [&](auto&& iterate, int kernels_per_iter) -> int {
+      if (job.iters <= 1) return 0;
+      if (use_graph_loop(st)) {
+        bool ran = false;
+        int r = run_loop(key, kernels_per_iter,
+                         [&](cudaStream_t cs, const GraphLoop* lp) {
+                           int q = iterate(1, cs, lp);
+                           return q ? q : iterate(2, cs, lp);
+                         },
+                         st, &ran);
+        if (r || ran) return r;
+      }
+      // Plain launches.  With profiling on (per-launch events) the host reads
+      // the active count after each iteration and stops where the device loop
+      // would, so that the profile covers the same kernels as a graph run.
+      const bool follow = profiling_enabled();
+      for (int j = 1; j < job.iters; ++j) {
+        int r = iterate(j, st, nullptr);
+        if (r) return r;
+        if (follow) {
+          int active = 0;
+          if ((r = check_cuda(cudaMemcpyAsync(&active, S.counter + 1, 4, cudaMemcpyDeviceToHost, st),
+                              "read active count")) ||
+              (r = check_cuda(cudaStreamSynchronize(st), "profiling sync")))
+            return r;
+          if (active == 0) break;
+        }
+      }
+      return 0;
+    };
     auto common = [&](Epilogue& e) {
       e.skip = skip;
       e.flags = job.flags;
@@ -146,7 +332,9 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       StackMaps& T4 = sm[6];
       if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, M[0].base, T.base, X[1].base, st)))
         return rc;
-      for (int j = 0; j < job.iters; ++j) {
+      // One iteration j on stream cs (inside a graph loop when lp != NULL).
+      auto iterate = [&](int j, cudaStream_t cs, const GraphLoop* lp) -> int {
+        int r;
         {
           Builder b;
           Epilogue& e = b.add(cbi, n, T, 0, T, 0, f1, NEWTON_B);  // T2 = T T
@@ -157,16 +345,16 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
             ex.D = X[(j + 1) & 1].base;
             common(ex);
           }
-          if ((rc = b.launch(st))) return rc;
+          if ((r = b.launch(cs))) return r;
         }
-        if (!residual && j == job.iters - 1) break;
+        if (!residual && j == job.iters - 1) return 0;
         StackMaps* P = &T2;
         if (p == 4) {
           Builder b;
           Epilogue& e = b.add(cbi, n, T2, 0, T2, 0, f1, NEWTON_B);  // T4 = T2 T2
           e.D = T4.base;
           common(e);
-          if ((rc = b.launch(st))) return rc;
+          if ((r = b.launch(cs))) return r;
           P = &T4;
         }
         {
@@ -179,12 +367,18 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
           e.res = residual ? S.res : nullptr;
           e.valid = valid;
           common(e);
-          if ((rc = b.launch(st))) return rc;
+          if ((r = b.launch(cs))) return r;
         }
-        if (residual &&
-            (rc = launch_check(S.res, S.prev, S.done, S.iters, valid, cb, n, job.tol, j + 1, kmin_newton(p),
-                               job.flags, st)))
-          return rc;
+        if (residual)
+          return launch_check(S.res, S.prev, S.done, S.iters, valid, cb, n, job.tol, S.counter, job.iters,
+                              kmin_newton(p), job.flags, lp, cs);
+        return 0;
+      };
+      if (residual) {
+        if ((rc = iterate(0, st, nullptr)) || (rc = run_rest(iterate, p == 4 ? 4 : 3))) return rc;
+      } else {
+        for (int j = 0; j < job.iters; ++j)
+          if ((rc = iterate(j, st, nullptr))) return rc;
       }
       if ((rc = launch_finalize(X[0].base, X[1].base, residual ? S.iters : nullptr, job.iters, S.sc, cb, n, out,
                                 job.flags, st)))
@@ -213,6 +407,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
             if ((rc = check_cuda(cudaMemsetAsync(S.done, 0, cb * 4, st), "memset done"))) return rc;
             if ((rc = check_cuda(cudaMemsetAsync(S.res, 0, cb * 4, st), "memset res"))) return rc;
             if ((rc = check_cuda(cudaMemsetAsync(S.prev, 0, cb * 4, st), "memset prev"))) return rc;
+            if ((rc = check_cuda(cudaMemsetAsync(S.counter, 0, 8, st), "memset counter"))) return rc;
           } else {
             if ((rc = launch_fill_iters(S.iters1, cb, job.iters, st))) return rc;
           }
@@ -220,7 +415,8 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
                                               st)))
             return rc;
         }
-        for (int j = 0; j < job.iters; ++j) {
+        auto iterate = [&](int j, cudaStream_t cs, const GraphLoop* lp) -> int {
+          int r;
           {
             Builder b;
             Epilogue& ey = b.add(cbi, n, Y[j & 1], 0, T, 0, f1, B_MN_MAJOR);  // Y <- Y T
@@ -231,9 +427,9 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
               ez.D = Z[(j + 1) & 1].base;
               common(ez);
             }
-            if ((rc = b.launch(st))) return rc;
+            if ((r = b.launch(cs))) return r;
           }
-          if (!residual && j == job.iters - 1) break;
+          if (!residual && j == job.iters - 1) return 0;
           {
             Builder b;
             Epilogue& e = b.add(cbi, n, Z[(j + 1) & 1], 0, Y[(j + 1) & 1], 0, f1, B_MN_MAJOR);  // T = (3I - Z Y)/2
@@ -243,12 +439,18 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
             e.res = residual ? S.res : nullptr;
             e.valid = valid;
             common(e);
-            if ((rc = b.launch(st))) return rc;
+            if ((r = b.launch(cs))) return r;
           }
-          if (residual &&
-              (rc = launch_check(S.res, S.prev, S.done, S.iters, valid, cb, n, job.tol, j + 1, kKminSqrt, job.flags,
-                                 st)))
-            return rc;
+          if (residual)
+            return launch_check(S.res, S.prev, S.done, S.iters, valid, cb, n, job.tol, S.counter, job.iters,
+                                kKminSqrt, job.flags, lp, cs);
+          return 0;
+        };
+        if (residual) {
+          if ((rc = iterate(0, st, nullptr)) || (rc = run_rest(iterate, 3))) return rc;
+        } else {
+          for (int j = 0; j < job.iters; ++j)
+            if ((rc = iterate(j, st, nullptr))) return rc;
         }
       }
       if ((rc = launch_finalize(Z[0].base, Z[1].base, residual ? S.iters : nullptr, job.iters, S.sc, cb, n, out,

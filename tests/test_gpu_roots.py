@@ -115,3 +115,30 @@ def test_nonfinite_flag(sb):
     X, it, st = run(sb, A32, p=4, eps=0.0, solver=sb.SOLVER_NEWTON, iters=5, tol=0.0)
     assert st & sb.DEVFLAG_NONFINITE
     assert np.all(np.isfinite(X[0]))
+
+
+@pytest.mark.parametrize("solver,per_iter", [(0, 4), (1, 3)])
+def test_graph_loop_matches_plain_launches(sb, solver, per_iter):
+    """Residual-checked iterations after the first run as a CUDA graph loop
+    that the device ends once every matrix is finished.  With profiling on
+    (per-launch events) the host issues the iterations one by one up to the
+    cap instead.  Both must give bit-identical roots and iteration counts, and
+    the graph loop must run about the iterations needed, not the cap's worth."""
+    A32 = workloads.spd_batch(6, 256, 1e3, seed=41).astype(np.float32)
+    kw = dict(p=4, eps=1e-6, solver=solver, iters=60, tol=1e-5)
+    sb.profile_enable(True)
+    try:
+        X1, it1, st1 = run(sb, A32, **kw)
+    finally:
+        sb.profile_enable(False)
+    n0 = sb.launch_count()
+    X2, it2, st2 = run(sb, A32, **kw)
+    n1 = sb.launch_count()
+    assert st1 == st2 == 0
+    assert np.array_equal(it1, it2)
+    assert np.array_equal(X1, X2)
+    stages = 2 if solver == 1 else 1
+    needed = int(np.max(it2))  # both stages for Newton-DB p = 4
+    # prologue, norm, finalize, report and per stage one extra loop pass at most
+    assert n1 - n0 <= 8 + per_iter * (needed + 2 * stages), (n1 - n0, needed)
+    assert n1 - n0 < per_iter * 60 * stages
