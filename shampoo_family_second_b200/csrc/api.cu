@@ -267,6 +267,8 @@ int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d
     args.g[i] = d_grads[i];
     args.w[i] = d_weights[i];
     args.ld[i] = static_cast<int>(h->cols[i]);
+    const size_t esize = c.grad_dtype == SHAMPOO_BF16 ? 2 : 4;
+    args.vec[i] = (h->cols[i] % 4 == 0 && reinterpret_cast<uintptr_t>(d_grads[i]) % (4 * esize) == 0) ? 1 : 0;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;

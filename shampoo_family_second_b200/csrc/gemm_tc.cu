@@ -201,6 +201,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int lane = threadIdx.x & 31;
   const int total = L.total_tiles;
   int* flags = L.g[0].ep.flags;
+  pdl_launch_dependents();  // the next launch may take the SMs this one frees
 
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -226,6 +227,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t taddr = *tmem_slot;
+  // Everything above overlaps the previous kernel; every global access below
+  // (operands, outputs, skip flags) waits for it to complete.
+  pdl_wait_prerequisites();
 
   if (warp < EPI_WARP0) {
     // Warps 0-7 (two whole warpgroups) run the light roles; each warpgroup
@@ -578,7 +582,22 @@ int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
   L.prof_slot = K_GEMM;
   const unsigned grid = static_cast<unsigned>(total < sms ? total : sms);
   ProfScope ps(K_GEMM, st, flops, 0.0);
-  gemm3x_tf32_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(L, maps, device_flop_slots());
+  // Programmatic stream serialization: the launch may begin (prologue only)
+  // while the previous kernel finishes; the kernel waits for it before any
+  // global access.
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  rc = check_cuda(cudaLaunchKernelEx(&cfg, gemm3x_tf32_kernel, L, maps, device_flop_slots()),
+                  "gemm3x_tf32_kernel launch");
+  if (rc) return rc;
   count_launch();
   return check_cuda(cudaGetLastError(), "gemm3x_tf32_kernel launch");
 }

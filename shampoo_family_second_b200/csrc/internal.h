@@ -151,6 +151,7 @@ struct StackArgs {
   const void* g[kMaxParams];
   float* w[kMaxParams];
   int ld[kMaxParams];
+  unsigned char vec[kMaxParams];  // rows of param i start 16-byte (fp32) / 8-byte (bf16) aligned
 };
 int launch_stack(const StackArgs& args, const int* d_table, int nb, int B, int grad_dtype, float* Gs, float* Gts,
                  float** blk_wptr, int* blk_ld, cudaStream_t st, double alg_bytes);

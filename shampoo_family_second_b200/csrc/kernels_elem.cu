@@ -35,38 +35,75 @@ __device__ __forceinline__ float load_grad(const void* g, size_t idx, int dtype)
 // tensors.  Block b of the table {param, row0, col0, r, c} is copied from the
 // row-major gradient into Gs[b] (B x B) and its transpose into Gt[b],
 // zero-padded beyond (r, c).  Also records where the block's weights live.
-// grid (B/32, B/32, nb), block (32, 8).
+// grid (ceil(B/128), B/32, nb), block (32, 8): a CTA moves a 32 x 128 piece.
+// Each thread loads 4 x 4 consecutive values (16-byte loads when the row is
+// aligned), writes them to Gs directly and through a shared-memory tile to
+// Gt; the tile's row stride (132 floats) keeps the 16-byte stores aligned.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ float4 load_grad4(const void* g, size_t idx, int dtype, bool vec, int valid_cols) {
+  // Values idx .. idx+3 of one row; columns beyond valid_cols read as 0.
+  if (vec && valid_cols >= 4) {
+    if (dtype == 1) {
+      const uint2 u = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(g) + idx);
+      return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                         __uint_as_float(u.y & 0xFFFF0000u));
+    }
+    return *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(g) + idx);
+  }
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (valid_cols > 0) v.x = load_grad(g, idx + 0, dtype);
+  if (valid_cols > 1) v.y = load_grad(g, idx + 1, dtype);
+  if (valid_cols > 2) v.z = load_grad(g, idx + 2, dtype);
+  if (valid_cols > 3) v.w = load_grad(g, idx + 3, dtype);
+  return v;
+}
+
 __global__ void stack_blocks_kernel(const __grid_constant__ StackArgs args, const int* __restrict__ table, int B,
-                                   int dtype, float* __restrict__ Gs, float* __restrict__ Gt, float** blk_wptr,
-                                   int* blk_ld) {
-  __shared__ float tile[32][33];
+                                    int dtype, float* __restrict__ Gs, float* __restrict__ Gt, float** blk_wptr,
+                                    int* blk_ld) {
+  pdl_launch_dependents();  // a following GEMM may start its prologue
+  constexpr int TC = 128, STRIDE = TC + 4;
+  __shared__ __align__(16) float tile[32 * STRIDE];
   const int b = blockIdx.z;
-  const int bi = blockIdx.y, bj = blockIdx.x;
+  const int r0 = blockIdx.y * 32;      // first row of the piece (block coordinates)
+  const int c0 = blockIdx.x * TC;      // first column
   const int tx = threadIdx.x, ty = threadIdx.y;
+  const int t = ty * 32 + tx;
   const int param = table[5 * b + 0];
   const int row0 = table[5 * b + 1], col0 = table[5 * b + 2];
   const int r = table[5 * b + 3], c = table[5 * b + 4];
   const void* g = args.g[param];
   const int ld = args.ld[param];
+  const bool vec = args.vec[param] != 0;
   const size_t nn = static_cast<size_t>(B) * B;
+  const int col = c0 + 4 * tx;  // this thread's 4 columns
+  if (col < B) {
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int row = bi * 32 + ty + 8 * k;
-    const int col = bj * 32 + tx;
-    float v = 0.f;
-    if (row < r && col < c) v = load_grad(g, static_cast<size_t>(row0 + row) * ld + col0 + col, dtype);
-    tile[ty + 8 * k][tx] = v;
-    Gs[b * nn + static_cast<size_t>(row) * B + col] = v;
+    for (int k = 0; k < 4; ++k) {
+      const int row = r0 + ty + 8 * k;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (row < r) v = load_grad4(g, static_cast<size_t>(row0 + row) * ld + col0 + col, dtype, vec, c - col);
+      *reinterpret_cast<float4*>(Gs + b * nn + static_cast<size_t>(row) * B + col) = v;
+      *reinterpret_cast<float4*>(&tile[(ty + 8 * k) * STRIDE + 4 * tx]) = v;
+    }
   }
   __syncthreads();
+  // Gt[b][c0 + j][r0 .. r0+31] = tile[0 .. 31][j]: 128 rows of 8 float4 each.
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const int row = bj * 32 + ty + 8 * k;  // row of G^T = column of G
-    const int col = bi * 32 + tx;
-    Gt[b * nn + static_cast<size_t>(row) * B + col] = tile[tx][ty + 8 * k];
+    const int idx = t + 256 * k;
+    const int j = idx >> 3;         // column of the piece = row of Gt
+    const int part = idx & 7;       // 4-row group
+    if (c0 + j < B) {
+      float4 v;
+      v.x = tile[(4 * part + 0) * STRIDE + j];
+      v.y = tile[(4 * part + 1) * STRIDE + j];
+      v.z = tile[(4 * part + 2) * STRIDE + j];
+      v.w = tile[(4 * part + 3) * STRIDE + j];
+      *reinterpret_cast<float4*>(Gt + b * nn + static_cast<size_t>(c0 + j) * B + r0 + 4 * part) = v;
+    }
   }
-  if (bi == 0 && bj == 0 && tx == 0 && ty == 0) {
+  if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0) {
     blk_wptr[b] = args.w[param] + static_cast<size_t>(row0) * ld + col0;
     blk_ld[b] = ld;
   }
@@ -129,6 +166,7 @@ __device__ __forceinline__ float effective_eps(float eps, float s) { return fmax
 __global__ void root_prologue_kernel(int kind, const float* __restrict__ A, int n, const int* __restrict__ valid,
                                      float eps, int p, const float* __restrict__ s, float* __restrict__ out0,
                                      float* __restrict__ out1, float* __restrict__ out2) {
+  pdl_launch_dependents();  // a following GEMM may start its prologue
   __shared__ float t1[32][33];
   __shared__ float t2[32][33];
   const int i = blockIdx.z;
@@ -167,6 +205,7 @@ __global__ void root_prologue_kernel(int kind, const float* __restrict__ A, int 
 // spectrum in (0, 1]); Y0' = Y, T0 = (3 I - Y) / 2, Z1 = T0.  Elementwise.
 __global__ void db_stage2_kernel(const float* Y0, const float* Y1, const int* __restrict__ iters, int n,
                                  float* Ynew0, float* __restrict__ T, float* __restrict__ Z1) {
+  pdl_launch_dependents();  // a following GEMM may start its prologue
   const int i = blockIdx.y;
   const size_t nn = static_cast<size_t>(n) * n;
   const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -200,6 +239,7 @@ __global__ void __launch_bounds__(1024) check_kernel(float* res, float* prev, in
                                                      const int* valid, int batch, int n, float tol, int* counter,
                                                      int cap, int kmin, int* flags, cudaGraphConditionalHandle cond,
                                                      int set_cond, int graph_kernels) {
+  pdl_launch_dependents();  // a following GEMM may start its prologue
   __shared__ int active;
   if (threadIdx.x == 0) active = 0;
   __syncthreads();
@@ -249,6 +289,7 @@ __global__ void __launch_bounds__(1024) check_kernel(float* res, float* prev, in
 __global__ void finalize_kernel(const float* __restrict__ X0, const float* __restrict__ X1,
                                 const int* __restrict__ iters, int default_iters, const float* __restrict__ sc, int n,
                                 float* __restrict__ out, int* flags) {
+  pdl_launch_dependents();  // a following GEMM may start its prologue
   __shared__ float t1[32][33];
   __shared__ float t2[32][33];
   const int i = blockIdx.z;
@@ -314,6 +355,7 @@ __global__ void cheb_coef_kernel(const float* __restrict__ s, int degree, int p,
 __global__ void cheb_prologue_kernel(const float* __restrict__ A, int n, const int* __restrict__ valid, float eps,
                                      const float* __restrict__ s, const float* __restrict__ coef, int degree,
                                      float* __restrict__ Xt, float* __restrict__ bd, float* __restrict__ bd1) {
+  pdl_launch_dependents();  // a following GEMM may start its prologue
   __shared__ float t1[32][33];
   __shared__ float t2[32][33];
   const int i = blockIdx.z;
@@ -358,7 +400,7 @@ int launch_stack(const StackArgs& args, const int* d_table, int nb, int B, int g
                  float** blk_wptr, int* blk_ld, cudaStream_t st, double alg_bytes) {
   if (nb == 0) return 0;
   ProfScope ps(K_STACK, st, 0.0, alg_bytes);
-  dim3 grid(B / 32, B / 32, nb), block(32, 8);
+  dim3 grid((B + 127) / 128, B / 32, nb), block(32, 8);
   stack_blocks_kernel<<<grid, block, 0, st>>>(args, d_table, B, grad_dtype, Gs, Gts, blk_wptr, blk_ld);
   count_launch();
   return check_cuda(cudaGetLastError(), "stack_blocks_kernel");
