@@ -7,8 +7,9 @@
 //   1. stack     gradient blocks -> Gs (B x B) and Gt (transposed), zero-padded
 //   2. stats     L <- beta L + Gs Gs^T, R <- beta R + Gt Gt^T     (one GEMM launch)
 //   3. roots     if step % refresh_every == 0: XL, XR of the damped, scaled stats
-//   4. apply     T = XL G (GEMM), then W -= lr T XR fused into the second
-//                GEMM's epilogue, masked to each block's real extent.
+//   4. apply     T = XL G (GEMM; on other steps it joins the launch of 2), then
+//                W -= lr T XR fused into the second GEMM's epilogue, masked to
+//                each block's real extent.
 #include <algorithm>
 #include <cstring>
 #include <new>
@@ -277,7 +278,15 @@ int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d
   if ((rc = launch_stack(args, h->d_table, nb, B, c.grad_dtype, h->Gs, h->Gt, h->blk_wptr, h->blk_ld, st,
                          h->stack_bytes)))
     return rc;
-  // 2. statistics: L <- beta L + G G^T (first nb matrices), R <- beta R + G^T G (next nb)
+  // 2. statistics: L <- beta L + G G^T (first nb matrices), R <- beta R + G^T G (next nb).
+  // On steps that keep the previous roots, the first apply product T = XL G
+  // depends on neither, so it joins the same launch.
+  const bool refresh = h->step % c.refresh_every == 0;
+  auto add_apply1 = [&](Builder& b) {
+    Epilogue& e = b.add(nb, B, h->mRoots, 0, h->mGt, 0, h->stats_flops_L);
+    e.D = h->Tap;
+    e.flags = h->d_status;
+  };
   {
     Builder b;
     Epilogue& eL = b.add(nb, B, h->mGs, 0, h->mGs, 0, h->stats_flops_L);
@@ -290,10 +299,11 @@ int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d
     eR.C = h->stats + plain_floats(nb, B);
     eR.D = h->stats + plain_floats(nb, B);
     eR.flags = h->d_status;
+    if (!refresh) add_apply1(b);
     if ((rc = b.launch(st))) return rc;
   }
   // 3. roots of all 2 nb damped statistics, every refresh_every steps
-  if (h->step % c.refresh_every == 0) {
+  if (refresh) {
     RootJob job;
     job.batch = 2 * nb;
     job.n = B;
@@ -310,15 +320,12 @@ int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d
     job.iters_used = nullptr;
     job.flags = h->d_status;
     if ((rc = run_inverse_roots(job, h->scratch + h->xl.root, h->xl.root_bytes, st))) return rc;
-  }
-  // 4. apply: T = XL G, then W -= lr T XR (masked scatter into the weights)
-  {
+    // 4a. apply, first product: T = XL G (with the fresh roots)
     Builder b;
-    Epilogue& e = b.add(nb, B, h->mRoots, 0, h->mGt, 0, h->stats_flops_L);
-    e.D = h->Tap;
-    e.flags = h->d_status;
+    add_apply1(b);
     if ((rc = b.launch(st))) return rc;
   }
+  // 4b. apply, second product: W -= lr T XR (masked scatter into the weights)
   {
     Builder b;
     Epilogue& e = b.add(nb, B, h->mTap, 0, h->mRoots, nb, h->stats_flops_R);
