@@ -160,8 +160,13 @@ int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, flo
                      cudaStream_t st);
 // kind: 0 = Newton (M0, T0 = ((p+1)I - M0)/p, X1 = T0)
 //       1 = Newton-DB (Y0 = A', T0 = (3I - A')/2, Z1 = T0)
+// Coupled-Newton scale: s = min(||A + eps I||_F, 1.25 x power-iteration estimate
+// of the largest eigenvalue), sc = s^{-1/p}, sf = ||A + eps I||_F.
+int launch_spectral_scale(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int iters,
+                          float* s, float* sc, float* sf, cudaStream_t st);
+// sf (nullable: s) sets the damping floor eps_eff = max(eps, 2^-24 sf).
 int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const int* valid, float eps, int p,
-                         const float* s, float* out0, float* out1, float* out2, cudaStream_t st);
+                         const float* s, const float* sf, float* out0, float* out1, float* out2, cudaStream_t st);
 // Second Newton-DB stage: Y0' = Y_par(i) (parity from iters), T0 = (3I - Y0')/2, Z1 = T0.
 int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters, int64_t batch, int n,
                               float* Ynew0, float* T, float* Z1, cudaStream_t st);

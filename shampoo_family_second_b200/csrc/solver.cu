@@ -53,7 +53,7 @@ int stacks_for(int solver) { return solver == 0 ? 7 : (solver == 1 ? 5 : 4); }
 
 constexpr size_t kAlign = 256;
 constexpr size_t kHeader = 64 * 1024;  // covers the alignment padding of the arrays
-constexpr int kVecInts = 7;            // s sc res prev done iters iters1
+constexpr int kVecInts = 8;            // s sc sf res prev done iters iters1
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // First iteration at which a stalled residual counts as stagnation: an
@@ -62,12 +62,14 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // square-root iteration, reaching 1/2 within 18 (resp. 20) iterations; a few
 // quadratic steps and a margin give the values below.
 int kmin_newton(int p) { return p == 4 ? 24 : 26; }
+constexpr int kPowerIters = 12;  // power-iteration steps of the coupled-Newton scale
 constexpr int kKminSqrt = 26;
 
 struct Layout {
   int* counter;  // [0] iterations done, [1] matrices still active (written by the check kernel)
   float* s;
   float* sc;
+  float* sf;  // Frobenius norm of A + eps I (the damping floor's reference)
   float* res;
   float* prev;
   int* done;
@@ -89,6 +91,7 @@ Layout carve(void* base, int64_t cb, int n, int solver) {
   L.counter = reinterpret_cast<int*>(take(8));
   L.s = reinterpret_cast<float*>(take(cb * 4));
   L.sc = reinterpret_cast<float*>(take(cb * 4));
+  L.sf = reinterpret_cast<float*>(take(cb * 4));
   L.res = reinterpret_cast<float*>(take(cb * 4));
   L.prev = reinterpret_cast<float*>(take(cb * 4));
   L.done = reinterpret_cast<int*>(take(cb * 4));
@@ -275,7 +278,14 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
     StackMaps sm[7];
     for (int k = 0; k < stacks_for(job.solver); ++k)
       if ((rc = make_stack_maps(sm[k], S.stack[k], cb, n))) return rc;
-    if ((rc = launch_frob_norm(A, cb, n, valid, job.eps, p, S.s, S.sc, st))) return rc;
+    // Coupled Newton scales by the power-iteration estimate (bounded by the
+    // Frobenius norm); Newton-DB (convergent only on (0, 2)) and Chebyshev
+    // (an exact upper bound is needed) by the Frobenius norm.
+    if (job.solver == 0) {
+      if ((rc = launch_spectral_scale(A, cb, n, valid, job.eps, p, kPowerIters, S.s, S.sc, S.sf, st))) return rc;
+    } else {
+      if ((rc = launch_frob_norm(A, cb, n, valid, job.eps, p, S.s, S.sc, st))) return rc;
+    }
     if (residual) {
       if ((rc = check_cuda(cudaMemsetAsync(S.done, 0, cb * 4, st), "memset done"))) return rc;
       if ((rc = check_cuda(cudaMemsetAsync(S.res, 0, cb * 4, st), "memset res"))) return rc;
@@ -330,7 +340,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       StackMaps& T = sm[4];
       StackMaps& T2 = sm[5];
       StackMaps& T4 = sm[6];
-      if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, M[0].base, T.base, X[1].base, st)))
+      if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, S.sf, M[0].base, T.base, X[1].base, st)))
         return rc;
       // One iteration j on stream cs (inside a graph loop when lp != NULL).
       auto iterate = [&](int j, cudaStream_t cs, const GraphLoop* lp) -> int {
@@ -392,7 +402,8 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       StackMaps* Y = &sm[0];
       StackMaps* Z = &sm[2];
       StackMaps& T = sm[4];
-      if ((rc = launch_root_prologue(1, A, cb, n, valid, job.eps, p, S.s, Y[0].base, T.base, Z[1].base, st)))
+      if ((rc = launch_root_prologue(1, A, cb, n, valid, job.eps, p, S.s, nullptr, Y[0].base, T.base, Z[1].base,
+                                     st)))
         return rc;
       const int stages = (p == 4) ? 2 : 1;
       for (int stage = 0; stage < stages; ++stage) {

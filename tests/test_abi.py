@@ -99,7 +99,7 @@ def test_scratch_sizes(sb):
     a = sb.inv_root_scratch_bytes(64, 1024, sb.SOLVER_NEWTON)
     b = sb.inv_root_scratch_bytes(128, 1024, sb.SOLVER_NEWTON)
     per = b - a
-    assert per == 64 * (7 * 1024 * 1024 * 4 + 4 * (7 + 64 + 2))   # Newton: 7 stacks per matrix
+    assert per == 64 * (7 * 1024 * 1024 * 4 + 4 * (8 + 64 + 2))   # Newton: 7 stacks per matrix
     assert sb.inv_root_scratch_bytes(64, 1024, sb.SOLVER_NEWTON_DB) < a
     assert sb.gemm_scratch_bytes(3, 256) == 0   # operands are split on chip
     # the no-alloc entry point's fixed 32 MiB covers one matrix of every supported size

@@ -142,3 +142,22 @@ def test_graph_loop_matches_plain_launches(sb, solver, per_iter):
     # prologue, norm, finalize, report and per stage one extra loop pass at most
     assert n1 - n0 <= 8 + per_iter * (needed + 2 * stages), (n1 - n0, needed)
     assert n1 - n0 < per_iter * 60 * stages
+
+
+def test_newton_uses_the_spectral_scale(sb):
+    """Coupled Newton scales by min(||A+eps I||_F, 1.25 x a power-iteration
+    estimate of the largest eigenvalue): on Wishart statistics (largest
+    eigenvalue about 0.15 of the Frobenius norm) it stops in fewer iterations
+    than the same iteration needs under Frobenius scaling, with the same root."""
+    from oracle import iter_mirror as im
+    rng = np.random.default_rng(12)
+    G = rng.standard_normal((4, 256, 256)).astype(np.float32)
+    A32 = np.einsum("bij,bkj->bik", G, G).astype(np.float32)
+    X, it, st = run(sb, A32, p=4, eps=1e-3, solver=sb.SOLVER_NEWTON, iters=60, tol=1e-5)
+    assert st == 0
+    for b in range(4):
+        A = A32[b].astype(np.float64)
+        _, k_frob, _ = im.coupled_newton(A, 4, 1e-3, 60, tol=1e-5, trace_tol=True)
+        assert it[b] < k_frob, (it[b], k_frob)
+        ref = oracle.inverse_root(A, 4, 1e-3)
+        assert oracle.rel_fro(X[b], ref) < root_gate(A, 4, 1e-3)

@@ -392,3 +392,23 @@ def test_rel_fro():
     assert osh.rel_fro(np.ones(4), np.ones(4)) == 0.0
     assert osh.rel_fro(np.array([1.0, 0]), np.array([2.0, 0])) == pytest.approx(0.5)
     assert osh.rel_fro(np.zeros(2), np.zeros(2)) == 0.0
+
+
+def test_spectral_scale_keeps_the_root_and_saves_iterations():
+    """The coupled-Newton scale min(||A+eps I||_F, 1.25 lam_est): the root is
+    scale-invariant ((cA)^{-1/p} = c^{-1/p} A^{-1/p}), so both scalings reach the
+    exact root; the spectral one starts the largest eigenvalue near 0.8 instead
+    of lam_max / ||A||_F and needs fewer iterations on Wishart statistics."""
+    from oracle import iter_mirror as im
+    rng = np.random.default_rng(8)
+    G = rng.standard_normal((256, 256))
+    A = G @ G.T
+    eps = 1e-3
+    ref = oracle.inverse_root(A, 4, eps)
+    Xf, kf, _ = im.coupled_newton(A, 4, eps, 80, tol=1e-10, trace_tol=True)
+    Xs, ks, _ = im.coupled_newton(A, 4, eps, 80, tol=1e-10, scale="spectral", trace_tol=True)
+    assert oracle.rel_fro(Xf, ref) < 1e-8 and oracle.rel_fro(Xs, ref) < 1e-8
+    assert ks <= kf - 2, (ks, kf)
+    lam = np.linalg.eigvalsh(A + eps * np.eye(256))[-1]
+    est = im.power_estimate(A + eps * np.eye(256))
+    assert 0.9 * lam <= est <= lam * (1 + 1e-12)
