@@ -56,7 +56,8 @@ WORKLOAD_NAMES = {
     "sweep": "inverse_root_sweep",
 }
 SWEEP_BATCH = {256: 512, 512: 128, 1024: 64}
-SOLVER_NAMES = {0: "coupled_newton", 1: "newton_db", 2: "chebyshev"}
+SOLVER_NAMES = {0: "coupled_newton", 1: "newton_db", 2: "chebyshev", 3: "coupled_newton_cubic"}
+SOLVER_IDS = {"newton": 0, "newton_db": 1, "chebyshev": 2, "newton_cubic": 3}
 
 
 # ---------------------------------------------------------------------------
@@ -351,7 +352,7 @@ def run_ours(args, wl):
     achieved = (g.alg_flops / max(g.launches, 1)) / (gemm_avg_ms * 1e-3) / 1e12 if g.launches else 0.0
     tf32_peak = peaks["bf16_tflops_sustained"] * TF32_PER_BF16
     peak = tf32_peak / SPLIT_PASSES
-    traffic = gemm_traffic_per_launch(g)
+    traffic = gemm_traffic_per_launch(wl)
     step_total_prof = sum(tl.total_ms for tl in tallies.values())
 
     result = {
@@ -418,16 +419,29 @@ def run_ours(args, wl):
         print(json.dumps(result), flush=True)
 
 
-def gemm_traffic_per_launch(g):
+TRAFFIC_SOURCES = ("gemm_tc.cu", "solver.cu", "api.cu")
+
+
+def traffic_source_sha():
+    """sha256 over the sources that decide the GEMM launch mix of a step."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "shampoo_family_second_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gemm_traffic_per_launch(wl):
     """DRAM bytes per GEMM launch from the committed ncu capture of this
-    workload's GEMM, if the capture was taken on the current kernel source."""
+    workload's GEMMs, if the capture was taken on the current sources with the
+    same workload and solver (else None)."""
     path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        import hashlib
-        src = open(os.path.join(ROOT, "shampoo_family_second_b200", "csrc", "gemm_tc.cu"), "rb").read()
-        if d.get("gemm_tc_sha256") != hashlib.sha256(src).hexdigest():
+        if (d.get("source_sha256") != traffic_source_sha() or d.get("workload_key") != wl.name
+                or d.get("solver") != SOLVER_NAMES[wl.solver]):
             return None
         return d.get("bytes_per_launch")
     except Exception:
@@ -531,7 +545,7 @@ def run_sweep(args):
     stream = torch.cuda.current_stream()
     n, kappa, p = args.sweep_n, args.sweep_kappa, args.sweep_p
     batch = args.sweep_batch or SWEEP_BATCH.get(n, 64)
-    solver = {"newton": 0, "newton_db": 1, "chebyshev": 2}[args.sweep_solver]
+    solver = SOLVER_IDS[args.sweep_solver]
     A64, Q64, lam64 = workloads.spd_batch(batch, n, kappa, seed=4321 + n + rank, return_parts=True)
     A = torch.from_numpy(A64.astype(np.float32)).to(device)
     X = torch.empty_like(A)
@@ -615,11 +629,13 @@ def main():
     ap.add_argument("--ring", type=int, default=8, help="distinct gradient sets kept on the device")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--solver", default=None, choices=["newton", "newton_db", "chebyshev", "newton_cubic"],
+                    help="inverse-root solver of the step workloads (default: the workload's own)")
     ap.add_argument("--sweep-n", type=int, default=512)
     ap.add_argument("--sweep-batch", type=int, default=0)
     ap.add_argument("--sweep-kappa", type=float, default=1e4)
     ap.add_argument("--sweep-p", type=int, default=4)
-    ap.add_argument("--sweep-solver", default="newton", choices=["newton", "newton_db", "chebyshev"])
+    ap.add_argument("--sweep-solver", default="newton", choices=["newton", "newton_db", "chebyshev", "newton_cubic"])
     ap.add_argument("--sweep-iters", type=int, default=25)
     ap.add_argument("--sweep-tol", type=float, default=0.0)
     ap.add_argument("--sweep-degree", type=int, default=32)
@@ -633,7 +649,10 @@ def main():
             return
         run_sweep(args)
         return
-    wl = workloads.workload(args.workload)
+    over = {}
+    if args.solver is not None:
+        over["solver"] = SOLVER_IDS[args.solver]
+    wl = workloads.workload(args.workload, **over)
     np.random.seed(0)
     if args.impl == "reference":
         run_reference(args, wl)

@@ -74,7 +74,11 @@ enum {
 enum {
   SHAMPOO_SOLVER_NEWTON = 0,    /* coupled Newton for A^{-1/p} (Guo & Higham 2006) */
   SHAMPOO_SOLVER_NEWTON_DB = 1, /* coupled Y/Z square-root iteration, twice for p = 4 */
-  SHAMPOO_SOLVER_CHEBYSHEV = 2  /* Chebyshev interpolant of x^{-1/p}, Clenshaw evaluation */
+  SHAMPOO_SOLVER_CHEBYSHEV = 2, /* Chebyshev interpolant of x^{-1/p}, Clenshaw evaluation */
+  SHAMPOO_SOLVER_NEWTON_CUBIC = 3 /* coupled Newton with the degree-2 binomial correction
+                                     T = I + (I-M)/p + (p+1)(I-M)^2/(2p^2) after a plain first
+                                     step: one more GEMM per iteration, cubic local convergence,
+                                     about a third fewer iterations */
 };
 
 /* Gradient element types. */
@@ -100,7 +104,7 @@ enum {
  *  root_p         2 or 4.
  *  solver         SHAMPOO_SOLVER_*.
  *  iters          iterations (tol = 0) or iteration cap (tol > 0) per Newton / Newton-DB
- *                 stage, >= 1; ignored by Chebyshev.
+ *                 stage, >= 1; ignored by Chebyshev.  NEWTON_CUBIC behaves as NEWTON here.
  *  tol            0: fixed iteration count; > 0: stop a matrix once
  *                 tr(I - M)/n (Newton) or tr(I - Z Y)/n (Newton-DB) <= tol.  Both iterations
  *                 keep every eigenvalue of M (or Z Y) at or below 1, so this trace bounds the

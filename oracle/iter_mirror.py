@@ -13,6 +13,11 @@ Newton on the GPU the power-iteration scale of spectral_scale.
 * Coupled Newton for A'^{-1/p} (Guo & Higham, "A Schur-Newton method for the
   matrix p-th root and its inverse", 2006): X_0 = I, M_0 = A';
   T = ((p + 1) I - M) / p;  X <- X T;  M <- T^p M.  M -> I, X -> A'^{-1/p}.
+* The same coupled form with a higher-degree correction: T is the degree-m
+  truncation sum_{j<=m} c_j (I - M)^j of the binomial series of
+  M^{-1/p} = (I - (I - M))^{-1/p}, c_0 = 1, c_j = c_{j-1} (j - 1 + 1/p) / j.
+  m = 1 gives the Newton T above; the CUDA solver's NEWTON_CUBIC takes m = 2
+  from the second iteration on, after one plain Newton step.
 * Newton-DB, read as the coupled Denman-Beavers-family square-root iteration
   in its multiplication-only (Newton-Schulz) form (Higham, "Functions of
   Matrices", 2008, sec. 6.3 and 6.8): Y_0 = A', Z_0 = I;
@@ -64,11 +69,32 @@ def spectral_scale(A: np.ndarray, eps: float):
     return Ad / s, s
 
 
+def binomial_coefficients(p: int, m: int):
+    """c_0..c_m of (1 - x)^{-1/p} = sum_j c_j x^j."""
+    c = [1.0]
+    for j in range(1, m + 1):
+        c.append(c[-1] * (j - 1 + 1.0 / p) / j)
+    return c
+
+
+def correction(M: np.ndarray, p: int, degree: int) -> np.ndarray:
+    """T = sum_{j<=degree} c_j (I - M)^j."""
+    eye = np.eye(M.shape[0])
+    D = eye - M
+    T = np.zeros_like(M)
+    P = eye
+    for cj in binomial_coefficients(p, degree):
+        T = T + cj * P
+        P = P @ D
+    return T
+
+
 def coupled_newton(A: np.ndarray, p: int, eps: float, iters: int, tol: float = 0.0, scale: str = "frobenius",
-                   trace_tol: bool = False):
+                   trace_tol: bool = False, degree: int = 1):
     """Returns (X, iterations run, final residual).  The residual is
     ||M - I||_F / sqrt(n), or tr(I - M) / n with trace_tol (the CUDA solver's
-    stopping test)."""
+    stopping test).  degree > 1 uses that correction degree from the second
+    iteration on (the first is a plain Newton step)."""
     M, s = (spectral_scale if scale == "spectral" else frobenius_scale)(A, eps)
     n = M.shape[0]
     eye = np.eye(n)
@@ -80,7 +106,7 @@ def coupled_newton(A: np.ndarray, p: int, eps: float, iters: int, tol: float = 0
     res = residual(M)
     k = 0
     while k < iters and not (tol > 0.0 and res <= tol):
-        T = ((p + 1) * eye - M) / p
+        T = ((p + 1) * eye - M) / p if (degree == 1 or k == 0) else correction(M, p, degree)
         X = X @ T
         M = np.linalg.matrix_power(T, p) @ M
         res = residual(M)

@@ -33,6 +33,7 @@ DEVFLAG_STAGNATED = 8
 SOLVER_NEWTON = 0
 SOLVER_NEWTON_DB = 1
 SOLVER_CHEBYSHEV = 2
+SOLVER_NEWTON_CUBIC = 3
 
 F32 = 0
 BF16 = 1

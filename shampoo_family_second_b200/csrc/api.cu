@@ -40,7 +40,7 @@ int validate_config(const shampoo_config* c) {
   if (!(c->eps >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "eps must be >= 0");
   if (!(c->lr == c->lr)) return set_error(SHAMPOO_ERR_INVALID_ARG, "lr is NaN");
   if (c->root_p != 2 && c->root_p != 4) return set_error(SHAMPOO_ERR_INVALID_ARG, "root_p must be 2 or 4");
-  if (c->solver < 0 || c->solver > 2) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", c->solver);
+  if (c->solver < 0 || c->solver > 3) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", c->solver);
   if (c->solver != SHAMPOO_SOLVER_CHEBYSHEV && (c->iters < 1 || c->iters > 1000))
     return set_error(SHAMPOO_ERR_INVALID_ARG, "iters must be in [1, 1000]");
   if (!(c->tol >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "tol must be >= 0");
@@ -381,7 +381,7 @@ void shampoo_destroy(shampoo_handle h) { delete h; }
 
 int inv_root_scratch_bytes(int64_t batch, int32_t n, int32_t solver, size_t* bytes) {
   if (!bytes) return set_error(SHAMPOO_ERR_INVALID_ARG, "bytes is NULL");
-  if (batch < 0 || n < 32 || n > 1024 || n % 32 || solver < 0 || solver > 2)
+  if (batch < 0 || n < 32 || n > 1024 || n % 32 || solver < 0 || solver > 3)
     return set_error(SHAMPOO_ERR_INVALID_ARG, "bad batch / n / solver");
   *bytes = root_scratch_header() + root_scratch_per_matrix(n, solver) * static_cast<size_t>(std::max<int64_t>(batch, 1));
   return SHAMPOO_OK;
@@ -396,7 +396,7 @@ int inv_root_batched(const float* d_A, float* d_X, int64_t batch, int32_t n, int
   if (n < 32 || n > 1024 || n % 32) return set_error(SHAMPOO_ERR_INVALID_ARG, "n %d: need a multiple of 32 in [32, 1024]", n);
   if (p != 2 && p != 4) return set_error(SHAMPOO_ERR_INVALID_ARG, "p must be 2 or 4");
   if (!(eps >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "eps must be >= 0");
-  if (solver < 0 || solver > 2) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", solver);
+  if (solver < 0 || solver > 3) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", solver);
   if (solver != SHAMPOO_SOLVER_CHEBYSHEV && (iters < 1 || iters > 1000))
     return set_error(SHAMPOO_ERR_INVALID_ARG, "iters must be in [1, 1000]");
   if (!(tol >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "tol must be >= 0");

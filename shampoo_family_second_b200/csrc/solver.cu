@@ -8,20 +8,34 @@
 //   coupled Newton  (Guo & Higham 2006): X0 = I, M0 = A'; T = ((p+1) I - M)/p;
 //                   X <- X T; M <- T^p M   (4 GEMMs per iteration for p = 4,
 //                   3 for p = 2);
+//   coupled Newton, second-degree correction: the same coupled form with T
+//                   the degree-2 truncation of the binomial series of
+//                   M^{-1/p} = (I - (I - M))^{-1/p}; the degree-1 truncation is
+//                   the Newton T above.  One more GEMM per iteration (T needs
+//                   M^2), cubic local convergence, and an eigenvalue mu << 1
+//                   of M grows by (1 + c1 + c2)^p instead of ((p+1)/p)^p per
+//                   iteration (3.91 against 2.44 at p = 4);
 //   Newton-DB       coupled Denman-Beavers-family square-root iteration in its
 //                   multiplication-only form: Y0 = A', Z0 = I;
 //                   T = (3 I - Z Y)/2; Y <- Y T; Z <- T Z (3 GEMMs); p = 4 runs
 //                   a second stage on Y ~ A'^{1/2};
 //   Chebyshev       Clenshaw evaluation of the degree-d interpolant of x^{-1/p}
 //                   on [a, 1] (d - 1 GEMMs).
-// Operand orientation.  The tensor core computes A B^T from row-major stacks
-// fastest (both operands K-major).  The iterates are symmetric in exact
-// arithmetic, so A B^T is the wanted product up to rounding, which leaves a
-// small antisymmetric component in the iterates.  Coupled Newton and the
-// Clenshaw recurrence are stable under it (it neither grows nor disturbs the
-// symmetric part), so they use A B^T.  The Newton-DB fixed point is unstable
-// along that direction (the error grows about 1.5x per iteration), so its
-// products are true products A B with B read MN-major.
+// Operand orientation.  The iterates are symmetric in exact arithmetic, so
+// A B^T (both operands K-major) equals the wanted product A B up to rounding,
+// but the rounding's antisymmetric part K then never dies out: in coupled
+// Newton it flips sign every iteration, is amplified with the small
+// eigenvalues during the linear phase (to ||K||_F ~ 0.08 at n = 256), and its
+// second-order term 2 (2 c2 + c1^2) K^T K shifts the fixed point of M above I
+// (by 2e-5 for the Newton T, 1e-4 with the second-degree correction; the
+// signed trace residual settles at -3e-6, resp. -2e-5, and the latter never
+// reaches a 1e-5 tolerance).  With true products A B (B read MN-major) K
+// decays quadratically with the rest of the error, the residual settles near
+// +3e-8 and M's eigenvalues within 3e-7 of 1, so both Newton forms use true
+// products.  The Newton-DB fixed point is outright unstable along K under
+// A B^T (the error grows about 1.5x per iteration): true products as well.
+// The Clenshaw recurrence is a fixed number of steps with no fixed point to
+// shift and keeps A B^T.
 // Convergence is measured by tr(I - M)/n (Newton) or tr(I - Z Y)/n (Newton-DB):
 // both iterations keep every eigenvalue of M (or Z Y) at or below 1, so the
 // trace bounds the largest eigenvalue error and ignores the antisymmetric
@@ -43,13 +57,13 @@
 namespace shampoo {
 namespace {
 
-constexpr int NEWTON_B = B_TRANSPOSED;
+constexpr int NEWTON_B = B_MN_MAJOR;
 
 // Scratch stacks per solver (plain fp32, n x n per matrix):
-//   Newton    : M0 M1 X0 X1 T T2 T4
+//   Newton    : M0 M1 X0 X1 T T2 T4 (both correction degrees)
 //   Newton-DB : Y0 Y1 Z0 Z1 T
 //   Chebyshev : Xt b0 b1 b2
-int stacks_for(int solver) { return solver == 0 ? 7 : (solver == 1 ? 5 : 4); }
+int stacks_for(int solver) { return (solver == 0 || solver == 3) ? 7 : (solver == 1 ? 5 : 4); }
 
 constexpr size_t kAlign = 256;
 constexpr size_t kHeader = 64 * 1024;  // covers the alignment padding of the arrays
@@ -60,8 +74,14 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // eigenvalue mu of M (scaled input 2^-24 <= mu << 1) grows by ((p+1)/p)^p per
 // coupled-Newton iteration (2.44 at p = 4, 2.25 at p = 2) and by 9/4 per
 // square-root iteration, reaching 1/2 within 18 (resp. 20) iterations; a few
-// quadratic steps and a margin give the values below.
-int kmin_newton(int p) { return p == 4 ? 24 : 26; }
+// quadratic steps and a margin give the values below.  With the
+// second-degree correction the growth is (1 + c1 + c2)^p (3.91 at p = 4,
+// 3.52 at p = 2), reaching 1/2 within 13 (resp. 14) iterations counting the
+// plain first step, followed by cubic steps.
+int kmin_newton(int p, bool order2) {
+  if (order2) return p == 4 ? 17 : 18;
+  return p == 4 ? 24 : 26;
+}
 constexpr int kPowerIters = 12;  // power-iteration steps of the coupled-Newton scale
 constexpr int kKminSqrt = 26;
 
@@ -281,7 +301,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
     // Coupled Newton scales by the power-iteration estimate (bounded by the
     // Frobenius norm); Newton-DB (convergent only on (0, 2)) and Chebyshev
     // (an exact upper bound is needed) by the Frobenius norm.
-    if (job.solver == 0) {
+    if (job.solver == 0 || job.solver == 3) {
       if ((rc = launch_spectral_scale(A, cb, n, valid, job.eps, p, kPowerIters, S.s, S.sc, S.sf, st))) return rc;
     } else {
       if ((rc = launch_frob_norm(A, cb, n, valid, job.eps, p, S.s, S.sc, st))) return rc;
@@ -333,47 +353,102 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       e.flags = job.flags;
     };
 
-    if (job.solver == 0) {
+    if (job.solver == 0 || job.solver == 3) {
       // ------------------------------------------------------------ coupled Newton
       StackMaps* M = &sm[0];  // M[0], M[1]
       StackMaps* X = &sm[2];  // X[0], X[1]
       StackMaps& T = sm[4];
       StackMaps& T2 = sm[5];
       StackMaps& T4 = sm[6];
+      // Second-degree correction (solver 3): from iteration 1 on,
+      // T = I + c1 (I - M) + c2 (I - M)^2 with c1 = 1/p, c2 = (p+1)/(2p^2),
+      // the first three terms of the binomial series of M^{-1/p} about I,
+      // which is one GEMM: T = c2 M M + (-c1 - 2 c2) M + (1 + c1 + c2) I.
+      // Iteration 0 is a plain Newton step; it maps every eigenvalue in
+      // (0, p+1) into (0, 1], where the second-degree steps keep eigenvalues
+      // increasing to 1.
+      const bool order2 = job.solver == 3;
+      const float c1 = 1.f / p, c2 = (p + 1.f) / (2.f * p * p);
       if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, S.sf, M[0].base, T.base, X[1].base, st)))
         return rc;
+      // With the second-degree correction the M update also writes
+      // D = I - M (exact in fp32 from the accumulator value), and T is formed
+      // from D: T = c2 D D + c1 D + I.  The product of D carries rounding
+      // relative to |D|^2 only, so T is as accurate as the Newton T = I + D/p
+      // (a product of M itself would add rounding of order |M|^2 = 1, above
+      // the residual tolerance).  The three stacks T, T2, T4 then rotate
+      // (p = 4, period 2; p = 2, period 1), so that no launch writes a stack
+      // that another of its tiles reads:
+      //   p = 4, j >= 1: D in Q[j&1], T -> Q[(j+1)&1], T2 -> Q2, T4 -> Q[j&1],
+      //                  next D -> Q[(j+1)&1];
+      //   p = 2, j >= 1: D in Q0, T -> Q1, T2 -> Q2, next D -> Q0;
+      //   j = 0 (plain step): T in Q0, T2 -> Q1, T4 -> Q2, next D -> Q1
+      //                  (p = 4) or Q0 (p = 2).
+      StackMaps* Q[3] = {&T, &T2, &T4};
       // One iteration j on stream cs (inside a graph loop when lp != NULL).
       auto iterate = [&](int j, cudaStream_t cs, const GraphLoop* lp) -> int {
         int r;
-        {
-          Builder b;
-          Epilogue& e = b.add(cbi, n, T, 0, T, 0, f1, NEWTON_B);  // T2 = T T
-          e.D = T2.base;
-          common(e);
+        StackMaps* Tb = Q[0];
+        StackMaps* T2b = Q[1];
+        StackMaps* T4b = Q[2];
+        StackMaps* Dnext = nullptr;
+        if (order2) {
           if (j >= 1) {
-            Epilogue& ex = b.add(cbi, n, X[j & 1], 0, T, 0, f1, NEWTON_B);  // X <- X T
+            StackMaps* Db = p == 4 ? Q[j & 1] : Q[0];
+            Tb = p == 4 ? Q[(j + 1) & 1] : Q[1];
+            T2b = Q[2];
+            T4b = Db;
+            Builder b;
+            Epilogue& e = b.add(cbi, n, *Db, 0, *Db, 0, f1, NEWTON_B);  // T = c2 D D + c1 D + I
+            e.alpha = c2;
+            e.C = Db->base;
+            e.beta = c1;
+            e.gamma = 1.f;
+            e.D = Tb->base;
+            common(e);
+            if ((r = b.launch(cs))) return r;
+          }
+          Dnext = p == 4 ? Q[(j + 1) & 1] : Q[0];
+        }
+        // The last iteration of a fixed count only needs X <- X T.
+        const bool last = !residual && j == job.iters - 1;
+        if (j >= 1 || !last) {
+          Builder b;
+          if (!last) {
+            Epilogue& e = b.add(cbi, n, *Tb, 0, *Tb, 0, f1, NEWTON_B);  // T2 = T T
+            e.D = T2b->base;
+            common(e);
+          }
+          if (j >= 1) {
+            Epilogue& ex = b.add(cbi, n, X[j & 1], 0, *Tb, 0, f1, NEWTON_B);  // X <- X T
             ex.D = X[(j + 1) & 1].base;
             common(ex);
           }
           if ((r = b.launch(cs))) return r;
         }
-        if (!residual && j == job.iters - 1) return 0;
-        StackMaps* P = &T2;
+        if (last) return 0;
+        StackMaps* P = T2b;
         if (p == 4) {
           Builder b;
-          Epilogue& e = b.add(cbi, n, T2, 0, T2, 0, f1, NEWTON_B);  // T4 = T2 T2
-          e.D = T4.base;
+          Epilogue& e = b.add(cbi, n, *T2b, 0, *T2b, 0, f1, NEWTON_B);  // T4 = T2 T2
+          e.D = T4b->base;
           common(e);
           if ((r = b.launch(cs))) return r;
-          P = &T4;
+          P = T4b;
         }
         {
           Builder b;
           Epilogue& e = b.add(cbi, n, *P, 0, M[j & 1], 0, f1, NEWTON_B);  // M <- T^p M
           e.D = M[(j + 1) & 1].base;
-          e.E = T.base;  // next T = ((p+1) I - M) / p
-          e.e_mul = -1.f / p;
-          e.e_add = static_cast<float>(p + 1) / p;
+          if (order2) {
+            e.E = Dnext->base;  // next D = I - M
+            e.e_mul = -1.f;
+            e.e_add = 1.f;
+          } else {
+            e.E = T.base;  // next T = ((p+1) I - M) / p
+            e.e_mul = -1.f / p;
+            e.e_add = static_cast<float>(p + 1) / p;
+          }
           e.res = residual ? S.res : nullptr;
           e.valid = valid;
           common(e);
@@ -381,11 +456,12 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
         }
         if (residual)
           return launch_check(S.res, S.prev, S.done, S.iters, valid, cb, n, job.tol, S.counter, job.iters,
-                              kmin_newton(p), job.flags, lp, cs);
+                              kmin_newton(p, order2), job.flags, lp, cs);
         return 0;
       };
       if (residual) {
-        if ((rc = iterate(0, st, nullptr)) || (rc = run_rest(iterate, p == 4 ? 4 : 3))) return rc;
+        const int per_iter = (p == 4 ? 4 : 3) + (order2 ? 1 : 0);
+        if ((rc = iterate(0, st, nullptr)) || (rc = run_rest(iterate, per_iter))) return rc;
       } else {
         for (int j = 0; j < job.iters; ++j)
           if ((rc = iterate(j, st, nullptr))) return rc;

@@ -36,9 +36,10 @@ def run(sb, A32, **kw):
 @pytest.mark.parametrize("n,batch", [(64, 4), (256, 3), (384, 2)])
 @pytest.mark.parametrize("p", [2, 4])
 @pytest.mark.parametrize("kappa", [1e2, 1e4])
-def test_newton_fixed(sb, n, batch, p, kappa):
+@pytest.mark.parametrize("solver", [0, 3])
+def test_newton_fixed(sb, n, batch, p, kappa, solver):
     A32 = workloads.spd_batch(batch, n, kappa, seed=n + p).astype(np.float32)
-    X, it, st = run(sb, A32, p=p, eps=0.0, solver=sb.SOLVER_NEWTON, iters=30, tol=0.0)
+    X, it, st = run(sb, A32, p=p, eps=0.0, solver=solver, iters=30, tol=0.0)
     assert st == 0
     assert np.all(it == 30)
     for b in range(batch):
@@ -48,14 +49,37 @@ def test_newton_fixed(sb, n, batch, p, kappa):
 
 
 @pytest.mark.parametrize("p", [2, 4])
-def test_newton_residual_mode(sb, p):
+@pytest.mark.parametrize("solver", [0, 3])
+def test_newton_residual_mode(sb, p, solver):
     A32 = workloads.spd_batch(4, 128, 1e3, seed=5).astype(np.float32)
-    X, it, st = run(sb, A32, p=p, eps=1e-6, solver=sb.SOLVER_NEWTON, iters=40, tol=1e-5)
+    X, it, st = run(sb, A32, p=p, eps=1e-6, solver=solver, iters=40, tol=1e-5)
     assert st == 0
     assert np.all(it > 0) and np.all(it < 40)
     for b in range(4):
         ref = oracle.inverse_root(A32[b].astype(np.float64), p, 1e-6)
         assert oracle.rel_fro(X[b], ref) < TOL
+
+
+@pytest.mark.parametrize("p", [2, 4])
+@pytest.mark.parametrize("kappa", [1e2, 1e4, 1e6])
+def test_cubic_newton_iterations_follow_the_float64_mirror(sb, p, kappa):
+    """The second-degree correction stops where its float64 restatement (same
+    spectral scale, same trace test) stops, give or take one iteration of fp32
+    rounding, and in fewer iterations than plain coupled Newton on the GPU."""
+    from oracle import iter_mirror as im
+    A32 = workloads.spd_batch(4, 256, kappa, seed=int(np.log10(kappa)) + 10 * p).astype(np.float32)
+    tol = 1e-5
+    X3, it3, st3 = run(sb, A32, p=p, eps=0.0, solver=sb.SOLVER_NEWTON_CUBIC, iters=40, tol=tol)
+    X0, it0, st0 = run(sb, A32, p=p, eps=0.0, solver=sb.SOLVER_NEWTON, iters=40, tol=tol)
+    assert st3 & ~sb.DEVFLAG_STAGNATED == 0 and st0 & ~sb.DEVFLAG_STAGNATED == 0
+    for b in range(4):
+        A = A32[b].astype(np.float64)
+        _, k, _ = im.coupled_newton(A, p, 0.0, 40, tol=tol, scale="spectral", trace_tol=True, degree=2)
+        assert abs(abs(int(it3[b])) - k) <= 1, (b, it3[b], k)
+        assert abs(int(it3[b])) < abs(int(it0[b])), (b, it3[b], it0[b])
+        ref = oracle.inverse_root(A, p, 0.0)
+        e3, e0 = oracle.rel_fro(X3[b], ref), oracle.rel_fro(X0[b], ref)
+        assert e3 < max(root_gate(A, p, 0.0), 1.5 * e0), (b, e3, e0)
 
 
 @pytest.mark.parametrize("p", [2, 4])
@@ -90,41 +114,54 @@ def test_not_converged_flag(sb):
     assert np.all(it == -2)
 
 
-@pytest.mark.parametrize("solver,kmin", [(0, 24), (1, 26)])
-def test_stagnation_stops_before_the_cap(sb, solver, kmin):
+@pytest.mark.parametrize("solver", [0, 1, 3])
+def test_rank_deficient_input_finishes_before_the_cap(sb, solver):
     """Rank-deficient input with eps = 0 (a 128 x 128 G^T G of rank 64, like
     the ragged blocks of the GPT-2 shapes): the null space sits at the damping
-    floor 2^-24 s, where fp32 rounding holds the residual far above tol.  The
-    solver must stop the iteration once the residual no longer improves (from
-    iteration kmin on), flag STAGNATED rather than NOT_CONVERGED, and stay
-    well below the cap.  The root is checked against the exact root on the
-    range space, and on the null space only for being finite (there it is set
-    by the damping floor alone; the exact root is infinite at eps = 0)."""
+    floor 2^-24 s.  The solver must end without NOT_CONVERGED (converged, or
+    stopped at a stagnated residual) well below the cap.  The root is checked
+    against the exact root on the range space, and on the null space only for
+    being finite (there it is set by the damping floor alone; the exact root
+    is infinite at eps = 0)."""
     rng = np.random.default_rng(31)
     G = rng.standard_normal((3, 64, 128)).astype(np.float32)
     A32 = np.einsum("bki,bkj->bij", G, G).astype(np.float32)
     cap = 80
     X, it, st = run(sb, A32, p=4, eps=0.0, solver=solver, iters=cap, tol=1e-5)
-    assert not st & sb.DEVFLAG_NOT_CONVERGED
-    if solver == 0:
-        assert st & sb.DEVFLAG_STAGNATED
-        assert np.all(it < 0) and np.all(-it >= kmin) and np.all(-it < cap), it
-        for b in range(3):
-            # range space (64 eigenvalues, well conditioned): the exact root there
-            lam, Q = np.linalg.eigh(A32[b].astype(np.float64))
-            rng_ = lam > 1e-3 * lam[-1]
-            assert rng_.sum() == 64
-            Qr = Q[:, rng_]
-            got = Qr.T @ X[b] @ Qr
-            ref = np.diag(lam[rng_] ** -0.25)
-            assert oracle.rel_fro(got, ref) < TOL, (b, oracle.rel_fro(got, ref))
-            assert np.all(np.isfinite(X[b]))
-    else:
-        # The square-root iteration lifts the damping floor's eigenvalues
-        # without stalling on this input: it converges (or stops at a
-        # stagnation) well before the cap.
-        assert st & ~sb.DEVFLAG_STAGNATED == 0
-        assert np.all(np.abs(it) < 2 * cap), it
+    assert st & ~sb.DEVFLAG_STAGNATED == 0, st
+    stages = 2 if solver == 1 else 1
+    assert np.all(np.abs(it) < stages * cap // 2), it
+    for b in range(3):
+        lam, Q = np.linalg.eigh(A32[b].astype(np.float64))
+        rng_ = lam > 1e-3 * lam[-1]
+        assert rng_.sum() == 64
+        Qr = Q[:, rng_]
+        got = Qr.T @ X[b] @ Qr
+        ref = np.diag(lam[rng_] ** -0.25)
+        assert oracle.rel_fro(got, ref) < TOL, (b, oracle.rel_fro(got, ref))
+        assert np.all(np.isfinite(X[b]))
+
+
+@pytest.mark.parametrize("solver,kmin", [(0, 24), (1, 26), (3, 17)])
+def test_stagnation_stops_before_the_cap(sb, solver, kmin):
+    """A tolerance below the fp32 resolution of the trace residual (1e-12;
+    the residual settles near 1e-8, where the fp32 iterate stops changing):
+    the solver must stop once the residual no longer improves, from iteration
+    kmin on, flag STAGNATED rather than NOT_CONVERGED, stay well below the
+    cap, and return the converged root.  The signed trace can land within
+    1e-12 of zero by chance on the way down, so a matrix may also end as
+    converged; most must stagnate."""
+    A32 = workloads.spd_batch(4, 128, 1e2, seed=33).astype(np.float32)
+    cap = 80
+    X, it, st = run(sb, A32, p=4, eps=0.0, solver=solver, iters=cap, tol=1e-12)
+    assert st & sb.DEVFLAG_STAGNATED and not st & sb.DEVFLAG_NOT_CONVERGED, st
+    stages = 2 if solver == 1 else 1
+    stag = it < 0
+    assert stag.sum() >= 2, it
+    assert np.all(-it[stag] >= kmin) and np.all(np.abs(it) < stages * cap), it
+    for b in range(4):
+        ref = oracle.inverse_root(A32[b].astype(np.float64), 4, 0.0)
+        assert oracle.rel_fro(X[b], ref) < TOL, (b, oracle.rel_fro(X[b], ref))
 
 
 def test_nonfinite_flag(sb):
@@ -135,7 +172,7 @@ def test_nonfinite_flag(sb):
     assert np.all(np.isfinite(X[0]))
 
 
-@pytest.mark.parametrize("solver,per_iter", [(0, 4), (1, 3)])
+@pytest.mark.parametrize("solver,per_iter", [(0, 4), (1, 3), (3, 5)])
 def test_graph_loop_matches_plain_launches(sb, solver, per_iter):
     """Residual-checked iterations after the first run as a CUDA graph loop
     that the device ends once every matrix is finished.  With profiling on

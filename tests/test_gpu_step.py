@@ -105,7 +105,7 @@ def test_ragged_blocks(sb, shapes):
     run_parity(sb, wl, wl.steps)
 
 
-@pytest.mark.parametrize("solver", [1, 2])
+@pytest.mark.parametrize("solver", [1, 2, 3])
 def test_other_solvers_in_step(sb, solver):
     # Chebyshev needs a spectral lower bound: eps large enough that a = eps / s
     # keeps the degree-32 interpolant within tolerance.

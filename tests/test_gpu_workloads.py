@@ -90,6 +90,18 @@ def test_lowrank_4x1024_b256(sb):
     run_workload(sb, wl, steps=11, k_blocks=4)
 
 
+def test_lowrank_4x1024_b256_plain_newton(sb):
+    """The 4 x 1024^2 workload with the plain (degree-1) coupled Newton step."""
+    wl = workloads.workload("lowrank", solver=workloads.SOLVER_NEWTON)
+    run_workload(sb, wl, steps=11, k_blocks=4)
+
+
+def test_gpt2_small_shapes_b512_plain_newton(sb):
+    """GPT-2-small layer shapes with the plain (degree-1) coupled Newton step."""
+    wl = workloads.workload("gpt2", solver=workloads.SOLVER_NEWTON)
+    run_workload(sb, wl, steps=2, k_blocks=6)
+
+
 def test_gpt2_small_shapes_b512(sb):
     """GPT-2-small layer shapes (456 blocks of 512, 252 ragged), root every step."""
     wl = workloads.workload("gpt2")

@@ -412,3 +412,49 @@ def test_spectral_scale_keeps_the_root_and_saves_iterations():
     lam = np.linalg.eigvalsh(A + eps * np.eye(256))[-1]
     est = im.power_estimate(A + eps * np.eye(256))
     assert 0.9 * lam <= est <= lam * (1 + 1e-12)
+
+
+@pytest.mark.parametrize("p", [2, 4])
+def test_correction_polynomial_is_third_order_in_the_scalar_root(p):
+    """The degree-2 correction T(mu) = c0 + c1 x + c2 x^2 (x = 1 - mu) must be
+    the Taylor polynomial of mu^{-1/p} about 1: its error against the power
+    function shrinks like x^3, with leading coefficient (1/p)(1/p + 1)(1/p + 2)/6.
+    A wrong c1 leaves an O(x) error, a wrong c2 an O(x^2) one."""
+    lead = (1 / p) * (1 / p + 1) * (1 / p + 2) / 6
+    for x in (1e-2, 2e-3):
+        mu = 1.0 - x
+        T = oim.correction(np.array([[mu]]), p, 2)[0, 0]
+        assert (mu ** (-1.0 / p) - T) / x ** 3 == pytest.approx(lead, rel=0.05)
+    # degree 1 is the coupled-Newton T = ((p + 1) - mu) / p
+    assert oim.correction(np.array([[0.3]]), p, 1)[0, 0] == pytest.approx((p + 1 - 0.3) / p)
+
+
+@pytest.mark.parametrize("p", [2, 4])
+def test_correction_keeps_eigenvalues_increasing_below_one(p):
+    """Truncating a series of positive terms underestimates mu^{-1/p}, so the
+    eigenvalue map mu -> mu T(mu)^p sends (0, 1] into (mu, 1]: the iterates
+    grow monotonically to 1 and the trace residual stays a bound.  Near 0 the
+    growth factor is (c0 + c1 + c2)^p."""
+    mu = np.concatenate([np.logspace(-24, -1, 200), np.linspace(0.1, 1.0, 400)])
+    f = np.array([m * oim.correction(np.array([[m]]), p, 2)[0, 0] ** p for m in mu])
+    assert np.all(f <= 1.0 + 1e-15) and np.all(f[:-1] > mu[:-1])
+    growth = f[0] / mu[0]
+    assert growth == pytest.approx(sum(oim.binomial_coefficients(p, 2)) ** p, rel=1e-6)
+    assert growth > ((p + 1) / p) ** p * 1.4
+
+
+@pytest.mark.parametrize("p", [2, 4])
+def test_cubic_newton_mirror_reaches_the_exact_root_in_fewer_iterations(p):
+    """Both correction degrees converge to the eigendecomposition root; the
+    degree-2 one in at most three quarters of the iterations on a spectrum
+    spanning 1e6, and a diagonal input gives the scalar closed form."""
+    A = workloads.spd_batch(1, 48, 1e6, seed=23)[0]
+    ref = oracle.inverse_root(A, p, 0.0)
+    X1, k1, _ = oim.coupled_newton(A, p, 0.0, 80, tol=1e-12, trace_tol=True)
+    X2, k2, _ = oim.coupled_newton(A, p, 0.0, 80, tol=1e-12, trace_tol=True, degree=2)
+    assert osh.rel_fro(X1, ref) < 1e-8 and osh.rel_fro(X2, ref) < 1e-8
+    assert k2 <= 0.75 * k1, (k1, k2)
+    d = np.array([1.0, 0.5, 1e-3, 1e-5])
+    Xd, _, _ = oim.coupled_newton(np.diag(d), p, 0.0, 80, tol=1e-14, trace_tol=True, degree=2)
+    assert np.allclose(np.diag(Xd), d ** (-1.0 / p), rtol=1e-10)
+    assert np.abs(Xd - np.diag(np.diag(Xd))).max() == 0.0

@@ -33,6 +33,7 @@ import numpy as np
 SOLVER_NEWTON = 0
 SOLVER_NEWTON_DB = 1
 SOLVER_CHEBYSHEV = 2
+SOLVER_NEWTON_CUBIC = 3
 
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
@@ -81,15 +82,15 @@ WORKLOADS = {
         steps=10, seed=1234 + 0),
     "lowrank": Workload(
         name="lowrank", shapes=((1024, 1024),) * 4, block=256, beta=0.95,
-        eps=1e-8, lr=1e-3, root_p=4, solver=SOLVER_NEWTON, iters=40, tol=1e-5,
+        eps=1e-8, lr=1e-3, root_p=4, solver=SOLVER_NEWTON_CUBIC, iters=40, tol=1e-5,
         refresh_every=10, steps=100, seed=1234 + 1),
     "gpt2": Workload(
         name="gpt2", shapes=_gpt2_shapes(), block=512, beta=0.999, eps=1e-12,
-        lr=1e-3, root_p=4, solver=SOLVER_NEWTON, iters=40, tol=1e-5,
+        lr=1e-3, root_p=4, solver=SOLVER_NEWTON_CUBIC, iters=40, tol=1e-5,
         refresh_every=1, steps=10, seed=1234 + 2),
     "llama": Workload(
         name="llama", shapes=_llama_shapes(), block=1024, beta=0.999,
-        eps=1e-10, lr=1e-3, root_p=4, solver=SOLVER_NEWTON, iters=40, tol=1e-5,
+        eps=1e-10, lr=1e-3, root_p=4, solver=SOLVER_NEWTON_CUBIC, iters=40, tol=1e-5,
         refresh_every=10, grad_dtype=DTYPE_BF16, steps=20, seed=1234 + 3),
 }
 
