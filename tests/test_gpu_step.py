@@ -196,3 +196,33 @@ def test_launch_count_increases(sb):
     torch.cuda.synchronize()
     # stack + stats + norm + prologue + 20 + 19 * 2 Newton launches + finalize + 2 apply
     assert sb.launch_count() - n0 == 1 + 1 + 1 + 1 + 20 + 19 * 2 + 1 + 2
+
+
+@pytest.mark.parametrize("block,shape", [(512, (700, 1024)), (1024, (1024, 2048))])
+def test_large_blocks_parity(sb, block, shape):
+    """Blocks of 512 (with a ragged block row of 188) and 1024 with the
+    workloads' solver: every statistic matches the float64 oracle and every
+    root passes its gate, over two steps with beta 0.9."""
+    wl = workloads.workload("tiny", shapes=(shape,), block=block, steps=2, iters=30, tol=1e-5, beta=0.9, eps=1e-4,
+                            solver=workloads.SOLVER_NEWTON_CUBIC)
+    opt = sb.Shampoo(wl.shapes, sb.config_from_workload(wl))
+    W = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    ref = oracle.ShampooOracle(wl.shapes, wl.block, wl.beta, wl.eps, wl.lr, wl.root_p, wl.refresh_every)
+    stream = workloads.GradientStream(wl)
+    for t in range(wl.steps):
+        G = stream.next()
+        opt.step(W, [torch.from_numpy(g).cuda() for g in G])
+        ref.step(G)
+    torch.cuda.synchronize()
+    L, R = opt.statistics()
+    L, R = L.cpu().numpy(), R.cpu().numpy()
+    for b, blk in enumerate(ref.table):
+        assert oracle.rel_fro(L[b, :blk.r, :blk.r].astype(np.float64), ref.L[b]) < TOL_STATS
+        assert oracle.rel_fro(R[b, :blk.c, :blk.c].astype(np.float64), ref.R[b]) < TOL_STATS
+    XL, XR = opt.roots()
+    XL, XR = XL.cpu().numpy().astype(np.float64), XR.cpu().numpy().astype(np.float64)
+    for b, blk in enumerate(ref.table):
+        for X, S, v in ((XL, ref.L[b], blk.r), (XR, ref.R[b], blk.c)):
+            er, gate, _ = root_checks(X[b, :v, :v], S, wl.root_p, wl.eps)
+            assert er < gate, (b, er, gate)
+    assert opt.status() & ~sb.DEVFLAG_STAGNATED == 0
