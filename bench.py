@@ -531,7 +531,11 @@ def run_reference(args, wl):
 def run_sweep(args):
     """Inverse-root solver sweep: stacked fp32 SPD matrices Q diag(lam) Q^T
     (Haar Q, log-uniform lam with condition number kappa), one
-    inv_root_batched call per step through the C ABI."""
+    inv_root_batched call per step through the C ABI.  With --sweep-grid every
+    (n, kappa, p, solver) of the sweep runs in turn, one JSON line each:
+    n in {256, 512, 1024}, kappa in {1e2, 1e4, 1e6, 1e8}, p in {2, 4}; coupled
+    Newton (both correction degrees) and Newton-DB residual-checked
+    (tol 1e-5, cap 40), Chebyshev at degrees 16 and 32."""
     import torch
     import shampoo_family_second_b200 as sb
 
@@ -543,10 +547,38 @@ def run_sweep(args):
         dist.init_process_group(backend="nccl", timeout=timedelta(seconds=120))
     device = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
-    n, kappa, p = args.sweep_n, args.sweep_kappa, args.sweep_p
+    if not args.sweep_grid:
+        sweep_case(args, sb, device, stream, rank, world, args.sweep_n, args.sweep_kappa, args.sweep_p,
+                   args.sweep_solver, args.sweep_iters, args.sweep_tol, args.sweep_degree)
+    else:
+        for n in (256, 512, 1024):
+            for kappa in (1e2, 1e4, 1e6, 1e8):
+                for p in (2, 4):
+                    for name, degree in (("newton", 0), ("newton_cubic", 0), ("newton_db", 0),
+                                         ("chebyshev", 16), ("chebyshev", 32)):
+                        sweep_case(args, sb, device, stream, rank, world, n, kappa, p, name, 40,
+                                   0.0 if name == "chebyshev" else 1e-5, degree or args.sweep_degree)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+_SWEEP_INPUT = {}
+
+
+def sweep_case(args, sb, device, stream, rank, world, n, kappa, p, solver_name, sweep_iters, sweep_tol,
+               sweep_degree):
+    """One (n, kappa, p, solver) case of the sweep: W untimed and K timed calls."""
+    import torch
     batch = args.sweep_batch or SWEEP_BATCH.get(n, 64)
-    solver = SOLVER_IDS[args.sweep_solver]
-    A64, Q64, lam64 = workloads.spd_batch(batch, n, kappa, seed=4321 + n + rank, return_parts=True)
+    solver = SOLVER_IDS[solver_name]
+    key = (batch, n, kappa, rank)
+    if _SWEEP_INPUT.get("key") != key:  # the grid reuses one input set across p and solvers
+        _SWEEP_INPUT.clear()
+        _SWEEP_INPUT["key"] = key
+        _SWEEP_INPUT["parts"] = workloads.spd_batch(batch, n, kappa, seed=4321 + n + rank, return_parts=True)
+    A64, Q64, lam64 = _SWEEP_INPUT["parts"]
     A = torch.from_numpy(A64.astype(np.float32)).to(device)
     X = torch.empty_like(A)
     scratch = torch.empty(sb.inv_root_scratch_bytes(batch, n, solver), dtype=torch.uint8, device=device)
@@ -554,7 +586,7 @@ def run_sweep(args):
     status = torch.zeros(1, dtype=torch.int32, device=device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     lo = 0.999 / kappa if solver == 2 else 0.0
-    kw = dict(p=p, eps=0.0, solver=solver, iters=args.sweep_iters, tol=args.sweep_tol, cheb_degree=args.sweep_degree,
+    kw = dict(p=p, eps=0.0, solver=solver, iters=sweep_iters, tol=sweep_tol, cheb_degree=sweep_degree,
               cheb_lo=lo, out=X, scratch=scratch, stream=stream)
 
     def one():
@@ -602,9 +634,9 @@ def run_sweep(args):
             "metric": METRIC, "value": job_throughput(batch * args.steps, world, total_ms), "unit": "inverse-roots/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": f"inverse_root_sweep_{batch}x{n}sq_kappa{kappa:.0e}_p{p}_{args.sweep_solver}",
-                       "n": n, "batch": batch, "kappa": kappa, "p": p, "solver": args.sweep_solver,
-                       "iters": args.sweep_iters, "tol": args.sweep_tol, "degree": args.sweep_degree,
+            "config": {"workload": f"inverse_root_sweep_{batch}x{n}sq_kappa{kappa:.0e}_p{p}_{solver_name}{sweep_degree if solver == 2 else ''}",
+                       "n": n, "batch": batch, "kappa": kappa, "p": p, "solver": solver_name,
+                       "iters": sweep_iters, "tol": sweep_tol, "degree": sweep_degree,
                        "l2": "256 MiB buffer written between timed calls, outside the events"},
             "iters_used": [int(it_host.min()), int(it_host.max())], "device_status": int(status.item()),
             "rel_err_vs_construction_sample": errs, "gpu_launches": int(launches), "clocks": clk,
@@ -613,10 +645,6 @@ def run_sweep(args):
                          "launches": g.launches, "avg_launch_ms": g.total_ms / max(g.launches, 1),
                          "peak_basis": f"{src} bf16 sustained x 1.1/2.25 / 3"},
         }), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
 
 
 def main():
@@ -639,6 +667,7 @@ def main():
     ap.add_argument("--sweep-iters", type=int, default=25)
     ap.add_argument("--sweep-tol", type=float, default=0.0)
     ap.add_argument("--sweep-degree", type=int, default=32)
+    ap.add_argument("--sweep-grid", action="store_true", help="run every (n, kappa, p, solver) case of the sweep")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -140,6 +140,15 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, ui
 
 // Orders this thread's ordinary shared-memory stores before later accesses
 // by the async proxy (the tensor core's operand reads, TMA writes).
+// 16-byte asynchronous copy global -> shared (cp.async, cached at L2 only),
+// and waiting for all of this thread's outstanding ones.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -95,17 +95,38 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmLaunch& L, int tile) {
   return c;
 }
 
+// Stages the C rows of the 32 x 32 chunk at (row0, c0) into the warp's shared
+// tile with asynchronous 16-byte copies, in the tile's swizzled layout (piece
+// k of row R at R * 32 + ((k ^ (R & 7)) << 2)); each 8-lane group copies one
+// 128-byte row piece.  The copies are waited for in epilogue_chunk.
+__device__ __forceinline__ void stage_c(const Epilogue& E, int n, int mat, int row0, int c0, float* tilebuf,
+                                        int lane) {
+  const float* base = E.C + static_cast<size_t>(mat) * n * n + static_cast<size_t>(row0) * n + c0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int R = 4 * j + (lane >> 3);
+    const int k = lane & 7;
+    cp_async_16(tilebuf + R * 32 + ((k ^ (R & 7)) << 2), base + static_cast<size_t>(R) * n + 4 * k);
+  }
+  cp_async_commit();
+}
+
 // Epilogue of one 32 x 32 chunk: rows row0 .. row0+31 (row row0 + lane in this
 // thread's registers, acc = its 32 sums for columns c0 .. c0+31).
-//   phase 1  each thread writes alpha * acc + gamma [r == c] for its row into
-//            the warp's shared tile (16-byte pieces XOR-swizzled by the row, so
-//            neither phase has bank conflicts) and adds its diagonal term to
-//            the residual;
+//   phase 0  (C set) the chunk's C rows arrive in the warp's shared tile by
+//            asynchronous copies (issued here, or earlier when c_staged), so
+//            all 32 rows are in flight at once and none waits on a register;
+//   phase 1  each thread writes alpha * acc + beta C + gamma [r == c] for its
+//            row into the warp's shared tile (16-byte pieces XOR-swizzled by
+//            the row, so neither phase has bank conflicts; C is read from the
+//            same place first) and adds its diagonal term to the residual;
 //   phase 2  each quarter-warp takes one row: 8 lanes x 16 bytes = one
-//            128-byte piece; beta C, the scale, the outputs D, E and the
-//            weight update are applied there.
+//            128-byte piece; the scale, the outputs D, E and the weight update
+//            are applied there.
+// Each element of C is read before the same thread group's store of that
+// element, so C may be the output D (statistics updated in place).
 __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int row0, int c0, const float* acc,
-                                               float* tilebuf, int lane, float& resid, bool& bad) {
+                                               float* tilebuf, int lane, float& resid, bool& bad, bool c_staged) {
   const Epilogue& E = G.ep;
   const int n = G.n;
   const int r = row0 + lane;
@@ -117,14 +138,27 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
     for (int j = 0; j < 32; ++j)
       if (j == dj && r < vsz) resid += 1.f - acc[j];
   }
+  if (E.C) {
+    if (!c_staged) stage_c(E, n, mat, row0, c0, tilebuf, lane);
+    cp_async_wait_all();
+    __syncwarp();
+  }
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
+    float4* slot = reinterpret_cast<float4*>(tilebuf + lane * 32 + ((k ^ (lane & 7)) << 2));
     float4 w;
     w.x = E.alpha * acc[4 * k + 0] + ((4 * k + 0 == dj) ? gam : 0.f);
     w.y = E.alpha * acc[4 * k + 1] + ((4 * k + 1 == dj) ? gam : 0.f);
     w.z = E.alpha * acc[4 * k + 2] + ((4 * k + 2 == dj) ? gam : 0.f);
     w.w = E.alpha * acc[4 * k + 3] + ((4 * k + 3 == dj) ? gam : 0.f);
-    *reinterpret_cast<float4*>(tilebuf + lane * 32 + ((k ^ (lane & 7)) << 2)) = w;
+    if (E.C) {
+      const float4 c = *slot;
+      w.x += E.beta * c.x;
+      w.y += E.beta * c.y;
+      w.z += E.beta * c.z;
+      w.w += E.beta * c.w;
+    }
+    *slot = w;
   }
   __syncwarp();
   const size_t nn = static_cast<size_t>(n) * n;
@@ -146,13 +180,6 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
     float4 v = *reinterpret_cast<const float4*>(tilebuf + R * 32 + ((kq ^ (R & 7)) << 2));
     if (gr < n) {
       const size_t off = static_cast<size_t>(mat) * nn + static_cast<size_t>(gr) * n + gc;
-      if (E.C) {
-        const float4 c = *reinterpret_cast<const float4*>(E.C + off);
-        v.x += E.beta * c.x;
-        v.y += E.beta * c.y;
-        v.z += E.beta * c.z;
-        v.w += E.beta * c.w;
-      }
       v.x *= sc;
       v.y *= sc;
       v.z *= sc;
@@ -401,6 +428,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       const GemmGroup& G = L.g[tc.gi];
       const int n = G.n;
       const int nseg = (n / BK + SEG - 1) / SEG;
+      // C of this warp's first chunk streams into its shared tile while the
+      // tile's MMAs run.
+      const int row0_first = tc.tm * BM + q * 32;
+      const int c0_first = tc.tn * BN + h * (BN / 2);
+      const bool staged0 = G.ep.C && row0_first < n && c0_first < n;
+      if (staged0) stage_c(G.ep, n, tc.mat, row0_first, c0_first, tilebuf, lane);
       float sum[BN / 2];
 #pragma unroll
       for (int j = 0; j < BN / 2; ++j) sum[j] = 0.f;
@@ -424,7 +457,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
       }
-      if (!ok) break;
+      if (!ok) {
+        cp_async_wait_all();  // no copy may still be landing when the CTA retires
+        break;
+      }
       float resid = 0.f;
       bool nonfinite = false;
       const int row0 = tc.tm * BM + q * 32;
@@ -432,7 +468,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c) {
           const int c0 = tc.tn * BN + h * (BN / 2) + c * 32;
-          if (c0 < n) epilogue_chunk(G, tc.mat, row0, c0, &sum[c * 32], tilebuf, lane, resid, nonfinite);
+          if (c0 < n) epilogue_chunk(G, tc.mat, row0, c0, &sum[c * 32], tilebuf, lane, resid, nonfinite, c == 0 && staged0);
         }
       }
       if (G.ep.res) {
