@@ -12,8 +12,10 @@
  *     W <- W - lr * XL G XR                                  (update)
  * with p = 4 by default (the notes' -1/4 powers) and p = 2 allowed (SOAP
  * abstract: Shampoo with the 1/2 power).  The roots come from an iterative
- * solver (coupled Newton, Newton-DB or Chebyshev) on Frobenius-scaled, damped
- * statistics.  All products run on the tensor cores as 3xTF32 (fp32-accurate)
+ * solver (coupled Newton with a first- or second-degree correction, Newton-DB
+ * or Chebyshev) on scaled, damped statistics (coupled Newton: the smaller of the
+ * Frobenius norm and 1.25 x a power-iteration estimate of the largest
+ * eigenvalue; the others: the Frobenius norm).  All products run on the tensor cores as 3xTF32 (fp32-accurate)
  * tcgen05 MMAs.
  *
  * Conventions (all entry points):
@@ -106,9 +108,11 @@ enum {
  *  iters          iterations (tol = 0) or iteration cap (tol > 0) per Newton / Newton-DB
  *                 stage, >= 1; ignored by Chebyshev.  NEWTON_CUBIC behaves as NEWTON here.
  *  tol            0: fixed iteration count; > 0: stop a matrix once
- *                 tr(I - M)/n (Newton) or tr(I - Z Y)/n (Newton-DB) <= tol.  Both iterations
- *                 keep every eigenvalue of M (or Z Y) at or below 1, so this trace bounds the
- *                 largest eigenvalue error (times n).
+ *                 |tr(I - M)|/n (Newton) or |tr(I - Z Y)|/n (Newton-DB) <= tol.  The
+ *                 iterations keep every eigenvalue of M (or Z Y) at or below 1, so this trace
+ *                 bounds the largest eigenvalue error (times n).  A matrix whose residual
+ *                 stops improving once every eigenvalue above fp32 resolution has converged
+ *                 stops there (SHAMPOO_DEVFLAG_STAGNATED).
  *  refresh_every  roots recomputed at steps t with t % refresh_every == 0 (t from 0), >= 1.
  *  cheb_degree    Chebyshev degree d in [2, 64].
  *  cheb_lo        Chebyshev interval: [lo / s, 1] with lo = cheb_lo if > 0 else eps,

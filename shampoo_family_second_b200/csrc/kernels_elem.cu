@@ -370,8 +370,7 @@ __global__ void __launch_bounds__(1024) check_kernel(float* res, float* prev, in
 
 // Output pass: X = sym(final iterate) * s^{-1/p}, with sym(Y) = (Y + Y^T)/2.
 // The principal root is symmetric; the iterates pick up a small
-// antisymmetric rounding component (the products are formed as A B^T), which
-// this removes.  The final iterate sits in buffer (iters[i] & 1).
+// antisymmetric rounding component, which this removes.  The final iterate sits in buffer (iters[i] & 1).
 // grid (n/32, n/32, batch), block (32, 8).
 __global__ void finalize_kernel(const float* __restrict__ X0, const float* __restrict__ X1,
                                 const int* __restrict__ iters, int default_iters, const float* __restrict__ sc, int n,

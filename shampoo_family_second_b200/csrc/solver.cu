@@ -11,10 +11,12 @@
 //   coupled Newton, second-degree correction: the same coupled form with T
 //                   the degree-2 truncation of the binomial series of
 //                   M^{-1/p} = (I - (I - M))^{-1/p}; the degree-1 truncation is
-//                   the Newton T above.  One more GEMM per iteration (T needs
-//                   M^2), cubic local convergence, and an eigenvalue mu << 1
-//                   of M grows by (1 + c1 + c2)^p instead of ((p+1)/p)^p per
-//                   iteration (3.91 against 2.44 at p = 4);
+//                   the Newton T above.  One more GEMM per iteration (T is
+//                   formed from D = I - M, which the M update writes, as
+//                   c2 D D + c1 D + I), cubic local convergence, and an
+//                   eigenvalue mu << 1 of M grows by (1 + c1 + c2)^p instead
+//                   of ((p+1)/p)^p per iteration (3.91 against 2.44 at p = 4);
+//                   the first iteration is a plain Newton step;
 //   Newton-DB       coupled Denman-Beavers-family square-root iteration in its
 //                   multiplication-only form: Y0 = A', Z0 = I;
 //                   T = (3 I - Z Y)/2; Y <- Y T; Z <- T Z (3 GEMMs); p = 4 runs
@@ -36,13 +38,14 @@
 // A B^T (the error grows about 1.5x per iteration): true products as well.
 // The Clenshaw recurrence is a fixed number of steps with no fixed point to
 // shift and keeps A B^T.
-// Convergence is measured by tr(I - M)/n (Newton) or tr(I - Z Y)/n (Newton-DB):
-// both iterations keep every eigenvalue of M (or Z Y) at or below 1, so the
-// trace bounds the largest eigenvalue error and ignores the antisymmetric
-// rounding component.
-// A' = (A + eps I)/||A + eps I||_F (Frobenius pre-scaling); the result is
-// unscaled by ||A + eps I||_F^{-1/p}.  With tol > 0 the residual
-// tr(I - M)/n (Newton) or tr(I - Z Y)/n (Newton-DB) is checked after every
+// Convergence is measured by |tr(I - M)|/n (Newton) or |tr(I - Z Y)|/n
+// (Newton-DB): the iterations keep every eigenvalue of M (or Z Y) at or below
+// 1 in exact arithmetic, so the trace bounds the largest eigenvalue error and
+// ignores any antisymmetric rounding component.
+// A' = (A + eps I)/s, unscaled by s^{-1/p} at the end.  Newton-DB and
+// Chebyshev take s = ||A + eps I||_F (Frobenius pre-scaling); coupled Newton
+// takes s = min(||A + eps I||_F, 1.25 x a power-iteration estimate of the
+// largest eigenvalue).  With tol > 0 the residual is checked after every
 // iteration and converged matrices drop out of later launches (their tiles
 // exit at once); iters is then the cap.
 #include <algorithm>
