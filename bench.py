@@ -422,13 +422,31 @@ def run_ours(args, wl):
 TRAFFIC_SOURCES = ("gemm_tc.cu", "solver.cu", "api.cu")
 
 
-def traffic_source_sha():
-    """sha256 over the sources that decide the GEMM launch mix of a step."""
+def code_only(text):
+    """C++ source without comments and blank space (the traffic record tracks
+    code, not its comments)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    lines = []
+    for line in text.splitlines():
+        line = re.sub(r"//.*$", "", line).strip()
+        if line:
+            lines.append(" ".join(line.split()))
+    return "\n".join(lines)
+
+
+def traffic_source_sha(read=None):
+    """sha256 over the code (comments dropped) of the sources that decide the
+    GEMM launch mix of a step.  `read(name)` returns a source's text (default:
+    the working tree)."""
     import hashlib
+    if read is None:
+        def read(name):
+            with open(os.path.join(ROOT, "shampoo_family_second_b200", "csrc", name)) as f:
+                return f.read()
     h = hashlib.sha256()
     for name in TRAFFIC_SOURCES:
-        with open(os.path.join(ROOT, "shampoo_family_second_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        h.update(code_only(read(name)).encode())
     return h.hexdigest()
 
 
