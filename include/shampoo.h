@@ -166,6 +166,15 @@ SHAMPOO_API int shampoo_init(const shampoo_config* cfg, int32_t nparams, const i
  * of nparams device pointers.  Enqueued on `stream`; no host sync. */
 SHAMPOO_API int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d_grads, void* stream);
 
+/* shampoo_step on strided views: ld (host, nparams entries; NULL = cols) gives
+ * the row stride, in elements, of d_weights[i] and d_grads[i] alike (cols[i] <=
+ * ld[i] < 2^31).  A parameter can then be a sub-matrix of a larger weight, e.g.
+ * the blocks one rank owns when the blocks are sharded across ranks.
+ * SHAMPOO_ERR_INVALID_ARG for a stride out of range; rows need no alignment
+ * (unaligned rows take the scalar load path). */
+SHAMPOO_API int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* const* d_grads,
+                                     const int64_t* ld, void* stream);
+
 /* Synchronises the handle's last stream, reads the device status word into
  * *status (0 = clean; else SHAMPOO_DEVFLAG_* bits) and returns SHAMPOO_OK, or
  * SHAMPOO_ERR_CUDA if the device reported an error.  reset != 0 clears the word. */

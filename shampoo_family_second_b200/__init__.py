@@ -51,7 +51,7 @@ KERNEL_NAMES = ("gemm3x_tf32", "stack_blocks", "frob_norm", "prologue", "check",
 # Exported symbols, in header order (tests compare this with include/shampoo.h).
 EXPORTS = (
     "shampoo_status_string", "shampoo_last_error", "shampoo_query_sizes", "shampoo_init", "shampoo_step",
-    "shampoo_get_status", "shampoo_block_table", "shampoo_state_views", "shampoo_set_step", "shampoo_destroy",
+    "shampoo_step_strided", "shampoo_get_status", "shampoo_block_table", "shampoo_state_views", "shampoo_set_step", "shampoo_destroy",
     "inv_root_scratch_bytes", "inv_root_batched", "inv_root_batched_noalloc", "shampoo_gemm_scratch_bytes",
     "shampoo_gemm_batched",
     "shampoo_profile_enable", "shampoo_profile_reset", "shampoo_profile_read", "shampoo_launch_count",
@@ -103,6 +103,7 @@ def _load():
         "shampoo_init": (ctypes.c_int, [ctypes.POINTER(Config), I32, ctypes.POINTER(I64), ctypes.POINTER(I64), P,
                                         ctypes.c_size_t, P, ctypes.c_size_t, P, ctypes.POINTER(P)]),
         "shampoo_step": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P), P]),
+        "shampoo_step_strided": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(I64), P]),
         "shampoo_get_status": (ctypes.c_int, [P, ctypes.POINTER(I32), I32]),
         "shampoo_block_table": (ctypes.c_int, [P, ctypes.POINTER(I32), ctypes.POINTER(I64)]),
         "shampoo_state_views": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
@@ -215,6 +216,7 @@ class Shampoo:
         self.nb = nb.value
         self._wbuf = (ctypes.c_void_p * len(self.shapes))()
         self._gbuf = (ctypes.c_void_p * len(self.shapes))()
+        self._ldbuf = (ctypes.c_int64 * len(self.shapes))()
 
     def __del__(self):
         h = getattr(self, "_h", None)
@@ -223,20 +225,32 @@ class Shampoo:
             self._h = None
 
     def step(self, weights, grads, stream=None):
+        """Weights and gradients may be row-strided views (for instance blocks
+        of larger tensors): unit column stride, and the same row stride for a
+        weight and its gradient."""
         import torch
         want = torch.bfloat16 if self.cfg.grad_dtype == BF16 else torch.float32
+        if len(weights) != len(self.shapes) or len(grads) != len(self.shapes):
+            raise ValueError("one weight and one gradient per shape")
+        strided = False
         for i, (w, g) in enumerate(zip(weights, grads)):
             if w.dtype != torch.float32 or g.dtype != want:
                 raise TypeError(f"param {i}: weights must be float32 and grads {want}")
             if tuple(w.shape) != self.shapes[i] or tuple(g.shape) != self.shapes[i]:
                 raise ValueError(f"param {i}: shape mismatch")
-            if not (w.is_contiguous() and g.is_contiguous()):
-                raise ValueError(f"param {i}: tensors must be contiguous")
+            rows, cols = self.shapes[i]
+            ldw = w.stride(0) if rows > 1 else cols
+            ldg = g.stride(0) if rows > 1 else cols
+            if (cols > 1 and (w.stride(1) != 1 or g.stride(1) != 1)) or ldw != ldg or ldw < cols:
+                raise ValueError(f"param {i}: weight and gradient need unit column stride and one row stride")
+            self._ldbuf[i] = ldw
+            strided |= ldw != cols
             self._wbuf[i] = w.data_ptr()
             self._gbuf[i] = g.data_ptr()
-        if len(weights) != len(self.shapes) or len(grads) != len(self.shapes):
-            raise ValueError("one weight and one gradient per shape")
-        _check(lib.shampoo_step(self._h, self._wbuf, self._gbuf, _stream_ptr(stream)))
+        if strided:
+            _check(lib.shampoo_step_strided(self._h, self._wbuf, self._gbuf, self._ldbuf, _stream_ptr(stream)))
+        else:
+            _check(lib.shampoo_step(self._h, self._wbuf, self._gbuf, _stream_ptr(stream)))
 
     def status(self, reset: bool = False) -> int:
         s = ctypes.c_int32(0)

@@ -258,6 +258,11 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
 }
 
 int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d_grads, void* stream) {
+  return shampoo_step_strided(h, d_weights, d_grads, nullptr, stream);
+}
+
+int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* const* d_grads, const int64_t* ld,
+                         void* stream) {
   if (!h) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle is NULL");
   if (!d_weights || !d_grads) return set_error(SHAMPOO_ERR_INVALID_ARG, "weights/grads array is NULL");
   const shampoo_config& c = h->cfg;
@@ -265,11 +270,16 @@ int shampoo_step(shampoo_handle h, float* const* d_weights, const void* const* d
   StackArgs args;
   for (int i = 0; i < h->nparams; ++i) {
     if (!d_weights[i] || !d_grads[i]) return set_error(SHAMPOO_ERR_INVALID_ARG, "param %d has a NULL pointer", i);
+    const int64_t ldi = ld ? ld[i] : h->cols[i];
+    if (ldi < h->cols[i] || ldi > 0x7fffffff)
+      return set_error(SHAMPOO_ERR_INVALID_ARG, "param %d: row stride %lld outside [cols, 2^31)", i,
+                       static_cast<long long>(ldi));
     args.g[i] = d_grads[i];
     args.w[i] = d_weights[i];
-    args.ld[i] = static_cast<int>(h->cols[i]);
+    args.ld[i] = static_cast<int>(ldi);
+    // 16-byte (fp32) / 8-byte (bf16) gradient loads need every row aligned.
     const size_t esize = c.grad_dtype == SHAMPOO_BF16 ? 2 : 4;
-    args.vec[i] = (h->cols[i] % 4 == 0 && reinterpret_cast<uintptr_t>(d_grads[i]) % (4 * esize) == 0) ? 1 : 0;
+    args.vec[i] = (ldi % 4 == 0 && reinterpret_cast<uintptr_t>(d_grads[i]) % (4 * esize) == 0) ? 1 : 0;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;

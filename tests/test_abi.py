@@ -118,3 +118,14 @@ def test_init_rejects_missing_buffers_without_cuda(sb):
     assert sb.lib.shampoo_init(ctypes.byref(cfg), 1, rows, cols, 256, 0, 512, 0, None, ctypes.byref(h)) == -3
     assert sb.lib.shampoo_init(ctypes.byref(cfg), 1, rows, cols, 255, 1 << 30, 512, 1 << 30, None,
                                ctypes.byref(h)) == -2
+
+
+def test_strided_step_refuses_a_null_handle():
+    """The strided step checks its arguments before any launch: a null handle
+    is refused with ERR_INVALID_ARG without touching the device."""
+    import ctypes
+    sb = pytest.importorskip("shampoo_family_second_b200")
+    ld = (ctypes.c_int64 * 1)(4)
+    w = (ctypes.c_void_p * 1)(None)
+    assert sb.lib.shampoo_step_strided(None, w, w, ld, None) == sb.ERR_INVALID_ARG
+    assert "handle" in sb.last_error()

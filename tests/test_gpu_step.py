@@ -226,3 +226,35 @@ def test_large_blocks_parity(sb, block, shape):
             er, gate, _ = root_checks(X[b, :v, :v], S, wl.root_p, wl.eps)
             assert er < gate, (b, er, gate)
     assert opt.status() & ~sb.DEVFLAG_STAGNATED == 0
+
+
+def test_strided_block_views_match_the_full_step(sb):
+    """Blocks are independent: the weights' blocks, given to the optimizer as
+    strided views (each block a parameter of its own, via the strided step),
+    end with exactly the weights of the optimizer over the full weights, and
+    so does the sharded optimizer on a single rank (one process, which owns
+    every block).  One weight has rows of 70 floats (no vector loads)."""
+    from shampoo_family_second_b200 import sharded
+    shapes = ((96, 80), (40, 70))
+    wl = workloads.workload("tiny", shapes=shapes, block=32, steps=3, iters=30, tol=1e-5, beta=0.9, eps=1e-4,
+                            solver=workloads.SOLVER_NEWTON_CUBIC)
+    cfg = sb.config_from_workload(wl)
+    blocks = sharded.block_list(shapes, 32)
+    full = sb.Shampoo(shapes, cfg)
+    per_block = sb.Shampoo([(b[3], b[4]) for b in blocks], cfg)
+    shard = sharded.ShardedShampoo(shapes, cfg)
+    W1, W2, W3 = ([torch.zeros(s, dtype=torch.float32, device="cuda") for s in shapes] for _ in range(3))
+    stream = workloads.GradientStream(wl)
+
+    def views(T):
+        return [T[p][r0:r0 + r, c0:c0 + c] for p, r0, c0, r, c in blocks]
+
+    for t in range(wl.steps):
+        G = [torch.from_numpy(g).cuda() for g in stream.next()]
+        full.step(W1, G)
+        per_block.step(views(W2), views(G))
+        shard.step(W3, G)
+    torch.cuda.synchronize()
+    for a, b, c in zip(W1, W2, W3):
+        assert torch.equal(a, b) and torch.equal(a, c)
+    assert full.status() & ~sb.DEVFLAG_STAGNATED == 0 and per_block.status() & ~sb.DEVFLAG_STAGNATED == 0

@@ -1,0 +1,139 @@
+"""Blocks sharded across ranks (shampoo_family_second_b200.sharded), on CPU.
+
+The partition is checked as host logic; the step's communication runs in
+real gloo process groups of world size 2, with the float64 oracle standing in
+for each rank's block compute (the CUDA optimizer cannot run on CPU ranks).
+Every rank must end with the same weights, equal to a single process that
+steps all blocks itself.
+"""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import oracle  # noqa: E402
+from shampoo_family_second_b200 import sharded  # noqa: E402
+
+SHAPES = [(96, 80), (40, 70), (64, 64)]
+B = 32
+HP = dict(beta=0.9, eps=1e-4, lr=1e-2, root_p=4, refresh_every=2)
+STEPS = 3
+
+
+class Cfg:
+    block = B
+
+
+def oracle_local_step(blocks):
+    """The float64 oracle over the given blocks, each a parameter of its own."""
+    ref = oracle.ShampooOracle([(b[3], b[4]) for b in blocks], B, HP["beta"], HP["eps"], HP["lr"], HP["root_p"],
+                               HP["refresh_every"])
+
+    def step(ws, gs):
+        P = ref.step([g.numpy() for g in gs])
+        for k, w in enumerate(ws):
+            w -= torch.from_numpy(HP["lr"] * P[k]).to(w.dtype)
+    return step
+
+
+def gradients(t, rank=None):
+    """Seeded gradients of step t; with a rank, that rank's local part
+    (rank 0: G + D, rank 1: G - D, averaging to G)."""
+    rng = np.random.default_rng(100 + t)
+    G = [rng.standard_normal(s).astype(np.float32) for s in SHAPES]
+    if rank is None:
+        return [torch.from_numpy(g) for g in G]
+    D = [np.random.default_rng(200 + t).standard_normal(s).astype(np.float32) for s in SHAPES]
+    sign = 1.0 if rank == 0 else -1.0
+    return [torch.from_numpy(g + np.float32(sign) * d) for g, d in zip(G, D)]
+
+
+def run_single(grads_reduced):
+    blocks = sharded.block_list(SHAPES, B)
+    opt = sharded.ShardedShampoo(SHAPES, Cfg, grads_reduced=grads_reduced, local_step=oracle_local_step(blocks))
+    W = [torch.zeros(s) for s in SHAPES]
+    for t in range(STEPS):
+        if grads_reduced:
+            G = gradients(t)
+        else:  # the average of the two ranks' local gradients, summed as the ranks sum them
+            g0, g1 = gradients(t, 0), gradients(t, 1)
+            G = [(a + b) / 2 for a, b in zip(g0, g1)]
+        opt.step(W, G)
+    return [w.numpy().copy() for w in W]
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, grads_reduced, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        blocks = sharded.block_list(SHAPES, B)
+        owner = sharded.partition_blocks(blocks, world)
+        mine = [blocks[i] for i, k in enumerate(owner) if k == rank]
+        opt = sharded.ShardedShampoo(SHAPES, Cfg, grads_reduced=grads_reduced, local_step=oracle_local_step(mine))
+        W = [torch.zeros(s) for s in SHAPES]
+        for t in range(STEPS):
+            opt.step(W, gradients(t) if grads_reduced else gradients(t, rank))
+        out_q.put((rank, len(mine), [w.numpy().copy() for w in W]))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def two_ranks(grads_reduced):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, grads_reduced, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return res
+
+
+def test_block_list_matches_the_oracle_table():
+    table = oracle.block_table(SHAPES, B)
+    assert sharded.block_list(SHAPES, B) == [(b.param, b.row0, b.col0, b.r, b.c) for b in table]
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 8, 40])
+def test_partition_covers_and_balances(world):
+    blocks = sharded.block_list(SHAPES, B)
+    owner = sharded.partition_blocks(blocks, world)
+    assert owner == sharded.partition_blocks(blocks, world)  # deterministic
+    assert len(owner) == len(blocks) and all(0 <= k < world for k in owner)
+    cost = [b[3] ** 3 + b[4] ** 3 for b in blocks]
+    load = [sum(c for c, k in zip(cost, owner) if k == r) for r in range(world)]
+    # greedy by decreasing cost: no rank exceeds another by more than one block's cost
+    assert max(load) - min(load) <= max(cost)
+    if world == 1:
+        assert set(owner) == {0}
+
+
+@pytest.mark.parametrize("grads_reduced", [True, False])
+def test_two_ranks_match_one_process(grads_reduced):
+    single = run_single(grads_reduced)
+    res = two_ranks(grads_reduced)
+    (r0, n0, W0), (r1, n1, W1) = res
+    assert n0 > 0 and n1 > 0 and n0 + n1 == len(sharded.block_list(SHAPES, B))
+    for a, b, s in zip(W0, W1, single):
+        assert np.array_equal(a, b)               # every rank holds the same weights
+        assert np.allclose(a, s, rtol=0, atol=1e-7), float(np.abs(a - s).max())
+        assert np.abs(s).max() > 1e-3             # the steps did move the weights
