@@ -137,3 +137,17 @@ def test_two_ranks_match_one_process(grads_reduced):
         assert np.array_equal(a, b)               # every rank holds the same weights
         assert np.allclose(a, s, rtol=0, atol=1e-7), float(np.abs(a - s).max())
         assert np.abs(s).max() > 1e-3             # the steps did move the weights
+
+
+@pytest.mark.parametrize("world", [2, 4, 8])
+def test_partition_balance_on_transformer_shapes(world):
+    """GPT-2-small layer shapes at block 512 (456 blocks, 252 ragged): the
+    busiest rank carries at most 2% more root cost than the average."""
+    layer = ((768, 2304), (768, 768), (768, 3072), (3072, 768))
+    shapes = [s for _ in range(12) for s in layer]
+    blocks = sharded.block_list(shapes, 512)
+    assert len(blocks) == 456
+    owner = sharded.partition_blocks(blocks, world)
+    cost = [b[3] ** 3 + b[4] ** 3 for b in blocks]
+    load = [sum(c for c, k in zip(cost, owner) if k == r) for r in range(world)]
+    assert max(load) <= 1.02 * sum(load) / world, load
