@@ -7,7 +7,7 @@ fp32 / bf16 buffers the GPU receives.  Roots are exact (symmetric
 eigendecomposition), not iterative: the iterative solvers of the CUDA path are
 ways of reaching this same result faster.
 
-Readings of the pages that this file fixes (each also listed in the design doc):
+Readings of the pages that this file fixes:
 
 * Blocking: each m x n weight is cut into a ceil(m/B) x ceil(n/B) grid of
   blocks aligned at multiples of B; the last block row / column is ragged.
