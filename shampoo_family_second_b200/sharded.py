@@ -133,8 +133,8 @@ class ShardedShampoo:
             self.local_step([self._view(weights[self.blocks[i][0]], i) for i in mine],
                             [self._view(grads[self.blocks[i][0]], i) for i in mine])
         else:
-            # sum the local gradients by block owner
-            gbuf = torch.zeros(self.world * self.seg_elems, dtype=grads[0].dtype, device=dev)
+            # sum the local gradients by block owner, in fp32 (also for bf16 gradients)
+            gbuf = torch.zeros(self.world * self.seg_elems, dtype=torch.float32, device=dev)
             for rank, seg in enumerate(self.segments):
                 self._pack(grads, seg, gbuf[rank * self.seg_elems:(rank + 1) * self.seg_elems])
             if self.world > 1:
