@@ -233,7 +233,8 @@ def test_strided_block_views_match_the_full_step(sb):
     strided views (each block a parameter of its own, via the strided step),
     end with exactly the weights of the optimizer over the full weights, and
     so does the sharded optimizer on a single rank (one process, which owns
-    every block).  One weight has rows of 70 floats (no vector loads)."""
+    every block), in place and with its blocks packed into contiguous
+    buffers.  One weight has rows of 70 floats (no vector loads)."""
     from shampoo_family_second_b200 import sharded
     shapes = ((96, 80), (40, 70))
     wl = workloads.workload("tiny", shapes=shapes, block=32, steps=3, iters=30, tol=1e-5, beta=0.9, eps=1e-4,
@@ -243,7 +244,8 @@ def test_strided_block_views_match_the_full_step(sb):
     full = sb.Shampoo(shapes, cfg)
     per_block = sb.Shampoo([(b[3], b[4]) for b in blocks], cfg)
     shard = sharded.ShardedShampoo(shapes, cfg)
-    W1, W2, W3 = ([torch.zeros(s, dtype=torch.float32, device="cuda") for s in shapes] for _ in range(3))
+    packed = sharded.ShardedShampoo(shapes, cfg, grads_reduced=False)  # blocks packed into contiguous buffers
+    W1, W2, W3, W4 = ([torch.zeros(s, dtype=torch.float32, device="cuda") for s in shapes] for _ in range(4))
     stream = workloads.GradientStream(wl)
 
     def views(T):
@@ -254,7 +256,8 @@ def test_strided_block_views_match_the_full_step(sb):
         full.step(W1, G)
         per_block.step(views(W2), views(G))
         shard.step(W3, G)
+        packed.step(W4, G)
     torch.cuda.synchronize()
-    for a, b, c in zip(W1, W2, W3):
-        assert torch.equal(a, b) and torch.equal(a, c)
+    for a, b, c, d in zip(W1, W2, W3, W4):
+        assert torch.equal(a, b) and torch.equal(a, c) and torch.equal(a, d)
     assert full.status() & ~sb.DEVFLAG_STAGNATED == 0 and per_block.status() & ~sb.DEVFLAG_STAGNATED == 0
