@@ -23,7 +23,13 @@ Readings of the pages that this file fixes:
   steps, counting from step 0) recompute the roots, then apply the update
   with the current roots (podcast cue 28: roots refreshed only every so many
   steps; the notes' listing: preconditioners before parameters).
-* No momentum and no grafting: the update uses the raw gradient.
+* No grafting.  Momentum is off by default (the update uses the raw
+  gradient); ``momentum = alpha > 0`` folds ordinary momentum in before
+  preconditioning (podcast cue 28: momentum 0.9 ahead of the
+  preconditioner): per block M <- alpha M + G from M = 0, the statistics still
+  take the raw G, and the update is XL M XR.
+* The diagonal variant for dimensions above about 1200 (podcast cue 28) never
+  applies to blocks, whose sides are at most the block size (<= 1024).
 """
 from __future__ import annotations
 
@@ -111,7 +117,7 @@ class ShampooOracle:
     """
 
     def __init__(self, shapes, block, beta, eps, lr, root_p=4, refresh_every=1,
-                 weights=None, blocks: Sequence[int] | None = None):
+                 weights=None, blocks: Sequence[int] | None = None, momentum: float = 0.0):
         self.shapes = [tuple(s) for s in shapes]
         self.B = int(block)
         self.beta = float(beta)
@@ -130,6 +136,8 @@ class ShampooOracle:
         self.R = {b: np.zeros((self.table[b].c,) * 2) for b in self.active}
         self.XL = {b: None for b in self.active}
         self.XR = {b: None for b in self.active}
+        self.momentum = float(momentum)
+        self.M = {b: np.zeros((self.table[b].r, self.table[b].c)) for b in self.active}
         self.t = 0
 
     def block_of(self, grads, b):
@@ -147,7 +155,11 @@ class ShampooOracle:
             if refresh:
                 self.XL[b] = inverse_root(self.L[b], self.p, self.eps)
                 self.XR[b] = inverse_root(self.R[b], self.p, self.eps)
-            P[b] = precondition(self.XL[b], G, self.XR[b])
+            if self.momentum > 0.0:
+                self.M[b] = self.momentum * self.M[b] + G
+                P[b] = precondition(self.XL[b], self.M[b], self.XR[b])
+            else:
+                P[b] = precondition(self.XL[b], G, self.XR[b])
             blk = self.table[b]
             self.W[blk.param][blk.row0:blk.row0 + blk.r,
                               blk.col0:blk.col0 + blk.c] -= self.lr * P[b]

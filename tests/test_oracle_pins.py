@@ -458,3 +458,53 @@ def test_cubic_newton_mirror_reaches_the_exact_root_in_fewer_iterations(p):
     Xd, _, _ = oim.coupled_newton(np.diag(d), p, 0.0, 80, tol=1e-14, trace_tol=True, degree=2)
     assert np.allclose(np.diag(Xd), d ** (-1.0 / p), rtol=1e-10)
     assert np.abs(Xd - np.diag(np.diag(Xd))).max() == 0.0
+
+
+# ---------------------------------------------------------------- momentum (podcast cue 28)
+
+@pytest.mark.parametrize("alpha", [0.5, 0.9])
+def test_momentum_constant_gradient_geometric_sum(alpha):
+    """A constant gradient G every step: the momentum buffer after t + 1 steps
+    is (1 + alpha + ... + alpha^t) G, so the preconditioned direction is the
+    momentum-free one scaled by (1 - alpha^(t+1)) / (1 - alpha), while the
+    statistics (and therefore the roots) are those of the raw gradient."""
+    rng = np.random.default_rng(41)
+    G = rng.standard_normal((24, 16))
+    kw = dict(shapes=[(24, 16)], block=32, beta=1.0, eps=1e-3, lr=1e-2, root_p=4, refresh_every=1)
+    plain = osh.ShampooOracle(**kw)
+    mom = osh.ShampooOracle(**kw, momentum=alpha)
+    for t in range(5):
+        Pp = plain.step([G])[0]
+        Pm = mom.step([G])[0]
+        factor = (1.0 - alpha ** (t + 1)) / (1.0 - alpha)
+        assert osh.rel_fro(Pm, factor * Pp) < 1e-12
+        assert np.array_equal(mom.L[0], plain.L[0]) and np.array_equal(mom.R[0], plain.R[0])
+
+
+def test_momentum_zero_is_the_plain_step():
+    rng = np.random.default_rng(42)
+    kw = dict(shapes=[(40, 70)], block=32, beta=0.9, eps=1e-4, lr=1e-2, root_p=4, refresh_every=2)
+    a, b = osh.ShampooOracle(**kw), osh.ShampooOracle(**kw, momentum=0.0)
+    for _ in range(3):
+        g = [rng.standard_normal((40, 70))]
+        Pa, Pb = a.step(g), b.step(g)
+        assert all(np.array_equal(Pa[k], Pb[k]) for k in Pa)
+    assert all(np.array_equal(x, y) for x, y in zip(a.W, b.W))
+
+
+def test_momentum_alternating_gradient_closed_form():
+    """Gradients G, -G, G, ...: the buffer is G (1 - alpha + alpha^2 - ...),
+    i.e. M_t = G (1 - (-alpha)^(t+1)) / (1 + alpha) times the sign of step t;
+    with fixed roots (refreshed at step 0 only, beta = 1 keeps G G^T growing
+    but roots stay those of step 0) the directions follow that closed form."""
+    alpha = 0.9
+    rng = np.random.default_rng(43)
+    G = rng.standard_normal((16, 24))
+    kw = dict(shapes=[(16, 24)], block=32, beta=1.0, eps=1e-3, lr=1e-2, root_p=4, refresh_every=1000)
+    mom = osh.ShampooOracle(**kw, momentum=alpha)
+    P0 = mom.step([G])[0]  # step 0: M = G, roots of G G^T
+    for t in range(1, 6):
+        sign = -1.0 if t % 2 else 1.0
+        P = mom.step([sign * G])[0]
+        expect = sign * (1.0 - (-alpha) ** (t + 1)) / (1.0 + alpha)
+        assert osh.rel_fro(P, expect * P0) < 1e-12
