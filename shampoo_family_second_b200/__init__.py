@@ -211,6 +211,7 @@ class Shampoo:
                                     self.state_bytes, self.scratch.data_ptr(), self.scratch_bytes,
                                     _stream_ptr(stream), ctypes.byref(h)))
         self._h = h
+        self._destroy = lib.shampoo_destroy
         nb = ctypes.c_int32(0)
         _check(lib.shampoo_block_table(self._h, ctypes.byref(nb), None))
         self.nb = nb.value
@@ -219,9 +220,12 @@ class Shampoo:
         self._ldbuf = (ctypes.c_int64 * len(self.shapes))()
 
     def __del__(self):
+        # The library handle is held by the instance: at interpreter shutdown
+        # the module's globals may already be cleared.
         h = getattr(self, "_h", None)
-        if h is not None and h.value:
-            lib.shampoo_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
             self._h = None
 
     def step(self, weights, grads, stream=None):
