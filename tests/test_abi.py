@@ -101,12 +101,26 @@ def test_scratch_sizes(sb):
     per = b - a
     assert per == 64 * (7 * 1024 * 1024 * 4 + 4 * (8 + 64 + 2))   # Newton: 7 stacks per matrix
     assert sb.inv_root_scratch_bytes(64, 1024, sb.SOLVER_NEWTON_DB) < a
+    # the second-degree correction reuses the Newton stacks (T, T^2, T^4 also hold D = I - M)
+    assert sb.inv_root_scratch_bytes(64, 1024, sb.SOLVER_NEWTON_CUBIC) == a
     assert sb.gemm_scratch_bytes(3, 256) == 0   # operands are split on chip
     # the no-alloc entry point's fixed 32 MiB covers one matrix of every supported size
-    for solver in (sb.SOLVER_NEWTON, sb.SOLVER_NEWTON_DB, sb.SOLVER_CHEBYSHEV):
+    for solver in (sb.SOLVER_NEWTON, sb.SOLVER_NEWTON_DB, sb.SOLVER_CHEBYSHEV, sb.SOLVER_NEWTON_CUBIC):
         assert sb.inv_root_scratch_bytes(1, 1024, solver) <= 32 << 20
     with pytest.raises(sb.ShampooError):
         sb.inv_root_scratch_bytes(4, 100, 0)
+    with pytest.raises(sb.ShampooError):   # no solver 4
+        sb.inv_root_scratch_bytes(4, 256, 4)
+
+
+def test_every_solver_is_accepted_by_the_step_config(sb):
+    """Each solver id of the header passes the step's argument checks (sizes
+    are queried without a GPU); an unknown id is refused."""
+    for solver in (sb.SOLVER_NEWTON, sb.SOLVER_NEWTON_DB, sb.SOLVER_NEWTON_CUBIC):
+        state, scratch = sb.query_sizes(sb.make_config(256, 0.95, 1e-8, 1e-3, solver=solver), [(1024, 1024)])
+        assert state > 0 and scratch > 0
+    with pytest.raises(sb.ShampooError):
+        sb.query_sizes(sb.make_config(256, 0.95, 1e-8, 1e-3, solver=4), [(1024, 1024)])
 
 
 def test_init_rejects_missing_buffers_without_cuda(sb):
