@@ -508,6 +508,27 @@ def time_oracle(wl, blocks, steps, warmup=0):
     return times, nref
 
 
+SINGLE_THREAD_WORKLOADS = ("tiny", "lowrank")
+
+
+def single_thread_oracle(wl, blocks, nb, steps, est_s_per_block, budget_s):
+    """The oracle over the same step window on one host thread (BLAS/LAPACK
+    limited to one thread), on a prefix of the block sample sized so that even
+    a run `cores` times slower than the multi-threaded one stays near
+    budget_s; None when the thread limit cannot be set."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return None
+    k = max(1, min(len(blocks), int(budget_s / max(est_s_per_block, 1e-6))))
+    sub = blocks[:k]
+    with threadpool_limits(limits=1):
+        times, nref = time_oracle(wl, sub, steps)
+    return {"value": 2 * len(sub) * nref / sum(times), "unit": "inverse-roots/s", "cores": 1,
+            "sample": (f"{len(sub)} of {nb} blocks, {steps} consecutive steps from step 0 ({nref} refresh), "
+                       f"float64 numpy/LAPACK eigh, 1 thread")}
+
+
 def cpu_baseline(wl, budget_s):
     cores = len(os.sched_getaffinity(0))
     blocks, nb = oracle_sample_plan(wl, budget_s)
@@ -515,9 +536,15 @@ def cpu_baseline(wl, budget_s):
     times, nref = time_oracle(wl, blocks, steps)
     roots = 2 * len(blocks) * nref
     value = roots / sum(times)
-    return {"value": value, "unit": "inverse-roots/s", "cores": cores, "kind": "oracle",
-            "sample": (f"{len(blocks)} of {nb} blocks, {steps} consecutive steps from step 0 "
-                       f"({nref} refresh), float64 numpy/LAPACK eigh, {cores} host threads")}
+    out = {"value": value, "unit": "inverse-roots/s", "cores": cores, "kind": "oracle",
+           "sample": (f"{len(blocks)} of {nb} blocks, {steps} consecutive steps from step 0 "
+                      f"({nref} refresh), float64 numpy/LAPACK eigh, {cores} host threads")}
+    if wl.name in SINGLE_THREAD_WORKLOADS:
+        per_block = sum(times) / len(blocks) * cores   # pessimistic one-thread time per block
+        one = single_thread_oracle(wl, blocks, nb, steps, per_block, min(budget_s, 20.0) / 2.0)
+        if one is not None:
+            out["single_thread"] = one
+    return out
 
 
 def run_reference(args, wl):

@@ -28,3 +28,14 @@ def test_traffic_record_is_well_formed():
     assert d["workload_key"] in ("lowrank", "gpt2", "llama")
     assert d["solver"] in bench.SOLVER_NAMES.values()
     assert len(d["source_sha256"]) == 64 and "ncu" in d["command"]
+
+
+def test_cpu_baseline_reports_a_single_thread_number():
+    """The oracle baseline of the default workload carries, beside the
+    multi-threaded rate, a one-thread rate on a bounded sample."""
+    import workloads
+    out = bench.cpu_baseline(workloads.workload("lowrank"), 2.0)
+    assert out["kind"] == "oracle" and out["value"] > 0 and out["cores"] >= 1
+    one = out.get("single_thread")
+    assert one is not None and one["cores"] == 1 and one["value"] > 0
+    assert "1 thread" in one["sample"]
