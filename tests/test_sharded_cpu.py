@@ -44,28 +44,30 @@ def oracle_local_step(blocks):
     return step
 
 
-def gradients(t, rank=None, world=2):
+def gradients(t, rank=None, world=2, shapes=None):
     """Seeded gradients of step t; with a rank, that rank's local part: G plus
     a rank-dependent term whose sum over the ranks is zero (rank 0: +D, rank
     1: -D, any further rank: 0)."""
+    shapes = SHAPES if shapes is None else shapes
     rng = np.random.default_rng(100 + t)
-    G = [rng.standard_normal(s).astype(np.float32) for s in SHAPES]
+    G = [rng.standard_normal(s).astype(np.float32) for s in shapes]
     if rank is None:
         return [torch.from_numpy(g) for g in G]
-    D = [np.random.default_rng(200 + t).standard_normal(s).astype(np.float32) for s in SHAPES]
+    D = [np.random.default_rng(200 + t).standard_normal(s).astype(np.float32) for s in shapes]
     sign = {0: 1.0, 1: -1.0}.get(rank, 0.0)
     return [torch.from_numpy(g + np.float32(sign) * d) for g, d in zip(G, D)]
 
 
-def run_single(grads_reduced, world=2):
-    blocks = sharded.block_list(SHAPES, B)
-    opt = sharded.ShardedShampoo(SHAPES, Cfg, grads_reduced=grads_reduced, local_step=oracle_local_step(blocks))
-    W = [torch.zeros(s) for s in SHAPES]
+def run_single(grads_reduced, world=2, shapes=None):
+    shapes = SHAPES if shapes is None else shapes
+    blocks = sharded.block_list(shapes, B)
+    opt = sharded.ShardedShampoo(shapes, Cfg, grads_reduced=grads_reduced, local_step=oracle_local_step(blocks))
+    W = [torch.zeros(s) for s in shapes]
     for t in range(STEPS):
         if grads_reduced:
-            G = gradients(t)
+            G = gradients(t, shapes=shapes)
         else:  # the average of the ranks' local gradients
-            parts = [gradients(t, k, world) for k in range(world)]
+            parts = [gradients(t, k, world, shapes) for k in range(world)]
             G = [sum(ps[1:], ps[0]) / world for ps in zip(*parts)]
         opt.step(W, G)
     return [w.numpy().copy() for w in W]
@@ -77,29 +79,30 @@ def free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, grads_reduced, out_q):
+def _worker(rank, world, port, grads_reduced, shapes, out_q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     from datetime import timedelta
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
     try:
-        blocks = sharded.block_list(SHAPES, B)
+        blocks = sharded.block_list(shapes, B)
         owner = sharded.partition_blocks(blocks, world)
         mine = [blocks[i] for i, k in enumerate(owner) if k == rank]
-        opt = sharded.ShardedShampoo(SHAPES, Cfg, grads_reduced=grads_reduced, local_step=oracle_local_step(mine))
-        W = [torch.zeros(s) for s in SHAPES]
+        opt = sharded.ShardedShampoo(shapes, Cfg, grads_reduced=grads_reduced, local_step=oracle_local_step(mine))
+        W = [torch.zeros(s) for s in shapes]
         for t in range(STEPS):
-            opt.step(W, gradients(t) if grads_reduced else gradients(t, rank, world))
+            opt.step(W, gradients(t, shapes=shapes) if grads_reduced else gradients(t, rank, world, shapes))
         out_q.put((rank, len(mine), [w.numpy().copy() for w in W]))
     finally:
         dist.barrier()
         dist.destroy_process_group()
 
 
-def run_ranks(grads_reduced, world=2):
+def run_ranks(grads_reduced, world=2, shapes=None):
+    shapes = SHAPES if shapes is None else shapes
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, grads_reduced, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, grads_reduced, shapes, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = sorted(q.get(timeout=180) for _ in procs)
@@ -161,3 +164,17 @@ def test_partition_balance_on_transformer_shapes(world):
     cost = [b[3] ** 3 + b[4] ** 3 for b in blocks]
     load = [sum(c for c, k in zip(cost, owner) if k == r) for r in range(world)]
     assert max(load) <= 1.02 * sum(load) / world, load
+
+
+@pytest.mark.parametrize("grads_reduced", [True, False])
+def test_more_ranks_than_blocks(grads_reduced):
+    """A 40 x 30 weight at block 32 has 2 blocks; with 3 ranks one rank owns
+    none.  It still takes part in every collective, and all ranks end with
+    the single-process weights."""
+    shapes = [(40, 30)]
+    single = run_single(grads_reduced, 3, shapes)
+    res = run_ranks(grads_reduced, 3, shapes)
+    assert sorted(n for _, n, _ in res) == [0, 1, 1]
+    for _, _, W in res:
+        for a, s_ in zip(W, single):
+            assert np.allclose(a, s_, rtol=0, atol=1e-6), float(np.abs(a - s_).max())
