@@ -16,7 +16,8 @@ Sources (web pages; cited by title and section/cue):
 * Podcast transcript "Preconditioned optimization without the full matrix
   cost" (Gupta, Koren, Singer 2018) — cue 20 (update rule), cue 22 (the
   two-sided quarter powers equal the Kronecker product form), cue 24 (memory
-  and cost), cue 28 (roots recomputed only every 20-100 steps).
+  and cost), cue 26 (order-k tensors), cue 28 (roots recomputed only every
+  20-100 steps; momentum ahead of the preconditioner).
 * "DASH: Faster Shampoo via Batched Block Preconditioning and Efficient
   Inverse-Root Solvers" — abstract (blocks stacked into 3D tensors; Newton-DB
   and Chebyshev inverse-root solvers; matrix scaling).
@@ -32,9 +33,14 @@ Modules:
                   evaluation on a matrix (the polynomial the Chebyshev solver
                   evaluates).  Pinned against numpy's Chebyshev routines and
                   polynomial exactness.
-* ``iter_mirror`` float64 restatements of the coupled-Newton and Newton-DB
-                  iterations, used only as a diagnostic (never as a parity
-                  gate).  Pinned by convergence to the exact root.
+* ``iter_mirror`` float64 restatements of the coupled-Newton (both correction
+                  degrees) and Newton-DB iterations, used only as a diagnostic
+                  (never as a parity gate).  Pinned by convergence to the
+                  exact root and by the correction's Taylor order.
+* ``tensor``      order-k tensor Shampoo (podcast cue 26): per-mode statistics,
+                  -1/(2k) roots, mode-wise contractions.  Pinned by the matrix
+                  case, a Kronecker brute force and a rank-one closed form
+                  (tests/test_oracle_tensor.py).
 """
 from .shampoo import (Block, block_table, inverse_root, accumulate,
                       precondition, ShampooOracle, rel_fro)
