@@ -178,3 +178,31 @@ def test_more_ranks_than_blocks(grads_reduced):
     for _, _, W in res:
         for a, s_ in zip(W, single):
             assert np.allclose(a, s_, rtol=0, atol=1e-6), float(np.abs(a - s_).max())
+
+
+def test_partition_properties_on_random_shapes():
+    """Random weight lists, block sizes and world sizes: the blocks tile every
+    weight exactly once, every block has one owner, and the greedy balance
+    bound holds (no rank carries more than the average plus one block's cost)."""
+    hypothesis = pytest.importorskip("hypothesis")
+    st = hypothesis.strategies
+
+    @hypothesis.settings(max_examples=60, deadline=None)
+    @hypothesis.given(shapes=st.lists(st.tuples(st.integers(1, 300), st.integers(1, 300)), min_size=1, max_size=6),
+                      block=st.sampled_from([32, 64, 128]), world=st.integers(1, 9))
+    def check(shapes, block, world):
+        blocks = sharded.block_list(shapes, block)
+        for p, (m, n) in enumerate(shapes):
+            cover = np.zeros((m, n), dtype=int)
+            for q, r0, c0, r, c in blocks:
+                if q == p:
+                    assert 0 < r <= block and 0 < c <= block
+                    cover[r0:r0 + r, c0:c0 + c] += 1
+            assert (cover == 1).all()
+        owner = sharded.partition_blocks(blocks, world)
+        assert len(owner) == len(blocks) and all(0 <= k < world for k in owner)
+        cost = [b[3] ** 3 + b[4] ** 3 for b in blocks]
+        load = [sum(c for c, k in zip(cost, owner) if k == r) for r in range(world)]
+        assert max(load) <= sum(load) / world + max(cost)
+
+    check()
