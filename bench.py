@@ -107,6 +107,15 @@ def phase_to_refresh(step, every):
     return -(-step // every) * every
 
 
+def split_step_ms(step_ms, every):
+    """Mean step time of the refresh steps and of the other steps of a window
+    that starts on a refresh step (step k refreshes when k % every == 0)."""
+    ref = [t for k, t in enumerate(step_ms) if k % every == 0]
+    other = [t for k, t in enumerate(step_ms) if k % every != 0]
+    return {"refresh_ms": sum(ref) / len(ref) if ref else None, "refresh_steps": len(ref),
+            "non_refresh_ms": sum(other) / len(other) if other else None, "non_refresh_steps": len(other)}
+
+
 class ClockSampler:
     """SM clocks and throttle reasons during the timed region.
 
@@ -410,6 +419,7 @@ def run_ours(args, wl):
             "overlap": f"host-to-device copies (each after an L2 flush) run up to {E2E_DEPTH} steps ahead on a copy stream",
         },
     }
+    result["step_ms_split"] = split_step_ms(step_ms, wl.refresh_every)   # this rank's timed steps
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget_s)
     if world > 1:

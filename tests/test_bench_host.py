@@ -39,3 +39,15 @@ def test_cpu_baseline_reports_a_single_thread_number():
     one = out.get("single_thread")
     assert one is not None and one["cores"] == 1 and one["value"] > 0
     assert "1 thread" in one["sample"]
+
+
+def test_step_time_split_by_refresh():
+    """A 20-step window starting on a refresh, refresh every 10: steps 0 and
+    10 are the refresh steps; every step counts once."""
+    ms = [5.0 if k % 10 == 0 else 0.2 for k in range(20)]
+    out = bench.split_step_ms(ms, 10)
+    assert out["refresh_steps"] == 2 and out["non_refresh_steps"] == 18
+    assert out["refresh_ms"] == 5.0 and abs(out["non_refresh_ms"] - 0.2) < 1e-12
+    every_step = bench.split_step_ms([3.0, 4.0], 1)       # refresh every step
+    assert every_step["refresh_ms"] == 3.5 and every_step["non_refresh_ms"] is None
+    assert bench.refresh_steps(20, 10) == out["refresh_steps"]
