@@ -117,7 +117,11 @@ enum {
  *  cheb_degree    Chebyshev degree d in [2, 64].
  *  cheb_lo        Chebyshev interval: [lo / s, 1] with lo = cheb_lo if > 0 else eps,
  *                 s = ||A + eps I||_F.
- *  grad_dtype     SHAMPOO_F32 or SHAMPOO_BF16 (weights and statistics are always fp32). */
+ *  grad_dtype     SHAMPOO_F32 or SHAMPOO_BF16 (weights and statistics are always fp32).
+ *  momentum       alpha in [0, 1): 0 = off (the update uses the raw gradient); > 0 keeps a
+ *                 per-block momentum M <- alpha M + G (from M = 0) ahead of the preconditioner,
+ *                 and the update becomes W <- W - lr XL M XR, while the statistics still take
+ *                 the raw G (podcast transcript, cue 28: momentum 0.9 before preconditioning). */
 typedef struct {
   int32_t block;
   float beta;
@@ -131,6 +135,7 @@ typedef struct {
   int32_t cheb_degree;
   float cheb_lo;
   int32_t grad_dtype;
+  float momentum;
 } shampoo_config;
 
 typedef struct shampoo_ctx* shampoo_handle;
@@ -191,6 +196,10 @@ SHAMPOO_API int shampoo_block_table(shampoo_handle h, int32_t* nb, int64_t* tabl
  * Ragged blocks hold zeros outside their r x r / c x c valid region. */
 SHAMPOO_API int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, float** rootR, int64_t* step);
 
+/* Device pointer to the momentum stack (nb, B, B) fp32 in the state (zero
+ * outside each block's r x c region), or NULL when momentum is off. */
+SHAMPOO_API int shampoo_momentum_view(shampoo_handle h, float** M);
+
 /* Sets the step counter (checkpoint resume: restore the state buffer bytes,
  * then the counter). */
 SHAMPOO_API int shampoo_set_step(shampoo_handle h, int64_t step);
@@ -199,16 +208,23 @@ SHAMPOO_API int shampoo_set_step(shampoo_handle h, int64_t step);
 SHAMPOO_API void shampoo_destroy(shampoo_handle h);
 
 /* Scratch bytes inv_root_batched needs to solve all `batch` matrices in one
- * pass.  Less (but at least the size for one matrix plus 64 KiB) makes it work
- * through the batch in chunks.  Host-only. */
+ * pass, for p = 2 or 4.  Less (but at least the size for one matrix plus
+ * 64 KiB) makes it work through the batch in chunks.  Host-only. */
 SHAMPOO_API int inv_root_scratch_bytes(int64_t batch, int32_t n, int32_t solver, size_t* bytes);
+
+/* inv_root_scratch_bytes for a given root order p in {2, 4, 6, 8}: coupled
+ * Newton with p = 6 or 8 keeps one more n x n iterate per matrix (T^p).
+ * Host-only. */
+SHAMPOO_API int inv_root_scratch_bytes_p(int64_t batch, int32_t n, int32_t solver, int32_t p, size_t* bytes);
 
 /* Batched inverse p-th roots: X_i ~ (A_i + eps I)^{-1/p} for symmetric
  * positive semi-definite A_i (the notes' L^{-1/4}, R^{-1/4}; SOAP abstract's
  * p = 2).  DASH abstract: batched inverse-root solvers with matrix scaling.
  *  d_A, d_X      device plain stacks (batch, n, n); n a multiple of 32 in [32, 1024].
  *                A is symmetrised ((A + A^T)/2) before use.
- *  p             2 or 4.   eps  damping >= 0.
+ *  p             2 or 4; also 6 or 8 (order-3 and order-4 tensor Shampoo's -1/(2k)
+ *                powers, podcast cue 26) with coupled Newton and Chebyshev.
+ *                eps  damping >= 0.
  *  solver, iters, tol, cheb_degree, cheb_lo   as in shampoo_config.
  *  d_scratch     device scratch, 256-byte aligned (see inv_root_scratch_bytes).
  *  d_iters_used  nullable device int32[batch]: iterations run per matrix
@@ -236,10 +252,67 @@ SHAMPOO_API int inv_root_batched(const float* d_A, float* d_X, int64_t batch, in
  * what must start at zero on every call.  Batches larger than the array are
  * solved in chunks (the largest need, coupled Newton at n = 1024, is 28 MiB
  * per matrix); a size whose scratch for one matrix exceeded the array would
- * return SHAMPOO_ERR_UNSUPPORTED. */
+ * return SHAMPOO_ERR_UNSUPPORTED.  With tol > 0 the iterations are plain
+ * kernel launches up to the cap (tiles of finished matrices exit at once),
+ * never a CUDA graph, whose instantiation may take device memory; results
+ * equal inv_root_batched's. */
 SHAMPOO_API int inv_root_batched_noalloc(const float* d_A, float* d_X, int64_t batch, int32_t n, int32_t p, float eps,
                                          int32_t solver, int32_t iters, float tol, int32_t cheb_degree,
                                          float cheb_lo, int32_t* d_iters_used, int32_t* d_status, void* stream);
+
+/* Order-k tensor Shampoo (podcast transcript "Preconditioned optimization
+ * without the full matrix cost", cue 26): for a parameter of order k in
+ * [2, 4] with dimensions d_0 .. d_{k-1} (each in [1, 1024]; larger gives
+ * SHAMPOO_ERR_UNSUPPORTED), one statistic per dimension,
+ *     H_i <- beta H_i + G_(i) G_(i)^T      (G_(i): mode-i unfolding of G, the
+ *                                           other indices in row-major order)
+ *     X_i = (H_i + eps I)^{-1/(2k)}        (every refresh_every steps)
+ *     W <- W - lr  G x_0 X_0 x_1 X_1 ... x_{k-1} X_{k-1}
+ * (x_i: contraction along dimension i).  The parameters are not blocked.
+ * Config fields used: beta, eps, lr, solver (coupled Newton either degree,
+ * Chebyshev; Newton-DB for order 2 only), iters, tol, refresh_every,
+ * cheb_degree, cheb_lo, grad_dtype; block and root_p are ignored, momentum
+ * must be 0.  orders[j] is the order of parameter j; dims holds all
+ * parameters' dimensions back to back.  Weights are fp32 and gradients
+ * grad_dtype, both row-major (natural layout), device pointers in host
+ * arrays.  Ownership, streams and errors as for shampoo_init / shampoo_step;
+ * nparams in [1, 256]. */
+typedef struct shampoo_tensor_ctx* shampoo_tensor_handle;
+SHAMPOO_API int shampoo_tensor_query_sizes(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
+                                           const int64_t* dims, size_t* state_bytes, size_t* scratch_bytes);
+SHAMPOO_API int shampoo_tensor_init(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
+                                    const int64_t* dims, void* d_state, size_t state_bytes, void* d_scratch,
+                                    size_t scratch_bytes, void* stream, shampoo_tensor_handle* out);
+SHAMPOO_API int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const void* const* d_grads,
+                                    void* stream);
+/* Device pointers to the statistic H_i and root X_i of mode `mode` of
+ * parameter `param`: npad x npad fp32 (npad = d_i rounded up to 32; zero /
+ * identity-scaled beyond d_i); *step: steps taken. */
+SHAMPOO_API int shampoo_tensor_views(shampoo_tensor_handle h, int32_t param, int32_t mode, float** H, float** X,
+                                     int32_t* npad, int64_t* step);
+/* As shampoo_get_status, for a tensor handle. */
+SHAMPOO_API int shampoo_tensor_get_status(shampoo_tensor_handle h, int32_t* status, int32_t reset);
+SHAMPOO_API void shampoo_tensor_destroy(shampoo_tensor_handle h);
+
+/* Block packing for blocks sharded across ranks (DASH abstract: the
+ * preconditioner blocks are distributed across devices): one launch moves
+ * nblocks r x c blocks between row-strided matrices and one packed fp32
+ * buffer holding the blocks back to back, each row-major.
+ *  d_table     device int64 [nblocks x 6]: {param, row0, col0, r, c, offset},
+ *              offset = the block's first float in d_packed.  Every block must
+ *              lie inside its matrix and the packed buffer (not checked on the
+ *              device).
+ *  d_params    host array of nparams device pointers; ld host array of their
+ *              row strides in elements (>= 1).
+ *  dtype       element type of the matrices: SHAMPOO_F32, or SHAMPOO_BF16 for
+ *              a gather (widened exactly).
+ *  direction   0: gather, d_packed = scale * block; 1: scatter, block = d_packed
+ *              (scale unused; fp32 matrices only).
+ *  max_rows, max_cols   largest r and c in the table (they size the grid).
+ * nblocks in [0, 65535], nparams in [1, 1024].  Enqueued on `stream`. */
+SHAMPOO_API int shampoo_pack_blocks(const int64_t* d_table, int32_t nblocks, int32_t nparams, void* const* d_params,
+                                    const int64_t* ld, int32_t dtype, float* d_packed, int32_t direction, float scale,
+                                    int32_t max_rows, int32_t max_cols, void* stream);
 
 /* The batched fp32-accurate product every stage uses, as a utility:
  * D_i = alpha A_i op(B_i) + beta C_i + gamma I for plain stacks (batch, n, n),

@@ -51,8 +51,12 @@ KERNEL_NAMES = ("gemm3x_tf32", "stack_blocks", "frob_norm", "prologue", "check",
 # Exported symbols, in header order (tests compare this with include/shampoo.h).
 EXPORTS = (
     "shampoo_status_string", "shampoo_last_error", "shampoo_query_sizes", "shampoo_init", "shampoo_step",
-    "shampoo_step_strided", "shampoo_get_status", "shampoo_block_table", "shampoo_state_views", "shampoo_set_step", "shampoo_destroy",
-    "inv_root_scratch_bytes", "inv_root_batched", "inv_root_batched_noalloc", "shampoo_gemm_scratch_bytes",
+    "shampoo_step_strided", "shampoo_get_status", "shampoo_block_table", "shampoo_state_views",
+    "shampoo_momentum_view", "shampoo_set_step", "shampoo_destroy",
+    "inv_root_scratch_bytes", "inv_root_scratch_bytes_p", "inv_root_batched", "inv_root_batched_noalloc",
+    "shampoo_tensor_query_sizes", "shampoo_tensor_init", "shampoo_tensor_step", "shampoo_tensor_views",
+    "shampoo_tensor_get_status", "shampoo_tensor_destroy", "shampoo_pack_blocks",
+    "shampoo_gemm_scratch_bytes",
     "shampoo_gemm_batched",
     "shampoo_profile_enable", "shampoo_profile_reset", "shampoo_profile_read", "shampoo_launch_count",
 )
@@ -71,20 +75,21 @@ class Config(ctypes.Structure):
         ("block", ctypes.c_int32), ("beta", ctypes.c_float), ("eps", ctypes.c_float), ("lr", ctypes.c_float),
         ("root_p", ctypes.c_int32), ("solver", ctypes.c_int32), ("iters", ctypes.c_int32), ("tol", ctypes.c_float),
         ("refresh_every", ctypes.c_int32), ("cheb_degree", ctypes.c_int32), ("cheb_lo", ctypes.c_float),
-        ("grad_dtype", ctypes.c_int32),
+        ("grad_dtype", ctypes.c_int32), ("momentum", ctypes.c_float),
     ]
 
 
 def make_config(block: int, beta: float, eps: float, lr: float, root_p: int = 4, solver: int = SOLVER_NEWTON,
                 iters: int = 40, tol: float = 1e-5, refresh_every: int = 1, cheb_degree: int = 32,
-                cheb_lo: float = 0.0, grad_dtype: int = F32) -> Config:
-    return Config(block, beta, eps, lr, root_p, solver, iters, tol, refresh_every, cheb_degree, cheb_lo, grad_dtype)
+                cheb_lo: float = 0.0, grad_dtype: int = F32, momentum: float = 0.0) -> Config:
+    return Config(block, beta, eps, lr, root_p, solver, iters, tol, refresh_every, cheb_degree, cheb_lo, grad_dtype,
+                  momentum)
 
 
 def config_from_workload(wl) -> Config:
     """Config of a ``workloads.Workload`` preset."""
     return make_config(wl.block, wl.beta, wl.eps, wl.lr, wl.root_p, wl.solver, wl.iters, wl.tol, wl.refresh_every,
-                       wl.cheb_degree, wl.cheb_lo, wl.grad_dtype)
+                       wl.cheb_degree, wl.cheb_lo, wl.grad_dtype, getattr(wl, "momentum", 0.0))
 
 
 def _load():
@@ -108,11 +113,24 @@ def _load():
         "shampoo_block_table": (ctypes.c_int, [P, ctypes.POINTER(I32), ctypes.POINTER(I64)]),
         "shampoo_state_views": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
                                                ctypes.POINTER(P), ctypes.POINTER(I64)]),
+        "shampoo_momentum_view": (ctypes.c_int, [P, ctypes.POINTER(P)]),
         "shampoo_set_step": (ctypes.c_int, [P, I64]),
         "shampoo_destroy": (None, [P]),
         "inv_root_scratch_bytes": (ctypes.c_int, [I64, I32, I32, sz]),
+        "inv_root_scratch_bytes_p": (ctypes.c_int, [I64, I32, I32, I32, sz]),
         "inv_root_batched": (ctypes.c_int, [P, P, I64, I32, I32, F, I32, I32, F, I32, F, P, ctypes.c_size_t, P, P, P]),
         "inv_root_batched_noalloc": (ctypes.c_int, [P, P, I64, I32, I32, F, I32, I32, F, I32, F, P, P, P]),
+        "shampoo_tensor_query_sizes": (ctypes.c_int, [ctypes.POINTER(Config), I32, ctypes.POINTER(I32),
+                                                      ctypes.POINTER(I64), sz, sz]),
+        "shampoo_tensor_init": (ctypes.c_int, [ctypes.POINTER(Config), I32, ctypes.POINTER(I32), ctypes.POINTER(I64),
+                                               P, ctypes.c_size_t, P, ctypes.c_size_t, P, ctypes.POINTER(P)]),
+        "shampoo_tensor_step": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P), P]),
+        "shampoo_tensor_views": (ctypes.c_int, [P, I32, I32, ctypes.POINTER(P), ctypes.POINTER(P),
+                                                ctypes.POINTER(I32), ctypes.POINTER(I64)]),
+        "shampoo_tensor_get_status": (ctypes.c_int, [P, ctypes.POINTER(I32), I32]),
+        "shampoo_tensor_destroy": (None, [P]),
+        "shampoo_pack_blocks": (ctypes.c_int, [P, I32, I32, ctypes.POINTER(P), ctypes.POINTER(I64), I32, P, I32, F,
+                                               I32, I32, P]),
         "shampoo_gemm_scratch_bytes": (ctypes.c_int, [I64, I32, sz]),
         "shampoo_gemm_batched": (ctypes.c_int, [P, P, P, P, I64, I32, I32, F, F, F, P, ctypes.c_size_t, P, P]),
         "shampoo_profile_enable": (None, [I32]),
@@ -171,9 +189,9 @@ def query_sizes(cfg: Config, shapes: Sequence[Tuple[int, int]]) -> Tuple[int, in
     return sb.value, xb.value
 
 
-def inv_root_scratch_bytes(batch: int, n: int, solver: int) -> int:
+def inv_root_scratch_bytes(batch: int, n: int, solver: int, p: int = 4) -> int:
     b = ctypes.c_size_t(0)
-    _check(lib.inv_root_scratch_bytes(batch, n, solver, ctypes.byref(b)))
+    _check(lib.inv_root_scratch_bytes_p(batch, n, solver, p, ctypes.byref(b)))
     return b.value
 
 
@@ -299,6 +317,18 @@ class Shampoo:
         XR = fl[(pxr - base) // 4:(pxr - base) // 4 + nb * B * B].view(nb, B, B)
         return XL, XR
 
+    def momentum(self):
+        """The momentum stack (nb, B, B) as a float32 view into the state
+        buffer, or None when momentum is off."""
+        import torch
+        ptr = ctypes.c_void_p()
+        _check(lib.shampoo_momentum_view(self._h, ctypes.byref(ptr)))
+        if not ptr.value:
+            return None
+        B, nb = self.cfg.block, self.nb
+        off = (ptr.value - self.state.data_ptr()) // 4
+        return self.state.view(torch.float32)[off:off + nb * B * B].view(nb, B, B)
+
     def set_step_count(self, step: int):
         """Sets the step counter (the refresh schedule counts from it)."""
         _check(lib.shampoo_set_step(self._h, int(step)))
@@ -310,6 +340,88 @@ class Shampoo:
     def load_state_dict(self, sd):
         self.state.copy_(sd["state"])
         _check(lib.shampoo_set_step(self._h, int(sd["step"])))
+
+
+def tensor_query_sizes(cfg: Config, shapes: Sequence[Sequence[int]]) -> Tuple[int, int]:
+    orders = (ctypes.c_int32 * len(shapes))(*[len(s) for s in shapes])
+    dims = _i64_array([d for s in shapes for d in s])
+    sb, xb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(lib.shampoo_tensor_query_sizes(ctypes.byref(cfg), len(shapes), orders, dims, ctypes.byref(sb),
+                                          ctypes.byref(xb)))
+    return sb.value, xb.value
+
+
+class TensorShampoo:
+    """Order-k tensor Shampoo over a fixed list of tensor weights (order 2 to
+    4, every dimension at most 1024): one statistic and one -1/(2k) root per
+    dimension, applied by contractions along each dimension.
+
+    ``step(weights, grads)`` updates the fp32 weights in place; gradients are
+    fp32 or bf16 (cfg.grad_dtype), natural row-major layout.  State and
+    scratch are torch allocations owned by this object."""
+
+    def __init__(self, shapes: Sequence[Sequence[int]], cfg: Config, device=None, stream=None):
+        import torch
+        self.shapes = [tuple(int(x) for x in s) for s in shapes]
+        self.cfg = cfg
+        self.device = torch.device("cuda" if device is None else device)
+        self.state_bytes, self.scratch_bytes = tensor_query_sizes(cfg, self.shapes)
+        self.state = torch.empty(self.state_bytes, dtype=torch.uint8, device=self.device)
+        self.scratch = torch.empty(self.scratch_bytes, dtype=torch.uint8, device=self.device)
+        orders = (ctypes.c_int32 * len(self.shapes))(*[len(s) for s in self.shapes])
+        dims = _i64_array([d for s in self.shapes for d in s])
+        h = ctypes.c_void_p(None)
+        with torch.cuda.device(self.device):
+            _check(lib.shampoo_tensor_init(ctypes.byref(cfg), len(self.shapes), orders, dims, self.state.data_ptr(),
+                                           self.state_bytes, self.scratch.data_ptr(), self.scratch_bytes,
+                                           _stream_ptr(stream), ctypes.byref(h)))
+        self._h = h
+        self._destroy = lib.shampoo_tensor_destroy
+        self._wbuf = (ctypes.c_void_p * len(self.shapes))()
+        self._gbuf = (ctypes.c_void_p * len(self.shapes))()
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        destroy = getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
+            self._h = None
+
+    def step(self, weights, grads, stream=None):
+        import torch
+        want = torch.bfloat16 if self.cfg.grad_dtype == BF16 else torch.float32
+        if len(weights) != len(self.shapes) or len(grads) != len(self.shapes):
+            raise ValueError("one weight and one gradient per shape")
+        for i, (w, g) in enumerate(zip(weights, grads)):
+            if w.dtype != torch.float32 or g.dtype != want:
+                raise TypeError(f"param {i}: weights must be float32 and grads {want}")
+            if tuple(w.shape) != self.shapes[i] or tuple(g.shape) != self.shapes[i]:
+                raise ValueError(f"param {i}: shape mismatch")
+            if not (w.is_contiguous() and g.is_contiguous()):
+                raise ValueError(f"param {i}: weight and gradient must be contiguous")
+            self._wbuf[i] = w.data_ptr()
+            self._gbuf[i] = g.data_ptr()
+        _check(lib.shampoo_tensor_step(self._h, self._wbuf, self._gbuf, _stream_ptr(stream)))
+
+    def status(self, reset: bool = False) -> int:
+        s = ctypes.c_int32(0)
+        _check(lib.shampoo_tensor_get_status(self._h, ctypes.byref(s), 1 if reset else 0))
+        return s.value
+
+    def mode_views(self, param: int, mode: int):
+        """(H, X) of one mode as float32 (npad, npad) views into the state; the
+        statistic's dimension d occupies the leading d x d block."""
+        import torch
+        ph, px = ctypes.c_void_p(), ctypes.c_void_p()
+        npad, step = ctypes.c_int32(0), ctypes.c_int64(0)
+        _check(lib.shampoo_tensor_views(self._h, param, mode, ctypes.byref(ph), ctypes.byref(px),
+                                        ctypes.byref(npad), ctypes.byref(step)))
+        fl = self.state.view(torch.float32)
+        base = self.state.data_ptr()
+        n = npad.value
+        H = fl[(ph.value - base) // 4:(ph.value - base) // 4 + n * n].view(n, n)
+        X = fl[(px.value - base) // 4:(px.value - base) // 4 + n * n].view(n, n)
+        return H, X
 
 
 # ---------------------------------------------------------------------------
@@ -330,7 +442,7 @@ def inv_root_batched(A, p: int = 4, eps: float = 0.0, solver: int = SOLVER_NEWTO
     batch, n = A.shape[0], A.shape[1]
     X = torch.empty_like(A) if out is None else out
     if scratch is None:
-        scratch = torch.empty(inv_root_scratch_bytes(batch, n, solver), dtype=torch.uint8, device=A.device)
+        scratch = torch.empty(inv_root_scratch_bytes(batch, n, solver, p), dtype=torch.uint8, device=A.device)
     iters_used = torch.zeros(batch, dtype=torch.int32, device=A.device)
     status = torch.zeros(1, dtype=torch.int32, device=A.device)
     with torch.cuda.device(A.device):
@@ -361,6 +473,43 @@ def gemm_batched(A, B, C=None, alpha: float = 1.0, beta: float = 0.0, gamma: flo
                                         status.data_ptr(),
                                         _stream_ptr(stream)))
     return D, status
+
+
+class BlockPacker:
+    """Moves a fixed list of blocks between matrices and a packed fp32 buffer
+    in one kernel launch per call (shampoo_pack_blocks).
+
+    ``blocks``: (param, row0, col0, r, c, offset) tuples, offset in floats of
+    the packed buffer.  The device table is built once."""
+
+    def __init__(self, blocks, device):
+        import torch
+        self.blocks = [tuple(int(x) for x in b) for b in blocks]
+        self.n = len(self.blocks)
+        self.table = torch.tensor(self.blocks if self.blocks else [[0] * 6], dtype=torch.int64, device=device)
+        self.max_rows = max([b[3] for b in self.blocks], default=1)
+        self.max_cols = max([b[4] for b in self.blocks], default=1)
+
+    def _call(self, mats, packed, direction, scale, stream):
+        import torch
+        if self.n == 0:
+            return
+        ptrs = (ctypes.c_void_p * len(mats))(*[m.data_ptr() for m in mats])
+        ld = _i64_array([m.stride(0) if m.dim() == 2 else m.shape[-1] for m in mats])
+        for m in mats:
+            if m.dim() != 2 or (m.shape[1] > 1 and m.stride(1) != 1):
+                raise ValueError("matrices must be 2-D with unit column stride")
+        dt = BF16 if mats[0].dtype == torch.bfloat16 else F32
+        if packed.dtype != torch.float32 or not packed.is_contiguous():
+            raise ValueError("the packed buffer must be contiguous float32")
+        _check(lib.shampoo_pack_blocks(self.table.data_ptr(), self.n, len(mats), ptrs, ld, dt, packed.data_ptr(),
+                                       direction, scale, self.max_rows, self.max_cols, _stream_ptr(stream)))
+
+    def gather(self, mats, packed, scale: float = 1.0, stream=None):
+        self._call(mats, packed, 0, scale, stream)
+
+    def scatter(self, packed, mats, stream=None):
+        self._call(mats, packed, 1, 1.0, stream)
 
 
 # ---------------------------------------------------------------------------

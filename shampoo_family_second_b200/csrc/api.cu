@@ -53,6 +53,8 @@ int validate_config(const shampoo_config* c) {
   }
   if (c->grad_dtype != SHAMPOO_F32 && c->grad_dtype != SHAMPOO_BF16)
     return set_error(SHAMPOO_ERR_INVALID_ARG, "grad_dtype must be SHAMPOO_F32 or SHAMPOO_BF16");
+  if (!(c->momentum >= 0.f) || !(c->momentum < 1.f))
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "momentum must be in [0, 1)");
   return SHAMPOO_OK;
 }
 
@@ -82,10 +84,11 @@ int build_table(int B, int32_t nparams, const int64_t* rows, const int64_t* cols
 // State layout (bytes, each part 256-aligned):
 //   status word | block table (nb x 5 int32) | valid extents (2nb int32: r of L_b, c of R_b)
 //   | wrows (nb) | wcols (nb) | statistics (2nb, B, B) | roots (2nb, B, B)
+//   | momentum (nb, B, B; only with momentum > 0)
 struct StateLayout {
-  size_t status, table, valid, wrows, wcols, stats, roots, total;
+  size_t status, table, valid, wrows, wcols, stats, roots, mom, total;
 };
-StateLayout state_layout(int nb, int B) {
+StateLayout state_layout(int nb, int B, bool momentum) {
   StateLayout s;
   size_t o = 0;
   s.status = o, o += al(4);
@@ -95,6 +98,8 @@ StateLayout state_layout(int nb, int B) {
   s.wcols = o, o += al(size_t(nb) * 4);
   s.stats = o, o += al(plain_floats(2 * nb, B) * 4);
   s.roots = o, o += al(plain_floats(2 * nb, B) * 4);
+  s.mom = o;
+  if (momentum) o += al(plain_floats(nb, B) * 4);
   s.total = o;
   return s;
 }
@@ -102,7 +107,7 @@ StateLayout state_layout(int nb, int B) {
 struct ScratchLayout {
   size_t gs, gt, tap, wptr, ld, root, root_bytes, total;
 };
-ScratchLayout scratch_layout(int nb, int B, int solver) {
+ScratchLayout scratch_layout(int nb, int B, int solver, int p) {
   ScratchLayout s;
   size_t o = 0;
   s.gs = o, o += al(plain_floats(nb, B) * 4);
@@ -111,7 +116,7 @@ ScratchLayout scratch_layout(int nb, int B, int solver) {
   s.wptr = o, o += al(size_t(nb) * 8);
   s.ld = o, o += al(size_t(nb) * 4);
   s.root = o;
-  const size_t per = root_scratch_per_matrix(B, solver);
+  const size_t per = root_scratch_per_matrix(B, solver, p);
   const size_t want = root_scratch_header() + per * size_t(2 * nb);
   s.root_bytes = std::min(want, std::max(kRootBudget, root_scratch_header() + per));
   o += al(s.root_bytes);
@@ -139,12 +144,13 @@ struct shampoo_ctx {
   int* d_wcols = nullptr;
   float* stats = nullptr;
   float* roots = nullptr;
+  float* mom = nullptr;  // momentum stack (momentum > 0 only)
   float* Gs = nullptr;
   float* Gt = nullptr;
   float* Tap = nullptr;
   float** blk_wptr = nullptr;
   int* blk_ld = nullptr;
-  StackMaps mGs, mGt, mRoots, mTap;
+  StackMaps mGs, mGt, mRoots, mTap, mMom;
   double stats_flops_L = 0, stats_flops_R = 0, stack_bytes = 0;
   int64_t step = 0;
   cudaStream_t last_stream = nullptr;
@@ -171,8 +177,8 @@ int shampoo_query_sizes(const shampoo_config* cfg, int32_t nparams, const int64_
   Shapes sh;
   if ((rc = build_table(cfg->block, nparams, rows, cols, sh))) return rc;
   if (!state_bytes || !scratch_bytes) return set_error(SHAMPOO_ERR_INVALID_ARG, "output pointer is NULL");
-  *state_bytes = state_layout(sh.nb, cfg->block).total;
-  *scratch_bytes = scratch_layout(sh.nb, cfg->block, cfg->solver).total;
+  *state_bytes = state_layout(sh.nb, cfg->block, cfg->momentum > 0.f).total;
+  *scratch_bytes = scratch_layout(sh.nb, cfg->block, cfg->solver, cfg->root_p).total;
   return SHAMPOO_OK;
 }
 
@@ -188,8 +194,8 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
   if (!aligned256(d_state) || !aligned256(d_scratch))
     return set_error(SHAMPOO_ERR_UNSUPPORTED, "state/scratch must be 256-byte aligned");
   const int B = cfg->block, nb = sh.nb;
-  StateLayout sl = state_layout(nb, B);
-  ScratchLayout xl = scratch_layout(nb, B, cfg->solver);
+  StateLayout sl = state_layout(nb, B, cfg->momentum > 0.f);
+  ScratchLayout xl = scratch_layout(nb, B, cfg->solver, cfg->root_p);
   if (state_bytes < sl.total) return set_error(SHAMPOO_ERR_WORKSPACE, "state %zu < %zu bytes", state_bytes, sl.total);
   if (scratch_bytes < xl.total)
     return set_error(SHAMPOO_ERR_WORKSPACE, "scratch %zu < %zu bytes", scratch_bytes, xl.total);
@@ -212,6 +218,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
   h->d_wcols = reinterpret_cast<int*>(h->state + sl.wcols);
   h->stats = reinterpret_cast<float*>(h->state + sl.stats);
   h->roots = reinterpret_cast<float*>(h->state + sl.roots);
+  h->mom = cfg->momentum > 0.f ? reinterpret_cast<float*>(h->state + sl.mom) : nullptr;
   h->Gs = reinterpret_cast<float*>(h->scratch + xl.gs);
   h->Gt = reinterpret_cast<float*>(h->scratch + xl.gt);
   h->Tap = reinterpret_cast<float*>(h->scratch + xl.tap);
@@ -229,6 +236,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
     fl += 2 * r * r * c;
     fr += 2 * r * c * c;
     sb += r * c * (cfg->grad_dtype == SHAMPOO_BF16 ? 2 : 4) + 8.0 * B * B;  // G read; Gs, Gt written
+    if (cfg->momentum > 0.f) sb += 8.0 * B * B;                                 // M read and written
   }
   h->stats_flops_L = fl / nb;
   h->stats_flops_R = fr / nb;
@@ -244,12 +252,14 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
       (rc = check_cuda(cudaMemsetAsync(h->d_status, 0, 4, st), "zero status")) ||
       (rc = check_cuda(cudaMemsetAsync(h->stats, 0, plain_floats(2 * nb, B) * 4, st), "zero statistics")) ||
       (rc = check_cuda(cudaMemsetAsync(h->roots, 0, plain_floats(2 * nb, B) * 4, st), "zero roots")) ||
+      (h->mom && (rc = check_cuda(cudaMemsetAsync(h->mom, 0, plain_floats(nb, B) * 4, st), "zero momentum"))) ||
       (rc = check_cuda(cudaStreamSynchronize(st), "init sync"))) {
     delete h;
     return rc;
   }
   if ((rc = make_stack_maps(h->mGs, h->Gs, nb, B)) || (rc = make_stack_maps(h->mGt, h->Gt, nb, B)) ||
-      (rc = make_stack_maps(h->mRoots, h->roots, 2 * nb, B)) || (rc = make_stack_maps(h->mTap, h->Tap, nb, B))) {
+      (rc = make_stack_maps(h->mRoots, h->roots, 2 * nb, B)) || (rc = make_stack_maps(h->mTap, h->Tap, nb, B)) ||
+      (h->mom && (rc = make_stack_maps(h->mMom, h->mom, nb, B)))) {
     delete h;
     return rc;
   }
@@ -284,27 +294,40 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;
   int rc;
-  // 1. partition / stack
-  if ((rc = launch_stack(args, h->d_table, nb, B, c.grad_dtype, h->Gs, h->Gt, h->blk_wptr, h->blk_ld, st,
-                         h->stack_bytes)))
+  // 1. partition / stack (and, with momentum, M <- alpha M + G per block)
+  if ((rc = launch_stack(args, h->d_table, nb, B, c.grad_dtype, h->Gs, h->Gt, h->mom, c.momentum, h->blk_wptr,
+                         h->blk_ld, st, h->stack_bytes)))
     return rc;
+  // Widened bf16 gradients are exact in tf32: their lo parts are zero, so
+  // the products that take G as an operand skip the MMAs with those parts.
+  const int g_exact = c.grad_dtype == SHAMPOO_BF16 ? 1 : 0;
   // 2. statistics: L <- beta L + G G^T (first nb matrices), R <- beta R + G^T G (next nb).
   // On steps that keep the previous roots, the first apply product T = XL G
-  // depends on neither, so it joins the same launch.
+  // (T = XL M with momentum, M read as a true product) depends on neither, so
+  // it joins the same launch.
   const bool refresh = h->step % c.refresh_every == 0;
   auto add_apply1 = [&](Builder& b) {
-    Epilogue& e = b.add(nb, B, h->mRoots, 0, h->mGt, 0, h->stats_flops_L);
-    e.D = h->Tap;
-    e.flags = h->d_status;
+    if (h->mom) {
+      Epilogue& e = b.add(nb, B, h->mRoots, 0, h->mMom, 0, h->stats_flops_L, B_MN_MAJOR);
+      e.D = h->Tap;
+      e.flags = h->d_status;
+    } else {
+      Epilogue& e = b.add(nb, B, h->mRoots, 0, h->mGt, 0, h->stats_flops_L);
+      b.L.g[b.L.ngroups - 1].b_exact = g_exact;
+      e.D = h->Tap;
+      e.flags = h->d_status;
+    }
   };
   {
     Builder b;
     Epilogue& eL = b.add(nb, B, h->mGs, 0, h->mGs, 0, h->stats_flops_L);
+    b.L.g[0].a_exact = b.L.g[0].b_exact = g_exact;
     eL.beta = c.beta;
     eL.C = h->stats;
     eL.D = h->stats;
     eL.flags = h->d_status;
     Epilogue& eR = b.add(nb, B, h->mGt, 0, h->mGt, 0, h->stats_flops_R);
+    b.L.g[1].a_exact = b.L.g[1].b_exact = g_exact;
     eR.beta = c.beta;
     eR.C = h->stats + plain_floats(nb, B);
     eR.D = h->stats + plain_floats(nb, B);
@@ -381,6 +404,12 @@ int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, f
   return SHAMPOO_OK;
 }
 
+int shampoo_momentum_view(shampoo_handle h, float** M) {
+  if (!h || !M) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle/M is NULL");
+  *M = h->mom;
+  return SHAMPOO_OK;
+}
+
 int shampoo_set_step(shampoo_handle h, int64_t step) {
   if (!h || step < 0) return set_error(SHAMPOO_ERR_INVALID_ARG, "bad handle or step");
   h->step = step;
@@ -390,21 +419,32 @@ int shampoo_set_step(shampoo_handle h, int64_t step) {
 void shampoo_destroy(shampoo_handle h) { delete h; }
 
 int inv_root_scratch_bytes(int64_t batch, int32_t n, int32_t solver, size_t* bytes) {
+  return inv_root_scratch_bytes_p(batch, n, solver, 4, bytes);
+}
+
+int inv_root_scratch_bytes_p(int64_t batch, int32_t n, int32_t solver, int32_t p, size_t* bytes) {
   if (!bytes) return set_error(SHAMPOO_ERR_INVALID_ARG, "bytes is NULL");
   if (batch < 0 || n < 32 || n > 1024 || n % 32 || solver < 0 || solver > 3)
     return set_error(SHAMPOO_ERR_INVALID_ARG, "bad batch / n / solver");
-  *bytes = root_scratch_header() + root_scratch_per_matrix(n, solver) * static_cast<size_t>(std::max<int64_t>(batch, 1));
+  if (p != 2 && p != 4 && p != 6 && p != 8) return set_error(SHAMPOO_ERR_INVALID_ARG, "p must be 2, 4, 6 or 8");
+  *bytes = root_scratch_header() +
+           root_scratch_per_matrix(n, solver, p) * static_cast<size_t>(std::max<int64_t>(batch, 1));
   return SHAMPOO_OK;
 }
 
-int inv_root_batched(const float* d_A, float* d_X, int64_t batch, int32_t n, int32_t p, float eps, int32_t solver,
-                     int32_t iters, float tol, int32_t cheb_degree, float cheb_lo, void* d_scratch,
-                     size_t scratch_bytes, int32_t* d_iters_used, int32_t* d_status, void* stream) {
+}  // extern "C"
+
+int shampoo::inv_root_batched_impl(const float* d_A, float* d_X, int64_t batch, int n, int p, float eps, int solver,
+                                   int iters, float tol, int cheb_degree, float cheb_lo, void* d_scratch,
+                                   size_t scratch_bytes, int* d_iters_used, int* d_status, cudaStream_t st,
+                                   bool plain_launches) {
   if (batch < 0) return set_error(SHAMPOO_ERR_INVALID_ARG, "batch < 0");
   if (batch == 0) return SHAMPOO_OK;
   if (!d_A || !d_X || !d_scratch) return set_error(SHAMPOO_ERR_INVALID_ARG, "NULL device pointer");
   if (n < 32 || n > 1024 || n % 32) return set_error(SHAMPOO_ERR_INVALID_ARG, "n %d: need a multiple of 32 in [32, 1024]", n);
-  if (p != 2 && p != 4) return set_error(SHAMPOO_ERR_INVALID_ARG, "p must be 2 or 4");
+  if (p != 2 && p != 4 && p != 6 && p != 8) return set_error(SHAMPOO_ERR_INVALID_ARG, "p must be 2, 4, 6 or 8");
+  if (solver == SHAMPOO_SOLVER_NEWTON_DB && p > 4)
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "Newton-DB computes p = 2 and p = 4 only");
   if (!(eps >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "eps must be >= 0");
   if (solver < 0 || solver > 3) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", solver);
   if (solver != SHAMPOO_SOLVER_CHEBYSHEV && (iters < 1 || iters > 1000))
@@ -433,8 +473,19 @@ int inv_root_batched(const float* d_A, float* d_X, int64_t batch, int32_t n, int
   job.X = d_X;
   job.iters_used = d_iters_used;
   job.flags = d_status;
-  return run_inverse_roots(job, d_scratch, scratch_bytes, static_cast<cudaStream_t>(stream));
+  job.plain_launches = plain_launches ? 1 : 0;
+  return run_inverse_roots(job, d_scratch, scratch_bytes, st);
 }
+
+extern "C" {
+
+int inv_root_batched(const float* d_A, float* d_X, int64_t batch, int32_t n, int32_t p, float eps, int32_t solver,
+                     int32_t iters, float tol, int32_t cheb_degree, float cheb_lo, void* d_scratch,
+                     size_t scratch_bytes, int32_t* d_iters_used, int32_t* d_status, void* stream) {
+  return inv_root_batched_impl(d_A, d_X, batch, n, p, eps, solver, iters, tol, cheb_degree, cheb_lo, d_scratch,
+                               scratch_bytes, d_iters_used, d_status, static_cast<cudaStream_t>(stream), false);
+}
+
 
 int shampoo_gemm_scratch_bytes(int64_t batch, int32_t n, size_t* bytes) {
   if (!bytes || batch < 0 || n < 32 || n > 4096 || n % 32)

@@ -99,9 +99,9 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmLaunch& L, int tile) {
 // tile with asynchronous 16-byte copies, in the tile's swizzled layout (piece
 // k of row R at R * 32 + ((k ^ (R & 7)) << 2)); each 8-lane group copies one
 // 128-byte row piece.  The copies are waited for in epilogue_chunk.
-__device__ __forceinline__ void stage_c(const Epilogue& E, int n, int mat, int row0, int c0, float* tilebuf,
+__device__ __forceinline__ void stage_c(const Epilogue& E, int m, int n, int mat, int row0, int c0, float* tilebuf,
                                         int lane) {
-  const float* base = E.C + static_cast<size_t>(mat) * n * n + static_cast<size_t>(row0) * n + c0;
+  const float* base = E.C + static_cast<size_t>(mat) * m * n + static_cast<size_t>(row0) * n + c0;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int R = 4 * j + (lane >> 3);
@@ -128,7 +128,8 @@ __device__ __forceinline__ void stage_c(const Epilogue& E, int n, int mat, int r
 __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int row0, int c0, const float* acc,
                                                float* tilebuf, int lane, float& resid, bool& bad, bool c_staged) {
   const Epilogue& E = G.ep;
-  const int n = G.n;
+  const int n = G.n;  // columns (the row stride of C, D, E)
+  const int m = G.m;  // rows
   const int r = row0 + lane;
   const int dj = r - c0;  // column of this row's diagonal element within the chunk
   const float gam = E.gamma_vec ? E.gamma_vec[static_cast<size_t>(mat) * E.gamma_stride] : E.gamma;
@@ -139,7 +140,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
       if (j == dj && r < vsz) resid += 1.f - acc[j];
   }
   if (E.C) {
-    if (!c_staged) stage_c(E, n, mat, row0, c0, tilebuf, lane);
+    if (!c_staged) stage_c(E, m, n, mat, row0, c0, tilebuf, lane);
     cp_async_wait_all();
     __syncwarp();
   }
@@ -161,7 +162,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
     *slot = w;
   }
   __syncwarp();
-  const size_t nn = static_cast<size_t>(n) * n;
+  const size_t nn = static_cast<size_t>(m) * n;
   const float sc = E.scale_vec ? E.scale_vec[mat] : 1.f;
   float* wbase = nullptr;
   int wld = 0, wr = 0, wc = 0;
@@ -178,7 +179,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
     const int gr = row0 + R;
     const int gc = c0 + 4 * kq;
     float4 v = *reinterpret_cast<const float4*>(tilebuf + R * 32 + ((kq ^ (R & 7)) << 2));
-    if (gr < n) {
+    if (gr < m) {
       const size_t off = static_cast<size_t>(mat) * nn + static_cast<size_t>(gr) * n + gc;
       v.x *= sc;
       v.y *= sc;
@@ -272,7 +273,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const TileCoord tc = tile_coord(L, tile);
           if (tc.skip) continue;
           const GemmGroup& G = L.g[tc.gi];
-          const int nk = G.n / BK;
+          const int nk = (G.k + BK - 1) / BK;
           const uint32_t tx_bytes = static_cast<uint32_t>(G.a_rows + G.b_rows) * BK * 4u;
           const void* amap = &maps.m[G.a_map];
           const void* bmap = &maps.m[G.b_map];
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const TileCoord tc = tile_coord(L, tile);
           if (tc.skip) continue;
           const GemmGroup& G = L.g[tc.gi];
-          const int nk = G.n / BK;
+          const int nk = (G.k + BK - 1) / BK;
           const uint32_t idesc = idesc_tf32(BM, BN, G.b_mn);
 #pragma unroll 1
           for (int kc = 0; kc < nk; ++kc, ++it) {
@@ -358,8 +359,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 dbl = smem_desc_k_sw64(b_lo + off);
               }
               mma_tf32(tbuf, dah, dbh, idesc, (first && ks == 0) ? 0u : 1u);
-              mma_tf32(tbuf, dah, dbl, idesc, 1u);
-              mma_tf32(tbuf, dal, dbh, idesc, 1u);
+              if (!G.b_exact) mma_tf32(tbuf, dah, dbl, idesc, 1u);
+              if (!G.a_exact) mma_tf32(tbuf, dal, dbh, idesc, 1u);
             }
             mma_commit(&empty[s]);
             if ((kc % SEG) == SEG - 1 || kc == nk - 1) {
@@ -381,7 +382,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileCoord tc = tile_coord(L, tile);
         if (tc.skip) continue;
-        const int nk = L.g[tc.gi].n / BK;
+        const GemmGroup& G = L.g[tc.gi];
+        const int nk = (G.k + BK - 1) / BK;
+        // An operand whose values are exact in tf32 needs no split: its hi
+        // part is the value as TMA wrote it, and its lo part is never read.
+        const bool keep_a = G.a_exact != 0, keep_b = G.b_exact != 0;
 #pragma unroll 1
         for (int kc = 0; kc < nk; ++kc, ++it) {
           const int s = it % STAGES;
@@ -393,6 +398,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int i = 0; i < RAW_BYTES / 16 / CONV_THREADS; ++i) {
             const int off = (i * CONV_THREADS + ct) * 16;
+            if (off < A_BYTES ? keep_a : keep_b) continue;
             const float4 x = *reinterpret_cast<const float4*>(base + off);
             float4 h, l;
             split_tf32(x.x, h.x, l.x);
@@ -427,13 +433,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (tc.skip) continue;
       const GemmGroup& G = L.g[tc.gi];
       const int n = G.n;
-      const int nseg = (n / BK + SEG - 1) / SEG;
+      const int m = G.m;
+      const int nseg = ((G.k + BK - 1) / BK + SEG - 1) / SEG;
       // C of this warp's first chunk streams into its shared tile while the
       // tile's MMAs run.
       const int row0_first = tc.tm * BM + q * 32;
       const int c0_first = tc.tn * BN + h * (BN / 2);
-      const bool staged0 = G.ep.C && row0_first < n && c0_first < n;
-      if (staged0) stage_c(G.ep, n, tc.mat, row0_first, c0_first, tilebuf, lane);
+      const bool staged0 = G.ep.C && row0_first < m && c0_first < n;
+      if (staged0) stage_c(G.ep, m, n, tc.mat, row0_first, c0_first, tilebuf, lane);
       float sum[BN / 2];
 #pragma unroll
       for (int j = 0; j < BN / 2; ++j) sum[j] = 0.f;
@@ -464,7 +471,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       float resid = 0.f;
       bool nonfinite = false;
       const int row0 = tc.tm * BM + q * 32;
-      if (row0 < n) {
+      if (row0 < m) {
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c) {
           const int c0 = tc.tn * BN + h * (BN / 2) + c * 32;
@@ -515,18 +522,21 @@ int get_encoder() {
 }
 }  // namespace
 
-// Tensor map over a plain stack (batch, n, n) fp32: dimensions (innermost
-// first) column = n, row = n, matrix = batch.  K-major operand tiles (box
-// box_rows x 16) use the 64-byte swizzle; MN-major tiles (mn_layout: 16 rows
-// of K x 32 columns) the 128-byte swizzle with 32-byte atoms, the only
-// MN-major tf32 layout of the tensor core.
-int encode_stack_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout) {
+// Tensor map over a stack (batch, rows, cols) of row-major fp32 matrices:
+// dimensions (innermost first) column = cols, row = rows, matrix = batch.
+// K-major operand tiles (box box_rows x 16) use the 64-byte swizzle; MN-major
+// tiles (mn_layout: 16 rows of K x 32 columns) the 128-byte swizzle with
+// 32-byte atoms, the only MN-major tf32 layout of the tensor core.  Boxes that
+// reach past rows or cols read zeros.
+int encode_stack_map(CUtensorMap* map, const float* base, int64_t batch, int rows, int cols, int box_rows,
+                     int mn_layout) {
   int rc = get_encoder();
   if (rc) return rc;
   if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return set_error(-2, "stack base not 16-byte aligned");
-  const cuuint64_t nn = static_cast<cuuint64_t>(n);
-  cuuint64_t dims[3] = {nn, nn, static_cast<cuuint64_t>(batch)};
-  cuuint64_t strides[2] = {nn * 4, nn * nn * 4};
+  if (cols % 4 != 0) return set_error(-2, "stack rows of %d floats are not 16-byte multiples", cols);
+  const cuuint64_t nr = static_cast<cuuint64_t>(rows), nc = static_cast<cuuint64_t>(cols);
+  cuuint64_t dims[3] = {nc, nr, static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {nc * 4, nr * nc * 4};
   // K-major boxes: BK columns (64 bytes) x box_rows rows; MN-major boxes: 32
   // columns (128 bytes) x box_rows (= BK) rows of K.
   cuuint32_t box[3] = {static_cast<cuuint32_t>(mn_layout ? 32 : BK), static_cast<cuuint32_t>(box_rows), 1};
@@ -540,14 +550,20 @@ int encode_stack_map(CUtensorMap* map, const float* base, int64_t batch, int n, 
   return 0;
 }
 
-int make_stack_maps(StackMaps& sm, const float* base, int64_t batch, int n) {
+int make_rect_maps(StackMaps& sm, const float* base, int64_t batch, int rows, int cols) {
   sm.base = const_cast<float*>(base);
-  sm.a_rows = n < BM ? n : BM;
-  sm.b_rows = n < BN ? n : BN;
-  int rc = encode_stack_map(&sm.a, base, batch, n, sm.a_rows, 0);
+  sm.rows = rows;
+  sm.cols = cols;
+  sm.a_rows = rows < BM ? rows : BM;
+  sm.b_rows = rows < BN ? rows : BN;
+  int rc = encode_stack_map(&sm.a, base, batch, rows, cols, sm.a_rows, 0);
   if (rc) return rc;
-  if ((rc = encode_stack_map(&sm.mn, base, batch, n, BK, 1))) return rc;
-  return encode_stack_map(&sm.b, base, batch, n, sm.b_rows, 0);
+  if ((rc = encode_stack_map(&sm.mn, base, batch, rows, cols, BK, 1))) return rc;
+  return encode_stack_map(&sm.b, base, batch, rows, cols, sm.b_rows, 0);
+}
+
+int make_stack_maps(StackMaps& sm, const float* base, int64_t batch, int n) {
+  return make_rect_maps(sm, base, batch, n, n);
 }
 
 Builder::Builder() : nmaps(0) {
@@ -560,6 +576,8 @@ Epilogue& Builder::add(int batch, int n, const StackMaps& a, int a_off, const St
   GemmGroup& g = L.g[L.ngroups++];
   g.batch = batch;
   g.n = n;
+  g.m = n;
+  g.k = n;
   M.m[nmaps] = a.a;
   g.a_map = nmaps++;
   M.m[nmaps] = bmode == B_MN_MAJOR ? b.mn : b.b;
@@ -572,6 +590,17 @@ Epilogue& Builder::add(int batch, int n, const StackMaps& a, int a_off, const St
   g.flops_per_matrix = flops_per_matrix;
   g.ep = epilogue_defaults();
   return g.ep;
+}
+
+Epilogue& Builder::add_rect(int batch, int Mr, int N, int K, const StackMaps& a, int a_off, const StackMaps& b,
+                            int b_off, double flops_per_matrix, int bmode) {
+  Epilogue& e = add(batch, N, a, a_off, b, b_off, flops_per_matrix, bmode);
+  GemmGroup& g = L.g[L.ngroups - 1];
+  g.m = Mr;
+  g.k = K;
+  g.a_rows = Mr < BM ? Mr : BM;
+  g.b_rows = N < BN ? N : BN;
+  return e;
 }
 
 int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
@@ -599,7 +628,7 @@ int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
   double flops = 0;
   for (int i = 0; i < L.ngroups; ++i) {
     GemmGroup& g = L.g[i];
-    g.tiles_m = (g.n + BM - 1) / BM;
+    g.tiles_m = (g.m + BM - 1) / BM;
     g.tiles_n = (g.n + BN - 1) / BN;
     g.cta_begin = static_cast<int>(total);
     total += static_cast<int64_t>(g.batch) * g.tiles_m * g.tiles_n;

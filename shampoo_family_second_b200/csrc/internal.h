@@ -50,11 +50,15 @@ struct Epilogue {
 
 struct GemmGroup {
   int batch;       // matrices in this group
-  int n;           // square size (multiple of 32)
+  int n;           // columns N of B and D (multiple of 32); square products: also M and K
+  int m, k;        // rows M of A and D (multiple of 32), depth K (multiple of 4)
   int a_map, b_map;  // tensor-map slots (A as 128-row boxes, B as 256-row boxes)
   int a_off, b_off;  // matrix index offsets into the mapped stacks
   int a_rows, b_rows;  // box rows of the two maps (min(tile, n))
   int b_mn;            // 1: B is read MN-major (D = A B); 0: K-major (D = A B^T)
+  int a_exact, b_exact;  // 1: every value of the operand is exact in tf32 (e.g. widened bf16), so its
+                         // lo part is zero: the MMAs with that lo part are skipped and its tiles are
+                         // not split
   int tiles_m, tiles_n, cta_begin;  // filled by launch_gemm (cta_begin: first tile of the group)
   double flops_per_matrix;          // algorithmic flops (profiling only)
   Epilogue ep;
@@ -78,7 +82,8 @@ constexpr int kTileN = 256;
 constexpr int kTileK = 16;
 
 // Host helpers -------------------------------------------------------------
-int encode_stack_map(CUtensorMap* map, const float* base, int64_t batch, int n, int box_rows, int mn_layout);
+int encode_stack_map(CUtensorMap* map, const float* base, int64_t batch, int rows, int cols, int box_rows,
+                     int mn_layout);
 int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st);
 Epilogue epilogue_defaults();
 
@@ -124,8 +129,11 @@ struct StackMaps {
   CUtensorMap mn;    // as MN-major B: 16 rows of K x 32 columns of N
   float* base;
   int a_rows, b_rows;
+  int rows, cols;    // shape of each matrix of the stack
 };
 int make_stack_maps(StackMaps& sm, const float* base, int64_t batch, int n);
+// A stack (batch, rows, cols) of row-major matrices (cols a multiple of 4).
+int make_rect_maps(StackMaps& sm, const float* base, int64_t batch, int rows, int cols);
 
 // How a group reads its B operand: as B^T (K-major; D = A B^T) or as B
 // (MN-major; D = A B).
@@ -140,6 +148,10 @@ struct Builder {
   // over matrices a_off.. of `a` and b_off.. of `b`.
   Epilogue& add(int batch, int n, const StackMaps& a, int a_off, const StackMaps& b, int b_off,
                 double flops_per_matrix, int bmode = B_TRANSPOSED);
+  // Rectangular: D_i (M x N) = epi(A_i op(B_i)), A_i M x K; B_i N x K (B_TRANSPOSED) or K x N
+  // (B_MN_MAJOR).  M and N multiples of 32, K a multiple of 4.
+  Epilogue& add_rect(int batch, int M, int N, int K, const StackMaps& a, int a_off, const StackMaps& b, int b_off,
+                     double flops_per_matrix, int bmode);
   int launch(cudaStream_t st) { return launch_gemm(L, M, st); }
 };
 
@@ -153,8 +165,9 @@ struct StackArgs {
   int ld[kMaxParams];
   unsigned char vec[kMaxParams];  // rows of param i start 16-byte (fp32) / 8-byte (bf16) aligned
 };
+// M (nullable): momentum stack, updated in place as M <- alpha M + G_b.
 int launch_stack(const StackArgs& args, const int* d_table, int nb, int B, int grad_dtype, float* Gs, float* Gts,
-                 float** blk_wptr, int* blk_ld, cudaStream_t st, double alg_bytes);
+                 float* M, float alpha, float** blk_wptr, int* blk_ld, cudaStream_t st, double alg_bytes);
 
 int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, float eps, int p, float* s, float* sc,
                      cudaStream_t st);
@@ -201,8 +214,15 @@ struct RootJob {
   float* X;          // output stack
   int* iters_used;   // device per-matrix iterations (nullable)
   int* flags;        // device status word (nullable)
+  int plain_launches = 0;  // 1: never build or run a CUDA graph loop (residual-checked loops are
+                           // issued as plain launches up to the cap)
 };
-size_t root_scratch_per_matrix(int n, int solver);
+// inv_root_batched with a switch for plain launches (shared by the public
+// entry points of api.cu and noalloc.cu).
+int inv_root_batched_impl(const float* d_A, float* d_X, int64_t batch, int n, int p, float eps, int solver, int iters,
+                          float tol, int cheb_degree, float cheb_lo, void* d_scratch, size_t scratch_bytes,
+                          int* d_iters_used, int* d_status, cudaStream_t st, bool plain_launches);
+size_t root_scratch_per_matrix(int n, int solver, int p);
 size_t root_scratch_header();
 int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, cudaStream_t st);
 

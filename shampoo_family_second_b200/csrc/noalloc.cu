@@ -17,7 +17,10 @@
 // All calls share the one array and it keeps the last call's contents: the
 // solver clears what it needs zeroed (its residual accumulators) on every call,
 // and calls whose work overlaps on the GPU (different streams, or different
-// host threads on the same device) race on it.
+// host threads on the same device) race on it.  With tol > 0 the iterations
+// run as plain kernel launches up to the cap (the tiles of matrices that have
+// finished exit at once) rather than as a CUDA graph loop, because
+// instantiating a graph may take device memory.
 #include <mutex>
 
 #include "../../include/shampoo.h"
@@ -60,7 +63,7 @@ int inv_root_batched_noalloc(const float* d_A, float* d_X, int64_t batch, int32_
                              int32_t* d_iters_used, int32_t* d_status, void* stream) {
   if (batch == 0) return SHAMPOO_OK;
   size_t per_matrix = 0;
-  int rc = inv_root_scratch_bytes(1, n, solver, &per_matrix);
+  int rc = inv_root_scratch_bytes_p(1, n, solver, p, &per_matrix);
   if (rc) return rc;
   if (per_matrix > kNoAllocScratchBytes)
     return set_error(SHAMPOO_ERR_UNSUPPORTED,
@@ -70,8 +73,11 @@ int inv_root_batched_noalloc(const float* d_A, float* d_X, int64_t batch, int32_
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch))) return rc;
   // The solver works through the batch in chunks that fit the fixed scratch.
-  return inv_root_batched(d_A, d_X, batch, n, p, eps, solver, iters, tol, cheb_degree, cheb_lo, scratch,
-                          kNoAllocScratchBytes, d_iters_used, d_status, stream);
+  // Residual-checked loops are issued as plain launches: a CUDA graph loop
+  // would instantiate a graph, which the runtime may back with device memory.
+  return inv_root_batched_impl(d_A, d_X, batch, n, p, eps, solver, iters, tol, cheb_degree, cheb_lo, scratch,
+                               kNoAllocScratchBytes, d_iters_used, d_status, static_cast<cudaStream_t>(stream),
+                               true);
 }
 
 }  // extern "C"

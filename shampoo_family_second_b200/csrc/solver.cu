@@ -63,10 +63,13 @@ namespace {
 constexpr int NEWTON_B = B_MN_MAJOR;
 
 // Scratch stacks per solver (plain fp32, n x n per matrix):
-//   Newton    : M0 M1 X0 X1 T T2 T4 (both correction degrees)
+//   Newton    : M0 M1 X0 X1 T T2 T4 (both correction degrees), and T^p for p = 6, 8
 //   Newton-DB : Y0 Y1 Z0 Z1 T
 //   Chebyshev : Xt b0 b1 b2
-int stacks_for(int solver) { return (solver == 0 || solver == 3) ? 7 : (solver == 1 ? 5 : 4); }
+int stacks_for(int solver, int p) {
+  if (solver == 0 || solver == 3) return p >= 6 ? 8 : 7;
+  return solver == 1 ? 5 : 4;
+}
 
 constexpr size_t kAlign = 256;
 constexpr size_t kHeader = 64 * 1024;  // covers the alignment padding of the arrays
@@ -82,8 +85,10 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // 3.52 at p = 2), reaching 1/2 within 13 (resp. 14) iterations counting the
 // plain first step, followed by cubic steps.
 int kmin_newton(int p, bool order2) {
-  if (order2) return p == 4 ? 17 : 18;
-  return p == 4 ? 24 : 26;
+  // p = 6, 8 grow small eigenvalues at least as fast as p = 4 ((7/6)^6 = 2.52,
+  // (9/8)^8 = 2.57; second degree 4.08, 4.17) and take its thresholds.
+  if (order2) return p >= 4 ? 17 : 18;
+  return p >= 4 ? 24 : 26;
 }
 constexpr int kPowerIters = 12;  // power-iteration steps of the coupled-Newton scale
 constexpr int kKminSqrt = 26;
@@ -99,10 +104,10 @@ struct Layout {
   int* iters;
   int* iters1;
   float* coef;
-  float* stack[7];
+  float* stack[8];
 };
 
-Layout carve(void* base, int64_t cb, int n, int solver) {
+Layout carve(void* base, int64_t cb, int n, int solver, int root_p) {
   Layout L;
   std::memset(&L, 0, sizeof(L));
   char* p = static_cast<char*>(base);
@@ -121,7 +126,7 @@ Layout carve(void* base, int64_t cb, int n, int solver) {
   L.iters = reinterpret_cast<int*>(take(cb * 4));
   L.iters1 = reinterpret_cast<int*>(take(cb * 4));
   L.coef = reinterpret_cast<float*>(take(cb * 4 * (kMaxChebDegree + 2)));
-  for (int k = 0; k < stacks_for(solver); ++k)
+  for (int k = 0; k < stacks_for(solver, root_p); ++k)
     L.stack[k] = reinterpret_cast<float*>(take(plain_floats(cb, n) * 4));
   return L;
 }
@@ -275,15 +280,15 @@ int run_loop(const LoopKey& key, int kernels_per_iter, Body&& body, cudaStream_t
 
 size_t root_scratch_header() { return kHeader; }
 
-size_t root_scratch_per_matrix(int n, int solver) {
-  return static_cast<size_t>(stacks_for(solver)) * n * n * 4 + 4 * (kVecInts + kMaxChebDegree + 2);
+size_t root_scratch_per_matrix(int n, int solver, int p) {
+  return static_cast<size_t>(stacks_for(solver, p)) * n * n * 4 + 4 * (kVecInts + kMaxChebDegree + 2);
 }
 
 int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, cudaStream_t st) {
   const int n = job.n;
   const int p = job.p;
   const bool residual = job.tol > 0.f && job.solver != 2;
-  const size_t per = root_scratch_per_matrix(n, job.solver);
+  const size_t per = root_scratch_per_matrix(n, job.solver, p);
   if (scratch_bytes < kHeader + per)
     return set_error(-3, "inverse-root scratch too small: %zu < %zu bytes", scratch_bytes, kHeader + per);
   const int64_t cb_max = std::min<int64_t>(job.batch, static_cast<int64_t>((scratch_bytes - kHeader) / per));
@@ -293,13 +298,13 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
   for (int64_t off = 0; off < job.batch; off += cb_cap) {
     const int64_t cb = std::min<int64_t>(cb_cap, job.batch - off);
     const int cbi = static_cast<int>(cb);
-    Layout S = carve(scratch, cb, n, job.solver);
+    Layout S = carve(scratch, cb, n, job.solver, p);
     const float* A = job.A + off * static_cast<int64_t>(n) * n;
     const int* valid = job.valid ? job.valid + off : nullptr;
     float* out = job.X + off * static_cast<int64_t>(n) * n;
     int* iters_out = job.iters_used ? job.iters_used + off : nullptr;
-    StackMaps sm[7];
-    for (int k = 0; k < stacks_for(job.solver); ++k)
+    StackMaps sm[8];
+    for (int k = 0; k < stacks_for(job.solver, p); ++k)
       if ((rc = make_stack_maps(sm[k], S.stack[k], cb, n))) return rc;
     // Coupled Newton scales by the power-iteration estimate (bounded by the
     // Frobenius norm); Newton-DB (convergent only on (0, 2)) and Chebyshev
@@ -323,7 +328,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
     // when available, else plain launches up to the cap.
     auto run_rest = [&](auto&& iterate, int kernels_per_iter) -> int {
       if (job.iters <= 1) return 0;
-      if (use_graph_loop(st)) {
+      if (!job.plain_launches && use_graph_loop(st)) {
         bool ran = false;
         int r = run_loop(key, kernels_per_iter,
                          [&](cudaStream_t cs, const GraphLoop* lp) {
@@ -363,6 +368,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       StackMaps& T = sm[4];
       StackMaps& T2 = sm[5];
       StackMaps& T4 = sm[6];
+      StackMaps& Tp = sm[7];  // T^6 or T^8 (p = 6, 8 only)
       // Second-degree correction (solver 3): from iteration 1 on,
       // T = I + c1 (I - M) + c2 (I - M)^2 with c1 = 1/p, c2 = (p+1)/(2p^2),
       // the first three terms of the binomial series of M^{-1/p} about I,
@@ -397,8 +403,8 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
         StackMaps* Dnext = nullptr;
         if (order2) {
           if (j >= 1) {
-            StackMaps* Db = p == 4 ? Q[j & 1] : Q[0];
-            Tb = p == 4 ? Q[(j + 1) & 1] : Q[1];
+            StackMaps* Db = p >= 4 ? Q[j & 1] : Q[0];
+            Tb = p >= 4 ? Q[(j + 1) & 1] : Q[1];
             T2b = Q[2];
             T4b = Db;
             Builder b;
@@ -411,7 +417,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
             common(e);
             if ((r = b.launch(cs))) return r;
           }
-          Dnext = p == 4 ? Q[(j + 1) & 1] : Q[0];
+          Dnext = p >= 4 ? Q[(j + 1) & 1] : Q[0];
         }
         // The last iteration of a fixed count only needs X <- X T.
         const bool last = !residual && j == job.iters - 1;
@@ -431,13 +437,21 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
         }
         if (last) return 0;
         StackMaps* P = T2b;
-        if (p == 4) {
+        if (p >= 4) {
           Builder b;
           Epilogue& e = b.add(cbi, n, *T2b, 0, *T2b, 0, f1, NEWTON_B);  // T4 = T2 T2
           e.D = T4b->base;
           common(e);
           if ((r = b.launch(cs))) return r;
           P = T4b;
+        }
+        if (p >= 6) {  // T6 = T4 T2, or T8 = T4 T4, into a stack no later launch of this iteration writes
+          Builder b;
+          Epilogue& e = b.add(cbi, n, *T4b, 0, p == 6 ? *T2b : *T4b, 0, f1, NEWTON_B);
+          e.D = Tp.base;
+          common(e);
+          if ((r = b.launch(cs))) return r;
+          P = &Tp;
         }
         {
           Builder b;
@@ -463,7 +477,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
         return 0;
       };
       if (residual) {
-        const int per_iter = (p == 4 ? 4 : 3) + (order2 ? 1 : 0);
+        const int per_iter = (p == 2 ? 3 : (p == 4 ? 4 : 5)) + (order2 ? 1 : 0);
         if ((rc = iterate(0, st, nullptr)) || (rc = run_rest(iterate, per_iter))) return rc;
       } else {
         for (int j = 0; j < job.iters; ++j)

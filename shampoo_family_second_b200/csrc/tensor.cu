@@ -1,0 +1,527 @@
+// Order-k tensor Shampoo (podcast transcript "Preconditioned optimization
+// without the full matrix cost", cue 26: one preconditioner per dimension of
+// the gradient tensor, built from the gradient contracted with itself over
+// every other dimension, applied by a contraction along its own dimension with
+// the power -1/(2k); the order of the modes does not matter).
+//
+// For a parameter of order k with dimensions d_0 .. d_{k-1}, every step:
+//   1. unfold   U_i = mode-i unfolding of G (d_i x prod_{l != i} d_l, the other
+//               indices in row-major order), zero-padded to npad_i x Kpad_i
+//               (multiples of 32);
+//   2. stats    H_i <- beta H_i + U_i U_i^T        (one GEMM launch, k groups);
+//   3. roots    every refresh_every steps, X_i = (H_i + eps I)^{-1/(2k)} for all
+//               modes of all parameters, batched by (npad, k);
+//   4. apply    V = X_0 U_0; then for i = 1 .. k-1: V <- X_i unfold_i(fold_{i-1}(V))
+//               (a permutation pass between the products), and the last
+//               fold writes W <- W - lr P into the weight.
+// Dimensions above 1024 are not supported (SHAMPOO_ERR_UNSUPPORTED).
+#include <algorithm>
+#include <cstring>
+#include <map>
+#include <new>
+#include <vector>
+
+#include "../../include/shampoo.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace shampoo;
+
+namespace {
+
+constexpr int kMaxOrder = 4;
+constexpr int kMaxTensorParams = 256;
+constexpr size_t kAlignT = 256;
+constexpr size_t kTensorRootBudget = size_t(8) << 30;
+
+size_t alt(size_t x) { return (x + kAlignT - 1) / kAlignT * kAlignT; }
+int up32(int64_t x) { return static_cast<int>((x + 31) / 32 * 32); }
+
+// Layout of one side of a permutation: the natural row-major tensor
+// (mode = -1) or the mode-`mode` unfolding with row stride `ld`.
+struct PermSide {
+  int mode;
+  int64_t ld;
+};
+
+struct PermArgs {
+  int k;
+  int dims[kMaxOrder];
+  const void* src;
+  int src_bf16;
+  PermSide s;
+  float* dst;
+  PermSide d;
+  int rows, cols;  // destination extent written (unfolding: padded rows x padded cols)
+  float lr;        // fold into the weight: dst[idx] -= lr * value
+  int update;
+};
+
+// Multi-index of column c of the mode-m unfolding (other indices row-major).
+__device__ __forceinline__ void unfold_col_index(const PermArgs& a, int m, int64_t c, int* idx) {
+#pragma unroll
+  for (int l = kMaxOrder - 1; l >= 0; --l) {
+    if (l >= a.k || l == m) continue;
+    idx[l] = static_cast<int>(c % a.dims[l]);
+    c /= a.dims[l];
+  }
+}
+
+__device__ __forceinline__ int64_t natural_offset(const PermArgs& a, const int* idx) {
+  int64_t o = 0;
+#pragma unroll
+  for (int l = 0; l < kMaxOrder; ++l)
+    if (l < a.k) o = o * a.dims[l] + idx[l];
+  return o;
+}
+
+__device__ __forceinline__ int64_t unfold_offset(const PermArgs& a, const PermSide& sd, const int* idx) {
+  int64_t c = 0;
+#pragma unroll
+  for (int l = 0; l < kMaxOrder; ++l)
+    if (l < a.k && l != sd.mode) c = c * a.dims[l] + idx[l];
+  return static_cast<int64_t>(idx[sd.mode]) * sd.ld + c;
+}
+
+// One thread per destination element.  Unfolding destinations are written
+// whole, zeros in the padding; a natural destination (the weight) is updated
+// in place, W[idx] -= lr * P[idx].
+__global__ void tensor_permute_kernel(const __grid_constant__ PermArgs a, int64_t total) {
+  pdl_launch_dependents();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= total) return;
+  int idx[kMaxOrder] = {0, 0, 0, 0};
+  bool inside = true;
+  int64_t dst_off;
+  if (a.d.mode < 0) {
+    int64_t r = t;
+#pragma unroll
+    for (int l = kMaxOrder - 1; l >= 0; --l) {
+      if (l >= a.k) continue;
+      idx[l] = static_cast<int>(r % a.dims[l]);
+      r /= a.dims[l];
+    }
+    dst_off = t;
+  } else {
+    const int row = static_cast<int>(t / a.cols);
+    const int64_t col = t - static_cast<int64_t>(row) * a.cols;
+    int64_t kcols = 1;
+#pragma unroll
+    for (int l = 0; l < kMaxOrder; ++l)
+      if (l < a.k && l != a.d.mode) kcols *= a.dims[l];
+    inside = row < a.dims[a.d.mode] && col < kcols;
+    if (inside) {
+      idx[a.d.mode] = row;
+      unfold_col_index(a, a.d.mode, col, idx);
+    }
+    dst_off = static_cast<int64_t>(row) * a.d.ld + col;
+  }
+  float v = 0.f;
+  if (inside) {
+    const int64_t so = a.s.mode < 0 ? natural_offset(a, idx) : unfold_offset(a, a.s, idx);
+    if (a.src_bf16) {
+      const uint16_t bits = reinterpret_cast<const uint16_t*>(a.src)[so];
+      v = __uint_as_float(static_cast<uint32_t>(bits) << 16);
+    } else {
+      v = reinterpret_cast<const float*>(a.src)[so];
+    }
+  }
+  if (a.update)
+    a.dst[dst_off] -= a.lr * v;
+  else
+    a.dst[dst_off] = v;
+}
+
+int launch_permute(const PermArgs& a, int64_t total, cudaStream_t st) {
+  if (total <= 0) return 0;
+  ProfScope ps(K_STACK, st, 0.0, 8.0 * total);
+  const unsigned grid = static_cast<unsigned>((total + 255) / 256);
+  tensor_permute_kernel<<<grid, 256, 0, st>>>(a, total);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "tensor_permute_kernel");
+}
+
+struct Mode {
+  int n, npad;
+  int64_t K;
+  int Kpad;
+  int group, slot;   // root group and index in its stacks
+  size_t u_off;      // float offset of U_i in the unfolding area (per parameter)
+};
+
+struct Param {
+  int k;
+  int dims[kMaxOrder];
+  int64_t size;
+  std::vector<Mode> modes;
+  size_t u_floats;   // all modes' unfoldings
+};
+
+struct Group {
+  int npad, p, count;
+  size_t h_off, x_off, valid_off;  // state byte offsets
+  std::vector<int> valid;
+};
+
+struct Plan {
+  std::vector<Param> params;
+  std::vector<Group> groups;
+  size_t state_status, state_total;
+  size_t u_area, v_floats, root_bytes, scratch_u, scratch_v0, scratch_v1, scratch_root, scratch_total;
+};
+
+int validate_tensor_config(const shampoo_config* c) {
+  if (!c) return set_error(SHAMPOO_ERR_INVALID_ARG, "config is NULL");
+  if (!(c->beta >= 0.f) || !(c->beta <= 1.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "beta must be in [0, 1]");
+  if (!(c->eps >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "eps must be >= 0");
+  if (!(c->lr == c->lr)) return set_error(SHAMPOO_ERR_INVALID_ARG, "lr is NaN");
+  if (c->solver < 0 || c->solver > 3) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", c->solver);
+  if (c->solver != SHAMPOO_SOLVER_CHEBYSHEV && (c->iters < 1 || c->iters > 1000))
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "iters must be in [1, 1000]");
+  if (!(c->tol >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "tol must be >= 0");
+  if (c->refresh_every < 1) return set_error(SHAMPOO_ERR_INVALID_ARG, "refresh_every must be >= 1");
+  if (c->solver == SHAMPOO_SOLVER_CHEBYSHEV) {
+    if (c->cheb_degree < 2 || c->cheb_degree > kMaxChebDegree)
+      return set_error(SHAMPOO_ERR_INVALID_ARG, "cheb_degree must be in [2, %d]", kMaxChebDegree);
+    if (!(c->cheb_lo > 0.f) && !(c->eps > 0.f))
+      return set_error(SHAMPOO_ERR_INVALID_ARG, "Chebyshev needs cheb_lo > 0 or eps > 0");
+  }
+  if (c->grad_dtype != SHAMPOO_F32 && c->grad_dtype != SHAMPOO_BF16)
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "grad_dtype must be SHAMPOO_F32 or SHAMPOO_BF16");
+  if (c->momentum != 0.f) return set_error(SHAMPOO_ERR_UNSUPPORTED, "tensor Shampoo takes no momentum");
+  return SHAMPOO_OK;
+}
+
+int make_plan(const shampoo_config* cfg, int32_t nparams, const int32_t* orders, const int64_t* dims, Plan& P) {
+  if (nparams < 1 || nparams > kMaxTensorParams)
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "nparams %d: need 1..%d", nparams, kMaxTensorParams);
+  if (!orders || !dims) return set_error(SHAMPOO_ERR_INVALID_ARG, "orders/dims is NULL");
+  P = Plan();
+  std::map<std::pair<int, int>, int> gid;
+  size_t di = 0;
+  for (int j = 0; j < nparams; ++j) {
+    Param pr;
+    pr.k = orders[j];
+    if (pr.k < 2 || pr.k > kMaxOrder) return set_error(SHAMPOO_ERR_INVALID_ARG, "param %d has order %d (2..4)", j, pr.k);
+    if (cfg->solver == SHAMPOO_SOLVER_NEWTON_DB && pr.k != 2)
+      return set_error(SHAMPOO_ERR_INVALID_ARG, "Newton-DB computes the -1/4 power only (order 2)");
+    pr.size = 1;
+    for (int l = 0; l < pr.k; ++l) {
+      const int64_t d = dims[di + l];
+      if (d < 1) return set_error(SHAMPOO_ERR_INVALID_ARG, "param %d dimension %d is %lld", j, l, (long long)d);
+      if (d > 1024) return set_error(SHAMPOO_ERR_UNSUPPORTED, "param %d dimension %d is %lld > 1024", j, l, (long long)d);
+      pr.dims[l] = static_cast<int>(d);
+      pr.size *= d;
+    }
+    if (pr.size > (int64_t(1) << 31)) return set_error(SHAMPOO_ERR_UNSUPPORTED, "param %d is too large", j);
+    di += pr.k;
+    const int p = 2 * pr.k;
+    pr.u_floats = 0;
+    for (int i = 0; i < pr.k; ++i) {
+      Mode m;
+      m.n = pr.dims[i];
+      m.npad = up32(m.n);
+      m.K = pr.size / m.n;
+      m.Kpad = up32(m.K);
+      auto key = std::make_pair(m.npad, p);
+      auto it = gid.find(key);
+      if (it == gid.end()) {
+        Group g;
+        g.npad = m.npad;
+        g.p = p;
+        g.count = 0;
+        it = gid.emplace(key, static_cast<int>(P.groups.size())).first;
+        P.groups.push_back(g);
+      }
+      m.group = it->second;
+      m.slot = P.groups[m.group].count++;
+      P.groups[m.group].valid.push_back(m.n);
+      m.u_off = pr.u_floats;
+      pr.u_floats += alt(static_cast<size_t>(m.npad) * m.Kpad * 4) / 4;
+      pr.modes.push_back(m);
+    }
+    P.params.push_back(pr);
+  }
+  // state: status | per group: valid, H stack, X stack
+  size_t o = 0;
+  P.state_status = o, o += alt(4);
+  for (Group& g : P.groups) {
+    const size_t mat = static_cast<size_t>(g.npad) * g.npad * 4;
+    g.valid_off = o, o += alt(static_cast<size_t>(g.count) * 4);
+    g.h_off = o, o += alt(mat * g.count);
+    g.x_off = o, o += alt(mat * g.count);
+  }
+  P.state_total = o;
+  // scratch: all unfoldings of the largest parameter | two product buffers | root solver
+  P.u_area = 0;
+  P.v_floats = 0;
+  for (const Param& pr : P.params) {
+    P.u_area = std::max(P.u_area, pr.u_floats);
+    for (const Mode& m : pr.modes) P.v_floats = std::max(P.v_floats, static_cast<size_t>(m.npad) * m.Kpad);
+  }
+  P.root_bytes = 0;
+  for (const Group& g : P.groups) {
+    const size_t per = root_scratch_per_matrix(g.npad, cfg->solver, g.p);
+    const size_t want = root_scratch_header() + per * g.count;
+    P.root_bytes = std::max(P.root_bytes, std::min(want, std::max(kTensorRootBudget, root_scratch_header() + per)));
+  }
+  o = 0;
+  P.scratch_u = o, o += alt(P.u_area * 4);
+  P.scratch_v0 = o, o += alt(P.v_floats * 4);
+  P.scratch_v1 = o, o += alt(P.v_floats * 4);
+  P.scratch_root = o, o += alt(P.root_bytes);
+  P.scratch_total = o;
+  return SHAMPOO_OK;
+}
+
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+
+}  // namespace
+
+struct shampoo_tensor_ctx {
+  shampoo_config cfg;
+  Plan plan;
+  char* state = nullptr;
+  char* scratch = nullptr;
+  int* d_status = nullptr;
+  std::vector<StackMaps> mH, mX;  // per group
+  int64_t step = 0;
+  cudaStream_t last_stream = nullptr;
+};
+
+extern "C" {
+
+int shampoo_tensor_query_sizes(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
+                               const int64_t* dims, size_t* state_bytes, size_t* scratch_bytes) {
+  int rc = validate_tensor_config(cfg);
+  if (rc) return rc;
+  Plan P;
+  if ((rc = make_plan(cfg, nparams, orders, dims, P))) return rc;
+  if (!state_bytes || !scratch_bytes) return set_error(SHAMPOO_ERR_INVALID_ARG, "output pointer is NULL");
+  *state_bytes = P.state_total;
+  *scratch_bytes = P.scratch_total;
+  return SHAMPOO_OK;
+}
+
+int shampoo_tensor_init(const shampoo_config* cfg, int32_t nparams, const int32_t* orders, const int64_t* dims,
+                        void* d_state, size_t state_bytes, void* d_scratch, size_t scratch_bytes, void* stream,
+                        shampoo_tensor_handle* out) {
+  int rc = validate_tensor_config(cfg);
+  if (rc) return rc;
+  if (!out) return set_error(SHAMPOO_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  Plan P;
+  if ((rc = make_plan(cfg, nparams, orders, dims, P))) return rc;
+  if (!d_state || !d_scratch) return set_error(SHAMPOO_ERR_INVALID_ARG, "state/scratch is NULL");
+  if (!aligned256(d_state) || !aligned256(d_scratch))
+    return set_error(SHAMPOO_ERR_UNSUPPORTED, "state/scratch must be 256-byte aligned");
+  if (state_bytes < P.state_total)
+    return set_error(SHAMPOO_ERR_WORKSPACE, "state %zu < %zu bytes", state_bytes, P.state_total);
+  if (scratch_bytes < P.scratch_total)
+    return set_error(SHAMPOO_ERR_WORKSPACE, "scratch %zu < %zu bytes", scratch_bytes, P.scratch_total);
+  shampoo_tensor_ctx* h = new (std::nothrow) shampoo_tensor_ctx;
+  if (!h) return set_error(SHAMPOO_ERR_INVALID_ARG, "out of host memory");
+  h->cfg = *cfg;
+  h->plan = P;
+  h->state = static_cast<char*>(d_state);
+  h->scratch = static_cast<char*>(d_scratch);
+  h->d_status = reinterpret_cast<int*>(h->state + P.state_status);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  rc = check_cuda(cudaMemsetAsync(h->state, 0, P.state_total, st), "zero tensor state");
+  for (size_t g = 0; g < P.groups.size() && !rc; ++g) {
+    const Group& G = P.groups[g];
+    rc = check_cuda(cudaMemcpyAsync(h->state + G.valid_off, G.valid.data(), G.valid.size() * 4,
+                                    cudaMemcpyHostToDevice, st),
+                    "upload valid extents");
+  }
+  if (!rc) rc = check_cuda(cudaStreamSynchronize(st), "tensor init sync");
+  h->mH.resize(P.groups.size());
+  h->mX.resize(P.groups.size());
+  for (size_t g = 0; g < P.groups.size() && !rc; ++g) {
+    const Group& G = P.groups[g];
+    if ((rc = make_stack_maps(h->mH[g], reinterpret_cast<float*>(h->state + G.h_off), G.count, G.npad))) break;
+    rc = make_stack_maps(h->mX[g], reinterpret_cast<float*>(h->state + G.x_off), G.count, G.npad);
+  }
+  if (rc) {
+    delete h;
+    return rc;
+  }
+  *out = h;
+  return SHAMPOO_OK;
+}
+
+int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const void* const* d_grads, void* stream) {
+  if (!h) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle is NULL");
+  if (!d_weights || !d_grads) return set_error(SHAMPOO_ERR_INVALID_ARG, "weights/grads array is NULL");
+  const Plan& P = h->plan;
+  const shampoo_config& c = h->cfg;
+  for (size_t j = 0; j < P.params.size(); ++j)
+    if (!d_weights[j] || !d_grads[j]) return set_error(SHAMPOO_ERR_INVALID_ARG, "param %zu has a NULL pointer", j);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  float* U = reinterpret_cast<float*>(h->scratch + P.scratch_u);
+  float* V[2] = {reinterpret_cast<float*>(h->scratch + P.scratch_v0),
+                 reinterpret_cast<float*>(h->scratch + P.scratch_v1)};
+  const bool refresh = h->step % c.refresh_every == 0;
+  const int g_exact = c.grad_dtype == SHAMPOO_BF16 ? 1 : 0;
+  int rc;
+  auto hptr = [&](const Mode& m) {
+    const Group& G = P.groups[m.group];
+    return reinterpret_cast<float*>(h->state + G.h_off) + static_cast<size_t>(m.slot) * G.npad * G.npad;
+  };
+  // 1-2. unfold every mode of every parameter and accumulate its statistic
+  // (one GEMM launch per parameter, one group per mode).  With a refresh
+  // pending, all statistics must be complete before the roots, so the
+  // unfoldings of the last parameter are the ones left for the apply below.
+  for (size_t j = 0; j < P.params.size(); ++j) {
+    const Param& pr = P.params[j];
+    std::vector<StackMaps> um(pr.k);
+    for (int i = 0; i < pr.k; ++i) {
+      const Mode& m = pr.modes[i];
+      PermArgs a;
+      std::memset(&a, 0, sizeof(a));
+      a.k = pr.k;
+      for (int l = 0; l < pr.k; ++l) a.dims[l] = pr.dims[l];
+      a.src = d_grads[j];
+      a.src_bf16 = c.grad_dtype == SHAMPOO_BF16;
+      a.s = PermSide{-1, 0};
+      a.dst = U + m.u_off;
+      a.d = PermSide{i, m.Kpad};
+      a.rows = m.npad;
+      a.cols = m.Kpad;
+      if ((rc = launch_permute(a, static_cast<int64_t>(m.npad) * m.Kpad, st))) return rc;
+      if ((rc = make_rect_maps(um[i], U + m.u_off, 1, m.npad, m.Kpad))) return rc;
+    }
+    Builder b;
+    for (int i = 0; i < pr.k; ++i) {
+      const Mode& m = pr.modes[i];
+      Epilogue& e = b.add_rect(1, m.npad, m.npad, m.Kpad, um[i], 0, um[i], 0, 2.0 * m.n * double(m.n) * m.K,
+                               B_TRANSPOSED);
+      b.L.g[i].a_exact = b.L.g[i].b_exact = g_exact;
+      e.beta = c.beta;
+      e.C = hptr(m);
+      e.D = hptr(m);
+      e.flags = h->d_status;
+    }
+    if ((rc = b.launch(st))) return rc;
+  }
+  // 3. roots X = (H + eps I)^{-1/(2k)}, batched per (npad, k)
+  if (refresh) {
+    for (size_t g = 0; g < P.groups.size(); ++g) {
+      const Group& G = P.groups[g];
+      RootJob job;
+      job.batch = G.count;
+      job.n = G.npad;
+      job.p = G.p;
+      job.solver = c.solver;
+      job.iters = c.iters;
+      job.cheb_degree = c.cheb_degree;
+      job.eps = c.eps;
+      job.tol = c.tol;
+      job.cheb_lo = c.cheb_lo;
+      job.A = reinterpret_cast<float*>(h->state + G.h_off);
+      job.valid = reinterpret_cast<int*>(h->state + G.valid_off);
+      job.X = reinterpret_cast<float*>(h->state + G.x_off);
+      job.iters_used = nullptr;
+      job.flags = h->d_status;
+      if ((rc = run_inverse_roots(job, h->scratch + P.scratch_root, P.root_bytes, st))) return rc;
+    }
+  }
+  // 4. apply: V = X_0 unfold_0(G), then mode by mode; the last fold updates W.
+  for (size_t j = 0; j < P.params.size(); ++j) {
+    const Param& pr = P.params[j];
+    const Mode& m0 = pr.modes[0];
+    {  // mode-0 unfolding of G (U holds the last parameter's unfoldings only)
+      PermArgs a;
+      std::memset(&a, 0, sizeof(a));
+      a.k = pr.k;
+      for (int l = 0; l < pr.k; ++l) a.dims[l] = pr.dims[l];
+      a.src = d_grads[j];
+      a.src_bf16 = c.grad_dtype == SHAMPOO_BF16;
+      a.s = PermSide{-1, 0};
+      a.dst = V[1];
+      a.d = PermSide{0, m0.Kpad};
+      a.rows = m0.npad;
+      a.cols = m0.Kpad;
+      if ((rc = launch_permute(a, static_cast<int64_t>(m0.npad) * m0.Kpad, st))) return rc;
+    }
+    // cur: mode-i unfolding of the partial product; out: X_i cur.  The next
+    // mode's permutation reads `out` into `cur`, so the two never trade roles.
+    float* cur = V[1];
+    float* out = V[0];
+    for (int i = 0; i < pr.k; ++i) {
+      const Mode& m = pr.modes[i];
+      if (i > 0) {  // cur <- mode-i unfolding of the previous product (held in `out` as mode i-1)
+        const Mode& mp = pr.modes[i - 1];
+        PermArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.k = pr.k;
+        for (int l = 0; l < pr.k; ++l) a.dims[l] = pr.dims[l];
+        a.src = out;
+        a.s = PermSide{i - 1, mp.Kpad};
+        a.dst = cur;
+        a.d = PermSide{i, m.Kpad};
+        a.rows = m.npad;
+        a.cols = m.Kpad;
+        if ((rc = launch_permute(a, static_cast<int64_t>(m.npad) * m.Kpad, st))) return rc;
+      }
+      StackMaps cm;
+      if ((rc = make_rect_maps(cm, cur, 1, m.npad, m.Kpad))) return rc;
+      Builder b;
+      Epilogue& e = b.add_rect(1, m.npad, m.Kpad, m.npad, h->mX[m.group], m.slot, cm, 0,
+                               2.0 * m.n * double(m.n) * m.K, B_MN_MAJOR);
+      if (i == 0) b.L.g[0].b_exact = g_exact;
+      e.D = out;
+      e.flags = h->d_status;
+      if ((rc = b.launch(st))) return rc;
+    }
+    {  // fold the last product (mode k-1 unfolding) into the weight: W -= lr P
+      const Mode& ml = pr.modes[pr.k - 1];
+      PermArgs a;
+      std::memset(&a, 0, sizeof(a));
+      a.k = pr.k;
+      for (int l = 0; l < pr.k; ++l) a.dims[l] = pr.dims[l];
+      a.src = out;
+      a.s = PermSide{pr.k - 1, ml.Kpad};
+      a.dst = d_weights[j];
+      a.d = PermSide{-1, 0};
+      a.update = 1;
+      a.lr = c.lr;
+      if ((rc = launch_permute(a, pr.size, st))) return rc;
+    }
+  }
+  h->step += 1;
+  return SHAMPOO_OK;
+}
+
+int shampoo_tensor_views(shampoo_tensor_handle h, int32_t param, int32_t mode, float** H, float** X, int32_t* npad,
+                         int64_t* step) {
+  if (!h) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle is NULL");
+  const Plan& P = h->plan;
+  if (param < 0 || param >= static_cast<int>(P.params.size()) || mode < 0 || mode >= P.params[param].k)
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "no mode %d of param %d", mode, param);
+  const Mode& m = P.params[param].modes[mode];
+  const Group& G = P.groups[m.group];
+  const size_t off = static_cast<size_t>(m.slot) * G.npad * G.npad;
+  if (H) *H = reinterpret_cast<float*>(h->state + G.h_off) + off;
+  if (X) *X = reinterpret_cast<float*>(h->state + G.x_off) + off;
+  if (npad) *npad = G.npad;
+  if (step) *step = h->step;
+  return SHAMPOO_OK;
+}
+
+int shampoo_tensor_get_status(shampoo_tensor_handle h, int32_t* status, int32_t reset) {
+  if (!h || !status) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle/status is NULL");
+  int rc = check_cuda(cudaStreamSynchronize(h->last_stream), "status sync");
+  if (rc) return rc;
+  int v = 0;
+  if ((rc = check_cuda(cudaMemcpy(&v, h->d_status, 4, cudaMemcpyDeviceToHost), "read status"))) return rc;
+  *status = v;
+  if (reset && (rc = check_cuda(cudaMemset(h->d_status, 0, 4), "reset status"))) return rc;
+  return SHAMPOO_OK;
+}
+
+void shampoo_tensor_destroy(shampoo_tensor_handle h) { delete h; }
+
+}  // extern "C"

@@ -19,6 +19,15 @@ relative error, against the float64 oracle, of an fp32 reference pipeline
 (float32 statistics and products, single-precision LAPACK roots) run on the
 same gradients; the gate is max(2e-3, 2 F_update).
 
+Apply gate (stage parity of the update).  The GPU's update of a block,
+Delta W / lr, is compared with the float64 product XL_gpu G XR_gpu of the
+GPU's own fp32 roots and the same gradient, which isolates the two apply
+products and the masked scatter into W from the roots' own error.  Each
+fp32-accurate product (3xTF32 with round-to-nearest segment sums) carries an
+elementwise error of order 2^-22 sum_k |a_ik| |b_kj|, so the gate is
+TOL_APPLY = 2e-5 times the cancellation factor
+|| |XL| |G| |XR| ||_F / ||XL G XR||_F (at least 1).
+
 Both fp32 references damp with eps_eff = max(eps, u ||A + eps I||_F), the
 damping the GPU solvers apply: statistics accumulated in fp32 can be
 indefinite at the level u ||A||, and a smaller eps is below fp32 resolution.
@@ -85,13 +94,15 @@ class Fp32ReferenceShampoo:
     """The blocked step in float32 with LAPACK roots: the update floor's
     reference (statistics, roots and products all in single precision)."""
 
-    def __init__(self, shapes, block, beta, eps, root_p, refresh_every, blocks):
+    def __init__(self, shapes, block, beta, eps, root_p, refresh_every, blocks, momentum=0.0):
         from oracle import block_table
         self.table = block_table(shapes, block)
         self.blocks = list(blocks)
         self.beta, self.eps, self.p, self.k = np.float32(beta), eps, root_p, refresh_every
         self.L = {b: np.zeros((self.table[b].r,) * 2, np.float32) for b in self.blocks}
         self.R = {b: np.zeros((self.table[b].c,) * 2, np.float32) for b in self.blocks}
+        self.alpha = np.float32(momentum)
+        self.M = {b: np.zeros((self.table[b].r, self.table[b].c), np.float32) for b in self.blocks}
         self.XL, self.XR = {}, {}
         self.t = 0
 
@@ -106,13 +117,32 @@ class Fp32ReferenceShampoo:
             if refresh:
                 self.XL[b] = lapack_fp32_root(self.L[b], self.p, self.eps).astype(np.float32)
                 self.XR[b] = lapack_fp32_root(self.R[b], self.p, self.eps).astype(np.float32)
-            P[b] = (self.XL[b] @ G @ self.XR[b]).astype(np.float64)
+            if self.alpha > 0:
+                self.M[b] = self.alpha * self.M[b] + G
+                P[b] = (self.XL[b] @ self.M[b] @ self.XR[b]).astype(np.float64)
+            else:
+                P[b] = (self.XL[b] @ G @ self.XR[b]).astype(np.float64)
         self.t += 1
         return P
 
 
 def update_gate(P_fp32, P_oracle):
     return max(BASE_TOL, 2.0 * rel_fro(P_fp32, P_oracle))
+
+
+TOL_APPLY = 2e-5
+
+
+def apply_check(P_gpu, XL, G, XR):
+    """(error, gate) of the GPU's update direction against the float64
+    product of the GPU's own roots and the gradient (the apply stage alone)."""
+    XL = np.asarray(XL, dtype=np.float64)
+    G = np.asarray(G, dtype=np.float64)
+    XR = np.asarray(XR, dtype=np.float64)
+    P64 = XL @ G @ XR
+    den = np.linalg.norm(P64)
+    cancel = np.linalg.norm(np.abs(XL) @ np.abs(G) @ np.abs(XR)) / den if den > 0 else 1.0
+    return rel_fro(P_gpu, P64), TOL_APPLY * max(1.0, cancel)
 
 
 def split_range_null(S, eps):
@@ -154,3 +184,39 @@ def root_checks(X, S, p, eps):
     above = np.maximum(0.0, mu - hi) / hi
     spread = float(max(below.max(), above.max()))
     return err, gate, spread
+
+
+class Fp32ReferenceTensorShampoo:
+    """Order-k tensor Shampoo in float32 with LAPACK roots (the update floor's
+    reference for the tensor path): fp32 statistics, single-precision
+    eigendecomposition roots with the power -1/(2k), fp32 mode products."""
+
+    def __init__(self, shape, beta, eps, refresh_every):
+        self.shape = tuple(shape)
+        self.k = len(self.shape)
+        self.beta, self.eps, self.every = np.float32(beta), eps, refresh_every
+        self.H = [np.zeros((n, n), np.float32) for n in self.shape]
+        self.X = [None] * self.k
+        self.t = 0
+
+    def step(self, G):
+        from oracle.tensor import mode_statistic, precondition_tensor
+        G = np.asarray(G, np.float32)
+        for i in range(self.k):
+            self.H[i] = (self.beta * self.H[i] + mode_statistic(G, i)).astype(np.float32)
+        if self.t % self.every == 0:
+            self.X = [lapack_fp32_root(H, 2 * self.k, self.eps).astype(np.float32) for H in self.H]
+        self.t += 1
+        return precondition_tensor(G, self.X).astype(np.float64)
+
+
+def tensor_apply_check(P_gpu, G, roots):
+    """(error, gate) of the tensor path's update direction against the float64
+    mode products of the GPU's own roots and the gradient (apply stage)."""
+    from oracle.tensor import precondition_tensor
+    G = np.asarray(G, dtype=np.float64)
+    roots = [np.asarray(X, dtype=np.float64) for X in roots]
+    P64 = precondition_tensor(G, roots)
+    den = np.linalg.norm(P64)
+    cancel = np.linalg.norm(precondition_tensor(np.abs(G), [np.abs(X) for X in roots])) / den if den > 0 else 1.0
+    return rel_fro(P_gpu, P64), TOL_APPLY * max(1.0, cancel)

@@ -143,3 +143,40 @@ def test_strided_step_refuses_a_null_handle():
     w = (ctypes.c_void_p * 1)(None)
     assert sb.lib.shampoo_step_strided(None, w, w, ld, None) == sb.ERR_INVALID_ARG
     assert "handle" in sb.last_error()
+
+
+def test_momentum_state_is_one_more_block_stack(sb):
+    """Momentum adds one (nb, B, B) fp32 stack to the state and nothing to the
+    scratch; alpha must lie in [0, 1)."""
+    shapes = [(1024, 768), (300, 512)]
+    off = sb.make_config(256, 0.95, 1e-8, 1e-3)
+    on = sb.make_config(256, 0.95, 1e-8, 1e-3, momentum=0.9)
+    s0, x0 = sb.query_sizes(off, shapes)
+    s1, x1 = sb.query_sizes(on, shapes)
+    nb = len(oracle.block_table(shapes, 256))
+    assert x1 == x0
+    assert s1 - s0 == nb * 256 * 256 * 4
+    for bad in (1.0, -0.1, float("nan")):
+        with pytest.raises(sb.ShampooError):
+            sb.query_sizes(sb.make_config(256, 0.95, 1e-8, 1e-3, momentum=bad), shapes)
+
+
+def test_tensor_sizes_and_validation(sb):
+    """Tensor Shampoo: orders 2..4, dimensions up to 1024; state holds one
+    statistic and one root per mode (padded to multiples of 32)."""
+    cfg = sb.make_config(32, 0.9, 1e-4, 1e-3, solver=3)
+    state, scratch = sb.tensor_query_sizes(cfg, [(3, 3, 64, 128)])
+    per_mode = [32, 32, 64, 128]
+    assert state >= sum(2 * n * n * 4 for n in per_mode)
+    assert scratch > 0
+    for bad in ([(5,)], [(2, 2, 2, 2, 2)], [(0, 4)]):
+        with pytest.raises(sb.ShampooError) as e:
+            sb.tensor_query_sizes(cfg, bad)
+        assert e.value.code == sb.ERR_INVALID_ARG
+    with pytest.raises(sb.ShampooError) as e:
+        sb.tensor_query_sizes(cfg, [(2048, 8)])
+    assert e.value.code == sb.ERR_UNSUPPORTED
+    db = sb.make_config(32, 0.9, 1e-4, 1e-3, solver=1)
+    sb.tensor_query_sizes(db, [(40, 50)])
+    with pytest.raises(sb.ShampooError):
+        sb.tensor_query_sizes(db, [(4, 5, 6)])

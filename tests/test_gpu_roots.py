@@ -217,3 +217,36 @@ def test_newton_uses_the_spectral_scale(sb):
         assert it[b] < k_frob, (it[b], k_frob)
         ref = oracle.inverse_root(A, 4, 1e-3)
         assert oracle.rel_fro(X[b], ref) < root_gate(A, 4, 1e-3)
+
+
+@pytest.mark.parametrize("p", [6, 8])
+@pytest.mark.parametrize("solver,tol", [(0, 0.0), (0, 1e-5), (3, 1e-5)])
+def test_newton_higher_orders(sb, p, solver, tol):
+    """Coupled Newton for the -1/6 and -1/8 powers of order-3 and order-4
+    tensor Shampoo (T^6 = T^4 T^2, T^8 = T^4 T^4 in one more stack): the exact
+    root within 2e-3 at kappa 1e3, residual-checked runs well below the cap."""
+    A32 = workloads.spd_batch(4, 192, 1e3, seed=60 + p).astype(np.float32)
+    X, it, st = run(sb, A32, p=p, eps=0.0, solver=solver, iters=40, tol=tol)
+    assert st == 0
+    if tol > 0:
+        assert np.all(it > 0) and np.all(it < 30), it
+    for b in range(4):
+        ref = oracle.inverse_root(A32[b].astype(np.float64), p, 0.0)
+        assert oracle.rel_fro(X[b], ref) < TOL, (b, oracle.rel_fro(X[b], ref))
+
+
+@pytest.mark.parametrize("p", [6, 8])
+def test_chebyshev_higher_orders(sb, p):
+    A32 = workloads.spd_batch(3, 128, 1e2, seed=61).astype(np.float32)
+    lo = 0.999e-2
+    X, it, st = run(sb, A32, p=p, eps=0.0, solver=sb.SOLVER_CHEBYSHEV, cheb_degree=24, cheb_lo=lo)
+    assert st == 0
+    for b in range(3):
+        ref = och.chebyshev_inverse_root(A32[b].astype(np.float64), p, 0.0, 24, lo=lo)
+        assert oracle.rel_fro(X[b], ref) < TOL
+
+
+def test_newton_db_refuses_higher_orders(sb):
+    A = torch.zeros((1, 64, 64), device="cuda")
+    with pytest.raises(sb.ShampooError):
+        sb.inv_root_batched(A, p=6, solver=sb.SOLVER_NEWTON_DB)

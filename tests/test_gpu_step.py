@@ -3,8 +3,11 @@
 Per step and per block: statistics (GPU fp32 L, R vs the float64 oracle's,
 1e-5 relative Frobenius), roots (the GPU roots vs the oracle's exact root of
 the GPU's own fp32 statistics: isolates the solver from fp32 statistics
-rounding), and the update P_b = -(W_t - W_{t-1}) / lr against the fully
-float64 pipeline, <= max(2e-3, 2 F_update) relative Frobenius per block.
+rounding), the update P_b = -(W_t - W_{t-1}) / lr against the float64
+product of the GPU's own roots and the gradient (the apply stage alone:
+2e-5 times the cancellation factor, parity.apply_check), and the same update
+against the fully float64 pipeline, <= max(2e-3, 2 F_update) relative
+Frobenius per block.
 
 Small ragged blocks have rank-deficient statistics (a 32 x 15 gradient
 block gives a 32 x 32 L of rank 15).  On the null space the root is set by
@@ -25,7 +28,7 @@ pytestmark = pytest.mark.gpu
 
 import oracle
 import workloads
-from parity import Fp32ReferenceShampoo, root_checks, root_gate, update_gate
+from parity import Fp32ReferenceShampoo, apply_check, root_checks, root_gate, update_gate
 
 TOL_UPDATE = 2e-3
 TOL_ROOT = 2e-3
@@ -53,7 +56,7 @@ def run_parity(sb, wl, steps, check_roots=True, blocks=None):
     assert [tuple(t) for t in table] == [(b.param, b.row0, b.col0, b.r, b.c) for b in ref.table]
     ref32 = Fp32ReferenceShampoo(wl.shapes, wl.block, wl.beta, wl.eps, wl.root_p, wl.refresh_every, ref.active)
     stream = workloads.GradientStream(wl)
-    worst = {"update": 0.0, "root": 0.0, "stats": 0.0}
+    worst = {"update": 0.0, "root": 0.0, "stats": 0.0, "apply": 0.0}
     for t in range(steps):
         grads = stream.next()
         if wl.grad_dtype == workloads.DTYPE_BF16:
@@ -65,15 +68,17 @@ def run_parity(sb, wl, steps, check_roots=True, blocks=None):
         P_ref = ref.step(grads)
         P_32 = ref32.step(grads)
         torch.cuda.synchronize()
-        dW = [((b - a) / wl.lr).cpu().numpy().astype(np.float64) for a, b in zip(W, before)]
+        dW = [((b.double() - a.double()) / wl.lr).cpu().numpy() for a, b in zip(W, before)]
         L, R = opt.statistics()
         L, R = L.cpu().numpy().astype(np.float64), R.cpu().numpy().astype(np.float64)
-        if check_roots and t % wl.refresh_every == 0:
-            XL, XR = opt.roots()
-            XL, XR = XL.cpu().numpy().astype(np.float64), XR.cpu().numpy().astype(np.float64)
+        XL, XR = opt.roots()
+        XL, XR = XL.cpu().numpy().astype(np.float64), XR.cpu().numpy().astype(np.float64)
         for b in ref.active:
             blk = ref.table[b]
             Pg = dW[blk.param][blk.row0:blk.row0 + blk.r, blk.col0:blk.col0 + blk.c]
+            ea, ga = apply_check(Pg, XL[b, :blk.r, :blk.r], ref.block_of(grads, b), XR[b, :blk.c, :blk.c])
+            worst["apply"] = max(worst["apply"], ea)
+            assert ea < ga, (t, b, "apply", ea, ga)
             e = oracle.rel_fro(Pg, P_ref[b])
             worst["update"] = max(worst["update"], e)
             assert e < update_gate(P_32[b], P_ref[b]), (t, b, "update", e)
@@ -89,7 +94,7 @@ def run_parity(sb, wl, steps, check_roots=True, blocks=None):
                         assert spread < NULL_SPREAD, (t, b, "null-space root", spread)
     assert opt.status() == 0
     print(f"\n{wl.name} {wl.shapes}: worst update {worst['update']:.2e}, root {worst['root']:.2e}, "
-          f"statistics {worst['stats']:.2e}")
+          f"apply {worst['apply']:.2e}, statistics {worst['stats']:.2e}")
     return worst
 
 
@@ -201,29 +206,41 @@ def test_launch_count_increases(sb):
 @pytest.mark.parametrize("block,shape", [(512, (700, 1024)), (1024, (1024, 2048))])
 def test_large_blocks_parity(sb, block, shape):
     """Blocks of 512 (with a ragged block row of 188) and 1024 with the
-    workloads' solver: every statistic matches the float64 oracle and every
-    root passes its gate, over two steps with beta 0.9."""
+    workloads' solver, over two steps with beta 0.9: every statistic matches
+    the float64 oracle, every root passes its gate, every block's update
+    matches the float64 product of the GPU's own roots and gradient (the
+    apply stage) and the fully float64 pipeline (end to end)."""
     wl = workloads.workload("tiny", shapes=(shape,), block=block, steps=2, iters=30, tol=1e-5, beta=0.9, eps=1e-4,
                             solver=workloads.SOLVER_NEWTON_CUBIC)
     opt = sb.Shampoo(wl.shapes, sb.config_from_workload(wl))
     W = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
     ref = oracle.ShampooOracle(wl.shapes, wl.block, wl.beta, wl.eps, wl.lr, wl.root_p, wl.refresh_every)
+    ref32 = Fp32ReferenceShampoo(wl.shapes, wl.block, wl.beta, wl.eps, wl.root_p, wl.refresh_every, ref.active)
     stream = workloads.GradientStream(wl)
     for t in range(wl.steps):
         G = stream.next()
+        before = [w.double() for w in W]
         opt.step(W, [torch.from_numpy(g).cuda() for g in G])
-        ref.step(G)
-    torch.cuda.synchronize()
+        P_ref = ref.step(G)
+        P_32 = ref32.step(G)
+        torch.cuda.synchronize()
+        dW = [((a - w.double()) / wl.lr).cpu().numpy() for a, w in zip(before, W)]
+        XL, XR = opt.roots()
+        XL, XR = XL.cpu().numpy().astype(np.float64), XR.cpu().numpy().astype(np.float64)
+        for b, blk in enumerate(ref.table):
+            Pg = dW[blk.param][blk.row0:blk.row0 + blk.r, blk.col0:blk.col0 + blk.c]
+            ea, ga = apply_check(Pg, XL[b, :blk.r, :blk.r], ref.block_of(G, b), XR[b, :blk.c, :blk.c])
+            assert ea < ga, (t, b, "apply", ea, ga)
+            e = oracle.rel_fro(Pg, P_ref[b])
+            assert e < update_gate(P_32[b], P_ref[b]), (t, b, "update", e)
     L, R = opt.statistics()
     L, R = L.cpu().numpy(), R.cpu().numpy()
     for b, blk in enumerate(ref.table):
         assert oracle.rel_fro(L[b, :blk.r, :blk.r].astype(np.float64), ref.L[b]) < TOL_STATS
         assert oracle.rel_fro(R[b, :blk.c, :blk.c].astype(np.float64), ref.R[b]) < TOL_STATS
-    XL, XR = opt.roots()
-    XL, XR = XL.cpu().numpy().astype(np.float64), XR.cpu().numpy().astype(np.float64)
     for b, blk in enumerate(ref.table):
-        for X, S, v in ((XL, ref.L[b], blk.r), (XR, ref.R[b], blk.c)):
-            er, gate, _ = root_checks(X[b, :v, :v], S, wl.root_p, wl.eps)
+        for X, S, v in ((XL, L, blk.r), (XR, R, blk.c)):
+            er, gate, _ = root_checks(X[b, :v, :v], S[b, :v, :v].astype(np.float64), wl.root_p, wl.eps)
             assert er < gate, (b, er, gate)
     assert opt.status() & ~sb.DEVFLAG_STAGNATED == 0
 

@@ -1,0 +1,95 @@
+"""The inverse-root solver sweep at its own batch shapes, gated.
+
+Inputs: the sweep's stacks 512 x 256^2, 128 x 512^2 and 64 x 1024^2 of SPD
+matrices Q diag(lam) Q^T (Haar Q, lam log-uniform with condition number kappa
+forced exactly), kappa in {1e2, 1e4, 1e6, 1e8}, cast to fp32; eps = 0.  Every
+case runs the whole stack on the GPU through the C ABI; the oracle checks two
+matrices of each (the first and the last), one by one.
+
+Solvers and gates (DASH abstract: Newton-DB and Chebyshev solvers; the
+coupled-Newton family is the reading of the Newton iterations):
+
+* coupled Newton (both correction degrees) and Newton-DB, residual-checked
+  (tol 1e-5, cap 40): against the exact root of the same fp32 matrix,
+  2e-3 relative Frobenius at kappa <= 1e4, and at kappa >= 1e6 the
+  conditioning floor max(2e-3, 2 F) (tests/parity.py: no fp32-input method can
+  do better than the root's own sensitivity to rounding its input, or than
+  single-precision LAPACK with the same damping);
+* Chebyshev, degree 16 and 32, interval [0.999/kappa, 1] in A's units:
+  polynomial parity, against the float64 Clenshaw evaluation of the same
+  interpolant on the same damped matrix (the GPU damps with
+  eps_eff = max(eps, 2^-24 ||A + eps I||_F)), 2e-3; its distance to the exact
+  root is a property of the degree.
+
+p in {2, 4} throughout.  The device status may only carry STAGNATED (a
+residual held up by fp32 rounding above tol), never NOT_CONVERGED.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle
+from oracle import chebyshev as och
+import workloads
+from parity import BASE_TOL, effective_eps, root_gate
+
+SOLVERS = (("newton", 0, 0), ("newton_cubic", 3, 0), ("newton_db", 1, 0), ("chebyshev16", 2, 16),
+           ("chebyshev32", 2, 32))
+CAP, TOL_RES = 40, 1e-5
+
+
+@pytest.fixture(scope="module")
+def sb():
+    import shampoo_family_second_b200 as sb
+    return sb
+
+
+CASES = [(batch, n, kappa) for batch, n in workloads.SWEEP_SHAPES for kappa in workloads.SWEEP_KAPPAS]
+
+
+@pytest.mark.parametrize("batch,n,kappa", CASES, ids=[f"{b}x{n}sq-kappa{k:.0e}" for b, n, k in CASES])
+def test_sweep_case(sb, batch, n, kappa):
+    A32 = workloads.spd_batch(batch, n, kappa, seed=4321 + n).astype(np.float32)
+    A = torch.from_numpy(A32).cuda()
+    samples = (0, batch - 1)
+    exact, gates = {}, {}
+    report = []
+    for p in (2, 4):
+        for s in samples:
+            A64 = A32[s].astype(np.float64)
+            exact[p, s] = oracle.inverse_root(A64, p, 0.0)
+            gates[p, s] = BASE_TOL if kappa <= 1e4 else root_gate(A64, p, 0.0)
+        for name, solver, degree in SOLVERS:
+            if solver == 2:
+                lo = 0.999 / kappa
+                X, it, st = sb.inv_root_batched(A, p=p, eps=0.0, solver=2, cheb_degree=degree, cheb_lo=lo)
+            else:
+                X, it, st = sb.inv_root_batched(A, p=p, eps=0.0, solver=solver, iters=CAP, tol=TOL_RES)
+            torch.cuda.synchronize()
+            st = int(st.item())
+            it = it.cpu().numpy()
+            assert st & ~sb.DEVFLAG_STAGNATED == 0, (name, p, st)
+            if solver == 2:
+                assert np.all(it == degree)
+            else:
+                stages = 2 if (solver == 1 and p == 4) else 1
+                assert np.all(np.abs(it) >= 1) and np.all(np.abs(it) <= stages * CAP), (name, p, it.min(), it.max())
+            for s in samples:
+                Xs = X[s].cpu().numpy().astype(np.float64)
+                assert np.all(np.isfinite(Xs))
+                A64 = A32[s].astype(np.float64)
+                if solver == 2:
+                    ref = och.chebyshev_inverse_root(A64, p, effective_eps(A64, 0.0), degree, lo=lo)
+                    e, gate = oracle.rel_fro(Xs, ref), BASE_TOL
+                    e_exact = oracle.rel_fro(Xs, exact[p, s])
+                else:
+                    e, gate = oracle.rel_fro(Xs, exact[p, s]), gates[p, s]
+                    e_exact = e
+                report.append((name, p, s, e, gate, e_exact, int(np.abs(it).max())))
+                assert e < gate, (name, p, s, e, gate)
+        del X
+    print(f"\nsweep {batch}x{n}^2 kappa {kappa:.0e}: " + "; ".join(
+        f"{nm} p{p} #{s}: {e:.1e}/{g:.1e}" + (f" (exact-root {ex:.1e})" if nm.startswith("cheb") else f" it {k}")
+        for nm, p, s, e, g, ex, k in report))

@@ -206,3 +206,90 @@ def test_partition_properties_on_random_shapes():
         assert max(load) <= sum(load) / world + max(cost)
 
     check()
+
+
+class FakeComm:
+    """In-process collectives for ranks run as threads: the reduce-scatter and
+    all-gather semantics of NCCL's reduce_scatter_tensor /
+    all_gather_into_tensor on flat tensors."""
+
+    def __init__(self, world):
+        import threading
+        self.world = world
+        self.bar = threading.Barrier(world)
+        self.slots = [None] * world
+
+    def reduce_scatter(self, rank):
+        def rs(out, inp):
+            self.slots[rank] = inp.clone()
+            self.bar.wait()
+            n = out.numel()
+            out.copy_(sum(s[rank * n:(rank + 1) * n] for s in self.slots))
+            self.bar.wait()
+        return rs
+
+    def all_gather(self, rank):
+        def ag(out, inp):
+            self.slots[rank] = inp.clone()
+            self.bar.wait()
+            out.copy_(torch.cat(self.slots))
+            self.bar.wait()
+        return ag
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("grads_reduced", [True, False])
+def test_injected_collectives_match_one_process(grads_reduced, world):
+    """The reduce-scatter / all-gather branch (the one NCCL takes) with its
+    packing and segment offsets, run with in-process collectives: every rank
+    (a thread) ends with the single-process weights."""
+    import threading
+    comm = FakeComm(world)
+    blocks = sharded.block_list(SHAPES, B)
+    owner = sharded.partition_blocks(blocks, world)
+    results = [None] * world
+    errors = []
+
+    def rank_main(rank):
+        try:
+            mine = [blocks[i] for i, k in enumerate(owner) if k == rank]
+            opt = sharded.ShardedShampoo(SHAPES, Cfg, grads_reduced=grads_reduced,
+                                         local_step=oracle_local_step(mine), world=world, rank=rank,
+                                         reduce_scatter=comm.reduce_scatter(rank), all_gather=comm.all_gather(rank))
+            W = [torch.zeros(s) for s in SHAPES]
+            for t in range(STEPS):
+                opt.step(W, gradients(t, shapes=SHAPES) if grads_reduced else gradients(t, rank, world))
+            results[rank] = [w.numpy().copy() for w in W]
+        except Exception as e:   # surfaced below
+            errors.append(e)
+            comm.bar.abort()
+
+    threads = [threading.Thread(target=rank_main, args=(r,)) for r in range(world)]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join(timeout=120)
+    assert not errors, errors
+    single = run_single(grads_reduced, world)
+    tol = 1e-7 if (grads_reduced or world == 2) else 1e-6
+    for W in results[1:]:
+        for a, b in zip(results[0], W):
+            assert np.array_equal(a, b)
+    for a, s in zip(results[0], single):
+        assert np.allclose(a, s, rtol=0, atol=tol), float(np.abs(a - s).max())
+
+
+def test_packed_offsets_tile_each_segment():
+    """Every block's packed range lies inside its owner's segment and the
+    ranges of one segment do not overlap."""
+    blocks = sharded.block_list(SHAPES, B)
+    for world in (1, 2, 3, 5):
+        owner = sharded.partition_blocks(blocks, world)
+        segments, offsets, seg = sharded.packed_offsets(blocks, owner, world)
+        for rank, sg in enumerate(segments):
+            used = np.zeros(seg, dtype=int)
+            for i in sg:
+                n = blocks[i][3] * blocks[i][4]
+                assert 0 <= offsets[i] and offsets[i] + n <= seg
+                used[offsets[i]:offsets[i] + n] += 1
+            assert used.max(initial=0) <= 1

@@ -67,3 +67,23 @@ def test_noalloc_largest_block_in_chunks(sb):
     Xr, Xn = X_ref.cpu().numpy().astype(np.float64), X.cpu().numpy().astype(np.float64)
     for b in range(2):
         assert oracle.rel_fro(Xn[b], Xr[b]) <= TOL
+
+
+def test_noalloc_residual_checked_chunks(sb):
+    """n = 1024, second-degree coupled Newton, tol 1e-5, batch 3: one matrix
+    per chunk of the fixed array, so the residual accumulators and the
+    iteration counter are reset for each chunk, and the iterations run as
+    plain launches.  Roots and iteration counts equal inv_root_batched's
+    (caller-owned scratch, one chunk, graph loop) on two calls in a row."""
+    for call in range(2):
+        A64 = workloads.spd_batch(3, 1024, 1e3, seed=70 + call)
+        A = torch.from_numpy(A64.astype(np.float32)).cuda()
+        X_ref, it_ref, st_ref = sb.inv_root_batched(A, p=4, eps=1e-6, solver=3, iters=40, tol=1e-5)
+        X, it, st = call_noalloc(sb, A, 4, 1e-6, 3, 40, 1e-5)
+        torch.cuda.synchronize()
+        assert int(st.item()) == int(st_ref.item()) == 0
+        assert torch.equal(it, it_ref)
+        assert int(it.min().item()) > 0
+        Xr, Xn = X_ref.cpu().numpy().astype(np.float64), X.cpu().numpy().astype(np.float64)
+        for b in range(3):
+            assert oracle.rel_fro(Xn[b], Xr[b]) <= TOL
