@@ -294,6 +294,47 @@ SHAMPOO_API int shampoo_tensor_views(shampoo_tensor_handle h, int32_t param, int
 SHAMPOO_API int shampoo_tensor_get_status(shampoo_tensor_handle h, int32_t* status, int32_t reset);
 SHAMPOO_API void shampoo_tensor_destroy(shampoo_tensor_handle h);
 
+/* SOAP: Adam run in the eigenbasis of Shampoo's preconditioner (pith.science
+ * record of "SOAP: Improving and Stabilizing Shampoo using Adam": abstract
+ * and claims; the basis is recomputed every refresh_every steps and kept in
+ * between), on the blocks and statistics of the blocked step.  Per block,
+ * step t (from 0):
+ *     G' = QL^T G QR,  m <- beta1 m + (1 - beta1) G,  v <- beta2 v + (1 - beta2) G'^2,
+ *     W <- W - lr QL [ (QL^T m QR / (1 - beta1^{t+1})) / (sqrt(v / (1 - beta2^{t+1})) + eps) ] QR^T,
+ *     L <- beta L + G G^T,  R <- beta R + G^T G,
+ *     if t % refresh_every == 0: QL, QR <- eigenbases of L, R (the identity before the
+ *     first refresh), v carried over as (PL o PL) v (PR o PR)^T, P = Q_new^T Q_old.
+ * The current gradient never enters its own projection (its rotation would have
+ * exact zeros that fp32 turns into rounding noise, which Adam's normalisation
+ * amplifies).  The bases come from eigh's method (cyclic Jacobi warm-started from
+ * the previous basis, then refine_iters refinement iterations).
+ * shampoo_config fields used: block, beta, lr, refresh_every, grad_dtype. */
+typedef struct {
+  float beta1;            /* Adam first-moment decay, [0, 1) */
+  float beta2;            /* Adam second-moment decay, [0, 1) */
+  float eps;              /* Adam epsilon, > 0 */
+  int32_t jacobi_sweeps;  /* eigensolver: Jacobi sweep cap per refresh, [1, 100] */
+  int32_t refine_iters;   /* eigensolver: refinement iterations per refresh, [0, 100] */
+} shampoo_soap_config;
+typedef struct shampoo_soap_ctx* shampoo_soap_handle;
+SHAMPOO_API int shampoo_soap_query_sizes(const shampoo_config* cfg, const shampoo_soap_config* sc, int32_t nparams,
+                                         const int64_t* rows, const int64_t* cols, size_t* state_bytes,
+                                         size_t* scratch_bytes);
+SHAMPOO_API int shampoo_soap_init(const shampoo_config* cfg, const shampoo_soap_config* sc, int32_t nparams,
+                                  const int64_t* rows, const int64_t* cols, void* d_state, size_t state_bytes,
+                                  void* d_scratch, size_t scratch_bytes, void* stream, shampoo_soap_handle* out);
+/* One SOAP step over every block; weights fp32, gradients grad_dtype, both
+ * contiguous row-major.  Enqueued on `stream`; no host sync. */
+SHAMPOO_API int shampoo_soap_step(shampoo_soap_handle h, float* const* d_weights, const void* const* d_grads,
+                                  void* stream);
+/* Device views of the state: statistics L, R; bases QL, QR (eigenvectors as
+ * columns); m (original coordinates) and v (eigenbasis), each (nb, B, B);
+ * *step: steps taken. */
+SHAMPOO_API int shampoo_soap_views(shampoo_soap_handle h, float** L, float** R, float** QL, float** QR, float** m,
+                                   float** v, int64_t* step);
+SHAMPOO_API int shampoo_soap_get_status(shampoo_soap_handle h, int32_t* status, int32_t reset);
+SHAMPOO_API void shampoo_soap_destroy(shampoo_soap_handle h);
+
 /* Block packing for blocks sharded across ranks (DASH abstract: the
  * preconditioner blocks are distributed across devices): one launch moves
  * nblocks r x c blocks between row-strided matrices and one packed fp32
@@ -313,6 +354,29 @@ SHAMPOO_API void shampoo_tensor_destroy(shampoo_tensor_handle h);
 SHAMPOO_API int shampoo_pack_blocks(const int64_t* d_table, int32_t nblocks, int32_t nparams, void* const* d_params,
                                     const int64_t* ld, int32_t dtype, float* d_packed, int32_t direction, float scale,
                                     int32_t max_rows, int32_t max_cols, void* stream);
+
+/* Batched symmetric eigendecomposition A_i = Q_i diag(lam_i) Q_i^T (the
+ * eigenbasis SOAP runs Adam in: pith.science SOAP record; the pages name no
+ * method).  warm_start = 0: cyclic Jacobi with the round-robin parallel
+ * ordering (Golub & Van Loan sec. 8.5) from A_i, at most jacobi_sweeps sweeps
+ * (SHAMPOO_DEVFLAG_NOT_CONVERGED if the off-diagonal mass stays above 1e-5 of
+ * ||A_i||_F), then refine_iters iterations of the GEMM-only refinement of
+ * Ogita & Aishima (2018); warm_start = 1: d_Q holds an approximate basis X on
+ * entry (e.g. the previous one): Jacobi runs on the nearly diagonal X^T A X,
+ * X is rotated by its eigenvectors, then the refinement runs.
+ *  d_A       device stack (batch, n, n), symmetrised before use; n a multiple
+ *            of 32 in [32, 1024].
+ *  d_Q       device stack (batch, n, n): eigenvectors as columns, in no
+ *            particular order (Jacobi's); in/out with warm_start = 1.
+ *  d_lam     nullable device (batch, n): eigenvalues, matching Q's columns.
+ *  d_scratch 256-byte aligned, eigh_scratch_bytes(batch, n) for one pass
+ *            (less, but at least one matrix's share, works in chunks).
+ *  d_status  nullable device int32: OR of SHAMPOO_DEVFLAG_*.
+ * Enqueued on `stream`; no host sync. */
+SHAMPOO_API int eigh_scratch_bytes(int64_t batch, int32_t n, size_t* bytes);
+SHAMPOO_API int eigh_batched(const float* d_A, float* d_Q, float* d_lam, int64_t batch, int32_t n,
+                             int32_t warm_start, int32_t jacobi_sweeps, int32_t refine_iters, void* d_scratch,
+                             size_t scratch_bytes, int32_t* d_status, void* stream);
 
 /* The batched fp32-accurate product every stage uses, as a utility:
  * D_i = alpha A_i op(B_i) + beta C_i + gamma I for plain stacks (batch, n, n),

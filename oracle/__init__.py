@@ -41,6 +41,12 @@ Modules:
                   -1/(2k) roots, mode-wise contractions.  Pinned by the matrix
                   case, a Kronecker brute force and a rank-one closed form
                   (tests/test_oracle_tensor.py).
+* ``soap``        SOAP (pith.science SOAP record: Adam run in the eigenbasis of
+                  Shampoo's preconditioner, basis recomputed at a fixed
+                  frequency).  Pinned by the constant-gradient and first-step
+                  closed forms (the latter from the SVD), the reduction to
+                  Adam on diagonal statistics, rotation equivariance and
+                  eigenvector-sign invariance (tests/test_oracle_soap.py).
 """
 from .shampoo import (Block, block_table, inverse_root, accumulate,
                       precondition, ShampooOracle, rel_fro)

@@ -55,7 +55,9 @@ EXPORTS = (
     "shampoo_momentum_view", "shampoo_set_step", "shampoo_destroy",
     "inv_root_scratch_bytes", "inv_root_scratch_bytes_p", "inv_root_batched", "inv_root_batched_noalloc",
     "shampoo_tensor_query_sizes", "shampoo_tensor_init", "shampoo_tensor_step", "shampoo_tensor_views",
-    "shampoo_tensor_get_status", "shampoo_tensor_destroy", "shampoo_pack_blocks",
+    "shampoo_tensor_get_status", "shampoo_tensor_destroy", "shampoo_soap_query_sizes", "shampoo_soap_init",
+    "shampoo_soap_step", "shampoo_soap_views", "shampoo_soap_get_status", "shampoo_soap_destroy",
+    "shampoo_pack_blocks", "eigh_scratch_bytes", "eigh_batched",
     "shampoo_gemm_scratch_bytes",
     "shampoo_gemm_batched",
     "shampoo_profile_enable", "shampoo_profile_reset", "shampoo_profile_read", "shampoo_launch_count",
@@ -66,6 +68,13 @@ class ShampooError(RuntimeError):
     def __init__(self, code: int, msg: str):
         super().__init__(f"{_status_name(code)}: {msg}")
         self.code = code
+
+
+class SoapConfig(ctypes.Structure):
+    """Mirror of ``shampoo_soap_config`` (include/shampoo.h)."""
+
+    _fields_ = [("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("jacobi_sweeps", ctypes.c_int32), ("refine_iters", ctypes.c_int32)]
 
 
 class Config(ctypes.Structure):
@@ -129,8 +138,19 @@ def _load():
                                                 ctypes.POINTER(I32), ctypes.POINTER(I64)]),
         "shampoo_tensor_get_status": (ctypes.c_int, [P, ctypes.POINTER(I32), I32]),
         "shampoo_tensor_destroy": (None, [P]),
+        "shampoo_soap_query_sizes": (ctypes.c_int, [ctypes.POINTER(Config), ctypes.POINTER(SoapConfig), I32,
+                                                    ctypes.POINTER(I64), ctypes.POINTER(I64), sz, sz]),
+        "shampoo_soap_init": (ctypes.c_int, [ctypes.POINTER(Config), ctypes.POINTER(SoapConfig), I32,
+                                             ctypes.POINTER(I64), ctypes.POINTER(I64), P, ctypes.c_size_t, P,
+                                             ctypes.c_size_t, P, ctypes.POINTER(P)]),
+        "shampoo_soap_step": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P), P]),
+        "shampoo_soap_views": (ctypes.c_int, [P] + [ctypes.POINTER(P)] * 6 + [ctypes.POINTER(I64)]),
+        "shampoo_soap_get_status": (ctypes.c_int, [P, ctypes.POINTER(I32), I32]),
+        "shampoo_soap_destroy": (None, [P]),
         "shampoo_pack_blocks": (ctypes.c_int, [P, I32, I32, ctypes.POINTER(P), ctypes.POINTER(I64), I32, P, I32, F,
                                                I32, I32, P]),
+        "eigh_scratch_bytes": (ctypes.c_int, [I64, I32, sz]),
+        "eigh_batched": (ctypes.c_int, [P, P, P, I64, I32, I32, I32, I32, P, ctypes.c_size_t, P, P]),
         "shampoo_gemm_scratch_bytes": (ctypes.c_int, [I64, I32, sz]),
         "shampoo_gemm_batched": (ctypes.c_int, [P, P, P, P, I64, I32, I32, F, F, F, P, ctypes.c_size_t, P, P]),
         "shampoo_profile_enable": (None, [I32]),
@@ -452,6 +472,33 @@ def inv_root_batched(A, p: int = 4, eps: float = 0.0, solver: int = SOLVER_NEWTO
     return X, iters_used, status
 
 
+def eigh_batched(A, Q=None, warm_start: bool = False, jacobi_sweeps: int = 15, refine_iters: int = 2,
+                 stream=None):
+    """Q_i (eigenvectors as columns) and lam_i of a float32 CUDA stack of
+    symmetric matrices A (batch, n, n); with warm_start, Q holds an
+    approximate basis on entry and is refined in place.  Returns
+    (Q, lam, status), all on the device."""
+    import torch
+    if A.dtype != torch.float32 or A.dim() != 3 or A.shape[1] != A.shape[2] or not A.is_cuda:
+        raise ValueError("A must be a float32 CUDA tensor (batch, n, n)")
+    A = A.contiguous()
+    batch, n = A.shape[0], A.shape[1]
+    if Q is None:
+        if warm_start:
+            raise ValueError("warm_start needs Q")
+        Q = torch.empty_like(A)
+    lam = torch.empty((batch, n), dtype=torch.float32, device=A.device)
+    b = ctypes.c_size_t(0)
+    _check(lib.eigh_scratch_bytes(batch, n, ctypes.byref(b)))
+    scratch = torch.empty(b.value, dtype=torch.uint8, device=A.device)
+    status = torch.zeros(1, dtype=torch.int32, device=A.device)
+    with torch.cuda.device(A.device):
+        _check(lib.eigh_batched(A.data_ptr(), Q.data_ptr(), lam.data_ptr(), batch, n, 1 if warm_start else 0,
+                                jacobi_sweeps, refine_iters, scratch.data_ptr(), scratch.numel(), status.data_ptr(),
+                                _stream_ptr(stream)))
+    return Q, lam, status
+
+
 def gemm_batched(A, B, C=None, alpha: float = 1.0, beta: float = 0.0, gamma: float = 0.0, trans_b: bool = True,
                  out=None, scratch=None, stream=None):
     """D_i = alpha A_i op(B_i) + beta C_i + gamma I on the tensor cores (3xTF32),
@@ -473,6 +520,86 @@ def gemm_batched(A, B, C=None, alpha: float = 1.0, beta: float = 0.0, gamma: flo
                                         status.data_ptr(),
                                         _stream_ptr(stream)))
     return D, status
+
+
+def make_soap_config(beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8, jacobi_sweeps: int = 15,
+                     refine_iters: int = 1) -> SoapConfig:
+    return SoapConfig(beta1, beta2, eps, jacobi_sweeps, refine_iters)
+
+
+class Soap:
+    """SOAP (Adam in the eigenbasis of Shampoo's preconditioner) over a fixed
+    list of 2-D weights, blocked like ``Shampoo``.  ``cfg`` gives block, beta,
+    lr, refresh_every and grad_dtype; ``sc`` the Adam and eigensolver
+    settings.  State and scratch are torch allocations owned by this object."""
+
+    def __init__(self, shapes: Sequence[Tuple[int, int]], cfg: Config, sc: SoapConfig, device=None, stream=None):
+        import torch
+        self.shapes = [tuple(int(x) for x in s) for s in shapes]
+        self.cfg, self.sc = cfg, sc
+        self.device = torch.device("cuda" if device is None else device)
+        rows = _i64_array([s[0] for s in self.shapes])
+        cols = _i64_array([s[1] for s in self.shapes])
+        sb_, xb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        _check(lib.shampoo_soap_query_sizes(ctypes.byref(cfg), ctypes.byref(sc), len(self.shapes), rows, cols,
+                                            ctypes.byref(sb_), ctypes.byref(xb)))
+        self.state_bytes, self.scratch_bytes = sb_.value, xb.value
+        self.state = torch.empty(self.state_bytes, dtype=torch.uint8, device=self.device)
+        self.scratch = torch.empty(self.scratch_bytes, dtype=torch.uint8, device=self.device)
+        h = ctypes.c_void_p(None)
+        with torch.cuda.device(self.device):
+            _check(lib.shampoo_soap_init(ctypes.byref(cfg), ctypes.byref(sc), len(self.shapes), rows, cols,
+                                         self.state.data_ptr(), self.state_bytes, self.scratch.data_ptr(),
+                                         self.scratch_bytes, _stream_ptr(stream), ctypes.byref(h)))
+        self._h = h
+        self._destroy = lib.shampoo_soap_destroy
+        self.nb = sum(-(-m // cfg.block) * -(-n // cfg.block) for m, n in self.shapes)
+        self._wbuf = (ctypes.c_void_p * len(self.shapes))()
+        self._gbuf = (ctypes.c_void_p * len(self.shapes))()
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        destroy = getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
+            self._h = None
+
+    def step(self, weights, grads, stream=None):
+        import torch
+        want = torch.bfloat16 if self.cfg.grad_dtype == BF16 else torch.float32
+        if len(weights) != len(self.shapes) or len(grads) != len(self.shapes):
+            raise ValueError("one weight and one gradient per shape")
+        for i, (w, g) in enumerate(zip(weights, grads)):
+            if w.dtype != torch.float32 or g.dtype != want:
+                raise TypeError(f"param {i}: weights must be float32 and grads {want}")
+            if tuple(w.shape) != self.shapes[i] or tuple(g.shape) != self.shapes[i]:
+                raise ValueError(f"param {i}: shape mismatch")
+            if not (w.is_contiguous() and g.is_contiguous()):
+                raise ValueError(f"param {i}: weight and gradient must be contiguous")
+            self._wbuf[i] = w.data_ptr()
+            self._gbuf[i] = g.data_ptr()
+        _check(lib.shampoo_soap_step(self._h, self._wbuf, self._gbuf, _stream_ptr(stream)))
+
+    def status(self, reset: bool = False) -> int:
+        s = ctypes.c_int32(0)
+        _check(lib.shampoo_soap_get_status(self._h, ctypes.byref(s), 1 if reset else 0))
+        return s.value
+
+    def views(self):
+        """dict of float32 (nb, B, B) views: L, R, QL, QR, m, v."""
+        import torch
+        ptrs = [ctypes.c_void_p() for _ in range(6)]
+        step = ctypes.c_int64(0)
+        _check(lib.shampoo_soap_views(self._h, *[ctypes.byref(p) for p in ptrs], ctypes.byref(step)))
+        fl = self.state.view(torch.float32)
+        base = self.state.data_ptr()
+        B, nb = self.cfg.block, self.nb
+        out = {}
+        for name, p in zip(("L", "R", "QL", "QR", "m", "v"), ptrs):
+            o = (p.value - base) // 4
+            out[name] = fl[o:o + nb * B * B].view(nb, B, B)
+        out["step"] = step.value
+        return out
 
 
 class BlockPacker:

@@ -128,6 +128,15 @@ bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) =
 
 }  // namespace
 
+int shampoo::build_block_table(int B, int32_t nparams, const int64_t* rows, const int64_t* cols,
+                               std::vector<int>& table) {
+  Shapes sh;
+  int rc = build_table(B, nparams, rows, cols, sh);
+  if (rc) return rc;
+  table = sh.table;
+  return SHAMPOO_OK;
+}
+
 struct shampoo_ctx {
   shampoo_config cfg;
   int nparams = 0;
@@ -295,8 +304,8 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
   h->last_stream = st;
   int rc;
   // 1. partition / stack (and, with momentum, M <- alpha M + G per block)
-  if ((rc = launch_stack(args, h->d_table, nb, B, c.grad_dtype, h->Gs, h->Gt, h->mom, c.momentum, h->blk_wptr,
-                         h->blk_ld, st, h->stack_bytes)))
+  if ((rc = launch_stack(args, h->d_table, nb, B, c.grad_dtype, h->Gs, h->Gt, h->mom, c.momentum, 1.f,
+                         h->blk_wptr, h->blk_ld, st, h->stack_bytes)))
     return rc;
   // Widened bf16 gradients are exact in tf32: their lo parts are zero, so
   // the products that take G as an operand skip the MMAs with those parts.

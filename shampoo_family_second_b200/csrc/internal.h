@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <vector>
 #include <cuda.h>  // CUtensorMap (type only; the driver entry point is fetched at run time)
 #include <cuda_runtime.h>
 
@@ -158,6 +159,10 @@ struct Builder {
 int launch_report(const int* iters, const int* add, const int* done, int64_t batch, int default_iters, int* out,
                   int* flags, bool residual, cudaStream_t st);
 
+// Block partition of a parameter set (api.cu): table gets nb x {param, row0,
+// col0, r, c}, in (param, block row, block column) order.
+int build_block_table(int B, int32_t nparams, const int64_t* rows, const int64_t* cols, std::vector<int>& table);
+
 // Elementwise / reduction kernels (kernels_elem.cu) ---------------------------
 struct StackArgs {
   const void* g[kMaxParams];
@@ -165,9 +170,10 @@ struct StackArgs {
   int ld[kMaxParams];
   unsigned char vec[kMaxParams];  // rows of param i start 16-byte (fp32) / 8-byte (bf16) aligned
 };
-// M (nullable): momentum stack, updated in place as M <- alpha M + G_b.
+// M (nullable): moment stack, updated in place as M <- alpha M + gscale G_b.
 int launch_stack(const StackArgs& args, const int* d_table, int nb, int B, int grad_dtype, float* Gs, float* Gts,
-                 float* M, float alpha, float** blk_wptr, int* blk_ld, cudaStream_t st, double alg_bytes);
+                 float* M, float alpha, float gscale, float** blk_wptr, int* blk_ld, cudaStream_t st,
+                 double alg_bytes);
 
 int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, float eps, int p, float* s, float* sc,
                      cudaStream_t st);
@@ -223,6 +229,13 @@ int inv_root_batched_impl(const float* d_A, float* d_X, int64_t batch, int n, in
                           float tol, int cheb_degree, float cheb_lo, void* d_scratch, size_t scratch_bytes,
                           int* d_iters_used, int* d_status, cudaStream_t st, bool plain_launches);
 size_t root_scratch_per_matrix(int n, int solver, int p);
+// Batched symmetric eigendecomposition (eigen.cu): Q (columns) and lam
+// (nullable) of the valid part of each A_i; warm_start = 0: cyclic Jacobi (at
+// most jacobi_sweeps) from scratch, then refine_iters refinement iterations;
+// warm_start = 1: Q holds an approximate basis on entry, refinement only.
+size_t eig_scratch_per_matrix(int n);
+int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const int* valid, int warm_start,
+             int jacobi_sweeps, int refine_iters, void* scratch, size_t scratch_bytes, int* flags, cudaStream_t st);
 size_t root_scratch_header();
 int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, cudaStream_t st);
 

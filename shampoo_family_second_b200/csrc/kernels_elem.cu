@@ -58,12 +58,14 @@ __device__ __forceinline__ float4 load_grad4(const void* g, size_t idx, int dtyp
   return v;
 }
 
-// With momentum (M != NULL) the same pass updates the block's momentum in
-// place, M_b <- alpha M_b + G_b (podcast cue 28: momentum ahead of the
-// preconditioner; the statistics keep the raw G in Gs and Gt).
+// With a moment stack (M != NULL) the same pass updates it in place,
+// M_b <- alpha M_b + gscale G_b: Shampoo's momentum ahead of the
+// preconditioner (podcast cue 28; gscale = 1) or Adam's first moment (SOAP;
+// alpha = beta1, gscale = 1 - beta1).  The statistics keep the raw G in Gs, Gt.
 __global__ void stack_blocks_kernel(const __grid_constant__ StackArgs args, const int* __restrict__ table, int B,
                                     int dtype, float* __restrict__ Gs, float* __restrict__ Gt,
-                                    float* __restrict__ M, float alpha, float** blk_wptr, int* blk_ld) {
+                                    float* __restrict__ M, float alpha, float gscale, float** blk_wptr,
+                                    int* blk_ld) {
   pdl_launch_dependents();  // a following GEMM may start its prologue
   constexpr int TC = 128, STRIDE = TC + 4;
   __shared__ __align__(16) float tile[32 * STRIDE];
@@ -90,10 +92,10 @@ __global__ void stack_blocks_kernel(const __grid_constant__ StackArgs args, cons
       if (M) {
         float4* mp = reinterpret_cast<float4*>(M + b * nn + static_cast<size_t>(row) * B + col);
         float4 m = *mp;
-        m.x = fmaf(alpha, m.x, v.x);
-        m.y = fmaf(alpha, m.y, v.y);
-        m.z = fmaf(alpha, m.z, v.z);
-        m.w = fmaf(alpha, m.w, v.w);
+        m.x = fmaf(alpha, m.x, gscale * v.x);
+        m.y = fmaf(alpha, m.y, gscale * v.y);
+        m.z = fmaf(alpha, m.z, gscale * v.z);
+        m.w = fmaf(alpha, m.w, gscale * v.w);
         *mp = m;
       }
       *reinterpret_cast<float4*>(&tile[(ty + 8 * k) * STRIDE + 4 * tx]) = v;
@@ -495,11 +497,13 @@ __global__ void fill_int_kernel(int* p, int64_t count, int value) {
 }  // namespace
 
 int launch_stack(const StackArgs& args, const int* d_table, int nb, int B, int grad_dtype, float* Gs, float* Gts,
-                 float* M, float alpha, float** blk_wptr, int* blk_ld, cudaStream_t st, double alg_bytes) {
+                 float* M, float alpha, float gscale, float** blk_wptr, int* blk_ld, cudaStream_t st,
+                 double alg_bytes) {
   if (nb == 0) return 0;
   ProfScope ps(K_STACK, st, 0.0, alg_bytes);
   dim3 grid((B + 127) / 128, B / 32, nb), block(32, 8);
-  stack_blocks_kernel<<<grid, block, 0, st>>>(args, d_table, B, grad_dtype, Gs, Gts, M, alpha, blk_wptr, blk_ld);
+  stack_blocks_kernel<<<grid, block, 0, st>>>(args, d_table, B, grad_dtype, Gs, Gts, M, alpha, gscale, blk_wptr,
+                                              blk_ld);
   count_launch();
   return check_cuda(cudaGetLastError(), "stack_blocks_kernel");
 }

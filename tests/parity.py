@@ -220,3 +220,50 @@ def tensor_apply_check(P_gpu, G, roots):
     den = np.linalg.norm(P64)
     cancel = np.linalg.norm(precondition_tensor(np.abs(G), [np.abs(X) for X in roots])) / den if den > 0 else 1.0
     return rel_fro(P_gpu, P64), TOL_APPLY * max(1.0, cancel)
+
+
+class Fp32ReferenceSoap:
+    """SOAP in float32 with single-precision LAPACK eigenbases: the update
+    floor's reference for the SOAP path (same order of operations as
+    oracle.soap.SoapOracle)."""
+
+    def __init__(self, shapes, block, beta, refresh_every, beta1, beta2, eps, blocks):
+        from oracle import block_table
+        self.table = block_table(shapes, block)
+        self.blocks = list(blocks)
+        f = np.float32
+        self.beta, self.k = f(beta), refresh_every
+        self.b1, self.b2, self.eps = f(beta1), f(beta2), f(eps)
+        self.L = {b: np.zeros((self.table[b].r,) * 2, f) for b in self.blocks}
+        self.R = {b: np.zeros((self.table[b].c,) * 2, f) for b in self.blocks}
+        self.QL = {b: np.eye(self.table[b].r, dtype=f) for b in self.blocks}
+        self.QR = {b: np.eye(self.table[b].c, dtype=f) for b in self.blocks}
+        self.m = {b: np.zeros((self.table[b].r, self.table[b].c), f) for b in self.blocks}
+        self.v = {b: np.zeros((self.table[b].r, self.table[b].c), f) for b in self.blocks}
+        self.t = 0
+
+    def step(self, grads):
+        refresh = self.t % self.k == 0
+        self.t += 1
+        c1 = np.float32(1.0 / (1.0 - float(self.b1) ** self.t))
+        c2 = np.float32(1.0 / (1.0 - float(self.b2) ** self.t))
+        out = {}
+        for b in self.blocks:
+            blk = self.table[b]
+            G = np.asarray(grads[blk.param][blk.row0:blk.row0 + blk.r, blk.col0:blk.col0 + blk.c], np.float32)
+            QL, QR = self.QL[b], self.QR[b]
+            Gr = QL.T @ G @ QR
+            self.m[b] = self.b1 * self.m[b] + (np.float32(1) - self.b1) * G
+            self.v[b] = self.b2 * self.v[b] + (np.float32(1) - self.b2) * Gr * Gr
+            Nr = (QL.T @ self.m[b] @ QR * c1) / (np.sqrt(self.v[b] * c2) + self.eps)
+            out[b] = (QL @ Nr @ QR.T).astype(np.float64)
+            self.L[b] = self.beta * self.L[b] + G @ G.T
+            self.R[b] = self.beta * self.R[b] + G.T @ G
+            if refresh:
+                QLn = scipy.linalg.eigh(0.5 * (self.L[b] + self.L[b].T), driver="evd")[1].astype(np.float32)
+                QRn = scipy.linalg.eigh(0.5 * (self.R[b] + self.R[b].T), driver="evd")[1].astype(np.float32)
+                PL = (QLn.T @ QL) ** 2
+                PR = (QRn.T @ QR) ** 2
+                self.v[b] = PL @ self.v[b] @ PR.T
+                self.QL[b], self.QR[b] = QLn, QRn
+        return out

@@ -180,3 +180,28 @@ def test_tensor_sizes_and_validation(sb):
     sb.tensor_query_sizes(db, [(40, 50)])
     with pytest.raises(sb.ShampooError):
         sb.tensor_query_sizes(db, [(4, 5, 6)])
+
+
+def test_eigh_argument_errors(sb):
+    b = ctypes.c_size_t(0)
+    assert sb.lib.eigh_scratch_bytes(4, 64, ctypes.byref(b)) == 0 and b.value >= 4 * 5 * 64 * 64 * 4
+    assert sb.lib.eigh_scratch_bytes(4, 48, ctypes.byref(b)) == sb.ERR_INVALID_ARG
+    assert sb.lib.eigh_batched(None, None, None, 0, 64, 0, 10, 2, None, 0, None, None) == 0
+    assert sb.lib.eigh_batched(None, None, None, 2, 64, 0, 10, 2, None, 0, None, None) == sb.ERR_INVALID_ARG
+
+
+def test_soap_sizes_and_validation(sb):
+    """SOAP keeps statistics, bases and their transposes (2 nb stacks each) and
+    the two moments (nb each): 8 nb block matrices of state."""
+    cfg = sb.make_config(128, 0.95, 0.0, 1e-3, refresh_every=10)
+    sc = sb.make_soap_config()
+    rows = (ctypes.c_int64 * 2)(256, 128)
+    cols = (ctypes.c_int64 * 2)(256, 384)
+    st, xs = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert sb.lib.shampoo_soap_query_sizes(ctypes.byref(cfg), ctypes.byref(sc), 2, rows, cols, ctypes.byref(st),
+                                           ctypes.byref(xs)) == 0
+    nb = 4 + 3
+    assert st.value >= 8 * nb * 128 * 128 * 4
+    for bad in (sb.make_soap_config(beta1=1.0), sb.make_soap_config(eps=0.0), sb.make_soap_config(jacobi_sweeps=0)):
+        assert sb.lib.shampoo_soap_query_sizes(ctypes.byref(cfg), ctypes.byref(bad), 2, rows, cols,
+                                               ctypes.byref(st), ctypes.byref(xs)) == sb.ERR_INVALID_ARG
