@@ -121,7 +121,12 @@ enum {
  *  momentum       alpha in [0, 1): 0 = off (the update uses the raw gradient); > 0 keeps a
  *                 per-block momentum M <- alpha M + G (from M = 0) ahead of the preconditioner,
  *                 and the update becomes W <- W - lr XL M XR, while the statistics still take
- *                 the raw G (podcast transcript, cue 28: momentum 0.9 before preconditioning). */
+ *                 the raw G (podcast transcript, cue 28: momentum 0.9 before preconditioning).
+ *  diag_threshold tensor Shampoo only (the blocked step's blocks never exceed 1024): a
+ *                 dimension longer than this keeps only the diagonal of its statistic
+ *                 (podcast transcript, cue 28: diagonal variant past a size threshold,
+ *                 decided per dimension).  <= 0: 1024, the largest root the solvers
+ *                 compute; at most 1024. */
 typedef struct {
   int32_t block;
   float beta;
@@ -136,6 +141,7 @@ typedef struct {
   float cheb_lo;
   int32_t grad_dtype;
   float momentum;
+  int32_t diag_threshold;
 } shampoo_config;
 
 typedef struct shampoo_ctx* shampoo_handle;
@@ -262,17 +268,20 @@ SHAMPOO_API int inv_root_batched_noalloc(const float* d_A, float* d_X, int64_t b
 
 /* Order-k tensor Shampoo (podcast transcript "Preconditioned optimization
  * without the full matrix cost", cue 26): for a parameter of order k in
- * [2, 4] with dimensions d_0 .. d_{k-1} (each in [1, 1024]; larger gives
- * SHAMPOO_ERR_UNSUPPORTED), one statistic per dimension,
+ * [2, 4] with dimensions d_0 .. d_{k-1} (each in [1, 2^20]), one statistic per
+ * dimension,
  *     H_i <- beta H_i + G_(i) G_(i)^T      (G_(i): mode-i unfolding of G, the
  *                                           other indices in row-major order)
  *     X_i = (H_i + eps I)^{-1/(2k)}        (every refresh_every steps)
  *     W <- W - lr  G x_0 X_0 x_1 X_1 ... x_{k-1} X_{k-1}
- * (x_i: contraction along dimension i).  The parameters are not blocked.
+ * (x_i: contraction along dimension i).  The parameters are not blocked.  A
+ * dimension longer than cfg.diag_threshold keeps the diagonal h_i of H_i
+ * (cue 28's diagonal variant) and scales its dimension by
+ * d_i = (h_i + eps)^{-1/(2k)} (0 where h_i + eps = 0).
  * Config fields used: beta, eps, lr, solver (coupled Newton either degree,
  * Chebyshev; Newton-DB for order 2 only), iters, tol, refresh_every,
- * cheb_degree, cheb_lo, grad_dtype; block and root_p are ignored, momentum
- * must be 0.  orders[j] is the order of parameter j; dims holds all
+ * cheb_degree, cheb_lo, grad_dtype, diag_threshold; block and root_p are
+ * ignored, momentum must be 0.  orders[j] is the order of parameter j; dims holds all
  * parameters' dimensions back to back.  Weights are fp32 and gradients
  * grad_dtype, both row-major (natural layout), device pointers in host
  * arrays.  Ownership, streams and errors as for shampoo_init / shampoo_step;
@@ -287,9 +296,10 @@ SHAMPOO_API int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_wei
                                     void* stream);
 /* Device pointers to the statistic H_i and root X_i of mode `mode` of
  * parameter `param`: npad x npad fp32 (npad = d_i rounded up to 32; zero /
- * identity-scaled beyond d_i); *step: steps taken. */
+ * identity-scaled beyond d_i), or, when *diagonal = 1, the d_i-vectors h_i and
+ * d_i of the diagonal variant (then *npad = d_i); *step: steps taken. */
 SHAMPOO_API int shampoo_tensor_views(shampoo_tensor_handle h, int32_t param, int32_t mode, float** H, float** X,
-                                     int32_t* npad, int64_t* step);
+                                     int32_t* npad, int32_t* diagonal, int64_t* step);
 /* As shampoo_get_status, for a tensor handle. */
 SHAMPOO_API int shampoo_tensor_get_status(shampoo_tensor_handle h, int32_t* status, int32_t reset);
 SHAMPOO_API void shampoo_tensor_destroy(shampoo_tensor_handle h);

@@ -15,6 +15,14 @@ Readings (as in the matrix oracle): statistics start at zero and decay by
 beta with no (1 - beta) factor; roots are of (H + eps I), by symmetric
 eigendecomposition; roots are refreshed every ``refresh_every`` steps from
 step 0; the update is W <- W - lr P.
+
+Diagonal variant (cue 28: past a size threshold, about 1200 in the paper's
+experiments, a dimension keeps only the diagonal of its statistic, decided
+independently per dimension): a mode with n_i > ``diag_threshold`` keeps
+h_i = diag(H_i), updated as h_i <- beta h_i + (sum over the other modes of
+G^2), and is preconditioned by the scaling d_i = (h_i + eps)^{-1/(2k)} along
+its dimension (d_i = 0 where h_i + eps = 0, which only happens with eps = 0
+on an index the gradient has never touched).
 """
 from __future__ import annotations
 
@@ -46,17 +54,35 @@ def precondition_tensor(G: np.ndarray, roots: Sequence[np.ndarray], order: Seque
     return P
 
 
-class TensorShampooOracle:
-    """Order-k Shampoo on one tensor parameter, one step at a time."""
+def mode_diagonal_statistic(G: np.ndarray, i: int) -> np.ndarray:
+    """diag(mode_statistic(G, i)): the sum of G^2 over every mode but i."""
+    others = tuple(j for j in range(G.ndim) if j != i)
+    return np.sum(np.asarray(G, dtype=np.float64) ** 2, axis=others)
 
-    def __init__(self, shape, beta: float, eps: float, lr: float, refresh_every: int = 1, weight=None):
+
+def diagonal_root(h: np.ndarray, p: int, eps: float) -> np.ndarray:
+    """(h + eps)^{-1/p} elementwise, 0 where h + eps = 0."""
+    x = np.asarray(h, dtype=np.float64) + eps
+    out = np.zeros_like(x)
+    pos = x > 0
+    out[pos] = x[pos] ** (-1.0 / p)
+    return out
+
+
+class TensorShampooOracle:
+    """Order-k Shampoo on one tensor parameter, one step at a time.  Modes
+    longer than ``diag_threshold`` (None: none) use the diagonal variant."""
+
+    def __init__(self, shape, beta: float, eps: float, lr: float, refresh_every: int = 1, weight=None,
+                 diag_threshold: int | None = None):
         self.shape = tuple(int(x) for x in shape)
         self.k = len(self.shape)
         self.beta = float(beta)
         self.eps = float(eps)
         self.lr = float(lr)
         self.refresh_every = int(refresh_every)
-        self.H: List[np.ndarray] = [np.zeros((n, n)) for n in self.shape]
+        self.diag = [diag_threshold is not None and n > diag_threshold for n in self.shape]
+        self.H: List[np.ndarray] = [np.zeros(n) if d else np.zeros((n, n)) for n, d in zip(self.shape, self.diag)]
         self.X: List[np.ndarray] = [None] * self.k
         self.W = np.zeros(self.shape) if weight is None else np.array(weight, dtype=np.float64)
         self.t = 0
@@ -66,10 +92,19 @@ class TensorShampooOracle:
         update; returns the preconditioned gradient P."""
         G = np.asarray(grad, dtype=np.float64)
         for i in range(self.k):
-            self.H[i] = self.beta * self.H[i] + mode_statistic(G, i)
+            stat = mode_diagonal_statistic(G, i) if self.diag[i] else mode_statistic(G, i)
+            self.H[i] = self.beta * self.H[i] + stat
         if self.t % self.refresh_every == 0:
-            self.X = [inverse_root(H, 2 * self.k, self.eps) for H in self.H]
-        P = precondition_tensor(G, self.X)
+            self.X = [diagonal_root(H, 2 * self.k, self.eps) if d else inverse_root(H, 2 * self.k, self.eps)
+                      for H, d in zip(self.H, self.diag)]
+        P = G
+        for i in range(self.k):
+            if self.diag[i]:
+                shape = [1] * self.k
+                shape[i] = self.shape[i]
+                P = P * self.X[i].reshape(shape)
+            else:
+                P = mode_product(P, self.X[i], i)
         self.W -= self.lr * P
         self.t += 1
         return P

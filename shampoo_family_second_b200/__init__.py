@@ -84,21 +84,22 @@ class Config(ctypes.Structure):
         ("block", ctypes.c_int32), ("beta", ctypes.c_float), ("eps", ctypes.c_float), ("lr", ctypes.c_float),
         ("root_p", ctypes.c_int32), ("solver", ctypes.c_int32), ("iters", ctypes.c_int32), ("tol", ctypes.c_float),
         ("refresh_every", ctypes.c_int32), ("cheb_degree", ctypes.c_int32), ("cheb_lo", ctypes.c_float),
-        ("grad_dtype", ctypes.c_int32), ("momentum", ctypes.c_float),
+        ("grad_dtype", ctypes.c_int32), ("momentum", ctypes.c_float), ("diag_threshold", ctypes.c_int32),
     ]
 
 
 def make_config(block: int, beta: float, eps: float, lr: float, root_p: int = 4, solver: int = SOLVER_NEWTON,
                 iters: int = 40, tol: float = 1e-5, refresh_every: int = 1, cheb_degree: int = 32,
-                cheb_lo: float = 0.0, grad_dtype: int = F32, momentum: float = 0.0) -> Config:
+                cheb_lo: float = 0.0, grad_dtype: int = F32, momentum: float = 0.0, diag_threshold: int = 0) -> Config:
     return Config(block, beta, eps, lr, root_p, solver, iters, tol, refresh_every, cheb_degree, cheb_lo, grad_dtype,
-                  momentum)
+                  momentum, diag_threshold)
 
 
 def config_from_workload(wl) -> Config:
     """Config of a ``workloads.Workload`` preset."""
     return make_config(wl.block, wl.beta, wl.eps, wl.lr, wl.root_p, wl.solver, wl.iters, wl.tol, wl.refresh_every,
-                       wl.cheb_degree, wl.cheb_lo, wl.grad_dtype, getattr(wl, "momentum", 0.0))
+                       wl.cheb_degree, wl.cheb_lo, wl.grad_dtype, getattr(wl, "momentum", 0.0),
+                       getattr(wl, "diag_threshold", 0))
 
 
 def _load():
@@ -135,7 +136,7 @@ def _load():
                                                P, ctypes.c_size_t, P, ctypes.c_size_t, P, ctypes.POINTER(P)]),
         "shampoo_tensor_step": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P), P]),
         "shampoo_tensor_views": (ctypes.c_int, [P, I32, I32, ctypes.POINTER(P), ctypes.POINTER(P),
-                                                ctypes.POINTER(I32), ctypes.POINTER(I64)]),
+                                                ctypes.POINTER(I32), ctypes.POINTER(I32), ctypes.POINTER(I64)]),
         "shampoo_tensor_get_status": (ctypes.c_int, [P, ctypes.POINTER(I32), I32]),
         "shampoo_tensor_destroy": (None, [P]),
         "shampoo_soap_query_sizes": (ctypes.c_int, [ctypes.POINTER(Config), ctypes.POINTER(SoapConfig), I32,
@@ -429,16 +430,20 @@ class TensorShampoo:
         return s.value
 
     def mode_views(self, param: int, mode: int):
-        """(H, X) of one mode as float32 (npad, npad) views into the state; the
-        statistic's dimension d occupies the leading d x d block."""
+        """(H, X) of one mode as float32 (npad, npad) views into the state (the
+        statistic's dimension d occupies the leading d x d block), or, for a
+        mode that keeps only its diagonal, the d-vectors (h, d)."""
         import torch
         ph, px = ctypes.c_void_p(), ctypes.c_void_p()
-        npad, step = ctypes.c_int32(0), ctypes.c_int64(0)
+        npad, diag, step = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int64(0)
         _check(lib.shampoo_tensor_views(self._h, param, mode, ctypes.byref(ph), ctypes.byref(px),
-                                        ctypes.byref(npad), ctypes.byref(step)))
+                                        ctypes.byref(npad), ctypes.byref(diag), ctypes.byref(step)))
         fl = self.state.view(torch.float32)
         base = self.state.data_ptr()
         n = npad.value
+        if diag.value:
+            return (fl[(ph.value - base) // 4:(ph.value - base) // 4 + n],
+                    fl[(px.value - base) // 4:(px.value - base) // 4 + n])
         H = fl[(ph.value - base) // 4:(ph.value - base) // 4 + n * n].view(n, n)
         X = fl[(px.value - base) // 4:(px.value - base) // 4 + n * n].view(n, n)
         return H, X

@@ -14,7 +14,10 @@
 //   4. apply    V = X_0 U_0; then for i = 1 .. k-1: V <- X_i unfold_i(fold_{i-1}(V))
 //               (a permutation pass between the products), and the last
 //               fold writes W <- W - lr P into the weight.
-// Dimensions above 1024 are not supported (SHAMPOO_ERR_UNSUPPORTED).
+// Diagonal variant (cue 28): a dimension longer than the threshold keeps only
+// h_i = diag(H_i) (the row sums of squares of U_i), is refreshed to
+// d_i = (h_i + eps)^{-1/(2k)} elementwise, and its "product" scales the rows
+// of the mode-i unfolding by d_i.
 #include <algorithm>
 #include <cstring>
 #include <map>
@@ -141,11 +144,53 @@ int launch_permute(const PermArgs& a, int64_t total, cudaStream_t st) {
   return check_cuda(cudaGetLastError(), "tensor_permute_kernel");
 }
 
+// Diagonal variant, statistics: h[x] <- beta h[x] + sum_c U[x][c]^2 over the
+// row x of the mode's unfolding (one warp per row, float64 sums).
+__global__ void row_sumsq_kernel(const float* __restrict__ U, int64_t ld, int n, int64_t K, float beta,
+                                 float* __restrict__ h) {
+  pdl_launch_dependents();
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n) return;
+  const float* row = U + static_cast<int64_t>(warp) * ld;
+  double acc = 0.0;
+  for (int64_t c = lane; c < K; c += 32) {
+    const double v = row[c];
+    acc += v * v;
+  }
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) h[warp] = static_cast<float>(static_cast<double>(beta) * h[warp] + acc);
+}
+
+// Diagonal variant, roots: d = (h + eps)^{-1/p}, 0 where h + eps = 0.
+__global__ void diag_root_kernel(const float* __restrict__ h, int n, float eps, float inv_p, float* __restrict__ d,
+                                 int* flags) {
+  const int x = blockIdx.x * blockDim.x + threadIdx.x;
+  if (x >= n) return;
+  const float v = h[x] + eps;
+  const float r = v > 0.f ? powf(v, -inv_p) : 0.f;
+  if (!isfinite(r)) raise_flag(flags, DEV_FLAG_NONFINITE);
+  d[x] = r;
+}
+
+// Diagonal variant, product along the mode: out[x][c] = d[x] cur[x][c] for
+// x < n (zero on the padded rows).
+__global__ void row_scale_kernel(const float* __restrict__ cur, const float* __restrict__ d, int n, int rows,
+                                 int64_t cols, float* __restrict__ out) {
+  pdl_launch_dependents();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<int64_t>(rows) * cols) return;
+  const int x = static_cast<int>(t / cols);
+  out[t] = x < n ? d[x] * cur[t] : 0.f;
+}
+
 struct Mode {
   int n, npad;
   int64_t K;
   int Kpad;
-  int group, slot;   // root group and index in its stacks
+  int diag;          // 1: diagonal variant (h, d vectors instead of H, X)
+  int group, slot;   // root group and index in its stacks (matrix modes)
+  size_t h_off, d_off;  // state byte offsets of h and d (diagonal modes)
   size_t u_off;      // float offset of U_i in the unfolding area (per parameter)
 };
 
@@ -189,6 +234,9 @@ int validate_tensor_config(const shampoo_config* c) {
   if (c->grad_dtype != SHAMPOO_F32 && c->grad_dtype != SHAMPOO_BF16)
     return set_error(SHAMPOO_ERR_INVALID_ARG, "grad_dtype must be SHAMPOO_F32 or SHAMPOO_BF16");
   if (c->momentum != 0.f) return set_error(SHAMPOO_ERR_UNSUPPORTED, "tensor Shampoo takes no momentum");
+  if (c->diag_threshold > 1024)
+    return set_error(SHAMPOO_ERR_INVALID_ARG, "diag_threshold %d above 1024, the largest root computed",
+                     c->diag_threshold);
   return SHAMPOO_OK;
 }
 
@@ -197,6 +245,7 @@ int make_plan(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
     return set_error(SHAMPOO_ERR_INVALID_ARG, "nparams %d: need 1..%d", nparams, kMaxTensorParams);
   if (!orders || !dims) return set_error(SHAMPOO_ERR_INVALID_ARG, "orders/dims is NULL");
   P = Plan();
+  const int thr = cfg->diag_threshold > 0 ? cfg->diag_threshold : 1024;
   std::map<std::pair<int, int>, int> gid;
   size_t di = 0;
   for (int j = 0; j < nparams; ++j) {
@@ -209,7 +258,8 @@ int make_plan(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
     for (int l = 0; l < pr.k; ++l) {
       const int64_t d = dims[di + l];
       if (d < 1) return set_error(SHAMPOO_ERR_INVALID_ARG, "param %d dimension %d is %lld", j, l, (long long)d);
-      if (d > 1024) return set_error(SHAMPOO_ERR_UNSUPPORTED, "param %d dimension %d is %lld > 1024", j, l, (long long)d);
+      if (d > (1 << 20)) return set_error(SHAMPOO_ERR_UNSUPPORTED, "param %d dimension %d is %lld > 2^20", j, l,
+                                          (long long)d);
       pr.dims[l] = static_cast<int>(d);
       pr.size *= d;
     }
@@ -223,6 +273,15 @@ int make_plan(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
       m.npad = up32(m.n);
       m.K = pr.size / m.n;
       m.Kpad = up32(m.K);
+      m.diag = m.n > thr ? 1 : 0;
+      m.group = m.slot = -1;
+      m.h_off = m.d_off = 0;
+      m.u_off = pr.u_floats;
+      pr.u_floats += alt(static_cast<size_t>(m.npad) * m.Kpad * 4) / 4;
+      if (m.diag) {
+        pr.modes.push_back(m);
+        continue;
+      }
       auto key = std::make_pair(m.npad, p);
       auto it = gid.find(key);
       if (it == gid.end()) {
@@ -236,8 +295,6 @@ int make_plan(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
       m.group = it->second;
       m.slot = P.groups[m.group].count++;
       P.groups[m.group].valid.push_back(m.n);
-      m.u_off = pr.u_floats;
-      pr.u_floats += alt(static_cast<size_t>(m.npad) * m.Kpad * 4) / 4;
       pr.modes.push_back(m);
     }
     P.params.push_back(pr);
@@ -251,6 +308,12 @@ int make_plan(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
     g.h_off = o, o += alt(mat * g.count);
     g.x_off = o, o += alt(mat * g.count);
   }
+  for (Param& pr : P.params)
+    for (Mode& m : pr.modes)
+      if (m.diag) {
+        m.h_off = o, o += alt(static_cast<size_t>(m.n) * 4);
+        m.d_off = o, o += alt(static_cast<size_t>(m.n) * 4);
+      }
   P.state_total = o;
   // scratch: all unfoldings of the largest parameter | two product buffers | root solver
   P.u_area = 0;
@@ -391,20 +454,29 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
       a.rows = m.npad;
       a.cols = m.Kpad;
       if ((rc = launch_permute(a, static_cast<int64_t>(m.npad) * m.Kpad, st))) return rc;
-      if ((rc = make_rect_maps(um[i], U + m.u_off, 1, m.npad, m.Kpad))) return rc;
+      if (!m.diag && (rc = make_rect_maps(um[i], U + m.u_off, 1, m.npad, m.Kpad))) return rc;
     }
     Builder b;
     for (int i = 0; i < pr.k; ++i) {
       const Mode& m = pr.modes[i];
+      if (m.diag) {
+        ProfScope ps(K_NORM, st, 0.0, 4.0 * m.n * double(m.Kpad));
+        const unsigned blocks = static_cast<unsigned>((static_cast<int64_t>(m.n) * 32 + 255) / 256);
+        row_sumsq_kernel<<<blocks, 256, 0, st>>>(U + m.u_off, m.Kpad, m.n, m.K, c.beta,
+                                                 reinterpret_cast<float*>(h->state + m.h_off));
+        count_launch();
+        if ((rc = check_cuda(cudaGetLastError(), "row_sumsq_kernel"))) return rc;
+        continue;
+      }
       Epilogue& e = b.add_rect(1, m.npad, m.npad, m.Kpad, um[i], 0, um[i], 0, 2.0 * m.n * double(m.n) * m.K,
                                B_TRANSPOSED);
-      b.L.g[i].a_exact = b.L.g[i].b_exact = g_exact;
+      b.L.g[b.L.ngroups - 1].a_exact = b.L.g[b.L.ngroups - 1].b_exact = g_exact;
       e.beta = c.beta;
       e.C = hptr(m);
       e.D = hptr(m);
       e.flags = h->d_status;
     }
-    if ((rc = b.launch(st))) return rc;
+    if (b.L.ngroups > 0 && (rc = b.launch(st))) return rc;
   }
   // 3. roots X = (H + eps I)^{-1/(2k)}, batched per (npad, k)
   if (refresh) {
@@ -427,6 +499,16 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
       job.flags = h->d_status;
       if ((rc = run_inverse_roots(job, h->scratch + P.scratch_root, P.root_bytes, st))) return rc;
     }
+    for (const Param& pr : P.params)
+      for (const Mode& m : pr.modes) {
+        if (!m.diag) continue;
+        ProfScope ps(K_FINALIZE, st, 0.0, 8.0 * m.n);
+        diag_root_kernel<<<static_cast<unsigned>((m.n + 255) / 256), 256, 0, st>>>(
+            reinterpret_cast<const float*>(h->state + m.h_off), m.n, c.eps, 1.f / (2 * pr.k),
+            reinterpret_cast<float*>(h->state + m.d_off), h->d_status);
+        count_launch();
+        if ((rc = check_cuda(cudaGetLastError(), "diag_root_kernel"))) return rc;
+      }
   }
   // 4. apply: V = X_0 unfold_0(G), then mode by mode; the last fold updates W.
   for (size_t j = 0; j < P.params.size(); ++j) {
@@ -466,6 +548,15 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
         a.cols = m.Kpad;
         if ((rc = launch_permute(a, static_cast<int64_t>(m.npad) * m.Kpad, st))) return rc;
       }
+      if (m.diag) {
+        ProfScope ps(K_FINALIZE, st, 0.0, 8.0 * m.npad * double(m.Kpad));
+        const int64_t total = static_cast<int64_t>(m.npad) * m.Kpad;
+        row_scale_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
+            cur, reinterpret_cast<const float*>(h->state + m.d_off), m.n, m.npad, m.Kpad, out);
+        count_launch();
+        if ((rc = check_cuda(cudaGetLastError(), "row_scale_kernel"))) return rc;
+        continue;
+      }
       StackMaps cm;
       if ((rc = make_rect_maps(cm, cur, 1, m.npad, m.Kpad))) return rc;
       Builder b;
@@ -496,12 +587,20 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
 }
 
 int shampoo_tensor_views(shampoo_tensor_handle h, int32_t param, int32_t mode, float** H, float** X, int32_t* npad,
-                         int64_t* step) {
+                         int32_t* diagonal, int64_t* step) {
   if (!h) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle is NULL");
   const Plan& P = h->plan;
   if (param < 0 || param >= static_cast<int>(P.params.size()) || mode < 0 || mode >= P.params[param].k)
     return set_error(SHAMPOO_ERR_INVALID_ARG, "no mode %d of param %d", mode, param);
   const Mode& m = P.params[param].modes[mode];
+  if (diagonal) *diagonal = m.diag;
+  if (step) *step = h->step;
+  if (m.diag) {
+    if (H) *H = reinterpret_cast<float*>(h->state + m.h_off);
+    if (X) *X = reinterpret_cast<float*>(h->state + m.d_off);
+    if (npad) *npad = m.n;
+    return SHAMPOO_OK;
+  }
   const Group& G = P.groups[m.group];
   const size_t off = static_cast<size_t>(m.slot) * G.npad * G.npad;
   if (H) *H = reinterpret_cast<float*>(h->state + G.h_off) + off;

@@ -162,8 +162,9 @@ def test_momentum_state_is_one_more_block_stack(sb):
 
 
 def test_tensor_sizes_and_validation(sb):
-    """Tensor Shampoo: orders 2..4, dimensions up to 1024; state holds one
-    statistic and one root per mode (padded to multiples of 32)."""
+    """Tensor Shampoo: orders 2..4; state holds one statistic and one root per
+    mode (padded to multiples of 32), or two vectors for a mode past the
+    diagonal threshold."""
     cfg = sb.make_config(32, 0.9, 1e-4, 1e-3, solver=3)
     state, scratch = sb.tensor_query_sizes(cfg, [(3, 3, 64, 128)])
     per_mode = [32, 32, 64, 128]
@@ -173,9 +174,15 @@ def test_tensor_sizes_and_validation(sb):
         with pytest.raises(sb.ShampooError) as e:
             sb.tensor_query_sizes(cfg, bad)
         assert e.value.code == sb.ERR_INVALID_ARG
+    # a dimension above the diagonal threshold keeps a vector: 2048 + 2048 floats, not 2048^2
+    state_d, _ = sb.tensor_query_sizes(cfg, [(2048, 8)])
+    assert state_d < 2 * 2048 * 2048 * 4
     with pytest.raises(sb.ShampooError) as e:
-        sb.tensor_query_sizes(cfg, [(2048, 8)])
+        sb.tensor_query_sizes(cfg, [((1 << 20) + 1, 2)])
     assert e.value.code == sb.ERR_UNSUPPORTED
+    with pytest.raises(sb.ShampooError) as e:
+        sb.tensor_query_sizes(sb.make_config(32, 0.9, 1e-4, 1e-3, solver=3, diag_threshold=2000), [(8, 8)])
+    assert e.value.code == sb.ERR_INVALID_ARG
     db = sb.make_config(32, 0.9, 1e-4, 1e-3, solver=1)
     sb.tensor_query_sizes(db, [(40, 50)])
     with pytest.raises(sb.ShampooError):

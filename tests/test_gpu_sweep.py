@@ -10,11 +10,17 @@ Solvers and gates (DASH abstract: Newton-DB and Chebyshev solvers; the
 coupled-Newton family is the reading of the Newton iterations):
 
 * coupled Newton (both correction degrees) and Newton-DB, residual-checked
-  (tol 1e-5, cap 40): against the exact root of the same fp32 matrix,
-  2e-3 relative Frobenius at kappa <= 1e4, and at kappa >= 1e6 the
-  conditioning floor max(2e-3, 2 F) (tests/parity.py: no fp32-input method can
-  do better than the root's own sensitivity to rounding its input, or than
-  single-precision LAPACK with the same damping);
+  (tol 1e-5, cap 40): against the exact root of the same fp32 matrix at the
+  gate max(2e-3, 2 F) (tests/parity.py: no fp32-input method can do better
+  than the root's own sensitivity to rounding its input, or than
+  single-precision LAPACK with the same damping; the gate is the plain 2e-3
+  wherever that floor is below 1e-3, which holds at kappa <= 1e4 except for
+  p = 2 at n = 1024, where the solvers' damping 2^-24 ||A||_F moves the
+  smallest eigenvalue 1e-4 by 0.45%).  At kappa = 1e8 the fp32 matrix itself
+  is not positive definite (its smallest eigenvalues 1e-8 sit below the
+  rounding of its largest, 1), so its undamped root does not exist; the
+  reference there is the exact root of the matrix with the damping the
+  solvers apply, eps_eff = 2^-24 ||A||_F, gated at its own floor;
 * Chebyshev, degree 16 and 32, interval [0.999/kappa, 1] in A's units:
   polynomial parity, against the float64 Clenshaw evaluation of the same
   interpolant on the same damped matrix (the GPU damps with
@@ -59,8 +65,9 @@ def test_sweep_case(sb, batch, n, kappa):
     for p in (2, 4):
         for s in samples:
             A64 = A32[s].astype(np.float64)
-            exact[p, s] = oracle.inverse_root(A64, p, 0.0)
-            gates[p, s] = BASE_TOL if kappa <= 1e4 else root_gate(A64, p, 0.0)
+            e_ref = 0.0 if np.linalg.eigvalsh(A64)[0] > 0.0 else effective_eps(A64, 0.0)
+            exact[p, s] = oracle.inverse_root(A64, p, e_ref)
+            gates[p, s] = root_gate(A64, p, e_ref)
         for name, solver, degree in SOLVERS:
             if solver == 2:
                 lo = 0.999 / kappa

@@ -85,3 +85,44 @@ def test_roots_use_the_order_dependent_power():
     for H, X in zip(t.H, t.X):
         n = H.shape[0]
         assert np.allclose(np.linalg.matrix_power(X, 6) @ (H + 1e-2 * np.eye(n)), np.eye(n), atol=1e-9)
+
+
+def test_diagonal_variant_equals_full_when_the_statistic_is_diagonal():
+    """A gradient whose mode-0 fibres are mutually orthogonal has a diagonal
+    mode-0 statistic, so the diagonal variant of that mode (a threshold below
+    its length) must give the full variant's update exactly."""
+    from oracle.tensor import TensorShampooOracle
+    rng = np.random.default_rng(11)
+    n0, n1, n2 = 6, 4, 5
+    seq = []
+    for _ in range(3):
+        Q = np.linalg.qr(rng.standard_normal((n1 * n2, n0)))[0]     # orthonormal columns
+        seq.append((Q * rng.uniform(0.5, 2.0, size=n0)).T.reshape(n0, n1, n2))
+    full = TensorShampooOracle((n0, n1, n2), 0.9, 1e-3, 1e-2)
+    diag = TensorShampooOracle((n0, n1, n2), 0.9, 1e-3, 1e-2, diag_threshold=5)   # only mode 0 (6 > 5)
+    assert diag.diag == [True, False, False]
+    for G in seq:
+        np.testing.assert_allclose(diag.step(G), full.step(G), atol=1e-12)
+
+
+def test_diagonal_variant_rank_one_closed_form():
+    """G = a (x) b (x) c: the diagonal statistics are a^2 |b|^2 |c|^2 etc., so
+    with every mode diagonal the first step is
+    G_ijk * prod over modes of (stat + eps)^{-1/6}."""
+    from oracle.tensor import TensorShampooOracle
+    rng = np.random.default_rng(12)
+    a, b, c = rng.standard_normal(5), rng.standard_normal(7), rng.standard_normal(3)
+    G = np.einsum("i,j,k->ijk", a, b, c)
+    eps = 1e-2
+    o = TensorShampooOracle(G.shape, 1.0, eps, 1.0, diag_threshold=0)
+    P = o.step(G)
+    na, nb, nc = a @ a, b @ b, c @ c
+    da = (a ** 2 * nb * nc + eps) ** (-1 / 6)
+    db = (b ** 2 * na * nc + eps) ** (-1 / 6)
+    dc = (c ** 2 * na * nb + eps) ** (-1 / 6)
+    np.testing.assert_allclose(P, G * np.einsum("i,j,k->ijk", da, db, dc), rtol=1e-12)
+
+
+def test_diagonal_root_of_an_untouched_index_is_zero():
+    from oracle.tensor import diagonal_root
+    np.testing.assert_array_equal(diagonal_root(np.array([0.0, 16.0]), 4, 0.0), np.array([0.0, 0.5]))

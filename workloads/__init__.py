@@ -58,6 +58,7 @@ class Workload:
     cheb_lo: float = 0.0
     grad_dtype: int = DTYPE_F32
     momentum: float = 0.0
+    diag_threshold: int = 0
     steps: int = 10
     seed: int = 1234
 
