@@ -58,7 +58,12 @@ WORKLOAD_NAMES = {
     "gpt2": "gpt2_small_shapes_b512",
     "llama": "llama_1b_shapes_b1024",
     "sweep": "inverse_root_sweep",
+    "soap": "soap_4x1024sq_b256",
+    "tensor": "tensor_conv3x3_stack",
 }
+# Convolution kernels (3 x 3 x C_in x C_out) of a ResNet-style stack, for
+# order-4 tensor Shampoo: 4 stages of 4 kernels at 64 .. 512 channels.
+CONV_SHAPES = tuple((3, 3, c, c) for c in (64, 128, 256, 512) for _ in range(4))
 SWEEP_BATCH = {256: 512, 512: 128, 1024: 64}
 SOLVER_NAMES = {0: "coupled_newton", 1: "newton_db", 2: "chebyshev", 3: "coupled_newton_cubic"}
 SOLVER_IDS = {"newton": 0, "newton_db": 1, "chebyshev": 2, "newton_cubic": 3}
@@ -437,7 +442,7 @@ def run_ours(args, wl):
             "params": len(wl.shapes), "param_elems": wl.n_params, "block": wl.block, "blocks": nb,
             "roots_per_refresh": roots_per_refresh, "refresh_every": wl.refresh_every,
             "refresh_steps_timed": nref, "solver": SOLVER_NAMES[wl.solver], "root_p": wl.root_p,
-            "iters_cap": wl.iters, "tol": wl.tol, "beta": wl.beta, "eps": wl.eps,
+            "iters_cap": wl.iters, "tol": wl.tol, "beta": wl.beta, "eps": wl.eps, "momentum": wl.momentum,
             "grad_dtype": "bf16" if wl.grad_dtype == workloads.DTYPE_BF16 else "f32",
             "arithmetic": "3xTF32 tcgen05 (fp32-accurate), fp32 state",
             "l2": "256 MiB buffer written between timed steps, outside the per-step events",
@@ -644,6 +649,93 @@ def run_reference(args, wl):
     }), flush=True)
 
 
+def run_other(args):
+    """SOAP or order-4 tensor Shampoo through their C-ABI handles: W untimed
+    and K timed steps, per-step CUDA events, the L2 flushed between steps.
+    SOAP runs on the 4 x 1024^2 low-rank workload (block 256, refresh every
+    10); tensor Shampoo on a stack of 3 x 3 convolution kernels (refresh every
+    10).  Units: eigenbases (SOAP) or inverse roots (tensor) per second, with
+    ms per step beside them."""
+    import torch
+    import shampoo_family_second_b200 as sb
+    rank, world, _ = dist_env()
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    gen = torch.Generator(device=device)
+    gen.manual_seed(77 + rank)
+    if args.workload == "soap":
+        wl = workloads.workload("lowrank")
+        cfg = sb.make_config(wl.block, wl.beta, 0.0, 3e-3, refresh_every=wl.refresh_every)
+        opt = sb.Soap(wl.shapes, cfg, sb.make_soap_config(jacobi_sweeps=15, refine_iters=1))
+        shapes, every = wl.shapes, wl.refresh_every
+        per_refresh = 2 * opt.nb
+        grads = device_gradients(wl, wl.seed + 1000 * rank, min(args.ring, args.steps + args.warmup), device)
+        unit = "eigenbases/s"
+    else:
+        shapes, every = CONV_SHAPES, 10
+        cfg = sb.make_config(32, 0.999, 1e-6, 1e-3, solver=sb.SOLVER_NEWTON_CUBIC, iters=40, tol=1e-5,
+                             refresh_every=every)
+        opt = sb.TensorShampoo(shapes, cfg)
+        per_refresh = sum(len(s) for s in shapes)
+        grads = [[torch.randn(s, generator=gen, device=device) * 0.01 for s in shapes]
+                 for _ in range(min(args.ring, args.steps + args.warmup))]
+        unit = "inverse-roots/s"
+    W = [torch.zeros(s, dtype=torch.float32, device=device) for s in shapes]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for t in range(args.warmup):
+        opt.step(W, grads[t % len(grads)])
+    # the timed window starts on a refresh step
+    k0 = args.warmup
+    pad = (-k0) % every
+    for t in range(pad):
+        opt.step(W, grads[(k0 + t) % len(grads)])
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(device.index or 0)
+    clocks.start()
+    l0 = sb.launch_count()
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        opt.step(W, grads[(k0 + pad + k) % len(grads)])
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    launches = sb.launch_count() - l0
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total = sum(step_ms)
+    nref = refresh_steps(args.steps, every)
+    sb.profile_reset()
+    sb.profile_enable(True)
+    for k in range(args.steps):
+        flush.zero_()
+        opt.step(W, grads[k % len(grads)])
+    torch.cuda.synchronize()
+    g = sb.profile_read(sb.KERNEL_GEMM)
+    sb.profile_enable(False)
+    peaks, src = load_peaks()
+    pb, ps_, kind = tensor_peaks(peaks, total)
+    ach = (g.alg_flops / g.launches) / (g.total_ms / g.launches * 1e-3) / 1e12 if g.launches else 0.0
+    status = opt.status()
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": per_refresh * nref / (total * 1e-3), "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAMES[args.workload], "params": len(shapes),
+                       "param_elems": int(sum(np.prod(s) for s in shapes)), "refresh_every": every,
+                       "per_refresh": per_refresh, "refresh_steps_timed": nref,
+                       "l2": "256 MiB buffer written between timed steps, outside the per-step events"},
+            "step_ms_split": split_step_ms(step_ms, every), "device_status": int(status),
+            "gpu_launches": int(launches), "clocks": clk,
+            "roofline": {"kernel": "gemm3x_tf32_kernel", "bound": "tensor", "achieved": ach,
+                         "peak": pb if kind == "burst" else ps_, "unit": "TFLOP/s",
+                         "frac_burst": ach / pb, "frac_sustained": ach / ps_, "peak_kind": kind,
+                         "launches": g.launches, "avg_launch_ms": g.total_ms / max(g.launches, 1),
+                         "peak_basis": f"{src} bf16 {kind} x 1.1/2.25 / 3"},
+        }), flush=True)
+
+
 def run_sweep(args):
     """Inverse-root solver sweep: stacked fp32 SPD matrices Q diag(lam) Q^T
     (Haar Q, log-uniform lam with condition number kappa), one
@@ -778,6 +870,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--solver", default=None, choices=["newton", "newton_db", "chebyshev", "newton_cubic"],
                     help="inverse-root solver of the step workloads (default: the workload's own)")
+    ap.add_argument("--momentum", type=float, default=None, help="momentum ahead of the preconditioner (step workloads)")
     ap.add_argument("--sweep-n", type=int, default=512)
     ap.add_argument("--sweep-batch", type=int, default=0)
     ap.add_argument("--sweep-kappa", type=float, default=1e4)
@@ -790,6 +883,13 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload in ("soap", "tensor"):
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the SOAP and tensor workloads are timed for the "
+                              "CUDA path only; the oracle arm covers the step workloads"}))
+            return
+        run_other(args)
+        return
     if args.workload == "sweep":
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the sweep is timed for the CUDA path only; "
@@ -800,6 +900,8 @@ def main():
     over = {}
     if args.solver is not None:
         over["solver"] = SOLVER_IDS[args.solver]
+    if args.momentum is not None:
+        over["momentum"] = args.momentum
     wl = workloads.workload(args.workload, **over)
     np.random.seed(0)
     if args.impl == "reference":

@@ -316,15 +316,16 @@ SHAMPOO_API void shampoo_tensor_destroy(shampoo_tensor_handle h);
  *     first refresh), v carried over as (PL o PL) v (PR o PR)^T, P = Q_new^T Q_old.
  * The current gradient never enters its own projection (its rotation would have
  * exact zeros that fp32 turns into rounding noise, which Adam's normalisation
- * amplifies).  The bases come from eigh's method (cyclic Jacobi warm-started from
- * the previous basis, then refine_iters refinement iterations).
+ * amplifies).  The bases come from eigh_batched's method (cyclic Jacobi
+ * warm-started from the previous basis, then refine_iters orthogonalisation
+ * steps).
  * shampoo_config fields used: block, beta, lr, refresh_every, grad_dtype. */
 typedef struct {
   float beta1;            /* Adam first-moment decay, [0, 1) */
   float beta2;            /* Adam second-moment decay, [0, 1) */
   float eps;              /* Adam epsilon, > 0 */
   int32_t jacobi_sweeps;  /* eigensolver: Jacobi sweep cap per refresh, [1, 100] */
-  int32_t refine_iters;   /* eigensolver: refinement iterations per refresh, [0, 100] */
+  int32_t refine_iters;   /* eigensolver: orthogonalisation steps per refresh, [0, 100] */
 } shampoo_soap_config;
 typedef struct shampoo_soap_ctx* shampoo_soap_handle;
 SHAMPOO_API int shampoo_soap_query_sizes(const shampoo_config* cfg, const shampoo_soap_config* sc, int32_t nparams,
@@ -370,10 +371,11 @@ SHAMPOO_API int shampoo_pack_blocks(const int64_t* d_table, int32_t nblocks, int
  * method).  warm_start = 0: cyclic Jacobi with the round-robin parallel
  * ordering (Golub & Van Loan sec. 8.5) from A_i, at most jacobi_sweeps sweeps
  * (SHAMPOO_DEVFLAG_NOT_CONVERGED if the off-diagonal mass stays above 1e-5 of
- * ||A_i||_F), then refine_iters iterations of the GEMM-only refinement of
- * Ogita & Aishima (2018); warm_start = 1: d_Q holds an approximate basis X on
- * entry (e.g. the previous one): Jacobi runs on the nearly diagonal X^T A X,
- * X is rotated by its eigenvectors, then the refinement runs.
+ * ||A_i||_F); warm_start = 1: d_Q holds an approximate basis X on entry (e.g.
+ * the previous one): Jacobi runs on the nearly diagonal X^T A X and X is
+ * rotated by its eigenvectors.  Then refine_iters Newton-Schulz steps toward
+ * the nearest orthogonal matrix (Bjorck & Bowie 1971), X <- 1.5 X - 0.5 X X^T X,
+ * each squaring X's departure from orthogonality.
  *  d_A       device stack (batch, n, n), symmetrised before use; n a multiple
  *            of 32 in [32, 1024].
  *  d_Q       device stack (batch, n, n): eigenvectors as columns, in no

@@ -331,18 +331,21 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
     Builder b;
     Epilogue& eL = b.add(nb, B, h->mGs, 0, h->mGs, 0, h->stats_flops_L);
     b.L.g[0].a_exact = b.L.g[0].b_exact = g_exact;
+    b.L.g[0].sym = 1;  // symmetric: the tiles below the diagonal are mirrored below
     eL.beta = c.beta;
     eL.C = h->stats;
     eL.D = h->stats;
     eL.flags = h->d_status;
     Epilogue& eR = b.add(nb, B, h->mGt, 0, h->mGt, 0, h->stats_flops_R);
     b.L.g[1].a_exact = b.L.g[1].b_exact = g_exact;
+    b.L.g[1].sym = 1;
     eR.beta = c.beta;
     eR.C = h->stats + plain_floats(nb, B);
     eR.D = h->stats + plain_floats(nb, B);
     eR.flags = h->d_status;
     if (!refresh) add_apply1(b);
     if ((rc = b.launch(st))) return rc;
+    if ((rc = launch_mirror_lower(h->stats, 2 * nb, B, st))) return rc;
   }
   // 3. roots of all 2 nb damped statistics, every refresh_every steps
   if (refresh) {

@@ -3,21 +3,21 @@
 // eigenbasis of Shampoo's preconditioner; Substack SOAP survey: the
 // eigendecompositions are Shampoo's bottleneck).  The pages name no method;
 // two published ones are used:
-//   cold start   cyclic Jacobi with the round-robin parallel ordering
-//                (Golub & Van Loan, "Matrix Computations", sec. 8.5): each
-//                round rotates n/2 disjoint index pairs (p, q), zeroing a_pq,
-//                as the two-sided update A <- J^T A J and V <- V J; one CTA per
-//                matrix, the working copy in global memory (L2 resident);
-//   warm start   from an approximate basis X: Jacobi on the nearly diagonal
-//                X^T A X (a few sweeps), X <- X V;
-//   polishing    iterative refinement of the basis (Ogita & Aishima 2018,
-//                "Iterative refinement for symmetric eigenvalue
-//                decomposition"), GEMM only:
-//                  R = I - X^T X,  S = X^T A X,  lam_i = s_ii / (1 - r_ii),
-//                  delta = 2 (||S - diag(lam)||_F + ||A||_F ||R||_F),
-//                  E_ij = (s_ij + lam_j r_ij) / (lam_j - lam_i) if |lam_i - lam_j| > delta
-//                         else r_ij / 2,
-//                  X <- X + X E  (quadratic convergence; E_ii = r_ii / 2).
+//   eigenvectors  cyclic Jacobi with the round-robin parallel ordering
+//                 (Golub & Van Loan, "Matrix Computations", sec. 8.5): each
+//                 round rotates n/2 disjoint index pairs (p, q), zeroing a_pq,
+//                 as the two-sided update A <- J^T A J and V <- V J; one CTA per
+//                 matrix, the working copy in global memory (L2 resident).  A
+//                 warm start from an approximate basis X runs Jacobi on the
+//                 nearly diagonal X^T A X (a few sweeps) and takes X V;
+//   orthogonality Newton-Schulz steps toward the nearest orthogonal matrix
+//                 (Bjorck & Bowie 1971): X <- X + X (I - X^T X) / 2 =
+//                 1.5 X - 0.5 X (X^T X), GEMM only.  The products of a warm start
+//                 carry 3xTF32 rounding into X's orthogonality; each step
+//                 squares that error.  (An eigenvector-correcting refinement
+//                 such as Ogita & Aishima's divides rounding in X^T A X by
+//                 eigenvalue gaps and, evaluated in fp32, degrades an
+//                 fp32-accurate basis; it is not used.)
 // Matrices of a ragged block use their leading `valid` x `valid` part; the
 // rest of Q is the identity.
 #include <algorithm>
@@ -172,70 +172,9 @@ __global__ void transpose_kernel(const float* __restrict__ X, int n, float* __re
         t[threadIdx.x][threadIdx.y + 8 * k];
 }
 
-// Refinement, phase 1 (one CTA per matrix): lam_i = s_ii / (1 - r_ii) and
-// delta = 2 (||S - diag(lam)||_F + ||A||_F ||R||_F) over the valid part.
-__global__ void refine_stats_kernel(const float* __restrict__ Rm, const float* __restrict__ S,
-                                    const float* __restrict__ A, int n, const int* __restrict__ valid,
-                                    float* __restrict__ lam, float* __restrict__ delta) {
-  __shared__ double red[3][32];
-  const int i = blockIdx.x, tid = threadIdx.x;
-  const int m = valid ? valid[i] : n;
-  const size_t nn = static_cast<size_t>(n) * n;
-  for (int j = tid; j < n; j += blockDim.x) {
-    const float r = Rm[i * nn + static_cast<size_t>(j) * n + j], s = S[i * nn + static_cast<size_t>(j) * n + j];
-    lam[static_cast<size_t>(i) * n + j] = j < m ? s / (1.f - r) : 0.f;
-  }
-  __syncthreads();
-  double so = 0.0, sa = 0.0, sr = 0.0;
-  for (size_t e = tid; e < static_cast<size_t>(m) * m; e += blockDim.x) {
-    const int r = static_cast<int>(e / m), c = static_cast<int>(e % m);
-    const size_t idx = i * nn + static_cast<size_t>(r) * n + c;
-    const double s = S[idx] - (r == c ? lam[static_cast<size_t>(i) * n + r] : 0.f);
-    so += s * s;
-    sa += static_cast<double>(A[idx]) * A[idx];
-    sr += static_cast<double>(Rm[idx]) * Rm[idx];
-  }
-  for (int o = 16; o > 0; o >>= 1) {
-    so += __shfl_xor_sync(0xffffffffu, so, o);
-    sa += __shfl_xor_sync(0xffffffffu, sa, o);
-    sr += __shfl_xor_sync(0xffffffffu, sr, o);
-  }
-  if ((tid & 31) == 0) red[0][tid >> 5] = so, red[1][tid >> 5] = sa, red[2][tid >> 5] = sr;
-  __syncthreads();
-  if (tid == 0) {
-    double a0 = 0, a1 = 0, a2 = 0;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) a0 += red[0][w], a1 += red[1][w], a2 += red[2][w];
-    delta[i] = static_cast<float>(2.0 * (sqrt(a0) + sqrt(a1) * sqrt(a2)));
-  }
-}
-
-// Refinement, phase 2 (elementwise): E on the valid part, 0 on the padding.
-__global__ void refine_update_kernel(const float* __restrict__ Rm, const float* __restrict__ S, int n,
-                                     const int* __restrict__ valid, const float* __restrict__ lam,
-                                     const float* __restrict__ delta, float* __restrict__ E) {
-  pdl_launch_dependents();
-  const int i = blockIdx.z;
-  const int r = blockIdx.y * 8 + threadIdx.y;
-  const int c = blockIdx.x * 32 + threadIdx.x;
-  const int m = valid ? valid[i] : n;
-  const size_t nn = static_cast<size_t>(n) * n;
-  const size_t idx = i * nn + static_cast<size_t>(r) * n + c;
-  float e = 0.f;
-  if (r < m && c < m) {
-    const float rr = Rm[idx];
-    if (r == c) {
-      e = 0.5f * rr;
-    } else {
-      const float li = lam[static_cast<size_t>(i) * n + r], lj = lam[static_cast<size_t>(i) * n + c];
-      e = (fabsf(li - lj) > delta[i]) ? (S[idx] + lj * rr) / (lj - li) : 0.5f * rr;
-    }
-  }
-  E[idx] = e;
-}
-
 }  // namespace
 
-size_t eig_scratch_per_matrix(int n) { return static_cast<size_t>(5) * n * n * 4 + 16 + 4 * static_cast<size_t>(n); }
+size_t eig_scratch_per_matrix(int n) { return static_cast<size_t>(5) * n * n * 4; }
 
 int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const int* valid, int warm_start,
              int jacobi_sweeps, int refine_iters, void* scratch, size_t scratch_bytes, int* flags, cudaStream_t st) {
@@ -253,12 +192,10 @@ int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const i
     const int* vi = valid ? valid + off : nullptr;
     float* base = static_cast<float*>(scratch);
     float* Xt = base;            // X^T
-    float* Rm = Xt + cb * nn;    // R = I - X^T X
-    float* T = Rm + cb * nn;     // A X
-    float* S = T + cb * nn;      // X^T A X
-    float* E = S + cb * nn;
-    float* lamw = E + cb * nn;   // cb x n
-    float* delta = lamw + cb * n;
+    float* Rm = Xt + cb * nn;    // the Jacobi working copy
+    float* T = Rm + cb * nn;     // A X, then the new basis
+    float* S = T + cb * nn;      // X^T A X, then X^T X
+    float* E = S + cb * nn;      // Jacobi's rotation of X^T A X
     const double f1 = 2.0 * n * static_cast<double>(n) * n;
     const int cbi = static_cast<int>(cb);
     StackMaps mA, mX, mXt, mT, mE;
@@ -316,50 +253,28 @@ int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const i
         count_launch();
         if ((rc = check_cuda(cudaGetLastError(), "transpose_kernel"))) return rc;
       }
-      {  // R = I - X^T X (= I - Xt Xt^T) and T = A X, one launch
+      {  // S = X^T X (= Xt Xt^T)
         Builder b;
-        Epilogue& er = b.add(cbi, n, mXt, 0, mXt, 0, f1, B_TRANSPOSED);
-        er.alpha = -1.f;
-        er.gamma = 1.f;
-        er.D = Rm;
-        er.flags = flags;
-        Epilogue& et = b.add(cbi, n, mA, 0, mX, 0, f1, B_MN_MAJOR);
-        et.D = T;
-        et.flags = flags;
-        if ((rc = b.launch(st))) return rc;
-      }
-      {  // S = X^T (A X)
-        Builder b;
-        Epilogue& e = b.add(cbi, n, mXt, 0, mT, 0, f1, B_MN_MAJOR);
+        Epilogue& e = b.add(cbi, n, mXt, 0, mXt, 0, f1, B_TRANSPOSED);
         e.D = S;
         e.flags = flags;
         if ((rc = b.launch(st))) return rc;
       }
-      {
-        ProfScope ps(K_CHECK, st, 0.0, 12.0 * cb * nn);
-        refine_stats_kernel<<<static_cast<unsigned>(cb), 512, 0, st>>>(Rm, S, Ai, n, vi, lamw, delta);
-        count_launch();
-        if ((rc = check_cuda(cudaGetLastError(), "refine_stats_kernel"))) return rc;
-        refine_update_kernel<<<dim3(n / 32, n / 8, static_cast<unsigned>(cb)), dim3(32, 8), 0, st>>>(
-            Rm, S, n, vi, lamw, delta, E);
-        count_launch();
-        if ((rc = check_cuda(cudaGetLastError(), "refine_update_kernel"))) return rc;
-      }
-      {  // X <- X + X E
+      StackMaps mS;
+      if ((rc = make_stack_maps(mS, S, cb, n))) return rc;
+      {  // X <- 1.5 X - 0.5 X (X^T X), into T, then back to Q
         Builder b;
-        Epilogue& e = b.add(cbi, n, mX, 0, mE, 0, f1, B_MN_MAJOR);
+        Epilogue& e = b.add(cbi, n, mX, 0, mS, 0, f1, B_MN_MAJOR);
+        e.alpha = -0.5f;
         e.C = Qi;
-        e.beta = 1.f;
-        e.D = Rm;  // R is no longer needed: X + X E lands there, then moves to Q below
+        e.beta = 1.5f;
+        e.D = T;
         e.flags = flags;
         if ((rc = b.launch(st))) return rc;
       }
-      if ((rc = check_cuda(cudaMemcpyAsync(Qi, Rm, cb * nn * 4, cudaMemcpyDeviceToDevice, st), "refined basis")))
+      if ((rc = check_cuda(cudaMemcpyAsync(Qi, T, cb * nn * 4, cudaMemcpyDeviceToDevice, st), "orthogonalised basis")))
         return rc;
     }
-    if (li && refine_iters > 0 &&
-        (rc = check_cuda(cudaMemcpyAsync(li, lamw, cb * n * 4, cudaMemcpyDeviceToDevice, st), "eigenvalues")))
-      return rc;
   }
   return 0;
 }

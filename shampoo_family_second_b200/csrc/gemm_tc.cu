@@ -34,6 +34,7 @@
 // need them.  Every wait is bounded (2 s); a time-out raises
 // DEV_FLAG_TIMEOUT, tells the other roles of the CTA to stop waiting, and the
 // CTA unwinds, releasing its TMEM.
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 
@@ -85,12 +86,27 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmLaunch& L, int tile) {
   while (gi + 1 < L.ngroups && tile >= L.g[gi + 1].cta_begin) ++gi;
   const GemmGroup& G = L.g[gi];
   const int local = tile - G.cta_begin;
-  const int tiles = G.tiles_m * G.tiles_n;
+  const int tiles = G.tiles_per;
   c.gi = gi;
   c.mat = local / tiles;
-  const int t = local - c.mat * tiles;
-  c.tm = t / G.tiles_n;
-  c.tn = t - c.tm * G.tiles_n;
+  int t = local - c.mat * tiles;
+  if (G.sym) {
+    // Symmetric result: tile column tn keeps the tile rows that reach the
+    // diagonal or above, tm * BM < (tn + 1) * BN, i.e. tm < 2 tn + 2.
+    int tn = 0;
+#pragma unroll 1
+    while (true) {
+      const int cnt = min(2 * tn + 2, G.tiles_m);
+      if (t < cnt) break;
+      t -= cnt;
+      ++tn;
+    }
+    c.tm = t;
+    c.tn = tn;
+  } else {
+    c.tm = t / G.tiles_n;
+    c.tn = t - c.tm * G.tiles_n;
+  }
   c.skip = G.ep.skip && G.ep.skip[c.mat];
   return c;
 }
@@ -197,10 +213,19 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
       }
       if (wbase && gr < wr) {
         float* wrow = wbase + static_cast<size_t>(gr) * wld + gc;
-        if (gc + 0 < wc) wrow[0] -= E.lr * v.x;
-        if (gc + 1 < wc) wrow[1] -= E.lr * v.y;
-        if (gc + 2 < wc) wrow[2] -= E.lr * v.z;
-        if (gc + 3 < wc) wrow[3] -= E.lr * v.w;
+        if (gc + 3 < wc && (reinterpret_cast<uintptr_t>(wrow) & 15) == 0) {
+          float4 w4 = *reinterpret_cast<float4*>(wrow);  // one 16-byte read-modify-write
+          w4.x -= E.lr * v.x;
+          w4.y -= E.lr * v.y;
+          w4.z -= E.lr * v.z;
+          w4.w -= E.lr * v.w;
+          *reinterpret_cast<float4*>(wrow) = w4;
+        } else {
+          if (gc + 0 < wc) wrow[0] -= E.lr * v.x;
+          if (gc + 1 < wc) wrow[1] -= E.lr * v.y;
+          if (gc + 2 < wc) wrow[2] -= E.lr * v.z;
+          if (gc + 3 < wc) wrow[3] -= E.lr * v.w;
+        }
       }
     }
   }
@@ -485,7 +510,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (__any_sync(0xffffffffu, nonfinite) && lane == 0) raise_flag(G.ep.flags, DEV_FLAG_NONFINITE);
       if (L.profile && ew == 0 && lane == 0 && prof_flops)
-        atomicAdd(&prof_flops[L.prof_slot], G.flops_per_matrix / (G.tiles_m * G.tiles_n));
+        atomicAdd(&prof_flops[L.prof_slot], G.flops_per_matrix / G.tiles_per);
     }
   }
 
@@ -630,8 +655,14 @@ int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
     GemmGroup& g = L.g[i];
     g.tiles_m = (g.m + BM - 1) / BM;
     g.tiles_n = (g.n + BN - 1) / BN;
+    if (g.sym && g.m != g.n) return set_error(-1, "a symmetric GEMM group must be square");
+    g.tiles_per = g.tiles_m * g.tiles_n;
+    if (g.sym) {
+      g.tiles_per = 0;
+      for (int tn = 0; tn < g.tiles_n; ++tn) g.tiles_per += std::min(2 * tn + 2, g.tiles_m);
+    }
     g.cta_begin = static_cast<int>(total);
-    total += static_cast<int64_t>(g.batch) * g.tiles_m * g.tiles_n;
+    total += static_cast<int64_t>(g.batch) * g.tiles_per;
     flops += g.flops_per_matrix * g.batch;
   }
   if (total == 0) return 0;

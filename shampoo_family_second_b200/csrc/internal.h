@@ -60,6 +60,9 @@ struct GemmGroup {
   int a_exact, b_exact;  // 1: every value of the operand is exact in tf32 (e.g. widened bf16), so its
                          // lo part is zero: the MMAs with that lo part are skipped and its tiles are
                          // not split
+  int sym;               // 1: D is symmetric (square, e.g. G G^T): only the tiles that reach the
+                         // diagonal or above are computed; launch_mirror_lower fills the rest
+  int tiles_per;         // tiles computed per matrix (filled by launch_gemm)
   int tiles_m, tiles_n, cta_begin;  // filled by launch_gemm (cta_begin: first tile of the group)
   double flops_per_matrix;          // algorithmic flops (profiling only)
   Epilogue ep;
@@ -209,6 +212,9 @@ int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, fl
                       float lo, const float* s, float* coef, float* sc, float* Xt, float* bd, float* bd1,
                       cudaStream_t st);
 int launch_fill_iters(int* iters, int64_t batch, int value, cudaStream_t st);
+// After a GEMM group with sym = 1: copies the transpose of the computed upper
+// part into the 32 x 32 blocks of the tiles it skipped (wholly below the diagonal).
+int launch_mirror_lower(float* D, int64_t batch, int n, cudaStream_t st);
 
 // Inverse-root solver (solver.cu) ---------------------------------------------
 struct RootJob {

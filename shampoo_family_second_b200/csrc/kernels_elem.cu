@@ -489,6 +489,27 @@ __global__ void cheb_prologue_kernel(const float* __restrict__ A, int n, const i
   }
 }
 
+// Lower blocks of a symmetric result whose GEMM skipped the tiles wholly below
+// the diagonal (tile row tm >= 2 tn + 2 of the 128 x 256 tiling): block (bi, bj)
+// of 32 x 32 takes the transpose of block (bj, bi), which the GEMM computed.
+// grid (n/32, n/32, batch), block (32, 8).
+__global__ void mirror_lower_kernel(float* __restrict__ D, int n) {
+  pdl_launch_dependents();
+  const int i = blockIdx.z, bi = blockIdx.y, bj = blockIdx.x;
+  const int tm = bi / (kTileM / 32), tn = bj / (kTileN / 32);
+  if (tm < 2 * tn + 2) return;  // computed by the GEMM
+  __shared__ float t[32][33];
+  const size_t nn = static_cast<size_t>(n) * n;
+  float* d = D + i * nn;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    t[threadIdx.y + 8 * k][threadIdx.x] = d[static_cast<size_t>(bj * 32 + threadIdx.y + 8 * k) * n + bi * 32 + threadIdx.x];
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    d[static_cast<size_t>(bi * 32 + threadIdx.y + 8 * k) * n + bj * 32 + threadIdx.x] = t[threadIdx.x][threadIdx.y + 8 * k];
+}
+
 __global__ void fill_int_kernel(int* p, int64_t count, int value) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i < count) p[i] = value;
@@ -584,6 +605,15 @@ int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, fl
   cheb_prologue_kernel<<<grid, block, 0, st>>>(A, n, valid, eps, s, coef, degree, Xt, bd, bd1);
   count_launch();
   return check_cuda(cudaGetLastError(), "cheb_prologue_kernel");
+}
+
+int launch_mirror_lower(float* D, int64_t batch, int n, cudaStream_t st) {
+  if (batch == 0 || n <= kTileN) return 0;  // one tile column: every tile is computed
+  ProfScope ps(K_FINALIZE, st, 0.0, 8.0 * batch * n * double(n) * 0.375);
+  dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
+  mirror_lower_kernel<<<grid, block, 0, st>>>(D, n);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "mirror_lower_kernel");
 }
 
 int launch_fill_iters(int* iters, int64_t batch, int value, cudaStream_t st) {

@@ -13,8 +13,9 @@
 //   4. back      W <- W - lr QL N' QR^T (the second product's epilogue updates W)
 //   5. stats     L <- beta L + G G^T, R <- beta R + G^T G
 //   6. refresh   if t % refresh_every == 0: new bases from L and R (batched
-//                eigensolver, warm-started from the current ones; the identity
-//                before the first refresh), and the second moment carried over,
+//                Jacobi, warm-started from the current ones, the identity before
+//                the first refresh; then orthogonalisation steps), and the
+//                second moment carried over,
 //                v <- (PL o PL) v (PR o PR)^T with P = Q_new^T Q_old.
 // The basis of a step is built from statistics without that step's gradient:
 // the current gradient never enters its own projection, whose exact zeros
@@ -370,17 +371,20 @@ int shampoo_soap_step(shampoo_soap_handle h, float* const* d_weights, const void
     Builder b;
     Epilogue& eL = b.add(nb, B, h->mGs, 0, h->mGs, 0, h->fl);
     b.L.g[0].a_exact = b.L.g[0].b_exact = g_exact;
+    b.L.g[0].sym = 1;
     eL.beta = c.beta;
     eL.C = h->stats;
     eL.D = h->stats;
     eL.flags = h->d_status;
     Epilogue& eR = b.add(nb, B, h->mGt, 0, h->mGt, 0, h->fr);
     b.L.g[1].a_exact = b.L.g[1].b_exact = g_exact;
+    b.L.g[1].sym = 1;
     eR.beta = c.beta;
     eR.C = h->stats + one;
     eR.D = h->stats + one;
     eR.flags = h->d_status;
     if ((rc = b.launch(st))) return rc;
+    if ((rc = launch_mirror_lower(h->stats, 2 * nb, B, st))) return rc;
   }
   // 6. refresh: new bases, the second moment carried over
   if (h->step % c.refresh_every == 0) {

@@ -471,12 +471,15 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
       Epilogue& e = b.add_rect(1, m.npad, m.npad, m.Kpad, um[i], 0, um[i], 0, 2.0 * m.n * double(m.n) * m.K,
                                B_TRANSPOSED);
       b.L.g[b.L.ngroups - 1].a_exact = b.L.g[b.L.ngroups - 1].b_exact = g_exact;
+      b.L.g[b.L.ngroups - 1].sym = 1;
       e.beta = c.beta;
       e.C = hptr(m);
       e.D = hptr(m);
       e.flags = h->d_status;
     }
     if (b.L.ngroups > 0 && (rc = b.launch(st))) return rc;
+    for (int i = 0; i < pr.k; ++i)
+      if (!pr.modes[i].diag && (rc = launch_mirror_lower(hptr(pr.modes[i]), 1, pr.modes[i].npad, st))) return rc;
   }
   // 3. roots X = (H + eps I)^{-1/(2k)}, batched per (npad, k)
   if (refresh) {

@@ -3,10 +3,10 @@
 Eigenvectors are unique only up to sign (and within clusters of equal
 eigenvalues), so the checks are on what is unique: the eigenvalues (against
 numpy's float64 eigh of the same fp32 matrix), and that Q is orthogonal and
-diagonalises A.  Cold start: cyclic Jacobi, then the GEMM-only refinement of
-Ogita & Aishima (2018).  Warm start from a perturbed exact basis: Jacobi on the
-nearly diagonal Q^T A Q, the rotated basis, then refinement; repeated calls
-stay at the fp32 floor.
+diagonalises A.  Cold start: cyclic Jacobi, then Newton-Schulz
+orthogonalisation steps.  Warm start from a perturbed exact basis: Jacobi on
+the nearly diagonal Q^T A Q, the rotated basis, then orthogonalisation;
+repeated calls stay at the fp32 floor.
 """
 import numpy as np
 import pytest
@@ -84,3 +84,18 @@ def test_warm_start_from_a_nearby_basis(sb):
         errs.append(max(checks(A32[b], Qh[b], lam.cpu().numpy()[b])[1] for b in range(2)))
     assert errs[1] < 0.1 * errs[0] or errs[1] < TOL, errs
     assert errs[-1] < TOL, errs
+
+
+def test_orthogonalisation_steps_do_not_degrade_the_basis(sb):
+    """Newton-Schulz orthogonalisation keeps an fp32-accurate Jacobi basis at
+    the fp32 floor (no step may make it worse than 2x the Jacobi result or
+    5e-6)."""
+    A32 = workloads.spd_batch(2, 256, 1e4, seed=40).astype(np.float32)
+    A = torch.from_numpy(A32).cuda()
+    res = []
+    for k in (0, 1, 2):
+        Q, lam, st = sb.eigh_batched(A, jacobi_sweeps=20, refine_iters=k)
+        torch.cuda.synchronize()
+        Qh, lh = Q.cpu().numpy(), lam.cpu().numpy()
+        res.append(max(checks(A32[b], Qh[b], lh[b])[0] for b in range(2)))
+    assert res[1] <= max(2 * res[0], 5e-6) and res[2] <= max(2 * res[0], 5e-6), res

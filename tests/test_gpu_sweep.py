@@ -17,10 +17,11 @@ coupled-Newton family is the reading of the Newton iterations):
   wherever that floor is below 1e-3, which holds at kappa <= 1e4 except for
   p = 2 at n = 1024, where the solvers' damping 2^-24 ||A||_F moves the
   smallest eigenvalue 1e-4 by 0.45%).  At kappa = 1e8 the fp32 matrix itself
-  is not positive definite (its smallest eigenvalues 1e-8 sit below the
-  rounding of its largest, 1), so its undamped root does not exist; the
-  reference there is the exact root of the matrix with the damping the
-  solvers apply, eps_eff = 2^-24 ||A||_F, gated at its own floor;
+  is not positive definite beyond its own rounding (its smallest eigenvalues
+  1e-8 sit below 4 u ||A||_F), so its undamped root is undefined or set by
+  rounding alone; the reference there is the exact root of the matrix with
+  the damping the solvers apply, eps_eff = 2^-24 ||A||_F, gated at its own
+  floor;
 * Chebyshev, degree 16 and 32, interval [0.999/kappa, 1] in A's units:
   polynomial parity, against the float64 Clenshaw evaluation of the same
   interpolant on the same damped matrix (the GPU damps with
@@ -65,9 +66,13 @@ def test_sweep_case(sb, batch, n, kappa):
     for p in (2, 4):
         for s in samples:
             A64 = A32[s].astype(np.float64)
-            e_ref = 0.0 if np.linalg.eigvalsh(A64)[0] > 0.0 else effective_eps(A64, 0.0)
+            # the undamped root where the fp32 matrix is positive definite beyond its own
+            # rounding (smallest eigenvalue above 4 u ||A||_F), else the damped one (R21)
+            lam_min = np.linalg.eigvalsh(A64)[0]
+            e_ref = 0.0 if lam_min > 4 * 2.0 ** -24 * np.linalg.norm(A64) else effective_eps(A64, 0.0)
             exact[p, s] = oracle.inverse_root(A64, p, e_ref)
             gates[p, s] = root_gate(A64, p, e_ref)
+            assert np.isfinite(gates[p, s]) and np.all(np.isfinite(exact[p, s]))
         for name, solver, degree in SOLVERS:
             if solver == 2:
                 lo = 0.999 / kappa
