@@ -84,9 +84,9 @@ int build_table(int B, int32_t nparams, const int64_t* rows, const int64_t* cols
 // State layout (bytes, each part 256-aligned):
 //   status word | block table (nb x 5 int32) | valid extents (2nb int32: r of L_b, c of R_b)
 //   | wrows (nb) | wcols (nb) | statistics (2nb, B, B) | roots (2nb, B, B)
-//   | momentum (nb, B, B; only with momentum > 0)
+//   | momentum (nb, B, B; only with momentum > 0) | power flag | power iterates (2nb, B)
 struct StateLayout {
-  size_t status, table, valid, wrows, wcols, stats, roots, mom, total;
+  size_t status, table, valid, wrows, wcols, stats, roots, mom, pflag, pvec, total;
 };
 StateLayout state_layout(int nb, int B, bool momentum) {
   StateLayout s;
@@ -100,6 +100,8 @@ StateLayout state_layout(int nb, int B, bool momentum) {
   s.roots = o, o += al(plain_floats(2 * nb, B) * 4);
   s.mom = o;
   if (momentum) o += al(plain_floats(nb, B) * 4);
+  s.pflag = o, o += al(4);
+  s.pvec = o, o += al(size_t(2) * nb * B * 4);
   s.total = o;
   return s;
 }
@@ -262,6 +264,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
       (rc = check_cuda(cudaMemsetAsync(h->stats, 0, plain_floats(2 * nb, B) * 4, st), "zero statistics")) ||
       (rc = check_cuda(cudaMemsetAsync(h->roots, 0, plain_floats(2 * nb, B) * 4, st), "zero roots")) ||
       (h->mom && (rc = check_cuda(cudaMemsetAsync(h->mom, 0, plain_floats(nb, B) * 4, st), "zero momentum"))) ||
+      (rc = check_cuda(cudaMemsetAsync(h->state + sl.pflag, 0, sl.total - sl.pflag, st), "zero power store")) ||
       (rc = check_cuda(cudaStreamSynchronize(st), "init sync"))) {
     delete h;
     return rc;
@@ -364,6 +367,8 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
     job.X = h->roots;
     job.iters_used = nullptr;
     job.flags = h->d_status;
+    job.power_vec = reinterpret_cast<float*>(h->state + h->sl.pvec);
+    job.power_warm = reinterpret_cast<int*>(h->state + h->sl.pflag);
     if ((rc = run_inverse_roots(job, h->scratch + h->xl.root, h->xl.root_bytes, st))) return rc;
     // 4a. apply, first product: T = XL G (with the fresh roots)
     Builder b;

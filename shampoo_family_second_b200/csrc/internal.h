@@ -184,11 +184,17 @@ int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, flo
 //       1 = Newton-DB (Y0 = A', T0 = (3I - A')/2, Z1 = T0)
 // Coupled-Newton scale: s = min(||A + eps I||_F, 1.25 x power-iteration estimate
 // of the largest eigenvalue), sc = s^{-1/p}, sf = ||A + eps I||_F.
+// vec (nullable): per-matrix store of the power iterate (batch x n floats);
+// with *warm != 0 the iteration starts from it for warm_iters steps (the root
+// prologue of the refresh's last chunk sets *warm).
 int launch_spectral_scale(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int iters,
-                          float* s, float* sc, float* sf, cudaStream_t st);
-// sf (nullable: s) sets the damping floor eps_eff = max(eps, 2^-24 sf).
+                          float* s, float* sc, float* sf, float* vec, const int* warm, int warm_iters,
+                          cudaStream_t st);
+// sf (nullable: s) sets the damping floor eps_eff = max(eps, 2^-24 sf);
+// set_flag (nullable) is set to 1 (a power-iterate store is filled).
 int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const int* valid, float eps, int p,
-                         const float* s, const float* sf, float* out0, float* out1, float* out2, cudaStream_t st);
+                         const float* s, const float* sf, float* out0, float* out1, float* out2, int* set_flag,
+                         cudaStream_t st);
 // Second Newton-DB stage: Y0' = Y_par(i) (parity from iters), T0 = (3I - Y0')/2, Z1 = T0.
 int launch_db_stage2_prologue(const float* Y0, const float* Y1, const int* iters, int64_t batch, int n,
                               float* Ynew0, float* T, float* Z1, cudaStream_t st);
@@ -228,6 +234,8 @@ struct RootJob {
   int* flags;        // device status word (nullable)
   int plain_launches = 0;  // 1: never build or run a CUDA graph loop (residual-checked loops are
                            // issued as plain launches up to the cap)
+  float* power_vec = nullptr;  // coupled Newton's scale: per-matrix power-iterate store (batch x n), or NULL
+  int* power_warm = nullptr;   // device flag: power_vec holds the previous refresh's iterates
 };
 // inv_root_batched with a switch for plain launches (shared by the public
 // entry points of api.cu and noalloc.cu).

@@ -170,10 +170,18 @@ __global__ void frob_norm_kernel(const float* __restrict__ A, int n, const int* 
 // largest scaled eigenvalue lands near 0.8 instead of lam_max / sf (0.1 to 0.3
 // on Wishart-like statistics), which saves iterations.  sc_i = s_i^{-1/p}.
 // One CTA of 512 threads per matrix; x and (A + eps I) x live in shared memory.
+// With a vector store (vec != NULL) the last normalised iterate of each matrix
+// is kept there, and when *warm != 0 the next call starts from it and runs
+// warm_iters steps instead of iters: statistics change little between
+// refreshes, so the previous dominant direction is already close.  The store
+// and its flag live in the caller's state, so a restored state restarts the
+// same way.
 __global__ void __launch_bounds__(512) spectral_scale_kernel(const float* __restrict__ A, int n,
                                                              const int* __restrict__ valid, float eps, double inv_p,
                                                              int iters, float* __restrict__ s,
-                                                             float* __restrict__ sc, float* __restrict__ sf) {
+                                                             float* __restrict__ sc, float* __restrict__ sf,
+                                                             float* __restrict__ vec, const int* __restrict__ warm,
+                                                             int warm_iters) {
   extern __shared__ float xy[];  // x[n], y[n]
   __shared__ double red[16];
   __shared__ double bcast;
@@ -208,18 +216,30 @@ __global__ void __launch_bounds__(512) spectral_scale_kernel(const float* __rest
   }
   double fro = sqrt(block_sum(acc));
   if (!(fro > 0.0)) fro = 1.0;  // all-zero matrix with eps = 0: keep the scale finite
-  // start vector: positive, with a fixed irregular pattern
+  // start vector: the stored one (warm), else positive with a fixed irregular pattern
+  const bool from_store = vec && warm && *warm;
+  float* xs = vec ? vec + static_cast<size_t>(i) * n : nullptr;
   double nx = 0.0;
   for (int j = tid; j < v; j += 512) {
-    const float t = 1.f + 0.3f * static_cast<float>((j * 7919) % 17) / 17.f;
+    const float t = from_store ? xs[j] : 1.f + 0.3f * static_cast<float>((j * 7919) % 17) / 17.f;
     x[j] = t;
     nx += static_cast<double>(t) * t;
   }
   nx = sqrt(block_sum(nx));
+  if (!(nx > 0.0)) {  // a stored zero vector (all-zero statistics): the fixed start
+    nx = 0.0;
+    for (int j = tid; j < v; j += 512) {
+      const float t = 1.f + 0.3f * static_cast<float>((j * 7919) % 17) / 17.f;
+      x[j] = t;
+      nx += static_cast<double>(t) * t;
+    }
+    nx = sqrt(block_sum(nx));
+  }
   for (int j = tid; j < v; j += 512) x[j] = static_cast<float>(x[j] / nx);
   __syncthreads();
   double lam = 0.0;
-  for (int k = 0; k < iters; ++k) {
+  const int steps = from_store ? warm_iters : iters;
+  for (int k = 0; k < steps; ++k) {
     double part = 0.0;
     for (int r = warp; r < v; r += 16) {
       const float* row = a + static_cast<size_t>(r) * n;
@@ -237,6 +257,8 @@ __global__ void __launch_bounds__(512) spectral_scale_kernel(const float* __rest
     for (int j = tid; j < v; j += 512) x[j] = static_cast<float>(y[j] / lam);
     __syncthreads();
   }
+  if (xs)
+    for (int j = tid; j < v; j += 512) xs[j] = x[j];
   if (tid == 0) {
     double sv = fro;
     if (lam > 0.0 && 1.25 * lam < fro) sv = 1.25 * lam;
@@ -245,6 +267,7 @@ __global__ void __launch_bounds__(512) spectral_scale_kernel(const float* __rest
     sc[i] = static_cast<float>(pow(sv, -inv_p));
   }
 }
+
 
 // Damping actually applied by the solvers: eps_eff = max(eps, u s) with
 // u = 2^-24 and s = ||A + eps I||_F.  Statistics accumulated in fp32 carry
@@ -264,10 +287,15 @@ __device__ __forceinline__ float effective_eps(float eps, float s) { return fmax
 //                           out2 = Z1 = T0.
 // grid (n/32, n/32, batch), block (32, 8).
 // ---------------------------------------------------------------------------
+// set_flag (nullable): written 1 by one thread (marks a power-iterate store as
+// filled; this kernel runs after the scale kernel that read the flag).
 __global__ void root_prologue_kernel(int kind, const float* __restrict__ A, int n, const int* __restrict__ valid,
                                      float eps, int p, const float* __restrict__ s, const float* __restrict__ sf,
-                                     float* __restrict__ out0, float* __restrict__ out1, float* __restrict__ out2) {
+                                     float* __restrict__ out0, float* __restrict__ out1, float* __restrict__ out2,
+                                     int* set_flag) {
   pdl_launch_dependents();  // a following GEMM may start its prologue
+  if (set_flag && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0 && threadIdx.y == 0)
+    *set_flag = 1;
   __shared__ float t1[32][33];
   __shared__ float t2[32][33];
   const int i = blockIdx.z;
@@ -539,21 +567,24 @@ int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, flo
 }
 
 int launch_spectral_scale(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int iters,
-                          float* s, float* sc, float* sf, cudaStream_t st) {
+                          float* s, float* sc, float* sf, float* vec, const int* warm, int warm_iters,
+                          cudaStream_t st) {
   if (batch == 0) return 0;
   ProfScope ps(K_NORM, st, 0.0, 4.0 * (iters + 1) * batch * n * n);
-  spectral_scale_kernel<<<static_cast<unsigned>(batch), 512, 2 * n * sizeof(float), st>>>(A, n, valid, eps, 1.0 / p,
-                                                                                         iters, s, sc, sf);
+  spectral_scale_kernel<<<static_cast<unsigned>(batch), 512, 2 * n * sizeof(float), st>>>(
+      A, n, valid, eps, 1.0 / p, iters, s, sc, sf, vec, warm, warm_iters);
   count_launch();
   return check_cuda(cudaGetLastError(), "spectral_scale_kernel");
 }
 
 int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const int* valid, float eps, int p,
-                         const float* s, const float* sf, float* out0, float* out1, float* out2, cudaStream_t st) {
+                         const float* s, const float* sf, float* out0, float* out1, float* out2, int* set_flag,
+                         cudaStream_t st) {
   if (batch == 0) return 0;
   ProfScope ps(K_PROLOGUE, st, 0.0, 16.0 * batch * n * n);
   dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
-  root_prologue_kernel<<<grid, block, 0, st>>>(kind, A, n, valid, eps, p, s, sf ? sf : s, out0, out1, out2);
+  root_prologue_kernel<<<grid, block, 0, st>>>(kind, A, n, valid, eps, p, s, sf ? sf : s, out0, out1, out2,
+                                               set_flag);
   count_launch();
   return check_cuda(cudaGetLastError(), "root_prologue_kernel");
 }

@@ -90,7 +90,8 @@ int kmin_newton(int p, bool order2) {
   if (order2) return p >= 4 ? 17 : 18;
   return p >= 4 ? 24 : 26;
 }
-constexpr int kPowerIters = 12;  // power-iteration steps of the coupled-Newton scale
+constexpr int kPowerIters = 12;     // power-iteration steps of the coupled-Newton scale
+constexpr int kPowerItersWarm = 4;  // ... from the previous refresh's iterate
 constexpr int kKminSqrt = 26;
 
 struct Layout {
@@ -310,7 +311,12 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
     // Frobenius norm); Newton-DB (convergent only on (0, 2)) and Chebyshev
     // (an exact upper bound is needed) by the Frobenius norm.
     if (job.solver == 0 || job.solver == 3) {
-      if ((rc = launch_spectral_scale(A, cb, n, valid, job.eps, p, kPowerIters, S.s, S.sc, S.sf, st))) return rc;
+      float* pv = job.power_vec ? job.power_vec + off * n : nullptr;
+      // one flag for all chunks: read by every chunk's scale kernel, set by the
+      // last chunk's root prologue
+      if ((rc = launch_spectral_scale(A, cb, n, valid, job.eps, p, kPowerIters, S.s, S.sc, S.sf, pv,
+                                      job.power_vec ? job.power_warm : nullptr, kPowerItersWarm, st)))
+        return rc;
     } else {
       if ((rc = launch_frob_norm(A, cb, n, valid, job.eps, p, S.s, S.sc, st))) return rc;
     }
@@ -378,7 +384,9 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       // increasing to 1.
       const bool order2 = job.solver == 3;
       const float c1 = 1.f / p, c2 = (p + 1.f) / (2.f * p * p);
-      if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, S.sf, M[0].base, T.base, X[1].base, st)))
+      int* set_flag = (job.power_vec && job.power_warm && off + cb == job.batch) ? job.power_warm : nullptr;
+      if ((rc = launch_root_prologue(0, A, cb, n, valid, job.eps, p, S.s, S.sf, M[0].base, T.base, X[1].base,
+                                     set_flag, st)))
         return rc;
       // With the second-degree correction the M update also writes
       // D = I - M (exact in fp32 from the accumulator value), and T is formed
@@ -496,7 +504,7 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       StackMaps* Z = &sm[2];
       StackMaps& T = sm[4];
       if ((rc = launch_root_prologue(1, A, cb, n, valid, job.eps, p, S.s, nullptr, Y[0].base, T.base, Z[1].base,
-                                     st)))
+                                     nullptr, st)))
         return rc;
       const int stages = (p == 4) ? 2 : 1;
       for (int stage = 0; stage < stages; ++stage) {
