@@ -380,7 +380,8 @@ SHAMPOO_API int shampoo_pack_blocks(const int64_t* d_table, int32_t nblocks, int
  *            of 32 in [32, 1024].
  *  d_Q       device stack (batch, n, n): eigenvectors as columns, in no
  *            particular order (Jacobi's); in/out with warm_start = 1.
- *  d_lam     nullable device (batch, n): eigenvalues, matching Q's columns.
+ *  d_lam     nullable device (batch, n): eigenvalues, matching Q's columns, as
+ *            Rayleigh quotients q_j^T A q_j of the final basis.
  *  d_scratch 256-byte aligned, eigh_scratch_bytes(batch, n) for one pass
  *            (less, but at least one matrix's share, works in chunks).
  *  d_status  nullable device int32: OR of SHAMPOO_DEVFLAG_*.

@@ -172,6 +172,24 @@ __global__ void transpose_kernel(const float* __restrict__ X, int n, float* __re
         t[threadIdx.x][threadIdx.y + 8 * k];
 }
 
+// Eigenvalues as Rayleigh quotients of the final basis: lam_j = q_j^T A q_j =
+// sum_i Q[i][j] (A Q)[i][j] (more accurate than the diagonal Jacobi's
+// rotations leave, which carries their accumulated rounding).  One thread per
+// column, rows in order (coalesced across the threads of a row).
+__global__ void rayleigh_kernel(const float* __restrict__ Q, const float* __restrict__ AQ, int n,
+                                const int* __restrict__ valid, float* __restrict__ lam) {
+  const int i = blockIdx.y;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  const int m = valid ? valid[i] : n;
+  const size_t nn = static_cast<size_t>(n) * n;
+  double acc = 0.0;
+  if (j < m)
+    for (int r = 0; r < m; ++r)
+      acc += static_cast<double>(Q[i * nn + static_cast<size_t>(r) * n + j]) * AQ[i * nn + static_cast<size_t>(r) * n + j];
+  lam[static_cast<size_t>(i) * n + j] = static_cast<float>(acc);
+}
+
 }  // namespace
 
 size_t eig_scratch_per_matrix(int n) { return static_cast<size_t>(5) * n * n * 4; }
@@ -181,7 +199,8 @@ int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const i
   if (batch == 0) return 0;
   const size_t per = eig_scratch_per_matrix(n);
   const size_t nn = static_cast<size_t>(n) * n;
-  const int64_t cb_max = static_cast<int64_t>(scratch_bytes / per);
+  // at most 65535 matrices per chunk (grid.y / grid.z of the per-matrix kernels)
+  const int64_t cb_max = std::min<int64_t>(static_cast<int64_t>(scratch_bytes / per), 65535);
   if (cb_max < 1) return set_error(-3, "eigensolver scratch too small: %zu < %zu bytes", scratch_bytes, per);
   int rc;
   for (int64_t off = 0; off < batch; off += cb_max) {
@@ -207,8 +226,8 @@ int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const i
     auto jacobi = [&](const float* in, float* vout) -> int {
       ProfScope ps(K_PROLOGUE, st, 0.0, 8.0 * cb * nn);
       // the Jacobi working copy lives in Rm
-      jacobi_eig_kernel<<<static_cast<unsigned>(cb), kJacobiThreads, 0, st>>>(in, n, vi, Rm, vout, li, jacobi_sweeps,
-                                                                          kJacobiTol, flags);
+      jacobi_eig_kernel<<<static_cast<unsigned>(cb), kJacobiThreads, 0, st>>>(in, n, vi, Rm, vout, nullptr,
+                                                                          jacobi_sweeps, kJacobiTol, flags);
       count_launch();
       return check_cuda(cudaGetLastError(), "jacobi_eig_kernel");
     };
@@ -274,6 +293,19 @@ int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const i
       }
       if ((rc = check_cuda(cudaMemcpyAsync(Qi, T, cb * nn * 4, cudaMemcpyDeviceToDevice, st), "orthogonalised basis")))
         return rc;
+    }
+    if (li) {  // eigenvalues: Rayleigh quotients of the final basis
+      {
+        Builder b;
+        Epilogue& e = b.add(cbi, n, mA, 0, mX, 0, f1, B_MN_MAJOR);  // T = A Q
+        e.D = T;
+        e.flags = flags;
+        if ((rc = b.launch(st))) return rc;
+      }
+      ProfScope ps(K_CHECK, st, 0.0, 8.0 * cb * nn);
+      rayleigh_kernel<<<dim3((n + 127) / 128, static_cast<unsigned>(cb)), 128, 0, st>>>(Qi, T, n, vi, li);
+      count_launch();
+      if ((rc = check_cuda(cudaGetLastError(), "rayleigh_kernel"))) return rc;
     }
   }
   return 0;

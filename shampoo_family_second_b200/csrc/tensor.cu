@@ -184,6 +184,66 @@ __global__ void row_scale_kernel(const float* __restrict__ cur, const float* __r
   out[t] = x < n ? d[x] * cur[t] : 0.f;
 }
 
+// Statistic of a short mode (n <= 32) whose unfolding is long (K up to
+// 10^6): one 32 x 32 GEMM tile would reduce all of K on one SM, so the Gram
+// matrix is summed in K-chunks instead.  Phase 1: each CTA stages 128-column
+// pieces of the n rows of its chunk in shared memory and accumulates its
+// thread's pairs (x <= y) in float64; phase 2 adds the chunks' partials in
+// chunk order and writes H <- beta H + sum (both triangles).
+constexpr int kGramChunk = 4096;
+constexpr int kGramPairs = 32 * 33 / 2;
+__global__ void __launch_bounds__(256) gram_small_kernel(const float* __restrict__ U, int64_t ld, int n, int64_t K,
+                                                         double* __restrict__ partial) {
+  __shared__ float tile[32][129];
+  const int chunk = blockIdx.x;
+  const int64_t c_begin = static_cast<int64_t>(chunk) * kGramChunk;
+  const int64_t c_end = c_begin + kGramChunk < K ? c_begin + kGramChunk : K;
+  const int npairs = n * (n + 1) / 2;
+  double acc[3] = {0.0, 0.0, 0.0};
+  int px[3], py[3];
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {  // pair index -> (x, y), x <= y, row by row
+    int pidx = threadIdx.x + 256 * q, x = 0;
+    while (pidx >= n - x && x < n) pidx -= n - x, ++x;
+    px[q] = x;
+    py[q] = x + pidx;
+  }
+  for (int64_t c0 = c_begin; c0 < c_end; c0 += 128) {
+    for (int e = threadIdx.x; e < 32 * 128; e += 256) {
+      const int r = e >> 7, c = e & 127;
+      const int64_t col = c0 + c;
+      tile[r][c] = (r < n && col < c_end) ? U[static_cast<int64_t>(r) * ld + col] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      if (threadIdx.x + 256 * q >= npairs) continue;
+      double a = 0.0;
+      for (int c = 0; c < 128; ++c) a += static_cast<double>(tile[px[q]][c]) * tile[py[q]][c];
+      acc[q] += a;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int q = 0; q < 3; ++q)
+    if (threadIdx.x + 256 * q < npairs) partial[static_cast<int64_t>(chunk) * kGramPairs + threadIdx.x + 256 * q] = acc[q];
+}
+
+__global__ void gram_reduce_kernel(const double* __restrict__ partial, int nchunks, int n, float beta,
+                                   float* __restrict__ H, int ldh) {
+  const int npairs = n * (n + 1) / 2;
+  for (int pidx0 = threadIdx.x; pidx0 < npairs; pidx0 += blockDim.x) {
+    double sum = 0.0;
+    for (int ch = 0; ch < nchunks; ++ch) sum += partial[static_cast<int64_t>(ch) * kGramPairs + pidx0];
+    int pidx = pidx0, x = 0;
+    while (pidx >= n - x) pidx -= n - x, ++x;
+    const int y = x + pidx;
+    const float v = static_cast<float>(static_cast<double>(beta) * H[x * ldh + y] + sum);
+    H[x * ldh + y] = v;
+    H[y * ldh + x] = v;
+  }
+}
+
 struct Mode {
   int n, npad;
   int64_t K;
@@ -212,8 +272,12 @@ struct Plan {
   std::vector<Param> params;
   std::vector<Group> groups;
   size_t state_status, state_total;
-  size_t u_area, v_floats, root_bytes, scratch_u, scratch_v0, scratch_v1, scratch_root, scratch_total;
+  size_t u_area, v_floats, root_bytes, gram_bytes;
+  size_t scratch_u, scratch_v0, scratch_v1, scratch_root, scratch_gram, scratch_total;
 };
+
+// A mode whose statistic takes the split-K path.
+bool small_mode(int npad, int64_t K) { return npad == 32 && K > 8 * kGramChunk; }
 
 int validate_tensor_config(const shampoo_config* c) {
   if (!c) return set_error(SHAMPOO_ERR_INVALID_ARG, "config is NULL");
@@ -322,6 +386,11 @@ int make_plan(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
     P.u_area = std::max(P.u_area, pr.u_floats);
     for (const Mode& m : pr.modes) P.v_floats = std::max(P.v_floats, static_cast<size_t>(m.npad) * m.Kpad);
   }
+  P.gram_bytes = 0;
+  for (const Param& pr : P.params)
+    for (const Mode& m : pr.modes)
+      if (!m.diag && small_mode(m.npad, m.K))
+        P.gram_bytes = std::max(P.gram_bytes, static_cast<size_t>((m.K + kGramChunk - 1) / kGramChunk) * kGramPairs * 8);
   P.root_bytes = 0;
   for (const Group& g : P.groups) {
     const size_t per = root_scratch_per_matrix(g.npad, cfg->solver, g.p);
@@ -333,6 +402,7 @@ int make_plan(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
   P.scratch_v0 = o, o += alt(P.v_floats * 4);
   P.scratch_v1 = o, o += alt(P.v_floats * 4);
   P.scratch_root = o, o += alt(P.root_bytes);
+  P.scratch_gram = o, o += alt(P.gram_bytes);
   P.scratch_total = o;
   return SHAMPOO_OK;
 }
@@ -468,6 +538,18 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
         if ((rc = check_cuda(cudaGetLastError(), "row_sumsq_kernel"))) return rc;
         continue;
       }
+      if (small_mode(m.npad, m.K)) {
+        ProfScope ps(K_NORM, st, 2.0 * m.n * double(m.n) * m.K, 4.0 * m.n * double(m.K));
+        double* partial = reinterpret_cast<double*>(h->scratch + P.scratch_gram);
+        const int nchunks = static_cast<int>((m.K + kGramChunk - 1) / kGramChunk);
+        gram_small_kernel<<<nchunks, 256, 0, st>>>(U + m.u_off, m.Kpad, m.n, m.K, partial);
+        count_launch();
+        if ((rc = check_cuda(cudaGetLastError(), "gram_small_kernel"))) return rc;
+        gram_reduce_kernel<<<1, 256, 0, st>>>(partial, nchunks, m.n, c.beta, hptr(m), m.npad);
+        count_launch();
+        if ((rc = check_cuda(cudaGetLastError(), "gram_reduce_kernel"))) return rc;
+        continue;
+      }
       Epilogue& e = b.add_rect(1, m.npad, m.npad, m.Kpad, um[i], 0, um[i], 0, 2.0 * m.n * double(m.n) * m.K,
                                B_TRANSPOSED);
       b.L.g[b.L.ngroups - 1].a_exact = b.L.g[b.L.ngroups - 1].b_exact = g_exact;
@@ -479,7 +561,9 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
     }
     if (b.L.ngroups > 0 && (rc = b.launch(st))) return rc;
     for (int i = 0; i < pr.k; ++i)
-      if (!pr.modes[i].diag && (rc = launch_mirror_lower(hptr(pr.modes[i]), 1, pr.modes[i].npad, st))) return rc;
+      if (!pr.modes[i].diag && !small_mode(pr.modes[i].npad, pr.modes[i].K) &&
+          (rc = launch_mirror_lower(hptr(pr.modes[i]), 1, pr.modes[i].npad, st)))
+        return rc;
   }
   // 3. roots X = (H + eps I)^{-1/(2k)}, batched per (npad, k)
   if (refresh) {

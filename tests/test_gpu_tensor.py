@@ -5,10 +5,11 @@ cost", cue 26: one statistic per dimension of the gradient tensor (the
 gradient contracted with itself over every other dimension), roots with the
 power -1/(2k), applied by contractions along each dimension.
 
-Shapes: a 3 x 3 convolution kernel (order 4: two tiny modes, padded to 32),
-an order-3 tensor with ragged dimensions, an order-2 tensor (the unblocked
-matrix case, p = 4), and bf16 gradients; all in one handle, so the unfolding
-area is reused across parameters.  Checked per step, parameter and mode:
+Shapes: 3 x 3 convolution kernels (order 4: two tiny modes, padded to 32; in
+the larger one their statistics take the split-K Gram path), an order-3
+tensor with ragged dimensions, an order-2 tensor (the unblocked matrix case,
+p = 4), and bf16 gradients; all in one handle, so the unfolding area is
+reused across parameters.  Checked per step, parameter and mode:
 statistics (1e-5 against the oracle's H_i), roots on refresh steps
 (root_checks on the GPU's own statistics with p = 2k), the apply stage (the
 float64 mode products of the GPU's own roots and the gradient, 2e-5 times the
@@ -28,7 +29,9 @@ from parity import Fp32ReferenceTensorShampoo, root_checks, tensor_apply_check, 
 
 TOL_STATS = 1e-5
 NULL_SPREAD = 0.10
-SHAPES = ((3, 3, 16, 40), (24, 40, 56), (64, 48), (5, 7, 9, 11))
+# (3, 3, 96, 400): its 3-long modes unfold to 115200 columns, which the split-K
+# Gram kernel reduces instead of a single GEMM tile
+SHAPES = ((3, 3, 16, 40), (24, 40, 56), (64, 48), (5, 7, 9, 11), (3, 3, 96, 400))
 
 
 @pytest.fixture(scope="module")
