@@ -95,7 +95,10 @@ enum {
   SHAMPOO_KERNEL_CHECK = 4,    /* residual check */
   SHAMPOO_KERNEL_FINALIZE = 5, /* unscale + output */
   SHAMPOO_KERNEL_CHEB_COEF = 6,/* Chebyshev coefficients */
-  SHAMPOO_KERNEL_KINDS = 7
+  SHAMPOO_KERNEL_SCALE = 7,    /* power-iteration spectral scale (coupled Newton) */
+  SHAMPOO_KERNEL_MIRROR = 8,   /* lower triangle of symmetric statistics from the upper */
+  SHAMPOO_KERNEL_EIGEN = 9,    /* Jacobi sweeps of the eigensolver */
+  SHAMPOO_KERNEL_KINDS = 10
 };
 
 /* Hyper-parameters of the blocked step.

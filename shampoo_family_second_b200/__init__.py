@@ -45,8 +45,9 @@ KERNEL_PROLOGUE = 3
 KERNEL_CHECK = 4
 KERNEL_FINALIZE = 5
 KERNEL_CHEB_COEF = 6
-KERNEL_KINDS = 7
-KERNEL_NAMES = ("gemm3x_tf32", "stack_blocks", "frob_norm", "prologue", "check", "finalize", "cheb_coef")
+KERNEL_KINDS = 10
+KERNEL_NAMES = ("gemm3x_tf32", "stack_blocks", "frob_norm", "prologue", "check", "finalize", "cheb_coef",
+                "spectral_scale", "mirror_lower", "jacobi_eig")
 
 # Exported symbols, in header order (tests compare this with include/shampoo.h).
 EXPORTS = (

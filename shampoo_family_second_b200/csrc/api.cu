@@ -164,6 +164,7 @@ struct shampoo_ctx {
   StackMaps mGs, mGt, mRoots, mTap, mMom;
   double stats_flops_L = 0, stats_flops_R = 0, stack_bytes = 0;
   int64_t step = 0;
+  int power_refreshed = 0;  // a refresh has stored power iterates (profiler byte count only)
   cudaStream_t last_stream = nullptr;
 };
 
@@ -369,7 +370,9 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
     job.flags = h->d_status;
     job.power_vec = reinterpret_cast<float*>(h->state + h->sl.pvec);
     job.power_warm = reinterpret_cast<int*>(h->state + h->sl.pflag);
+    job.power_warm_hint = h->power_refreshed;
     if ((rc = run_inverse_roots(job, h->scratch + h->xl.root, h->xl.root_bytes, st))) return rc;
+    h->power_refreshed = 1;
     // 4a. apply, first product: T = XL G (with the fresh roots)
     Builder b;
     add_apply1(b);

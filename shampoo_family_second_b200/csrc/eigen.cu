@@ -224,7 +224,7 @@ int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const i
       return rc;
     dim3 tgrid(n / 32, n / 32, static_cast<unsigned>(cb)), tblock(32, 8);
     auto jacobi = [&](const float* in, float* vout) -> int {
-      ProfScope ps(K_PROLOGUE, st, 0.0, 8.0 * cb * nn);
+      ProfScope ps(K_EIGEN, st, 0.0, 8.0 * cb * nn);
       // the Jacobi working copy lives in Rm
       jacobi_eig_kernel<<<static_cast<unsigned>(cb), kJacobiThreads, 0, st>>>(in, n, vi, Rm, vout, nullptr,
                                                                           jacobi_sweeps, kJacobiTol, flags);

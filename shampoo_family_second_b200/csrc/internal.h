@@ -104,7 +104,10 @@ enum KernelKind : int {
   K_CHECK = 4,
   K_FINALIZE = 5,
   K_CHEB_COEF = 6,
-  K_COUNT = 7,
+  K_SCALE = 7,
+  K_MIRROR = 8,
+  K_EIGEN = 9,
+  K_COUNT = 10,
 };
 struct ProfScope {
   ProfScope(int kind, cudaStream_t st, double alg_flops, double alg_bytes);
@@ -189,7 +192,7 @@ int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, flo
 // prologue of the refresh's last chunk sets *warm).
 int launch_spectral_scale(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int iters,
                           float* s, float* sc, float* sf, float* vec, const int* warm, int warm_iters,
-                          cudaStream_t st);
+                          int warm_hint, cudaStream_t st);
 // sf (nullable: s) sets the damping floor eps_eff = max(eps, 2^-24 sf);
 // set_flag (nullable) is set to 1 (a power-iterate store is filled).
 int launch_root_prologue(int kind, const float* A, int64_t batch, int n, const int* valid, float eps, int p,
@@ -236,6 +239,7 @@ struct RootJob {
                            // issued as plain launches up to the cap)
   float* power_vec = nullptr;  // coupled Newton's scale: per-matrix power-iterate store (batch x n), or NULL
   int* power_warm = nullptr;   // device flag: power_vec holds the previous refresh's iterates
+  int power_warm_hint = 0;     // host's view of that flag, used only for the profiler's byte count
 };
 // inv_root_batched with a switch for plain launches (shared by the public
 // entry points of api.cu and noalloc.cu).

@@ -568,9 +568,9 @@ int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, flo
 
 int launch_spectral_scale(const float* A, int64_t batch, int n, const int* valid, float eps, int p, int iters,
                           float* s, float* sc, float* sf, float* vec, const int* warm, int warm_iters,
-                          cudaStream_t st) {
+                          int warm_hint, cudaStream_t st) {
   if (batch == 0) return 0;
-  ProfScope ps(K_NORM, st, 0.0, 4.0 * (iters + 1) * batch * n * n);
+  ProfScope ps(K_SCALE, st, 0.0, 4.0 * ((warm_hint ? warm_iters : iters) + 1) * batch * n * n);
   spectral_scale_kernel<<<static_cast<unsigned>(batch), 512, 2 * n * sizeof(float), st>>>(
       A, n, valid, eps, 1.0 / p, iters, s, sc, sf, vec, warm, warm_iters);
   count_launch();
@@ -640,7 +640,7 @@ int launch_cheb_setup(const float* A, int64_t batch, int n, const int* valid, fl
 
 int launch_mirror_lower(float* D, int64_t batch, int n, cudaStream_t st) {
   if (batch == 0 || n <= kTileN) return 0;  // one tile column: every tile is computed
-  ProfScope ps(K_FINALIZE, st, 0.0, 8.0 * batch * n * double(n) * 0.375);
+  ProfScope ps(K_MIRROR, st, 0.0, 8.0 * batch * n * double(n) * 0.375);
   dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
   mirror_lower_kernel<<<grid, block, 0, st>>>(D, n);
   count_launch();

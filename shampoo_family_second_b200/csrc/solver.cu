@@ -315,7 +315,8 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       // one flag for all chunks: read by every chunk's scale kernel, set by the
       // last chunk's root prologue
       if ((rc = launch_spectral_scale(A, cb, n, valid, job.eps, p, kPowerIters, S.s, S.sc, S.sf, pv,
-                                      job.power_vec ? job.power_warm : nullptr, kPowerItersWarm, st)))
+                                      job.power_vec ? job.power_warm : nullptr, kPowerItersWarm,
+                                      job.power_vec && job.power_warm_hint, st)))
         return rc;
     } else {
       if ((rc = launch_frob_norm(A, cb, n, valid, job.eps, p, S.s, S.sc, st))) return rc;
