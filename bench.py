@@ -65,8 +65,12 @@ WORKLOAD_NAMES = {
 # order-4 tensor Shampoo: 4 stages of 4 kernels at 64 .. 512 channels.
 CONV_SHAPES = tuple((3, 3, c, c) for c in (64, 128, 256, 512) for _ in range(4))
 SWEEP_BATCH = {256: 512, 512: 128, 1024: 64}
-SOLVER_NAMES = {0: "coupled_newton", 1: "newton_db", 2: "chebyshev", 3: "coupled_newton_cubic"}
-SOLVER_IDS = {"newton": 0, "newton_db": 1, "chebyshev": 2, "newton_cubic": 3}
+SOLVER_NAMES = {0: "coupled_newton", 1: "newton_db", 2: "chebyshev", 3: "coupled_newton_cubic",
+                4: "coupled_newton_cubic_f64"}
+SOLVER_IDS = {"newton": 0, "newton_db": 1, "chebyshev": 2, "newton_cubic": 3, "newton_cubic_f64": 4}
+# fp64 tensor-core rate of a B200 (NVIDIA's nominal figure; no measured fp64 peak exists on this
+# pool): the denominator of the fp64-iterate solver's product
+FP64_NOMINAL_TFLOPS = 40.0
 
 
 # ---------------------------------------------------------------------------
@@ -824,12 +828,25 @@ def sweep_case(args, sb, device, stream, rank, world, n, kappa, p, solver_name, 
         flush.zero_()
         one()
     torch.cuda.synchronize()
-    g = sb.profile_read(sb.KERNEL_GEMM)
+    f64 = solver == SOLVER_IDS["newton_cubic_f64"]
+    g = sb.profile_read(sb.KERNEL_GEMM_F64 if f64 else sb.KERNEL_GEMM)
     sb.profile_enable(False)
     peaks, src = load_peaks()
     peak_burst, peak_sust, peak_kind = tensor_peaks(peaks, total_ms)
     peak = peak_burst if peak_kind == "burst" else peak_sust
     ach = (g.alg_flops / g.launches) / (g.total_ms / g.launches * 1e-3) / 1e12 if g.launches else 0.0
+    if f64:
+        roofline = {"kernel": "dgemm_kernel", "bound": "tensor", "achieved": ach, "peak": FP64_NOMINAL_TFLOPS,
+                    "unit": "TFLOP/s", "frac": ach / FP64_NOMINAL_TFLOPS, "traffic": None,
+                    "launches": g.launches, "avg_launch_ms": g.total_ms / max(g.launches, 1),
+                    "peak_basis": "nominal B200 fp64 tensor-core rate (not measured on this pool)"}
+    else:
+        roofline = {"kernel": "gemm3x_tf32_kernel", "bound": "tensor", "achieved": ach, "peak": peak,
+                    "unit": "TFLOP/s", "frac": ach / peak if peak else None, "traffic": None,
+                    "launches": g.launches, "avg_launch_ms": g.total_ms / max(g.launches, 1),
+                    "peak_kind": peak_kind, "frac_burst": ach / peak_burst if peak_burst else None,
+                    "frac_sustained": ach / peak_sust if peak_sust else None,
+                    "peak_basis": f"{src} bf16 {peak_kind} x 1.1/2.25 / 3"}
     it_host = iters.cpu().numpy()
     # error of a few roots against the construction's own root Q lam^{-1/p} Q^T
     # (of the float64 matrix: includes the fp32 rounding of A, amplified ~kappa u / p)
@@ -849,12 +866,7 @@ def sweep_case(args, sb, device, stream, rank, world, n, kappa, p, solver_name, 
                        "l2": "256 MiB buffer written between timed calls, outside the events"},
             "iters_used": [int(it_host.min()), int(it_host.max())], "device_status": int(status.item()),
             "rel_err_vs_construction_sample": errs, "gpu_launches": int(launches), "clocks": clk,
-            "roofline": {"kernel": "gemm3x_tf32_kernel", "bound": "tensor", "achieved": ach, "peak": peak,
-                         "unit": "TFLOP/s", "frac": ach / peak if peak else None, "traffic": None,
-                         "launches": g.launches, "avg_launch_ms": g.total_ms / max(g.launches, 1),
-                         "peak_kind": peak_kind, "frac_burst": ach / peak_burst if peak_burst else None,
-                         "frac_sustained": ach / peak_sust if peak_sust else None,
-                         "peak_basis": f"{src} bf16 {peak_kind} x 1.1/2.25 / 3"},
+            "roofline": roofline,
         }), flush=True)
 
 
@@ -868,14 +880,14 @@ def main():
     ap.add_argument("--ring", type=int, default=8, help="distinct gradient sets kept on the device")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--solver", default=None, choices=["newton", "newton_db", "chebyshev", "newton_cubic"],
+    ap.add_argument("--solver", default=None, choices=sorted(SOLVER_IDS),
                     help="inverse-root solver of the step workloads (default: the workload's own)")
     ap.add_argument("--momentum", type=float, default=None, help="momentum ahead of the preconditioner (step workloads)")
     ap.add_argument("--sweep-n", type=int, default=512)
     ap.add_argument("--sweep-batch", type=int, default=0)
     ap.add_argument("--sweep-kappa", type=float, default=1e4)
     ap.add_argument("--sweep-p", type=int, default=4)
-    ap.add_argument("--sweep-solver", default="newton", choices=["newton", "newton_db", "chebyshev", "newton_cubic"])
+    ap.add_argument("--sweep-solver", default="newton", choices=sorted(SOLVER_IDS))
     ap.add_argument("--sweep-iters", type=int, default=25)
     ap.add_argument("--sweep-tol", type=float, default=0.0)
     ap.add_argument("--sweep-degree", type=int, default=32)

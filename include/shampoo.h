@@ -77,10 +77,17 @@ enum {
   SHAMPOO_SOLVER_NEWTON = 0,    /* coupled Newton for A^{-1/p} (Guo & Higham 2006) */
   SHAMPOO_SOLVER_NEWTON_DB = 1, /* coupled Y/Z square-root iteration, twice for p = 4 */
   SHAMPOO_SOLVER_CHEBYSHEV = 2, /* Chebyshev interpolant of x^{-1/p}, Clenshaw evaluation */
-  SHAMPOO_SOLVER_NEWTON_CUBIC = 3 /* coupled Newton with the degree-2 binomial correction
+  SHAMPOO_SOLVER_NEWTON_CUBIC = 3, /* coupled Newton with the degree-2 binomial correction
                                      T = I + (I-M)/p + (p+1)(I-M)^2/(2p^2) after a plain first
                                      step: one more GEMM per iteration, cubic local convergence,
                                      about a third fewer iterations */
+  SHAMPOO_SOLVER_NEWTON_CUBIC_F64 = 4 /* the same iteration (scale, damping, stopping rule) with
+                                     fp64 iterates on the fp64 tensor-core instruction: the
+                                     root of the damped input to the last fp32 bit of the
+                                     output, for statistics whose condition number puts the
+                                     fp32 iterates' error ((1/p) 2^-24 kappa) above tolerance;
+                                     scratch holds fp64 stacks (twice the bytes), and the
+                                     products run at the fp64 rate */
 };
 
 /* Gradient element types. */
@@ -98,7 +105,8 @@ enum {
   SHAMPOO_KERNEL_SCALE = 7,    /* power-iteration spectral scale (coupled Newton) */
   SHAMPOO_KERNEL_MIRROR = 8,   /* lower triangle of symmetric statistics from the upper */
   SHAMPOO_KERNEL_EIGEN = 9,    /* Jacobi sweeps of the eigensolver */
-  SHAMPOO_KERNEL_KINDS = 10
+  SHAMPOO_KERNEL_GEMM_F64 = 10,/* fp64 GEMM of the fp64-iterate solver */
+  SHAMPOO_KERNEL_KINDS = 11
 };
 
 /* Hyper-parameters of the blocked step.
@@ -259,9 +267,10 @@ SHAMPOO_API int inv_root_batched(const float* d_A, float* d_X, int64_t batch, in
  * All calls share the array: calls whose work overlaps on the GPU (other
  * streams or host threads on the same device) race on it.  The solver clears
  * what must start at zero on every call.  Batches larger than the array are
- * solved in chunks (the largest need, coupled Newton at n = 1024, is 28 MiB
- * per matrix); a size whose scratch for one matrix exceeded the array would
- * return SHAMPOO_ERR_UNSUPPORTED.  With tol > 0 the iterations are plain
+ * solved in chunks (the largest need of the fp32 solvers at p <= 4, coupled
+ * Newton at n = 1024, is 28 MiB per matrix); a size whose scratch for one
+ * matrix exceeds the array (p = 6, 8 at n = 1024; fp64 iterates from n = 800)
+ * returns SHAMPOO_ERR_UNSUPPORTED.  With tol > 0 the iterations are plain
  * kernel launches up to the cap (tiles of finished matrices exit at once),
  * never a CUDA graph, whose instantiation may take device memory; results
  * equal inv_root_batched's. */
@@ -407,6 +416,17 @@ SHAMPOO_API int shampoo_gemm_scratch_bytes(int64_t batch, int32_t n, size_t* byt
 SHAMPOO_API int shampoo_gemm_batched(const float* d_A, const float* d_B, const float* d_C, float* d_D, int64_t batch, int32_t n,
                          int32_t op_b, float alpha, float beta, float gamma, void* d_scratch, size_t scratch_bytes,
                          int32_t* d_status, void* stream);
+
+/* The fp64 product of the fp64-iterate solver (SHAMPOO_SOLVER_NEWTON_CUBIC_F64),
+ * as a utility: D_i = alpha A_i B_i + beta C_i + gamma I for row-major fp64
+ * stacks (batch, n, n) on the fp64 tensor-core instruction (mma m8n8k4).
+ * d_C may be NULL (then beta is ignored) and may equal d_D; d_D must not
+ * overlap d_A or d_B.  n a multiple of 16 in [16, 4096], batch <= 65535, all
+ * four 16-byte aligned.  Enqueued on `stream`; no host sync; non-finite outputs
+ * raise SHAMPOO_DEVFLAG_NONFINITE in d_status (nullable). */
+SHAMPOO_API int shampoo_dgemm_batched(const double* d_A, const double* d_B, const double* d_C, double* d_D,
+                                      int64_t batch, int32_t n, double alpha, double beta, double gamma,
+                                      int32_t* d_status, void* stream);
 
 /* Profiling (process-wide).  When enabled, every kernel launch of the library
  * is bracketed by CUDA events on its own stream and tallied per kind with its

@@ -34,6 +34,7 @@ SOLVER_NEWTON = 0
 SOLVER_NEWTON_DB = 1
 SOLVER_CHEBYSHEV = 2
 SOLVER_NEWTON_CUBIC = 3
+SOLVER_NEWTON_CUBIC_F64 = 4
 
 F32 = 0
 BF16 = 1
@@ -45,9 +46,13 @@ KERNEL_PROLOGUE = 3
 KERNEL_CHECK = 4
 KERNEL_FINALIZE = 5
 KERNEL_CHEB_COEF = 6
-KERNEL_KINDS = 10
+KERNEL_SCALE = 7
+KERNEL_MIRROR = 8
+KERNEL_EIGEN = 9
+KERNEL_GEMM_F64 = 10
+KERNEL_KINDS = 11
 KERNEL_NAMES = ("gemm3x_tf32", "stack_blocks", "frob_norm", "prologue", "check", "finalize", "cheb_coef",
-                "spectral_scale", "mirror_lower", "jacobi_eig")
+                "spectral_scale", "mirror_lower", "jacobi_eig", "dgemm_f64")
 
 # Exported symbols, in header order (tests compare this with include/shampoo.h).
 EXPORTS = (
@@ -61,6 +66,7 @@ EXPORTS = (
     "shampoo_pack_blocks", "eigh_scratch_bytes", "eigh_batched",
     "shampoo_gemm_scratch_bytes",
     "shampoo_gemm_batched",
+    "shampoo_dgemm_batched",
     "shampoo_profile_enable", "shampoo_profile_reset", "shampoo_profile_read", "shampoo_launch_count",
 )
 
@@ -155,6 +161,8 @@ def _load():
         "eigh_batched": (ctypes.c_int, [P, P, P, I64, I32, I32, I32, I32, P, ctypes.c_size_t, P, P]),
         "shampoo_gemm_scratch_bytes": (ctypes.c_int, [I64, I32, sz]),
         "shampoo_gemm_batched": (ctypes.c_int, [P, P, P, P, I64, I32, I32, F, F, F, P, ctypes.c_size_t, P, P]),
+        "shampoo_dgemm_batched": (ctypes.c_int, [P, P, P, P, I64, I32, ctypes.c_double, ctypes.c_double,
+                                                 ctypes.c_double, P, P]),
         "shampoo_profile_enable": (None, [I32]),
         "shampoo_profile_reset": (None, []),
         "shampoo_profile_read": (ctypes.c_int, [I32, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_double),
@@ -525,6 +533,25 @@ def gemm_batched(A, B, C=None, alpha: float = 1.0, beta: float = 0.0, gamma: flo
                                         0 if trans_b else 1, alpha, beta, gamma, scratch.data_ptr(), scratch.numel(),
                                         status.data_ptr(),
                                         _stream_ptr(stream)))
+    return D, status
+
+
+def dgemm_batched(A, B, C=None, alpha: float = 1.0, beta: float = 0.0, gamma: float = 0.0, out=None,
+                  stream=None):
+    """D_i = alpha A_i B_i + beta C_i + gamma I in fp64 on the fp64 tensor-core
+    instruction (the products of SOLVER_NEWTON_CUBIC_F64)."""
+    import torch
+    for t in (A, B) + ((C,) if C is not None else ()):
+        if t.dtype != torch.float64 or t.dim() != 3 or not t.is_cuda:
+            raise ValueError("operands must be float64 CUDA tensors (batch, n, n)")
+    A, B = A.contiguous(), B.contiguous()
+    C = None if C is None else C.contiguous()
+    batch, n = A.shape[0], A.shape[1]
+    D = torch.empty_like(A) if out is None else out
+    status = torch.zeros(1, dtype=torch.int32, device=A.device)
+    with torch.cuda.device(A.device):
+        _check(lib.shampoo_dgemm_batched(A.data_ptr(), B.data_ptr(), _ptr(C), D.data_ptr(), batch, n, alpha, beta,
+                                         gamma, status.data_ptr(), _stream_ptr(stream)))
     return D, status
 
 

@@ -40,7 +40,7 @@ int validate_config(const shampoo_config* c) {
   if (!(c->eps >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "eps must be >= 0");
   if (!(c->lr == c->lr)) return set_error(SHAMPOO_ERR_INVALID_ARG, "lr is NaN");
   if (c->root_p != 2 && c->root_p != 4) return set_error(SHAMPOO_ERR_INVALID_ARG, "root_p must be 2 or 4");
-  if (c->solver < 0 || c->solver > 3) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", c->solver);
+  if (c->solver < 0 || c->solver > kMaxSolver) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", c->solver);
   if (c->solver != SHAMPOO_SOLVER_CHEBYSHEV && (c->iters < 1 || c->iters > 1000))
     return set_error(SHAMPOO_ERR_INVALID_ARG, "iters must be in [1, 1000]");
   if (!(c->tol >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "tol must be >= 0");
@@ -444,7 +444,7 @@ int inv_root_scratch_bytes(int64_t batch, int32_t n, int32_t solver, size_t* byt
 
 int inv_root_scratch_bytes_p(int64_t batch, int32_t n, int32_t solver, int32_t p, size_t* bytes) {
   if (!bytes) return set_error(SHAMPOO_ERR_INVALID_ARG, "bytes is NULL");
-  if (batch < 0 || n < 32 || n > 1024 || n % 32 || solver < 0 || solver > 3)
+  if (batch < 0 || n < 32 || n > 1024 || n % 32 || solver < 0 || solver > kMaxSolver)
     return set_error(SHAMPOO_ERR_INVALID_ARG, "bad batch / n / solver");
   if (p != 2 && p != 4 && p != 6 && p != 8) return set_error(SHAMPOO_ERR_INVALID_ARG, "p must be 2, 4, 6 or 8");
   *bytes = root_scratch_header() +
@@ -466,7 +466,7 @@ int shampoo::inv_root_batched_impl(const float* d_A, float* d_X, int64_t batch, 
   if (solver == SHAMPOO_SOLVER_NEWTON_DB && p > 4)
     return set_error(SHAMPOO_ERR_INVALID_ARG, "Newton-DB computes p = 2 and p = 4 only");
   if (!(eps >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "eps must be >= 0");
-  if (solver < 0 || solver > 3) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", solver);
+  if (solver < 0 || solver > kMaxSolver) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", solver);
   if (solver != SHAMPOO_SOLVER_CHEBYSHEV && (iters < 1 || iters > 1000))
     return set_error(SHAMPOO_ERR_INVALID_ARG, "iters must be in [1, 1000]");
   if (!(tol >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "tol must be >= 0");

@@ -21,6 +21,7 @@ constexpr int kMaxGroups = 4;
 constexpr int kMaxMaps = 2 * kMaxGroups;
 constexpr int kMaxParams = 1024;
 constexpr int kMaxChebDegree = 64;
+constexpr int kMaxSolver = 4;  // SHAMPOO_SOLVER_NEWTON_CUBIC_F64
 
 // Epilogue of one GEMM group.  For matrix i of the group and element (r, c):
 //   v = scale_i * (alpha * acc + beta * C_i[r][c] + gamma_i * [r == c])
@@ -107,7 +108,8 @@ enum KernelKind : int {
   K_SCALE = 7,
   K_MIRROR = 8,
   K_EIGEN = 9,
-  K_COUNT = 10,
+  K_GEMM_F64 = 10,
+  K_COUNT = 11,
 };
 struct ProfScope {
   ProfScope(int kind, cudaStream_t st, double alg_flops, double alg_bytes);
@@ -224,6 +226,30 @@ int launch_fill_iters(int* iters, int64_t batch, int value, cudaStream_t st);
 // After a GEMM group with sym = 1: copies the transpose of the computed upper
 // part into the 32 x 32 blocks of the tiles it skipped (wholly below the diagonal).
 int launch_mirror_lower(float* D, int64_t batch, int n, cudaStream_t st);
+
+// fp64 products of the fp64-iterate solver (solver_f64.cu): per matrix,
+// D = alpha A B + beta C + gamma I (true product, row-major n x n operands),
+// optionally E = e_mul D + e_add I and res[m] += sum over the valid diagonal
+// of (1 - D).  C may be D itself; A and B must not be written by the launch.
+struct DGemmGroup {
+  const double* A = nullptr;
+  const double* B = nullptr;
+  const double* C = nullptr;
+  double* D = nullptr;
+  double* E = nullptr;
+  double alpha = 1.0, beta = 0.0, gamma = 0.0, e_mul = 0.0, e_add = 0.0;
+  float* res = nullptr;
+};
+int launch_dgemm(const DGemmGroup* groups, int ngroups, int64_t batch, int n, const int* valid, const int* skip,
+                 int* flags, cudaStream_t st);
+// M0 = (sym(A) + eps_eff I)/s (identity on the padding), T = ((p+1) I - M0)/p,
+// X1 = T; eps_eff = max(eps, eps_floor_rel * sf).  A is fp32 or (a_is_f64) fp64.
+int launch_prologue_f64(const void* A, int a_is_f64, int64_t batch, int n, const int* valid, float eps,
+                        float eps_floor_rel, int p, const float* s, const float* sf, double* M0, double* T,
+                        double* X1, int* set_flag, cudaStream_t st);
+// out = sym(X_final) s^{-1/p} in fp32; X_final = X1 if (iters or default_iters) is odd, else X0.
+int launch_finalize_f64(const double* X0, const double* X1, const int* iters, int default_iters, const float* s,
+                        int p, int64_t batch, int n, float* out, int* flags, cudaStream_t st);
 
 // Inverse-root solver (solver.cu) ---------------------------------------------
 struct RootJob {

@@ -67,9 +67,11 @@ constexpr int NEWTON_B = B_MN_MAJOR;
 //   Newton-DB : Y0 Y1 Z0 Z1 T
 //   Chebyshev : Xt b0 b1 b2
 int stacks_for(int solver, int p) {
-  if (solver == 0 || solver == 3) return p >= 6 ? 8 : 7;
+  if (solver == 0 || solver == 3 || solver == 4) return p >= 6 ? 8 : 7;
   return solver == 1 ? 5 : 4;
 }
+// Bytes per stack element: fp64 iterates for solver 4, fp32 otherwise.
+size_t stack_elem_bytes(int solver) { return solver == 4 ? 8 : 4; }
 
 constexpr size_t kAlign = 256;
 constexpr size_t kHeader = 64 * 1024;  // covers the alignment padding of the arrays
@@ -128,7 +130,7 @@ Layout carve(void* base, int64_t cb, int n, int solver, int root_p) {
   L.iters1 = reinterpret_cast<int*>(take(cb * 4));
   L.coef = reinterpret_cast<float*>(take(cb * 4 * (kMaxChebDegree + 2)));
   for (int k = 0; k < stacks_for(solver, root_p); ++k)
-    L.stack[k] = reinterpret_cast<float*>(take(plain_floats(cb, n) * 4));
+    L.stack[k] = reinterpret_cast<float*>(take(plain_floats(cb, n) * stack_elem_bytes(solver)));
   return L;
 }
 
@@ -282,7 +284,8 @@ int run_loop(const LoopKey& key, int kernels_per_iter, Body&& body, cudaStream_t
 size_t root_scratch_header() { return kHeader; }
 
 size_t root_scratch_per_matrix(int n, int solver, int p) {
-  return static_cast<size_t>(stacks_for(solver, p)) * n * n * 4 + 4 * (kVecInts + kMaxChebDegree + 2);
+  return static_cast<size_t>(stacks_for(solver, p)) * n * n * stack_elem_bytes(solver) +
+         4 * (kVecInts + kMaxChebDegree + 2);
 }
 
 int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, cudaStream_t st) {
@@ -293,7 +296,8 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
   if (scratch_bytes < kHeader + per)
     return set_error(-3, "inverse-root scratch too small: %zu < %zu bytes", scratch_bytes, kHeader + per);
   const int64_t cb_max = std::min<int64_t>(job.batch, static_cast<int64_t>((scratch_bytes - kHeader) / per));
-  const int64_t cb_cap = std::min<int64_t>(cb_max, 65535);  // grid.z limit of the prologues
+  // grid.z limit of the prologues (and of the fp64 GEMM's two groups)
+  const int64_t cb_cap = std::min<int64_t>(cb_max, job.solver == 4 ? 32767 : 65535);
   const double f1 = 2.0 * n * static_cast<double>(n) * n;  // one GEMM(n), algorithmic
   int rc = 0;
   for (int64_t off = 0; off < job.batch; off += cb_cap) {
@@ -305,12 +309,13 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
     float* out = job.X + off * static_cast<int64_t>(n) * n;
     int* iters_out = job.iters_used ? job.iters_used + off : nullptr;
     StackMaps sm[8];
-    for (int k = 0; k < stacks_for(job.solver, p); ++k)
-      if ((rc = make_stack_maps(sm[k], S.stack[k], cb, n))) return rc;
+    if (job.solver != 4)  // the fp64 GEMM reads its operands without tensor maps
+      for (int k = 0; k < stacks_for(job.solver, p); ++k)
+        if ((rc = make_stack_maps(sm[k], S.stack[k], cb, n))) return rc;
     // Coupled Newton scales by the power-iteration estimate (bounded by the
     // Frobenius norm); Newton-DB (convergent only on (0, 2)) and Chebyshev
     // (an exact upper bound is needed) by the Frobenius norm.
-    if (job.solver == 0 || job.solver == 3) {
+    if (job.solver == 0 || job.solver == 3 || job.solver == 4) {
       float* pv = job.power_vec ? job.power_vec + off * n : nullptr;
       // one flag for all chunks: read by every chunk's scale kernel, set by the
       // last chunk's root prologue
@@ -368,7 +373,95 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       e.flags = job.flags;
     };
 
-    if (job.solver == 0 || job.solver == 3) {
+    if (job.solver == 4) {
+      // ------------------------------------------------ coupled Newton, fp64 iterates
+      // The second-degree iteration of solver 3 below, step for step, with the
+      // same stack rotation, on fp64 stacks through the fp64 GEMM.
+      double* Mb[2] = {reinterpret_cast<double*>(S.stack[0]), reinterpret_cast<double*>(S.stack[1])};
+      double* Xb[2] = {reinterpret_cast<double*>(S.stack[2]), reinterpret_cast<double*>(S.stack[3])};
+      double* Q[3] = {reinterpret_cast<double*>(S.stack[4]), reinterpret_cast<double*>(S.stack[5]),
+                      reinterpret_cast<double*>(S.stack[6])};
+      double* Tp = reinterpret_cast<double*>(S.stack[7]);
+      const double c1 = 1.0 / p, c2 = (p + 1.0) / (2.0 * p * p);
+      int* set_flag = (job.power_vec && job.power_warm && off + cb == job.batch) ? job.power_warm : nullptr;
+      // fp32 input: the damping floor is the fp32 rounding of A (2^-24 ||A + eps I||_F, as
+      // for the fp32 solvers), below which the input itself may be indefinite
+      if ((rc = launch_prologue_f64(A, 0, cb, n, valid, job.eps, 5.9604645e-8f, p, S.s, S.sf, Mb[0], Q[0], Xb[1],
+                                    set_flag, st)))
+        return rc;
+      auto dg = [](const double* a, const double* b, double* d) {
+        DGemmGroup g;
+        g.A = a;
+        g.B = b;
+        g.D = d;
+        return g;
+      };
+      auto iterate = [&](int j, cudaStream_t cs, const GraphLoop* lp) -> int {
+        int r;
+        double* Tb = Q[0];
+        double* T2b = Q[1];
+        double* T4b = Q[2];
+        if (j >= 1) {
+          double* Db = p >= 4 ? Q[j & 1] : Q[0];
+          Tb = p >= 4 ? Q[(j + 1) & 1] : Q[1];
+          T2b = Q[2];
+          T4b = Db;
+          DGemmGroup g = dg(Db, Db, Tb);  // T = c2 D D + c1 D + I
+          g.C = Db;
+          g.alpha = c2;
+          g.beta = c1;
+          g.gamma = 1.0;
+          if ((r = launch_dgemm(&g, 1, cb, n, valid, skip, job.flags, cs))) return r;
+        }
+        double* Dnext = p >= 4 ? Q[(j + 1) & 1] : Q[0];
+        const bool last = !residual && j == job.iters - 1;
+        {
+          DGemmGroup g[2];
+          int ng = 0;
+          if (!last) g[ng++] = dg(Tb, Tb, T2b);                      // T2 = T T
+          if (j >= 1) g[ng++] = dg(Xb[j & 1], Tb, Xb[(j + 1) & 1]);  // X <- X T
+          if (ng && (r = launch_dgemm(g, ng, cb, n, valid, skip, job.flags, cs))) return r;
+        }
+        if (last) return 0;
+        double* P = T2b;
+        if (p >= 4) {
+          DGemmGroup g = dg(T2b, T2b, T4b);  // T4 = T2 T2
+          if ((r = launch_dgemm(&g, 1, cb, n, valid, skip, job.flags, cs))) return r;
+          P = T4b;
+        }
+        if (p >= 6) {
+          DGemmGroup g = dg(T4b, p == 6 ? T2b : T4b, Tp);
+          if ((r = launch_dgemm(&g, 1, cb, n, valid, skip, job.flags, cs))) return r;
+          P = Tp;
+        }
+        {
+          DGemmGroup g = dg(P, Mb[j & 1], Mb[(j + 1) & 1]);  // M <- T^p M, next D = I - M
+          g.E = Dnext;
+          g.e_mul = -1.0;
+          g.e_add = 1.0;
+          g.res = residual ? S.res : nullptr;
+          if ((r = launch_dgemm(&g, 1, cb, n, valid, skip, job.flags, cs))) return r;
+        }
+        if (residual)
+          return launch_check(S.res, S.prev, S.done, S.iters, valid, cb, n, job.tol, S.counter, job.iters,
+                              kmin_newton(p, true), job.flags, lp, cs);
+        return 0;
+      };
+      if (residual) {
+        const int per_iter = (p == 2 ? 3 : (p == 4 ? 4 : 5)) + 1;
+        if ((rc = iterate(0, st, nullptr)) || (rc = run_rest(iterate, per_iter))) return rc;
+      } else {
+        for (int j = 0; j < job.iters; ++j)
+          if ((rc = iterate(j, st, nullptr))) return rc;
+      }
+      if ((rc = launch_finalize_f64(Xb[0], Xb[1], residual ? S.iters : nullptr, job.iters, S.s, p, cb, n, out,
+                                    job.flags, st)))
+        return rc;
+      if ((iters_out || residual) &&
+          (rc = launch_report(residual ? S.iters : nullptr, nullptr, residual ? S.done : nullptr, cb, job.iters,
+                              iters_out, job.flags, residual, st)))
+        return rc;
+    } else if (job.solver == 0 || job.solver == 3) {
       // ------------------------------------------------------------ coupled Newton
       StackMaps* M = &sm[0];  // M[0], M[1]
       StackMaps* X = &sm[2];  // X[0], X[1]

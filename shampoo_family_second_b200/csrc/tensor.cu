@@ -284,7 +284,7 @@ int validate_tensor_config(const shampoo_config* c) {
   if (!(c->beta >= 0.f) || !(c->beta <= 1.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "beta must be in [0, 1]");
   if (!(c->eps >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "eps must be >= 0");
   if (!(c->lr == c->lr)) return set_error(SHAMPOO_ERR_INVALID_ARG, "lr is NaN");
-  if (c->solver < 0 || c->solver > 3) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", c->solver);
+  if (c->solver < 0 || c->solver > kMaxSolver) return set_error(SHAMPOO_ERR_INVALID_ARG, "unknown solver %d", c->solver);
   if (c->solver != SHAMPOO_SOLVER_CHEBYSHEV && (c->iters < 1 || c->iters > 1000))
     return set_error(SHAMPOO_ERR_INVALID_ARG, "iters must be in [1, 1000]");
   if (!(c->tol >= 0.f)) return set_error(SHAMPOO_ERR_INVALID_ARG, "tol must be >= 0");

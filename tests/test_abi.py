@@ -111,18 +111,24 @@ def test_scratch_sizes(sb):
         assert sb.inv_root_scratch_bytes(1, 1024, solver) <= 32 << 20
     with pytest.raises(sb.ShampooError):
         sb.inv_root_scratch_bytes(4, 100, 0)
-    with pytest.raises(sb.ShampooError):   # no solver 4
-        sb.inv_root_scratch_bytes(4, 256, 4)
+    # fp64 iterates: the same 7 stacks at 8 bytes per element; beyond the
+    # no-alloc array at n = 1024
+    f64 = sb.inv_root_scratch_bytes(128, 1024, sb.SOLVER_NEWTON_CUBIC_F64) - \
+        sb.inv_root_scratch_bytes(64, 1024, sb.SOLVER_NEWTON_CUBIC_F64)
+    assert f64 == 64 * (7 * 1024 * 1024 * 8 + 4 * (8 + 64 + 2))
+    assert sb.inv_root_scratch_bytes(1, 1024, sb.SOLVER_NEWTON_CUBIC_F64) > 32 << 20
+    with pytest.raises(sb.ShampooError):   # no solver 5
+        sb.inv_root_scratch_bytes(4, 256, 5)
 
 
 def test_every_solver_is_accepted_by_the_step_config(sb):
     """Each solver id of the header passes the step's argument checks (sizes
     are queried without a GPU); an unknown id is refused."""
-    for solver in (sb.SOLVER_NEWTON, sb.SOLVER_NEWTON_DB, sb.SOLVER_NEWTON_CUBIC):
+    for solver in (sb.SOLVER_NEWTON, sb.SOLVER_NEWTON_DB, sb.SOLVER_NEWTON_CUBIC, sb.SOLVER_NEWTON_CUBIC_F64):
         state, scratch = sb.query_sizes(sb.make_config(256, 0.95, 1e-8, 1e-3, solver=solver), [(1024, 1024)])
         assert state > 0 and scratch > 0
     with pytest.raises(sb.ShampooError):
-        sb.query_sizes(sb.make_config(256, 0.95, 1e-8, 1e-3, solver=4), [(1024, 1024)])
+        sb.query_sizes(sb.make_config(256, 0.95, 1e-8, 1e-3, solver=5), [(1024, 1024)])
 
 
 def test_init_rejects_missing_buffers_without_cuda(sb):

@@ -1,0 +1,158 @@
+"""fp64 iterates (SOLVER_NEWTON_CUBIC_F64) and their fp64 product.
+
+The fp32-accurate solvers miss the exact root by about (1/p) 2^-24 kappa (the
+plateau at kappa >= 1e6).  The fp64-iterate solver runs the same iteration
+(scale, damping eps_eff = max(eps, 2^-24 ||A + eps I||_F), stopping rule) in
+fp64, so its output must be the exact root of the damped fp32 input,
+sym(A) + eps_eff I, to the rounding of the fp32 output: gated here at 1e-6
+relative Frobenius at every condition number up to 1e8, against the oracle's
+eigendecomposition root of that damped matrix (DASH abstract: inverse matrix
+roots of the preconditioner blocks; the iteration is the reading of the
+Newton family).
+
+The product itself (``shampoo_dgemm_batched``) is checked against float64
+products: a few ulps of fp64 (1e-13), bit-exact on small integers.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle
+import workloads
+from parity import apply_check, effective_eps
+
+TOL_DGEMM = 1e-13
+TOL_ROOT_F64 = 1e-6
+
+
+@pytest.fixture(scope="module")
+def sb():
+    import shampoo_family_second_b200 as sb
+    return sb
+
+
+def rel(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+@pytest.mark.parametrize("n", [16, 32, 96, 256, 1024])
+def test_dgemm_matches_float64(sb, n):
+    rng = np.random.default_rng(100 + n)
+    batch = 3
+    A = rng.standard_normal((batch, n, n))
+    B = rng.standard_normal((batch, n, n))
+    D, status = sb.dgemm_batched(torch.from_numpy(A).cuda(), torch.from_numpy(B).cuda())
+    D = D.cpu().numpy()
+    for i in range(batch):
+        assert rel(D[i], A[i] @ B[i]) < TOL_DGEMM, (n, i, rel(D[i], A[i] @ B[i]))
+    assert int(status.item()) == 0
+
+
+def test_dgemm_epilogue_and_layout(sb):
+    """alpha, beta, gamma with C the output itself; small-integer operands make
+    every product exact, so a transposed fragment or a swapped operand shows
+    as a bit difference."""
+    rng = np.random.default_rng(9)
+    n, batch = 160, 2   # 2.5 tiles of 64: a ragged last tile row and column
+    A = rng.integers(-8, 9, (batch, n, n)).astype(np.float64)
+    B = rng.integers(-8, 9, (batch, n, n)).astype(np.float64)
+    C = rng.integers(-8, 9, (batch, n, n)).astype(np.float64)
+    Ct = torch.from_numpy(C.copy()).cuda()
+    D, status = sb.dgemm_batched(torch.from_numpy(A).cuda(), torch.from_numpy(B).cuda(), Ct, alpha=-0.5, beta=0.75,
+                                 gamma=2.0, out=Ct)
+    D = D.cpu().numpy()
+    for i in range(batch):
+        ref = -0.5 * (A[i] @ B[i]) + 0.75 * C[i] + 2.0 * np.eye(n)
+        assert np.array_equal(D[i], ref)
+    assert int(status.item()) == 0
+
+
+def exact_damped_root(A32, p, eps):
+    """The oracle's root of sym(A) + eps_eff I, eps_eff the solvers' damping."""
+    A64 = np.asarray(A32, dtype=np.float64)
+    e = effective_eps(A64, eps)
+    return oracle.inverse_root(0.5 * (A64 + A64.T) + e * np.eye(A64.shape[0]), p, 0.0)
+
+
+@pytest.mark.parametrize("n,batch", [(64, 4), (256, 3), (1024, 2)])
+@pytest.mark.parametrize("p", [2, 4])
+@pytest.mark.parametrize("kappa", [1e2, 1e6, 1e8])
+def test_f64_iterates_give_the_exact_root(sb, n, batch, p, kappa):
+    A32 = workloads.spd_batch(batch, n, kappa, seed=7 * n + p).astype(np.float32)
+    X, it, st = sb.inv_root_batched(torch.from_numpy(A32).cuda(), p=p, eps=0.0, solver=sb.SOLVER_NEWTON_CUBIC_F64,
+                                    iters=40, tol=1e-12)
+    torch.cuda.synchronize()
+    st = int(st.item())
+    it = it.cpu().numpy()
+    X = X.cpu().numpy().astype(np.float64)
+    assert st & ~sb.DEVFLAG_STAGNATED == 0, st
+    assert np.all(np.abs(it) >= 1) and np.all(np.abs(it) < 40), it
+    errs = []
+    for b in range(batch):
+        e = oracle.rel_fro(X[b], exact_damped_root(A32[b], p, 0.0))
+        errs.append(e)
+        assert e < TOL_ROOT_F64, (b, e)
+    print(f"\nfp64 iterates {batch}x{n}^2 kappa {kappa:.0e} p {p}: worst {max(errs):.1e}, "
+          f"iterations {np.abs(it).min()}-{np.abs(it).max()}")
+
+
+def test_f64_fixed_count_and_graph_loop(sb):
+    """Fixed iteration counts and the residual-checked graph loop agree with
+    plain launches (profiling on) bit for bit."""
+    A32 = workloads.spd_batch(5, 192, 1e5, seed=77).astype(np.float32)
+    At = torch.from_numpy(A32).cuda()
+    X0, it0, st0 = sb.inv_root_batched(At, p=4, eps=1e-6, solver=sb.SOLVER_NEWTON_CUBIC_F64, iters=25, tol=0.0)
+    kw = dict(p=4, eps=1e-6, solver=sb.SOLVER_NEWTON_CUBIC_F64, iters=40, tol=1e-12)
+    sb.profile_enable(True)
+    try:
+        X1, it1, st1 = sb.inv_root_batched(At, **kw)
+        torch.cuda.synchronize()
+    finally:
+        sb.profile_enable(False)
+    X2, it2, st2 = sb.inv_root_batched(At, **kw)
+    torch.cuda.synchronize()
+    assert int(st0.item()) == 0 and np.all(it0.cpu().numpy() == 25)
+    assert int(st1.item()) == int(st2.item())
+    assert np.array_equal(it1.cpu().numpy(), it2.cpu().numpy())
+    assert torch.equal(X1, X2)
+    for b in range(5):
+        ref = exact_damped_root(A32[b], 4, 1e-6)
+        assert oracle.rel_fro(X0[b].cpu().numpy().astype(np.float64), ref) < TOL_ROOT_F64
+        assert oracle.rel_fro(X2[b].cpu().numpy().astype(np.float64), ref) < TOL_ROOT_F64
+
+
+@pytest.mark.parametrize("shapes", [[(64, 32)], [(100, 45), (33, 96)]])
+def test_f64_iterates_in_the_step(sb, shapes):
+    """The blocked step with fp64 iterates: on every refresh the roots equal
+    the exact roots of the GPU's own damped fp32 statistics over the whole
+    block, null space included (with fp64 iterates the damping alone fixes the
+    null-space root), and the update equals the float64 product of those
+    roots and the gradient (the apply stage)."""
+    wl = workloads.workload("tiny", shapes=tuple(shapes), block=32, beta=0.9, eps=1e-4, lr=1e-3,
+                            solver=4, iters=40, tol=1e-12, refresh_every=2)
+    cfg = sb.config_from_workload(wl)
+    opt = sb.Shampoo(wl.shapes, cfg)
+    W = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    table = [tuple(t) for t in opt.block_table()]
+    stream = workloads.GradientStream(wl)
+    worst = 0.0
+    for t in range(5):
+        grads = stream.next()
+        before = [w.clone() for w in W]
+        opt.step(W, [torch.from_numpy(g).cuda() for g in grads])
+        torch.cuda.synchronize()
+        L, R = [x.cpu().numpy() for x in opt.statistics()]
+        XL, XR = [x.cpu().numpy().astype(np.float64) for x in opt.roots()]
+        for b, (param, r0, c0, r, c) in enumerate(table):
+            if t % wl.refresh_every == 0:
+                for X, S, v in ((XL, L, r), (XR, R, c)):
+                    e = oracle.rel_fro(X[b, :v, :v], exact_damped_root(S[b, :v, :v], wl.root_p, wl.eps))
+                    worst = max(worst, e)
+                    assert e < TOL_ROOT_F64, (t, b, e)
+            Pg = ((before[param] - W[param]).double() / wl.lr).cpu().numpy()[r0:r0 + r, c0:c0 + c]
+            ea, ga = apply_check(Pg, XL[b, :r, :r], grads[param][r0:r0 + r, c0:c0 + c], XR[b, :c, :c])
+            assert ea < ga, (t, b, ea, ga)
+    assert opt.status() & ~sb.DEVFLAG_STAGNATED == 0
+    print(f"\nfp64 iterates in the step {shapes}: worst root {worst:.1e}")

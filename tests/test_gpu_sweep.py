@@ -28,6 +28,10 @@ coupled-Newton family is the reading of the Newton iterations):
   eps_eff = max(eps, 2^-24 ||A + eps I||_F)), 2e-3; its distance to the exact
   root is a property of the degree.
 
+* coupled Newton with fp64 iterates (tol 1e-12): against the exact root of
+  the damped input sym(A) + eps_eff I it computes, at 1e-6 for every kappa
+  (its error against the undamped root is reported beside it).
+
 p in {2, 4} throughout.  The device status may only carry STAGNATED (a
 residual held up by fp32 rounding above tol), never NOT_CONVERGED.
 """
@@ -43,7 +47,8 @@ import workloads
 from parity import BASE_TOL, effective_eps, root_gate
 
 SOLVERS = (("newton", 0, 0), ("newton_cubic", 3, 0), ("newton_db", 1, 0), ("chebyshev16", 2, 16),
-           ("chebyshev32", 2, 32))
+           ("chebyshev32", 2, 32), ("newton_cubic_f64", 4, 0))
+TOL_F64 = 1e-6
 CAP, TOL_RES = 40, 1e-5
 
 
@@ -78,7 +83,8 @@ def test_sweep_case(sb, batch, n, kappa):
                 lo = 0.999 / kappa
                 X, it, st = sb.inv_root_batched(A, p=p, eps=0.0, solver=2, cheb_degree=degree, cheb_lo=lo)
             else:
-                X, it, st = sb.inv_root_batched(A, p=p, eps=0.0, solver=solver, iters=CAP, tol=TOL_RES)
+                X, it, st = sb.inv_root_batched(A, p=p, eps=0.0, solver=solver, iters=CAP,
+                                                tol=1e-12 if solver == 4 else TOL_RES)
             torch.cuda.synchronize()
             st = int(st.item())
             it = it.cpu().numpy()
@@ -96,6 +102,11 @@ def test_sweep_case(sb, batch, n, kappa):
                     ref = och.chebyshev_inverse_root(A64, p, effective_eps(A64, 0.0), degree, lo=lo)
                     e, gate = oracle.rel_fro(Xs, ref), BASE_TOL
                     e_exact = oracle.rel_fro(Xs, exact[p, s])
+                elif solver == 4:
+                    # fp64 iterates: the exact root of the damped input itself
+                    damped = 0.5 * (A64 + A64.T) + effective_eps(A64, 0.0) * np.eye(n)
+                    e, gate = oracle.rel_fro(Xs, oracle.inverse_root(damped, p, 0.0)), TOL_F64
+                    e_exact = oracle.rel_fro(Xs, exact[p, s])
                 else:
                     e, gate = oracle.rel_fro(Xs, exact[p, s]), gates[p, s]
                     e_exact = e
@@ -103,5 +114,6 @@ def test_sweep_case(sb, batch, n, kappa):
                 assert e < gate, (name, p, s, e, gate)
         del X
     print(f"\nsweep {batch}x{n}^2 kappa {kappa:.0e}: " + "; ".join(
-        f"{nm} p{p} #{s}: {e:.1e}/{g:.1e}" + (f" (exact-root {ex:.1e})" if nm.startswith("cheb") else f" it {k}")
+        f"{nm} p{p} #{s}: {e:.1e}/{g:.1e}" + (f" (exact-root {ex:.1e})" if nm.startswith("cheb") or nm.endswith("f64")
+                                              else "") + ("" if nm.startswith("cheb") else f" it {k}")
         for nm, p, s, e, g, ex, k in report))
