@@ -644,7 +644,8 @@ def run_reference(args, wl):
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "inverse-roots/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(timed) / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD_NAMES.get(wl.name, wl.name), "block": wl.block,
                    "refresh_every": wl.refresh_every, "sampled_blocks": len(blocks), "blocks": nb},
         "cpu_baseline": {"value": value, "unit": "inverse-roots/s", "cores": cores, "kind": "oracle",

@@ -87,7 +87,12 @@ enum {
                                      output, for statistics whose condition number puts the
                                      fp32 iterates' error ((1/p) 2^-24 kappa) above tolerance;
                                      scratch holds fp64 stacks (twice the bytes), and the
-                                     products run at the fp64 rate */
+                                     products run at the fp64 rate.  In the blocked step it
+                                     also keeps L and R in fp64 (their products on the fp64
+                                     MMA, the gradients widened exactly; Frobenius scaling;
+                                     damping floor n 2^-53 ||L + eps I||_F): with fp32
+                                     statistics the update's error floor would stay that of
+                                     fp32 rounding whatever the iterates' precision */
 };
 
 /* Gradient element types. */
@@ -208,8 +213,10 @@ SHAMPOO_API int shampoo_get_status(shampoo_handle h, int32_t* status, int32_t re
 SHAMPOO_API int shampoo_block_table(shampoo_handle h, int32_t* nb, int64_t* table);
 
 /* Device pointers into the state (owned by the caller's state buffer):
- * L: plain stack (nb, B, B) of left statistics; R: (nb, B, B) right statistics;
- * rootL / rootR: (nb, B, B) stacks of XL and XR; *step: steps taken.
+ * L: plain stack (nb, B, B) of left statistics; R: (nb, B, B) right statistics
+ * (fp32; fp64 values behind the float pointers when cfg.solver is
+ * SHAMPOO_SOLVER_NEWTON_CUBIC_F64); rootL / rootR: (nb, B, B) fp32 stacks of
+ * XL and XR; *step: steps taken.
  * Ragged blocks hold zeros outside their r x r / c x c valid region. */
 SHAMPOO_API int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, float** rootR, int64_t* step);
 

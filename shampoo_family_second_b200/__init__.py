@@ -326,14 +326,19 @@ class Shampoo:
         return self._views()[1]
 
     def statistics(self):
-        """(L, R) as float32 views (nb, B, B) into the state buffer."""
+        """(L, R) as views (nb, B, B) into the state buffer: float32, or float64
+        with the fp64-iterate solver (which keeps the statistics in fp64)."""
         import torch
         (pl, pr, _, _), _ = self._views()
         B, nb = self.cfg.block, self.nb
         base = self.state.data_ptr()
-        fl = self.state.view(torch.float32) if (self.state_bytes % 4 == 0) else None
-        L = fl[(pl - base) // 4:(pl - base) // 4 + nb * B * B].view(nb, B, B)
-        R = fl[(pr - base) // 4:(pr - base) // 4 + nb * B * B].view(nb, B, B)
+        if self.cfg.solver == SOLVER_NEWTON_CUBIC_F64:
+            dt, es = torch.float64, 8
+        else:
+            dt, es = torch.float32, 4
+        fl = self.state[:self.state_bytes - self.state_bytes % es].view(dt)
+        L = fl[(pl - base) // es:(pl - base) // es + nb * B * B].view(nb, B, B)
+        R = fl[(pr - base) // es:(pr - base) // es + nb * B * B].view(nb, B, B)
         return L, R
 
     def roots(self):

@@ -83,12 +83,17 @@ int build_table(int B, int32_t nparams, const int64_t* rows, const int64_t* cols
 
 // State layout (bytes, each part 256-aligned):
 //   status word | block table (nb x 5 int32) | valid extents (2nb int32: r of L_b, c of R_b)
-//   | wrows (nb) | wcols (nb) | statistics (2nb, B, B) | roots (2nb, B, B)
+//   | wrows (nb) | wcols (nb) | statistics (2nb, B, B; fp64 with the fp64-iterate solver) | roots (2nb, B, B)
 //   | momentum (nb, B, B; only with momentum > 0) | power flag | power iterates (2nb, B)
+// Bytes per statistics element: the fp64-iterate solver keeps L and R in
+// fp64 in the blocked step (fp32 statistics would set the update's error
+// floor whatever the iterates' precision).
+size_t stats_elem_bytes(int solver) { return solver == SHAMPOO_SOLVER_NEWTON_CUBIC_F64 ? 8 : 4; }
+
 struct StateLayout {
   size_t status, table, valid, wrows, wcols, stats, roots, mom, pflag, pvec, total;
 };
-StateLayout state_layout(int nb, int B, bool momentum) {
+StateLayout state_layout(int nb, int B, bool momentum, size_t stats_elem) {
   StateLayout s;
   size_t o = 0;
   s.status = o, o += al(4);
@@ -96,7 +101,7 @@ StateLayout state_layout(int nb, int B, bool momentum) {
   s.valid = o, o += al(size_t(2) * nb * 4);
   s.wrows = o, o += al(size_t(nb) * 4);
   s.wcols = o, o += al(size_t(nb) * 4);
-  s.stats = o, o += al(plain_floats(2 * nb, B) * 4);
+  s.stats = o, o += al(plain_floats(2 * nb, B) * stats_elem);
   s.roots = o, o += al(plain_floats(2 * nb, B) * 4);
   s.mom = o;
   if (momentum) o += al(plain_floats(nb, B) * 4);
@@ -165,6 +170,7 @@ struct shampoo_ctx {
   double stats_flops_L = 0, stats_flops_R = 0, stack_bytes = 0;
   int64_t step = 0;
   int power_refreshed = 0;  // a refresh has stored power iterates (profiler byte count only)
+  bool stats_f64 = false;   // L, R kept in fp64 (fp64-iterate solver)
   cudaStream_t last_stream = nullptr;
 };
 
@@ -189,7 +195,7 @@ int shampoo_query_sizes(const shampoo_config* cfg, int32_t nparams, const int64_
   Shapes sh;
   if ((rc = build_table(cfg->block, nparams, rows, cols, sh))) return rc;
   if (!state_bytes || !scratch_bytes) return set_error(SHAMPOO_ERR_INVALID_ARG, "output pointer is NULL");
-  *state_bytes = state_layout(sh.nb, cfg->block, cfg->momentum > 0.f).total;
+  *state_bytes = state_layout(sh.nb, cfg->block, cfg->momentum > 0.f, stats_elem_bytes(cfg->solver)).total;
   *scratch_bytes = scratch_layout(sh.nb, cfg->block, cfg->solver, cfg->root_p).total;
   return SHAMPOO_OK;
 }
@@ -206,7 +212,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
   if (!aligned256(d_state) || !aligned256(d_scratch))
     return set_error(SHAMPOO_ERR_UNSUPPORTED, "state/scratch must be 256-byte aligned");
   const int B = cfg->block, nb = sh.nb;
-  StateLayout sl = state_layout(nb, B, cfg->momentum > 0.f);
+  StateLayout sl = state_layout(nb, B, cfg->momentum > 0.f, stats_elem_bytes(cfg->solver));
   ScratchLayout xl = scratch_layout(nb, B, cfg->solver, cfg->root_p);
   if (state_bytes < sl.total) return set_error(SHAMPOO_ERR_WORKSPACE, "state %zu < %zu bytes", state_bytes, sl.total);
   if (scratch_bytes < xl.total)
@@ -229,6 +235,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
   h->d_wrows = reinterpret_cast<int*>(h->state + sl.wrows);
   h->d_wcols = reinterpret_cast<int*>(h->state + sl.wcols);
   h->stats = reinterpret_cast<float*>(h->state + sl.stats);
+  h->stats_f64 = cfg->solver == SHAMPOO_SOLVER_NEWTON_CUBIC_F64;
   h->roots = reinterpret_cast<float*>(h->state + sl.roots);
   h->mom = cfg->momentum > 0.f ? reinterpret_cast<float*>(h->state + sl.mom) : nullptr;
   h->Gs = reinterpret_cast<float*>(h->scratch + xl.gs);
@@ -262,7 +269,8 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
   if ((rc = up(h->d_table, sh.table.data(), sh.table.size() * 4)) || (rc = up(h->d_valid, valid.data(), valid.size() * 4)) ||
       (rc = up(h->d_wrows, wr.data(), wr.size() * 4)) || (rc = up(h->d_wcols, wc.data(), wc.size() * 4)) ||
       (rc = check_cuda(cudaMemsetAsync(h->d_status, 0, 4, st), "zero status")) ||
-      (rc = check_cuda(cudaMemsetAsync(h->stats, 0, plain_floats(2 * nb, B) * 4, st), "zero statistics")) ||
+      (rc = check_cuda(cudaMemsetAsync(h->stats, 0, plain_floats(2 * nb, B) * stats_elem_bytes(cfg->solver), st),
+                       "zero statistics")) ||
       (rc = check_cuda(cudaMemsetAsync(h->roots, 0, plain_floats(2 * nb, B) * 4, st), "zero roots")) ||
       (h->mom && (rc = check_cuda(cudaMemsetAsync(h->mom, 0, plain_floats(nb, B) * 4, st), "zero momentum"))) ||
       (rc = check_cuda(cudaMemsetAsync(h->state + sl.pflag, 0, sl.total - sl.pflag, st), "zero power store")) ||
@@ -331,7 +339,28 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
       e.flags = h->d_status;
     }
   };
-  {
+  if (h->stats_f64) {
+    // fp64 statistics: L <- beta L + Gs Gt and R <- beta R + Gt Gs (Gt = Gs^T,
+    // true products) on the fp64 MMA, the fp32 stacks widened exactly
+    double* L64 = reinterpret_cast<double*>(h->stats);
+    DGemmGroup g[2];
+    g[0].A = h->Gs;
+    g[0].B = h->Gt;
+    g[0].C = L64;
+    g[0].D = L64;
+    g[0].beta = c.beta;
+    g[1].A = h->Gt;
+    g[1].B = h->Gs;
+    g[1].C = L64 + plain_floats(nb, B);
+    g[1].D = L64 + plain_floats(nb, B);
+    g[1].beta = c.beta;
+    if ((rc = launch_dgemm(g, 2, nb, B, nullptr, nullptr, h->d_status, st, true))) return rc;
+    if (!refresh) {
+      Builder b;
+      add_apply1(b);
+      if ((rc = b.launch(st))) return rc;
+    }
+  } else {
     Builder b;
     Epilogue& eL = b.add(nb, B, h->mGs, 0, h->mGs, 0, h->stats_flops_L);
     b.L.g[0].a_exact = b.L.g[0].b_exact = g_exact;
@@ -363,13 +392,16 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
     job.eps = c.eps;
     job.tol = c.tol;
     job.cheb_lo = c.cheb_lo;
-    job.A = h->stats;
+    job.A = h->stats_f64 ? nullptr : h->stats;
+    job.A64 = h->stats_f64 ? reinterpret_cast<const double*>(h->stats) : nullptr;
     job.valid = h->d_valid;
     job.X = h->roots;
     job.iters_used = nullptr;
     job.flags = h->d_status;
-    job.power_vec = reinterpret_cast<float*>(h->state + h->sl.pvec);
-    job.power_warm = reinterpret_cast<int*>(h->state + h->sl.pflag);
+    if (!h->stats_f64) {  // fp64 statistics are scaled by their Frobenius norm
+      job.power_vec = reinterpret_cast<float*>(h->state + h->sl.pvec);
+      job.power_warm = reinterpret_cast<int*>(h->state + h->sl.pflag);
+    }
     job.power_warm_hint = h->power_refreshed;
     if ((rc = run_inverse_roots(job, h->scratch + h->xl.root, h->xl.root_bytes, st))) return rc;
     h->power_refreshed = 1;

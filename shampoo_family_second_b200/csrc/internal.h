@@ -232,8 +232,8 @@ int launch_mirror_lower(float* D, int64_t batch, int n, cudaStream_t st);
 // optionally E = e_mul D + e_add I and res[m] += sum over the valid diagonal
 // of (1 - D).  C may be D itself; A and B must not be written by the launch.
 struct DGemmGroup {
-  const double* A = nullptr;
-  const double* B = nullptr;
+  const void* A = nullptr;  // double, or float with f32_operands (widened exactly)
+  const void* B = nullptr;
   const double* C = nullptr;
   double* D = nullptr;
   double* E = nullptr;
@@ -241,7 +241,10 @@ struct DGemmGroup {
   float* res = nullptr;
 };
 int launch_dgemm(const DGemmGroup* groups, int ngroups, int64_t batch, int n, const int* valid, const int* skip,
-                 int* flags, cudaStream_t st);
+                 int* flags, cudaStream_t st, bool f32_operands = false);
+// s = sf = ||A + eps I||_F (valid block) of fp64 matrices.
+int launch_frob_f64(const double* A, int64_t batch, int n, const int* valid, float eps, float* s, float* sf,
+                    cudaStream_t st);
 // M0 = (sym(A) + eps_eff I)/s (identity on the padding), T = ((p+1) I - M0)/p,
 // X1 = T; eps_eff = max(eps, eps_floor_rel * sf).  A is fp32 or (a_is_f64) fp64.
 int launch_prologue_f64(const void* A, int a_is_f64, int64_t batch, int n, const int* valid, float eps,
@@ -266,6 +269,8 @@ struct RootJob {
   float* power_vec = nullptr;  // coupled Newton's scale: per-matrix power-iterate store (batch x n), or NULL
   int* power_warm = nullptr;   // device flag: power_vec holds the previous refresh's iterates
   int power_warm_hint = 0;     // host's view of that flag, used only for the profiler's byte count
+  const double* A64 = nullptr;  // fp64 input stack instead of A (fp64-iterate solver only): scaled by
+                                // its Frobenius norm and damped at the fp64 statistics' rounding
 };
 // inv_root_batched with a switch for plain launches (shared by the public
 // entry points of api.cu and noalloc.cu).

@@ -291,20 +291,25 @@ size_t root_scratch_per_matrix(int n, int solver, int p) {
 int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, cudaStream_t st) {
   const int n = job.n;
   const int p = job.p;
+  if (job.A64 && job.solver != 4) return set_error(-1, "fp64 input needs the fp64-iterate solver");
   const bool residual = job.tol > 0.f && job.solver != 2;
   const size_t per = root_scratch_per_matrix(n, job.solver, p);
   if (scratch_bytes < kHeader + per)
     return set_error(-3, "inverse-root scratch too small: %zu < %zu bytes", scratch_bytes, kHeader + per);
   const int64_t cb_max = std::min<int64_t>(job.batch, static_cast<int64_t>((scratch_bytes - kHeader) / per));
-  // grid.z limit of the prologues (and of the fp64 GEMM's two groups)
-  const int64_t cb_cap = std::min<int64_t>(cb_max, job.solver == 4 ? 32767 : 65535);
+  // grid.z limit of the prologues (and of the fp64 GEMM's two groups); the
+  // chunks are then balanced, so that no last chunk runs a few matrices alone
+  const int64_t cb_lim = std::min<int64_t>(cb_max, job.solver == 4 ? 32767 : 65535);
+  const int64_t nchunks = (job.batch + cb_lim - 1) / cb_lim;
+  const int64_t cb_cap = (job.batch + nchunks - 1) / nchunks;
   const double f1 = 2.0 * n * static_cast<double>(n) * n;  // one GEMM(n), algorithmic
   int rc = 0;
   for (int64_t off = 0; off < job.batch; off += cb_cap) {
     const int64_t cb = std::min<int64_t>(cb_cap, job.batch - off);
     const int cbi = static_cast<int>(cb);
     Layout S = carve(scratch, cb, n, job.solver, p);
-    const float* A = job.A + off * static_cast<int64_t>(n) * n;
+    const float* A = job.A ? job.A + off * static_cast<int64_t>(n) * n : nullptr;
+    const double* A64 = job.A64 ? job.A64 + off * static_cast<int64_t>(n) * n : nullptr;
     const int* valid = job.valid ? job.valid + off : nullptr;
     float* out = job.X + off * static_cast<int64_t>(n) * n;
     int* iters_out = job.iters_used ? job.iters_used + off : nullptr;
@@ -315,7 +320,9 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
     // Coupled Newton scales by the power-iteration estimate (bounded by the
     // Frobenius norm); Newton-DB (convergent only on (0, 2)) and Chebyshev
     // (an exact upper bound is needed) by the Frobenius norm.
-    if (job.solver == 0 || job.solver == 3 || job.solver == 4) {
+    if (A64) {
+      if ((rc = launch_frob_f64(A64, cb, n, valid, job.eps, S.s, S.sf, st))) return rc;
+    } else if (job.solver == 0 || job.solver == 3 || job.solver == 4) {
       float* pv = job.power_vec ? job.power_vec + off * n : nullptr;
       // one flag for all chunks: read by every chunk's scale kernel, set by the
       // last chunk's root prologue
@@ -384,10 +391,14 @@ int run_inverse_roots(const RootJob& job, void* scratch, size_t scratch_bytes, c
       double* Tp = reinterpret_cast<double*>(S.stack[7]);
       const double c1 = 1.0 / p, c2 = (p + 1.0) / (2.0 * p * p);
       int* set_flag = (job.power_vec && job.power_warm && off + cb == job.batch) ? job.power_warm : nullptr;
-      // fp32 input: the damping floor is the fp32 rounding of A (2^-24 ||A + eps I||_F, as
-      // for the fp32 solvers), below which the input itself may be indefinite
-      if ((rc = launch_prologue_f64(A, 0, cb, n, valid, job.eps, 5.9604645e-8f, p, S.s, S.sf, Mb[0], Q[0], Xb[1],
-                                    set_flag, st)))
+      // The damping floor is the input's own rounding, below which it may be
+      // indefinite: 2^-24 ||A + eps I||_F for fp32 input (as for the fp32
+      // solvers); for fp64 statistics n 2^-53 ||A + eps I||_F, the size of
+      // their accumulated rounding
+      const float floor_rel = A64 ? static_cast<float>(n * 1.1102230246251565e-16) : 5.9604645e-8f;
+      if ((rc = launch_prologue_f64(A64 ? static_cast<const void*>(A64) : static_cast<const void*>(A), A64 ? 1 : 0,
+                                    cb, n, valid, job.eps, floor_rel, p, S.s, S.sf, Mb[0], Q[0], Xb[1], set_flag,
+                                    st)))
         return rc;
       auto dg = [](const double* a, const double* b, double* d) {
         DGemmGroup g;

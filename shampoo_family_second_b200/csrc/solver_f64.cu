@@ -29,11 +29,15 @@ constexpr int kDT = 64;                 // CTA tile: 64 x 64 outputs
 constexpr int kDK = 16;                 // K per stage
 constexpr int kDStages = 3;
 constexpr int kDThreads = 128;          // 4 warps, 2 x 2 quarters of 32 x 32
-constexpr int kAStride = kDK + 4;       // doubles per A row in shared memory
-constexpr int kBStride = kDT + 8;       // doubles per B row
-constexpr int kAStage = kDT * kAStride; // doubles per A stage
+constexpr int kAStride = kDK + 4;       // elements per A row in shared memory
+constexpr int kBStride = kDT + 8;       // elements per B row
+constexpr int kAStage = kDT * kAStride; // elements per A stage
 constexpr int kBStage = kDK * kBStride;
-constexpr size_t kDSmem = sizeof(double) * kDStages * (kAStage + kBStage);
+// Operands are fp64, or fp32 widened exactly when fragments are loaded (the
+// statistics of fp32 / bf16 gradient stacks).  Both paddings keep every
+// fragment load at the minimum number of shared-memory wavefronts.
+template <class TIn>
+constexpr size_t dsmem_bytes() { return sizeof(TIn) * kDStages * (kAStage + kBStage); }
 
 struct DArgs {
   DGemmGroup g[2];
@@ -65,6 +69,7 @@ __device__ __forceinline__ void dmma8x8x4(double (&d)[2], double a, double b) {
 
 // grid (ceil(n/64), ceil(n/64), ngroups * batch), block 128.  Every operand is
 // a row-major n x n matrix; the product is the true product A B.
+template <class TIn>
 __global__ void __launch_bounds__(kDThreads) dgemm_kernel(DArgs args) {
   const int z = blockIdx.z;
   const int gi = z / args.batch, m = z - gi * args.batch;
@@ -72,36 +77,41 @@ __global__ void __launch_bounds__(kDThreads) dgemm_kernel(DArgs args) {
   const DGemmGroup& G = args.g[gi];
   const int n = args.n;
   const size_t nn = static_cast<size_t>(n) * n;
-  const double* A = G.A + m * nn;
-  const double* B = G.B + m * nn;
+  const TIn* A = static_cast<const TIn*>(G.A) + m * nn;
+  const TIn* B = static_cast<const TIn*>(G.B) + m * nn;
   const int row0 = blockIdx.y * kDT, col0 = blockIdx.x * kDT;
 
-  extern __shared__ __align__(16) double dsm[];
-  double* As = dsm;
-  double* Bs = dsm + kDStages * kAStage;
+  extern __shared__ __align__(16) unsigned char dsm_raw[];
+  TIn* As = reinterpret_cast<TIn*>(dsm_raw);
+  TIn* Bs = As + kDStages * kAStage;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int wm = warp >> 1, wn = warp & 1;
+  constexpr int kPer = 16 / sizeof(TIn);      // elements per 16-byte piece
+  constexpr int kAPieces = kDK / kPer;        // pieces per A row (8 fp64, 4 fp32)
+  constexpr int kBPieces = kDT / kPer;        // pieces per B row (32 fp64, 16 fp32)
+  constexpr int kLoads = kDT * kAPieces / kDThreads;  // per thread and operand (4 fp64, 2 fp32)
+  static_assert(kDK * kBPieces == kDT * kAPieces, "A and B stages have the same number of pieces");
 
   auto load_stage = [&](int stage, int kt) {
     const int k0 = kt * kDK;
-    double* as = As + stage * kAStage;
-    double* bs = Bs + stage * kBStage;
+    TIn* as = As + stage * kAStage;
+    TIn* bs = Bs + stage * kBStage;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int idx = tid + q * kDThreads;  // 512 pieces of 16 bytes: 64 rows x 8
-      const int r = idx >> 3, c = idx & 7;
+    for (int q = 0; q < kLoads; ++q) {
+      const int idx = tid + q * kDThreads;  // 64 rows x kAPieces
+      const int r = idx / kAPieces, c = idx % kAPieces;
       const bool ok = row0 + r < n;
-      const double* src = ok ? A + static_cast<size_t>(row0 + r) * n + k0 + 2 * c : A;
-      cp_async16(as + r * kAStride + 2 * c, src, ok);
+      const TIn* src = ok ? A + static_cast<size_t>(row0 + r) * n + k0 + kPer * c : A;
+      cp_async16(as + r * kAStride + kPer * c, src, ok);
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int idx = tid + q * kDThreads;  // 16 rows x 32 pieces
-      const int k = idx >> 5, c = idx & 31;
-      const bool ok = col0 + 2 * c < n;
-      const double* src = ok ? B + static_cast<size_t>(k0 + k) * n + col0 + 2 * c : B;
-      cp_async16(bs + k * kBStride + 2 * c, src, ok);
+    for (int q = 0; q < kLoads; ++q) {
+      const int idx = tid + q * kDThreads;  // 16 rows x kBPieces
+      const int k = idx / kBPieces, c = idx % kBPieces;
+      const bool ok = col0 + kPer * c < n;
+      const TIn* src = ok ? B + static_cast<size_t>(k0 + k) * n + col0 + kPer * c : B;
+      cp_async16(bs + k * kBStride + kPer * c, src, ok);
     }
   };
 
@@ -124,15 +134,15 @@ __global__ void __launch_bounds__(kDThreads) dgemm_kernel(DArgs args) {
     __syncthreads();  // stage kt landed for every thread; stage kt - 1 is free
     if (kt + kDStages - 1 < KT) load_stage((kt + kDStages - 1) % kDStages, kt + kDStages - 1);
     cp_async_commit();
-    const double* as = As + (kt % kDStages) * kAStage;
-    const double* bs = Bs + (kt % kDStages) * kBStage;
+    const TIn* as = As + (kt % kDStages) * kAStage;
+    const TIn* bs = Bs + (kt % kDStages) * kBStage;
 #pragma unroll
     for (int kk = 0; kk < kDK; kk += 4) {
       double a[4], b[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = as[(ar + 8 * i) * kAStride + kk + ak];
+      for (int i = 0; i < 4; ++i) a[i] = static_cast<double>(as[(ar + 8 * i) * kAStride + kk + ak]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = bs[(kk + bk) * kBStride + bc + 8 * j];
+      for (int j = 0; j < 4; ++j) b[j] = static_cast<double>(bs[(kk + bk) * kBStride + bc + 8 * j]);
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -256,25 +266,66 @@ __global__ void finalize_f64_kernel(const double* __restrict__ X0, const double*
   if (bad) raise_flag(flags, DEV_FLAG_NONFINITE);
 }
 
+// Scale of an fp64 input: s = sf = ||A + eps I||_F over the valid block, an
+// upper bound of the largest eigenvalue, in fp64.  One CTA per matrix.
+__global__ void frob_f64_kernel(const double* __restrict__ A, int n, const int* __restrict__ valid, float eps,
+                                float* __restrict__ s, float* __restrict__ sf) {
+  const int i = blockIdx.x;
+  const int v = valid ? valid[i] : n;
+  const double* a = A + static_cast<size_t>(i) * n * n;
+  double acc = 0.0;
+  for (int r = threadIdx.y; r < v; r += blockDim.y)
+    for (int c = threadIdx.x; c < v; c += blockDim.x) {
+      const double x = a[static_cast<size_t>(r) * n + c] + (r == c ? static_cast<double>(eps) : 0.0);
+      acc += x * x;
+    }
+  __shared__ double part[32];
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  const int w = (threadIdx.y * blockDim.x + threadIdx.x) >> 5;
+  if ((threadIdx.x & 31) == 0) part[w] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0 && threadIdx.y == 0) {
+    double t = 0.0;
+    for (int k = 0; k < static_cast<int>(blockDim.x * blockDim.y / 32); ++k) t += part[k];
+    const float f = static_cast<float>(sqrt(t));
+    s[i] = f > 0.f ? f : 1.f;  // an all-zero block: any scale
+    sf[i] = f;
+  }
+}
+
 }  // namespace
 
+int launch_frob_f64(const double* A, int64_t batch, int n, const int* valid, float eps, float* s, float* sf,
+                    cudaStream_t st) {
+  if (batch == 0) return 0;
+  ProfScope ps(K_SCALE, st, 0.0, 8.0 * batch * n * n);
+  frob_f64_kernel<<<static_cast<unsigned>(batch), dim3(32, 16), 0, st>>>(A, n, valid, eps, s, sf);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "frob_f64_kernel");
+}
+
 int launch_dgemm(const DGemmGroup* groups, int ngroups, int64_t batch, int n, const int* valid, const int* skip,
-                 int* flags, cudaStream_t st) {
+                 int* flags, cudaStream_t st, bool f32_operands) {
   if (batch == 0) return 0;
   if (ngroups < 1 || ngroups > 2 || n % kDK != 0 || batch * ngroups > 65535)
     return set_error(SHAMPOO_ERR_INVALID_ARG, "dgemm: %d groups, n %d, batch %lld", ngroups, n,
                      static_cast<long long>(batch));
-  static bool attr_set[64] = {};  // per device
+  static bool attr_set[64][2] = {};  // per device and operand type
   int dev = 0;
   int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
   if (rc) return rc;
   if (dev < 0 || dev >= 64) return set_error(SHAMPOO_ERR_UNSUPPORTED, "device %d", dev);
-  if (!attr_set[dev]) {
-    rc = check_cuda(cudaFuncSetAttribute(dgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kDSmem)),
-                    "cudaFuncSetAttribute(dgemm_kernel)");
+  if (!attr_set[dev][f32_operands]) {
+    rc = f32_operands ? check_cuda(cudaFuncSetAttribute(dgemm_kernel<float>,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                        static_cast<int>(dsmem_bytes<float>())),
+                                   "cudaFuncSetAttribute(dgemm_kernel<float>)")
+                      : check_cuda(cudaFuncSetAttribute(dgemm_kernel<double>,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                        static_cast<int>(dsmem_bytes<double>())),
+                                   "cudaFuncSetAttribute(dgemm_kernel<double>)");
     if (rc) return rc;
-    attr_set[dev] = true;
+    attr_set[dev][f32_operands] = true;
   }
   DArgs a;
   for (int g = 0; g < ngroups; ++g) a.g[g] = groups[g];
@@ -285,9 +336,13 @@ int launch_dgemm(const DGemmGroup* groups, int ngroups, int64_t batch, int n, co
   a.skip = skip;
   a.flags = flags;
   const double flops = 2.0 * n * static_cast<double>(n) * n * batch * ngroups;
-  ProfScope ps(K_GEMM_F64, st, flops, 24.0 * n * static_cast<double>(n) * batch * ngroups);
+  ProfScope ps(K_GEMM_F64, st, flops, (f32_operands ? 24.0 : 32.0) * n * static_cast<double>(n) * batch * ngroups);
   const unsigned tiles = static_cast<unsigned>((n + kDT - 1) / kDT);
-  dgemm_kernel<<<dim3(tiles, tiles, static_cast<unsigned>(batch * ngroups)), kDThreads, kDSmem, st>>>(a);
+  const dim3 grid(tiles, tiles, static_cast<unsigned>(batch * ngroups));
+  if (f32_operands)
+    dgemm_kernel<float><<<grid, kDThreads, dsmem_bytes<float>(), st>>>(a);
+  else
+    dgemm_kernel<double><<<grid, kDThreads, dsmem_bytes<double>(), st>>>(a);
   count_launch();
   return check_cuda(cudaGetLastError(), "dgemm_kernel");
 }

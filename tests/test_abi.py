@@ -106,7 +106,7 @@ def test_scratch_sizes(sb):
     # the second-degree correction reuses the Newton stacks (T, T^2, T^4 also hold D = I - M)
     assert sb.inv_root_scratch_bytes(64, 1024, sb.SOLVER_NEWTON_CUBIC) == a
     assert sb.gemm_scratch_bytes(3, 256) == 0   # operands are split on chip
-    # the no-alloc entry point's fixed 32 MiB covers one matrix of every supported size
+    # the no-alloc entry point's fixed 32 MiB covers one matrix of every fp32 solver at every size
     for solver in (sb.SOLVER_NEWTON, sb.SOLVER_NEWTON_DB, sb.SOLVER_CHEBYSHEV, sb.SOLVER_NEWTON_CUBIC):
         assert sb.inv_root_scratch_bytes(1, 1024, solver) <= 32 << 20
     with pytest.raises(sb.ShampooError):

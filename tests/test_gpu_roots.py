@@ -250,3 +250,4 @@ def test_newton_db_refuses_higher_orders(sb):
     A = torch.zeros((1, 64, 64), device="cuda")
     with pytest.raises(sb.ShampooError):
         sb.inv_root_batched(A, p=6, solver=sb.SOLVER_NEWTON_DB)
+
