@@ -449,7 +449,9 @@ int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, f
   if (!h) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle is NULL");
   const int nb = h->shapes.nb, B = h->cfg.block;
   if (L) *L = h->stats;
-  if (R) *R = h->stats + plain_floats(nb, B);
+  if (R)  // R follows the nb L matrices, whose elements are fp64 with the fp64-iterate solver
+    *R = h->stats_f64 ? reinterpret_cast<float*>(reinterpret_cast<double*>(h->stats) + plain_floats(nb, B))
+                      : h->stats + plain_floats(nb, B);
   if (rootL) *rootL = h->roots;
   if (rootR) *rootR = h->roots + plain_floats(nb, B);
   if (step) *step = h->step;
