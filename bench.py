@@ -61,6 +61,18 @@ WORKLOAD_NAMES = {
     "soap": "soap_4x1024sq_b256",
     "tensor": "tensor_conv3x3_stack",
 }
+LLAMA_LAYER = 7  # weights per Llama layer (q, k, v, o, gate, up, down)
+
+
+def workload_label(wl):
+    """The workload's name; a Llama workload cut to fewer layers (--layers, for
+    small profiling captures) says so."""
+    name = WORKLOAD_NAMES.get(wl.name, wl.name)
+    if wl.name == "llama" and len(wl.shapes) != len(workloads.WORKLOADS["llama"].shapes):
+        name += f"_{len(wl.shapes) // LLAMA_LAYER}layers"
+    return name
+
+
 # Convolution kernels (3 x 3 x C_in x C_out) of a ResNet-style stack, for
 # order-4 tensor Shampoo: 4 stages of 4 kernels at 64 .. 512 channels.
 CONV_SHAPES = tuple((3, 3, c, c) for c in (64, 128, 256, 512) for _ in range(4))
@@ -442,7 +454,7 @@ def run_ours(args, wl):
         "dtype": "f32",
         "data": "synthetic",
         "config": {
-            "workload": WORKLOAD_NAMES.get(wl.name, wl.name),
+            "workload": workload_label(wl),
             "params": len(wl.shapes), "param_elems": wl.n_params, "block": wl.block, "blocks": nb,
             "roots_per_refresh": roots_per_refresh, "refresh_every": wl.refresh_every,
             "refresh_steps_timed": nref, "solver": SOLVER_NAMES[wl.solver], "root_p": wl.root_p,
@@ -538,7 +550,7 @@ def gemm_traffic_per_launch(wl):
     try:
         with open(path) as f:
             d = json.load(f)
-        if (d.get("source_sha256") != traffic_source_sha() or d.get("workload_key") != wl.name
+        if (d.get("source_sha256") != traffic_source_sha() or d.get("workload_key") != workload_label(wl)
                 or d.get("solver") != SOLVER_NAMES[wl.solver]):
             return None
         return d.get("bytes_per_launch")
@@ -884,6 +896,8 @@ def main():
     ap.add_argument("--solver", default=None, choices=sorted(SOLVER_IDS),
                     help="inverse-root solver of the step workloads (default: the workload's own)")
     ap.add_argument("--momentum", type=float, default=None, help="momentum ahead of the preconditioner (step workloads)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="Llama workload cut to its first N layers (small profiling captures; 0: all 16)")
     ap.add_argument("--sweep-n", type=int, default=512)
     ap.add_argument("--sweep-batch", type=int, default=0)
     ap.add_argument("--sweep-kappa", type=float, default=1e4)
@@ -915,6 +929,10 @@ def main():
         over["solver"] = SOLVER_IDS[args.solver]
     if args.momentum is not None:
         over["momentum"] = args.momentum
+    if args.layers:
+        if args.workload != "llama":
+            ap.error("--layers applies to the llama workload")
+        over["shapes"] = workloads.WORKLOADS["llama"].shapes[:LLAMA_LAYER * args.layers]
     wl = workloads.workload(args.workload, **over)
     np.random.seed(0)
     if args.impl == "reference":

@@ -167,6 +167,11 @@ struct shampoo_ctx {
   float** blk_wptr = nullptr;
   int* blk_ld = nullptr;
   StackMaps mGs, mGt, mRoots, mTap, mMom;
+  // bf16 gradients with fp32 statistics: G and G^T also as bf16 stacks (in the
+  // Gs region), the statistics' operands on the kind::f16 MMA
+  uint16_t* Gs16 = nullptr;
+  uint16_t* Gt16 = nullptr;
+  StackMaps mGs16, mGt16;
   double stats_flops_L = 0, stats_flops_R = 0, stack_bytes = 0;
   int64_t step = 0;
   int power_refreshed = 0;  // a refresh has stored power iterates (profiler byte count only)
@@ -242,6 +247,10 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
   h->Gt = reinterpret_cast<float*>(h->scratch + xl.gt);
   h->Tap = reinterpret_cast<float*>(h->scratch + xl.tap);
   h->blk_wptr = reinterpret_cast<float**>(h->scratch + xl.wptr);
+  if (cfg->grad_dtype == SHAMPOO_BF16 && !h->stats_f64) {
+    h->Gs16 = reinterpret_cast<uint16_t*>(h->scratch + xl.gs);
+    h->Gt16 = h->Gs16 + plain_floats(nb, B);
+  }
   h->blk_ld = reinterpret_cast<int*>(h->scratch + xl.ld);
 
   std::vector<int> valid(2 * nb), wr(nb), wc(nb);
@@ -280,7 +289,9 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
   }
   if ((rc = make_stack_maps(h->mGs, h->Gs, nb, B)) || (rc = make_stack_maps(h->mGt, h->Gt, nb, B)) ||
       (rc = make_stack_maps(h->mRoots, h->roots, 2 * nb, B)) || (rc = make_stack_maps(h->mTap, h->Tap, nb, B)) ||
-      (h->mom && (rc = make_stack_maps(h->mMom, h->mom, nb, B)))) {
+      (h->mom && (rc = make_stack_maps(h->mMom, h->mom, nb, B))) ||
+      (h->Gs16 && ((rc = make_stack_maps_bf16(h->mGs16, h->Gs16, nb, B)) ||
+                   (rc = make_stack_maps_bf16(h->mGt16, h->Gt16, nb, B))))) {
     delete h;
     return rc;
   }
@@ -317,7 +328,7 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
   int rc;
   // 1. partition / stack (and, with momentum, M <- alpha M + G per block)
   if ((rc = launch_stack(args, h->d_table, nb, B, c.grad_dtype, h->Gs, h->Gt, h->mom, c.momentum, 1.f,
-                         h->blk_wptr, h->blk_ld, st, h->stack_bytes)))
+                         h->blk_wptr, h->blk_ld, st, h->stack_bytes, h->Gs16, h->Gt16)))
     return rc;
   // Widened bf16 gradients are exact in tf32: their lo parts are zero, so
   // the products that take G as an operand skip the MMAs with those parts.
@@ -362,14 +373,15 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
     }
   } else {
     Builder b;
-    Epilogue& eL = b.add(nb, B, h->mGs, 0, h->mGs, 0, h->stats_flops_L);
+    // bf16 gradients: both statistics products on the kind::f16 MMA (G exact in bf16)
+    Epilogue& eL = b.add(nb, B, h->Gs16 ? h->mGs16 : h->mGs, 0, h->Gs16 ? h->mGs16 : h->mGs, 0, h->stats_flops_L);
     b.L.g[0].a_exact = b.L.g[0].b_exact = g_exact;
     b.L.g[0].sym = 1;  // symmetric: the tiles below the diagonal are mirrored below
     eL.beta = c.beta;
     eL.C = h->stats;
     eL.D = h->stats;
     eL.flags = h->d_status;
-    Epilogue& eR = b.add(nb, B, h->mGt, 0, h->mGt, 0, h->stats_flops_R);
+    Epilogue& eR = b.add(nb, B, h->Gs16 ? h->mGt16 : h->mGt, 0, h->Gs16 ? h->mGt16 : h->mGt, 0, h->stats_flops_R);
     b.L.g[1].a_exact = b.L.g[1].b_exact = g_exact;
     b.L.g[1].sym = 1;
     eR.beta = c.beta;

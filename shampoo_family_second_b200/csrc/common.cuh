@@ -206,6 +206,18 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
+// D (TMEM, fp32) (+)= A B with bf16 A and B in shared memory (kind::f16, K = 16
+// per instruction: the same 32 bytes of K per row as a kind::tf32 MMA).
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on an mbarrier once all previously issued MMAs of this thread are done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -273,6 +285,12 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128_32b(uint32_t saddr, uint3
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, int b_mn = 0) {
   return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(b_mn & 1) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+// The same descriptor for kind::f16 with bf16 A and B (type code 1 in both
+// operand fields), fp32 accumulation, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 }  // namespace shampoo

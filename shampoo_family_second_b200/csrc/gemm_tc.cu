@@ -71,6 +71,11 @@ static_assert(256 * LIGHT_REGS + 256 * HEAVY_REGS == THREADS * LAUNCH_REGS, "reg
 static_assert((RAW_BYTES / 16) % CONV_THREADS == 0, "converter work divides evenly");
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
+// K per ring chunk (one 64-byte stage row): 16 fp32 values, or 32 bf16; and
+// chunks per accumulation segment, so that a segment is 64 deep either way.
+__device__ __forceinline__ int chunk_k(const GemmGroup& G) { return G.bf16 ? 2 * BK : BK; }
+__device__ __forceinline__ int seg_chunks(const GemmGroup& G) { return G.bf16 ? SEG / 2 : SEG; }
+
 struct TileCoord {
   int gi, mat, tm, tn;
   bool skip;
@@ -298,8 +303,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           const TileCoord tc = tile_coord(L, tile);
           if (tc.skip) continue;
           const GemmGroup& G = L.g[tc.gi];
-          const int nk = (G.k + BK - 1) / BK;
-          const uint32_t tx_bytes = static_cast<uint32_t>(G.a_rows + G.b_rows) * BK * 4u;
+          const int ck = chunk_k(G);
+          const int nk = (G.k + ck - 1) / ck;
+          const uint32_t tx_bytes = static_cast<uint32_t>(G.a_rows + G.b_rows) * BK * 4u;  // 64 bytes a row
           const void* amap = &maps.m[G.a_map];
           const void* bmap = &maps.m[G.b_map];
           const int am = G.a_off + tc.mat;
@@ -314,7 +320,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint8_t* sa = smem + s * STAGE_BYTES;
             uint8_t* sb = sa + A_BYTES;
             mbar_arrive_expect_tx(&full[s], tx_bytes);
-            tma_load_3d(sa, amap, &full[s], kc * BK, tc.tm * BM, am);
+            tma_load_3d(sa, amap, &full[s], kc * ck, tc.tm * BM, am);
             if (G.b_mn) {
               // B[k][n] row-major: 16 K-rows x 32 N-columns per copy, one copy per
               // 32-column block of the tile, blocks MN_BLOCK bytes apart.
@@ -323,7 +329,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               for (int q = 0; q < nblk; ++q)
                 tma_load_3d(sb + q * MN_BLOCK, bmap, &full[s], tc.tn * BN + q * 32, kc * BK, bm);
             } else {
-              tma_load_3d(sb, bmap, &full[s], kc * BK, tc.tn * BN, bm);
+              tma_load_3d(sb, bmap, &full[s], kc * ck, tc.tn * BN, bm);
             }
           }
         }
@@ -348,12 +354,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           const TileCoord tc = tile_coord(L, tile);
           if (tc.skip) continue;
           const GemmGroup& G = L.g[tc.gi];
-          const int nk = (G.k + BK - 1) / BK;
-          const uint32_t idesc = idesc_tf32(BM, BN, G.b_mn);
+          const int ck = chunk_k(G), sc = seg_chunks(G);
+          const int nk = (G.k + ck - 1) / ck;
+          const bool f16 = G.bf16 != 0;
+          const uint32_t idesc = f16 ? idesc_bf16(BM, BN) : idesc_tf32(BM, BN, G.b_mn);
 #pragma unroll 1
           for (int kc = 0; kc < nk; ++kc, ++it) {
             const int s = it % STAGES;
-            const bool first = (kc % SEG) == 0;
+            const bool first = (kc % sc) == 0;
             const uint32_t b = sg & 1;
             const uint32_t tbuf = taddr + b * BN;
             if (first && sg >= 2 &&
@@ -383,12 +391,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                 dbh = smem_desc_k_sw64(b_hi + off);
                 dbl = smem_desc_k_sw64(b_lo + off);
               }
-              mma_tf32(tbuf, dah, dbh, idesc, (first && ks == 0) ? 0u : 1u);
-              if (!G.b_exact) mma_tf32(tbuf, dah, dbl, idesc, 1u);
-              if (!G.a_exact) mma_tf32(tbuf, dal, dbh, idesc, 1u);
+              if (f16) {
+                mma_bf16(tbuf, dah, dbh, idesc, (first && ks == 0) ? 0u : 1u);
+              } else {
+                mma_tf32(tbuf, dah, dbh, idesc, (first && ks == 0) ? 0u : 1u);
+                if (!G.b_exact) mma_tf32(tbuf, dah, dbl, idesc, 1u);
+                if (!G.a_exact) mma_tf32(tbuf, dal, dbh, idesc, 1u);
+              }
             }
             mma_commit(&empty[s]);
-            if ((kc % SEG) == SEG - 1 || kc == nk - 1) {
+            if ((kc % sc) == sc - 1 || kc == nk - 1) {
               mma_commit(&acc_full[b]);
               ++sg;
             }
@@ -408,7 +420,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const TileCoord tc = tile_coord(L, tile);
         if (tc.skip) continue;
         const GemmGroup& G = L.g[tc.gi];
-        const int nk = (G.k + BK - 1) / BK;
+        const int ck = chunk_k(G);
+        const int nk = (G.k + ck - 1) / ck;
         // An operand whose values are exact in tf32 needs no split: its hi
         // part is the value as TMA wrote it, and its lo part is never read.
         const bool keep_a = G.a_exact != 0, keep_b = G.b_exact != 0;
@@ -459,7 +472,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const GemmGroup& G = L.g[tc.gi];
       const int n = G.n;
       const int m = G.m;
-      const int nseg = ((G.k + BK - 1) / BK + SEG - 1) / SEG;
+      const int ck = chunk_k(G), sc = seg_chunks(G);
+      const int nseg = ((G.k + ck - 1) / ck + sc - 1) / sc;
       // C of this warp's first chunk streams into its shared tile while the
       // tile's MMAs run.
       const int row0_first = tc.tm * BM + q * 32;
@@ -553,20 +567,23 @@ int get_encoder() {
 // tiles (mn_layout: 16 rows of K x 32 columns) the 128-byte swizzle with
 // 32-byte atoms, the only MN-major tf32 layout of the tensor core.  Boxes that
 // reach past rows or cols read zeros.
-int encode_stack_map(CUtensorMap* map, const float* base, int64_t batch, int rows, int cols, int box_rows,
-                     int mn_layout) {
+int encode_stack_map(CUtensorMap* map, const void* base, int64_t batch, int rows, int cols, int box_rows,
+                     int mn_layout, int bf16) {
   int rc = get_encoder();
   if (rc) return rc;
+  const int es = bf16 ? 2 : 4;  // element bytes
   if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return set_error(-2, "stack base not 16-byte aligned");
-  if (cols % 4 != 0) return set_error(-2, "stack rows of %d floats are not 16-byte multiples", cols);
+  if ((cols * es) % 16 != 0) return set_error(-2, "stack rows of %d elements are not 16-byte multiples", cols);
   const cuuint64_t nr = static_cast<cuuint64_t>(rows), nc = static_cast<cuuint64_t>(cols);
   cuuint64_t dims[3] = {nc, nr, static_cast<cuuint64_t>(batch)};
-  cuuint64_t strides[2] = {nc * 4, nr * nc * 4};
-  // K-major boxes: BK columns (64 bytes) x box_rows rows; MN-major boxes: 32
-  // columns (128 bytes) x box_rows (= BK) rows of K.
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(mn_layout ? 32 : BK), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint64_t strides[2] = {nc * es, nr * nc * es};
+  // K-major boxes: 64 bytes of K (BK fp32 or 2 BK bf16 columns) x box_rows
+  // rows; MN-major boxes (fp32 only): 32 columns (128 bytes) x box_rows (= BK)
+  // rows of K.
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(mn_layout ? 32 : 64 / es), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+  CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                        const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
                         mn_layout ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -581,14 +598,27 @@ int make_rect_maps(StackMaps& sm, const float* base, int64_t batch, int rows, in
   sm.cols = cols;
   sm.a_rows = rows < BM ? rows : BM;
   sm.b_rows = rows < BN ? rows : BN;
-  int rc = encode_stack_map(&sm.a, base, batch, rows, cols, sm.a_rows, 0);
+  sm.bf16 = 0;
+  int rc = encode_stack_map(&sm.a, base, batch, rows, cols, sm.a_rows, 0, 0);
   if (rc) return rc;
-  if ((rc = encode_stack_map(&sm.mn, base, batch, rows, cols, BK, 1))) return rc;
-  return encode_stack_map(&sm.b, base, batch, rows, cols, sm.b_rows, 0);
+  if ((rc = encode_stack_map(&sm.mn, base, batch, rows, cols, BK, 1, 0))) return rc;
+  return encode_stack_map(&sm.b, base, batch, rows, cols, sm.b_rows, 0, 0);
 }
 
 int make_stack_maps(StackMaps& sm, const float* base, int64_t batch, int n) {
   return make_rect_maps(sm, base, batch, n, n);
+}
+
+int make_stack_maps_bf16(StackMaps& sm, const void* base, int64_t batch, int n) {
+  std::memset(&sm, 0, sizeof(sm));
+  sm.base = nullptr;  // not an fp32 stack
+  sm.rows = sm.cols = n;
+  sm.a_rows = n < BM ? n : BM;
+  sm.b_rows = n < BN ? n : BN;
+  sm.bf16 = 1;
+  int rc = encode_stack_map(&sm.a, base, batch, n, n, sm.a_rows, 0, 1);
+  if (rc) return rc;
+  return encode_stack_map(&sm.b, base, batch, n, n, sm.b_rows, 0, 1);
 }
 
 Builder::Builder() : nmaps(0) {
@@ -608,6 +638,10 @@ Epilogue& Builder::add(int batch, int n, const StackMaps& a, int a_off, const St
   M.m[nmaps] = bmode == B_MN_MAJOR ? b.mn : b.b;
   g.b_map = nmaps++;
   g.b_mn = bmode == B_MN_MAJOR ? 1 : 0;
+  // bf16 stacks (both operands, K-major): kind::f16 MMAs; their values are
+  // exact, so nothing is split
+  g.bf16 = (a.bf16 && b.bf16 && bmode != B_MN_MAJOR) ? 1 : 0;
+  if (g.bf16) g.a_exact = g.b_exact = 1;
   g.a_off = a_off;
   g.b_off = b_off;
   g.a_rows = a.a_rows;

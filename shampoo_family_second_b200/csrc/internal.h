@@ -61,6 +61,7 @@ struct GemmGroup {
   int a_exact, b_exact;  // 1: every value of the operand is exact in tf32 (e.g. widened bf16), so its
                          // lo part is zero: the MMAs with that lo part are skipped and its tiles are
                          // not split
+  int bf16;              // 1: both operands are bf16 stacks: kind::f16 MMAs, 32 K per 64-byte stage row
   int sym;               // 1: D is symmetric (square, e.g. G G^T): only the tiles that reach the
                          // diagonal or above are computed; launch_mirror_lower fills the rest
   int tiles_per;         // tiles computed per matrix (filled by launch_gemm)
@@ -87,8 +88,8 @@ constexpr int kTileN = 256;
 constexpr int kTileK = 16;
 
 // Host helpers -------------------------------------------------------------
-int encode_stack_map(CUtensorMap* map, const float* base, int64_t batch, int rows, int cols, int box_rows,
-                     int mn_layout);
+int encode_stack_map(CUtensorMap* map, const void* base, int64_t batch, int rows, int cols, int box_rows,
+                     int mn_layout, int bf16);
 int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st);
 Epilogue epilogue_defaults();
 
@@ -139,8 +140,12 @@ struct StackMaps {
   float* base;
   int a_rows, b_rows;
   int rows, cols;    // shape of each matrix of the stack
+  int bf16;          // 1: a bf16 stack (K-major maps only, 32 columns per box)
 };
 int make_stack_maps(StackMaps& sm, const float* base, int64_t batch, int n);
+// A stack (batch, n, n) of bf16 matrices, as K-major A and B operands of the
+// kind::f16 MMA (both operands of a group must be bf16 stacks).
+int make_stack_maps_bf16(StackMaps& sm, const void* base, int64_t batch, int n);
 // A stack (batch, rows, cols) of row-major matrices (cols a multiple of 4).
 int make_rect_maps(StackMaps& sm, const float* base, int64_t batch, int rows, int cols);
 
@@ -179,9 +184,11 @@ struct StackArgs {
   unsigned char vec[kMaxParams];  // rows of param i start 16-byte (fp32) / 8-byte (bf16) aligned
 };
 // M (nullable): moment stack, updated in place as M <- alpha M + gscale G_b.
+// Gs16 / Gt16 (nullable, bf16 gradients only): G and G^T also as packed bf16
+// stacks; with Gs16 the fp32 Gs is not written.
 int launch_stack(const StackArgs& args, const int* d_table, int nb, int B, int grad_dtype, float* Gs, float* Gts,
                  float* M, float alpha, float gscale, float** blk_wptr, int* blk_ld, cudaStream_t st,
-                 double alg_bytes);
+                 double alg_bytes, uint16_t* Gs16 = nullptr, uint16_t* Gt16 = nullptr);
 
 int launch_frob_norm(const float* A, int64_t batch, int n, const int* valid, float eps, int p, float* s, float* sc,
                      cudaStream_t st);

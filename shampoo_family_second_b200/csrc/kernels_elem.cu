@@ -62,10 +62,17 @@ __device__ __forceinline__ float4 load_grad4(const void* g, size_t idx, int dtyp
 // M_b <- alpha M_b + gscale G_b: Shampoo's momentum ahead of the
 // preconditioner (podcast cue 28; gscale = 1) or Adam's first moment (SOAP;
 // alpha = beta1, gscale = 1 - beta1).  The statistics keep the raw G in Gs, Gt.
+// Four values exact in bf16 (widened bf16 gradients) as packed bf16: their
+// upper halves, element 0 in the low half-word.
+__device__ __forceinline__ uint2 pack_bf16x4(float4 v) {
+  return make_uint2((__float_as_uint(v.x) >> 16) | (__float_as_uint(v.y) & 0xFFFF0000u),
+                    (__float_as_uint(v.z) >> 16) | (__float_as_uint(v.w) & 0xFFFF0000u));
+}
+
 __global__ void stack_blocks_kernel(const __grid_constant__ StackArgs args, const int* __restrict__ table, int B,
                                     int dtype, float* __restrict__ Gs, float* __restrict__ Gt,
                                     float* __restrict__ M, float alpha, float gscale, float** blk_wptr,
-                                    int* blk_ld) {
+                                    int* blk_ld, uint16_t* __restrict__ Gs16, uint16_t* __restrict__ Gt16) {
   pdl_launch_dependents();  // a following GEMM may start its prologue
   constexpr int TC = 128, STRIDE = TC + 4;
   __shared__ __align__(16) float tile[32 * STRIDE];
@@ -88,7 +95,10 @@ __global__ void stack_blocks_kernel(const __grid_constant__ StackArgs args, cons
       const int row = r0 + ty + 8 * k;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (row < r) v = load_grad4(g, static_cast<size_t>(row0 + row) * ld + col0 + col, dtype, vec, c - col);
-      *reinterpret_cast<float4*>(Gs + b * nn + static_cast<size_t>(row) * B + col) = v;
+      if (Gs16)  // bf16 gradients: the statistics read G as bf16
+        *reinterpret_cast<uint2*>(Gs16 + b * nn + static_cast<size_t>(row) * B + col) = pack_bf16x4(v);
+      else
+        *reinterpret_cast<float4*>(Gs + b * nn + static_cast<size_t>(row) * B + col) = v;
       if (M) {
         float4* mp = reinterpret_cast<float4*>(M + b * nn + static_cast<size_t>(row) * B + col);
         float4 m = *mp;
@@ -115,6 +125,8 @@ __global__ void stack_blocks_kernel(const __grid_constant__ StackArgs args, cons
       v.z = tile[(4 * part + 2) * STRIDE + j];
       v.w = tile[(4 * part + 3) * STRIDE + j];
       *reinterpret_cast<float4*>(Gt + b * nn + static_cast<size_t>(c0 + j) * B + r0 + 4 * part) = v;
+      if (Gt16) *reinterpret_cast<uint2*>(Gt16 + b * nn + static_cast<size_t>(c0 + j) * B + r0 + 4 * part) =
+          pack_bf16x4(v);
     }
   }
   if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0) {
@@ -547,12 +559,14 @@ __global__ void fill_int_kernel(int* p, int64_t count, int value) {
 
 int launch_stack(const StackArgs& args, const int* d_table, int nb, int B, int grad_dtype, float* Gs, float* Gts,
                  float* M, float alpha, float gscale, float** blk_wptr, int* blk_ld, cudaStream_t st,
-                 double alg_bytes) {
+                 double alg_bytes, uint16_t* Gs16, uint16_t* Gt16) {
   if (nb == 0) return 0;
+  if ((Gs16 || Gt16) && grad_dtype != 1)
+    return set_error(-1, "bf16 stacks need bf16 gradients (other values are not exact in bf16)");
   ProfScope ps(K_STACK, st, 0.0, alg_bytes);
   dim3 grid((B + 127) / 128, B / 32, nb), block(32, 8);
   stack_blocks_kernel<<<grid, block, 0, st>>>(args, d_table, B, grad_dtype, Gs, Gts, M, alpha, gscale, blk_wptr,
-                                              blk_ld);
+                                              blk_ld, Gs16, Gt16);
   count_launch();
   return check_cuda(cudaGetLastError(), "stack_blocks_kernel");
 }

@@ -25,7 +25,7 @@ def test_traffic_record_is_well_formed():
     with open(os.path.join(bench.ROOT, "profiles", "gemm_traffic.json")) as f:
         d = json.load(f)
     assert d["bytes_per_launch"] > 0 and d["captured_launches"] > 0
-    assert d["workload_key"] in ("lowrank", "gpt2", "llama")
+    assert d["workload_key"] in bench.WORKLOAD_NAMES.values() or d["workload_key"].startswith("llama_1b_shapes")
     assert d["solver"] in bench.SOLVER_NAMES.values()
     assert len(d["source_sha256"]) == 64 and "ncu" in d["command"]
 
@@ -51,3 +51,13 @@ def test_step_time_split_by_refresh():
     every_step = bench.split_step_ms([3.0, 4.0], 1)       # refresh every step
     assert every_step["refresh_ms"] == 3.5 and every_step["non_refresh_ms"] is None
     assert bench.refresh_steps(20, 10) == out["refresh_steps"]
+
+
+def test_workload_label_marks_a_cut_llama_workload():
+    """--layers cuts the Llama workload for small profiling captures; its label
+    (and so the traffic record's key) must not be the full workload's."""
+    import workloads
+    full = workloads.workload("llama")
+    cut = workloads.workload("llama", shapes=full.shapes[:bench.LLAMA_LAYER * 2])
+    assert bench.workload_label(full) == "llama_1b_shapes_b1024"
+    assert bench.workload_label(cut) == "llama_1b_shapes_b1024_2layers"
