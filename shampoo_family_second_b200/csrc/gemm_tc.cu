@@ -72,9 +72,14 @@ static_assert((RAW_BYTES / 16) % CONV_THREADS == 0, "converter work divides even
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 // K per ring chunk (one 64-byte stage row): 16 fp32 values, or 32 bf16; and
-// chunks per accumulation segment, so that a segment is 64 deep either way.
+// chunks per accumulation segment: 64 deep for fp32 operands, 128 for bf16.
+// The bf16 statistics issue one fast MMA per 16 K, and with 64-deep segments
+// the epilogue's drains and round-to-nearest adds (32K per segment and tile)
+// paced the launch (tensor pipe 13.5% active on the statistics launch of one
+// Llama layer); their products are exact, so the longer segment only adds
+// truncated fp32 accumulation of exact terms.
 __device__ __forceinline__ int chunk_k(const GemmGroup& G) { return G.bf16 ? 2 * BK : BK; }
-__device__ __forceinline__ int seg_chunks(const GemmGroup& G) { return G.bf16 ? SEG / 2 : SEG; }
+__device__ __forceinline__ int seg_chunks(const GemmGroup&) { return SEG; }
 
 struct TileCoord {
   int gi, mat, tm, tn;

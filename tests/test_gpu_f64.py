@@ -149,7 +149,10 @@ def test_f64_iterates_in_the_step(sb, shapes):
     opt = sb.Shampoo(wl.shapes, cfg)
     W = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
     table = [tuple(t) for t in opt.block_table()]
-    ref = oracle.ShampooOracle(wl.shapes, wl.block, wl.beta, wl.eps, wl.lr, wl.root_p, wl.refresh_every)
+    # the config carries beta as fp32 (0.9 -> 0.8999999762): at fp64 precision the oracle takes
+    # the same value
+    ref = oracle.ShampooOracle(wl.shapes, wl.block, float(np.float32(wl.beta)), wl.eps, wl.lr, wl.root_p,
+                               wl.refresh_every)
     stream = workloads.GradientStream(wl)
     worst = 0.0
     for t in range(5):
