@@ -111,7 +111,11 @@ enum {
   SHAMPOO_KERNEL_MIRROR = 8,   /* lower triangle of symmetric statistics from the upper */
   SHAMPOO_KERNEL_EIGEN = 9,    /* Jacobi sweeps of the eigensolver */
   SHAMPOO_KERNEL_GEMM_F64 = 10,/* fp64 GEMM of the fp64-iterate solver */
-  SHAMPOO_KERNEL_KINDS = 11
+  SHAMPOO_KERNEL_PERMUTE = 11, /* tensor Shampoo: unfoldings and mode products' permutes */
+  SHAMPOO_KERNEL_GRAM = 12,    /* tensor Shampoo: split-K statistics of short modes */
+  SHAMPOO_KERNEL_DIAG = 13,    /* tensor Shampoo: the diagonal variant's sums, roots and scaling */
+  SHAMPOO_KERNEL_SOAP = 14,    /* SOAP: Adam in the eigenbasis, basis transposes, carry-over */
+  SHAMPOO_KERNEL_KINDS = 15
 };
 
 /* Hyper-parameters of the blocked step.

@@ -235,7 +235,7 @@ int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const i
       if ((rc = jacobi(Ai, Qi))) return rc;
     } else {
       {  // Xt = X^T
-        ProfScope ps(K_FINALIZE, st, 0.0, 8.0 * cb * nn);
+        ProfScope ps(K_EIGEN, st, 0.0, 8.0 * cb * nn);
         transpose_kernel<<<tgrid, tblock, 0, st>>>(Qi, n, Xt);
         count_launch();
         if ((rc = check_cuda(cudaGetLastError(), "transpose_kernel"))) return rc;
@@ -267,7 +267,7 @@ int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const i
     }
     for (int it = 0; it < refine_iters; ++it) {
       {
-        ProfScope ps(K_FINALIZE, st, 0.0, 8.0 * cb * nn);
+        ProfScope ps(K_EIGEN, st, 0.0, 8.0 * cb * nn);
         transpose_kernel<<<tgrid, tblock, 0, st>>>(Qi, n, Xt);
         count_launch();
         if ((rc = check_cuda(cudaGetLastError(), "transpose_kernel"))) return rc;
@@ -302,7 +302,7 @@ int run_eigh(const float* A, float* Q, float* lam, int64_t batch, int n, const i
         e.flags = flags;
         if ((rc = b.launch(st))) return rc;
       }
-      ProfScope ps(K_CHECK, st, 0.0, 8.0 * cb * nn);
+      ProfScope ps(K_EIGEN, st, 0.0, 8.0 * cb * nn);
       rayleigh_kernel<<<dim3((n + 127) / 128, static_cast<unsigned>(cb)), 128, 0, st>>>(Qi, T, n, vi, li);
       count_launch();
       if ((rc = check_cuda(cudaGetLastError(), "rayleigh_kernel"))) return rc;

@@ -110,7 +110,11 @@ enum KernelKind : int {
   K_MIRROR = 8,
   K_EIGEN = 9,
   K_GEMM_F64 = 10,
-  K_COUNT = 11,
+  K_PERMUTE = 11,
+  K_GRAM = 12,
+  K_DIAG = 13,
+  K_SOAP = 14,
+  K_COUNT = 15,
 };
 struct ProfScope {
   ProfScope(int kind, cudaStream_t st, double alg_flops, double alg_bytes);

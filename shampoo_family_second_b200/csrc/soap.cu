@@ -342,7 +342,7 @@ int shampoo_soap_step(shampoo_soap_handle h, float* const* d_weights, const void
     const double t = static_cast<double>(h->step + 1);
     const float c1 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(sc.beta1), t)));
     const float c2 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(sc.beta2), t)));
-    ProfScope ps(K_FINALIZE, st, 0.0, 20.0 * one);
+    ProfScope ps(K_SOAP, st, 0.0, 20.0 * one);
     soap_adam_kernel<<<dim3(B / 32, B / 8, nb), dim3(32, 8), 0, st>>>(h->Grot, h->Mrot, h->v, h->d_wrows, h->d_wcols,
                                                                      B, sc.beta2, c1, c2, sc.eps, h->Grot,
                                                                      h->d_status);
@@ -394,7 +394,7 @@ int shampoo_soap_step(shampoo_soap_handle h, float* const* d_weights, const void
                        h->scratch + h->xl.eig, h->xl.eig_bytes, h->d_status, st)))
       return rc;
     {
-      ProfScope ps(K_FINALIZE, st, 0.0, 16.0 * one);
+      ProfScope ps(K_SOAP, st, 0.0, 16.0 * one);
       transpose_stack_kernel<<<dim3(B / 32, B / 32, 2 * nb), dim3(32, 8), 0, st>>>(h->Q, B, h->Qt);
       count_launch();
       if ((rc = check_cuda(cudaGetLastError(), "transpose_stack_kernel"))) return rc;
@@ -407,7 +407,7 @@ int shampoo_soap_step(shampoo_soap_handle h, float* const* d_weights, const void
       if ((rc = b.launch(st))) return rc;
     }
     {
-      ProfScope ps(K_FINALIZE, st, 0.0, 16.0 * one);
+      ProfScope ps(K_SOAP, st, 0.0, 16.0 * one);
       const size_t cnt = 2 * one;
       square_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, st>>>(h->P, cnt);
       count_launch();

@@ -137,7 +137,7 @@ __global__ void tensor_permute_kernel(const __grid_constant__ PermArgs a, int64_
 
 int launch_permute(const PermArgs& a, int64_t total, cudaStream_t st) {
   if (total <= 0) return 0;
-  ProfScope ps(K_STACK, st, 0.0, 8.0 * total);
+  ProfScope ps(K_PERMUTE, st, 0.0, 8.0 * total);
   const unsigned grid = static_cast<unsigned>((total + 255) / 256);
   tensor_permute_kernel<<<grid, 256, 0, st>>>(a, total);
   count_launch();
@@ -530,7 +530,7 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
     for (int i = 0; i < pr.k; ++i) {
       const Mode& m = pr.modes[i];
       if (m.diag) {
-        ProfScope ps(K_NORM, st, 0.0, 4.0 * m.n * double(m.Kpad));
+        ProfScope ps(K_DIAG, st, 0.0, 4.0 * m.n * double(m.Kpad));
         const unsigned blocks = static_cast<unsigned>((static_cast<int64_t>(m.n) * 32 + 255) / 256);
         row_sumsq_kernel<<<blocks, 256, 0, st>>>(U + m.u_off, m.Kpad, m.n, m.K, c.beta,
                                                  reinterpret_cast<float*>(h->state + m.h_off));
@@ -539,7 +539,7 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
         continue;
       }
       if (small_mode(m.npad, m.K)) {
-        ProfScope ps(K_NORM, st, 2.0 * m.n * double(m.n) * m.K, 4.0 * m.n * double(m.K));
+        ProfScope ps(K_GRAM, st, 2.0 * m.n * double(m.n) * m.K, 4.0 * m.n * double(m.K));
         double* partial = reinterpret_cast<double*>(h->scratch + P.scratch_gram);
         const int nchunks = static_cast<int>((m.K + kGramChunk - 1) / kGramChunk);
         gram_small_kernel<<<nchunks, 256, 0, st>>>(U + m.u_off, m.Kpad, m.n, m.K, partial);
@@ -589,7 +589,7 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
     for (const Param& pr : P.params)
       for (const Mode& m : pr.modes) {
         if (!m.diag) continue;
-        ProfScope ps(K_FINALIZE, st, 0.0, 8.0 * m.n);
+        ProfScope ps(K_DIAG, st, 0.0, 8.0 * m.n);
         diag_root_kernel<<<static_cast<unsigned>((m.n + 255) / 256), 256, 0, st>>>(
             reinterpret_cast<const float*>(h->state + m.h_off), m.n, c.eps, 1.f / (2 * pr.k),
             reinterpret_cast<float*>(h->state + m.d_off), h->d_status);
@@ -636,7 +636,7 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
         if ((rc = launch_permute(a, static_cast<int64_t>(m.npad) * m.Kpad, st))) return rc;
       }
       if (m.diag) {
-        ProfScope ps(K_FINALIZE, st, 0.0, 8.0 * m.npad * double(m.Kpad));
+        ProfScope ps(K_DIAG, st, 0.0, 8.0 * m.npad * double(m.Kpad));
         const int64_t total = static_cast<int64_t>(m.npad) * m.Kpad;
         row_scale_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
             cur, reinterpret_cast<const float*>(h->state + m.d_off), m.n, m.npad, m.Kpad, out);
