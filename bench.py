@@ -777,7 +777,8 @@ def run_sweep(args):
     (n, kappa, p, solver) of the sweep runs in turn, one JSON line each:
     n in {256, 512, 1024}, kappa in {1e2, 1e4, 1e6, 1e8}, p in {2, 4}; coupled
     Newton (both correction degrees) and Newton-DB residual-checked
-    (tol 1e-5, cap 40), Chebyshev at degrees 16 and 32."""
+    (tol 1e-5, cap 40), Chebyshev at degrees 16 and 32, and the fp64-iterate
+    solver (tol 1e-12, cap 40)."""
     import torch
     import shampoo_family_second_b200 as sb
 
@@ -797,9 +798,10 @@ def run_sweep(args):
             for kappa in (1e2, 1e4, 1e6, 1e8):
                 for p in (2, 4):
                     for name, degree in (("newton", 0), ("newton_cubic", 0), ("newton_db", 0),
-                                         ("chebyshev", 16), ("chebyshev", 32)):
-                        sweep_case(args, sb, device, stream, rank, world, n, kappa, p, name, 40,
-                                   0.0 if name == "chebyshev" else 1e-5, degree or args.sweep_degree)
+                                         ("chebyshev", 16), ("chebyshev", 32), ("newton_cubic_f64", 0)):
+                        tol = 0.0 if name == "chebyshev" else (1e-12 if name.endswith("f64") else 1e-5)
+                        sweep_case(args, sb, device, stream, rank, world, n, kappa, p, name, 40, tol,
+                                   degree or args.sweep_degree)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
