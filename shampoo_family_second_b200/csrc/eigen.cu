@@ -133,9 +133,10 @@ __global__ void __launch_bounds__(kJacobiThreads) jacobi_eig_kernel(const float*
         *rq = s * x + c * y;
       }
       __syncthreads();
-      // columns: A <- A J and V <- V J (columns p and q of every pair)
+      // columns: A <- A J and V <- V J (columns p and q of every pair); the
+      // pair index runs fastest, so a warp's accesses fall in one or two rows
       for (int e = tid; e < pairs * m; e += blockDim.x) {
-        const int k = e / m, row = e % m;
+        const int k = e % pairs, row = e / pairs;
         const int p = pq[k][0], q = pq[k][1];
         if (q >= m || cs[k][1] == 0.f) continue;
         const float c = cs[k][0], s = cs[k][1];

@@ -315,6 +315,17 @@ __global__ void __launch_bounds__(THREADS, 1)
           const void* bmap = &maps.m[G.b_map];
           const int am = G.a_off + tc.mat;
           const int bm = G.b_off + tc.mat;
+          if (G.ep.C) {
+            // The epilogue reads the tile's C rows a chunk at a time, each one
+            // memory latency after the last; ask for them in L2 now, a whole
+            // tile of MMAs ahead.
+            const int r0 = tc.tm * BM, c0 = tc.tn * BN;
+            const int rows = min(BM, G.m - r0), cols = min(BN, G.n - c0);
+            const float* cbase = G.ep.C + static_cast<size_t>(tc.mat) * G.m * G.n + static_cast<size_t>(r0) * G.n + c0;
+#pragma unroll 1
+            for (int r = 0; r < rows; ++r)
+              prefetch_l2_bulk(cbase + static_cast<size_t>(r) * G.n, static_cast<uint32_t>(cols) * 4u);
+          }
 #pragma unroll 1
           for (int kc = 0; kc < nk; ++kc, ++it) {
             const int s = it % STAGES;
