@@ -151,6 +151,18 @@ __device__ __forceinline__ void stage_c(const Epilogue& E, int m, int n, int mat
 //            are applied there.
 // Each element of C is read before the same thread group's store of that
 // element, so C may be the output D (statistics updated in place).
+// Epilogue features a launch uses, as a kernel template mask: every line the
+// epilogue's four inlined chunk sites carry costs all launches of a kernel
+// built with it (with the weight update in every launch, the solver products
+// at n = 256 ran 20% slower), so each launch runs the kernel built with only
+// the features its groups use.
+enum : int {
+  F_W = 1,  // weight update (the second apply product)
+  F_C = 2,  // C operand (beta C), staged through shared memory
+  F_E = 4,  // second output E and the trace residual
+};
+
+template <int kF>
 __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int row0, int c0, const float* acc,
                                                float* tilebuf, int lane, float& resid, bool& bad, bool c_staged) {
   const Epilogue& E = G.ep;
@@ -159,13 +171,13 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
   const int r = row0 + lane;
   const int dj = r - c0;  // column of this row's diagonal element within the chunk
   const float gam = E.gamma_vec ? E.gamma_vec[static_cast<size_t>(mat) * E.gamma_stride] : E.gamma;
-  if (E.res) {
+  if ((kF & F_E) && E.res) {
     const int vsz = E.valid ? E.valid[mat] : n;
 #pragma unroll
     for (int j = 0; j < 32; ++j)
       if (j == dj && r < vsz) resid += 1.f - acc[j];
   }
-  if (E.C) {
+  if ((kF & F_C) && E.C) {
     if (!c_staged) stage_c(E, m, n, mat, row0, c0, tilebuf, lane);
     cp_async_wait_all();
     __syncwarp();
@@ -178,7 +190,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
     w.y = E.alpha * acc[4 * k + 1] + ((4 * k + 1 == dj) ? gam : 0.f);
     w.z = E.alpha * acc[4 * k + 2] + ((4 * k + 2 == dj) ? gam : 0.f);
     w.w = E.alpha * acc[4 * k + 3] + ((4 * k + 3 == dj) ? gam : 0.f);
-    if (E.C) {
+    if ((kF & F_C) && E.C) {
       const float4 c = *slot;
       w.x += E.beta * c.x;
       w.y += E.beta * c.y;
@@ -192,7 +204,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
   const float sc = E.scale_vec ? E.scale_vec[mat] : 1.f;
   float* wbase = nullptr;
   int wld = 0, wr = 0, wc = 0;
-  if (E.wptr) {
+  if ((kF & F_W) && E.wptr) {
     wbase = E.wptr[mat];
     wld = E.wld[mat];
     wr = E.wrows[mat];
@@ -213,7 +225,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
       v.w *= sc;
       bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
       if (E.D) *reinterpret_cast<float4*>(E.D + off) = v;
-      if (E.E) {
+      if ((kF & F_E) && E.E) {
         float4 e;
         e.x = E.e_mul * v.x + ((gr == gc + 0) ? E.e_add : 0.f);
         e.y = E.e_mul * v.y + ((gr == gc + 1) ? E.e_add : 0.f);
@@ -221,7 +233,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
         e.w = E.e_mul * v.w + ((gr == gc + 3) ? E.e_add : 0.f);
         *reinterpret_cast<float4*>(E.E + off) = e;
       }
-      if (wbase && gr < wr) {
+      if ((kF & F_W) && wbase && gr < wr) {
         float* wrow = wbase + static_cast<size_t>(gr) * wld + gc;
         if (gc + 3 < wc && (reinterpret_cast<uintptr_t>(wrow) & 15) == 0) {
           float4 w4 = *reinterpret_cast<float4*>(wrow);  // one 16-byte read-modify-write
@@ -246,6 +258,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int mat, int 
 // gridDim.x, ...  The shared-memory ring and the two TMEM buffers carry over
 // from one tile to the next, so the epilogue of a tile (register sums ->
 // global stores) overlaps the MMAs of the next one.
+template <int kF>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm3x_tf32_kernel(const __grid_constant__ GemmLaunch L, const __grid_constant__ TmaMaps maps,
                        double* prof_flops) {
@@ -315,17 +328,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           const void* bmap = &maps.m[G.b_map];
           const int am = G.a_off + tc.mat;
           const int bm = G.b_off + tc.mat;
-          if (G.ep.C) {
-            // The epilogue reads the tile's C rows a chunk at a time, each one
-            // memory latency after the last; ask for them in L2 now, a whole
-            // tile of MMAs ahead.
-            const int r0 = tc.tm * BM, c0 = tc.tn * BN;
-            const int rows = min(BM, G.m - r0), cols = min(BN, G.n - c0);
-            const float* cbase = G.ep.C + static_cast<size_t>(tc.mat) * G.m * G.n + static_cast<size_t>(r0) * G.n + c0;
-#pragma unroll 1
-            for (int r = 0; r < rows; ++r)
-              prefetch_l2_bulk(cbase + static_cast<size_t>(r) * G.n, static_cast<uint32_t>(cols) * 4u);
-          }
 #pragma unroll 1
           for (int kc = 0; kc < nk; ++kc, ++it) {
             const int s = it % STAGES;
@@ -494,7 +496,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // tile's MMAs run.
       const int row0_first = tc.tm * BM + q * 32;
       const int c0_first = tc.tn * BN + h * (BN / 2);
-      const bool staged0 = G.ep.C && row0_first < m && c0_first < n;
+      const bool staged0 = (kF & F_C) && G.ep.C && row0_first < m && c0_first < n;
       if (staged0) stage_c(G.ep, m, n, tc.mat, row0_first, c0_first, tilebuf, lane);
       float sum[BN / 2];
 #pragma unroll
@@ -530,10 +532,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c) {
           const int c0 = tc.tn * BN + h * (BN / 2) + c * 32;
-          if (c0 < n) epilogue_chunk(G, tc.mat, row0, c0, &sum[c * 32], tilebuf, lane, resid, nonfinite, c == 0 && staged0);
+          if (c0 < n)
+            epilogue_chunk<kF>(G, tc.mat, row0, c0, &sum[c * 32], tilebuf, lane, resid, nonfinite, c == 0 && staged0);
         }
       }
-      if (G.ep.res) {
+      if ((kF & F_E) && G.ep.res) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) resid += __shfl_xor_sync(0xffffffffu, resid, o);
         if (lane == 0 && resid != 0.f) atomicAdd(&G.ep.res[tc.mat], resid);
@@ -678,8 +681,22 @@ Epilogue& Builder::add_rect(int batch, int Mr, int N, int K, const StackMaps& a,
   return e;
 }
 
+// The kernel built for feature mask f (F_W | F_C | F_E).
+const void* gemm_kernel(int f) {
+  switch (f & 7) {
+    case 0: return reinterpret_cast<const void*>(gemm3x_tf32_kernel<0>);
+    case 1: return reinterpret_cast<const void*>(gemm3x_tf32_kernel<1>);
+    case 2: return reinterpret_cast<const void*>(gemm3x_tf32_kernel<2>);
+    case 3: return reinterpret_cast<const void*>(gemm3x_tf32_kernel<3>);
+    case 4: return reinterpret_cast<const void*>(gemm3x_tf32_kernel<4>);
+    case 5: return reinterpret_cast<const void*>(gemm3x_tf32_kernel<5>);
+    case 6: return reinterpret_cast<const void*>(gemm3x_tf32_kernel<6>);
+    default: return reinterpret_cast<const void*>(gemm3x_tf32_kernel<7>);
+  }
+}
+
 int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
-  static unsigned attr_mask = 0;  // devices on which the smem attribute is set
+  static unsigned attr_mask = 0;  // devices on which both kernels' attributes are set
   int dev = 0;
   int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
   if (rc) return rc;
@@ -687,17 +704,26 @@ int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
     // The register hand-over inside the kernel (setmaxnreg) balances only if
     // the CTA is launched with exactly LAUNCH_REGS registers per thread; with
     // fewer, the epilogue warps' request could never be met.
-    cudaFuncAttributes fa;
-    rc = check_cuda(cudaFuncGetAttributes(&fa, gemm3x_tf32_kernel), "cudaFuncGetAttributes(gemm)");
-    if (rc) return rc;
-    if (fa.numRegs != LAUNCH_REGS)
-      return set_error(-2, "gemm3x_tf32_kernel was built with %d registers per thread; the register split "
-                       "needs exactly %d", fa.numRegs, LAUNCH_REGS);
-    rc = check_cuda(cudaFuncSetAttribute(gemm3x_tf32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES),
-                    "cudaFuncSetAttribute(gemm)");
-    if (rc) return rc;
+    for (int f = 0; f < 8; ++f) {
+      const void* k = gemm_kernel(f);
+      cudaFuncAttributes fa;
+      rc = check_cuda(cudaFuncGetAttributes(&fa, k), "cudaFuncGetAttributes(gemm)");
+      if (rc) return rc;
+      if (fa.numRegs != LAUNCH_REGS)
+        return set_error(-2, "gemm3x_tf32_kernel was built with %d registers per thread; the register split "
+                         "needs exactly %d", fa.numRegs, LAUNCH_REGS);
+      rc = check_cuda(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
+                      "cudaFuncSetAttribute(gemm)");
+      if (rc) return rc;
+    }
     attr_mask |= 1u << dev;
+  }
+  int features = 0;  // the epilogue features some group uses: the kernel built with those
+  for (int i = 0; i < L.ngroups; ++i) {
+    const Epilogue& e = L.g[i].ep;
+    if (e.wptr) features |= F_W;
+    if (e.C) features |= F_C;
+    if (e.E || e.res) features |= F_E;
   }
   int64_t total = 0;
   double flops = 0;
@@ -741,8 +767,10 @@ int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  rc = check_cuda(cudaLaunchKernelEx(&cfg, gemm3x_tf32_kernel, L, maps, device_flop_slots()),
-                  "gemm3x_tf32_kernel launch");
+  void* args[3] = {&L, const_cast<TmaMaps*>(&maps), nullptr};
+  double* slots = device_flop_slots();
+  args[2] = &slots;
+  rc = check_cuda(cudaLaunchKernelExC(&cfg, gemm_kernel(features), args), "gemm3x_tf32_kernel launch");
   if (rc) return rc;
   count_launch();
   return check_cuda(cudaGetLastError(), "gemm3x_tf32_kernel launch");
