@@ -221,8 +221,25 @@ SHAMPOO_API int shampoo_block_table(shampoo_handle h, int32_t* nb, int64_t* tabl
  * (fp32; fp64 values behind the float pointers when cfg.solver is
  * SHAMPOO_SOLVER_NEWTON_CUBIC_F64); rootL / rootR: (nb, B, B) fp32 stacks of
  * XL and XR; *step: steps taken.
- * Ragged blocks hold zeros outside their r x r / c x c valid region. */
+ * Ragged blocks hold zeros outside their r x r / c x c valid region.
+ * The statistics are symmetric, and a step updates only their tiles on or
+ * above the diagonal (every element (i, j) with j >= i, and the diagonal
+ * tiles whole); the rest is copied from its transpose on refresh steps only,
+ * since only the roots read it.  Between refreshes, call
+ * shampoo_sync_statistics before reading L or R as full matrices.  A saved
+ * and restored state needs no sync: the next refresh fills the rest again. */
 SHAMPOO_API int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, float** rootR, int64_t* step);
+
+/* Fills the part of every statistics matrix below its diagonal tiles from
+ * the transpose of the part above (one pass over the L and R stacks),
+ * enqueued on `stream`: reads of L and R ordered after it see the full
+ * symmetric matrices.  No-op where every tile is computed: fp32 statistics
+ * with B <= 256 (one tile column of 256), fp64 statistics with B <= 64 (one
+ * tile of 64).  Statistics as in the
+ * notes' matrix-case listing (L = sum G G^T, R = sum G^T G, both symmetric).
+ * SHAMPOO_ERR_INVALID_ARG for a NULL handle; SHAMPOO_ERR_CUDA if the launch
+ * fails. */
+SHAMPOO_API int shampoo_sync_statistics(shampoo_handle h, void* stream);
 
 /* Device pointer to the momentum stack (nb, B, B) fp32 in the state (zero
  * outside each block's r x c region), or NULL when momentum is off. */

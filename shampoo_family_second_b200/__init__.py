@@ -63,7 +63,7 @@ KERNEL_NAMES = ("gemm3x_tf32", "stack_blocks", "frob_norm", "prologue", "check",
 EXPORTS = (
     "shampoo_status_string", "shampoo_last_error", "shampoo_query_sizes", "shampoo_init", "shampoo_step",
     "shampoo_step_strided", "shampoo_get_status", "shampoo_block_table", "shampoo_state_views",
-    "shampoo_momentum_view", "shampoo_set_step", "shampoo_destroy",
+    "shampoo_sync_statistics", "shampoo_momentum_view", "shampoo_set_step", "shampoo_destroy",
     "inv_root_scratch_bytes", "inv_root_scratch_bytes_p", "inv_root_batched", "inv_root_batched_noalloc",
     "shampoo_tensor_query_sizes", "shampoo_tensor_init", "shampoo_tensor_step", "shampoo_tensor_views",
     "shampoo_tensor_get_status", "shampoo_tensor_destroy", "shampoo_soap_query_sizes", "shampoo_soap_init",
@@ -136,6 +136,7 @@ def _load():
         "shampoo_state_views": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
                                                ctypes.POINTER(P), ctypes.POINTER(I64)]),
         "shampoo_momentum_view": (ctypes.c_int, [P, ctypes.POINTER(P)]),
+        "shampoo_sync_statistics": (ctypes.c_int, [P, P]),
         "shampoo_set_step": (ctypes.c_int, [P, I64]),
         "shampoo_destroy": (None, [P]),
         "inv_root_scratch_bytes": (ctypes.c_int, [I64, I32, I32, sz]),
@@ -330,10 +331,14 @@ class Shampoo:
     def step_count(self) -> int:
         return self._views()[1]
 
-    def statistics(self):
+    def statistics(self, stream=None):
         """(L, R) as views (nb, B, B) into the state buffer: float32, or float64
-        with the fp64-iterate solver (which keeps the statistics in fp64)."""
+        with the fp64-iterate solver (which keeps the statistics in fp64).
+        The part of fp32 statistics below the diagonal tiles is first filled in
+        on ``stream`` (default: the current stream), as steps without a root
+        refresh leave it stale."""
         import torch
+        _check(lib.shampoo_sync_statistics(self._h, _stream_ptr(stream)))
         (pl, pr, _, _), _ = self._views()
         B, nb = self.cfg.block, self.nb
         base = self.state.data_ptr()

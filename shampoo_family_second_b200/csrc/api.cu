@@ -365,7 +365,9 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
     g[1].C = L64 + plain_floats(nb, B);
     g[1].D = L64 + plain_floats(nb, B);
     g[1].beta = c.beta;
-    if ((rc = launch_dgemm(g, 2, nb, B, nullptr, nullptr, h->d_status, st, true))) return rc;
+    // symmetric: the tiles below the diagonal are filled in on refresh steps
+    if ((rc = launch_dgemm(g, 2, nb, B, nullptr, nullptr, h->d_status, st, true, true))) return rc;
+    if (refresh && (rc = launch_mirror_lower_f64(L64, 2 * int64_t(nb), B, st))) return rc;
     if (!refresh) {
       Builder b;
       add_apply1(b);
@@ -376,7 +378,7 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
     // bf16 gradients: both statistics products on the kind::f16 MMA (G exact in bf16)
     Epilogue& eL = b.add(nb, B, h->Gs16 ? h->mGs16 : h->mGs, 0, h->Gs16 ? h->mGs16 : h->mGs, 0, h->stats_flops_L);
     b.L.g[0].a_exact = b.L.g[0].b_exact = g_exact;
-    b.L.g[0].sym = 1;  // symmetric: the tiles below the diagonal are mirrored below
+    b.L.g[0].sym = 1;  // symmetric: the tiles below the diagonal come from the mirror pass
     eL.beta = c.beta;
     eL.C = h->stats;
     eL.D = h->stats;
@@ -390,7 +392,9 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
     eR.flags = h->d_status;
     if (!refresh) add_apply1(b);
     if ((rc = b.launch(st))) return rc;
-    if ((rc = launch_mirror_lower(h->stats, 2 * nb, B, st))) return rc;
+    // Only the roots read the tiles below the diagonal, so they are filled in
+    // on refresh steps alone (shampoo_sync_statistics fills them for readers).
+    if (refresh && (rc = launch_mirror_lower(h->stats, 2 * nb, B, st))) return rc;
   }
   // 3. roots of all 2 nb damped statistics, every refresh_every steps
   if (refresh) {
@@ -468,6 +472,14 @@ int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, f
   if (rootR) *rootR = h->roots + plain_floats(nb, B);
   if (step) *step = h->step;
   return SHAMPOO_OK;
+}
+
+int shampoo_sync_statistics(shampoo_handle h, void* stream) {
+  if (!h) return set_error(SHAMPOO_ERR_INVALID_ARG, "handle is NULL");
+  const int64_t batch = 2 * int64_t(h->shapes.nb);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (h->stats_f64) return launch_mirror_lower_f64(reinterpret_cast<double*>(h->stats), batch, h->cfg.block, st);
+  return launch_mirror_lower(h->stats, batch, h->cfg.block, st);
 }
 
 int shampoo_momentum_view(shampoo_handle h, float** M) {

@@ -251,8 +251,11 @@ struct DGemmGroup {
   double alpha = 1.0, beta = 0.0, gamma = 0.0, e_mul = 0.0, e_add = 0.0;
   float* res = nullptr;
 };
+// sym: the results are symmetric; tiles wholly below the diagonal are skipped
+// (launch_mirror_lower_f64 fills them).
 int launch_dgemm(const DGemmGroup* groups, int ngroups, int64_t batch, int n, const int* valid, const int* skip,
-                 int* flags, cudaStream_t st, bool f32_operands = false);
+                 int* flags, cudaStream_t st, bool f32_operands = false, bool sym = false);
+int launch_mirror_lower_f64(double* D, int64_t batch, int n, cudaStream_t st);
 // s = sf = ||A + eps I||_F (valid block) of fp64 matrices.
 int launch_frob_f64(const double* A, int64_t batch, int n, const int* valid, float eps, float* s, float* sf,
                     cudaStream_t st);

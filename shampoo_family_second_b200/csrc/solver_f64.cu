@@ -47,6 +47,7 @@ struct DArgs {
   const int* valid;
   const int* skip;
   int* flags;
+  int sym;  // symmetric results: tiles wholly below the diagonal are skipped
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pred) {
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(kDThreads) dgemm_kernel(DArgs args) {
   const int z = blockIdx.z;
   const int gi = z / args.batch, m = z - gi * args.batch;
   if (args.skip && args.skip[m]) return;  // converged matrix: its iterates are final
+  if (args.sym && blockIdx.y > blockIdx.x) return;  // mirror_lower_f64_kernel fills it from its transpose
   const DGemmGroup& G = args.g[gi];
   const int n = args.n;
   const size_t nn = static_cast<size_t>(n) * n;
@@ -194,6 +196,25 @@ __global__ void __launch_bounds__(kDThreads) dgemm_kernel(DArgs args) {
   if (bad) raise_flag(args.flags, DEV_FLAG_NONFINITE);
 }
 
+// Lower part of a symmetric fp64 result whose product skipped the 64 x 64 tiles
+// wholly below the diagonal: block (bi, bj) of 32 x 32 in such a tile takes
+// the transpose of block (bj, bi), which was computed.  grid (n/32, n/32,
+// batch), block (32, 8).
+__global__ void mirror_lower_f64_kernel(double* __restrict__ D, int n) {
+  const int i = blockIdx.z, bi = blockIdx.y, bj = blockIdx.x;
+  if (bi / (kDT / 32) <= bj / (kDT / 32)) return;  // computed by the product
+  __shared__ double t[32][33];
+  const size_t nn = static_cast<size_t>(n) * n;
+  double* d = D + i * nn;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    t[threadIdx.y + 8 * k][threadIdx.x] = d[static_cast<size_t>(bj * 32 + threadIdx.y + 8 * k) * n + bi * 32 + threadIdx.x];
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    d[static_cast<size_t>(bi * 32 + threadIdx.y + 8 * k) * n + bj * 32 + threadIdx.x] = t[threadIdx.x][threadIdx.y + 8 * k];
+}
+
 // Damping and scaling in fp64, the first plain Newton step, and X1 = T0:
 // M0 = (sym(A) + eps_eff I) / s on the valid block and the identity on the
 // padding; T0 = ((p+1) I - M0) / p.  A is fp32 (kind 0) or fp64 (kind 1).
@@ -305,7 +326,7 @@ int launch_frob_f64(const double* A, int64_t batch, int n, const int* valid, flo
 }
 
 int launch_dgemm(const DGemmGroup* groups, int ngroups, int64_t batch, int n, const int* valid, const int* skip,
-                 int* flags, cudaStream_t st, bool f32_operands) {
+                 int* flags, cudaStream_t st, bool f32_operands, bool sym) {
   if (batch == 0) return 0;
   if (ngroups < 1 || ngroups > 2 || n % kDK != 0 || batch * ngroups > 65535)
     return set_error(SHAMPOO_ERR_INVALID_ARG, "dgemm: %d groups, n %d, batch %lld", ngroups, n,
@@ -335,9 +356,14 @@ int launch_dgemm(const DGemmGroup* groups, int ngroups, int64_t batch, int n, co
   a.valid = valid;
   a.skip = skip;
   a.flags = flags;
-  const double flops = 2.0 * n * static_cast<double>(n) * n * batch * ngroups;
-  ProfScope ps(K_GEMM_F64, st, flops, (f32_operands ? 24.0 : 32.0) * n * static_cast<double>(n) * batch * ngroups);
+  a.sym = sym ? 1 : 0;
   const unsigned tiles = static_cast<unsigned>((n + kDT - 1) / kDT);
+  // computed fraction: every tile, or those on and above the diagonal
+  const double frac = sym ? (tiles + 1.0) / (2.0 * tiles) : 1.0;
+  const double flops = 2.0 * n * static_cast<double>(n) * n * batch * ngroups * frac;
+  ProfScope ps(K_GEMM_F64, st, flops,
+               (f32_operands ? 8.0 : 16.0) * n * static_cast<double>(n) * batch * ngroups +
+                   16.0 * frac * n * static_cast<double>(n) * batch * ngroups);
   const dim3 grid(tiles, tiles, static_cast<unsigned>(batch * ngroups));
   if (f32_operands)
     dgemm_kernel<float><<<grid, kDThreads, dsmem_bytes<float>(), st>>>(a);
@@ -345,6 +371,16 @@ int launch_dgemm(const DGemmGroup* groups, int ngroups, int64_t batch, int n, co
     dgemm_kernel<double><<<grid, kDThreads, dsmem_bytes<double>(), st>>>(a);
   count_launch();
   return check_cuda(cudaGetLastError(), "dgemm_kernel");
+}
+
+int launch_mirror_lower_f64(double* D, int64_t batch, int n, cudaStream_t st) {
+  if (batch == 0 || n <= kDT) return 0;  // one tile: computed whole
+  const double t = (n + kDT - 1) / kDT;
+  ProfScope ps(K_MIRROR, st, 0.0, 16.0 * batch * n * double(n) * (t - 1.0) / (2.0 * t));
+  dim3 grid(n / 32, n / 32, static_cast<unsigned>(batch)), block(32, 8);
+  mirror_lower_f64_kernel<<<grid, block, 0, st>>>(D, n);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "mirror_lower_f64_kernel");
 }
 
 int launch_prologue_f64(const void* A, int a_is_f64, int64_t batch, int n, const int* valid, float eps,

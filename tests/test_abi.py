@@ -151,6 +151,8 @@ def test_strided_step_refuses_a_null_handle():
     w = (ctypes.c_void_p * 1)(None)
     assert sb.lib.shampoo_step_strided(None, w, w, ld, None) == sb.ERR_INVALID_ARG
     assert "handle" in sb.last_error()
+    assert sb.lib.shampoo_sync_statistics(None, None) == sb.ERR_INVALID_ARG
+    assert "handle" in sb.last_error()
 
 
 def test_momentum_state_is_one_more_block_stack(sb):

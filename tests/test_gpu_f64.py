@@ -208,3 +208,89 @@ def test_f64_step_meets_2e3_end_to_end(sb):
     assert opt.status() & ~sb.DEVFLAG_STAGNATED == 0
     print(f"\nfp64 step, 4 x 1024^2 B 256, 11 steps: end-to-end update median {np.median(errs):.1e}, "
           f"max {max(errs):.1e}")
+
+
+def run_f64_layer_shapes(sb, name, steps, k_blocks):
+    """A layer-shaped workload at full size with fp64 statistics and iterates,
+    checked on sampled blocks (blocks are independent; the GPU steps every
+    block): statistics against the float64 oracle's to fp64 rounding; on
+    refresh steps every root against the oracle's root (the fully float64
+    pipeline) at 2e-3; the apply stage against XL_gpu G XR_gpu in float64;
+    and the update against the fully float64 pipeline at 2e-3 outright.
+
+    The roots are not held here to the exact damped root of the GPU's own
+    statistics at 1e-6 (the tests above do that up to condition 1e8): with
+    eps 1e-12 the null space of a rank-deficient ragged block scales to
+    eigenvalues near 1e-10 of the largest, and fp64 iterates carry about
+    10 u64 kappa / p (a few 1e-6) there, a part of the root that the update
+    never uses (a gradient block lies in the range of its statistics)."""
+    from test_gpu_workloads import filler_gradient, per_shape_blocks, sample_blocks, to_device
+    wl = workloads.workload(name, solver=4, tol=1e-12, iters=40)
+    table = oracle.block_table(wl.shapes, wl.block)
+    blocks = sorted(set(sample_blocks(table, k_blocks, wl.seed)) | set(per_shape_blocks(table, wl.shapes, wl.seed)))
+    params = sorted({table[b].param for b in blocks})
+    opt = sb.Shampoo(wl.shapes, sb.config_from_workload(wl))
+    # the config carries beta as fp32; the oracle takes the same value
+    ref = oracle.ShampooOracle(wl.shapes, wl.block, float(np.float32(wl.beta)), wl.eps, wl.lr, wl.root_p,
+                               wl.refresh_every, blocks=blocks)
+    W = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    stream = workloads.GradientStream(wl, params=params)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(wl.seed + 99)
+    errs, worst_root, worst_stats = [], 0.0, 0.0
+    for t in range(steps):
+        mine = dict(zip(params, stream.next()))
+        grads = [mine.get(i) for i in range(len(wl.shapes))]
+        G = [to_device(grads[i], wl.grad_dtype) if i in mine else filler_gradient(wl, s, gen)
+             for i, s in enumerate(wl.shapes)]
+        before = {p: W[p].double() for p in params}
+        opt.step(W, G)
+        P_ref = ref.step(grads)
+        torch.cuda.synchronize()
+        L, R = opt.statistics()
+        XL, XR = opt.roots()
+        for b in blocks:
+            blk = ref.table[b]
+            sl = (slice(blk.row0, blk.row0 + blk.r), slice(blk.col0, blk.col0 + blk.c))
+            Lg = L[b, :blk.r, :blk.r].cpu().numpy()
+            Rg = R[b, :blk.c, :blk.c].cpu().numpy()
+            assert Lg.dtype == np.float64
+            es = max(oracle.rel_fro(Lg, ref.L[b]), oracle.rel_fro(Rg, ref.R[b]))
+            worst_stats = max(worst_stats, es)
+            assert es < 1e-12, (t, b, "stats", es)
+            xl = XL[b, :blk.r, :blk.r].cpu().numpy().astype(np.float64)
+            xr = XR[b, :blk.c, :blk.c].cpu().numpy().astype(np.float64)
+            if t % wl.refresh_every == 0:
+                for X, ref_root in ((xl, ref.XL[b]), (xr, ref.XR[b])):
+                    e = oracle.rel_fro(X, ref_root)
+                    worst_root = max(worst_root, e)
+                    assert e < 2e-3, (t, b, "root", e)
+            Pg = ((before[blk.param][sl] - W[blk.param][sl].double()) / wl.lr).cpu().numpy()
+            ea, ga = apply_check(Pg, xl, ref.block_of(grads, b), xr)
+            assert ea < ga, (t, b, "apply", ea, ga)
+            e = oracle.rel_fro(Pg, P_ref[b])
+            errs.append(e)
+            assert e < 2e-3, (t, b, "update", e)
+        del G
+    assert opt.status() & ~sb.DEVFLAG_STAGNATED == 0
+    print(f"\nfp64 step, {name} ({len(blocks)} sampled blocks x {steps} steps): statistics {worst_stats:.1e}, "
+          f"root {worst_root:.1e}, end-to-end update median {np.median(errs):.1e}, max {max(errs):.1e}")
+
+
+def test_f64_step_meets_2e3_on_gpt2_shapes(sb):
+    """GPT-2-small layer shapes (456 blocks of 512, ragged edges, rank-deficient
+    right statistics on the 256-row blocks), root every step: with fp64
+    statistics and iterates every sampled block's update meets 2e-3 against
+    the fully float64 pipeline, where the fp32 pipeline (and fp32 LAPACK)
+    reach only 7.6e-2 on the ragged blocks."""
+    run_f64_layer_shapes(sb, "gpt2", steps=3, k_blocks=6)
+
+
+@pytest.mark.slow
+def test_f64_step_meets_2e3_on_llama_shapes(sb):
+    """Llama-1B layer shapes (1024 blocks of 1024, bf16 gradients), 11 steps
+    (refreshes at 0 and 10): with fp64 statistics and iterates every sampled
+    block's update meets 2e-3 against the fully float64 pipeline, where fp32
+    statistics from one square Gaussian gradient (condition 1e9 and more) miss
+    it on the step-0 roots."""
+    run_f64_layer_shapes(sb, "llama", steps=11, k_blocks=3)

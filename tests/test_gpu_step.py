@@ -245,6 +245,43 @@ def test_large_blocks_parity(sb, block, shape):
     assert opt.status() & ~sb.DEVFLAG_STAGNATED == 0
 
 
+def test_statistics_between_refreshes(sb):
+    """Steps without a refresh update only the statistics tiles on or above the
+    diagonal; the rest is filled from the transpose on refresh steps (before
+    the roots) and by statistics() for readers.  Blocks of 512 (two tile
+    columns, a ragged block row of 188), refresh every 3 steps, 7 steps: the
+    statistics read after every step equal the float64 oracle's; the roots of
+    the refreshes at steps 3 and 6, taken after two steps that left the lower
+    tiles stale, pass their gate against the GPU's own statistics; every
+    update matches XL_gpu G XR_gpu in float64."""
+    wl = workloads.workload("tiny", shapes=((700, 1024),), block=512, steps=7, iters=30, tol=1e-5, beta=0.9,
+                            eps=1e-4, refresh_every=3, solver=workloads.SOLVER_NEWTON_CUBIC)
+    opt = sb.Shampoo(wl.shapes, sb.config_from_workload(wl))
+    W = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    ref = oracle.ShampooOracle(wl.shapes, wl.block, wl.beta, wl.eps, wl.lr, wl.root_p, wl.refresh_every)
+    stream = workloads.GradientStream(wl)
+    for t in range(wl.steps):
+        G = stream.next()
+        before = [w.double() for w in W]
+        opt.step(W, [torch.from_numpy(g).cuda() for g in G])
+        ref.step(G)
+        torch.cuda.synchronize()
+        dW = [((a - w.double()) / wl.lr).cpu().numpy() for a, w in zip(before, W)]
+        XL, XR = [x.cpu().numpy().astype(np.float64) for x in opt.roots()]
+        L, R = [x.cpu().numpy().astype(np.float64) for x in opt.statistics()]
+        for b, blk in enumerate(ref.table):
+            assert oracle.rel_fro(L[b, :blk.r, :blk.r], ref.L[b]) < TOL_STATS, (t, b)
+            assert oracle.rel_fro(R[b, :blk.c, :blk.c], ref.R[b]) < TOL_STATS, (t, b)
+            if t % wl.refresh_every == 0:
+                for X, S, v in ((XL, L, blk.r), (XR, R, blk.c)):
+                    er, gate, _ = root_checks(X[b, :v, :v], S[b, :v, :v], wl.root_p, wl.eps)
+                    assert er < gate, (t, b, er, gate)
+            Pg = dW[blk.param][blk.row0:blk.row0 + blk.r, blk.col0:blk.col0 + blk.c]
+            ea, ga = apply_check(Pg, XL[b, :blk.r, :blk.r], ref.block_of(G, b), XR[b, :blk.c, :blk.c])
+            assert ea < ga, (t, b, "apply", ea, ga)
+    assert opt.status() & ~sb.DEVFLAG_STAGNATED == 0
+
+
 def test_strided_block_views_match_the_full_step(sb):
     """Blocks are independent: the weights' blocks, given to the optimizer as
     strided views (each block a parameter of its own, via the strided step),
