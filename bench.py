@@ -438,7 +438,43 @@ def run_ours(args, wl):
     peak = peak_burst if peak_kind == "burst" else peak_sust
     traffic = gemm_traffic_per_launch(wl)
     step_total_prof = sum(tl.total_ms for tl in tallies.values())
+    roofline = {
+        "kernel": "gemm3x_tf32_kernel",
+        "bound": "tensor",
+        "achieved": achieved,
+        "peak": peak,
+        "unit": "TFLOP/s",
+        "frac": achieved / peak if peak else None,
+        "traffic": traffic,
+        "peak_kind": peak_kind,
+        "frac_burst": achieved / peak_burst if peak_burst else None,
+        "frac_sustained": achieved / peak_sust if peak_sust else None,
+        "peak_basis": (f"{peak_src} bf16 {peak_kind} ({peaks['bf16_tflops']} burst, "
+                       f"{peaks['bf16_tflops_sustained']} sustained TF/s) x {TF32_PER_BF16:.4f} "
+                       f"(nominal tf32/bf16) / {SPLIT_PASSES} (3xTF32 passes): fp32-equivalent "
+                       "algorithmic flops; frac is also the issued tf32 fraction; burst peak for a timed "
+                       f"window under {BURST_WINDOW_MS:.0f} ms, sustained above"),
+        "launches": g.launches, "avg_launch_ms": gemm_avg_ms,
+        "share_of_step_kernel_time": g.total_ms / step_total_prof if step_total_prof else None,
+        "refresh_steps": nref_prof,
+    }
+    d64 = tallies[sb.KERNEL_GEMM_F64]
+    if d64.total_ms > g.total_ms:
+        # fp64 statistics and iterates: the fp64 product dominates the step
+        ach64 = d64.alg_flops / (d64.total_ms * 1e-3) / 1e12 if d64.total_ms > 0 else 0.0
+        roofline = {
+            "kernel": "dgemm_kernel", "bound": "tensor", "achieved": ach64, "peak": FP64_NOMINAL_TFLOPS,
+            "unit": "TFLOP/s", "frac": ach64 / FP64_NOMINAL_TFLOPS, "traffic": None,
+            "peak_basis": "nominal B200 fp64 tensor-core rate (not measured on this pool); executed fp64 flops",
+            "launches": d64.launches, "avg_launch_ms": d64.total_ms / max(d64.launches, 1),
+            "share_of_step_kernel_time": d64.total_ms / step_total_prof if step_total_prof else None,
+            "refresh_steps": nref_prof,
+            "gemm3x_tf32": {"achieved_tflops": achieved, "frac": achieved / peak if peak else None,
+                            "peak_kind": peak_kind,
+                            "share_of_step_kernel_time": g.total_ms / step_total_prof if step_total_prof else None},
+        }
 
+    fp64_mode = wl.solver == SOLVER_IDS["newton_cubic_f64"]
     rate = (lambda units, ms: units / (ms * 1e-3) if ms > 0 else 0.0)
     result = {
         "metric": METRIC,
@@ -451,7 +487,7 @@ def run_ours(args, wl):
         "higher_is_better": True,
         "scaling": "strong",
         "vs_baseline": None,
-        "dtype": "f32",
+        "dtype": "f64" if fp64_mode else "f32",
         "data": "synthetic",
         "config": {
             "workload": workload_label(wl),
@@ -460,7 +496,8 @@ def run_ours(args, wl):
             "refresh_steps_timed": nref, "solver": SOLVER_NAMES[wl.solver], "root_p": wl.root_p,
             "iters_cap": wl.iters, "tol": wl.tol, "beta": wl.beta, "eps": wl.eps, "momentum": wl.momentum,
             "grad_dtype": "bf16" if wl.grad_dtype == workloads.DTYPE_BF16 else "f32",
-            "arithmetic": "3xTF32 tcgen05 (fp32-accurate), fp32 state",
+            "arithmetic": ("fp64 statistics and iterates (mma.sync f64), fp32 roots, 3xTF32 tcgen05 apply"
+                           if fp64_mode else "3xTF32 tcgen05 (fp32-accurate), fp32 state"),
             "l2": "256 MiB buffer written between timed steps, outside the per-step events",
             "parallelism": (f"blocks sharded over {world} ranks (reduce-scatter of local gradients by block "
                             "owner, all-gather of updated blocks; NCCL)") if world > 1 else "single GPU",
@@ -468,26 +505,7 @@ def run_ours(args, wl):
         "device_status": int(status),
         "gpu_launches": int(launches),
         "clocks": clk,
-        "roofline": {
-            "kernel": "gemm3x_tf32_kernel",
-            "bound": "tensor",
-            "achieved": achieved,
-            "peak": peak,
-            "unit": "TFLOP/s",
-            "frac": achieved / peak if peak else None,
-            "traffic": traffic,
-            "peak_kind": peak_kind,
-            "frac_burst": achieved / peak_burst if peak_burst else None,
-            "frac_sustained": achieved / peak_sust if peak_sust else None,
-            "peak_basis": (f"{peak_src} bf16 {peak_kind} ({peaks['bf16_tflops']} burst, "
-                           f"{peaks['bf16_tflops_sustained']} sustained TF/s) x {TF32_PER_BF16:.4f} "
-                           f"(nominal tf32/bf16) / {SPLIT_PASSES} (3xTF32 passes): fp32-equivalent "
-                           "algorithmic flops; frac is also the issued tf32 fraction; burst peak for a timed "
-                           f"window under {BURST_WINDOW_MS:.0f} ms, sustained above"),
-            "launches": g.launches, "avg_launch_ms": gemm_avg_ms,
-            "share_of_step_kernel_time": g.total_ms / step_total_prof if step_total_prof else None,
-            "refresh_steps": nref_prof,
-        },
+        "roofline": roofline,
         "kernels": {sb.KERNEL_NAMES[k]: {"launches": v.launches, "ms": round(v.total_ms, 4),
                                          "alg_tflop": round(v.alg_flops / 1e12, 6),
                                          "alg_gb": round(v.alg_bytes / 1e9, 6)}

@@ -110,16 +110,27 @@ StateLayout state_layout(int nb, int B, bool momentum, size_t stats_elem) {
   s.total = o;
   return s;
 }
-// Scratch layout: Gs | Gt | Tapply (nb matrices each) | blk_wptr (nb ptrs) | blk_ld (nb) | solver scratch
+// bf16 gradients with fp32 statistics and no momentum: the first apply
+// product reads the roots XL as three bf16 planes (split once per refresh) and
+// G^T from the bf16 stack, all on the bf16 MMA; no fp32 G^T stack is kept.
+bool apply_planes(const shampoo_config* c) {
+  return c->grad_dtype == SHAMPOO_BF16 && c->solver != SHAMPOO_SOLVER_NEWTON_CUBIC_F64 && !(c->momentum > 0.f);
+}
+
+// Scratch layout: Gs | Gt (none with XL planes) | Tapply | XL planes (3 nb bf16 matrices, with XL planes only)
+//   | blk_wptr (nb ptrs) | blk_ld (nb) | solver scratch
 struct ScratchLayout {
-  size_t gs, gt, tap, wptr, ld, root, root_bytes, total;
+  size_t gs, gt, tap, xlp, wptr, ld, root, root_bytes, total;
 };
-ScratchLayout scratch_layout(int nb, int B, int solver, int p) {
+ScratchLayout scratch_layout(int nb, int B, int solver, int p, bool planes) {
   ScratchLayout s;
   size_t o = 0;
   s.gs = o, o += al(plain_floats(nb, B) * 4);
-  s.gt = o, o += al(plain_floats(nb, B) * 4);
+  s.gt = o;
+  if (!planes) o += al(plain_floats(nb, B) * 4);
   s.tap = o, o += al(plain_floats(nb, B) * 4);
+  s.xlp = o;
+  if (planes) o += al(plain_floats(nb, B) * 3 * 2);
   s.wptr = o, o += al(size_t(nb) * 8);
   s.ld = o, o += al(size_t(nb) * 4);
   s.root = o;
@@ -172,6 +183,12 @@ struct shampoo_ctx {
   uint16_t* Gs16 = nullptr;
   uint16_t* Gt16 = nullptr;
   StackMaps mGs16, mGt16;
+  // XL as three bf16 planes (apply_planes): rebuilt after every refresh, and
+  // before the next apply whenever the roots may have changed otherwise
+  // (a new handle, shampoo_set_step after restoring a state)
+  uint16_t* xlp = nullptr;
+  StackMaps mXlp;
+  bool planes_stale = true;
   double stats_flops_L = 0, stats_flops_R = 0, stack_bytes = 0;
   int64_t step = 0;
   int power_refreshed = 0;  // a refresh has stored power iterates (profiler byte count only)
@@ -201,7 +218,7 @@ int shampoo_query_sizes(const shampoo_config* cfg, int32_t nparams, const int64_
   if ((rc = build_table(cfg->block, nparams, rows, cols, sh))) return rc;
   if (!state_bytes || !scratch_bytes) return set_error(SHAMPOO_ERR_INVALID_ARG, "output pointer is NULL");
   *state_bytes = state_layout(sh.nb, cfg->block, cfg->momentum > 0.f, stats_elem_bytes(cfg->solver)).total;
-  *scratch_bytes = scratch_layout(sh.nb, cfg->block, cfg->solver, cfg->root_p).total;
+  *scratch_bytes = scratch_layout(sh.nb, cfg->block, cfg->solver, cfg->root_p, apply_planes(cfg)).total;
   return SHAMPOO_OK;
 }
 
@@ -218,7 +235,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
     return set_error(SHAMPOO_ERR_UNSUPPORTED, "state/scratch must be 256-byte aligned");
   const int B = cfg->block, nb = sh.nb;
   StateLayout sl = state_layout(nb, B, cfg->momentum > 0.f, stats_elem_bytes(cfg->solver));
-  ScratchLayout xl = scratch_layout(nb, B, cfg->solver, cfg->root_p);
+  ScratchLayout xl = scratch_layout(nb, B, cfg->solver, cfg->root_p, apply_planes(cfg));
   if (state_bytes < sl.total) return set_error(SHAMPOO_ERR_WORKSPACE, "state %zu < %zu bytes", state_bytes, sl.total);
   if (scratch_bytes < xl.total)
     return set_error(SHAMPOO_ERR_WORKSPACE, "scratch %zu < %zu bytes", scratch_bytes, xl.total);
@@ -244,7 +261,8 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
   h->roots = reinterpret_cast<float*>(h->state + sl.roots);
   h->mom = cfg->momentum > 0.f ? reinterpret_cast<float*>(h->state + sl.mom) : nullptr;
   h->Gs = reinterpret_cast<float*>(h->scratch + xl.gs);
-  h->Gt = reinterpret_cast<float*>(h->scratch + xl.gt);
+  h->Gt = apply_planes(cfg) ? nullptr : reinterpret_cast<float*>(h->scratch + xl.gt);
+  h->xlp = apply_planes(cfg) ? reinterpret_cast<uint16_t*>(h->scratch + xl.xlp) : nullptr;
   h->Tap = reinterpret_cast<float*>(h->scratch + xl.tap);
   h->blk_wptr = reinterpret_cast<float**>(h->scratch + xl.wptr);
   if (cfg->grad_dtype == SHAMPOO_BF16 && !h->stats_f64) {
@@ -263,7 +281,8 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
     wc[b] = sh.table[5 * b + 4];
     fl += 2 * r * r * c;
     fr += 2 * r * c * c;
-    sb += r * c * (cfg->grad_dtype == SHAMPOO_BF16 ? 2 : 4) + 8.0 * B * B;  // G read; Gs, Gt written
+    // G read; G and G^T written: fp32 (or bf16 both plus fp32 G^T), bf16 both with XL planes
+    sb += r * c * (cfg->grad_dtype == SHAMPOO_BF16 ? 2 : 4) + (apply_planes(cfg) ? 4.0 : 8.0) * B * B;
     if (cfg->momentum > 0.f) sb += 8.0 * B * B;                                 // M read and written
   }
   h->stats_flops_L = fl / nb;
@@ -287,7 +306,8 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
     delete h;
     return rc;
   }
-  if ((rc = make_stack_maps(h->mGs, h->Gs, nb, B)) || (rc = make_stack_maps(h->mGt, h->Gt, nb, B)) ||
+  if ((rc = make_stack_maps(h->mGs, h->Gs, nb, B)) || (h->Gt && (rc = make_stack_maps(h->mGt, h->Gt, nb, B))) ||
+      (h->xlp && (rc = make_stack_maps_bf16(h->mXlp, h->xlp, 3 * int64_t(nb), B))) ||
       (rc = make_stack_maps(h->mRoots, h->roots, 2 * nb, B)) || (rc = make_stack_maps(h->mTap, h->Tap, nb, B)) ||
       (h->mom && (rc = make_stack_maps(h->mMom, h->mom, nb, B))) ||
       (h->Gs16 && ((rc = make_stack_maps_bf16(h->mGs16, h->Gs16, nb, B)) ||
@@ -338,8 +358,18 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
   // (T = XL M with momentum, M read as a true product) depends on neither, so
   // it joins the same launch.
   const bool refresh = h->step % c.refresh_every == 0;
+  if (h->xlp && h->planes_stale && !refresh) {  // roots not split since they were last set
+    if ((rc = launch_split_planes(h->roots, plain_floats(nb, B), h->xlp, st))) return rc;
+    h->planes_stale = false;
+  }
   auto add_apply1 = [&](Builder& b) {
-    if (h->mom) {
+    if (h->xlp) {  // T = (XL0 + XL1 + XL2) G: three bf16 planes of XL against G^T in bf16
+      Epilogue& e = b.add(nb, B, h->mXlp, 0, h->mGt16, 0, h->stats_flops_L);
+      b.L.g[b.L.ngroups - 1].a_planes = 3;
+      b.L.g[b.L.ngroups - 1].a_plane_stride = nb;
+      e.D = h->Tap;
+      e.flags = h->d_status;
+    } else if (h->mom) {
       Epilogue& e = b.add(nb, B, h->mRoots, 0, h->mMom, 0, h->stats_flops_L, B_MN_MAJOR);
       e.D = h->Tap;
       e.flags = h->d_status;
@@ -421,6 +451,10 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
     job.power_warm_hint = h->power_refreshed;
     if ((rc = run_inverse_roots(job, h->scratch + h->xl.root, h->xl.root_bytes, st))) return rc;
     h->power_refreshed = 1;
+    if (h->xlp) {
+      if ((rc = launch_split_planes(h->roots, plain_floats(nb, B), h->xlp, st))) return rc;
+      h->planes_stale = false;
+    }
     // 4a. apply, first product: T = XL G (with the fresh roots)
     Builder b;
     add_apply1(b);
@@ -491,6 +525,7 @@ int shampoo_momentum_view(shampoo_handle h, float** M) {
 int shampoo_set_step(shampoo_handle h, int64_t step) {
   if (!h || step < 0) return set_error(SHAMPOO_ERR_INVALID_ARG, "bad handle or step");
   h->step = step;
+  h->planes_stale = true;  // the roots may have been restored
   return SHAMPOO_OK;
 }
 

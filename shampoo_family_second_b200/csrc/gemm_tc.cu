@@ -323,7 +323,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           const GemmGroup& G = L.g[tc.gi];
           const int ck = chunk_k(G);
           const int nk = (G.k + ck - 1) / ck;
-          const uint32_t tx_bytes = static_cast<uint32_t>(G.a_rows + G.b_rows) * BK * 4u;  // 64 bytes a row
+          const int planes = G.a_planes > 1 ? G.a_planes : 1;
+          const uint32_t tx_bytes = static_cast<uint32_t>(G.a_rows * planes + G.b_rows) * BK * 4u;  // 64 B a row
           const void* amap = &maps.m[G.a_map];
           const void* bmap = &maps.m[G.b_map];
           const int am = G.a_off + tc.mat;
@@ -339,6 +340,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint8_t* sb = sa + A_BYTES;
             mbar_arrive_expect_tx(&full[s], tx_bytes);
             tma_load_3d(sa, amap, &full[s], kc * ck, tc.tm * BM, am);
+            // further bf16 planes of A land in the lo areas (A lo, then the first half of B lo)
+            for (int q = 1; q < planes; ++q)
+              tma_load_3d(sa + RAW_BYTES + (q - 1) * A_BYTES, amap, &full[s], kc * ck, tc.tm * BM,
+                          am + q * G.a_plane_stride);
             if (G.b_mn) {
               // B[k][n] row-major: 16 K-rows x 32 N-columns per copy, one copy per
               // 32-column block of the tile, blocks MN_BLOCK bytes apart.
@@ -411,6 +416,10 @@ __global__ void __launch_bounds__(THREADS, 1)
               }
               if (f16) {
                 mma_bf16(tbuf, dah, dbh, idesc, (first && ks == 0) ? 0u : 1u);
+                if (G.a_planes > 1) {  // A = plane 0 + plane 1 + plane 2, each product exact in fp32
+                  mma_bf16(tbuf, dal, dbh, idesc, 1u);
+                  mma_bf16(tbuf, smem_desc_k_sw64(a_lo + A_BYTES + off), dbh, idesc, 1u);
+                }
               } else {
                 mma_tf32(tbuf, dah, dbh, idesc, (first && ks == 0) ? 0u : 1u);
                 if (!G.b_exact) mma_tf32(tbuf, dah, dbl, idesc, 1u);
@@ -732,6 +741,9 @@ int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
     g.tiles_m = (g.m + BM - 1) / BM;
     g.tiles_n = (g.n + BN - 1) / BN;
     if (g.sym && g.m != g.n) return set_error(-1, "a symmetric GEMM group must be square");
+    // planes 1 and 2 of A land in the stage's lo areas, which only bf16 groups leave unused
+    if (g.a_planes > 3 || (g.a_planes > 1 && (!g.bf16 || g.a_rows > BM)))
+      return set_error(-1, "A in %d planes needs a bf16 group of at most 3 planes", g.a_planes);
     g.tiles_per = g.tiles_m * g.tiles_n;
     if (g.sym) {
       g.tiles_per = 0;

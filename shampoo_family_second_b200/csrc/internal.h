@@ -62,6 +62,9 @@ struct GemmGroup {
                          // lo part is zero: the MMAs with that lo part are skipped and its tiles are
                          // not split
   int bf16;              // 1: both operands are bf16 stacks: kind::f16 MMAs, 32 K per 64-byte stage row
+  int a_planes;          // bf16 only: A is the exact sum of this many bf16 planes (0 or 1: one), plane q
+                         // at matrix a_off + mat + q * a_plane_stride of A's stack; one MMA per plane
+  int a_plane_stride;
   int sym;               // 1: D is symmetric (square, e.g. G G^T): only the tiles that reach the
                          // diagonal or above are computed; launch_mirror_lower fills the rest
   int tiles_per;         // tiles computed per matrix (filled by launch_gemm)
@@ -114,7 +117,8 @@ enum KernelKind : int {
   K_GRAM = 12,
   K_DIAG = 13,
   K_SOAP = 14,
-  K_COUNT = 15,
+  K_PLANES = 15,
+  K_COUNT = 16,
 };
 struct ProfScope {
   ProfScope(int kind, cudaStream_t st, double alg_flops, double alg_bytes);
@@ -237,6 +241,9 @@ int launch_fill_iters(int* iters, int64_t batch, int value, cudaStream_t st);
 // After a GEMM group with sym = 1: copies the transpose of the computed upper
 // part into the 32 x 32 blocks of the tiles it skipped (wholly below the diagonal).
 int launch_mirror_lower(float* D, int64_t batch, int n, cudaStream_t st);
+// planes[q * count + i], q = 0, 1, 2: bf16 values whose sum is X[i] exactly
+// (each the nearest bf16 to what the previous planes leave); count % 4 == 0.
+int launch_split_planes(const float* X, int64_t count, uint16_t* planes, cudaStream_t st);
 
 // fp64 products of the fp64-iterate solver (solver_f64.cu): per matrix,
 // D = alpha A B + beta C + gamma I (true product, row-major n x n operands),

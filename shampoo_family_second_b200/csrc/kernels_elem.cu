@@ -3,7 +3,10 @@
 // solvers, the residual check, the unscale / output pass, and the Chebyshev
 // coefficient setup.  All reads and writes are coalesced (transposes go through
 // a 32 x 33 shared-memory tile) and each kernel touches each byte once.
+#include <algorithm>
 #include <cmath>
+
+#include <cuda_bf16.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -124,7 +127,7 @@ __global__ void stack_blocks_kernel(const __grid_constant__ StackArgs args, cons
       v.y = tile[(4 * part + 1) * STRIDE + j];
       v.z = tile[(4 * part + 2) * STRIDE + j];
       v.w = tile[(4 * part + 3) * STRIDE + j];
-      *reinterpret_cast<float4*>(Gt + b * nn + static_cast<size_t>(c0 + j) * B + r0 + 4 * part) = v;
+      if (Gt) *reinterpret_cast<float4*>(Gt + b * nn + static_cast<size_t>(c0 + j) * B + r0 + 4 * part) = v;
       if (Gt16) *reinterpret_cast<uint2*>(Gt16 + b * nn + static_cast<size_t>(c0 + j) * B + r0 + 4 * part) =
           pack_bf16x4(v);
     }
@@ -550,6 +553,32 @@ __global__ void mirror_lower_kernel(float* __restrict__ D, int n) {
     d[static_cast<size_t>(bi * 32 + threadIdx.y + 8 * k) * n + bj * 32 + threadIdx.x] = t[threadIdx.x][threadIdx.y + 8 * k];
 }
 
+// X split into three bf16 planes whose sum is X exactly: each plane is the
+// nearest bf16 to what the previous ones leave (the remainder of a fp32 value
+// after rounding its leading 8 significant bits is exact in fp32, and after
+// two such steps at most 8 significant bits are left, which bf16 holds).  The
+// roots stay fixed between refreshes, so the first apply product reads them
+// in this form on the bf16 MMA, each plane times the bf16 gradient exact in
+// fp32.  Grid-stride over float4 groups.
+__global__ void split_planes_kernel(const float4* __restrict__ X, int64_t n4, uint2* __restrict__ P) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 x = X[i];
+    float r[4] = {x.x, x.y, x.z, x.w};
+    uint32_t h[3][4];
+#pragma unroll
+    for (int q = 0; q < 3; ++q)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat16 b = __float2bfloat16_rn(r[k]);
+        h[q][k] = __bfloat16_as_ushort(b);
+        r[k] -= __bfloat162float(b);
+      }
+#pragma unroll
+    for (int q = 0; q < 3; ++q) P[q * n4 + i] = make_uint2(h[q][0] | (h[q][1] << 16), h[q][2] | (h[q][3] << 16));
+  }
+}
+
 __global__ void fill_int_kernel(int* p, int64_t count, int value) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i < count) p[i] = value;
@@ -659,6 +688,18 @@ int launch_mirror_lower(float* D, int64_t batch, int n, cudaStream_t st) {
   mirror_lower_kernel<<<grid, block, 0, st>>>(D, n);
   count_launch();
   return check_cuda(cudaGetLastError(), "mirror_lower_kernel");
+}
+
+int launch_split_planes(const float* X, int64_t count, uint16_t* planes, cudaStream_t st) {
+  if (count == 0) return 0;
+  if (count % 4 || (reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(planes)) & 15)
+    return set_error(-1, "split_planes: %lld values, or unaligned buffers", static_cast<long long>(count));
+  ProfScope ps(K_PLANES, st, 0.0, 10.0 * count);
+  const int64_t n4 = count / 4;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 148 * 16));
+  split_planes_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(X), n4, reinterpret_cast<uint2*>(planes));
+  count_launch();
+  return check_cuda(cudaGetLastError(), "split_planes_kernel");
 }
 
 int launch_fill_iters(int* iters, int64_t batch, int value, cudaStream_t st) {

@@ -2,10 +2,10 @@
 //
 // When profiling is enabled every kernel launch of the library is bracketed by
 // two CUDA events recorded on the stream it is launched on, and tallied per
-// kernel kind together with its algorithmic flops and bytes.  The GEMM kernel
-// adds its executed algorithmic flops on the device (tiles of converged
-// matrices that exit early add nothing), so achieved TFLOP/s stay exact when
-// the residual-checked solvers skip work.
+// kernel kind together with its algorithmic flops and bytes.  The GEMM kernels
+// (3xTF32 and fp64) add their executed algorithmic flops on the device (tiles
+// of converged matrices that exit early add nothing), so achieved TFLOP/s stay
+// exact when the residual-checked solvers skip work.
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -158,7 +158,7 @@ int shampoo_profile_read(int32_t kind, int64_t* launches, double* total_ms, doub
   if (e != cudaSuccess) return check_cuda(e, "profile flops");
   if (launches) *launches = g_count[kind];
   if (total_ms) *total_ms = g_ms[kind];
-  if (alg_flops) *alg_flops = (kind == K_GEMM) ? dev[K_GEMM] : g_flops[kind];
+  if (alg_flops) *alg_flops = (kind == K_GEMM || kind == K_GEMM_F64) ? dev[kind] : g_flops[kind];
   if (alg_bytes) *alg_bytes = g_bytes[kind];
   return SHAMPOO_OK;
 }

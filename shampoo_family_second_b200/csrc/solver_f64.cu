@@ -48,6 +48,7 @@ struct DArgs {
   const int* skip;
   int* flags;
   int sym;  // symmetric results: tiles wholly below the diagonal are skipped
+  double* prof_flops;  // profiling on: executed algorithmic flops accumulate here
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pred) {
@@ -76,6 +77,10 @@ __global__ void __launch_bounds__(kDThreads) dgemm_kernel(DArgs args) {
   const int gi = z / args.batch, m = z - gi * args.batch;
   if (args.skip && args.skip[m]) return;  // converged matrix: its iterates are final
   if (args.sym && blockIdx.y > blockIdx.x) return;  // mirror_lower_f64_kernel fills it from its transpose
+  if (args.prof_flops && threadIdx.x == 0)  // tiles that ran, so skipped matrices add nothing
+    atomicAdd(&args.prof_flops[K_GEMM_F64],
+              2.0 * min(kDT, args.n - static_cast<int>(blockIdx.y) * kDT) *
+                  min(kDT, args.n - static_cast<int>(blockIdx.x) * kDT) * args.n);
   const DGemmGroup& G = args.g[gi];
   const int n = args.n;
   const size_t nn = static_cast<size_t>(n) * n;
@@ -357,6 +362,7 @@ int launch_dgemm(const DGemmGroup* groups, int ngroups, int64_t batch, int n, co
   a.skip = skip;
   a.flags = flags;
   a.sym = sym ? 1 : 0;
+  a.prof_flops = device_flop_slots();
   const unsigned tiles = static_cast<unsigned>((n + kDT - 1) / kDT);
   // computed fraction: every tile, or those on and above the diagonal
   const double frac = sym ? (tiles + 1.0) / (2.0 * tiles) : 1.0;

@@ -180,6 +180,47 @@ def test_checkpoint_resume_bit_identical(sb):
     assert b.step_count == a.step_count == wl.steps
 
 
+def test_bf16_checkpoint_resume_between_refreshes(sb):
+    """bf16 gradients, blocks of 256 with ragged edges, refresh every 3 steps.
+    The first apply product reads the roots as three bf16 planes, split after
+    each refresh; a handle restored from a checkpoint taken after step 3
+    resumes at step 4, which does not refresh, so it must split the restored
+    roots first.  Both runs end with bit-identical weights, and every update
+    of the resumed run matches XL_gpu G XR_gpu in float64 (the apply stage)."""
+    shapes = ((300, 520), (256, 200))
+    wl = workloads.workload("tiny", shapes=shapes, block=256, grad_dtype=workloads.DTYPE_BF16, steps=8,
+                            iters=30, tol=1e-5, beta=0.9, eps=1e-4, refresh_every=3,
+                            solver=workloads.SOLVER_NEWTON_CUBIC)
+    cfg = sb.config_from_workload(wl)
+    stream = workloads.GradientStream(wl)
+    host = [stream.next() for _ in range(wl.steps)]
+    grads = [[bf16_tensor(g).cuda() for g in gs] for gs in host]
+    a = sb.Shampoo(wl.shapes, cfg)
+    Wa = [torch.zeros(s, device="cuda") for s in wl.shapes]
+    for t in range(wl.steps):
+        a.step(Wa, grads[t])
+        if t == 3:
+            ckpt = {k: (v.clone() if torch.is_tensor(v) else v) for k, v in a.state_dict().items()}
+            Wckpt = [w.clone() for w in Wa]
+    b = sb.Shampoo(wl.shapes, cfg)
+    b.load_state_dict(ckpt)
+    Wb = Wckpt
+    table = [tuple(x) for x in b.block_table()]
+    for t in range(4, wl.steps):
+        before = [w.double() for w in Wb]
+        b.step(Wb, grads[t])
+        torch.cuda.synchronize()
+        XL, XR = [x.cpu().numpy().astype(np.float64) for x in b.roots()]
+        for k, (param, r0, c0, r, c) in enumerate(table):
+            Pg = ((before[param] - Wb[param].double()) / wl.lr).cpu().numpy()[r0:r0 + r, c0:c0 + c]
+            G = host[t][param][r0:r0 + r, c0:c0 + c]
+            ea, ga = apply_check(Pg, XL[k, :r, :r], G, XR[k, :c, :c])
+            assert ea < ga, (t, k, ea, ga)
+    for x, y in zip(Wa, Wb):
+        assert torch.equal(x, y)
+    assert b.status() & ~sb.DEVFLAG_STAGNATED == 0
+
+
 def test_nonfinite_gradient_sets_status(sb):
     wl = workloads.workload("tiny", steps=1)
     opt = sb.Shampoo(wl.shapes, sb.config_from_workload(wl))
