@@ -55,10 +55,11 @@ KERNEL_GRAM = 12
 KERNEL_DIAG = 13
 KERNEL_SOAP = 14
 KERNEL_PLANES = 15
-KERNEL_KINDS = 16
+KERNEL_MODE_SMALL = 16
+KERNEL_KINDS = 17
 KERNEL_NAMES = ("gemm3x_tf32", "stack_blocks", "frob_norm", "prologue", "check", "finalize", "cheb_coef",
                 "spectral_scale", "mirror_lower", "jacobi_eig", "dgemm_f64", "tensor_permute", "gram_small",
-                "diag_modes", "soap_elementwise", "split_planes")
+                "diag_modes", "soap_elementwise", "split_planes", "tensor_mode_small")
 
 # Exported symbols, in header order (tests compare this with include/shampoo.h).
 EXPORTS = (

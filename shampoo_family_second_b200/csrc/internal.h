@@ -118,7 +118,8 @@ enum KernelKind : int {
   K_DIAG = 13,
   K_SOAP = 14,
   K_PLANES = 15,
-  K_COUNT = 16,
+  K_MODE_SMALL = 16,
+  K_COUNT = 17,
 };
 struct ProfScope {
   ProfScope(int kind, cudaStream_t st, double alg_flops, double alg_bytes);

@@ -14,6 +14,13 @@
 //   4. apply    V = X_0 U_0; then for i = 1 .. k-1: V <- X_i unfold_i(fold_{i-1}(V))
 //               (a permutation pass between the products), and the last
 //               fold writes W <- W - lr P into the weight.
+// Short modes (d_i <= 32, e.g. the 3 x 3 spatial modes of a convolution
+// kernel) skip the unfolding, whose 32-row padding would be most of its
+// bytes: their statistic is summed over the tensor's fibres along the mode
+// in its natural layout, and their product is applied to those fibres in
+// place of a layout change (one pass, read and write once).  They go first;
+// the longer modes follow as above.  The modes commute, so the order does
+// not change the result.
 // Diagonal variant (cue 28): a dimension longer than the threshold keeps only
 // h_i = diag(H_i) (the row sums of squares of U_i), is refreshed to
 // d_i = (h_i + eps)^{-1/(2k)} elementwise, and its "product" scales the rows
@@ -184,35 +191,64 @@ __global__ void row_scale_kernel(const float* __restrict__ cur, const float* __r
   out[t] = x < n ? d[x] * cur[t] : 0.f;
 }
 
-// Statistic of a short mode (n <= 32) whose unfolding is long (K up to
-// 10^6): one 32 x 32 GEMM tile would reduce all of K on one SM, so the Gram
-// matrix is summed in K-chunks instead.  Phase 1: each CTA stages 128-column
-// pieces of the n rows of its chunk in shared memory and accumulates its
-// thread's pairs (x <= y) in float64; phase 2 adds the chunks' partials in
-// chunk order and writes H <- beta H + sum (both triangles).
+// Short-mode statistics are summed in K-chunks of 4096 fibres (kGramChunk),
+// each chunk's n (n + 1) / 2 pair sums in float64 (at most kGramPairs);
+// gram_reduce_kernel then adds the chunks' partials in chunk order and writes
+// H <- beta H + sum (both triangles).
 constexpr int kGramChunk = 4096;
 constexpr int kGramPairs = 32 * 33 / 2;
-__global__ void __launch_bounds__(256) gram_small_kernel(const float* __restrict__ U, int64_t ld, int n, int64_t K,
-                                                         double* __restrict__ partial) {
+
+__global__ void gram_reduce_kernel(const double* __restrict__ partial, int nchunks, int n, float beta,
+                                   float* __restrict__ H, int ldh) {
+  const int npairs = n * (n + 1) / 2;
+  for (int pidx0 = threadIdx.x; pidx0 < npairs; pidx0 += blockDim.x) {
+    double sum = 0.0;
+    for (int ch = 0; ch < nchunks; ++ch) sum += partial[static_cast<int64_t>(ch) * kGramPairs + pidx0];
+    int pidx = pidx0, x = 0;
+    while (pidx >= n - x) pidx -= n - x, ++x;
+    const int y = x + pidx;
+    const float v = static_cast<float>(static_cast<double>(beta) * H[x * ldh + y] + sum);
+    H[x * ldh + y] = v;
+    H[y * ldh + x] = v;
+  }
+}
+
+// Statistic of a short mode from the natural layout: the fibres along mode m
+// (fixed other indices; element j of fibre f at (f / S) n S + j S + f % S,
+// S the product of the later dimensions) are the columns of the mode's
+// unfolding, so the Gram sum over fibres is the unfolding's.  Each CTA takes
+// one chunk: it stages 128 fibres at a time in shared memory (n rows) and
+// accumulates its threads' pairs (x <= y) in float64.  A single 32 x 32 GEMM
+// tile would have to sweep all of K (up to 10^6) alone.
+__global__ void __launch_bounds__(256) gram_natural_kernel(const void* __restrict__ src, int src_bf16, int n,
+                                                           int64_t S, int64_t fibers,
+                                                           double* __restrict__ partial) {
   __shared__ float tile[32][129];
   const int chunk = blockIdx.x;
-  const int64_t c_begin = static_cast<int64_t>(chunk) * kGramChunk;
-  const int64_t c_end = c_begin + kGramChunk < K ? c_begin + kGramChunk : K;
+  const int64_t f_begin = static_cast<int64_t>(chunk) * kGramChunk;
+  const int64_t f_end = f_begin + kGramChunk < fibers ? f_begin + kGramChunk : fibers;
   const int npairs = n * (n + 1) / 2;
   double acc[3] = {0.0, 0.0, 0.0};
   int px[3], py[3];
 #pragma unroll
-  for (int q = 0; q < 3; ++q) {  // pair index -> (x, y), x <= y, row by row
+  for (int q = 0; q < 3; ++q) {
     int pidx = threadIdx.x + 256 * q, x = 0;
     while (pidx >= n - x && x < n) pidx -= n - x, ++x;
     px[q] = x;
     py[q] = x + pidx;
   }
-  for (int64_t c0 = c_begin; c0 < c_end; c0 += 128) {
+  for (int64_t f0 = f_begin; f0 < f_end; f0 += 128) {
     for (int e = threadIdx.x; e < 32 * 128; e += 256) {
       const int r = e >> 7, c = e & 127;
-      const int64_t col = c0 + c;
-      tile[r][c] = (r < n && col < c_end) ? U[static_cast<int64_t>(r) * ld + col] : 0.f;
+      const int64_t f = f0 + c;
+      float v = 0.f;
+      if (r < n && f < f_end) {
+        const int64_t o = f / S;
+        const int64_t off = o * n * S + static_cast<int64_t>(r) * S + (f - o * S);
+        v = src_bf16 ? __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(src)[off]) << 16)
+                     : reinterpret_cast<const float*>(src)[off];
+      }
+      tile[r][c] = v;
     }
     __syncthreads();
 #pragma unroll
@@ -229,18 +265,107 @@ __global__ void __launch_bounds__(256) gram_small_kernel(const float* __restrict
     if (threadIdx.x + 256 * q < npairs) partial[static_cast<int64_t>(chunk) * kGramPairs + threadIdx.x + 256 * q] = acc[q];
 }
 
-__global__ void gram_reduce_kernel(const double* __restrict__ partial, int nchunks, int n, float beta,
-                                   float* __restrict__ H, int ldh) {
-  const int npairs = n * (n + 1) / 2;
-  for (int pidx0 = threadIdx.x; pidx0 < npairs; pidx0 += blockDim.x) {
-    double sum = 0.0;
-    for (int ch = 0; ch < nchunks; ++ch) sum += partial[static_cast<int64_t>(ch) * kGramPairs + pidx0];
-    int pidx = pidx0, x = 0;
-    while (pidx >= n - x) pidx -= n - x, ++x;
-    const int y = x + pidx;
-    const float v = static_cast<float>(static_cast<double>(beta) * H[x * ldh + y] + sum);
-    H[x * ldh + y] = v;
-    H[y * ldh + x] = v;
+// The same statistic for modes of at most 8: with a handful of pairs the
+// staged tile leaves most threads idle, so here each thread takes every
+// blockDim-th fibre of the chunk and keeps all N (N + 1) / 2 pair sums of its
+// fibres in float64 registers; the CTA then adds its threads' sums in a fixed
+// order (per warp by shuffles, then warp by warp).
+template <int N>
+__global__ void __launch_bounds__(256) gram_tiny_kernel(const void* __restrict__ src, int src_bf16, int64_t S,
+                                                        int64_t fibers, double* __restrict__ partial) {
+  constexpr int kPairs = N * (N + 1) / 2;
+  __shared__ double red[8][kPairs];
+  const int64_t f_begin = static_cast<int64_t>(blockIdx.x) * kGramChunk;
+  const int64_t f_end = f_begin + kGramChunk < fibers ? f_begin + kGramChunk : fibers;
+  double acc[kPairs];
+#pragma unroll
+  for (int q = 0; q < kPairs; ++q) acc[q] = 0.0;
+  for (int64_t f = f_begin + threadIdx.x; f < f_end; f += blockDim.x) {
+    const int64_t o = f / S;
+    const int64_t base = o * N * S + (f - o * S);
+    double x[N];
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const int64_t off = base + static_cast<int64_t>(j) * S;
+      x[j] = src_bf16 ? __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(src)[off]) << 16)
+                      : reinterpret_cast<const float*>(src)[off];
+    }
+    int q = 0;
+#pragma unroll
+    for (int a = 0; a < N; ++a)
+#pragma unroll
+      for (int b = a; b < N; ++b) acc[q++] += x[a] * x[b];
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int q = 0; q < kPairs; ++q) {
+    double v = acc[q];
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0) red[warp][q] = v;
+  }
+  __syncthreads();
+  for (int q = threadIdx.x; q < kPairs; q += blockDim.x) {
+    double v = 0.0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) v += red[w][q];
+    partial[static_cast<int64_t>(blockIdx.x) * kGramPairs + q] = v;
+  }
+}
+
+int launch_gram_natural(const void* src, int src_bf16, int n, int64_t S, int64_t fibers, double* partial,
+                        cudaStream_t st) {
+  const unsigned nchunks = static_cast<unsigned>((fibers + kGramChunk - 1) / kGramChunk);
+  switch (n) {
+#define GRAM_TINY(N) \
+  case N: gram_tiny_kernel<N><<<nchunks, 256, 0, st>>>(src, src_bf16, S, fibers, partial); break;
+    GRAM_TINY(1) GRAM_TINY(2) GRAM_TINY(3) GRAM_TINY(4) GRAM_TINY(5) GRAM_TINY(6) GRAM_TINY(7) GRAM_TINY(8)
+#undef GRAM_TINY
+    default: gram_natural_kernel<<<nchunks, 256, 0, st>>>(src, src_bf16, n, S, fibers, partial);
+  }
+  count_launch();
+  return check_cuda(cudaGetLastError(), n <= 8 ? "gram_tiny_kernel" : "gram_natural_kernel");
+}
+
+// Product along a short mode in the natural layout: every fibre x (n values,
+// stride S) becomes X x, X the mode's n x n root (row stride ldx); with
+// `update` the result goes into the weight, dst -= lr X x.  One thread a
+// fibre, grid-stride; consecutive threads take consecutive fibres, so every
+// load and store is coalesced.
+__global__ void __launch_bounds__(256) mode_small_kernel(const void* __restrict__ src, int src_bf16,
+                                                         float* __restrict__ dst, int update, float lr,
+                                                         const float* __restrict__ X, int ldx, int n, int64_t S,
+                                                         int64_t fibers) {
+  pdl_launch_dependents();
+  __shared__ float xs[32][33];
+  for (int e = threadIdx.x; e < 32 * 32; e += blockDim.x) {
+    const int r = e >> 5, c = e & 31;
+    xs[r][c] = (r < n && c < n) ? X[r * ldx + c] : 0.f;
+  }
+  __syncthreads();
+  for (int64_t f = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; f < fibers;
+       f += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t o = f / S;
+    const int64_t base = o * n * S + (f - o * S);
+    float x[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      x[j] = 0.f;
+      if (j < n) {
+        const int64_t off = base + static_cast<int64_t>(j) * S;
+        x[j] = src_bf16 ? __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(src)[off]) << 16)
+                        : reinterpret_cast<const float*>(src)[off];
+      }
+    }
+#pragma unroll 1
+    for (int i = 0; i < n; ++i) {
+      float acc = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) acc = fmaf(xs[i][j], x[j], acc);
+      float* d = dst + base + static_cast<int64_t>(i) * S;
+      if (update)
+        *d -= lr * acc;
+      else
+        *d = acc;
+    }
   }
 }
 
@@ -277,7 +402,8 @@ struct Plan {
 };
 
 // A mode whose statistic takes the split-K path.
-bool small_mode(int npad, int64_t K) { return npad == 32 && K > 8 * kGramChunk; }
+// A mode handled in the natural layout (no unfolding): at most 32 long and not diagonal.
+bool short_mode(const Mode& m) { return !m.diag && m.n <= 32; }
 
 int validate_tensor_config(const shampoo_config* c) {
   if (!c) return set_error(SHAMPOO_ERR_INVALID_ARG, "config is NULL");
@@ -389,7 +515,7 @@ int make_plan(const shampoo_config* cfg, int32_t nparams, const int32_t* orders,
   P.gram_bytes = 0;
   for (const Param& pr : P.params)
     for (const Mode& m : pr.modes)
-      if (!m.diag && small_mode(m.npad, m.K))
+      if (short_mode(m))
         P.gram_bytes = std::max(P.gram_bytes, static_cast<size_t>((m.K + kGramChunk - 1) / kGramChunk) * kGramPairs * 8);
   P.root_bytes = 0;
   for (const Group& g : P.groups) {
@@ -503,21 +629,29 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
     const Group& G = P.groups[m.group];
     return reinterpret_cast<float*>(h->state + G.h_off) + static_cast<size_t>(m.slot) * G.npad * G.npad;
   };
-  // 1-2. unfold every mode of every parameter and accumulate its statistic
-  // (one GEMM launch per parameter, one group per mode).  With a refresh
-  // pending, all statistics must be complete before the roots, so the
-  // unfoldings of the last parameter are the ones left for the apply below.
+  // stride of mode i in the natural layout: the product of the later dimensions
+  auto stride_after = [](const Param& pr, int i) {
+    int64_t S = 1;
+    for (int l = i + 1; l < pr.k; ++l) S *= pr.dims[l];
+    return S;
+  };
+  const int bf16 = c.grad_dtype == SHAMPOO_BF16 ? 1 : 0;
+  // 1-2. unfold every long mode of every parameter and accumulate its
+  // statistic (one GEMM launch per parameter, one group per mode); short
+  // modes sum theirs from the gradient's natural layout.  With a refresh
+  // pending, all statistics must be complete before the roots.
   for (size_t j = 0; j < P.params.size(); ++j) {
     const Param& pr = P.params[j];
     std::vector<StackMaps> um(pr.k);
     for (int i = 0; i < pr.k; ++i) {
       const Mode& m = pr.modes[i];
+      if (short_mode(m)) continue;
       PermArgs a;
       std::memset(&a, 0, sizeof(a));
       a.k = pr.k;
       for (int l = 0; l < pr.k; ++l) a.dims[l] = pr.dims[l];
       a.src = d_grads[j];
-      a.src_bf16 = c.grad_dtype == SHAMPOO_BF16;
+      a.src_bf16 = bf16;
       a.s = PermSide{-1, 0};
       a.dst = U + m.u_off;
       a.d = PermSide{i, m.Kpad};
@@ -538,16 +672,16 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
         if ((rc = check_cuda(cudaGetLastError(), "row_sumsq_kernel"))) return rc;
         continue;
       }
-      if (small_mode(m.npad, m.K)) {
-        ProfScope ps(K_GRAM, st, 2.0 * m.n * double(m.n) * m.K, 4.0 * m.n * double(m.K));
+      if (short_mode(m)) {
         double* partial = reinterpret_cast<double*>(h->scratch + P.scratch_gram);
         const int nchunks = static_cast<int>((m.K + kGramChunk - 1) / kGramChunk);
-        gram_small_kernel<<<nchunks, 256, 0, st>>>(U + m.u_off, m.Kpad, m.n, m.K, partial);
-        count_launch();
-        if ((rc = check_cuda(cudaGetLastError(), "gram_small_kernel"))) return rc;
-        gram_reduce_kernel<<<1, 256, 0, st>>>(partial, nchunks, m.n, c.beta, hptr(m), m.npad);
-        count_launch();
-        if ((rc = check_cuda(cudaGetLastError(), "gram_reduce_kernel"))) return rc;
+        {
+          ProfScope ps(K_GRAM, st, 2.0 * m.n * double(m.n) * m.K, (bf16 ? 2.0 : 4.0) * m.n * double(m.K));
+          if ((rc = launch_gram_natural(d_grads[j], bf16, m.n, stride_after(pr, i), m.K, partial, st))) return rc;
+          gram_reduce_kernel<<<1, 256, 0, st>>>(partial, nchunks, m.n, c.beta, hptr(m), m.npad);
+          count_launch();
+          if ((rc = check_cuda(cudaGetLastError(), "gram_reduce_kernel"))) return rc;
+        }
         continue;
       }
       Epilogue& e = b.add_rect(1, m.npad, m.npad, m.Kpad, um[i], 0, um[i], 0, 2.0 * m.n * double(m.n) * m.K,
@@ -561,7 +695,7 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
     }
     if (b.L.ngroups > 0 && (rc = b.launch(st))) return rc;
     for (int i = 0; i < pr.k; ++i)
-      if (!pr.modes[i].diag && !small_mode(pr.modes[i].npad, pr.modes[i].K) &&
+      if (!pr.modes[i].diag && !short_mode(pr.modes[i]) &&
           (rc = launch_mirror_lower(hptr(pr.modes[i]), 1, pr.modes[i].npad, st)))
         return rc;
   }
@@ -597,38 +731,63 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
         if ((rc = check_cuda(cudaGetLastError(), "diag_root_kernel"))) return rc;
       }
   }
-  // 4. apply: V = X_0 unfold_0(G), then mode by mode; the last fold updates W.
+  // 4. apply: the short modes' products on the natural layout first, then the
+  // long modes on unfoldings (mode by mode); the last product updates W.
+  auto xptr = [&](const Mode& m) {
+    const Group& G = P.groups[m.group];
+    return reinterpret_cast<const float*>(h->state + G.x_off) + static_cast<size_t>(m.slot) * G.npad * G.npad;
+  };
   for (size_t j = 0; j < P.params.size(); ++j) {
     const Param& pr = P.params[j];
-    const Mode& m0 = pr.modes[0];
-    {  // mode-0 unfolding of G (U holds the last parameter's unfoldings only)
+    std::vector<int> shorts, longs;
+    for (int i = 0; i < pr.k; ++i) (short_mode(pr.modes[i]) ? shorts : longs).push_back(i);
+    const void* src = d_grads[j];  // natural layout of the partial product
+    int src_bf16 = bf16;
+    for (size_t q = 0; q < shorts.size(); ++q) {
+      const Mode& m = pr.modes[shorts[q]];
+      const bool last = longs.empty() && q + 1 == shorts.size();
+      float* dst = last ? d_weights[j] : (src == V[0] ? V[1] : V[0]);
+      const int64_t fibers = pr.size / m.n;
+      ProfScope ps(K_MODE_SMALL, st, 2.0 * m.n * double(m.n) * fibers, ((src_bf16 ? 2.0 : 4.0) + (last ? 8.0 : 4.0)) * pr.size);
+      const unsigned grid = static_cast<unsigned>(std::min<int64_t>((fibers + 255) / 256, 148 * 8));
+      mode_small_kernel<<<grid, 256, 0, st>>>(src, src_bf16, dst, last ? 1 : 0, c.lr, xptr(m), m.npad, m.n,
+                                              stride_after(pr, shorts[q]), fibers);
+      count_launch();
+      if ((rc = check_cuda(cudaGetLastError(), "mode_small_kernel"))) return rc;
+      src = dst;
+      src_bf16 = 0;
+    }
+    if (longs.empty()) continue;
+    // cur: unfolding of the partial product along the current mode; out: X_i cur.
+    // The next mode's permutation reads `out` into `cur`, so the two never trade roles.
+    float* cur = src == V[1] ? V[0] : V[1];
+    float* out = cur == V[1] ? V[0] : V[1];
+    {  // first long mode's unfolding of the natural partial product
+      const Mode& m0 = pr.modes[longs[0]];
       PermArgs a;
       std::memset(&a, 0, sizeof(a));
       a.k = pr.k;
       for (int l = 0; l < pr.k; ++l) a.dims[l] = pr.dims[l];
-      a.src = d_grads[j];
-      a.src_bf16 = c.grad_dtype == SHAMPOO_BF16;
+      a.src = src;
+      a.src_bf16 = src_bf16;
       a.s = PermSide{-1, 0};
-      a.dst = V[1];
-      a.d = PermSide{0, m0.Kpad};
+      a.dst = cur;
+      a.d = PermSide{longs[0], m0.Kpad};
       a.rows = m0.npad;
       a.cols = m0.Kpad;
       if ((rc = launch_permute(a, static_cast<int64_t>(m0.npad) * m0.Kpad, st))) return rc;
     }
-    // cur: mode-i unfolding of the partial product; out: X_i cur.  The next
-    // mode's permutation reads `out` into `cur`, so the two never trade roles.
-    float* cur = V[1];
-    float* out = V[0];
-    for (int i = 0; i < pr.k; ++i) {
+    for (size_t q = 0; q < longs.size(); ++q) {
+      const int i = longs[q];
       const Mode& m = pr.modes[i];
-      if (i > 0) {  // cur <- mode-i unfolding of the previous product (held in `out` as mode i-1)
-        const Mode& mp = pr.modes[i - 1];
+      if (q > 0) {  // cur <- mode-i unfolding of the previous product (held in `out` as that mode's)
+        const Mode& mp = pr.modes[longs[q - 1]];
         PermArgs a;
         std::memset(&a, 0, sizeof(a));
         a.k = pr.k;
         for (int l = 0; l < pr.k; ++l) a.dims[l] = pr.dims[l];
         a.src = out;
-        a.s = PermSide{i - 1, mp.Kpad};
+        a.s = PermSide{longs[q - 1], mp.Kpad};
         a.dst = cur;
         a.d = PermSide{i, m.Kpad};
         a.rows = m.npad;
@@ -649,19 +808,19 @@ int shampoo_tensor_step(shampoo_tensor_handle h, float* const* d_weights, const 
       Builder b;
       Epilogue& e = b.add_rect(1, m.npad, m.Kpad, m.npad, h->mX[m.group], m.slot, cm, 0,
                                2.0 * m.n * double(m.n) * m.K, B_MN_MAJOR);
-      if (i == 0) b.L.g[0].b_exact = g_exact;
+      if (q == 0 && shorts.empty()) b.L.g[0].b_exact = g_exact;  // the raw (widened bf16) gradient
       e.D = out;
       e.flags = h->d_status;
       if ((rc = b.launch(st))) return rc;
     }
-    {  // fold the last product (mode k-1 unfolding) into the weight: W -= lr P
-      const Mode& ml = pr.modes[pr.k - 1];
+    {  // fold the last product (its mode's unfolding) into the weight: W -= lr P
+      const Mode& ml = pr.modes[longs.back()];
       PermArgs a;
       std::memset(&a, 0, sizeof(a));
       a.k = pr.k;
       for (int l = 0; l < pr.k; ++l) a.dims[l] = pr.dims[l];
       a.src = out;
-      a.s = PermSide{pr.k - 1, ml.Kpad};
+      a.s = PermSide{longs.back(), ml.Kpad};
       a.dst = d_weights[j];
       a.d = PermSide{-1, 0};
       a.update = 1;
