@@ -28,7 +28,10 @@ tensors one kernel launch (shampoo_pack_blocks) gathers or scatters a whole
 block list; buffers are allocated once.
 
 Communication uses torch.distributed (NCCL on GPUs); every step runs the same
-collectives in the same order on all ranks.  ``reduce_scatter(out, inp)`` and
+collectives in the same order on all ranks.  Whenever a process group is
+initialised (or collectives are injected) the collective path runs, also with
+a single rank, where the exchange is a copy; only a single process without a
+group skips it.  ``reduce_scatter(out, inp)`` and
 ``all_gather(out, inp)`` (flat tensors: out = the rank's segment of the sum
 of inp over ranks; out = every rank's inp, back to back) may be injected to
 replace them, and ``local_step`` replaces the blocks' compute (the CUDA
@@ -111,6 +114,7 @@ class ShardedShampoo:
         self.device = torch.device(device) if device is not None else None
         self._rs = reduce_scatter if reduce_scatter is not None else self._default_reduce_scatter
         self._ag = all_gather if all_gather is not None else self._default_all_gather
+        self.collective = self.world > 1 or self.distributed or reduce_scatter is not None or all_gather is not None
         self._bufs = None
         self._packers = None
         self.local_optimizer = None
@@ -209,21 +213,21 @@ class ShardedShampoo:
         if self.grads_reduced:
             self.local_step([self._view(weights[self.blocks[i][0]], i) for i in self.owned],
                             [self._view(grads[self.blocks[i][0]], i) for i in self.owned])
-            if self.world > 1:
+            if self.collective:
                 self._gather("own", weights, b["wmine"][:n])
         else:
             gall = b["gall"][:self.world * n]
             self._gather("all", grads, gall, 1.0 / self.world)
             gmine = b["gmine"][:n]
-            if self.world > 1:
+            if self.collective:
                 self._rs(gmine, gall)
             else:
                 gmine.copy_(gall)
             self._gather("own", weights, b["wmine"][:n])
             self.local_step(self._own_views(b["wmine"]), self._own_views(gmine))
-            if self.world == 1:
+            if not self.collective:
                 self._scatter("own", b["wmine"], weights)
-        if self.world > 1:
+        if self.collective:
             wall = b["wall"][:self.world * n]
             self._ag(wall, b["wmine"][:n])
             self._scatter("all", wall, weights)

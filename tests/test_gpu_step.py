@@ -180,6 +180,44 @@ def test_checkpoint_resume_bit_identical(sb):
     assert b.step_count == a.step_count == wl.steps
 
 
+def test_sharded_collectives_on_a_single_rank_nccl_group(sb, tmp_path):
+    """The sharded optimizer's collective path on NCCL, with one rank (every
+    GPU call here has one GPU, and ranks that wait on each other cannot share
+    one): the packed reduce-scatter of local gradients and the all-gather of
+    updated blocks run as NCCL calls on the real packed buffers, where with a
+    single rank each is a copy.  Both gradient modes end with weights
+    bit-identical to the unsharded step."""
+    from datetime import timedelta
+
+    import torch.distributed as dist
+    from shampoo_family_second_b200 import sharded
+    if dist.is_initialized():
+        pytest.skip("a process group is already initialised in this process")
+    store = dist.FileStore(str(tmp_path / "store"), 1)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=timedelta(seconds=60))
+    try:
+        shapes = ((96, 80), (40, 70))
+        wl = workloads.workload("tiny", shapes=shapes, block=32, steps=3, iters=30, tol=1e-5, beta=0.9, eps=1e-4,
+                                solver=workloads.SOLVER_NEWTON_CUBIC)
+        cfg = sb.config_from_workload(wl)
+        full = sb.Shampoo(shapes, cfg)
+        reduced = sharded.ShardedShampoo(shapes, cfg)
+        packed = sharded.ShardedShampoo(shapes, cfg, grads_reduced=False)
+        assert reduced.collective and packed.collective and dist.get_backend() == "nccl"
+        W1, W2, W3 = ([torch.zeros(s, dtype=torch.float32, device="cuda") for s in shapes] for _ in range(3))
+        stream = workloads.GradientStream(wl)
+        for _ in range(wl.steps):
+            G = [torch.from_numpy(g).cuda() for g in stream.next()]
+            full.step(W1, G)
+            reduced.step(W2, G)
+            packed.step(W3, G)
+        torch.cuda.synchronize()
+        for a, b, c in zip(W1, W2, W3):
+            assert torch.equal(a, b) and torch.equal(a, c)
+    finally:
+        dist.destroy_process_group()
+
+
 def test_bf16_checkpoint_resume_between_refreshes(sb):
     """bf16 gradients, blocks of 256 with ragged edges, refresh every 3 steps.
     The first apply product reads the roots as three bf16 planes, split after
