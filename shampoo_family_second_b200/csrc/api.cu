@@ -116,13 +116,19 @@ StateLayout state_layout(int nb, int B, bool momentum, size_t stats_elem) {
 bool apply_planes(const shampoo_config* c) {
   return c->grad_dtype == SHAMPOO_BF16 && c->solver != SHAMPOO_SOLVER_NEWTON_CUBIC_F64 && !(c->momentum > 0.f);
 }
+// Roots kept for several steps: the second apply product reads XR split into
+// its tf32 hi and lo parts (once per refresh) instead of splitting it on chip
+// every step.  With a refresh every step the split pass would cost more than
+// it saves.
+bool presplit_xr(const shampoo_config* c) { return c->refresh_every > 1; }
 
 // Scratch layout: Gs | Gt (none with XL planes) | Tapply | XL planes (3 nb bf16 matrices, with XL planes only)
-//   | blk_wptr (nb ptrs) | blk_ld (nb) | solver scratch
+//   | XR split (nb tf32 hi, then nb lo matrices; with refresh_every > 1 only) | blk_wptr (nb ptrs) | blk_ld (nb)
+//   | solver scratch
 struct ScratchLayout {
-  size_t gs, gt, tap, xlp, wptr, ld, root, root_bytes, total;
+  size_t gs, gt, tap, xlp, xrs, wptr, ld, root, root_bytes, total;
 };
-ScratchLayout scratch_layout(int nb, int B, int solver, int p, bool planes) {
+ScratchLayout scratch_layout(int nb, int B, int solver, int p, bool planes, bool xr_split) {
   ScratchLayout s;
   size_t o = 0;
   s.gs = o, o += al(plain_floats(nb, B) * 4);
@@ -131,6 +137,8 @@ ScratchLayout scratch_layout(int nb, int B, int solver, int p, bool planes) {
   s.tap = o, o += al(plain_floats(nb, B) * 4);
   s.xlp = o;
   if (planes) o += al(plain_floats(nb, B) * 3 * 2);
+  s.xrs = o;
+  if (xr_split) o += al(plain_floats(2 * nb, B) * 4);
   s.wptr = o, o += al(size_t(nb) * 8);
   s.ld = o, o += al(size_t(nb) * 4);
   s.root = o;
@@ -188,6 +196,10 @@ struct shampoo_ctx {
   // (a new handle, shampoo_set_step after restoring a state)
   uint16_t* xlp = nullptr;
   StackMaps mXlp;
+  // XR split into its tf32 hi and lo parts (the second apply's right operand),
+  // rebuilt on the same schedule as the XL planes
+  float* xrs = nullptr;
+  StackMaps mXrs;
   bool planes_stale = true;
   double stats_flops_L = 0, stats_flops_R = 0, stack_bytes = 0;
   int64_t step = 0;
@@ -218,7 +230,8 @@ int shampoo_query_sizes(const shampoo_config* cfg, int32_t nparams, const int64_
   if ((rc = build_table(cfg->block, nparams, rows, cols, sh))) return rc;
   if (!state_bytes || !scratch_bytes) return set_error(SHAMPOO_ERR_INVALID_ARG, "output pointer is NULL");
   *state_bytes = state_layout(sh.nb, cfg->block, cfg->momentum > 0.f, stats_elem_bytes(cfg->solver)).total;
-  *scratch_bytes = scratch_layout(sh.nb, cfg->block, cfg->solver, cfg->root_p, apply_planes(cfg)).total;
+  *scratch_bytes =
+      scratch_layout(sh.nb, cfg->block, cfg->solver, cfg->root_p, apply_planes(cfg), presplit_xr(cfg)).total;
   return SHAMPOO_OK;
 }
 
@@ -235,7 +248,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
     return set_error(SHAMPOO_ERR_UNSUPPORTED, "state/scratch must be 256-byte aligned");
   const int B = cfg->block, nb = sh.nb;
   StateLayout sl = state_layout(nb, B, cfg->momentum > 0.f, stats_elem_bytes(cfg->solver));
-  ScratchLayout xl = scratch_layout(nb, B, cfg->solver, cfg->root_p, apply_planes(cfg));
+  ScratchLayout xl = scratch_layout(nb, B, cfg->solver, cfg->root_p, apply_planes(cfg), presplit_xr(cfg));
   if (state_bytes < sl.total) return set_error(SHAMPOO_ERR_WORKSPACE, "state %zu < %zu bytes", state_bytes, sl.total);
   if (scratch_bytes < xl.total)
     return set_error(SHAMPOO_ERR_WORKSPACE, "scratch %zu < %zu bytes", scratch_bytes, xl.total);
@@ -263,6 +276,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
   h->Gs = reinterpret_cast<float*>(h->scratch + xl.gs);
   h->Gt = apply_planes(cfg) ? nullptr : reinterpret_cast<float*>(h->scratch + xl.gt);
   h->xlp = apply_planes(cfg) ? reinterpret_cast<uint16_t*>(h->scratch + xl.xlp) : nullptr;
+  h->xrs = presplit_xr(cfg) ? reinterpret_cast<float*>(h->scratch + xl.xrs) : nullptr;
   h->Tap = reinterpret_cast<float*>(h->scratch + xl.tap);
   h->blk_wptr = reinterpret_cast<float**>(h->scratch + xl.wptr);
   if (cfg->grad_dtype == SHAMPOO_BF16 && !h->stats_f64) {
@@ -308,6 +322,7 @@ int shampoo_init(const shampoo_config* cfg, int32_t nparams, const int64_t* rows
   }
   if ((rc = make_stack_maps(h->mGs, h->Gs, nb, B)) || (h->Gt && (rc = make_stack_maps(h->mGt, h->Gt, nb, B))) ||
       (h->xlp && (rc = make_stack_maps_bf16(h->mXlp, h->xlp, 3 * int64_t(nb), B))) ||
+      (h->xrs && (rc = make_stack_maps(h->mXrs, h->xrs, 2 * int64_t(nb), B))) ||
       (rc = make_stack_maps(h->mRoots, h->roots, 2 * nb, B)) || (rc = make_stack_maps(h->mTap, h->Tap, nb, B)) ||
       (h->mom && (rc = make_stack_maps(h->mMom, h->mom, nb, B))) ||
       (h->Gs16 && ((rc = make_stack_maps_bf16(h->mGs16, h->Gs16, nb, B)) ||
@@ -358,10 +373,17 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
   // (T = XL M with momentum, M read as a true product) depends on neither, so
   // it joins the same launch.
   const bool refresh = h->step % c.refresh_every == 0;
-  if (h->xlp && h->planes_stale && !refresh) {  // roots not split since they were last set
-    if ((rc = launch_split_planes(h->roots, plain_floats(nb, B), h->xlp, st))) return rc;
+  // The apply products' split forms of the roots: XL as bf16 planes (bf16
+  // gradients), XR as tf32 hi and lo parts.
+  auto split_roots = [&]() -> int {
+    int r;
+    const int64_t cnt = plain_floats(nb, B);
+    if (h->xlp && (r = launch_split_planes(h->roots, cnt, h->xlp, st))) return r;
+    if (h->xrs && (r = launch_split_tf32(h->roots + cnt, cnt, h->xrs, h->xrs + cnt, st))) return r;
     h->planes_stale = false;
-  }
+    return SHAMPOO_OK;
+  };
+  if (h->planes_stale && !refresh && (rc = split_roots())) return rc;  // roots not split since they were set
   auto add_apply1 = [&](Builder& b) {
     if (h->xlp) {  // T = (XL0 + XL1 + XL2) G: three bf16 planes of XL against G^T in bf16
       Epilogue& e = b.add(nb, B, h->mXlp, 0, h->mGt16, 0, h->stats_flops_L);
@@ -451,10 +473,7 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
     job.power_warm_hint = h->power_refreshed;
     if ((rc = run_inverse_roots(job, h->scratch + h->xl.root, h->xl.root_bytes, st))) return rc;
     h->power_refreshed = 1;
-    if (h->xlp) {
-      if ((rc = launch_split_planes(h->roots, plain_floats(nb, B), h->xlp, st))) return rc;
-      h->planes_stale = false;
-    }
+    if ((rc = split_roots())) return rc;
     // 4a. apply, first product: T = XL G (with the fresh roots)
     Builder b;
     add_apply1(b);
@@ -463,7 +482,12 @@ int shampoo_step_strided(shampoo_handle h, float* const* d_weights, const void* 
   // 4b. apply, second product: W -= lr T XR (masked scatter into the weights)
   {
     Builder b;
-    Epilogue& e = b.add(nb, B, h->mTap, 0, h->mRoots, nb, h->stats_flops_R);
+    Epilogue& e = h->xrs ? b.add(nb, B, h->mTap, 0, h->mXrs, 0, h->stats_flops_R)  // XR as its hi and lo parts
+                         : b.add(nb, B, h->mTap, 0, h->mRoots, nb, h->stats_flops_R);
+    if (h->xrs) {
+      b.L.g[0].b_presplit = 1;
+      b.L.g[0].b_plane_stride = nb;
+    }
     e.wptr = h->blk_wptr;
     e.wld = h->blk_ld;
     e.wrows = h->d_wrows;

@@ -324,7 +324,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int ck = chunk_k(G);
           const int nk = (G.k + ck - 1) / ck;
           const int planes = G.a_planes > 1 ? G.a_planes : 1;
-          const uint32_t tx_bytes = static_cast<uint32_t>(G.a_rows * planes + G.b_rows) * BK * 4u;  // 64 B a row
+          const uint32_t tx_bytes =  // 64 bytes a box row
+              static_cast<uint32_t>(G.a_rows * planes + G.b_rows * (G.b_presplit ? 2 : 1)) * BK * 4u;
           const void* amap = &maps.m[G.a_map];
           const void* bmap = &maps.m[G.b_map];
           const int am = G.a_off + tc.mat;
@@ -353,6 +354,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tma_load_3d(sb + q * MN_BLOCK, bmap, &full[s], tc.tn * BN + q * 32, kc * BK, bm);
             } else {
               tma_load_3d(sb, bmap, &full[s], kc * ck, tc.tn * BN, bm);
+              if (G.b_presplit)  // B's lo parts, split ahead of the launch, straight into the B lo area
+                tma_load_3d(sb + RAW_BYTES, bmap, &full[s], kc * ck, tc.tn * BN, bm + G.b_plane_stride);
             }
           }
         }
@@ -451,7 +454,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int nk = (G.k + ck - 1) / ck;
         // An operand whose values are exact in tf32 needs no split: its hi
         // part is the value as TMA wrote it, and its lo part is never read.
-        const bool keep_a = G.a_exact != 0, keep_b = G.b_exact != 0;
+        // A presplit B arrives as its hi and lo parts (two TMA loads).
+        const bool keep_a = G.a_exact != 0, keep_b = G.b_exact != 0 || G.b_presplit != 0;
 #pragma unroll 1
         for (int kc = 0; kc < nk; ++kc, ++it) {
           const int s = it % STAGES;
@@ -744,6 +748,8 @@ int launch_gemm(GemmLaunch& L, const TmaMaps& maps, cudaStream_t st) {
     // planes 1 and 2 of A land in the stage's lo areas, which only bf16 groups leave unused
     if (g.a_planes > 3 || (g.a_planes > 1 && (!g.bf16 || g.a_rows > BM)))
       return set_error(-1, "A in %d planes needs a bf16 group of at most 3 planes", g.a_planes);
+    if (g.b_presplit && (g.bf16 || g.b_mn || g.b_exact || g.b_rows > BN))
+      return set_error(-1, "a presplit B needs an fp32 K-major operand with lo parts");
     g.tiles_per = g.tiles_m * g.tiles_n;
     if (g.sym) {
       g.tiles_per = 0;

@@ -65,6 +65,8 @@ struct GemmGroup {
   int a_planes;          // bf16 only: A is the exact sum of this many bf16 planes (0 or 1: one), plane q
                          // at matrix a_off + mat + q * a_plane_stride of A's stack; one MMA per plane
   int a_plane_stride;
+  int b_presplit;        // fp32 K-major B given as tf32 hi parts (matrix b_off + mat) and lo parts (matrix
+  int b_plane_stride;    // b_off + mat + b_plane_stride) of split_tf32: B's tiles are not split on chip
   int sym;               // 1: D is symmetric (square, e.g. G G^T): only the tiles that reach the
                          // diagonal or above are computed; launch_mirror_lower fills the rest
   int tiles_per;         // tiles computed per matrix (filled by launch_gemm)
@@ -245,6 +247,9 @@ int launch_mirror_lower(float* D, int64_t batch, int n, cudaStream_t st);
 // planes[q * count + i], q = 0, 1, 2: bf16 values whose sum is X[i] exactly
 // (each the nearest bf16 to what the previous planes leave); count % 4 == 0.
 int launch_split_planes(const float* X, int64_t count, uint16_t* planes, cudaStream_t st);
+// hi[i], lo[i] = split_tf32(X[i]) (the on-chip split of the 3xTF32 product,
+// stored); count % 4 == 0.
+int launch_split_tf32(const float* X, int64_t count, float* hi, float* lo, cudaStream_t st);
 
 // fp64 products of the fp64-iterate solver (solver_f64.cu): per matrix,
 // D = alpha A B + beta C + gamma I (true product, row-major n x n operands),

@@ -579,6 +579,25 @@ __global__ void split_planes_kernel(const float4* __restrict__ X, int64_t n4, ui
   }
 }
 
+// The 3xTF32 product's operand split (split_tf32, the converter warps' own
+// function), stored: hi[i] + lo[i] = X[i].  The roots XR stay fixed between
+// refreshes, so the second apply product reads them split from HBM and its
+// converters split only T.  Grid-stride over float4 groups.
+__global__ void split_tf32_kernel(const float4* __restrict__ X, int64_t n4, float4* __restrict__ hi,
+                                  float4* __restrict__ lo) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 x = X[i];
+    float4 h, l;
+    split_tf32(x.x, h.x, l.x);
+    split_tf32(x.y, h.y, l.y);
+    split_tf32(x.z, h.z, l.z);
+    split_tf32(x.w, h.w, l.w);
+    hi[i] = h;
+    lo[i] = l;
+  }
+}
+
 __global__ void fill_int_kernel(int* p, int64_t count, int value) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i < count) p[i] = value;
@@ -700,6 +719,20 @@ int launch_split_planes(const float* X, int64_t count, uint16_t* planes, cudaStr
   split_planes_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(X), n4, reinterpret_cast<uint2*>(planes));
   count_launch();
   return check_cuda(cudaGetLastError(), "split_planes_kernel");
+}
+
+int launch_split_tf32(const float* X, int64_t count, float* hi, float* lo, cudaStream_t st) {
+  if (count == 0) return 0;
+  if (count % 4 ||
+      (reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(hi) | reinterpret_cast<uintptr_t>(lo)) & 15)
+    return set_error(-1, "split_tf32: %lld values, or unaligned buffers", static_cast<long long>(count));
+  ProfScope ps(K_PLANES, st, 0.0, 12.0 * count);
+  const int64_t n4 = count / 4;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 148 * 16));
+  split_tf32_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(X), n4, reinterpret_cast<float4*>(hi),
+                                          reinterpret_cast<float4*>(lo));
+  count_launch();
+  return check_cuda(cudaGetLastError(), "split_tf32_kernel");
 }
 
 int launch_fill_iters(int* iters, int64_t batch, int value, cudaStream_t st) {

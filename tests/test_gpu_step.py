@@ -278,7 +278,8 @@ def test_launch_count_increases(sb):
     n0 = sb.launch_count()
     opt.step(W, [torch.randn(wl.shapes[0], device="cuda")])
     torch.cuda.synchronize()
-    # stack + stats + norm + prologue + 20 + 19 * 2 Newton launches + finalize + 2 apply
+    # stack + stats + norm + prologue + 20 + 19 * 2 Newton launches + finalize + 2 apply (a root
+    # refresh every step: the second apply splits XR on chip, with no split pass)
     assert sb.launch_count() - n0 == 1 + 1 + 1 + 1 + 20 + 19 * 2 + 1 + 2
 
 
