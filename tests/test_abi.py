@@ -55,6 +55,30 @@ def test_query_sizes_memory_is_quadratic_per_block(sb):
         assert scratch > 3 * nb * wl.block ** 2 * 4
 
 
+def test_scratch_holds_the_split_roots_where_they_pay(sb):
+    """Scratch per (B x B) block element, beside the solver's: G and G^T
+    (fp32 both, or bf16 both), T (fp32), the XL planes (three bf16, bf16
+    gradients without momentum only) and the stored tf32 split of XR (hi and
+    lo, fp32, only when roots are kept for several steps).  Checked as exact
+    differences between configurations, so the solver's share cancels."""
+    shapes = [(1024, 1024)]
+    nb, B = 4, 512
+    elems = nb * B * B
+
+    def scratch(**kw):
+        base = dict(block=B, beta=0.95, eps=1e-8, lr=1e-3, solver=sb.SOLVER_NEWTON_CUBIC)
+        base.update(kw)
+        return sb.query_sizes(sb.make_config(**base), shapes)[1]
+
+    f32_every = scratch(refresh_every=1)
+    f32_ten = scratch(refresh_every=10)
+    bf16_ten = scratch(refresh_every=10, grad_dtype=sb.BF16)
+    bf16_mom = scratch(refresh_every=10, grad_dtype=sb.BF16, momentum=0.9)
+    assert f32_ten - f32_every == 2 * elems * 4            # XR hi and lo
+    assert bf16_ten - f32_ten == 3 * elems * 2 - elems * 4  # XL planes in, the fp32 G^T stack out
+    assert bf16_mom == f32_ten                              # momentum: fp32 G^T kept, no planes
+
+
 @pytest.mark.parametrize("field,value", [("block", 48), ("block", 2048), ("root_p", 3), ("solver", 7),
                                          ("iters", 0), ("refresh_every", 0), ("beta", 1.5), ("eps", -1.0),
                                          ("grad_dtype", 5)])
