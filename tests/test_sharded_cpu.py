@@ -131,13 +131,15 @@ def test_partition_covers_and_balances(world):
         assert set(owner) == {0}
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [1, 2, 3])
 @pytest.mark.parametrize("grads_reduced", [True, False])
 def test_ranks_match_one_process(grads_reduced, world):
-    """2 ranks (even split) and 3 (uneven segments; the middle rank's slice of
-    the gradient reduction): every rank ends with the same weights as one
-    process stepping every block.  Sums of three local gradients may round
-    differently in the collective, hence a looser bound there."""
+    """1 rank (a process group of one: the collective path runs, each
+    exchange a copy), 2 ranks (even split) and 3 (uneven segments; the middle
+    rank's slice of the gradient reduction): every rank ends with the same
+    weights as one process stepping every block.  Sums of three local
+    gradients may round differently in the collective, hence a looser bound
+    there."""
     single = run_single(grads_reduced, world)
     res = run_ranks(grads_reduced, world)
     counts = [n for _, n, _ in res]
