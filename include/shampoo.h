@@ -227,7 +227,12 @@ SHAMPOO_API int shampoo_block_table(shampoo_handle h, int32_t* nb, int64_t* tabl
  * tiles whole); the rest is copied from its transpose on refresh steps only,
  * since only the roots read it.  Between refreshes, call
  * shampoo_sync_statistics before reading L or R as full matrices.  A saved
- * and restored state needs no sync: the next refresh fills the rest again. */
+ * and restored state needs no sync: the next refresh fills the rest again.
+ * The apply products read the roots in split forms derived from them after
+ * every refresh (XL as bf16 planes, XR as tf32 hi and lo parts, in the
+ * scratch); roots written through these pointers take effect after
+ * shampoo_set_step, which has the forms derived again before the next
+ * apply. */
 SHAMPOO_API int shampoo_state_views(shampoo_handle h, float** L, float** R, float** rootL, float** rootR, int64_t* step);
 
 /* Fills the part of every statistics matrix below its diagonal tiles from
@@ -246,7 +251,8 @@ SHAMPOO_API int shampoo_sync_statistics(shampoo_handle h, void* stream);
 SHAMPOO_API int shampoo_momentum_view(shampoo_handle h, float** M);
 
 /* Sets the step counter (checkpoint resume: restore the state buffer bytes,
- * then the counter). */
+ * then the counter).  The next step first derives the apply products' split
+ * forms of the roots again (see shampoo_state_views). */
 SHAMPOO_API int shampoo_set_step(shampoo_handle h, int64_t step);
 
 /* Frees the host-side handle (the caller's device buffers are untouched). */
